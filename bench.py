@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule hot path on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl {native,reference}] [--no-also] [--no-e2e]
+
+A step is one pass of the layer over one batch of synthetic input (seeded,
+recipe in gated_delta_rule_forward_b200/inputs.py).  The headline workload is
+the 350M-model layer shape: Gated DeltaNet forward, bf16 q/k/v/o, fp32 state,
+B=8 T=2048 H=8 dk=dv=128.  The line also carries the other workloads
+("also": DeltaNet on the same shape, KDA / KLA / GDN-2 at the 1.3B-model
+shape, the 65536-token forward and the 256 x 16 decode step), each with its
+own roofline.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronisation on each side, CUDA events on the launching stream, max
+over ranks.  Two input sets are rotated so that a step never finds its inputs
+in L2 (each set is larger than the 126 MB L2).  Multi-GPU (torchrun) is weak
+scaling: every rank runs its own batch, with no data-path collective.
+
+--impl reference times the fp64 CPU oracle (the only reference that exists)
+on the machine's host cores, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (variant, B, T, H, dk, dv); decode workloads use N = B and no T
+    "gdn_fwd_350m": ("gdn", 8, 2048, 8, 128, 128),
+    "deltanet_fwd_350m": ("deltanet", 8, 2048, 8, 128, 128),
+    "kda_fwd_1p3b": ("kda", 4, 4096, 16, 128, 128),
+    "kla_fwd_1p3b": ("kla", 4, 4096, 16, 128, 128),
+    "gdn2_fwd_1p3b": ("gdn2", 4, 4096, 16, 128, 128),
+    "gdn_fwd_64k": ("gdn", 1, 65536, 16, 128, 128),
+    "kla_fwd_64k": ("kla", 1, 65536, 16, 128, 128),
+    "gdn_decode_256x16": ("gdn", 256, None, 16, 128, 128),
+}
+DEFAULT = "gdn_fwd_350m"
+METRIC = "gated-delta-rule layer tokens/s (fwd, decode) at 1 B200; % of bf16 TC / HBM roofline"
+KERNEL_SOURCES = {
+    "chunk64_tc": ["gated_delta_rule_forward_b200/csrc/chunk_tc.cu"],
+    "token_bf16io": ["gated_delta_rule_forward_b200/csrc/token_fwd.cu"],
+    "token_f32io": ["gated_delta_rule_forward_b200/csrc/token_fwd.cu"],
+    "decode": ["gated_delta_rule_forward_b200/csrc/decode.cu"],
+}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def source_hash(kernel):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES.get(kernel, []) + ["gated_delta_rule_forward_b200/csrc/common.cuh"]:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
+            if f[2] == source_hash(kernel):
+                return float(f[3])
+    return None
+
+
+def fwd_bytes(variant, B, T, H, dk, dv, io_bytes=2):
+    """Algorithmic HBM bytes of one forward launch: every input read once, o and
+    the final state written once, no initial state (zeros)."""
+    th = B * T * H
+    b = th * (2 * dk + 2 * dv) * io_bytes
+    if variant != "gdn2":
+        b += th * 4                                    # beta / eta
+    if variant in ("gdn", "kla"):
+        b += th * 4                                    # scalar log decay
+    elif variant in ("kda", "gdn2"):
+        b += th * dk * 4                               # channel-wise log decay
+    if variant == "gdn2":
+        b += 2 * th * dk * 4                           # erase and write gates
+    b += B * H * dk * dv * 4                           # final state
+    return b
+
+
+def decode_bytes(variant, N, H, dk, dv, io_bytes=2):
+    nh = N * H
+    b = nh * dk * dv * 4 * 2 + nh * (2 * dk + 2 * dv) * io_bytes
+    if variant != "gdn2":
+        b += nh * 4
+    if variant in ("gdn", "kla"):
+        b += nh * 4
+    elif variant in ("kda", "gdn2"):
+        b += nh * dk * 4
+    if variant == "gdn2":
+        b += 2 * nh * dk * 4
+    return b
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.samples, self.proc, self.gpu = [], None, gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for t, s in self.samples if t0 - 0.15 <= t <= t1 + 0.15] or [s for _, s in self.samples]
+        if not rows:
+            return None
+        sm = sorted(float(r[0]) for r in rows if r[0].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.strip() == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- native arm
+def make_device_sets(name, seed):
+    """Two device-resident input sets of a forward workload (and the host copy)."""
+    from gated_delta_rule_forward_b200.inputs import make_inputs
+    variant, B, T, H, dk, dv = WORKLOADS[name]
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=seed)
+    dev = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    # second set: the same tensors rolled along the head axis (distinct values and addresses)
+    dev2 = {k: (None if v is None else torch.roll(v, 1, dims=-2 if v.dim() == 4 else -1).contiguous())
+            for k, v in dev.items()}
+    return [dev, dev2], d
+
+
+def gates(d):
+    return {k: d[k] for k in ("beta", "log_g", "erase_b", "write_w")}
+
+
+def run_forward_workload(name, K, W, world, e2e=False, seed=0):
+    import gated_delta_rule_forward_b200 as gdr
+    variant, B, T, H, dk, dv = WORKLOADS[name]
+    sets, host = make_device_sets(name, seed)
+    outs = [torch.empty(B, T, H, dv, device="cuda", dtype=torch.bfloat16) for _ in sets]
+    finals = [torch.empty(B, H, dk, dv, device="cuda", dtype=torch.float32) for _ in sets]
+    kernel = gdr.forward_kernel_name(variant, torch.bfloat16, B, T, H, dk, dv, 0)
+    launches = gdr.forward_launches(variant, torch.bfloat16, B, T, H, dk, dv, 0)
+
+    def step(i):
+        d = sets[i % 2]
+        gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), out=outs[i % 2],
+                    final_state=finals[i % 2], chunk=0)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_wall0 = time.time()
+    for i in range(K):
+        starts[i].record()
+        step(i)
+        ends[i].record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = starts[0].elapsed_time(ends[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    launch_ms = sum(per) / K                  # one kernel per step: its average duration
+    res = {
+        "workload": name, "variant": variant, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+        "kernel": kernel, "launches_per_step": launches, "ms_per_step": total_ms / K,
+        "launch_ms": launch_ms, "tokens_per_step": B * T, "wall": (t_wall0, t_wall1),
+        "alg_bytes": fwd_bytes(variant, B, T, H, dk, dv),
+    }
+    res["value"] = world * B * T * K / (total_ms / 1e3)
+    if e2e:
+        res["e2e"] = forward_e2e(name, host, K, W, world)
+    return res
+
+
+def forward_e2e(name, host, K, W, world):
+    """Public-API throughput with host buffers: pinned H2D of the step's inputs,
+    the forward, and D2H of the output, all inside the timed region."""
+    import gated_delta_rule_forward_b200 as gdr
+    variant, B, T, H, dk, dv = WORKLOADS[name]
+    pinned = {k: (None if v is None else v.pin_memory()) for k, v in host.items()}
+    o_host = torch.empty(B, T, H, dv, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values() if v is not None)
+    d2h = o_host.numel() * o_host.element_size()
+
+    def step():
+        d = {k: (None if v is None else v.to("cuda", non_blocking=True)) for k, v in pinned.items()}
+        o, _ = gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), output_final_state=False)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"value": world * B * T * K / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
+
+
+def run_decode_workload(name, K, W, world):
+    import gated_delta_rule_forward_b200 as gdr
+    from gated_delta_rule_forward_b200.inputs import make_decode_inputs, random_state
+    variant, N, _, H, dk, dv = WORKLOADS[name]
+    steps = [{k: (None if v is None else v.cuda()) for k, v in
+              make_decode_inputs(variant, N, H, s, dk, dv).items()} for s in range(4)]
+    state = random_state(N, H, dk, dv, 7).cuda()
+    out = torch.empty(N, H, dv, device="cuda", dtype=torch.bfloat16)
+
+    def step(i):
+        d = steps[i % 4]
+        gdr.decode_step(d["q"], d["k"], d["v"], state, variant=variant, **gates(d), out=out)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(K):
+        step(i)
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"workload": name, "variant": variant, "N": N, "H": H, "dk": dk, "dv": dv, "kernel": "decode",
+            "launches_per_step": 1, "ms_per_step": ms / K, "launch_ms": ms / K,
+            "value": world * N * K / (ms / 1e3), "alg_bytes": decode_bytes(variant, N, H, dk, dv)}
+
+
+def roofline(res, peaks):
+    achieved = res["alg_bytes"] / (res["launch_ms"] / 1e3) / 1e9
+    traffic = recorded_traffic(res["kernel"], res["workload"])
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+            "peak_source": peaks["source"], "alg_bytes_per_launch": res["alg_bytes"]}
+
+
+def cpu_baseline(name):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    import oracle
+    from gated_delta_rule_forward_b200.inputs import make_inputs
+    variant, B, T, H, dk, dv = WORKLOADS[name]
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+    oracle.forward(variant, **{k: (None if v is None else v[:, :64]) for k, v in d.items()})  # build/load
+    passes, t0 = 0, time.perf_counter()
+    while passes == 0 or time.perf_counter() - t0 < 2.0:     # >= 2 s wall on all host cores
+        oracle.forward(variant, **d)
+        passes += 1
+    dt = time.perf_counter() - t0
+    return {"value": passes * B * T / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{passes} pass(es) of the whole workload ({B} x {T} tokens x {H} heads), fp64, "
+                      f"{dt:.2f} s wall"}
+
+
+def native(args):
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    peaks = load_peaks()
+    sampler = ClockSampler(local)
+    sampler.start()
+    t0 = time.time()
+    main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
+    t1 = time.time()
+    also = []
+    if not args.no_also:
+        for name in WORKLOADS:
+            if name == args.workload:
+                continue
+            k = max(3, args.steps // 4) if "64k" in name else args.steps
+            r = (run_decode_workload(name, k, args.warmup, world) if WORKLOADS[name][2] is None
+                 else run_forward_workload(name, k, args.warmup, world))
+            r["roofline"] = roofline(r, peaks)
+            r["unit"] = "tokens/s"
+            r.pop("wall", None)
+            also.append(r)
+    sampler.stop()
+    clocks = sampler.summary(*main["wall"])
+    cpu = cpu_baseline(args.workload) if rank == 0 and world == 1 else None
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    variant, B, T, H, dk, dv = WORKLOADS[args.workload]
+    line = {
+        "metric": METRIC, "value": round(main["value"], 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms_per_step"], 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; q,k L2-normalised, v ~ N(0,1), sigmoid / -softplus gates)",
+        "config": {"workload": args.workload, "variant": variant, "batch_per_gpu": B, "seq_len": T,
+                   "heads": H, "dk": dk, "dv": dv, "global_batch": B * world, "kernel": main["kernel"],
+                   "state": "fp32", "parallelism": f"dp{world}",
+                   "l2": "inputs > L2; two input sets rotated between steps"},
+        "roofline": roofline(main, peaks),
+        "cpu_baseline": cpu,
+        "e2e": main.get("e2e"),
+        "gpu_launches": main["launches_per_step"] * args.steps,
+        "clocks": clocks,
+        "also": also,
+        "wall_s": round(t1 - t0, 2),
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import oracle
+    from gated_delta_rule_forward_b200.inputs import make_inputs
+    variant, B, T, H, dk, dv = WORKLOADS[args.workload]
+    if T is None:
+        raise SystemExit("reference arm supports the forward workloads")
+    d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+    for _ in range(args.warmup):
+        oracle.forward(variant, **d)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(variant, **d)
+    dt = time.perf_counter() - t0
+    value = T * args.steps / dt
+    cores = oracle.max_threads()
+    sample = f"1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "variant": variant, "batch_per_gpu": B, "seq_len": T,
+                   "heads": H, "dk": dk, "dv": dv, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT, choices=[w for w, v in WORKLOADS.items() if v[2]])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-also", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference(args)
+    else:
+        native(args)
+
+
+if __name__ == "__main__":
+    main()

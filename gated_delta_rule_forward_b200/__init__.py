@@ -1,0 +1,12 @@
+"""B200-native gated delta-rule linear attention (DeltaNet, Gated DeltaNet,
+KDA, Gated DeltaNet-2, KLA): chunked forward and recurrent decode.
+
+The compute lives in libgdr.so (hand-written CUDA for sm_100a, C ABI in
+include/gdr.h); this package is its thin Python binding.  Importing the
+package does not load the library; the first call does, and raises if the
+library is missing.
+"""
+from .ops import VARIANTS, decode_step, forward, forward_kernel_name, forward_launches  # noqa: F401
+from ._lib import GdrError  # noqa: F401
+
+__all__ = ["forward", "decode_step", "forward_launches", "forward_kernel_name", "VARIANTS", "GdrError"]

@@ -1,0 +1,198 @@
+// libgdr C ABI: argument validation, kernel selection, launch-error mapping.
+// The operation each entry point performs is specified in include/gdr.h.
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "gdr.h"
+#include "chunk_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+gdr_status_t fail(gdr_status_t st, const std::string &why) {
+  g_last_error = why;
+  return st;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool injected_launch_fault() {
+  const char *f = std::getenv("GDR_FAULT");
+  return f && std::strcmp(f, "launch") == 0;
+}
+
+gdr_status_t check_cuda(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return GDR_OK;
+  return fail(GDR_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool valid_variant(int v) { return v >= GDR_DELTANET && v <= GDR_KLA; }
+bool valid_dim(int d) { return d == 64 || d == 128; }
+
+enum class Kernel { None, Token, ChunkTC };
+
+// Which kernel a forward call runs, or None with a status and reason.
+Kernel select_forward(int variant, int dtype, int dk, int dv, int chunk, gdr_status_t *st,
+                      std::string *why) {
+  *st = GDR_OK;
+  const bool tc = dtype == GDR_BF16 && gdr_chunk_tc_supported(variant, dk, dv);
+  if (chunk == 1) return Kernel::Token;
+  if (chunk == 0) return tc ? Kernel::ChunkTC : Kernel::Token;
+  if (chunk == 64) {
+    if (tc) return Kernel::ChunkTC;
+    *st = GDR_ERR_UNSUPPORTED;
+    *why = "chunk=64 tensor-core kernel needs bf16 I/O and a supported (variant, dk, dv)";
+    return Kernel::None;
+  }
+  *st = GDR_ERR_INVALID_ARG;
+  *why = "chunk must be 0 (auto), 1 (per-token) or 64 (chunked tensor-core)";
+  return Kernel::None;
+}
+
+gdr_status_t validate_common(int variant, int dtype, int dk, int dv) {
+  if (!valid_variant(variant)) return fail(GDR_ERR_INVALID_ARG, "variant out of range");
+  if (dtype != GDR_F32 && dtype != GDR_BF16) return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_F32 or GDR_BF16");
+  if (!valid_dim(dk) || !valid_dim(dv)) return fail(GDR_ERR_UNSUPPORTED, "dk and dv must each be 64 or 128");
+  return GDR_OK;
+}
+
+gdr_status_t validate_gates(int variant, const float *beta, const float *log_g, const float *erase_b,
+                            const float *write_w) {
+  if (variant != GDR_GDN2 && !beta) return fail(GDR_ERR_INVALID_ARG, "beta (eta for KLA) is required");
+  if (variant != GDR_DELTANET && !log_g) return fail(GDR_ERR_INVALID_ARG, "log_g is required for this variant");
+  if (variant == GDR_GDN2 && (!erase_b || !write_w))
+    return fail(GDR_ERR_INVALID_ARG, "GDN-2 needs erase_b and write_w");
+  const void *ptrs[4] = {beta, log_g, erase_b, write_w};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "a gate pointer is not 16-byte aligned");
+  return GDR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr_version(void) { return 100; }
+
+const char *gdr_status_string(gdr_status_t s) {
+  switch (s) {
+    case GDR_OK: return "GDR_OK";
+    case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+    case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+    case GDR_ERR_ALIGNMENT: return "GDR_ERR_ALIGNMENT";
+    case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+    case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+  }
+  return "GDR_UNKNOWN_STATUS";
+}
+
+const char *gdr_last_error(void) { return g_last_error.c_str(); }
+
+size_t gdr_forward_workspace_size(int, int, int, int, int, int, int, int) { return 0; }
+
+int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  if (!valid_variant(variant) || (dtype != 0 && dtype != 1) || !valid_dim(dk) || !valid_dim(dv)) return 0;
+  if (B < 0 || T < 0 || H < 0) return 0;
+  gdr_status_t st;
+  std::string why;
+  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  if (kern == Kernel::None) return 0;
+  if ((long)B * H == 0) return 0;
+  if (T == 0) return 1;  // state copy or clear
+  return kern == Kernel::ChunkTC ? gdr_chunk_tc_launches(B, T, H, dk, dv) : 1;
+}
+
+const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  if (gdr_forward_launches(variant, dtype, B, T, H, dk, dv, chunk) == 0 && (long)B * H * T != 0) return "none";
+  gdr_status_t st;
+  std::string why;
+  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  if (kern == Kernel::ChunkTC) return "chunk64_tc";
+  if (kern == Kernel::Token) return dtype == GDR_BF16 ? "token_bf16io" : "token_f32io";
+  return "none";
+}
+
+gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                                 const gdr_fwd_args_t *a, float eps, float scale, int chunk,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  gdr_status_t st = validate_common(variant, dtype, dk, dv);
+  if (st != GDR_OK) return st;
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
+  if (!a) return fail(GDR_ERR_INVALID_ARG, "args is NULL");
+  std::string why;
+  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  if (kern == Kernel::None) return fail(st, why);
+  if ((long)B * H == 0) return GDR_OK;  // nothing to do
+  if (T > 0) {
+    if (!a->q || !a->k || !a->v || !a->o) return fail(GDR_ERR_INVALID_ARG, "q, k, v and o are required");
+    const void *io[4] = {a->q, a->k, a->v, a->o};
+    for (const void *p : io)
+      if (!aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "q, k, v and o must be 16-byte aligned");
+    st = validate_gates(variant, a->beta, a->log_g, a->erase_b, a->write_w);
+    if (st != GDR_OK) return st;
+  }
+  if ((a->initial_state && !aligned16(a->initial_state)) || (a->final_state && !aligned16(a->final_state)))
+    return fail(GDR_ERR_ALIGNMENT, "state pointers must be 16-byte aligned");
+  if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be >= 0");
+  if (injected_launch_fault()) return fail(GDR_ERR_CUDA, "injected launch failure (GDR_FAULT=launch)");
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    // No tokens: the final state is the initial state.
+    if (!a->final_state) return GDR_OK;
+    const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+    if (a->initial_state == a->final_state) return GDR_OK;
+    if (a->initial_state)
+      return check_cuda(cudaMemcpyAsync(a->final_state, a->initial_state, bytes, cudaMemcpyDeviceToDevice, s),
+                        "state copy");
+    return check_cuda(cudaMemsetAsync(a->final_state, 0, bytes, s), "state clear");
+  }
+
+  gdr::FwdProblem p;
+  p.variant = variant; p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
+  p.bf16_io = dtype == GDR_BF16;
+  p.q = a->q; p.k = a->k; p.v = a->v;
+  p.beta = a->beta; p.log_g = a->log_g; p.erase_b = a->erase_b; p.write_w = a->write_w;
+  p.s0 = a->initial_state; p.s_final = a->final_state; p.o = a->o;
+  p.eps = eps; p.scale = scale;
+  if (kern == Kernel::ChunkTC) {
+    std::string err;
+    const cudaError_t e = gdr_launch_chunk_tc(p, s, &err);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_tc: " + err + cudaGetErrorString(e));
+    return GDR_OK;
+  }
+  return check_cuda(gdr_launch_token_forward(p, s), "token_fwd launch");
+}
+
+gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv, const void *q, const void *k,
+                             const void *v, const float *beta, const float *log_g, const float *erase_b,
+                             const float *write_w, float *state, void *o, float eps, float scale, void *stream) {
+  gdr_status_t st = validate_common(variant, dtype, dk, dv);
+  if (st != GDR_OK) return st;
+  if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "N and H must be >= 0");
+  if ((long)N * H == 0) return GDR_OK;
+  if (!q || !k || !v || !o || !state) return fail(GDR_ERR_INVALID_ARG, "q, k, v, o and state are required");
+  const void *io[5] = {q, k, v, o, state};
+  for (const void *p : io)
+    if (!aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "q, k, v, o and state must be 16-byte aligned");
+  st = validate_gates(variant, beta, log_g, erase_b, write_w);
+  if (st != GDR_OK) return st;
+  if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be >= 0");
+  if (injected_launch_fault()) return fail(GDR_ERR_CUDA, "injected launch failure (GDR_FAULT=launch)");
+  gdr::DecodeProblem p;
+  p.variant = variant; p.N = N; p.H = H; p.dk = dk; p.dv = dv;
+  p.bf16_io = dtype == GDR_BF16;
+  p.q = q; p.k = k; p.v = v;
+  p.beta = beta; p.log_g = log_g; p.erase_b = erase_b; p.write_w = write_w;
+  p.state = state; p.o = o; p.eps = eps; p.scale = scale;
+  return check_cuda(gdr_launch_decode(p, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,12 @@
+// Chunked tensor-core forward (tcgen05 + TMEM + TMA, chunk C = 64, bf16 I/O).
+#pragma once
+#include <string>
+
+#include "common.cuh"
+
+// True when the chunked kernel covers (variant, dk, dv) with bf16 I/O.
+bool gdr_chunk_tc_supported(int variant, int dk, int dv);
+// Kernel launches one forward call makes on this path.
+int gdr_chunk_tc_launches(int B, int T, int H, int dk, int dv);
+// Enqueue the forward; on failure *err names the failing step.
+cudaError_t gdr_launch_chunk_tc(const gdr::FwdProblem &p, cudaStream_t stream, std::string *err);

@@ -1,0 +1,169 @@
+// Per-token forward of the gated delta rule: the exact-arithmetic path.
+//
+// One warp owns one (batch, head) and eight value columns of the state; the
+// dk x 8 fp32 slice lives in registers for the whole sequence (lane l holds
+// rows l, l+32, ...).  Each token applies, in fp32,
+//     S~ = Diag(g) S;   x = S~^T k;   y = S~^T q
+//     S  = S~ - a x^T + c v^T
+//     o  = scale * (y - (a.q) x + (c.q) v)          (= S^T (scale q))
+// which is the recurrence of "Kaczmarz Linear Attention" (KLA update rule)
+// and of the erase/write form read from "Gated DeltaNet-2" (technical core).
+// Reading x and y from S~ in one pass and correcting y afterwards gives the
+// same result as reading S after the update, with one reduction round.
+//
+// This kernel serves fp32 I/O (where the 1e-4 relative bar rules out bf16
+// tensor-core operands), chunk == 1 requests, and shapes the chunked kernel
+// does not cover.  Columns are independent, so the slicing is exact.
+#include "common.cuh"
+
+namespace gdr {
+namespace {
+
+template <int DK, typename IO, int VAR>
+__global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
+  constexpr int R = DK / 32;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int ngroups = p.dv / 8;
+  if (gw >= p.B * p.H * ngroups) return;
+  const int cg = gw % ngroups;
+  const int bh = gw / ngroups;
+  const int b = bh / p.H, h = bh % p.H;
+  const int c0 = cg * 8;
+  const int dv = p.dv;
+  const IO *__restrict__ q = static_cast<const IO *>(p.q);
+  const IO *__restrict__ k = static_cast<const IO *>(p.k);
+  const IO *__restrict__ v = static_cast<const IO *>(p.v);
+  IO *__restrict__ o = static_cast<IO *>(p.o);
+
+  float S[R][8];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (p.s0) {
+      const float4 *src = reinterpret_cast<const float4 *>(
+          p.s0 + ((size_t)bh * DK + lane + 32 * r) * dv + c0);
+      float4 a = __ldg(src), bq = __ldg(src + 1);
+      S[r][0] = a.x; S[r][1] = a.y; S[r][2] = a.z; S[r][3] = a.w;
+      S[r][4] = bq.x; S[r][5] = bq.y; S[r][6] = bq.z; S[r][7] = bq.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) S[r][c] = 0.f;
+    }
+  }
+
+  for (int t = 0; t < p.T; ++t) {
+    const size_t th = ((size_t)b * p.T + t) * p.H + h;
+    float kv[R], qv[R], g[R], ea[R], wc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      kv[r] = ld_io<IO>(k + th * DK + lane + 32 * r);
+      qv[r] = ld_io<IO>(q + th * DK + lane + 32 * r);
+    }
+    float vv[8];
+    ld8<IO>(v + th * dv + c0, vv);
+    if constexpr (scalar_decay(VAR)) {
+      const float gs = expf(__ldg(p.log_g + th));
+#pragma unroll
+      for (int r = 0; r < R; ++r) g[r] = gs;
+    } else if constexpr (channel_decay(VAR)) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) g[r] = expf(__ldg(p.log_g + th * DK + lane + 32 * r));
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) g[r] = 1.f;
+    }
+    if constexpr (VAR == kGDN2) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        ea[r] = __ldg(p.erase_b + th * DK + lane + 32 * r) * kv[r];
+        wc[r] = __ldg(p.write_w + th * DK + lane + 32 * r) * kv[r];
+      }
+    }
+
+    // decay, then the two readouts and the scalar dot products of this lane
+    float x[8], y[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) { x[c] = 0.f; y[c] = 0.f; }
+    float s1 = 0.f, s2 = 0.f;   // (k.q, k.k) or ((b.k).q, (w.k).q)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        S[r][c] *= g[r];
+        x[c] = fmaf(S[r][c], kv[r], x[c]);
+        y[c] = fmaf(S[r][c], qv[r], y[c]);
+      }
+      if constexpr (VAR == kGDN2) {
+        s1 = fmaf(ea[r], qv[r], s1);
+        s2 = fmaf(wc[r], qv[r], s2);
+      } else {
+        s1 = fmaf(kv[r], qv[r], s1);
+        s2 = fmaf(kv[r], kv[r], s2);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) { x[c] = warp_sum(x[c]); y[c] = warp_sum(y[c]); }
+    s1 = warp_sum(s1);
+    if constexpr (VAR == kKLA || VAR == kGDN2) s2 = warp_sum(s2);
+
+    float out[8];
+    if constexpr (VAR == kGDN2) {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) S[r][c] = fmaf(-ea[r], x[c], fmaf(wc[r], vv[c], S[r][c]));
+#pragma unroll
+      for (int c = 0; c < 8; ++c) out[c] = p.scale * (y[c] - s1 * x[c] + s2 * vv[c]);
+    } else {
+      float step = __ldg(p.beta + th);                      // beta_t, or eta_t for KLA
+      if constexpr (VAR == kKLA) step = step / (s2 + p.eps);  // Kaczmarz step
+      float e[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) e[c] = vv[c] - x[c];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float a = step * kv[r];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) S[r][c] = fmaf(a, e[c], S[r][c]);
+      }
+      const float akq = step * s1;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) out[c] = p.scale * fmaf(akq, e[c], y[c]);
+    }
+    if (lane == 0) st8<IO>(o + th * dv + c0, out);
+  }
+
+  if (p.s_final) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float4 *dst = reinterpret_cast<float4 *>(p.s_final + ((size_t)bh * DK + lane + 32 * r) * dv + c0);
+      dst[0] = make_float4(S[r][0], S[r][1], S[r][2], S[r][3]);
+      dst[1] = make_float4(S[r][4], S[r][5], S[r][6], S[r][7]);
+    }
+  }
+}
+
+template <int DK, typename IO>
+cudaError_t launch_dk_io(const FwdProblem &p, cudaStream_t s) {
+  const long warps = (long)p.B * p.H * (p.dv / 8);
+  const dim3 grid((unsigned)((warps + 3) / 4)), block(128);
+  switch (p.variant) {
+    case kDeltaNet: token_fwd_kernel<DK, IO, kDeltaNet><<<grid, block, 0, s>>>(p); break;
+    case kGatedDeltaNet: token_fwd_kernel<DK, IO, kGatedDeltaNet><<<grid, block, 0, s>>>(p); break;
+    case kKDA: token_fwd_kernel<DK, IO, kKDA><<<grid, block, 0, s>>>(p); break;
+    case kGDN2: token_fwd_kernel<DK, IO, kGDN2><<<grid, block, 0, s>>>(p); break;
+    case kKLA: token_fwd_kernel<DK, IO, kKLA><<<grid, block, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace gdr
+
+cudaError_t gdr_launch_token_forward(const gdr::FwdProblem &p, cudaStream_t s) {
+  using namespace gdr;
+  if (p.dk == 128) return p.bf16_io ? launch_dk_io<128, __nv_bfloat16>(p, s) : launch_dk_io<128, float>(p, s);
+  if (p.dk == 64) return p.bf16_io ? launch_dk_io<64, __nv_bfloat16>(p, s) : launch_dk_io<64, float>(p, s);
+  return cudaErrorInvalidValue;
+}

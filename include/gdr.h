@@ -1,0 +1,154 @@
+/*
+ * gdr.h -- C ABI of libgdr, the B200 (sm_100a) gated delta-rule library.
+ *
+ * The operation.  Per (batch, head) the library carries a state
+ * S in R^{dk x dv} (fp32) through the tokens t = 0 .. T-1:
+ *
+ *     S~_t = Diag(g_t) S_{t-1}                      (decay of the old state)
+ *     x_t  = S~_t^T k_t                             (readout at the key)
+ *     S_t  = S~_t - a_t x_t^T + c_t v_t^T           (erase, then write)
+ *     o_t  = S_t^T (scale * q_t)                    (readout after the update)
+ *
+ * and the five variants choose g, a and c:
+ *
+ *   GDR_DELTANET        g = 1                 a = c = beta_t k_t
+ *   GDR_GATED_DELTANET  g = alpha_t (scalar)  a = c = beta_t k_t
+ *   GDR_KDA             g in R^{dk}           a = c = beta_t k_t
+ *   GDR_GDN2            g in R^{dk}           a = b_t (.) k_t,  c = w_t (.) k_t
+ *   GDR_KLA             g = alpha_t (scalar)  a = c = beta_t k_t with
+ *                                             beta_t = eta_t / (||k_t||^2 + eps)
+ *
+ * Sources: "Kaczmarz Linear Attention" (gist.science/ja/paper/2605.08587),
+ * sections "problem definition" and "KLA update rule" (decayed state, residual
+ * e_t = v_t - S~^T k_t, update S_t = S~ + beta_t k_t e_t^T, Kaczmarz step) and
+ * section "implementation" (KLA keeps the state shape and the chunkwise solver
+ * of Gated DeltaNet and only changes the diagonal coefficient matrix);
+ * "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention"
+ * (ai-auto-bdv.pages.dev/blog/arxiv-260522791/), sections "what is new" and
+ * "technical core" (channel-wise decay of KDA; separate channel-wise erase
+ * gate b_t and write gate w_t; the chunkwise WY algorithm with the decay
+ * absorbed into asymmetric erase factors).  The GDN-2 form above is the
+ * reading of that page's garbled formula that reduces to KDA when
+ * b_t = w_t = beta_t, as the page states it must.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory, keeps no pointer after the call returns and
+ *    never synchronises: work is enqueued on `stream` (a cudaStream_t passed as
+ *    void*; NULL means the legacy default stream) and the call returns.
+ *  - Layouts are dense and row-major: q, k [B,T,H,dk]; v, o [B,T,H,dv];
+ *    per-token scalars [B,T,H]; per-token channel vectors [B,T,H,dk];
+ *    states [B,H,dk,dv].  q, k, v, o use the I/O dtype; all gates and the
+ *    states are fp32.
+ *  - Every tensor pointer must be 16-byte aligned.
+ *  - Decay is passed in log space: log_g = log(g) <= 0 (the chunked kernels
+ *    need cumulative log-decay).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call launches nothing and returns a status other than GDR_OK.
+ *    gdr_last_error() then gives a one-line reason (thread-local).
+ *  - A launch failure is reported as GDR_ERR_CUDA.  Faults inside a kernel
+ *    surface, as usual in CUDA, at the caller's next synchronisation.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_DELTANET = 0,
+    GDR_GATED_DELTANET = 1,
+    GDR_KDA = 2,
+    GDR_GDN2 = 3,
+    GDR_KLA = 4
+} gdr_variant_t;
+
+typedef enum {
+    GDR_F32 = 0,   /* q, k, v, o in fp32 */
+    GDR_BF16 = 1   /* q, k, v, o in bf16 */
+} gdr_dtype_t;
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,   /* NULL where required, non-positive size, bad enum */
+    GDR_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for */
+    GDR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    GDR_ERR_CUDA = 4,          /* a CUDA launch or driver call failed */
+    GDR_ERR_TIMEOUT = 5        /* reserved for bounded device-side waits */
+} gdr_status_t;
+
+/* Forward-call tensors.  Unused entries are NULL. */
+typedef struct {
+    const void *q;               /* [B,T,H,dk] I/O dtype */
+    const void *k;               /* [B,T,H,dk] I/O dtype */
+    const void *v;               /* [B,T,H,dv] I/O dtype */
+    const float *beta;           /* [B,T,H]: beta_t (DeltaNet, GDN, KDA) or eta_t (KLA); GDN-2: unused */
+    const float *log_g;          /* [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA, GDN-2); DeltaNet: unused */
+    const float *erase_b;        /* [B,T,H,dk] GDN-2 only */
+    const float *write_w;        /* [B,T,H,dk] GDN-2 only */
+    const float *initial_state;  /* [B,H,dk,dv] or NULL for zeros */
+    float *final_state;          /* [B,H,dk,dv] or NULL; may be the same buffer as initial_state */
+    void *o;                     /* [B,T,H,dv] I/O dtype, written for every token */
+} gdr_fwd_args_t;
+
+/*
+ * Bytes of device workspace gdr_forward_chunked needs for this problem.  The
+ * current kernels keep everything on chip and return 0; callers should still
+ * ask and pass a buffer of at least this size.
+ */
+size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
+                                  int dk, int dv, int chunk);
+
+/*
+ * Whole-sequence forward of B sequences of T tokens and H heads.
+ *
+ * chunk selects the algorithm:
+ *   0  automatic: the chunked tensor-core kernel (tcgen05 + TMEM + TMA, C = 64)
+ *      where it exists for (variant, dtype, dk, dv), else the per-token kernel;
+ *   1  the per-token kernel (fp32 state in registers, exact fp32 arithmetic,
+ *      any supported shape; the path used for fp32 I/O);
+ *   64 the chunked tensor-core kernel only (GDR_ERR_UNSUPPORTED where absent).
+ * Shapes: B, T, H >= 1; dk in {64, 128}; dv in {64, 128}.
+ * eps is used by KLA only; scale multiplies q.
+ * workspace may be NULL when gdr_forward_workspace_size(...) is 0.
+ */
+gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                                 const gdr_fwd_args_t *args, float eps, float scale, int chunk,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode token for N independent sequences and H heads.
+ * q, k [N,H,dk]; v, o [N,H,dv] (I/O dtype); beta [N,H]; log_g [N,H] or
+ * [N,H,dk]; erase_b, write_w [N,H,dk]; state [N,H,dk,dv] fp32, read and
+ * updated in place.  Gate roles as in gdr_fwd_args_t.
+ */
+gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv,
+                             const void *q, const void *k, const void *v,
+                             const float *beta, const float *log_g,
+                             const float *erase_b, const float *write_w,
+                             float *state, void *o, float eps, float scale, void *stream);
+
+/*
+ * Kernel launches one gdr_forward_chunked call with these arguments makes
+ * (0 if the call would be rejected), and a short name of the kernel that runs
+ * ("chunk64_tc", "token_f32io", "token_bf16io", ...).  Host-only, no GPU work.
+ */
+int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk);
+const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                                    int chunk);
+
+/* Human-readable name of a status, and the reason for the last rejected call. */
+const char *gdr_status_string(gdr_status_t status);
+const char *gdr_last_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

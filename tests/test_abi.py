@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI (no GPU work).
+
+Every call that passes validation here runs with GDR_FAULT=launch, which makes
+the library return GDR_ERR_CUDA before any CUDA call; pointer values are
+placeholders that are never dereferenced, and no test launches a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_forward_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000            # 16-byte aligned placeholder address, never dereferenced
+MISALIGNED = 0x10008
+
+
+@pytest.fixture(autouse=True)
+def _no_launch(monkeypatch):
+    monkeypatch.setenv("GDR_FAULT", "launch")
+    yield
+
+
+@pytest.fixture(scope="module")
+def L():
+    return _lib.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(gdr_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol(L):
+    syms = declared_symbols()
+    assert {"gdr_forward_chunked", "gdr_decode_step", "gdr_status_string"} <= syms
+    for s in sorted(syms):
+        assert hasattr(L, s), f"{s} declared in include/ but not exported"
+    assert set(_lib.EXPORTS) == syms
+
+
+def test_status_strings(L):
+    for code, name in _lib.STATUS.items():
+        assert L.gdr_status_string(code).decode() == name
+    assert L.gdr_version() >= 100
+
+
+def args(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, log_g=FAKE, erase_b=FAKE, write_w=FAKE,
+             initial_state=None, final_state=FAKE, o=FAKE)
+    a.update(over)
+    return _lib.FwdArgs(**a)
+
+
+def fwd(L, variant=1, dtype=1, B=2, T=8, H=2, dk=128, dv=128, a=None, eps=1e-6, chunk=0):
+    a = a if a is not None else args()
+    return L.gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, ctypes.byref(a), eps, 1.0, chunk,
+                                 None, 0, None)
+
+
+def test_valid_call_reaches_launch(L):
+    # passes validation, stops at the injected launch failure
+    assert fwd(L) == 4
+    assert "injected" in L.gdr_last_error().decode()
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(variant=7), 1), (dict(variant=-1), 1), (dict(dtype=5), 1),
+    (dict(dk=96), 2), (dict(dv=256), 2), (dict(B=-1), 1), (dict(T=-3), 1),
+    (dict(chunk=32), 1), (dict(eps=-1.0), 1),
+])
+def test_bad_arguments(L, over, code):
+    assert fwd(L, **over) == code
+    assert L.gdr_last_error().decode()
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "o"])
+def test_missing_tensor(L, field):
+    assert fwd(L, a=args(**{field: None})) == 1
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "o", "beta", "log_g", "final_state"])
+def test_misaligned(L, field):
+    assert fwd(L, a=args(**{field: MISALIGNED})) == 3
+
+
+@pytest.mark.parametrize("variant,field", [
+    (0, "beta"), (1, "beta"), (1, "log_g"), (2, "log_g"), (3, "erase_b"), (3, "write_w"),
+    (3, "log_g"), (4, "beta"), (4, "log_g")])
+def test_required_gates(L, variant, field):
+    assert fwd(L, variant=variant, a=args(**{field: None})) == 1
+
+
+def test_unused_gates_may_be_null(L):
+    assert fwd(L, variant=0, a=args(log_g=None, erase_b=None, write_w=None)) == 4
+    assert fwd(L, variant=3, a=args(beta=None)) == 4
+
+
+def test_empty_batch_is_a_noop(L):
+    assert fwd(L, B=0) == 0
+    assert fwd(L, H=0, a=args(q=None, k=None, v=None, o=None)) == 0
+
+
+def test_chunk_selection(L):
+    # the per-token kernel exists for every shape and dtype
+    for v in range(5):
+        for dt in (0, 1):
+            assert L.gdr_forward_kernel_name(v, dt, 2, 100, 2, 64, 128, 1).decode().startswith("token")
+            assert L.gdr_forward_launches(v, dt, 2, 100, 2, 64, 128, 1) == 1
+    # fp32 I/O never takes the tensor-core kernel
+    assert fwd(L, dtype=0, chunk=64) == 2
+    assert L.gdr_forward_kernel_name(1, 0, 8, 2048, 8, 128, 128, 0).decode() == "token_f32io"
+    assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 7) == 0
+
+
+def test_decode_validation(L):
+    i = ctypes.c_void_p
+    def dec(variant=1, dtype=1, N=4, H=2, dk=128, dv=128, q=FAKE, state=FAKE, beta=FAKE, log_g=FAKE,
+            eb=FAKE, ww=FAKE):
+        return L.gdr_decode_step(variant, dtype, N, H, dk, dv, i(q) if q else None, i(FAKE), i(FAKE),
+                                 i(beta) if beta else None, i(log_g) if log_g else None,
+                                 i(eb) if eb else None, i(ww) if ww else None,
+                                 i(state) if state else None, i(FAKE), 1e-6, 1.0, None)
+    assert dec() == 4
+    assert dec(N=0) == 0
+    assert dec(state=None) == 1
+    assert dec(state=MISALIGNED) == 3
+    assert dec(q=MISALIGNED) == 3
+    assert dec(dk=32) == 2
+    assert dec(variant=3, eb=None) == 1
+    assert dec(variant=2, log_g=None) == 1
+    assert dec(variant=0, log_g=None) == 4
+
+
+def test_workspace_is_zero(L):
+    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 0

@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle.
+
+Every case feeds the same seeded inputs (gated_delta_rule_forward_b200.inputs)
+to both sides; the oracle sees the I/O-dtype-rounded values up-cast exactly.
+Tolerances are in tests/parity_util.py.  ``chunk`` 1 is the per-token kernel,
+64 the chunked tensor-core kernel (skipped where the library reports it does
+not cover the case).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_forward_b200 as gdr
+import oracle
+from gated_delta_rule_forward_b200.inputs import make_decode_inputs, make_inputs, random_state
+from parity_util import assert_close, assert_gpu_close, gate_kwargs, select, to_dev
+
+pytestmark = pytest.mark.gpu
+VARS = ["deltanet", "gdn", "kda", "gdn2", "kla"]
+
+
+def kernel_or_skip(variant, dtype, B, T, H, dk, dv, chunk):
+    name = gdr.forward_kernel_name(variant, dtype, B, T, H, dk, dv, chunk)
+    if name == "none":
+        pytest.skip(f"no kernel for chunk={chunk} {variant} {dtype} dk={dk} dv={dv}")
+    return name
+
+
+def run_both(variant, B, T, H, dk, dv, dtype, chunk, seed=0, s0=True, **gen):
+    kernel_or_skip(variant, dtype, B, T, H, dk, dv, chunk)
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=dtype, seed=seed, **gen)
+    S0 = random_state(B, H, dk, dv, seed + 1) if s0 else None
+    dd = to_dev(d)
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant=variant, **gate_kwargs(dd),
+                       initial_state=None if S0 is None else S0.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=S0)
+    return o, S, o_ref, S_ref
+
+
+# ----------------------------------------------------------------- config 0 (fp32)
+def test_config0_gdn_fp32():
+    """GDN fp32, B=1 H=2 T=256 dk=dv=64, seed 0: max rel error 1e-4."""
+    o, S, o_ref, S_ref = run_both("gdn", 1, 256, 2, 64, 64, torch.float32, chunk=0, s0=False)
+    assert_close(o, o_ref, torch.float32, "o")
+    assert_close(S, S_ref, torch.float32, "S")
+
+
+# ----------------------------------------------------------------- small, ragged
+@pytest.mark.parametrize("chunk", [1, 64])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("variant", VARS)
+def test_small_ragged(variant, dtype, chunk):
+    o, S, o_ref, S_ref = run_both(variant, 2, 137, 3, 128, 128, dtype, chunk, seed=3)
+    assert_close(o, o_ref, dtype, "o")
+    assert_close(S, S_ref, dtype, "S")
+
+
+@pytest.mark.parametrize("chunk", [1, 64])
+@pytest.mark.parametrize("dkdv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("variant", ["gdn", "kda", "gdn2"])
+def test_head_dims(variant, dkdv, chunk):
+    dk, dv = dkdv
+    o, S, o_ref, S_ref = run_both(variant, 1, 100, 2, dk, dv, torch.bfloat16, chunk, seed=5)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
+@pytest.mark.parametrize("chunk", [1, 64])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 128, 191])
+def test_sequence_lengths(T, chunk):
+    for variant in ("gdn", "kda"):
+        o, S, o_ref, S_ref = run_both(variant, 2, T, 2, 128, 128, torch.bfloat16, chunk, seed=T)
+        assert_close(o, o_ref, torch.bfloat16, f"{variant} o")
+        assert_close(S, S_ref, torch.bfloat16, f"{variant} S")
+
+
+@pytest.mark.parametrize("chunk", [1, 64])
+def test_zero_initial_state_and_no_final_state(chunk):
+    kernel_or_skip("gdn", torch.bfloat16, 2, 70, 2, 128, 128, chunk)
+    d = make_inputs("gdn", 2, 70, 2, dtype=torch.bfloat16, seed=9)
+    dd = to_dev(d)
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant="gdn", **gate_kwargs(dd),
+                       output_final_state=False, chunk=chunk)
+    assert S is None
+    o_ref, _ = oracle.forward("gdn", **d)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+
+
+@pytest.mark.parametrize("chunk", [1, 64])
+def test_state_in_place(chunk):
+    """final_state may be the initial_state buffer."""
+    kernel_or_skip("kda", torch.bfloat16, 2, 90, 2, 128, 128, chunk)
+    d = make_inputs("kda", 2, 90, 2, dtype=torch.bfloat16, seed=12)
+    S0 = random_state(2, 2, 128, 128, 13)
+    dd = to_dev(d)
+    buf = S0.cuda()
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant="kda", **gate_kwargs(dd),
+                       initial_state=buf, final_state=buf, chunk=chunk)
+    assert S.data_ptr() == buf.data_ptr()
+    o_ref, S_ref = oracle.forward("kda", **d, initial_state=S0)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(buf, S_ref, torch.bfloat16, "S")
+
+
+def test_empty_sequence_copies_state():
+    S0 = random_state(2, 3, 128, 128, 1).cuda()
+    q = torch.empty(2, 0, 3, 128, device="cuda", dtype=torch.bfloat16)
+    beta = torch.empty(2, 0, 3, device="cuda")
+    o, S = gdr.forward(q, q, q, variant="gdn", beta=beta, log_g=beta, initial_state=S0)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 0, 3, 128) and torch.equal(S, S0)
+    o, S = gdr.forward(q, q, q, variant="gdn", beta=beta, log_g=beta)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S).item() == 0
+
+
+# ----------------------------------------------------------------- consistency
+@pytest.mark.parametrize("chunk", [1, 64])
+def test_deterministic(chunk):
+    kernel_or_skip("gdn2", torch.bfloat16, 2, 300, 4, 128, 128, chunk)
+    d = to_dev(make_inputs("gdn2", 2, 300, 4, dtype=torch.bfloat16, seed=2))
+    a = gdr.forward(d["q"], d["k"], d["v"], variant="gdn2", **gate_kwargs(d), chunk=chunk)
+    b = gdr.forward(d["q"], d["k"], d["v"], variant="gdn2", **gate_kwargs(d), chunk=chunk)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("chunk", [1, 64])
+@pytest.mark.parametrize("variant", VARS)
+def test_resume_split(variant, chunk):
+    """forward over [0,T) == forward over [0,T1) then [T1,T) from the carried state."""
+    kernel_or_skip(variant, torch.bfloat16, 2, 200, 2, 128, 128, chunk)
+    d = to_dev(make_inputs(variant, 2, 200, 2, dtype=torch.bfloat16, seed=4))
+    o, S = gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gate_kwargs(d), chunk=chunk)
+    a = select(d, t=slice(0, 77))
+    b = select(d, t=slice(77, 200))
+    oa, Sa = gdr.forward(a["q"], a["k"], a["v"], variant=variant, **gate_kwargs(a), chunk=chunk)
+    ob, Sb = gdr.forward(b["q"], b["k"], b["v"], variant=variant, **gate_kwargs(b), chunk=chunk,
+                         initial_state=Sa)
+    assert_gpu_close(torch.cat([oa, ob], 1), o, "o")
+    assert_gpu_close(Sb, S, "S")
+
+
+def test_kla_is_gdn_with_kaczmarz_beta():
+    """KLA = Gated DeltaNet with beta_t = eta_t / (||k_t||^2 + eps) ("Kaczmarz Linear
+    Attention", implementation: only the diagonal coefficient matrix changes)."""
+    for chunk in (1, 64):
+        if gdr.forward_kernel_name("kla", torch.bfloat16, 2, 150, 2, 128, 128, chunk) == "none":
+            continue
+        d = to_dev(make_inputs("kla", 2, 150, 2, dtype=torch.bfloat16, seed=8))
+        o1, S1 = gdr.forward(d["q"], d["k"], d["v"], variant="kla", **gate_kwargs(d), eps=1e-6, chunk=chunk)
+        kk = d["k"].float().pow(2).sum(-1)
+        beta = (d["beta"] / (kk + 1e-6)).contiguous()
+        o2, S2 = gdr.forward(d["q"], d["k"], d["v"], variant="gdn", beta=beta, log_g=d["log_g"], chunk=chunk)
+        assert_gpu_close(o2, o1, "o", tol=1e-2)
+        assert_gpu_close(S2, S1, "S", tol=1e-2)
+
+
+def test_gdn2_tied_equals_kda_gpu():
+    """GDN-2 with b_t = w_t = beta_t equals KDA ("Gated DeltaNet-2", what is new)."""
+    for chunk in (1, 64):
+        if gdr.forward_kernel_name("gdn2", torch.bfloat16, 2, 150, 2, 128, 128, chunk) == "none":
+            continue
+        dk = to_dev(make_inputs("kda", 2, 150, 2, dtype=torch.bfloat16, seed=6))
+        d2 = to_dev(make_inputs("gdn2", 2, 150, 2, dtype=torch.bfloat16, seed=6, gdn2_tied=True))
+        assert torch.equal(dk["q"], d2["q"]) and torch.equal(dk["log_g"], d2["log_g"])
+        o1, S1 = gdr.forward(dk["q"], dk["k"], dk["v"], variant="kda", **gate_kwargs(dk), chunk=chunk)
+        o2, S2 = gdr.forward(d2["q"], d2["k"], d2["v"], variant="gdn2", **gate_kwargs(d2), chunk=chunk)
+        assert_gpu_close(o2, o1, "o", tol=1e-2)
+        assert_gpu_close(S2, S1, "S", tol=1e-2)
+
+
+@pytest.mark.parametrize("variant", VARS)
+def test_forward_equals_decode_steps(variant):
+    """A forward over T tokens equals T single-token decode steps."""
+    B, T, H = 3, 20, 2
+    d = to_dev(make_inputs(variant, B, T, H, dtype=torch.bfloat16, seed=10))
+    S0 = random_state(B, H, 128, 128, 11).cuda()
+    o, S = gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gate_kwargs(d), initial_state=S0)
+    state = S0.clone()
+    outs = []
+    for t in range(T):
+        s = select(d, t=t)
+        outs.append(gdr.decode_step(s["q"], s["k"], s["v"], state, variant=variant, **gate_kwargs(s)))
+    assert_gpu_close(torch.stack(outs, 1), o, "o")
+    assert_gpu_close(state, S, "S")
+
+
+# ----------------------------------------------------------------- decode vs oracle
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("variant", VARS)
+def test_decode_step_parity(variant, dtype):
+    N, H = 7, 3
+    S0 = random_state(N, H, 128, 128, 3)
+    state = S0.cuda()
+    S_ref = S0.double().numpy()
+    for step in range(4):
+        d = make_decode_inputs(variant, N, H, step, dtype=dtype)
+        dd = to_dev(d)
+        o = gdr.decode_step(dd["q"], dd["k"], dd["v"], state, variant=variant, **gate_kwargs(dd))
+        o_ref, S_ref = oracle.decode_step(variant, d["q"], d["k"], d["v"], S_ref, **gate_kwargs(d))
+        assert_close(o, o_ref, dtype, f"o step {step}")
+    assert_close(state, S_ref, dtype, "state")
+
+
+@pytest.mark.parametrize("dkdv", [(64, 64), (64, 128), (128, 64)])
+def test_decode_head_dims(dkdv):
+    dk, dv = dkdv
+    S0 = random_state(5, 2, dk, dv, 4)
+    state = S0.cuda()
+    d = make_decode_inputs("gdn2", 5, 2, 0, dk=dk, dv=dv)
+    dd = to_dev(d)
+    o = gdr.decode_step(dd["q"], dd["k"], dd["v"], state, variant="gdn2", **gate_kwargs(dd))
+    o_ref, S_ref = oracle.decode_step("gdn2", d["q"], d["k"], d["v"], S0, **gate_kwargs(d))
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(state, S_ref, torch.bfloat16, "state")
