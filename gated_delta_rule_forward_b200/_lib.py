@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libgdr.so")
 EXPORTS = (
     "gdr_forward_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
     "gdr_forward_launches", "gdr_forward_kernel_name", "gdr_status_string",
-    "gdr_last_error", "gdr_version",
+    "gdr_last_error", "gdr_version", "gdr_device_status",
 )
 
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_ALIGNMENT",
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             L.gdr_status_string.restype = ctypes.c_char_p
             L.gdr_last_error.argtypes = []
             L.gdr_last_error.restype = ctypes.c_char_p
+            L.gdr_device_status.argtypes = [vp]
+            L.gdr_device_status.restype = i
             L.gdr_version.argtypes = []
             L.gdr_version.restype = i
             _lib = L

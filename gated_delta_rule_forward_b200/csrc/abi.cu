@@ -93,6 +93,13 @@ const char *gdr_status_string(gdr_status_t s) {
 
 const char *gdr_last_error(void) { return g_last_error.c_str(); }
 
+gdr_status_t gdr_device_status(void *stream) {
+  const int e = gdr_read_device_error(static_cast<cudaStream_t>(stream));
+  if (e < 0) return fail(GDR_ERR_CUDA, "synchronisation or symbol read failed");
+  if (e > 0) return fail(GDR_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  return GDR_OK;
+}
+
 size_t gdr_forward_workspace_size(int, int, int, int, int, int, int, int) { return 0; }
 
 int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {

@@ -10,3 +10,6 @@ bool gdr_chunk_tc_supported(int variant, int dk, int dv);
 int gdr_chunk_tc_launches(int B, int T, int H, int dk, int dv);
 // Enqueue the forward; on failure *err names the failing step.
 cudaError_t gdr_launch_chunk_tc(const gdr::FwdProblem &p, cudaStream_t stream, std::string *err);
+// Synchronise `stream`, then read and clear the device error word (1 when a
+// bounded wait inside a kernel gave up, 0 otherwise, -1 on a CUDA error).
+int gdr_read_device_error(cudaStream_t stream);

@@ -140,6 +140,15 @@ int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, in
 const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                     int chunk);
 
+/*
+ * Synchronises `stream`, then reads and clears the library's device-side
+ * error word.  Returns GDR_ERR_TIMEOUT if a bounded wait inside a kernel
+ * (an mbarrier wait that ran past its limit of about a second) gave up since
+ * the last call -- that kernel then skipped its remaining work and released
+ * its tensor memory -- GDR_ERR_CUDA if the synchronisation failed, else GDR_OK.
+ */
+gdr_status_t gdr_device_status(void *stream);
+
 /* Human-readable name of a status, and the reason for the last rejected call. */
 const char *gdr_status_string(gdr_status_t status);
 const char *gdr_last_error(void);
