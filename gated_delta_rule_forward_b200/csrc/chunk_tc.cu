@@ -9,44 +9,46 @@
 //     u_t = v_t - Gamma_t S0^T k_t - sum_{r<t} beta_r (Gamma_t/Gamma_r)(k_t.k_r) u_r
 //  => (I + A) U = V - Diag(Gamma) K S0,   A_tr = beta_r (Gamma_t/Gamma_r) k_t.k_r  (r < t)
 //  => U = T V - (T Diag(Gamma)) K S0 = U' - W S0,  T = (I + A)^{-1}
-//     O = Diag(Gamma) Q S0 + P U,           P_tr = beta_r (Gamma_t/Gamma_r) q_t.k_r (r <= t)
+//     O = Diag(scale Gamma) Q S0 + P U,     P_tr = scale beta_r (Gamma_t/Gamma_r) q_t.k_r (r <= t)
 //     S_C = Gamma_C S0 + K^T Diag(beta_r Gamma_C / Gamma_r) U
 // This is the chunkwise WY / UT form that "Gated DeltaNet-2" (technical core)
 // and "Kaczmarz Linear Attention" (implementation) describe: the decay enters
 // only through the asymmetric factors Gamma_t/Gamma_r of the erase terms, and
-// KLA differs from Gated DeltaNet only in the diagonal Diag(beta).  Here KLA's
+// KLA differs from Gated DeltaNet only in the diagonal Diag(beta).  KLA's
 // ||k_t||^2 is the diagonal of K K^T, which the kernel computes anyway.
 //
-// One CTA owns one (batch, head, 64-column slice of v) and sweeps the chunks
-// in order; the fp32 state slice (128 x 64) stays in registers (thread i holds
-// row i) for the whole sequence.  Per chunk:
-//   MMA1  [K;Q] K^T            (M128 N64 K128)  -> G = K K^T, H = Q K^T
-//   SIMT  A, P (decay, beta, scale), KLA beta, T = (I + A)^{-1}
-//   MMA2  W = T Diag(Gamma) K  (M64 N128 K64),   U' = T V (M64 N64 K64)
-//   MMA3  E = U' - W S0        (M64 N64 K128, negated A, accumulating on U')
-//         Y = Q S0             (M64 N64 K128)
-//   MMA4  dS = K^T Diag(w) E   (M128 N64 K64),   Z = P E (M64 N64 K64)
-//   SIMT  S = Gamma_C S + dS;  o_t = scale Gamma_t y_t + z_t
-// Operands are bf16 in shared memory (128-byte swizzled tiles; q, k, v arrive
-// by TMA, the rest is written by the threads), accumulators fp32 in TMEM.
-// The operands that carry the state and the residuals -- S0, E, Diag(w) E and
-// P -- are split into two bf16 terms x = hi + lo (hi = bf16(x), lo =
-// bf16(x - hi)), and each product takes the hi*hi, hi*lo and lo*hi terms, so
-// those products keep ~16 bits of precision; a single bf16 rounding there
-// (2^-9 relative) would leave errors of a few percent of the output RMS on
-// heavy-tailed outputs.  T, W and the raw q, k, v tiles stay single bf16.
-// No cluster, no multicast.
+// One CTA of 8 warps owns one (batch, head, 64-column slice of v) and sweeps
+// the chunks in order.  The fp32 state slice (128 x 64) lives in registers:
+// warp w holds rows 32 (w % 4) + lane, columns 32 (w / 4) .. +31.  Per chunk:
+//   MMA1  [K;Q] K^T (bf16)              M128 N64  K128 -> G = K K^T | H = Q K^T
+//   SIMT  A, P (decay, beta, scale; KLA beta from diag G); fp16 copies of K
+//         and Diag(scale Gamma) Q; T = (I + A)^{-1} by a 16x16-blocked solve
+//   MMA2  W = T Diag(Gamma) K (bf16)     M64  N128 K64
+//         [0; T] V (bf16)                M128 N64  K64  -> lanes 64-127: U'
+//   MMA3  + [Diag(scale Gamma) Q; -W] S0 (fp16)  M128 N64 K128
+//         -> lanes 0-63: Diag(scale Gamma) Q S0, lanes 64-127: E = U' - W S0
+//   MMA4  dS = K^T Diag(w) E (fp16)      M128 N64  K64
+//         + [P; *] E (fp16)              M128 N64  K64  -> lanes 0-63: O
+//   SIMT  S = Gamma_C S + dS; o rows
+// q, k, v arrive by 4-d TMA (128-byte swizzle, two stages, no multicast); all
+// other operands are written by the threads into swizzled tiles.  The
+// operands that carry the state and the residuals (S0, E, Diag(w) E, P, W and
+// the q/k copies they meet) are fp16: its 11-bit significand keeps those
+// products near 2^-12 relative error, where bf16 (8 bits) left a few percent
+// of the output RMS on heavy-tailed outputs.  fp16's range limits |S|, |E| to
+// 6.5e4; a kernel that sees larger values raises the range flag that
+// gdr_device_status() reports.  T, its Gamma-scaled copy and raw q, k, v stay
+// bf16.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <cstdio>
 #include <mutex>
 
 #include "chunk_tc.cuh"
 #include "tc_util.cuh"
 
-// Device-side error word: set (never cleared by a kernel) when a bounded wait
-// gives up; read and cleared by gdr_device_status().
+// Device-side error word, read and cleared by gdr_device_status():
+// bit 0 = a bounded wait gave up, bit 1 = an fp16 operand left its range.
 __device__ int g_gdr_device_error = 0;
 
 namespace gdr {
@@ -56,28 +58,27 @@ namespace {
 constexpr int C = 64;         // chunk length
 constexpr int DK = 128;       // key dim handled by this kernel
 constexpr int BV = 64;        // value columns per CTA
-constexpr int NTHREADS = 128;
+constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr float F16_SAFE = 60000.f;
 
-// shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // 2 stages x [Kb0 | Qb0 | Kb1 | Qb1], 8 KB each
+// shared memory map (bytes from a 1024-aligned base); 8 KB tiles are 64 rows x 128 B
+constexpr uint32_t OFF_KQ = 0;          // 2 stages x [Kb0 | Qb0 | Kb1 | Qb1] bf16 (TMA)
 constexpr uint32_t KQ_STAGE = 32768;
-constexpr uint32_t OFF_V = 65536;       // 2 stages x 8 KB
+constexpr uint32_t OFF_V = 65536;       // 2 stages x V bf16 (TMA)
 constexpr uint32_t V_STAGE = 8192;
-constexpr uint32_t OFF_W = 81920;       // W: [b0 | b1]
-constexpr uint32_t OFF_TP = 98304;      // T Diag(Gamma)
-constexpr uint32_t OFF_TT = 106496;     // T
-constexpr uint32_t OFF_P = 114688;      // P hi
-constexpr uint32_t OFF_PL = 122880;     // P lo
-constexpr uint32_t OFF_E = 131072;      // E hi   [r][v]
-constexpr uint32_t OFF_EL = 139264;     // E lo
-constexpr uint32_t OFF_EW = 147456;     // Diag(w) E hi
-constexpr uint32_t OFF_EWL = 155648;    // Diag(w) E lo
-constexpr uint32_t OFF_S = 163840;      // S0 hi [i][v], 128 rows
-constexpr uint32_t OFF_SL = 180224;     // S0 lo
-constexpr uint32_t OFF_A = 196608;      // A^T fp32, 64 x 68
-constexpr uint32_t A_LD = 68;
-constexpr uint32_t OFF_SC = OFF_A + 64 * A_LD * 4;   // scalars: 5 x 64 floats
+constexpr uint32_t OFF_QW = 81920;      // fp16 [Qg b0 | -W b0 | Qg b1 | -W b1]
+constexpr uint32_t OFF_K16 = 114688;    // fp16 [K b0 | K b1]
+constexpr uint32_t OFF_ZT = 131072;     // bf16 [zero | T]
+constexpr uint32_t OFF_TP = 147456;     // bf16 T Diag(Gamma)
+constexpr uint32_t OFF_P = 155648;      // fp16 P (rows 0-63 of an M128 operand; E16 follows)
+constexpr uint32_t OFF_E = 163840;      // fp16 E  [r][v]
+constexpr uint32_t OFF_EW = 172032;     // fp16 Diag(w) E
+constexpr uint32_t OFF_TF = OFF_QW;     // fp32 T during the solve, 64 x 72 (aliases Qg / -W)
+constexpr uint32_t OFF_S = 180224;      // fp16 S0 [i][v], 128 rows
+constexpr uint32_t OFF_A = 196608;      // fp32 A^T [r][t], 64 x 72
+constexpr uint32_t LD = 72;             // row stride (floats) of A^T and T: conflict-free MMA fragments
+constexpr uint32_t OFF_SC = OFF_A + 64 * LD * 4;   // scalars: 5 x 64 floats
 constexpr uint32_t OFF_BAR = OFF_SC + 5 * 64 * 4;    // 3 mbarriers + TMEM slot
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // + alignment slack
@@ -86,17 +87,16 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // TMEM columns (fp32 accumulators)
 constexpr uint32_t COL_G = 0;     // M128 x 64: G (lanes 0-63), H (lanes 64-127)
 constexpr uint32_t COL_W = 64;    // M64 x 128
-constexpr uint32_t COL_E = 192;   // M64 x 64: U', then E
-constexpr uint32_t COL_Y = 256;   // M64 x 64: Q S0
-constexpr uint32_t COL_S = 320;   // M128 x 64: dS
-constexpr uint32_t COL_Z = 384;   // M64 x 64: P E
+constexpr uint32_t COL_YE = 192;  // M128 x 64: lanes 0-63 Q S0 (+ P E), lanes 64-127 U' then E
+constexpr uint32_t COL_S = 256;   // M128 x 64: dS
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t ID_M128_N64_KK = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_M64_N128_KMN = idesc_bf16(64, 128, false, true);
-constexpr uint32_t ID_M64_N64_KMN = idesc_bf16(64, 64, false, true);
-constexpr uint32_t ID_M64_N64_KMN_NEG = idesc_bf16(64, 64, false, true, true);
-constexpr uint32_t ID_M128_N64_MNMN = idesc_bf16(128, 64, true, true);
+constexpr uint32_t ID_G = idesc_bf16(128, 64, false, false);        // [K;Q] K^T
+constexpr uint32_t ID_W = idesc_bf16(64, 128, false, true);         // T' K
+constexpr uint32_t ID_U = idesc_bf16(128, 64, false, true);         // [0;T] V
+constexpr uint32_t ID_YE = idesc_f16(128, 64, false, true);         // [Qg;-W] S0
+constexpr uint32_t ID_DS = idesc_f16(128, 64, true, true);          // K^T Ew
+constexpr uint32_t ID_PE = idesc_f16(128, 64, false, true);         // [P;*] E
 
 struct Params {
   int T, H, dv;
@@ -106,14 +106,8 @@ struct Params {
   float eps, scale;
 };
 
-// Store a row of 64 floats as two bf16 rows: hi = bf16(x), lo = bf16(x - hi).
-__device__ __forceinline__ void st_row64_split(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t r, const float *x) {
-  float lo[64];
-#pragma unroll
-  for (int j = 0; j < 64; ++j) lo[j] = x[j] - __bfloat162float(__float2bfloat16_rn(x[j]));
-  st_row64(hi_tile, r, x);
-  st_row64(lo_tile, r, lo);
-}
+// Round to tf32 and keep as float: the solve stores its operands pre-rounded.
+__device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
 
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -122,6 +116,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;            // TMEM lane quadrant, column half
+  const int row = quad * 32 + lane;                       // this thread's TMEM lane (M128 layout)
   const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
   const int NC = (p.T + C - 1) / C;
 
@@ -133,7 +129,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float *sc_wf = sc_g2 + 64;                                 // beta_r Gamma_C / Gamma_r
   float *sc_G = sc_wf + 64;                                  // Gamma_t
   float *sc_tmp = sc_G + 64;
-  float *At = reinterpret_cast<float *>(sm + OFF_A);        // At[r][t] = A[t][r]
+  float *At = reinterpret_cast<float *>(sm + OFF_A);        // At[r * LD + t] = A[t][r]
+  float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -148,13 +145,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
+  // zero tile (rows 0-63 of the [0; T] operand)
+  for (int i = tid; i < 512; i += NTHREADS)
+    reinterpret_cast<uint4 *>(sm + OFF_ZT)[i] = make_uint4(0u, 0u, 0u, 0u);
 
-  // state row i = tid, columns v0 .. v0+63, fp32 in registers
-  float S[64];
+  // state: row `row`, columns v0 + 32 half .. +31
+  float S[32];
   {
-    const float *src = p.s0 ? p.s0 + ((static_cast<size_t>(b) * p.H + h) * DK + tid) * p.dv + v0 : nullptr;
+    const float *src =
+        p.s0 ? p.s0 + ((static_cast<size_t>(b) * p.H + h) * DK + row) * p.dv + v0 + 32 * half : nullptr;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 8; ++j) {
       float4 f = src ? __ldg(reinterpret_cast<const float4 *>(src) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
       S[4 * j] = f.x; S[4 * j + 1] = f.y; S[4 * j + 2] = f.z; S[4 * j + 3] = f.w;
     }
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
 
   auto issue_chunk = [&](int c, int s) {
     uint8_t *kq = sm + OFF_KQ + s * KQ_STAGE;
@@ -177,107 +178,155 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     issue_chunk(0, 0);
     if (NC > 1) issue_chunk(1, 1);
   }
-  st_row64_split(sm + OFF_S, sm + OFF_SL, tid, S);
+  // fp16 S0 tile, this thread's 32 columns = four 16-byte chunks of row `row`
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
+
+  // gates of chunk 0 (prefetched one chunk ahead from here on)
+  float pf_lg = 0.f, pf_bt = 0.f;
+  auto load_gates = [&](int c) {
+    pf_lg = 0.f;
+    pf_bt = 0.f;
+    const int t = c * C + tid;
+    if (tid < 64 && t < p.T) {
+      const size_t th = (static_cast<size_t>(b) * p.T + t) * p.H + h;
+      if constexpr (scalar_decay(VAR)) pf_lg = __ldg(p.log_g + th);
+      pf_bt = __ldg(p.beta + th);
+    }
+  };
+  load_gates(0);
   fence_async_smem();
   __syncthreads();
 
   uint32_t mma_phase = 0;
   int bad = 0;
-  const uint32_t s_tile = smem_u32(sm + OFF_S), sl_tile = smem_u32(sm + OFF_SL);
+  float smax = 0.f;                                    // largest |fp16 operand| seen (range check)
+  const uint32_t s_tile = smem_u32(sm + OFF_S);
 
   for (int c = 0; c < NC; ++c) {
     const int s = c & 1;
     const int t0 = c * C;
     const uint32_t kq = smem_u32(sm + OFF_KQ + s * KQ_STAGE);
     const uint32_t vt = smem_u32(sm + OFF_V + s * V_STAGE);
+    uint8_t *kq_ptr = sm + OFF_KQ + s * KQ_STAGE;
 
-    // ---- (a) gates: beta_t, cumulative log2 decay
+    // ---- (a) gates: beta_t, cumulative log2 decay; prefetch the next chunk's
     if (tid < 64) {
-      const int t = t0 + tid;
-      float lg = 0.f, bt = 0.f;
-      if (t < p.T) {
-        const size_t th = (static_cast<size_t>(b) * p.T + t) * p.H + h;
-        if constexpr (scalar_decay(VAR)) lg = __ldg(p.log_g + th);
-        bt = __ldg(p.beta + th);
-      }
-      float x = lg * LOG2E;  // inclusive scan within the warp
+      float x = pf_lg * LOG2E;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
       sc_tmp[tid] = x;
-      sc_beta[tid] = bt;
+      sc_beta[tid] = pf_bt;
     }
+    if (c + 1 < NC) load_gates(c + 1);
     __syncthreads();
-    if (tid < 64) sc_g2[tid] = sc_tmp[tid] + (tid >= 32 ? sc_tmp[31] : 0.f);
+    if (tid < 64) {
+      const float g2 = sc_tmp[tid] + (tid >= 32 ? sc_tmp[31] : 0.f);
+      sc_g2[tid] = g2;
+      sc_G[tid] = ex2(g2);
+    }
 
     // ---- (b) chunk inputs landed?
     if (!mbar_wait(&bar_full[s], (c >> 1) & 1)) bad = 1;
     if (__syncthreads_or(bad)) break;
 
-    // ---- (c) MMA1: [K;Q] K^T
+    // ---- (c) MMA1: [K;Q] K^T; meanwhile the fp16 copy of K
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), ID_M128_N64_KK, kk > 0);
+        mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), ID_G, kk > 0);
       }
       mma_commit(bar_mma);
+    }
+    {
+      // fp16 copy of K: 2 atoms x 64 rows x 8 chunks = 1024 chunks; 4 per thread
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int idx = it * NTHREADS + tid;
+        const int kb = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+        const uint32_t off = sw128(r, j);
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4 *>(kq_ptr + kb * 16384 + off), x);
+        st_chunk_f16(sm + OFF_K16 + kb * 8192 + off, x);
+      }
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
     mma_phase ^= 1;
     tc_fence_after();
 
-    // ---- (d) A (warps 0-1, rows t = tid), P (warps 2-3, rows t = tid - 64)
+    // ---- (d) A (lanes 0-63) and P (lanes 64-127); this thread: 32 columns
     {
-      float g[64];
-      tmem_ld64(tmem + lane_base + COL_G, g);
-      const int row = tid & 63;
+      float g[32];
+      tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
+      const int t = row & 63;
+      const int r0 = 32 * half;
       if constexpr (VAR == kKLA) {
-        if (warp < 2) {
+        if (quad < 2 && (t >> 5) == half) {
           float kk = 0.f;
 #pragma unroll
-          for (int r = 0; r < 64; ++r) kk = (r == row) ? g[r] : kk;
-          const float eta = sc_beta[row];
-          sc_beta[row] = (eta == 0.f) ? 0.f : eta / (kk + p.eps);   // Kaczmarz step
+          for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
+          const float eta = sc_beta[t];
+          sc_beta[t] = (eta == 0.f) ? 0.f : eta / (kk + p.eps);   // Kaczmarz step
         }
       }
       __syncthreads();
+      // decay factors 2^(g2_t - g2_r) = rowf_t * colf_r with the reference at the
+      // first column of each 32-column half (rowf <= 1 where used, colf >= 1);
+      // exact per element when the chunk's decay span could overflow the split
+      const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
       if (tid < 64) {
         sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - sc_g2[tid]);
-        sc_G[tid] = ex2(sc_g2[tid]);
+        sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - sc_g2[tid]);
       }
-      const float g2t = sc_g2[row];
-      if (warp < 2) {
+      __syncthreads();
+      const float g2t = sc_g2[t];
+      const float rowf = (t >= r0) ? ex2(g2t - sc_g2[r0]) : 0.f;
+      float fac[32];
+      if (fast) {
 #pragma unroll
-        for (int r = 0; r < 64; ++r) {
-          const float a = (r < row) ? g[r] * sc_beta[r] * ex2(g2t - sc_g2[r]) : 0.f;
-          At[r * A_LD + row] = a;
+        for (int r4 = 0; r4 < 32; r4 += 4) {
+          const float4 cb = *reinterpret_cast<const float4 *>(sc_tmp + r0 + r4);
+          fac[r4 + 0] = cb.x * rowf; fac[r4 + 1] = cb.y * rowf;
+          fac[r4 + 2] = cb.z * rowf; fac[r4 + 3] = cb.w * rowf;
         }
       } else {
 #pragma unroll
-        for (int r = 0; r < 64; ++r) g[r] = (r <= row) ? p.scale * g[r] * sc_beta[r] * ex2(g2t - sc_g2[r]) : 0.f;
-        st_row64_split(sm + OFF_P, sm + OFF_PL, row, g);
+        for (int r = 0; r < 32; ++r) fac[r] = sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]);
+      }
+      if (quad < 2) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * fac[r]) : 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_P + sw128(t, 4 * half + j), g + 8 * j);
       }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ---- (e) T = (I + A)^{-1} (warps 0-1, column n = tid)
-    if (warp < 2) {
-      const int n = tid;
-      float x[64];
+    // ---- (e) T = (I + A)^{-1}, 16x16-blocked.  Diagonal blocks D_i by forward
+    // substitution (fp32, one thread per column); then, level by level (i - j = 1, 2, 3),
+    // X = sum_{l=j}^{i-1} A_il T_lj and T_ij = -D_i X with warp-level tf32 MMAs, one
+    // warp per 16x8 half block (X is parked in the unused upper block (j, i) of Tf).
+    if (tid < 64) {
+      const int bk = tid >> 4, j = tid & 15, o = 16 * bk;
+      float x[16];
 #pragma unroll
-      for (int m = 0; m < 64; ++m) x[m] = (m == n) ? 1.f : 0.f;
-      // right-looking substitution: x[m] -= A[m][l] x[l] for m > l
+      for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
 #pragma unroll
-      for (int l = 0; l < 63; ++l) {
+      for (int l = 0; l < 15; ++l) {
         const float xl = x[l];
-        const float *col = At + l * A_LD;   // A[.][l]
+        const float *col = At + (o + l) * LD + o;   // A[o + m][o + l], m = 0..15
 #pragma unroll
-        for (int m4 = (l + 1) & ~3; m4 < 64; m4 += 4) {
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+          if (m4 + 3 <= l) continue;
           const float4 a4 = *reinterpret_cast<const float4 *>(col + m4);
           if (m4 + 0 > l) x[m4 + 0] = fmaf(-a4.x, xl, x[m4 + 0]);
           if (m4 + 1 > l) x[m4 + 1] = fmaf(-a4.y, xl, x[m4 + 1]);
@@ -285,147 +334,211 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (m4 + 3 > l) x[m4 + 3] = fmaf(-a4.w, xl, x[m4 + 3]);
         }
       }
-      const float Gn = sc_G[n];
-      __nv_bfloat16 *tt = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TT);
-      __nv_bfloat16 *tp = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TP);
 #pragma unroll
-      for (int m = 0; m < 64; ++m) {
-        const uint32_t off = (sw128(m, n >> 3) >> 1) + (n & 7);
-        tt[off] = __float2bfloat16_rn(x[m]);
-        tp[off] = __float2bfloat16_rn(x[m] * Gn);
+      for (int m = 0; m < 16; ++m) Tf[(o + m) * LD + o + j] = tf32r(x[m]);
+    }
+    __syncthreads();
+    {
+      const int fg = lane >> 2, ft = lane & 3;   // fragment row group / thread in group
+#pragma unroll
+      for (int lev = 1; lev <= 3; ++lev) {
+        if (warp < 2 * (4 - lev)) {
+          const int i = lev + (warp >> 1), jb = i - lev, nh = warp & 1;
+          // X[:, half nh] = A[16i.., 16jb .. 16i) * T[16jb .. 16i, 16jb + 8nh ..]   (K = 16 lev)
+          float xa[4] = {0.f, 0.f, 0.f, 0.f};
+          const int nb = 16 * jb + 8 * nh + fg;
+#pragma unroll
+          for (int ks = 0; ks < 2 * lev; ++ks) {
+            const int k0 = 16 * jb + 8 * ks;
+            uint32_t a[4];
+            a[0] = __float_as_uint(At[(k0 + ft) * LD + 16 * i + fg]);
+            a[1] = __float_as_uint(At[(k0 + ft) * LD + 16 * i + fg + 8]);
+            a[2] = __float_as_uint(At[(k0 + ft + 4) * LD + 16 * i + fg]);
+            a[3] = __float_as_uint(At[(k0 + ft + 4) * LD + 16 * i + fg + 8]);
+            mma_tf32_16x8x8(xa, a, __float_as_uint(Tf[(k0 + ft) * LD + nb]),
+                            __float_as_uint(Tf[(k0 + ft + 4) * LD + nb]));
+          }
+          {
+            const int n = 16 * i + 8 * nh + 2 * ft;     // scratch: upper block (jb, i)
+            Tf[(16 * jb + fg) * LD + n] = tf32r(xa[0]);
+            Tf[(16 * jb + fg) * LD + n + 1] = tf32r(xa[1]);
+            Tf[(16 * jb + fg + 8) * LD + n] = tf32r(xa[2]);
+            Tf[(16 * jb + fg + 8) * LD + n + 1] = tf32r(xa[3]);
+          }
+          __syncwarp();
+          // T_ij[:, half nh] = -D_i X[:, half nh]   (K = 16)
+          float ta[4] = {0.f, 0.f, 0.f, 0.f};
+          const int nx = 16 * i + 8 * nh + fg;
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = 8 * ks;
+            uint32_t a[4];
+            a[0] = __float_as_uint(-Tf[(16 * i + fg) * LD + 16 * i + k0 + ft]);
+            a[1] = __float_as_uint(-Tf[(16 * i + fg + 8) * LD + 16 * i + k0 + ft]);
+            a[2] = __float_as_uint(-Tf[(16 * i + fg) * LD + 16 * i + k0 + ft + 4]);
+            a[3] = __float_as_uint(-Tf[(16 * i + fg + 8) * LD + 16 * i + k0 + ft + 4]);
+            mma_tf32_16x8x8(ta, a, __float_as_uint(Tf[(16 * jb + k0 + ft) * LD + nx]),
+                            __float_as_uint(Tf[(16 * jb + k0 + ft + 4) * LD + nx]));
+          }
+          {
+            const int n = 16 * jb + 8 * nh + 2 * ft;
+            Tf[(16 * i + fg) * LD + n] = tf32r(ta[0]);
+            Tf[(16 * i + fg) * LD + n + 1] = tf32r(ta[1]);
+            Tf[(16 * i + fg + 8) * LD + n] = tf32r(ta[2]);
+            Tf[(16 * i + fg + 8) * LD + n + 1] = tf32r(ta[3]);
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // T and T Diag(Gamma) as bf16 tiles (rows m, 16 columns per thread); upper part zero
+    {
+      const int m = tid >> 2, n0 = (tid & 3) * 16;
+      float tv[16], tg[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int n = n0 + e;
+        tv[e] = (n <= m) ? tv[e] : 0.f;
+        tg[e] = tv[e] * sc_G[n];
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        st_chunk_bf16(sm + OFF_ZT + 8192 + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
+        st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
       }
     }
     fence_async_smem();
     __syncthreads();
 
-    // ---- (f) MMA2: W = T Diag(Gamma) K, U' = T V
+    // ---- (f) MMA2: W = T Diag(Gamma) K ; lanes 64-127 of YE = T V (lanes 0-63 = 0)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_TT);
+      const uint32_t tp = smem_u32(sm + OFF_TP), zt = smem_u32(sm + OFF_ZT);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
-                 ID_M64_N128_KMN, kk > 0);
+        mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024), ID_W, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_E, sdesc(tt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024),
-                 ID_M64_N64_KMN, kk > 0);
+        mma_bf16(tmem + COL_YE, sdesc(zt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), ID_U, kk > 0);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
     mma_phase ^= 1;
     tc_fence_after();
 
-    // ---- (g) W (M64 layout: warp w, lanes 0-15 hold rows 16w + lane) -> bf16 tile
+    // ---- (g) -W (M64 layout: rows 16 quad + lane for lane < 16) -> fp16, columns 64 half ..;
+    // and the fp16 copy of Diag(scale Gamma) Q (the T scratch that shared this tile is dead)
     {
-      float w[64];
-      tmem_ld64(tmem + lane_base + COL_W, w);
-      if (lane < 16) st_row64(sm + OFF_W, warp * 16 + lane, w);
-      tmem_ld64(tmem + lane_base + COL_W + 64, w);
-      if (lane < 16) st_row64(sm + OFF_W + 8192, warp * 16 + lane, w);
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int idx = it * NTHREADS + tid;
+        const int kb = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+        const uint32_t off = sw128(r, j);
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4 *>(kq_ptr + kb * 16384 + 8192 + off), x);
+        const float f = p.scale * sc_G[r];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] *= f;
+        st_chunk_f16(sm + OFF_QW + kb * 16384 + off, x);
+      }
+    }
+    {
+      float w[32];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+        if (lane < 16) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            smax = fmaxf(smax, fabsf(w[e]));
+            w[e] = -w[e];
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_chunk_f16(sm + OFF_QW + half * 16384 + 8192 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        }
+      }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---- (h) MMA3: E = U' - W (S0hi + S0lo) ; Y = Q (S0hi + S0lo)
+    // ---- (h) MMA3: YE += [Diag(scale Gamma) Q; -W] S0
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t wt = smem_u32(sm + OFF_W), qt = kq + 8192;
+      const uint32_t qw = smem_u32(sm + OFF_QW);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t st = part ? sl_tile : s_tile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + COL_E, sdesc(wt + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                   sdesc(st + kk * 2048, 8192, 1024), ID_M64_N64_KMN_NEG, 1);
-      }
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t st = part ? sl_tile : s_tile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + COL_Y, sdesc(qt + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc(st + kk * 2048, 8192, 1024), ID_M64_N64_KMN, part + kk > 0);
-      }
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(s_tile + kk * 2048, 8192, 1024), ID_YE, 1);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
     mma_phase ^= 1;
     tc_fence_after();
 
-    // ---- (i) E -> bf16 tiles E and Diag(w) E  (rows r = 16w + lane)
-    {
-      float e[64];
-      tmem_ld64(tmem + lane_base + COL_E, e);
-      if (lane < 16) {
-        const int r = warp * 16 + lane;
-        st_row64_split(sm + OFF_E, sm + OFF_EL, r, e);
-        const float wr = sc_wf[r];
+    // ---- (i) E (lanes 64-127) -> fp16 tiles E and Diag(w) E
+    if (quad >= 2) {
+      float e[32];
+      tmem_ld32(tmem + lane_base + COL_YE + 32 * half, e);
+      const int r = row - 64;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) e[j] *= wr;
-        st_row64_split(sm + OFF_EW, sm + OFF_EWL, r, e);
-      }
+      for (int j = 0; j < 32; ++j) smax = fmaxf(smax, fabsf(e[j]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_E + sw128(r, 4 * half + j), e + 8 * j);
+      const float wr = sc_wf[r];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) e[j] *= wr;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_EW + sw128(r, 4 * half + j), e + 8 * j);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---- (j) MMA4: dS = K^T Diag(w) (Ehi + Elo) ; Z = Phi Ehi + Phi Elo + Plo Ehi
+    // ---- (j) MMA4: dS = K^T Diag(w) E ; YE += [P; *] E
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ew = smem_u32(sm + OFF_EW), ewl = smem_u32(sm + OFF_EWL);
-      const uint32_t et = smem_u32(sm + OFF_E), etl = smem_u32(sm + OFF_EL);
-      const uint32_t pt = smem_u32(sm + OFF_P), ptl = smem_u32(sm + OFF_PL);
+      const uint32_t k16 = smem_u32(sm + OFF_K16), ew = smem_u32(sm + OFF_EW);
+      const uint32_t et = smem_u32(sm + OFF_E), pt = smem_u32(sm + OFF_P);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t bt = part ? ewl : ew;
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_S, sdesc(k16 + kk * 2048, 8192, 1024), sdesc(ew + kk * 2048, 8192, 1024), ID_DS,
+                 kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_S, sdesc(kq + kk * 2048, 16384, 1024), sdesc(bt + kk * 2048, 8192, 1024),
-                   ID_M128_N64_MNMN, part + kk > 0);
-      }
-#pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        const uint32_t at = part == 2 ? ptl : pt;
-        const uint32_t bt = part == 1 ? etl : et;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_Z, sdesc(at + kk * 32, 16, 1024), sdesc(bt + kk * 2048, 8192, 1024),
-                   ID_M64_N64_KMN, part + kk > 0);
-      }
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_PE, 1);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
     mma_phase ^= 1;
     tc_fence_after();
 
-    // ---- (k) state update (row i = tid) and output rows (16w + lane)
+    // ---- (k) state update (all lanes) and output rows (lanes 0-63)
     {
-      float d[64];
-      tmem_ld64(tmem + lane_base + COL_S, d);
+      float d[32];
+      tmem_ld32(tmem + lane_base + COL_S + 32 * half, d);
       const float gc = ex2(sc_g2[63]);
 #pragma unroll
-      for (int j = 0; j < 64; ++j) S[j] = fmaf(gc, S[j], d[j]);
-      st_row64_split(sm + OFF_S, sm + OFF_SL, tid, S);
-      float y[64];
-      tmem_ld64(tmem + lane_base + COL_Y, y);
-      tmem_ld64(tmem + lane_base + COL_Z, d);
-      const int tr = (warp * 16 + lane) & 63;
-      const float fy = p.scale * sc_G[tr];
+      for (int j = 0; j < 32; ++j) {
+        S[j] = fmaf(gc, S[j], d[j]);
+        smax = fmaxf(smax, fabsf(S[j]));
+      }
 #pragma unroll
-      for (int j = 0; j < 64; ++j) d[j] = fmaf(fy, y[j], d[j]);
-      const int t = t0 + warp * 16 + lane;
-      if (lane < 16 && t < p.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + v0);
+      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
+      if (quad < 2) {
+        tmem_ld32(tmem + lane_base + COL_YE + 32 * half, d);
+        const int t = t0 + row;
+        if (t < p.T) {
+          uint8_t *dst = reinterpret_cast<uint8_t *>(
+              p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + v0 + 32 * half);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(d[8 * j + 0], d[8 * j + 1]);
-          u.y = pack_bf16x2(d[8 * j + 2], d[8 * j + 3]);
-          u.z = pack_bf16x2(d[8 * j + 4], d[8 * j + 5]);
-          u.w = pack_bf16x2(d[8 * j + 6], d[8 * j + 7]);
-          dst[j] = u;
+          for (int j = 0; j < 4; ++j) st_chunk_bf16(dst + 16 * j, d + 8 * j);
         }
       }
     }
@@ -438,11 +551,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 
   if (bad) {
-    if (tid == 0) atomicExch(&g_gdr_device_error, 1);
-  } else if (p.s_final) {
-    float4 *dst = reinterpret_cast<float4 *>(p.s_final + ((static_cast<size_t>(b) * p.H + h) * DK + tid) * p.dv + v0);
+    if (tid == 0) atomicOr(&g_gdr_device_error, 1);
+  } else {
+    if (smax > F16_SAFE) atomicOr(&g_gdr_device_error, 2);
+    if (p.s_final) {
+      float4 *dst = reinterpret_cast<float4 *>(
+          p.s_final + ((static_cast<size_t>(b) * p.H + h) * DK + row) * p.dv + v0 + 32 * half);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+      for (int j = 0; j < 8; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace gdr {
@@ -91,6 +92,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  tmem_ld16(taddr, v);
+  tmem_ld16(taddr + 16, v + 16);
+  tmem_wait_ld();
+}
+
 // 64 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   tmem_ld16(taddr, v);
@@ -127,6 +135,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor of tcgen05.mma kind::f16: fp16 x fp16 -> fp32.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false) {
+  return (1u << 4)                                  // D format: f32; A, B format 0: f16
+         | ((neg_a ? 1u : 0u) << 13)
+         | ((a_mn ? 1u : 0u) << 15)
+         | ((b_mn ? 1u : 0u) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A * B, issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -142,6 +160,23 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// ---------------------------------------------------------------- warp-level MMA (tf32)
+// D (16x8, f32) += A (16x8, tf32, row) * B (8x8, tf32, col).  Fragment layout per
+// lane (g = lane / 4, t = lane % 4): a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]},
+// b = {B[t][g], B[t+4][g]}, d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // ---------------------------------------------------------------- small math
@@ -171,6 +206,25 @@ __device__ __forceinline__ void st_row64(uint8_t *tile, uint32_t r, const float 
     u.w = pack_bf16x2(x[8 * j + 6], x[8 * j + 7]);
     *reinterpret_cast<uint4 *>(tile + sw128(r, j)) = u;
   }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Store 8 floats as one 16-byte chunk of bf16 / fp16 values.
+__device__ __forceinline__ void st_chunk_bf16(uint8_t *addr, const float *x) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]); u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]); u.w = pack_bf16x2(x[6], x[7]);
+  *reinterpret_cast<uint4 *>(addr) = u;
+}
+__device__ __forceinline__ void st_chunk_f16(uint8_t *addr, const float *x) {
+  uint4 u;
+  u.x = pack_f16x2(x[0], x[1]); u.y = pack_f16x2(x[2], x[3]);
+  u.z = pack_f16x2(x[4], x[5]); u.w = pack_f16x2(x[6], x[7]);
+  *reinterpret_cast<uint4 *>(addr) = u;
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float *x) {
