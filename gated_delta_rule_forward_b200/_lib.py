@@ -19,7 +19,7 @@ EXPORTS = (
 )
 
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_ALIGNMENT",
-          4: "GDR_ERR_CUDA", 5: "GDR_ERR_TIMEOUT"}
+          4: "GDR_ERR_CUDA", 5: "GDR_ERR_TIMEOUT", 6: "GDR_ERR_RANGE"}
 
 
 class FwdArgs(ctypes.Structure):

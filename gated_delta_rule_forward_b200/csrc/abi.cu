@@ -87,6 +87,7 @@ const char *gdr_status_string(gdr_status_t s) {
     case GDR_ERR_ALIGNMENT: return "GDR_ERR_ALIGNMENT";
     case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
     case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+    case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
   }
   return "GDR_UNKNOWN_STATUS";
 }
@@ -96,7 +97,8 @@ const char *gdr_last_error(void) { return g_last_error.c_str(); }
 gdr_status_t gdr_device_status(void *stream) {
   const int e = gdr_read_device_error(static_cast<cudaStream_t>(stream));
   if (e < 0) return fail(GDR_ERR_CUDA, "synchronisation or symbol read failed");
-  if (e > 0) return fail(GDR_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  if (e & 1) return fail(GDR_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  if (e & 2) return fail(GDR_ERR_RANGE, "a chunked-kernel operand left its representable range");
   return GDR_OK;
 }
 

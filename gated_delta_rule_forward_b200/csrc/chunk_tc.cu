@@ -39,12 +39,9 @@
 // 6.5e4; a kernel that sees larger values raises the range flag that
 // gdr_device_status() reports.  T, its Gamma-scaled copy and raw q, k, v stay
 // bf16.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "chunk_tc.cuh"
+#include "chunk_common.cuh"
+#include "tma_host.cuh"
 #include "tc_util.cuh"
 
 // Device-side error word, read and cleared by gdr_device_status():
@@ -77,7 +74,6 @@ constexpr uint32_t OFF_EW = 172032;     // fp16 Diag(w) E
 constexpr uint32_t OFF_TF = OFF_QW;     // fp32 T during the solve, 64 x 72 (aliases Qg / -W)
 constexpr uint32_t OFF_S = 180224;      // fp16 S0 [i][v], 128 rows
 constexpr uint32_t OFF_A = 196608;      // fp32 A^T [r][t], 64 x 72
-constexpr uint32_t LD = 72;             // row stride (floats) of A^T and T: conflict-free MMA fragments
 constexpr uint32_t OFF_SC = OFF_A + 64 * LD * 4;   // scalars: 5 x 64 floats
 constexpr uint32_t OFF_BAR = OFF_SC + 5 * 64 * 4;    // 3 mbarriers + TMEM slot
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
@@ -106,8 +102,6 @@ struct Params {
   float eps, scale;
 };
 
-// Round to tf32 and keep as float: the solve stores its operands pre-rounded.
-__device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
 
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -311,86 +305,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
 
-    // ---- (e) T = (I + A)^{-1}, 16x16-blocked.  Diagonal blocks D_i by forward
-    // substitution (fp32, one thread per column); then, level by level (i - j = 1, 2, 3),
-    // X = sum_{l=j}^{i-1} A_il T_lj and T_ij = -D_i X with warp-level tf32 MMAs, one
-    // warp per 16x8 half block (X is parked in the unused upper block (j, i) of Tf).
-    if (tid < 64) {
-      const int bk = tid >> 4, j = tid & 15, o = 16 * bk;
-      float x[16];
-#pragma unroll
-      for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
-#pragma unroll
-      for (int l = 0; l < 15; ++l) {
-        const float xl = x[l];
-        const float *col = At + (o + l) * LD + o;   // A[o + m][o + l], m = 0..15
-#pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
-          if (m4 + 3 <= l) continue;
-          const float4 a4 = *reinterpret_cast<const float4 *>(col + m4);
-          if (m4 + 0 > l) x[m4 + 0] = fmaf(-a4.x, xl, x[m4 + 0]);
-          if (m4 + 1 > l) x[m4 + 1] = fmaf(-a4.y, xl, x[m4 + 1]);
-          if (m4 + 2 > l) x[m4 + 2] = fmaf(-a4.z, xl, x[m4 + 2]);
-          if (m4 + 3 > l) x[m4 + 3] = fmaf(-a4.w, xl, x[m4 + 3]);
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < 16; ++m) Tf[(o + m) * LD + o + j] = tf32r(x[m]);
-    }
-    __syncthreads();
-    {
-      const int fg = lane >> 2, ft = lane & 3;   // fragment row group / thread in group
-#pragma unroll
-      for (int lev = 1; lev <= 3; ++lev) {
-        if (warp < 2 * (4 - lev)) {
-          const int i = lev + (warp >> 1), jb = i - lev, nh = warp & 1;
-          // X[:, half nh] = A[16i.., 16jb .. 16i) * T[16jb .. 16i, 16jb + 8nh ..]   (K = 16 lev)
-          float xa[4] = {0.f, 0.f, 0.f, 0.f};
-          const int nb = 16 * jb + 8 * nh + fg;
-#pragma unroll
-          for (int ks = 0; ks < 2 * lev; ++ks) {
-            const int k0 = 16 * jb + 8 * ks;
-            uint32_t a[4];
-            a[0] = __float_as_uint(At[(k0 + ft) * LD + 16 * i + fg]);
-            a[1] = __float_as_uint(At[(k0 + ft) * LD + 16 * i + fg + 8]);
-            a[2] = __float_as_uint(At[(k0 + ft + 4) * LD + 16 * i + fg]);
-            a[3] = __float_as_uint(At[(k0 + ft + 4) * LD + 16 * i + fg + 8]);
-            mma_tf32_16x8x8(xa, a, __float_as_uint(Tf[(k0 + ft) * LD + nb]),
-                            __float_as_uint(Tf[(k0 + ft + 4) * LD + nb]));
-          }
-          {
-            const int n = 16 * i + 8 * nh + 2 * ft;     // scratch: upper block (jb, i)
-            Tf[(16 * jb + fg) * LD + n] = tf32r(xa[0]);
-            Tf[(16 * jb + fg) * LD + n + 1] = tf32r(xa[1]);
-            Tf[(16 * jb + fg + 8) * LD + n] = tf32r(xa[2]);
-            Tf[(16 * jb + fg + 8) * LD + n + 1] = tf32r(xa[3]);
-          }
-          __syncwarp();
-          // T_ij[:, half nh] = -D_i X[:, half nh]   (K = 16)
-          float ta[4] = {0.f, 0.f, 0.f, 0.f};
-          const int nx = 16 * i + 8 * nh + fg;
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const int k0 = 8 * ks;
-            uint32_t a[4];
-            a[0] = __float_as_uint(-Tf[(16 * i + fg) * LD + 16 * i + k0 + ft]);
-            a[1] = __float_as_uint(-Tf[(16 * i + fg + 8) * LD + 16 * i + k0 + ft]);
-            a[2] = __float_as_uint(-Tf[(16 * i + fg) * LD + 16 * i + k0 + ft + 4]);
-            a[3] = __float_as_uint(-Tf[(16 * i + fg + 8) * LD + 16 * i + k0 + ft + 4]);
-            mma_tf32_16x8x8(ta, a, __float_as_uint(Tf[(16 * jb + k0 + ft) * LD + nx]),
-                            __float_as_uint(Tf[(16 * jb + k0 + ft + 4) * LD + nx]));
-          }
-          {
-            const int n = 16 * jb + 8 * nh + 2 * ft;
-            Tf[(16 * i + fg) * LD + n] = tf32r(ta[0]);
-            Tf[(16 * i + fg) * LD + n + 1] = tf32r(ta[1]);
-            Tf[(16 * i + fg + 8) * LD + n] = tf32r(ta[2]);
-            Tf[(16 * i + fg + 8) * LD + n + 1] = tf32r(ta[3]);
-          }
-        }
-        __syncthreads();
-      }
-    }
+    // ---- (e) T = (I + A)^{-1}
+    solve_unit_lower_64(At, Tf, tid, warp, lane);
     // T and T Diag(Gamma) as bf16 tiles (rows m, 16 columns per thread); upper part zero
     {
       const int m = tid >> 2, n0 = (tid & 3) * 16;
@@ -569,33 +485,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// [B, T, H, D] bf16 tensor, box of 64 (D) x 1 (H) x 64 (T) x 1 (B), 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int D) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 64, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int VAR>
 cudaError_t launch_variant(const FwdProblem &p, cudaStream_t stream, std::string *err) {
   // per call: the attribute is per device, and callers may switch devices
@@ -629,7 +518,7 @@ cudaError_t launch_variant(const FwdProblem &p, cudaStream_t stream, std::string
 
 bool gdr_chunk_tc_supported(int variant, int dk, int dv) {
   using namespace gdr;
-  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA;
+  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA;
   return v && dk == 128 && (dv == 64 || dv == 128);
 }
 
@@ -641,6 +530,7 @@ cudaError_t gdr_launch_chunk_tc(const gdr::FwdProblem &p, cudaStream_t stream, s
     case kDeltaNet: return tc::launch_variant<kDeltaNet>(p, stream, err);
     case kGatedDeltaNet: return tc::launch_variant<kGatedDeltaNet>(p, stream, err);
     case kKLA: return tc::launch_variant<kKLA>(p, stream, err);
+    case kKDA: return gdr_launch_chunk_chan(p, stream, err);
     default: *err = "variant not covered: "; return cudaErrorInvalidValue;
   }
 }
@@ -650,5 +540,7 @@ int gdr_read_device_error(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
   if (cudaMemcpyFromSymbol(&h, g_gdr_device_error, sizeof(int)) != cudaSuccess) return -1;
   if (h) cudaMemcpyToSymbol(g_gdr_device_error, &zero, sizeof(int));
-  return h;
+  const int hc = gdr_read_chan_error();
+  if (hc < 0) return -1;
+  return h | hc;
 }

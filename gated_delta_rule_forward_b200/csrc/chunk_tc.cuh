@@ -13,3 +13,6 @@ cudaError_t gdr_launch_chunk_tc(const gdr::FwdProblem &p, cudaStream_t stream, s
 // Synchronise `stream`, then read and clear the device error word (1 when a
 // bounded wait inside a kernel gave up, 0 otherwise, -1 on a CUDA error).
 int gdr_read_device_error(cudaStream_t stream);
+// Channel-wise decay kernel (chunk_tc_chan.cu) and its error word.
+cudaError_t gdr_launch_chunk_chan(const gdr::FwdProblem &p, cudaStream_t stream, std::string *err);
+int gdr_read_chan_error();

@@ -150,6 +150,12 @@ def decode_step(q, k, v, state, *, variant, beta=None, log_g=None, erase_b=None,
     return out
 
 
+def device_status(stream=None, device=None) -> None:
+    """Synchronise and raise GdrError if a kernel reported a timeout or a range fault."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    check(lib().gdr_device_status(_stream(stream, dev)))
+
+
 def forward_launches(variant, dtype, B, T, H, dk, dv, chunk=0) -> int:
     """Kernel launches one forward call makes (host-only query)."""
     return int(lib().gdr_forward_launches(variant_id(variant), _DTYPES[dtype], B, T, H, dk, dv, chunk))

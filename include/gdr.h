@@ -77,7 +77,8 @@ typedef enum {
     GDR_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for */
     GDR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
     GDR_ERR_CUDA = 4,          /* a CUDA launch or driver call failed */
-    GDR_ERR_TIMEOUT = 5        /* reserved for bounded device-side waits */
+    GDR_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (see gdr_device_status) */
+    GDR_ERR_RANGE = 6          /* a chunked-kernel operand left its representable range */
 } gdr_status_t;
 
 /* Forward-call tensors.  Unused entries are NULL. */
@@ -142,10 +143,17 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
 
 /*
  * Synchronises `stream`, then reads and clears the library's device-side
- * error word.  Returns GDR_ERR_TIMEOUT if a bounded wait inside a kernel
- * (an mbarrier wait that ran past its limit of about a second) gave up since
- * the last call -- that kernel then skipped its remaining work and released
- * its tensor memory -- GDR_ERR_CUDA if the synchronisation failed, else GDR_OK.
+ * error word.  Returns, since the previous call:
+ *   GDR_ERR_TIMEOUT  a bounded wait inside a kernel (an mbarrier wait past its
+ *                    limit of about a second) gave up; that kernel skipped its
+ *                    remaining work and released its tensor memory;
+ *   GDR_ERR_RANGE    a chunked-kernel operand left its range: an fp16 carry
+ *                    operand (state, residual, W) above 6e4 in magnitude, or a
+ *                    channel-wise decay spanning more than 2^120 within one
+ *                    64-token chunk; the results of that call are unreliable
+ *                    and chunk=1 (per-token fp32) is the safe path;
+ *   GDR_ERR_CUDA     the synchronisation failed;
+ *   GDR_OK           otherwise.
  */
 gdr_status_t gdr_device_status(void *stream);
 
