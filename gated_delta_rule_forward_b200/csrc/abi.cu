@@ -34,23 +34,47 @@ gdr_status_t check_cuda(cudaError_t e, const char *what) {
 bool valid_variant(int v) { return v >= GDR_DELTANET && v <= GDR_KLA; }
 bool valid_dim(int d) { return d == 64 || d == 128; }
 
-enum class Kernel { None, Token, ChunkTC };
+enum class Kernel { None, Token, ChunkTC, Split };
 
-// Which kernel a forward call runs, or None with a status and reason.
-Kernel select_forward(int variant, int dtype, int dk, int dv, int chunk, gdr_status_t *st,
-                      std::string *why) {
+bool split_ok(int variant, int dtype, int dk, int dv) {
+  return dtype == GDR_BF16 && gdr_split_supported(variant, dk, dv);
+}
+
+// Which kernel a forward call runs, or None with a status and reason.  `ws`
+// is the workspace the caller passes; the automatic choice takes the
+// two-kernel path only when the workspace is large enough for it.
+Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk, size_t ws,
+                      gdr_status_t *st, std::string *why) {
   *st = GDR_OK;
   const bool tc = dtype == GDR_BF16 && gdr_chunk_tc_supported(variant, dk, dv);
+  const bool sp = split_ok(variant, dtype, dk, dv);
+  const size_t need = sp ? gdr_split_workspace_bytes(B, T, H, dv) : 0;
   if (chunk == 1) return Kernel::Token;
-  if (chunk == 0) return tc ? Kernel::ChunkTC : Kernel::Token;
+  if (chunk == 0) {
+    if (sp && ws >= need) return Kernel::Split;
+    return tc ? Kernel::ChunkTC : Kernel::Token;
+  }
   if (chunk == 64) {
     if (tc) return Kernel::ChunkTC;
     *st = GDR_ERR_UNSUPPORTED;
     *why = "chunk=64 tensor-core kernel needs bf16 I/O and a supported (variant, dk, dv)";
     return Kernel::None;
   }
+  if (chunk == 65) {
+    if (!sp) {
+      *st = GDR_ERR_UNSUPPORTED;
+      *why = "chunk=65 two-kernel path needs bf16 I/O, dk = 128 and DeltaNet / Gated DeltaNet / KLA";
+      return Kernel::None;
+    }
+    if (ws < need) {
+      *st = GDR_ERR_INVALID_ARG;
+      *why = "chunk=65 needs gdr_forward_workspace_size() bytes of workspace";
+      return Kernel::None;
+    }
+    return Kernel::Split;
+  }
   *st = GDR_ERR_INVALID_ARG;
-  *why = "chunk must be 0 (auto), 1 (per-token) or 64 (chunked tensor-core)";
+  *why = "chunk must be 0 (auto), 1 (per-token), 64 (chunked, one kernel) or 65 (chunked, two kernels)";
   return Kernel::None;
 }
 
@@ -102,25 +126,35 @@ gdr_status_t gdr_device_status(void *stream) {
   return GDR_OK;
 }
 
-size_t gdr_forward_workspace_size(int, int, int, int, int, int, int, int) { return 0; }
+size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  if (!valid_variant(variant) || !valid_dim(dk) || !valid_dim(dv) || B <= 0 || T <= 0 || H <= 0) return 0;
+  if ((chunk == 0 || chunk == 65) && split_ok(variant, dtype, dk, dv)) return gdr_split_workspace_bytes(B, T, H, dv);
+  return 0;
+}
+
+// The kernel a call with a workspace of gdr_forward_workspace_size() bytes runs.
+static Kernel planned_kernel(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  gdr_status_t st;
+  std::string why;
+  const size_t ws = gdr_forward_workspace_size(variant, dtype, B, T, H, dk, dv, chunk);
+  return select_forward(variant, dtype, B, T, H, dk, dv, chunk, ws, &st, &why);
+}
 
 int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
   if (!valid_variant(variant) || (dtype != 0 && dtype != 1) || !valid_dim(dk) || !valid_dim(dv)) return 0;
   if (B < 0 || T < 0 || H < 0) return 0;
-  gdr_status_t st;
-  std::string why;
-  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  const Kernel kern = planned_kernel(variant, dtype, B, T, H, dk, dv, chunk);
   if (kern == Kernel::None) return 0;
   if ((long)B * H == 0) return 0;
   if (T == 0) return 1;  // state copy or clear
+  if (kern == Kernel::Split) return 2;
   return kern == Kernel::ChunkTC ? gdr_chunk_tc_launches(B, T, H, dk, dv) : 1;
 }
 
 const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
   if (gdr_forward_launches(variant, dtype, B, T, H, dk, dv, chunk) == 0 && (long)B * H * T != 0) return "none";
-  gdr_status_t st;
-  std::string why;
-  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  const Kernel kern = planned_kernel(variant, dtype, B, T, H, dk, dv, chunk);
+  if (kern == Kernel::Split) return "chunk64_split";
   if (kern == Kernel::ChunkTC) return "chunk64_tc";
   if (kern == Kernel::Token) return dtype == GDR_BF16 ? "token_bf16io" : "token_f32io";
   return "none";
@@ -129,14 +163,14 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
 gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                  const gdr_fwd_args_t *a, float eps, float scale, int chunk,
                                  void *workspace, size_t workspace_bytes, void *stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   gdr_status_t st = validate_common(variant, dtype, dk, dv);
   if (st != GDR_OK) return st;
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
   if (!a) return fail(GDR_ERR_INVALID_ARG, "args is NULL");
+  if (!workspace) workspace_bytes = 0;
+  if (workspace && !aligned16(workspace)) return fail(GDR_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   std::string why;
-  const Kernel kern = select_forward(variant, dtype, dk, dv, chunk, &st, &why);
+  const Kernel kern = select_forward(variant, dtype, B, T, H, dk, dv, chunk, workspace_bytes, &st, &why);
   if (kern == Kernel::None) return fail(st, why);
   if ((long)B * H == 0) return GDR_OK;  // nothing to do
   if (T > 0) {
@@ -171,6 +205,12 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
   p.beta = a->beta; p.log_g = a->log_g; p.erase_b = a->erase_b; p.write_w = a->write_w;
   p.s0 = a->initial_state; p.s_final = a->final_state; p.o = a->o;
   p.eps = eps; p.scale = scale;
+  if (kern == Kernel::Split) {
+    std::string err;
+    const cudaError_t e = gdr_launch_split(p, workspace, s, &err);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_split: " + err + cudaGetErrorString(e));
+    return GDR_OK;
+  }
   if (kern == Kernel::ChunkTC) {
     std::string err;
     const cudaError_t e = gdr_launch_chunk_tc(p, s, &err);

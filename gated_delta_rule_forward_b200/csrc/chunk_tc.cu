@@ -541,6 +541,7 @@ int gdr_read_device_error(cudaStream_t stream) {
   if (cudaMemcpyFromSymbol(&h, g_gdr_device_error, sizeof(int)) != cudaSuccess) return -1;
   if (h) cudaMemcpyToSymbol(g_gdr_device_error, &zero, sizeof(int));
   const int hc = gdr_read_chan_error();
-  if (hc < 0) return -1;
-  return h | hc;
+  const int hs = gdr_read_split_error();
+  if (hc < 0 || hs < 0) return -1;
+  return h | hc | hs;
 }

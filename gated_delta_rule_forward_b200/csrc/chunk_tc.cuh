@@ -16,3 +16,8 @@ int gdr_read_device_error(cudaStream_t stream);
 // Channel-wise decay kernel (chunk_tc_chan.cu) and its error word.
 cudaError_t gdr_launch_chunk_chan(const gdr::FwdProblem &p, cudaStream_t stream, std::string *err);
 int gdr_read_chan_error();
+// Two-kernel path (chunk_split.cu): chunk-parallel preparation + sequential carry.
+bool gdr_split_supported(int variant, int dk, int dv);
+size_t gdr_split_workspace_bytes(int B, int T, int H, int dv);
+cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err);
+int gdr_read_split_error();

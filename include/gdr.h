@@ -96,9 +96,12 @@ typedef struct {
 } gdr_fwd_args_t;
 
 /*
- * Bytes of device workspace gdr_forward_chunked needs for this problem.  The
- * current kernels keep everything on chip and return 0; callers should still
- * ask and pass a buffer of at least this size.
+ * Bytes of device workspace gdr_forward_chunked uses for this problem and
+ * `chunk` choice: B * H * ceil(T/64) records of 25 KB + 8 KB per 64 value
+ * columns for the two-kernel chunked path (chunk 0 or 65 with bf16 I/O,
+ * dk = 128, DeltaNet / Gated DeltaNet / KLA), 0 otherwise.  The workspace is
+ * caller-owned scratch, overwritten by every call; its contents are not
+ * needed after the call completes on the stream.
  */
 size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
                                   int dk, int dv, int chunk);
@@ -106,15 +109,25 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
 /*
  * Whole-sequence forward of B sequences of T tokens and H heads.
  *
- * chunk selects the algorithm:
- *   0  automatic: the chunked tensor-core kernel (tcgen05 + TMEM + TMA, C = 64)
- *      where it exists for (variant, dtype, dk, dv), else the per-token kernel;
+ * chunk selects the algorithm (all chunked paths use C = 64 tokens per chunk
+ * and tcgen05 tensor cores with TMEM accumulators fed by TMA):
+ *   0  automatic: the two-kernel chunked path when it covers the case and the
+ *      workspace is at least gdr_forward_workspace_size() bytes, else the
+ *      one-kernel chunked path where it exists, else the per-token kernel;
  *   1  the per-token kernel (fp32 state in registers, exact fp32 arithmetic,
  *      any supported shape; the path used for fp32 I/O);
- *   64 the chunked tensor-core kernel only (GDR_ERR_UNSUPPORTED where absent).
- * Shapes: B, T, H >= 1; dk in {64, 128}; dv in {64, 128}.
- * eps is used by KLA only; scale multiplies q.
- * workspace may be NULL when gdr_forward_workspace_size(...) is 0.
+ *   64 the one-kernel chunked path (each CTA prepares and carries its chunks;
+ *      no workspace): DeltaNet, Gated DeltaNet, KLA and KDA with bf16 I/O,
+ *      dk = 128;
+ *   65 the two-kernel chunked path: a chunk-parallel preparation kernel (the
+ *      S-independent products of every chunk, into the workspace) then the
+ *      sequential carry kernel: DeltaNet, Gated DeltaNet, KLA with bf16 I/O,
+ *      dk = 128; needs the workspace.
+ * A chunk value whose path does not cover the case returns GDR_ERR_UNSUPPORTED.
+ * Shapes: B, T, H >= 0; dk in {64, 128}; dv in {64, 128}.  T = 0 copies
+ * initial_state to final_state (or clears it); B * H = 0 does nothing.
+ * eps is used by KLA only; scale multiplies q.  workspace must be 16-byte
+ * aligned; it may be NULL (with workspace_bytes ignored) for paths that use none.
  */
 gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                  const gdr_fwd_args_t *args, float eps, float scale, int chunk,

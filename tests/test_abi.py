@@ -139,5 +139,22 @@ def test_decode_validation(L):
     assert dec(variant=0, log_g=None) == 4
 
 
-def test_workspace_is_zero(L):
-    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 0
+def test_workspace_sizes(L):
+    # two-kernel path: one 41 KB record per (b, h, 64-token chunk) for dv = 128
+    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * 41984
+    assert L.gdr_forward_workspace_size(1, 1, 2, 65, 3, 128, 64, 65) == 2 * 3 * 2 * (41984 - 8192)
+    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 64) == 0   # one-kernel path
+    assert L.gdr_forward_workspace_size(1, 0, 8, 2048, 8, 128, 128, 0) == 0    # fp32: per-token
+    assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 0    # KDA: one kernel
+    assert L.gdr_forward_kernel_name(1, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
+    assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == 2
+    assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_tc"
+
+
+def test_split_needs_workspace(L):
+    assert fwd(L, chunk=65) == 1                      # no workspace passed
+    a = args()
+    assert L.gdr_forward_chunked(1, 1, 2, 8, 2, 128, 128, ctypes.byref(a), 1e-6, 1.0, 65,
+                                 ctypes.c_void_p(FAKE), 1 << 20, None) == 4   # reaches the launch
+    assert L.gdr_forward_chunked(1, 1, 2, 8, 2, 128, 128, ctypes.byref(a), 1e-6, 1.0, 65,
+                                 ctypes.c_void_p(MISALIGNED), 1 << 20, None) == 3
