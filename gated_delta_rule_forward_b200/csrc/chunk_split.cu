@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     mma_commit(bar_mma);
   }
   if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+  bad = __syncthreads_or(bad);
   mma_phase ^= 1;
   tc_fence_after();
 
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     mma_commit(bar_mma);
   }
   if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+  bad = __syncthreads_or(bad);
   mma_phase ^= 1;
   tc_fence_after();
 
