@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libgdr.so")
 EXPORTS = (
     "gdr_forward_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
     "gdr_forward_launches", "gdr_forward_kernel_name", "gdr_status_string",
-    "gdr_last_error", "gdr_version", "gdr_device_status",
+    "gdr_last_error", "gdr_version", "gdr_device_status", "gdr_forward_chunked_noalloc",
 )
 
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_ALIGNMENT",
@@ -46,6 +46,8 @@ def lib() -> ctypes.CDLL:
             L.gdr_forward_workspace_size.restype = sz
             L.gdr_forward_chunked.argtypes = [i] * 7 + [ctypes.POINTER(FwdArgs), f, f, i, vp, sz, vp]
             L.gdr_forward_chunked.restype = i
+            L.gdr_forward_chunked_noalloc.argtypes = [i] * 7 + [ctypes.POINTER(FwdArgs), f, f, vp]
+            L.gdr_forward_chunked_noalloc.restype = i
             L.gdr_decode_step.argtypes = [i] * 6 + [vp] * 3 + [vp] * 4 + [vp, vp, f, f, vp]
             L.gdr_decode_step.restype = i
             L.gdr_forward_launches.argtypes = [i] * 8

@@ -220,6 +220,40 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
   return check_cuda(gdr_launch_token_forward(p, s), "token_fwd launch");
 }
 
+gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                                         const gdr_fwd_args_t *a, float eps, float scale, void *stream) {
+  gdr_status_t st = validate_common(variant, dtype, dk, dv);
+  if (st != GDR_OK) return st;
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
+  if (!a) return fail(GDR_ERR_INVALID_ARG, "args is NULL");
+  if (!split_ok(variant, dtype, dk, dv))
+    return fail(GDR_ERR_UNSUPPORTED,
+                "the no-allocation entry point covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O and dk = 128");
+  const size_t need = gdr_split_workspace_bytes(B, T, H, dv);
+  const size_t have = gdr_split_fixed_scratch_bytes();
+  if (need > have)
+    return fail(GDR_ERR_UNSUPPORTED,
+                "problem needs " + std::to_string(need) + " bytes of scratch but the fixed scratch holds " +
+                    std::to_string(have) + " (B * H * ceil(T / 64) must be at most " +
+                    std::to_string(have / (need / ((size_t)B * H * ((T + 63) / 64)))) + " for this dv)");
+  if ((long)B * H == 0 || T == 0) return gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, a, eps, scale, 65,
+                                                             nullptr, 0, stream);
+  if (!a->q || !a->k || !a->v || !a->o) return fail(GDR_ERR_INVALID_ARG, "q, k, v and o are required");
+  const void *io[4] = {a->q, a->k, a->v, a->o};
+  for (const void *p : io)
+    if (!aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "q, k, v and o must be 16-byte aligned");
+  st = validate_gates(variant, a->beta, a->log_g, a->erase_b, a->write_w);
+  if (st != GDR_OK) return st;
+  if ((a->initial_state && !aligned16(a->initial_state)) || (a->final_state && !aligned16(a->final_state)))
+    return fail(GDR_ERR_ALIGNMENT, "state pointers must be 16-byte aligned");
+  if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be >= 0");
+  if (injected_launch_fault()) return fail(GDR_ERR_CUDA, "injected launch failure (GDR_FAULT=launch)");
+  void *scratch = nullptr;
+  const cudaError_t e = gdr_split_fixed_scratch(&scratch);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("fixed scratch lookup: ") + cudaGetErrorString(e));
+  return gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, a, eps, scale, 65, scratch, have, stream);
+}
+
 gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv, const void *q, const void *k,
                              const void *v, const float *beta, const float *log_g, const float *erase_b,
                              const float *write_w, float *state, void *o, float eps, float scale, void *stream) {

@@ -21,6 +21,8 @@
 //     REC_U   fp16 U' per 64-column value slice                  8 KB x NS
 //     REC_P   fp16 P (rows t, columns r)                          8 KB
 //     REC_SC  fp32 scale Gamma_t [64], w_r [64], Gamma_C          1 KB
+#include <mutex>
+
 #include "chunk_common.cuh"
 #include "chunk_tc.cuh"
 #include "tc_util.cuh"
@@ -28,6 +30,15 @@
 
 // Device-side error word of this file (see gdr_device_status()).
 __device__ int g_gdr_split_error = 0;
+
+// Fixed scratch for gdr_forward_chunked_noalloc(): the two-kernel path's
+// workspace for callers that cannot allocate device memory.  It is part of
+// this library's device image, so every GPU that loads the library holds it
+// until the process exits.  All calls share it; the preparation kernel fully
+// rewrites the records a call uses before the carry kernel reads them, so
+// nothing needs clearing between calls, and calls that overlap on the GPU race.
+constexpr size_t kFixedScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_split_fixed_scratch[kFixedScratchBytes];
 
 namespace gdr {
 namespace tc {
@@ -602,4 +613,28 @@ int gdr_read_split_error() {
   if (cudaMemcpyFromSymbol(&h, g_gdr_split_error, sizeof(int)) != cudaSuccess) return -1;
   if (h) cudaMemcpyToSymbol(g_gdr_split_error, &zero, sizeof(int));
   return h;
+}
+
+size_t gdr_split_fixed_scratch_bytes() { return kFixedScratchBytes; }
+
+// Device address of the fixed scratch on the current device.  Host code only
+// holds a stand-in for the array, so the address is looked up with
+// cudaGetSymbolAddress, once per device, while that device is current.
+cudaError_t gdr_split_fixed_scratch(void **ptr) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_split_fixed_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }

@@ -21,3 +21,6 @@ bool gdr_split_supported(int variant, int dk, int dv);
 size_t gdr_split_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err);
 int gdr_read_split_error();
+// Fixed scratch of the no-allocation entry point (chunk_split.cu).
+size_t gdr_split_fixed_scratch_bytes();
+cudaError_t gdr_split_fixed_scratch(void **ptr);

@@ -134,6 +134,35 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Forward for callers that cannot allocate device memory at call time: a
+ * serving runtime whose device memory is planned up front and that forbids
+ * allocation on its request path, or a host program that drives this
+ * library without a device allocator of its own.  It runs the two-kernel
+ * chunked path (chunk = 65 of gdr_forward_chunked) with the library's own
+ * fixed scratch instead of a caller workspace, and allocates nothing.  The
+ * pages have no counterpart to this entry point; it is a deployment
+ * convenience.
+ *
+ * Arguments, layouts and results are those of gdr_forward_chunked.  It covers
+ * DeltaNet, Gated DeltaNet and KLA with bf16 I/O, dk = 128, dv in {64, 128};
+ * anything else returns GDR_ERR_UNSUPPORTED.
+ *
+ * The fixed scratch is a 32 MiB device array in the library's device image:
+ * every GPU that loads the library holds it until the process exits.  A call
+ * needs B * H * ceil(T / 64) records of 41 KB (dv = 128) or 33 KB (dv = 64),
+ * i.e. B * H * ceil(T / 64) <= 799 (dv = 128) or <= 992 (dv = 64); larger
+ * problems return GDR_ERR_UNSUPPORTED with the limit in gdr_last_error().
+ * The first call on each device looks up the array's device address (and may
+ * load the library's device code); make that first call before any stream
+ * capture.  All calls share the array and each call rewrites what it uses
+ * before reading it, so nothing needs clearing; calls whose execution
+ * overlaps on the GPU (different streams, or different host threads) race on
+ * the array and must be serialised by the caller.
+ */
+gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                                         const gdr_fwd_args_t *args, float eps, float scale, void *stream);
+
+/*
  * One recurrent decode token for N independent sequences and H heads.
  * q, k [N,H,dk]; v, o [N,H,dv] (I/O dtype); beta [N,H]; log_g [N,H] or
  * [N,H,dk]; erase_b, write_w [N,H,dk]; state [N,H,dk,dv] fp32, read and
