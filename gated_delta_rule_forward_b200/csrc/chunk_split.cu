@@ -312,6 +312,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 }
 
 // ------------------------------------------------------------------ carry kernel
+// Software-pipelined over chunks: the critical path is MMA3(c) -> E -> dS(c)
+// -> S -> MMA3(c+1); the fp16 copies for chunk c+1 are made while MMA4(c)
+// runs, and the output rows of chunk c are written while MMA3(c+1) runs.
+// TMEM output tiles and the Diag(w) K copy are double-buffered for that.
 namespace carry {
 constexpr uint32_t STAGE = 82944;       // 81 KB per chunk stage
 constexpr uint32_t S_KQ = 0;            // bf16 raw [Kb0 | Qb0 | Kb1 | Qb1] (TMA)
@@ -319,16 +323,16 @@ constexpr uint32_t S_QW = 32768;        // fp16 [Qg b0 | -W b0 | Qg b1 | -W b1] 
 constexpr uint32_t S_P = 65536;         // fp16 P (bulk); the U' tile follows as rows 64-127 of [P; *]
 constexpr uint32_t S_U = 73728;         // fp16 U' of this slice (bulk)
 constexpr uint32_t S_SC = 81920;        // fp32 scale Gamma_t [64], w_r [64], Gamma_C (bulk)
-constexpr uint32_t OFF_KT = 2 * STAGE;  // fp16 Diag(w) K [Kb0 | Kb1]
-constexpr uint32_t OFF_E = OFF_KT + 16384;
+constexpr uint32_t OFF_KT = 2 * STAGE;  // 2 x fp16 Diag(w) K [Kb0 | Kb1]
+constexpr uint32_t OFF_E = OFF_KT + 2 * 16384;
 constexpr uint32_t OFF_S = OFF_E + 8192;
 constexpr uint32_t OFF_BAR = OFF_S + 16384;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(STAGE % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_S % 1024 == 0, "alignment");
-constexpr uint32_t COL_YE = 0;    // M128 x 64
-constexpr uint32_t COL_S = 64;    // M128 x 64
-constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t COL_YE = 0;    // 2 x (M128 x 64): lanes 0-63 Qg S0 + P E, lanes 64-127 -W S0
+constexpr uint32_t COL_S = 128;   // M128 x 64: dS
+constexpr uint32_t TMEM_COLS = 256;
 }  // namespace carry
 
 struct CarryParams {
@@ -351,9 +355,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int sl = blockIdx.x, v0 = 64 * sl, h = blockIdx.y, b = blockIdx.z;
   const int NS = p.dv / 64, NC = p.NC;
 
-  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [2]
-  uint64_t *bar_mma = bar_full + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_full + 3);
+  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [2] chunk inputs
+  uint64_t *bar_e = bar_full + 2;                                    // MMA3 done
+  uint64_t *bar_s = bar_full + 3;                                    // dS done
+  uint64_t *bar_o = bar_full + 4;                                    // P E done
+  uint64_t *bar_drain = bar_full + 5;                                // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_full + 6);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -362,7 +369,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (tid == 0) {
     mbar_init(&bar_full[0], 1);
     mbar_init(&bar_full[1], 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar_e, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -383,8 +393,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   const size_t rb = rec_bytes(NS);
   const uint8_t *recs = p.ws + (static_cast<size_t>(b) * p.H + h) * NC * rb;
+  const uint32_t s_tile = smem_u32(sm + OFF_S), e_tile = smem_u32(sm + OFF_E);
 
+  // load phases issued into / seen landing in stage 0 (low 16 bits) and 1 (high 16 bits)
+  uint32_t n_issued = 0, n_landed = 0;
   auto issue_chunk = [&](int c, int s) {
+    n_issued += 1u << (16 * s);
     uint8_t *st = sm + s * STAGE;
     const uint8_t *rec = recs + c * rb;
     uint64_t *bar = &bar_full[s];
@@ -399,29 +413,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bulk_load(st + S_U, rec + rec_u(NS) + sl * 8192, 8192, bar);
     bulk_load(st + S_SC, rec + rec_sc(NS), 1024, bar);
   };
-  if (tid == 0) {
-    issue_chunk(0, 0);
-    if (NC > 1) issue_chunk(1, 1);
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
-  fence_async_smem();
-  __syncthreads();
-
-  uint32_t mma_phase = 0;
-  int bad = 0;
-  float smax = 0.f;
-  const uint32_t s_tile = smem_u32(sm + OFF_S);
-
-  for (int c = 0; c < NC; ++c) {
-    const int s = c & 1;
+  // fp16 Diag(scale Gamma) Q into the stage and fp16 Diag(w) K into buffer kbuf
+  // (1024 + 1024 sixteen-byte chunks, 8 per thread)
+  auto convert = [&](int s, int kbuf) {
     uint8_t *st = sm + s * STAGE;
     const float *rs = reinterpret_cast<const float *>(st + S_SC);
-
-    if (!mbar_wait(&bar_full[s], (c >> 1) & 1)) bad = 1;
-    if (__syncthreads_or(bad)) break;
-
-    // fp16 Diag(scale Gamma) Q into the stage, fp16 Diag(w) K (1024 + 1024 chunks, 8 per thread)
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       const int u = it * NTHREADS + tid;
@@ -432,29 +428,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float f = rs[isq ? r : 64 + r];
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] *= f;
-      st_chunk_f16(isq ? st + S_QW + kb * 16384 + off : sm + OFF_KT + kb * 8192 + off, x);
+      st_chunk_f16(isq ? st + S_QW + kb * 16384 + off : sm + OFF_KT + kbuf * 16384 + kb * 8192 + off, x);
     }
-    fence_async_smem();
-    __syncthreads();
-
-    // MMA3: YE = [Qg; -W] S0 -> lanes 0-63: Qg S0, lanes 64-127: -W S0
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qw = smem_u32(st + S_QW);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(s_tile + kk * 2048, 8192, 1024), idesc_f16(128, 64, false, true), kk > 0);
-      mma_commit(bar_mma);
-    }
-    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
-    mma_phase ^= 1;
+  };
+  // YE[yb] = [Qg; -W] S0 of stage s
+  auto issue_mma3 = [&](int s, int yb) {
     tc_fence_after();
+    const uint32_t qw = smem_u32(sm + s * STAGE + S_QW);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tmem + COL_YE + 64 * yb, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+               sdesc(s_tile + kk * 2048, 8192, 1024), idesc_f16(128, 64, false, true), kk > 0);
+    mma_commit(bar_e);
+  };
 
-    // E = U' - W S0 (lanes 64-127) -> fp16
+  int bad = 0;
+  float smax = 0.f;
+  if (tid == 0) {
+    issue_chunk(0, 0);
+    if (NC > 1) issue_chunk(1, 1);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
+  if (mbar_wait(&bar_full[0], 0)) n_landed += 1;
+  else bad = 1;
+  bad = __syncthreads_or(bad);
+  if (!bad) convert(0, 0);
+  fence_async_smem();
+  bad = __syncthreads_or(bad);
+  if (!bad && tid == 0) issue_mma3(0, 0);
+
+  for (int c = 0; c < NC && !bad; ++c) {
+    const int s = c & 1, yb = c & 1;
+    uint8_t *st = sm + s * STAGE;
+    const float *rs = reinterpret_cast<const float *>(st + S_SC);
+    const uint32_t ye = tmem + COL_YE + 64 * yb;
+
+    // (1) E = U' - W S0 (lanes 64-127) -> fp16
+    if (!mbar_wait(bar_e, c & 1)) bad = 1;
+    tc_fence_after();
     if (quad >= 2) {
       float e[32], u[8];
-      tmem_ld32(tmem + lane_base + COL_YE + 32 * half, e);
+      tmem_ld32(lane_base + ye + 32 * half, e);
       const int r = row - 64;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -477,27 +492,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    if ((bad = __syncthreads_or(bad))) break;
 
-    // MMA4: dS = (Diag(w) K)^T E ; YE += [P; *] E
+    // (2) dS = (Diag(w) K)^T E ; YE[yb] += [P; *] E
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t kt = smem_u32(sm + OFF_KT), et = smem_u32(sm + OFF_E), pt = smem_u32(st + S_P);
+      const uint32_t kt = smem_u32(sm + OFF_KT + yb * 16384), pt = smem_u32(st + S_P);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_S, sdesc(kt + kk * 2048, 8192, 1024), sdesc(et + kk * 2048, 8192, 1024),
+        mma_bf16(tmem + COL_S, sdesc(kt + kk * 2048, 8192, 1024), sdesc(e_tile + kk * 2048, 8192, 1024),
                  idesc_f16(128, 64, true, true), kk > 0);
+      mma_commit(bar_s);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024),
+        mma_bf16(ye, sdesc(pt + kk * 32, 16, 1024), sdesc(e_tile + kk * 2048, 8192, 1024),
                  idesc_f16(128, 64, false, true), 1);
-      mma_commit(bar_mma);
+      mma_commit(bar_o);
     }
-    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
-    mma_phase ^= 1;
-    tc_fence_after();
 
-    // state update (all lanes) and output rows (lanes 0-63)
+    // (3) while MMA4 runs: the next chunk's fp16 copies
+    if (c + 1 < NC) {
+      if (!mbar_wait(&bar_full[s ^ 1], ((c + 1) >> 1) & 1)) {
+        bad = 1;
+      } else {
+        n_landed += 1u << (16 * (s ^ 1));
+        convert(s ^ 1, yb ^ 1);
+      }
+    }
+
+    // (4) state update: S = Gamma_C S + dS -> fp16 tile; then MMA3 of the next chunk
+    if (!mbar_wait(bar_s, c & 1)) bad = 1;
+    tc_fence_after();
     {
       float d[32];
       tmem_ld32(tmem + lane_base + COL_S + 32 * half, d);
@@ -509,25 +534,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
-      if (quad < 2) {
-        tmem_ld32(tmem + lane_base + COL_YE + 32 * half, d);
-        const int t = c * C + row;
-        if (t < p.T) {
-          uint8_t *dst = reinterpret_cast<uint8_t *>(
-              p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + v0 + 32 * half);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) st_chunk_bf16(dst + 16 * j, d + 8 * j);
-        }
-      }
     }
     fence_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(bad)) break;
+    if ((bad = __syncthreads_or(bad))) break;
+    if (tid == 0 && c + 1 < NC) issue_mma3(s ^ 1, yb ^ 1);
+
+    // (5) while MMA3 of the next chunk runs: output rows of this chunk (lanes 0-63)
+    if (!mbar_wait(bar_o, c & 1)) bad = 1;
+    tc_fence_after();
+    if (quad < 2) {
+      float d[32];
+      tmem_ld32(lane_base + ye + 32 * half, d);
+      const int t = c * C + row;
+      if (t < p.T) {
+        uint8_t *dst = reinterpret_cast<uint8_t *>(
+            p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + v0 + 32 * half);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_bf16(dst + 16 * j, d + 8 * j);
+      }
+    }
+    tc_fence_before();
+    if ((bad = __syncthreads_or(bad))) break;
     if (tid == 0 && c + 2 < NC) issue_chunk(c + 2, s);
   }
 
   if (bad) {
-    if (tid == 0) atomicOr(&g_gdr_split_error, 1);
+    // a wait gave up: report it, then let this CTA's MMAs and copies in
+    // flight finish (each wait again bounded) before TMEM is released
+    if (tid == 0) {
+      atomicOr(&g_gdr_split_error, 1);
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0);
+      for (int st = 0; st < 2; ++st) {
+        const uint32_t got = (n_landed >> (16 * st)) & 0xffff, sent = (n_issued >> (16 * st)) & 0xffff;
+        if (got < sent) mbar_wait(&bar_full[st], got & 1);
+      }
+    }
   } else {
     if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
     if (p.s_final) {
