@@ -6,21 +6,28 @@
 // KLA update rule and implementation; "Gated DeltaNet-2", technical core):
 //     T = (I + A)^{-1},  W = T Diag(Gamma) K,  U' = T V,  E = U' - W S0
 //     O = Diag(scale Gamma) Q S0 + P E,   S_C = Gamma_C S0 + K^T Diag(w) E.
-// Everything that does not depend on S0 -- A, P, the solve, W, U' -- is the
-// bulk of the work and is independent across chunks.  The preparation kernel
-// computes it with one CTA per (batch, head, chunk) over the whole machine (two
-// CTAs per SM) instead of inside the sequential sweep, and it is shared by all
-// value slices of a head.  The carry kernel then does only what depends on the
-// state: [Diag(scale Gamma) Q; -W] S0, E, K^T Diag(w) E and P E, and the state
-// update, one CTA per (batch, head, 64-column value slice).
+// Everything that does not depend on S0 -- A, P, the solve, W, U' and the
+// scaled copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K -- is the bulk of
+// the work and is independent across chunks.  The preparation kernel computes
+// it with one CTA per (batch, head, chunk) over the whole machine (two CTAs
+// per SM) instead of inside the sequential sweep.  The carry kernel then does
+// only what depends on the state, one CTA per (batch, head), in transposed
+// form so that the state is the tensor-memory operand of every product:
+//     Y_W = S0^T (-W)^T,  Y_Q = S0^T Qg^T,  E^T = U'^T + Y_W,
+//     dS^T = E^T Kt,  O^T = Y_Q + E^T P^T,  S_C^T = Gamma_C S0^T + dS^T.
+// Lane v of tensor memory is value column v; S^T and E^T are written there in
+// fp16 by the threads that own them and read by the MMAs from there, so the
+// sweep moves no operand through shared memory except the record itself.
 //
-// Workspace record per (b, h, chunk), all tile images in the 128-byte-swizzled
-// layout the tensor cores read, so the carry kernel bulk-copies them into
-// shared memory unchanged:
-//     REC_W   fp16 -W, K-major atoms [d_k 0-63 | 64-127]         16 KB
-//     REC_U   fp16 U' per 64-column value slice                  8 KB x NS
-//     REC_P   fp16 P (rows t, columns r)                          8 KB
-//     REC_SC  fp32 scale Gamma_t [64], w_r [64], Gamma_C          1 KB
+// Workspace record per (b, h, chunk).  The tiles the MMAs read are images of
+// the 128-byte-swizzled shared-memory layout, so the carry kernel bulk-copies
+// the whole record into shared memory unchanged:
+//     REC_WQ  fp16 [-W; Qg] per d_k atom: [-W 0-63 | Qg 0-63 | -W 64-127 | Qg 64-127],
+//             rows t, K-major (the N = 128 operand of one product)   32 KB
+//     REC_K   fp16 Kt, rows t, atoms [d_k 0-63 | 64-127] (read as the MN-major operand)  16 KB
+//     REC_P   fp16 P, rows t, columns r                            8 KB
+//     REC_U   fp16 U'^T, rows v, columns t (swizzled 16-byte chunks) 8 KB per 64 values
+//     REC_SC  fp32 Gamma_C, padded to 16 bytes
 #include <mutex>
 
 #include "chunk_common.cuh"
@@ -50,10 +57,12 @@ constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float F16_SAFE = 60000.f;
 
-__host__ __device__ constexpr uint32_t rec_u(int) { return 16384; }
-__host__ __device__ constexpr uint32_t rec_p(int ns) { return 16384 + 8192 * ns; }
-__host__ __device__ constexpr uint32_t rec_sc(int ns) { return rec_p(ns) + 8192; }
-__host__ __device__ constexpr uint32_t rec_bytes(int ns) { return rec_sc(ns) + 1024; }
+constexpr uint32_t REC_WQ = 0;
+constexpr uint32_t REC_K = 32768;
+constexpr uint32_t REC_P = 49152;
+constexpr uint32_t REC_U = 57344;
+__host__ __device__ constexpr uint32_t rec_sc(int ns) { return REC_U + 8192 * ns; }
+__host__ __device__ constexpr uint32_t rec_bytes(int ns) { return rec_sc(ns) + 16; }
 
 // ------------------------------------------------------------------ preparation kernel
 namespace prep {
@@ -69,7 +78,7 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T, "layout");
 constexpr uint32_t COL_G = 0;     // M128 x 64 (dead before W)
 constexpr uint32_t COL_W = 0;     // M64 x 128
-constexpr uint32_t COL_U = 128;   // M64 x dv
+constexpr uint32_t COL_U = 128;   // M128 x 64: U'^T
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prep
 
@@ -120,6 +129,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
     tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
     for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+  }
+  if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
+    for (int i = tid; i < 512; i += NTHREADS)
+      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   // gates: beta_t, cumulative log2 decay, Gamma_t
   if (tid < 64) {
@@ -212,7 +225,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
       for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + rec_p(NS) + sw128(t, 4 * half + j), g + 8 * j);
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
     }
   }
   tc_fence_before();
@@ -239,17 +252,29 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
     }
   }
-  // per-row scalars of the record: scale Gamma_t, w_r, Gamma_C
-  if (tid < 64) {
-    float *rs = reinterpret_cast<float *>(rec + rec_sc(NS));
-    rs[tid] = p.scale * sc_G[tid];
-    rs[64 + tid] = sc_wf[tid];
-    if (tid == 0) rs[128] = sc_G[63];
+  // Gamma_C, and the fp16 copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K
+  // (2048 sixteen-byte chunks in the swizzled image of the bf16 tiles)
+  if (tid == 0) *reinterpret_cast<float4 *>(rec + rec_sc(NS)) = make_float4(sc_G[63], 0.f, 0.f, 0.f);
+  float qkmax = 0.f;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int u = it * NTHREADS + tid;
+    const int isq = u >> 10, kb = (u >> 9) & 1, r = (u >> 3) & 63, j = u & 7;
+    const uint32_t off = sw128(r, j);
+    float x[8];
+    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KQ + kb * 16384 + isq * 8192 + off), x);
+    const float f = isq ? p.scale * sc_G[r] : sc_wf[r];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      x[e] *= f;
+      qkmax = fmaxf(qkmax, fabsf(x[e]));
+    }
+    st_chunk_f16(rec + (isq ? REC_WQ + kb * 16384 + 8192 : REC_K + kb * 8192) + off, x);
   }
   fence_async_smem();
   __syncthreads();
 
-  // MMA2: W = T Diag(Gamma) K (M64 N128); U' = T V (M64 N dv)
+  // MMA2: W = T Diag(Gamma) K (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
   if (!bad && tid == 0) {
     tc_fence_after();
     const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
@@ -257,10 +282,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
                idesc_bf16(64, 128, false, true), kk > 0);
-    const uint32_t id_u = NS == 2 ? idesc_bf16(64, 128, false, true) : idesc_bf16(64, 64, false, true);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_U, sdesc(tt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), id_u, kk > 0);
+      mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+               idesc_bf16(128, 64, true, false), kk > 0);
     mma_commit(bar_mma);
   }
   if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
@@ -268,9 +293,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   mma_phase ^= 1;
   tc_fence_after();
 
-  // -W and U' (M64 layout: rows 16 quad + lane, lane < 16) -> fp16 record tiles.
-  // Column half `half` of W is d_k atom `half`; of U' it is value slice `half`.
-  float wmax = 0.f;
+  // -W (M64 layout: rows 16 quad + lane, lane < 16; column half `half` is d_k
+  // atom `half`) and U'^T (lane v = value column, columns t) -> fp16 record tiles
+  float wmax = qkmax;
   if (!bad) {
     float w[32];
 #pragma unroll
@@ -284,21 +309,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          st_chunk_f16(rec + half * 8192 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
       }
     }
-    if (half < NS) {
+    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
+    if (row < p.dv) {
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tmem + lane_base + COL_U + 64 * half + 32 * part, w);
-        if (lane < 16) {
+      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
 #pragma unroll
-          for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_chunk_f16(rec + rec_u(NS) + half * 8192 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
-        }
-      }
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
     }
   }
   if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
@@ -312,27 +331,30 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 }
 
 // ------------------------------------------------------------------ carry kernel
-// Software-pipelined over chunks: the critical path is MMA3(c) -> E -> dS(c)
-// -> S -> MMA3(c+1); the fp16 copies for chunk c+1 are made while MMA4(c)
-// runs, and the output rows of chunk c are written while MMA3(c+1) runs.
-// TMEM output tiles and the Diag(w) K copy are double-buffered for that.
+// One CTA per (b, h) sweeps the chunks in order, warp-specialised: warp 16
+// issues the record copies and the MMAs; compute warp w (0-15) owns value
+// column v = 32 (w mod 4) + lane of S^T (its tensor-memory lane) and the
+// quarter w / 4 of its d_k range (fp32 registers), of E^T's tokens and of the
+// output tokens.  The two sides hand over through mbarriers only:
+//     issuer:  Y(c) = S^T [-W; Qg]^T -> bar_e      compute: E^T(c) -> bar_ea
+//              dS^T(c), Y_Q += E^T P^T -> bar_s/o           S^T(c) -> bar_sa
+//              record c+2 (after bar_done of c-1)           output rows (c) -> bar_done
+// Y is double-buffered so Y(c+1) runs while the output rows of c are written;
+// records arrive by bulk copy two chunks ahead of their use.
 namespace carry {
-constexpr uint32_t STAGE = 82944;       // 81 KB per chunk stage
-constexpr uint32_t S_KQ = 0;            // bf16 raw [Kb0 | Qb0 | Kb1 | Qb1] (TMA)
-constexpr uint32_t S_QW = 32768;        // fp16 [Qg b0 | -W b0 | Qg b1 | -W b1] (Qg by threads, -W bulk)
-constexpr uint32_t S_P = 65536;         // fp16 P (bulk); the U' tile follows as rows 64-127 of [P; *]
-constexpr uint32_t S_U = 73728;         // fp16 U' of this slice (bulk)
-constexpr uint32_t S_SC = 81920;        // fp32 scale Gamma_t [64], w_r [64], Gamma_C (bulk)
-constexpr uint32_t OFF_KT = 2 * STAGE;  // 2 x fp16 Diag(w) K [Kb0 | Kb1]
-constexpr uint32_t OFF_E = OFF_KT + 2 * 16384;
-constexpr uint32_t OFF_S = OFF_E + 8192;
-constexpr uint32_t OFF_BAR = OFF_S + 16384;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+constexpr int NSTAGE = 3;
+constexpr int NCOMPUTE = 16;
+constexpr int NTHREADS_CARRY = (NCOMPUTE + 1) * 32;
+constexpr uint32_t STAGE = 74752;        // record image (<= 73744 bytes), 1 KB aligned
+constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(STAGE % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_S % 1024 == 0, "alignment");
-constexpr uint32_t COL_YE = 0;    // 2 x (M128 x 64): lanes 0-63 Qg S0 + P E, lanes 64-127 -W S0
-constexpr uint32_t COL_S = 128;   // M128 x 64: dS
-constexpr uint32_t TMEM_COLS = 256;
+static_assert(STAGE % 1024 == 0 && STAGE >= 73744, "stage layout");
+constexpr uint32_t COL_Y = 0;      // 2 x 128: [(-W S0)^T | (Qg S0)^T + (P E)^T], [v][t]
+constexpr uint32_t COL_DS = 256;   // 128: dS^T, [v][i]
+constexpr uint32_t COL_SA = 384;   // 64: fp16 S^T, d_k packed two per column (MMA operand)
+constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column (MMA operand)
+constexpr uint32_t TMEM_COLS = 512;
 }  // namespace carry
 
 struct CarryParams {
@@ -343,241 +365,253 @@ struct CarryParams {
   __nv_bfloat16 *o;
 };
 
-__global__ void __launch_bounds__(NTHREADS, 1)
-    chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const CarryParams p) {
+// Bounded wait that also gives up once another warp has raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const long long start = clock64();
+  while (!mbar_try_wait(bar, phase)) {
+    if (*abort) return false;
+    if (clock64() - start > (1ll << 31)) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
   using namespace carry;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
-  const int row = quad * 32 + lane;
-  const int sl = blockIdx.x, v0 = 64 * sl, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int NS = p.dv / 64, NC = p.NC;
 
-  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [2] chunk inputs
-  uint64_t *bar_e = bar_full + 2;                                    // MMA3 done
-  uint64_t *bar_s = bar_full + 3;                                    // dS done
-  uint64_t *bar_o = bar_full + 4;                                    // P E done
-  uint64_t *bar_drain = bar_full + 5;                                // error path only
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_full + 6);
+  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
+  uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
+  uint64_t *bar_s = bar_e + 1;            // dS^T(c) done
+  uint64_t *bar_o = bar_e + 2;            // E^T P^T (c) done
+  uint64_t *bar_ea = bar_e + 3;           // E^T(c) in tensor memory (16 warps)
+  uint64_t *bar_sa = bar_e + 4;           // S^T in tensor memory (16 warps)
+  uint64_t *bar_done = bar_e + 5;         // chunk c's Y read and stage released (16 warps)
+  uint64_t *bar_drain = bar_e + 6;        // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 7);
+  volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 8);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&bar_full[0], 1);
-    mbar_init(&bar_full[1], 1);
+    for (int i = 0; i < NSTAGE; ++i) mbar_init(&bar_full[i], 1);
     mbar_init(bar_e, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_ea, NCOMPUTE);
+    mbar_init(bar_sa, NCOMPUTE);
+    mbar_init(bar_done, NCOMPUTE);
     mbar_init(bar_drain, 1);
+    *abort = 0;
     fence_mbar_init();
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-  }
-  float S[32];
-  {
-    const float *src =
-        p.s0 ? p.s0 + ((static_cast<size_t>(b) * p.H + h) * DK + row) * p.dv + v0 + 32 * half : nullptr;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float4 f = src ? __ldg(reinterpret_cast<const float4 *>(src) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      S[4 * j] = f.x; S[4 * j + 1] = f.y; S[4 * j + 2] = f.z; S[4 * j + 3] = f.w;
-    }
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-  const size_t rb = rec_bytes(NS);
-  const uint8_t *recs = p.ws + (static_cast<size_t>(b) * p.H + h) * NC * rb;
-  const uint32_t s_tile = smem_u32(sm + OFF_S), e_tile = smem_u32(sm + OFF_E);
+  const uint32_t rb = rec_bytes(NS);
 
-  // load phases issued into / seen landing in stage 0 (low 16 bits) and 1 (high 16 bits)
-  uint32_t n_issued = 0, n_landed = 0;
-  auto issue_chunk = [&](int c, int s) {
-    n_issued += 1u << (16 * s);
-    uint8_t *st = sm + s * STAGE;
-    const uint8_t *rec = recs + c * rb;
-    uint64_t *bar = &bar_full[s];
-    mbar_expect_tx(bar, 4 * 8192 + 2 * 8192 + 8192 + 8192 + 1024);
-    tma_load_4d(st + S_KQ + 0, &tm_k, bar, 0, h, c * C, b);
-    tma_load_4d(st + S_KQ + 8192, &tm_q, bar, 0, h, c * C, b);
-    tma_load_4d(st + S_KQ + 16384, &tm_k, bar, 64, h, c * C, b);
-    tma_load_4d(st + S_KQ + 24576, &tm_q, bar, 64, h, c * C, b);
-    bulk_load(st + S_QW + 8192, rec + 0, 8192, bar);
-    bulk_load(st + S_QW + 24576, rec + 8192, 8192, bar);
-    bulk_load(st + S_P, rec + rec_p(NS), 8192, bar);
-    bulk_load(st + S_U, rec + rec_u(NS) + sl * 8192, 8192, bar);
-    bulk_load(st + S_SC, rec + rec_sc(NS), 1024, bar);
-  };
-  // fp16 Diag(scale Gamma) Q into the stage and fp16 Diag(w) K into buffer kbuf
-  // (1024 + 1024 sixteen-byte chunks, 8 per thread)
-  auto convert = [&](int s, int kbuf) {
-    uint8_t *st = sm + s * STAGE;
-    const float *rs = reinterpret_cast<const float *>(st + S_SC);
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int u = it * NTHREADS + tid;
-      const int isq = u >> 10, kb = (u >> 9) & 1, r = (u >> 3) & 63, j = u & 7;
-      const uint32_t off = sw128(r, j);
-      float x[8];
-      unpack8(*reinterpret_cast<const uint4 *>(st + S_KQ + kb * 16384 + isq * 8192 + off), x);
-      const float f = rs[isq ? r : 64 + r];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] *= f;
-      st_chunk_f16(isq ? st + S_QW + kb * 16384 + off : sm + OFF_KT + kbuf * 16384 + kb * 8192 + off, x);
-    }
-  };
-  // YE[yb] = [Qg; -W] S0 of stage s
-  auto issue_mma3 = [&](int s, int yb) {
-    tc_fence_after();
-    const uint32_t qw = smem_u32(sm + s * STAGE + S_QW);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tmem + COL_YE + 64 * yb, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-               sdesc(s_tile + kk * 2048, 8192, 1024), idesc_f16(128, 64, false, true), kk > 0);
-    mma_commit(bar_e);
-  };
-
-  int bad = 0;
+  // issuer's view of the record copies: stage has a copy in flight / phase parity to wait for
+  uint32_t pend = 0, par = 0;
   float smax = 0.f;
-  if (tid == 0) {
-    issue_chunk(0, 0);
-    if (NC > 1) issue_chunk(1, 1);
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
-  if (mbar_wait(&bar_full[0], 0)) n_landed += 1;
-  else bad = 1;
-  bad = __syncthreads_or(bad);
-  if (!bad) convert(0, 0);
-  fence_async_smem();
-  bad = __syncthreads_or(bad);
-  if (!bad && tid == 0) issue_mma3(0, 0);
+  float S[32];
+  const int quad = warp & 3, part = (warp >> 2) & 3;
+  const int v = quad * 32 + lane;
+  const bool has_v = quad * 32 < p.dv;   // warp-uniform (d_v is 64 or 128)
+  const uint32_t lrow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
 
-  for (int c = 0; c < NC && !bad; ++c) {
-    const int s = c & 1, yb = c & 1;
-    uint8_t *st = sm + s * STAGE;
-    const float *rs = reinterpret_cast<const float *>(st + S_SC);
-    const uint32_t ye = tmem + COL_YE + 64 * yb;
-
-    // (1) E = U' - W S0 (lanes 64-127) -> fp16
-    if (!mbar_wait(bar_e, c & 1)) bad = 1;
-    tc_fence_after();
-    if (quad >= 2) {
-      float e[32], u[8];
-      tmem_ld32(lane_base + ye + 32 * half, e);
-      const int r = row - 64;
+  if (warp == NCOMPUTE) {
+    // ---------------------------------------------------------------- issuer
+    if (lane == 0) {
+      const uint8_t *recs = p.ws + (static_cast<size_t>(b) * p.H + h) * NC * rb;
+      auto issue_chunk = [&](int c) {
+        const int s = c % NSTAGE;
+        mbar_expect_tx(&bar_full[s], rb);
+        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, rb, &bar_full[s]);
+        pend |= 1u << s;
+      };
+      auto wait_full = [&](int c) -> bool {
+        const int s = c % NSTAGE;
+        if (!wait_or_abort(&bar_full[s], (c / NSTAGE) & 1, abort)) return false;
+        pend &= ~(1u << s);
+        par ^= 1u << s;
+        return true;
+      };
+      auto issue_y = [&](int c) {   // Y(c) = S^T [-W; Qg]^T
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(st + S_U + sw128(r, 4 * half + j));
-        const __half2 *hp = reinterpret_cast<const __half2 *>(&raw);
-#pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
-          const float2 f = __half22float2(hp[q2]);
-          u[2 * q2] = f.x;
-          u[2 * q2 + 1] = f.y;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
+                 sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
+                 kk > 0);
+        mma_commit(bar_e);
+      };
+      for (int c = 0; c < NSTAGE && c < NC; ++c) issue_chunk(c);
+      bool ok = wait_or_abort(bar_sa, 0, abort) && wait_full(0);
+      if (ok) issue_y(0);
+      // Waits follow the order in which the compute warps arrive (done(c-1)
+      // before E(c) before S(c)), so no barrier can complete a phase the
+      // issuer has not waited for yet.
+      for (int c = 0; ok && c < NC; ++c) {
+        // chunk c-1 fully consumed: its stage takes record c+2
+        if (c >= 1) {
+          if (!(ok = wait_or_abort(bar_done, (c - 1) & 1, abort))) break;
+          if (c + 2 < NC) issue_chunk(c + 2);
         }
+        // dS^T = E^T Kt ; Y_Q += E^T P^T
+        if (!(ok = wait_or_abort(bar_ea, c & 1, abort))) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
 #pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) {
-          e[8 * j + e8] += u[e8];
-          smax = fmaxf(smax, fabsf(e[8 * j + e8]));
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + COL_DS, tmem + COL_EA + 8 * kk, sdesc(st + REC_K + kk * 2048, 8192, 1024),
+                 idesc_f16(128, 128, false, true), kk > 0);
+        mma_commit(bar_s);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 8 * kk, sdesc(st + REC_P + kk * 32, 16, 1024),
+                 idesc_f16(128, 64, false, false), 1);
+        mma_commit(bar_o);
+        if (c + 1 < NC) {
+          if (!(ok = wait_or_abort(bar_sa, (c + 1) & 1, abort) && wait_full(c + 1))) break;
+          issue_y(c + 1);
         }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_E + sw128(r, 4 * half + j), e + 8 * j);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    if ((bad = __syncthreads_or(bad))) break;
-
-    // (2) dS = (Diag(w) K)^T E ; YE[yb] += [P; *] E
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t kt = smem_u32(sm + OFF_KT + yb * 16384), pt = smem_u32(st + S_P);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_S, sdesc(kt + kk * 2048, 8192, 1024), sdesc(e_tile + kk * 2048, 8192, 1024),
-                 idesc_f16(128, 64, true, true), kk > 0);
-      mma_commit(bar_s);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(ye, sdesc(pt + kk * 32, 16, 1024), sdesc(e_tile + kk * 2048, 8192, 1024),
-                 idesc_f16(128, 64, false, true), 1);
-      mma_commit(bar_o);
-    }
-
-    // (3) while MMA4 runs: the next chunk's fp16 copies
-    if (c + 1 < NC) {
-      if (!mbar_wait(&bar_full[s ^ 1], ((c + 1) >> 1) & 1)) {
-        bad = 1;
-      } else {
-        n_landed += 1u << (16 * (s ^ 1));
-        convert(s ^ 1, yb ^ 1);
-      }
-    }
-
-    // (4) state update: S = Gamma_C S + dS -> fp16 tile; then MMA3 of the next chunk
-    if (!mbar_wait(bar_s, c & 1)) bad = 1;
-    tc_fence_after();
-    {
-      float d[32];
-      tmem_ld32(tmem + lane_base + COL_S + 32 * half, d);
-      const float gc = rs[128];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        S[j] = fmaf(gc, S[j], d[j]);
-        smax = fmaxf(smax, fabsf(S[j]));
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_S + sw128(row, 4 * half + j), S + 8 * j);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    if ((bad = __syncthreads_or(bad))) break;
-    if (tid == 0 && c + 1 < NC) issue_mma3(s ^ 1, yb ^ 1);
-
-    // (5) while MMA3 of the next chunk runs: output rows of this chunk (lanes 0-63)
-    if (!mbar_wait(bar_o, c & 1)) bad = 1;
-    tc_fence_after();
-    if (quad < 2) {
-      float d[32];
-      tmem_ld32(lane_base + ye + 32 * half, d);
-      const int t = c * C + row;
-      if (t < p.T) {
-        uint8_t *dst = reinterpret_cast<uint8_t *>(
-            p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + v0 + 32 * half);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) st_chunk_bf16(dst + 16 * j, d + 8 * j);
-      }
-    }
-    tc_fence_before();
-    if ((bad = __syncthreads_or(bad))) break;
-    if (tid == 0 && c + 2 < NC) issue_chunk(c + 2, s);
-  }
-
-  if (bad) {
-    // a wait gave up: report it, then let this CTA's MMAs and copies in
-    // flight finish (each wait again bounded) before TMEM is released
-    if (tid == 0) {
-      atomicOr(&g_gdr_split_error, 1);
-      mma_commit(bar_drain);
-      mbar_wait(bar_drain, 0);
-      for (int st = 0; st < 2; ++st) {
-        const uint32_t got = (n_landed >> (16 * st)) & 0xffff, sent = (n_issued >> (16 * st)) & 0xffff;
-        if (got < sent) mbar_wait(&bar_full[st], got & 1);
       }
     }
   } else {
-    if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
-    if (p.s_final) {
-      float4 *dst = reinterpret_cast<float4 *>(
-          p.s_final + ((static_cast<size_t>(b) * p.H + h) * DK + row) * p.dv + v0 + 32 * half);
+    // ---------------------------------------------------------------- compute warps
+    {
+      const size_t base = ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+      for (int k = 0; k < 32; ++k)
+        S[k] = (p.s0 != nullptr && has_v) ? __ldg(p.s0 + base + static_cast<size_t>(k) * p.dv) : 0.f;
+    }
+    auto store_state = [&]() {
+      uint32_t r[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
+      tmem_st16(lrow + COL_SA + 16 * part, r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sa);
+    };
+    store_state();
+    for (int c = 0; c < NC; ++c) {
+      uint8_t *st = sm + (c % NSTAGE) * STAGE;
+      const uint32_t y = lrow + COL_Y + 128 * (c & 1);
+
+      // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15
+      bool ok = wait_or_abort(&bar_full[c % NSTAGE], (c / NSTAGE) & 1, abort) &&
+                wait_or_abort(bar_e, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
+        float e[16];
+        tmem_ld16(y + 16 * part, e);
+        tmem_wait_ld();
+        if (has_v) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(st + REC_U + sw128(v, 2 * part + j));
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __half22float2(hp[q2]);
+              e[8 * j + 2 * q2] += f.x;
+              e[8 * j + 2 * q2 + 1] += f.y;
+            }
+          }
+        }
+        uint32_t r[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          smax = fmaxf(smax, fmaxf(fabsf(e[2 * m]), fabsf(e[2 * m + 1])));
+          r[m] = pack_f16x2(e[2 * m], e[2 * m + 1]);
+        }
+        tmem_st8(lrow + COL_EA + 8 * part, r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ea);
+      }
+
+      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31
+      ok = wait_or_abort(bar_s, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
+        const float gc = *reinterpret_cast<const float *>(st + rec_sc(NS));
+        float d[32];
+        tmem_ld32(lrow + COL_DS + 32 * part, d);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          S[m] = fmaf(gc, S[m], d[m]);
+          smax = fmaxf(smax, fabsf(S[m]));
+        }
+        store_state();
+      }
+
+      // output rows: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
+      // through this warp's 1 KB of the stage's (now unused) U'^T tile into 16-byte stores
+      ok = wait_or_abort(bar_o, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
+        float yo[16];
+        tmem_ld16(y + 64 + 16 * part, yo);
+        tmem_wait_ld();
+        if (has_v) {
+          uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            *reinterpret_cast<__nv_bfloat16 *>(tile + m * 64 + lane * 2) = __float2bfloat16_rn(yo[m]);
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
+            const int t = c * C + 16 * part + tr;
+            const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
+            if (t < p.T)
+              *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
+                                         8 * piece) = val;
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_done);
+      }
+    }
+  }
+
+  __syncthreads();
+  const bool failed = *abort != 0;
+  if (failed) {
+    // a wait gave up: report it, then let the MMAs and copies in flight
+    // finish (each wait again bounded) before tensor memory is released
+    if (warp == NCOMPUTE && lane == 0) {
+      atomicOr(&g_gdr_split_error, 1);
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0);
+      for (int s = 0; s < NSTAGE; ++s)
+        if (pend >> s & 1u) mbar_wait(&bar_full[s], par >> s & 1u);
+    }
+  } else if (warp < NCOMPUTE) {
+    if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
+    if (p.s_final != nullptr && has_v) {
+      float *dst = p.s_final + ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
     }
   }
   tc_fence_before();
@@ -620,7 +654,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   cp.T = p.T; cp.H = p.H; cp.dv = p.dv; cp.NC = NC;
   cp.ws = static_cast<const uint8_t *>(ws); cp.s0 = p.s0; cp.s_final = p.s_final;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<<<dim3(p.dv / 64, p.H, p.B), NTHREADS, carry::SMEM_BYTES, stream>>>(mq, mk, cp);
+  chunk_carry_kernel<<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;

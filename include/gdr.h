@@ -97,8 +97,8 @@ typedef struct {
 
 /*
  * Bytes of device workspace gdr_forward_chunked uses for this problem and
- * `chunk` choice: B * H * ceil(T/64) records of 25 KB + 8 KB per 64 value
- * columns for the two-kernel chunked path (chunk 0 or 65 with bf16 I/O,
+ * `chunk` choice: B * H * ceil(T/64) records of 56 KB + 8 KB per 64 value
+ * columns + 16 bytes for the two-kernel chunked path (chunk 0 or 65 with bf16 I/O,
  * dk = 128, DeltaNet / Gated DeltaNet / KLA), 0 otherwise.  The workspace is
  * caller-owned scratch, overwritten by every call; its contents are not
  * needed after the call completes on the stream.
@@ -149,8 +149,8 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
  *
  * The fixed scratch is a 32 MiB device array in the library's device image:
  * every GPU that loads the library holds it until the process exits.  A call
- * needs B * H * ceil(T / 64) records of 41 KB (dv = 128) or 33 KB (dv = 64),
- * i.e. B * H * ceil(T / 64) <= 799 (dv = 128) or <= 992 (dv = 64); larger
+ * needs B * H * ceil(T / 64) records of 73744 bytes (dv = 128) or 65552 bytes
+ * (dv = 64), i.e. B * H * ceil(T / 64) <= 455 (dv = 128) or <= 511 (dv = 64); larger
  * problems return GDR_ERR_UNSUPPORTED with the limit in gdr_last_error().
  * The first call on each device looks up the array's device address (and may
  * load the library's device code); make that first call before any stream

@@ -140,9 +140,10 @@ def test_decode_validation(L):
 
 
 def test_workspace_sizes(L):
-    # two-kernel path: one 41 KB record per (b, h, 64-token chunk) for dv = 128
-    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * 41984
-    assert L.gdr_forward_workspace_size(1, 1, 2, 65, 3, 128, 64, 65) == 2 * 3 * 2 * (41984 - 8192)
+    # two-kernel path: one record per (b, h, 64-token chunk): -W, Qg, Kt (16 KB each),
+    # P (8 KB), U'^T (8 KB per 64 value columns) and Gamma_C (16 bytes)
+    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 16)
+    assert L.gdr_forward_workspace_size(1, 1, 2, 65, 3, 128, 64, 65) == 2 * 3 * 2 * (57344 + 8192 + 16)
     assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 64) == 0   # one-kernel path
     assert L.gdr_forward_workspace_size(1, 0, 8, 2048, 8, 128, 128, 0) == 0    # fp32: per-token
     assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 0    # KDA: one kernel

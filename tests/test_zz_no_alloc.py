@@ -55,11 +55,14 @@ def test_noalloc_matches_workspace_path_twice(variant, dv):
 
 
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
-    B, T, H = 8, 8192, 8                    # 8 * 8 * 128 records > 799
+    B, T, H = 8, 8192, 8                    # 8 * 8 * 128 records, more than 32 MiB holds
+    record = _lib.lib().gdr_forward_workspace_size(1, 1, 1, 64, 1, 128, 128, 65)
+    limit = (32 << 20) // record
+    assert B * H * (T // 64) > limit
     q = torch.empty(1, device="cuda", dtype=torch.bfloat16)
     a = _lib.FwdArgs(q=q.data_ptr(), k=q.data_ptr(), v=q.data_ptr(), beta=q.data_ptr(),
                      log_g=q.data_ptr(), erase_b=None, write_w=None, initial_state=None,
                      final_state=None, o=q.data_ptr())
     st = _lib.lib().gdr_forward_chunked_noalloc(1, 1, B, T, H, 128, 128, ctypes.byref(a), 1e-6, 1.0, None)
     assert st == 2
-    assert "799" in _lib.lib().gdr_last_error().decode()
+    assert str(limit) in _lib.lib().gdr_last_error().decode()
