@@ -50,11 +50,14 @@ WORKLOADS = {
 }
 DEFAULT = "gdn_fwd_350m"
 METRIC = "gated-delta-rule layer tokens/s (fwd, decode) at 1 B200; % of bf16 TC / HBM roofline"
-KERNEL_SOURCES = {
-    "chunk64_tc": ["gated_delta_rule_forward_b200/csrc/chunk_tc.cu"],
-    "token_bf16io": ["gated_delta_rule_forward_b200/csrc/token_fwd.cu"],
-    "token_f32io": ["gated_delta_rule_forward_b200/csrc/token_fwd.cu"],
-    "decode": ["gated_delta_rule_forward_b200/csrc/decode.cu"],
+_CSRC = "gated_delta_rule_forward_b200/csrc/"
+_TC = [_CSRC + f for f in ("chunk_common.cuh", "tc_util.cuh", "tma_host.cuh")]
+KERNEL_SOURCES = {   # sources whose text keys a recorded ncu traffic figure
+    "chunk64_split": [_CSRC + "chunk_split.cu"] + _TC,
+    "chunk64_tc": [_CSRC + "chunk_tc.cu", _CSRC + "chunk_tc_chan.cu"] + _TC,
+    "token_bf16io": [_CSRC + "token_fwd.cu"],
+    "token_f32io": [_CSRC + "token_fwd.cu"],
+    "decode": [_CSRC + "decode.cu"],
 }
 
 
@@ -77,7 +80,8 @@ def source_hash(kernel):
 
 
 def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    """DRAM bytes per step (all launches of one forward / decode call) from a
+    committed ncu summary, if it was taken on the current kernel sources."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -276,7 +280,7 @@ def forward_e2e(name, host, K, W, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
 
 
-def run_decode_workload(name, K, W, world):
+def run_decode_workload(name, K, W, world, e2e=False):
     import gated_delta_rule_forward_b200 as gdr
     from gated_delta_rule_forward_b200.inputs import make_decode_inputs, random_state
     variant, N, _, H, dk, dv = WORKLOADS[name]
@@ -294,6 +298,44 @@ def run_decode_workload(name, K, W, world):
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    s.record()
+    for i in range(K):
+        step(i)
+    e.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    res = {"workload": name, "variant": variant, "N": N, "H": H, "dk": dk, "dv": dv, "kernel": "decode",
+           "launches_per_step": 1, "ms_per_step": ms / K, "launch_ms": ms / K, "tokens_per_step": N,
+           "value": world * N * K / (ms / 1e3), "alg_bytes": decode_bytes(variant, N, H, dk, dv),
+           "wall": (t_wall0, t_wall1)}
+    if e2e:
+        res["e2e"] = decode_e2e(name, steps, state, K, W, world)
+    return res
+
+
+def decode_e2e(name, dev_steps, state, K, W, world):
+    """Public-API decode throughput with host buffers: pinned H2D of the step's
+    token inputs, the step (state resident on the device), D2H of the output."""
+    import gated_delta_rule_forward_b200 as gdr
+    variant, N, _, H, dk, dv = WORKLOADS[name]
+    pinned = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()} for d in dev_steps]
+    o_host = torch.empty(N, H, dv, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values() if v is not None)
+    d2h = o_host.numel() * o_host.element_size()
+
+    def step(i):
+        d = {k: (None if v is None else v.to("cuda", non_blocking=True)) for k, v in pinned[i % len(pinned)].items()}
+        o = gdr.decode_step(d["q"], d["k"], d["v"], state, variant=variant, **gates(d))
+        o_host.copy_(o, non_blocking=True)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for i in range(K):
         step(i)
@@ -301,24 +343,37 @@ def run_decode_workload(name, K, W, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"workload": name, "variant": variant, "N": N, "H": H, "dk": dk, "dv": dv, "kernel": "decode",
-            "launches_per_step": 1, "ms_per_step": ms / K, "launch_ms": ms / K,
-            "value": world * N * K / (ms / 1e3), "alg_bytes": decode_bytes(variant, N, H, dk, dv)}
+    return {"value": world * N * K / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
 
 
 def roofline(res, peaks):
+    """Algorithmic bytes of one call over its event-timed duration.  A call of the
+    two-kernel path is one preparation and one carry launch; the pair is timed
+    together (the workspace between them is not algorithmic traffic)."""
     achieved = res["alg_bytes"] / (res["launch_ms"] / 1e3) / 1e9
     traffic = recorded_traffic(res["kernel"], res["workload"])
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-            "peak_source": peaks["source"], "alg_bytes_per_launch": res["alg_bytes"]}
+            "peak_source": peaks["source"], "alg_bytes_per_launch": res["alg_bytes"],
+            "launches_timed": res["launches_per_step"]}
 
 
 def cpu_baseline(name):
     """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
     import oracle
-    from gated_delta_rule_forward_b200.inputs import make_inputs
+    from gated_delta_rule_forward_b200.inputs import make_decode_inputs, make_inputs, random_state
     variant, B, T, H, dk, dv = WORKLOADS[name]
+    if T is None:   # decode: whole steps of all N sequences
+        d = make_decode_inputs(variant, B, H, 0, dk, dv)
+        S = random_state(B, H, dk, dv, 7)
+        passes, t0 = 0, time.perf_counter()
+        while passes == 0 or time.perf_counter() - t0 < 2.0:
+            _, S = oracle.decode_step(variant, d["q"], d["k"], d["v"], S, **gates(d))
+            passes += 1
+        dt = time.perf_counter() - t0
+        return {"value": passes * B / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                "sample": f"{passes} decode step(s) of all {B} sequences x {H} heads, fp64, {dt:.2f} s wall"}
     d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
     oracle.forward(variant, **{k: (None if v is None else v[:, :64]) for k, v in d.items()})  # build/load
     passes, t0 = 0, time.perf_counter()
@@ -341,7 +396,10 @@ def native(args):
     sampler = ClockSampler(local)
     sampler.start()
     t0 = time.time()
-    main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
+    if WORKLOADS[args.workload][2] is None:
+        main = run_decode_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
+    else:
+        main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
     t1 = time.time()
     also = []
     if not args.no_also:
@@ -363,13 +421,15 @@ def native(args):
     if rank != 0:
         return
     variant, B, T, H, dk, dv = WORKLOADS[args.workload]
+    shape = ({"sequences_per_gpu": B, "heads": H, "dk": dk, "dv": dv, "tokens_per_step": B} if T is None else
+             {"batch_per_gpu": B, "seq_len": T, "heads": H, "dk": dk, "dv": dv})
     line = {
         "metric": METRIC, "value": round(main["value"], 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms_per_step"], 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; q,k L2-normalised, v ~ N(0,1), sigmoid / -softplus gates)",
-        "config": {"workload": args.workload, "variant": variant, "batch_per_gpu": B, "seq_len": T,
-                   "heads": H, "dk": dk, "dv": dv, "global_batch": B * world, "kernel": main["kernel"],
+        "config": {"workload": args.workload, "variant": variant, **shape, "global_batch": B * world,
+                   "kernel": main["kernel"],
                    "state": "fp32", "parallelism": f"dp{world}",
                    "l2": "inputs > L2; two input sets rotated between steps"},
         "roofline": roofline(main, peaks),
@@ -389,20 +449,27 @@ def reference(args):
     if rank != 0:
         return
     import oracle
-    from gated_delta_rule_forward_b200.inputs import make_inputs
+    from gated_delta_rule_forward_b200.inputs import make_decode_inputs, make_inputs, random_state
     variant, B, T, H, dk, dv = WORKLOADS[args.workload]
-    if T is None:
-        raise SystemExit("reference arm supports the forward workloads")
-    d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+    if T is None:   # decode: one step of all N sequences per step
+        d = make_decode_inputs(variant, B, H, 0, dk, dv)
+        S = random_state(B, H, dk, dv, 7)
+        run = lambda: oracle.decode_step(variant, d["q"], d["k"], d["v"], S, **gates(d))
+        tokens = B
+        sample = f"one decode step of all {B} sequences x {H} heads per step, fp64"
+    else:           # forward: one of the B sequences per step
+        d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+        run = lambda: oracle.forward(variant, **d)
+        tokens = T
+        sample = f"1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
     for _ in range(args.warmup):
-        oracle.forward(variant, **d)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.forward(variant, **d)
+        run()
     dt = time.perf_counter() - t0
-    value = T * args.steps / dt
+    value = tokens * args.steps / dt
     cores = oracle.max_threads()
-    sample = f"1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
@@ -422,7 +489,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT, choices=[w for w, v in WORKLOADS.items() if v[2]])
+    ap.add_argument("--workload", default=DEFAULT, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-also", action="store_true", help="only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
