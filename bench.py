@@ -181,11 +181,18 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Maximum of a per-rank scalar (a device time) over all ranks."""
     if world == 1:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cpu" if torch.distributed.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, ms_max, world):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- native arm
@@ -243,7 +250,7 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
         "launch_ms": launch_ms, "tokens_per_step": B * T, "wall": (t_wall0, t_wall1),
         "alg_bytes": fwd_bytes(variant, B, T, H, dk, dv),
     }
-    res["value"] = world * B * T * K / (total_ms / 1e3)
+    res["value"] = job_throughput(B * T, K, total_ms, world)
     if e2e:
         res["e2e"] = forward_e2e(name, host, K, W, world)
     return res
@@ -276,7 +283,7 @@ def forward_e2e(name, host, K, W, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"value": world * B * T * K / (ms / 1e3), "unit": "tokens/s",
+    return {"value": job_throughput(B * T, K, ms, world), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
 
 
@@ -309,7 +316,7 @@ def run_decode_workload(name, K, W, world, e2e=False):
     ms = max_over_ranks(s.elapsed_time(e), world)
     res = {"workload": name, "variant": variant, "N": N, "H": H, "dk": dk, "dv": dv, "kernel": "decode",
            "launches_per_step": 1, "ms_per_step": ms / K, "launch_ms": ms / K, "tokens_per_step": N,
-           "value": world * N * K / (ms / 1e3), "alg_bytes": decode_bytes(variant, N, H, dk, dv),
+           "value": job_throughput(N, K, ms, world), "alg_bytes": decode_bytes(variant, N, H, dk, dv),
            "wall": (t_wall0, t_wall1)}
     if e2e:
         res["e2e"] = decode_e2e(name, steps, state, K, W, world)
@@ -343,7 +350,7 @@ def decode_e2e(name, dev_steps, state, K, W, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"value": world * N * K / (ms / 1e3), "unit": "tokens/s",
+    return {"value": job_throughput(N, K, ms, world), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
 
 
@@ -399,7 +406,8 @@ def native(args):
     if WORKLOADS[args.workload][2] is None:
         main = run_decode_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
     else:
-        main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
+        main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e,
+                                    seed=rank)   # each rank its own sequences
     t1 = time.time()
     also = []
     if not args.no_also:
