@@ -28,6 +28,7 @@
 //     REC_P   fp16 P, rows t, columns r                            8 KB
 //     REC_U   fp16 U'^T, rows v, columns t (swizzled 16-byte chunks) 8 KB per 64 values
 //     REC_SC  fp32 Gamma_C, padded to 16 bytes
+#include <algorithm>
 #include <mutex>
 
 #include "chunk_common.cuh"
@@ -83,7 +84,7 @@ constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prep
 
 struct PrepParams {
-  int T, H, dv, NC;
+  int B, T, H, dv, NC;
   const float *beta, *log_g;
   uint8_t *ws;
   float eps, scale;
@@ -99,13 +100,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int NS = p.dv / 64;
-  const int t0 = c * C;
+  const int total = p.NC * p.H * p.B;   // records, chunk index fastest
 
   uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
   uint64_t *bar_mma = bar_in + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 2);
+  uint64_t *bar_drain = bar_in + 2;     // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);
   float *sc_g2 = sc_beta + 64;
   float *sc_wf = sc_g2 + 64;
@@ -113,214 +114,265 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   float *sc_tmp = sc_G + 64;
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
-  uint8_t *rec = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c) * rec_bytes(NS);
 
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(bar_in, 1);
-    mbar_init(bar_mma, 1);
-    fence_mbar_init();
+  // TMA loads of record r's K, Q and V (thread 0)
+  auto issue_inputs = [&](int r) {
+    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const int t0 = c * C;
     mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
     tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
     tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
     tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
     tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
     for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
-  }
-  if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
-    for (int i = tid; i < 512; i += NTHREADS)
-      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
-  }
-  // gates: beta_t, cumulative log2 decay, Gamma_t
-  if (tid < 64) {
-    const int t = t0 + tid;
-    float lg = 0.f, bt = 0.f;
+  };
+  // log decay and beta of token `tid` of record r (threads 0-63)
+  auto load_gates = [&](int r, float &lg, float &bt) {
+    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const int t = c * C + tid;
+    lg = 0.f;
+    bt = 0.f;
     if (t < p.T) {
       const size_t th = (static_cast<size_t>(b) * p.T + t) * p.H + h;
       if constexpr (scalar_decay(VAR)) lg = __ldg(p.log_g + th);
       bt = __ldg(p.beta + th);
     }
-    float x = lg * LOG2E;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    sc_tmp[tid] = x;
-    sc_beta[tid] = bt;
+  };
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
   }
+  bool in_flight = false;   // thread 0: a record's loads are outstanding on bar_in
+  if (tid == 0) {
+    mbar_init(bar_in, 1);
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    if (static_cast<int>(blockIdx.x) < total) {
+      issue_inputs(blockIdx.x);
+      in_flight = true;
+    }
+  }
+  if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
+    for (int i = tid; i < 512; i += NTHREADS)
+      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  float lg_next = 0.f, bt_next = 0.f;
+  if (tid < 64 && static_cast<int>(blockIdx.x) < total) load_gates(blockIdx.x, lg_next, bt_next);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-  if (tid < 64) {
-    const float g2 = sc_tmp[tid] + (tid >= 32 ? sc_tmp[31] : 0.f);
-    sc_g2[tid] = g2;
-    sc_G[tid] = ex2(g2);
-  }
-  int bad = 0;
-  if (!mbar_wait(bar_in, 0)) bad = 1;
-  bad = __syncthreads_or(bad);
   const uint32_t kq = smem_u32(sm + OFF_KQ);
-  uint32_t mma_phase = 0;
+  uint32_t mma_phase = 0, in_phase = 0;
+  int bad = 0;
+  float wmax = 0.f;
 
-  // MMA1: [K;Q] K^T
-  if (!bad && tid == 0) {
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
-      mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), idesc_bf16(128, 64, false, false), kk > 0);
-    }
-    mma_commit(bar_mma);
-  }
-  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
-  bad = __syncthreads_or(bad);
-  mma_phase ^= 1;
-  tc_fence_after();
-
-  // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
-  if (!bad) {
-    float g[32];
-    tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
-    const int t = row & 63;
-    const int r0 = 32 * half;
-    if constexpr (VAR == kKLA) {
-      if (quad < 2 && (t >> 5) == half) {
-        float kk = 0.f;
-#pragma unroll
-        for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
-        const float eta = sc_beta[t];
-        sc_beta[t] = (eta == 0.f) ? 0.f : eta / (kk + p.eps);   // Kaczmarz step
-      }
-    }
-    __syncthreads();
-    const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
+  // Persistent over records: the next record's loads are issued as soon as
+  // MMA2 has consumed this record's inputs, and land during the epilogue.
+  for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    uint8_t *rec = p.ws + static_cast<size_t>(r) * rec_bytes(NS);
+    // gates: beta_t, cumulative log2 decay, Gamma_t
     if (tid < 64) {
-      sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - sc_g2[tid]);
-      sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - sc_g2[tid]);
+      float x = lg_next * LOG2E;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      sc_tmp[tid] = x;
+      sc_beta[tid] = bt_next;
+      if (r + static_cast<int>(gridDim.x) < total) load_gates(r + gridDim.x, lg_next, bt_next);
     }
     __syncthreads();
-    const float g2t = sc_g2[t];
-    const float rowf = (t >= r0) ? ex2(g2t - sc_g2[r0]) : 0.f;
-    float fac[32];
-    if (fast) {
+    if (tid < 64) {
+      const float g2 = sc_tmp[tid] + (tid >= 32 ? sc_tmp[31] : 0.f);
+      sc_g2[tid] = g2;
+      sc_G[tid] = ex2(g2);
+    }
+    if (!mbar_wait(bar_in, in_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    if (bad) break;
+    in_phase ^= 1;
+    if (tid == 0) in_flight = false;
+
+    // MMA1: [K;Q] K^T
+    if (!bad && tid == 0) {
+      tc_fence_after();
 #pragma unroll
-      for (int r4 = 0; r4 < 32; r4 += 4) {
-        const float4 cb = *reinterpret_cast<const float4 *>(sc_tmp + r0 + r4);
-        fac[r4 + 0] = cb.x * rowf; fac[r4 + 1] = cb.y * rowf;
-        fac[r4 + 2] = cb.z * rowf; fac[r4 + 3] = cb.w * rowf;
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), idesc_bf16(128, 64, false, false), kk > 0);
       }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 32; ++r) fac[r] = sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]);
+      mma_commit(bar_mma);
     }
-    if (quad < 2) {
-#pragma unroll
-      for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * fac[r]) : 0.f;
-    } else {
-#pragma unroll
-      for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // T = (I + A)^{-1}; T and T Diag(Gamma) as bf16 tiles
-  solve_unit_lower_64(At, Tf, tid, warp, lane);
-  {
-    const int m = tid >> 2, n0 = (tid & 3) * 16;
-    float tv[16], tg[16];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
-      tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
-    }
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
-      tg[e] = tv[e] * sc_G[n0 + e];
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
-      st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
-    }
-  }
-  // Gamma_C, and the fp16 copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K
-  // (2048 sixteen-byte chunks in the swizzled image of the bf16 tiles)
-  if (tid == 0) *reinterpret_cast<float4 *>(rec + rec_sc(NS)) = make_float4(sc_G[63], 0.f, 0.f, 0.f);
-  float qkmax = 0.f;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int u = it * NTHREADS + tid;
-    const int isq = u >> 10, kb = (u >> 9) & 1, r = (u >> 3) & 63, j = u & 7;
-    const uint32_t off = sw128(r, j);
-    float x[8];
-    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KQ + kb * 16384 + isq * 8192 + off), x);
-    const float f = isq ? p.scale * sc_G[r] : sc_wf[r];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      x[e] *= f;
-      qkmax = fmaxf(qkmax, fabsf(x[e]));
-    }
-    st_chunk_f16(rec + (isq ? REC_WQ + kb * 16384 + 8192 : REC_K + kb * 8192) + off, x);
-  }
-  fence_async_smem();
-  __syncthreads();
-
-  // MMA2: W = T Diag(Gamma) K (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
-  if (!bad && tid == 0) {
+    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    mma_phase ^= 1;
     tc_fence_after();
-    const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
-               idesc_bf16(64, 128, false, true), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
-               idesc_bf16(128, 64, true, false), kk > 0);
-    mma_commit(bar_mma);
-  }
-  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
-  bad = __syncthreads_or(bad);
-  mma_phase ^= 1;
-  tc_fence_after();
 
-  // -W (M64 layout: rows 16 quad + lane, lane < 16; column half `half` is d_k
-  // atom `half`) and U'^T (lane v = value column, columns t) -> fp16 record tiles
-  float wmax = qkmax;
-  if (!bad) {
-    float w[32];
+    // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
+    if (!bad) {
+      float g[32];
+      tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
+      const int t = row & 63;
+      const int r0 = 32 * half;
+      if constexpr (VAR == kKLA) {
+        if (quad < 2 && (t >> 5) == half) {
+          float kk = 0.f;
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
-      if (lane < 16) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          wmax = fmaxf(wmax, fabsf(w[e]));
-          w[e] = -w[e];
+          for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
+          const float eta = sc_beta[t];
+          sc_beta[t] = (eta == 0.f) ? 0.f : eta / (kk + p.eps);   // Kaczmarz step
         }
+      }
+      __syncthreads();
+      const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
+      if (tid < 64) {
+        sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - sc_g2[tid]);
+        sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - sc_g2[tid]);
+      }
+      __syncthreads();
+      const float g2t = sc_g2[t];
+      const float rowf = (t >= r0) ? ex2(g2t - sc_g2[r0]) : 0.f;
+      float fac[32];
+      if (fast) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        for (int r4 = 0; r4 < 32; r4 += 4) {
+          const float4 cb = *reinterpret_cast<const float4 *>(sc_tmp + r0 + r4);
+          fac[r4 + 0] = cb.x * rowf; fac[r4 + 1] = cb.y * rowf;
+          fac[r4 + 2] = cb.z * rowf; fac[r4 + 3] = cb.w * rowf;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) fac[r] = sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]);
+      }
+      if (quad < 2) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * fac[r]) : 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
       }
     }
-    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
-    if (row < p.dv) {
+    tc_fence_before();
+    __syncthreads();
+
+    // T = (I + A)^{-1}; T and T Diag(Gamma) as bf16 tiles
+    solve_unit_lower_64(At, Tf, tid, warp, lane);
+    {
+      const int m = tid >> 2, n0 = (tid & 3) * 16;
+      float tv[16], tg[16];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+      }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+      for (int e = 0; e < 16; ++e) {
+        tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+        tg[e] = tv[e] * sc_G[n0 + e];
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
+        st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
+      }
     }
+    // Gamma_C, and the fp16 copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K
+    // (2048 sixteen-byte chunks in the swizzled image of the bf16 tiles)
+    if (tid == 0) *reinterpret_cast<float4 *>(rec + rec_sc(NS)) = make_float4(sc_G[63], 0.f, 0.f, 0.f);
+    float qkmax = 0.f;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int u = it * NTHREADS + tid;
+      const int isq = u >> 10, kb = (u >> 9) & 1, r = (u >> 3) & 63, j = u & 7;
+      const uint32_t off = sw128(r, j);
+      float x[8];
+      unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KQ + kb * 16384 + isq * 8192 + off), x);
+      const float f = isq ? p.scale * sc_G[r] : sc_wf[r];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[e] *= f;
+        qkmax = fmaxf(qkmax, fabsf(x[e]));
+      }
+      st_chunk_f16(rec + (isq ? REC_WQ + kb * 16384 + 8192 : REC_K + kb * 8192) + off, x);
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // MMA2: W = T Diag(Gamma) K (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
+    if (!bad && tid == 0) {
+      tc_fence_after();
+      const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
+                 idesc_bf16(64, 128, false, true), kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+                 idesc_bf16(128, 64, true, false), kk > 0);
+      mma_commit(bar_mma);
+    }
+    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    mma_phase ^= 1;
+    tc_fence_after();
+
+    // this record's inputs are consumed: start the next record's loads
+    if (!bad && r + static_cast<int>(gridDim.x) < total && tid == 0) {
+      issue_inputs(r + gridDim.x);
+      in_flight = true;
+    }
+
+    // -W (M64 layout: rows 16 quad + lane, lane < 16; column half `half` is d_k
+    // atom `half`) and U'^T (lane v = value column, columns t) -> fp16 record tiles
+    wmax = fmaxf(wmax, qkmax);
+    if (!bad) {
+      float w[32];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+        if (lane < 16) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            wmax = fmaxf(wmax, fabsf(w[e]));
+            w[e] = -w[e];
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        }
+      }
+      tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
+      if (row < p.dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+      }
+    }
+    // tensor-memory reads done before the next record's MMA1
+    tc_fence_before();
+    __syncthreads();
+    if (bad) break;
   }
-  if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
+
+  if (bad && tid == 0) {
+    // a wait gave up: report it, then let the MMAs and loads in flight
+    // finish (each wait again bounded) before tensor memory is released
+    atomicOr(&g_gdr_split_error, 1);
+    mma_commit(bar_drain);
+    mbar_wait(bar_drain, 0);
+    if (in_flight) mbar_wait(bar_in, in_phase);
+  }
   if (wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
   tc_fence_before();
   __syncthreads();
@@ -626,6 +678,10 @@ template <int VAR>
 cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
+  // all of the unified L1 as shared memory, so that two preparation CTAs fit on an SM
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(chunk_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)carry::SMEM_BYTES);
@@ -641,10 +697,26 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   }
   const int NC = (p.T + C - 1) / C;
   PrepParams pp;
-  pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = static_cast<uint8_t *>(ws);
   pp.eps = p.eps; pp.scale = p.scale;
-  chunk_prep_kernel<VAR><<<dim3(NC, p.H, p.B), NTHREADS, prep::SMEM_BYTES, stream>>>(mq, mk, mv, pp);
+  // persistent grid: as many CTAs as fit on the device at once, none idle
+  int dev = 0, sms = 0, per_sm = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_prep_kernel<VAR>, NTHREADS, prep::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    *err = "occupancy query: ";
+    return e;
+  }
+  // The occupancy query reports one CTA per SM for this kernel, yet two are
+  // resident at once (105 KB of shared memory and 128 x 256 registers each),
+  // so the grid is sized for at least two.  A CTA that does not fit only
+  // starts later; no CTA waits on another.
+  const long long records = static_cast<long long>(NC) * p.H * p.B;
+  const int grid = static_cast<int>(std::min<long long>(records, static_cast<long long>(std::max(per_sm, 2)) * sms));
+  chunk_prep_kernel<VAR><<<grid, NTHREADS, prep::SMEM_BYTES, stream>>>(mq, mk, mv, pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = "prep launch: ";
