@@ -48,7 +48,7 @@ Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int d
   *st = GDR_OK;
   const bool tc = dtype == GDR_BF16 && gdr_chunk_tc_supported(variant, dk, dv);
   const bool sp = split_ok(variant, dtype, dk, dv);
-  const size_t need = sp ? gdr_split_workspace_bytes(B, T, H, dv) : 0;
+  const size_t need = sp ? gdr_split_workspace_bytes(variant, B, T, H, dv) : 0;
   if (chunk == 1) return Kernel::Token;
   if (chunk == 0) {
     if (sp && ws >= need) return Kernel::Split;
@@ -63,7 +63,7 @@ Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int d
   if (chunk == 65) {
     if (!sp) {
       *st = GDR_ERR_UNSUPPORTED;
-      *why = "chunk=65 two-kernel path needs bf16 I/O, dk = 128 and DeltaNet / Gated DeltaNet / KLA";
+      *why = "chunk=65 two-kernel path needs bf16 I/O, dk = 128 and DeltaNet / Gated DeltaNet / KLA / KDA";
       return Kernel::None;
     }
     if (ws < need) {
@@ -128,7 +128,7 @@ gdr_status_t gdr_device_status(void *stream) {
 
 size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
   if (!valid_variant(variant) || !valid_dim(dk) || !valid_dim(dv) || B <= 0 || T <= 0 || H <= 0) return 0;
-  if ((chunk == 0 || chunk == 65) && split_ok(variant, dtype, dk, dv)) return gdr_split_workspace_bytes(B, T, H, dv);
+  if ((chunk == 0 || chunk == 65) && split_ok(variant, dtype, dk, dv)) return gdr_split_workspace_bytes(variant, B, T, H, dv);
   return 0;
 }
 
@@ -229,7 +229,7 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
   if (!split_ok(variant, dtype, dk, dv))
     return fail(GDR_ERR_UNSUPPORTED,
                 "the no-allocation entry point covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O and dk = 128");
-  const size_t need = gdr_split_workspace_bytes(B, T, H, dv);
+  const size_t need = gdr_split_workspace_bytes(variant, B, T, H, dv);
   const size_t have = gdr_split_fixed_scratch_bytes();
   if (need > have)
     return fail(GDR_ERR_UNSUPPORTED,

@@ -64,6 +64,8 @@ constexpr uint32_t REC_P = 49152;
 constexpr uint32_t REC_U = 57344;
 __host__ __device__ constexpr uint32_t rec_sc(int ns) { return REC_U + 8192 * ns; }
 __host__ __device__ constexpr uint32_t rec_bytes(int ns) { return rec_sc(ns) + 16; }
+// channel decay: Gamma_C is a vector of d_k = 128 floats
+__host__ __device__ constexpr uint32_t rec_bytes_chan(int ns) { return rec_sc(ns) + 4 * 128; }
 
 // ------------------------------------------------------------------ preparation kernel
 namespace prep {
@@ -382,6 +384,291 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   }
 }
 
+// ------------------------------------------------------------------ preparation kernel, channel decay
+// KDA ("Gated DeltaNet-2", what is new / technical core: a decay vector g_t in
+// R^{dk} on the state rows).  The chunk-local products take the decay inside,
+// factored around the chunk's middle token m with G_t[i] = e^{gamma_t[i] - gamma_m[i]}:
+//     A_tr = beta_r [K o G; .](K o G^-1)^T,  P_tr = beta_r [.; scale Q o G](K o G^-1)^T,
+//     W = T (K o e^gamma),  Qg = scale Q o e^gamma,  Kt_r = beta_r k_r o e^{gamma_C - gamma_r},
+// and the state decays row by row with e^{gamma_C}.  The factors G span beyond
+// fp16's range and one bf16 rounding of them leaves ~2.5% of the output RMS,
+// so MMA1 takes tf32 operands (fp32 range, an 11-bit significand), in two
+// 64-channel halves.  The record is the scalar-decay record with Gamma_C a
+// vector of d_k values.
+namespace prepc {
+constexpr float SPAN_SAFE = 120.f;      // |gamma_t - gamma_m| (log2 units) the fp32 factors carry
+constexpr uint32_t OFF_KQ = 0;          // bf16 [Kb0 | Qb0 | Kb1 | Qb1] (TMA)
+constexpr uint32_t OFF_V = 32768;       // bf16 V, one 8 KB box per value slice (TMA)
+constexpr uint32_t OFF_LG = 49152;      // fp32 [64][128]: log g (TMA), then G
+constexpr uint32_t OFF_R = 81920;       // phase-shared region
+constexpr uint32_t OFF_XF = OFF_R;              // (c) tf32 [K o G; Q o G], 128 rows x 2 atoms of 32 channels
+constexpr uint32_t OFF_YF = OFF_R + 32768;      // (c) tf32 K o G^-1, 64 rows x 2 atoms
+constexpr uint32_t OFF_KG = OFF_R + 49152;      // (c..f) bf16 K o e^gamma [Kb0 | Kb1]
+constexpr uint32_t OFF_A = OFF_R;               // (d, e) fp32 A^T, 64 x LD
+constexpr uint32_t OFF_TF = OFF_R + 18432;      // (e) fp32 T, 64 x LD
+constexpr uint32_t OFF_T = OFF_R + 36864;       // (e, f) bf16 T
+constexpr uint32_t OFF_SC = OFF_R + 65536;      // beta [64], gamma_m [128], scratch [128]
+constexpr uint32_t OFF_BAR = OFF_SC + 320 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+static_assert(OFF_TF + 64 * LD * 4 <= OFF_T && OFF_T + 8192 <= OFF_KG, "phase region layout");
+static_assert(OFF_XF % 1024 == 0 && OFF_YF % 1024 == 0 && OFF_KG % 1024 == 0 && OFF_T % 1024 == 0, "alignment");
+constexpr uint32_t COL_G = 0;     // M128 x 64
+constexpr uint32_t COL_W = 64;    // M64 x 128
+constexpr uint32_t COL_U = 192;   // M128 x 64: U'^T
+constexpr uint32_t TMEM_COLS = 256;
+}  // namespace prepc
+
+__device__ __forceinline__ void unpack4_bf16(uint2 u, float *x) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    chunk_prep_chan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                           const PrepParams p) {
+  using namespace prepc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + lane;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int NS = p.dv / 64;
+  const int t0 = c * C;
+
+  uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+  uint64_t *bar_lg = bar_in + 1;
+  uint64_t *bar_mma = bar_in + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
+  float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);   // [64]
+  float *sc_gm = sc_beta + 64;                               // [128] gamma_m (log2 units)
+  float *sc_tmp = sc_gm + 128;                               // [128]
+  float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
+  float *At = reinterpret_cast<float *>(sm + OFF_A);
+  float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
+  uint8_t *rec = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c) * rec_bytes_chan(NS);
+  uint8_t *kq_ptr = sm + OFF_KQ;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_in, 1);
+    mbar_init(bar_lg, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    mbar_expect_tx(bar_lg, 64 * DK * 4);
+    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, t0, b);
+    mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
+    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+  }
+  if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
+    for (int i = tid; i < 512; i += NTHREADS)
+      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (tid < 64) {
+    const int t = t0 + tid;
+    sc_beta[tid] = (t < p.T) ? __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h) : 0.f;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  int bad = 0, range = 0;
+
+  // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
+  if (!mbar_wait(bar_lg, 0)) bad = 1;
+  bad = __syncthreads_or(bad);
+  if (!bad) {
+    const int ch = tid & 127, hh = tid >> 7;
+    float run = 0.f;
+#pragma unroll 8
+    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+      run += Gr[t * DK + ch] * LOG2E;
+      Gr[t * DK + ch] = run;
+    }
+    if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
+    __syncthreads();
+    const float gm = sc_tmp[ch];
+    if (hh == 0) sc_gm[ch] = gm;
+#pragma unroll 8
+    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+      float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
+      if (d > SPAN_SAFE || d < -SPAN_SAFE) {
+        range = 1;
+        d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
+      }
+      Gr[t * DK + ch] = ex2(d);
+    }
+  }
+  __syncthreads();
+  // Gamma_C per channel into the record
+  if (!bad && tid < DK)
+    reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * ex2(sc_gm[tid]);
+
+  // (b) inputs landed?
+  if (!mbar_wait(bar_in, 0)) bad = 1;
+  bad = __syncthreads_or(bad);
+  uint32_t mma_phase = 0;
+  float qkmax = 0.f;
+
+  // (c) MMA1 in two 64-channel halves; the record's Kt and Qg, and K o e^gamma for MMA2
+#pragma unroll 1
+  for (int hp = 0; hp < 2 && !bad; ++hp) {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
+      const int t = u >> 4, j4 = u & 15;
+      const int ch0 = 64 * hp + 4 * j4;
+      const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);   // 4 values of a 16-bit tile row
+      float kx[4], qx[4];
+      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+      const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
+      const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
+      const float4 m4 = *reinterpret_cast<const float4 *>(sc_gm + ch0);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
+      const float em[4] = {ex2(m4.x), ex2(m4.y), ex2(m4.z), ex2(m4.w)};
+      const float bt = sc_beta[t];
+      float kg[4], qg[4], ig[4], kt[4], qo[4], ke[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float inv = __frcp_rn(g[e]);
+        kg[e] = tf32r(kx[e] * g[e]);
+        qg[e] = tf32r(p.scale * qx[e] * g[e]);
+        ig[e] = tf32r(kx[e] * inv);
+        kt[e] = bt * kx[e] * (g63[e] * inv);
+        qo[e] = p.scale * qx[e] * g[e] * em[e];
+        ke[e] = kx[e] * g[e] * em[e];
+        qkmax = fmaxf(qkmax, fmaxf(fabsf(kt[e]), fabsf(qo[e])));
+      }
+      const uint32_t xa = (j4 >> 3) * 16384, ya = (j4 >> 3) * 8192;
+      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(t, j4 & 7)) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(64 + t, j4 & 7)) = make_float4(qg[0], qg[1], qg[2], qg[3]);
+      *reinterpret_cast<float4 *>(sm + OFF_YF + ya + sw128(t, j4 & 7)) = make_float4(ig[0], ig[1], ig[2], ig[3]);
+      *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
+          make_uint2(pack_f16x2(kt[0], kt[1]), pack_f16x2(kt[2], kt[3]));
+      *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
+          make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
+      *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
+          make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(yf + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 64, false, false),
+                 hp + kk > 0);
+      mma_commit(bar_mma);
+    }
+    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    mma_phase ^= 1;
+    tc_fence_after();
+  }
+
+  // (d) A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
+  if (!bad) {
+    float g[32];
+    tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
+    const int t = row & 63;
+    const int r0 = 32 * half;
+    if (quad < 2) {
+#pragma unroll
+      for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * sc_beta[r0 + r]) : 0.f;
+    } else {
+#pragma unroll
+      for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? g[r] * sc_beta[r0 + r] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // (e) T = (I + A)^{-1} as a bf16 tile
+  solve_unit_lower_64(At, Tf, tid, warp, lane);
+  {
+    const int m = tid >> 2, n0 = (tid & 3) * 16;
+    float tv[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+      tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
+  }
+  fence_async_smem();
+  __syncthreads();
+
+  // (f) MMA2: W = T (K o e^gamma) (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
+  if (!bad && tid == 0) {
+    tc_fence_after();
+    const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+               idesc_bf16(64, 128, false, true), kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+               idesc_bf16(128, 64, true, false), kk > 0);
+    mma_commit(bar_mma);
+  }
+  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+  bad = __syncthreads_or(bad);
+  tc_fence_after();
+
+  // (g) -W (M64 layout) and U'^T -> fp16 record tiles
+  float wmax = qkmax;
+  if (!bad) {
+    float w[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          wmax = fmaxf(wmax, fabsf(w[e]));
+          w[e] = -w[e];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+      }
+    }
+    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
+    if (row < p.dv) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+    }
+  }
+  if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
+  if (range || wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ carry kernel
 // One CTA per (b, h) sweeps the chunks in order, warp-specialised: warp 16
 // issues the record copies and the MMAs; compute warp w (0-15) owns value
@@ -397,11 +684,11 @@ namespace carry {
 constexpr int NSTAGE = 3;
 constexpr int NCOMPUTE = 16;
 constexpr int NTHREADS_CARRY = (NCOMPUTE + 1) * 32;
-constexpr uint32_t STAGE = 74752;        // record image (<= 73744 bytes), 1 KB aligned
+constexpr uint32_t STAGE = 74752;        // record image (<= 74240 bytes), 1 KB aligned
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(STAGE % 1024 == 0 && STAGE >= 73744, "stage layout");
+static_assert(STAGE % 1024 == 0 && STAGE >= rec_bytes(2) && STAGE >= rec_bytes_chan(2), "stage layout");
 constexpr uint32_t COL_Y = 0;      // 2 x 128: [(-W S0)^T | (Qg S0)^T + (P E)^T], [v][t]
 constexpr uint32_t COL_DS = 256;   // 128: dS^T, [v][i]
 constexpr uint32_t COL_SA = 384;   // 64: fp16 S^T, d_k packed two per column (MMA operand)
@@ -411,6 +698,7 @@ constexpr uint32_t TMEM_COLS = 512;
 
 struct CarryParams {
   int T, H, dv, NC;
+  uint32_t rec_bytes;    // bytes per record
   const uint8_t *ws;
   const float *s0;
   float *s_final;
@@ -431,6 +719,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
   return true;
 }
 
+// CHAN: Gamma_C is a vector of d_k values (channel decay), else a scalar.
+template <bool CHAN>
 __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
   using namespace carry;
   extern __shared__ uint8_t smem_raw[];
@@ -469,7 +759,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t rb = rec_bytes(NS);
+  const uint32_t rb = p.rec_bytes;
 
   // issuer's view of the record copies: stage has a copy in flight / phase parity to wait for
   uint32_t pend = 0, par = 0;
@@ -597,17 +887,18 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         if (lane == 0) mbar_arrive(bar_ea);
       }
 
-      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31
+      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row
+      // for channel decay)
       ok = wait_or_abort(bar_s, c & 1, abort);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       {
-        const float gc = *reinterpret_cast<const float *>(st + rec_sc(NS));
+        const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
         float d[32];
         tmem_ld32(lrow + COL_DS + 32 * part, d);
 #pragma unroll
         for (int m = 0; m < 32; ++m) {
-          S[m] = fmaf(gc, S[m], d[m]);
+          S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d[m]);
           smax = fmaxf(smax, fabsf(S[m]));
         }
         store_state();
@@ -675,16 +966,13 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 }
 
 template <int VAR>
-cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
   // all of the unified L1 as shared memory, so that two preparation CTAs fit on an SM
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)carry::SMEM_BYTES);
   if (e != cudaSuccess) {
     *err = "cudaFuncSetAttribute: ";
     return e;
@@ -695,10 +983,9 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
     *err = "cuTensorMapEncodeTiled failed: ";
     return cudaErrorInvalidValue;
   }
-  const int NC = (p.T + C - 1) / C;
   PrepParams pp;
   pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
-  pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = static_cast<uint8_t *>(ws);
+  pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
   // persistent grid: as many CTAs as fit on the device at once, none idle
   int dev = 0, sms = 0, per_sm = 0;
@@ -718,18 +1005,61 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   const int grid = static_cast<int>(std::min<long long>(records, static_cast<long long>(std::max(per_sm, 2)) * sms));
   chunk_prep_kernel<VAR><<<grid, NTHREADS, prep::SMEM_BYTES, stream>>>(mq, mk, mv, pp);
   e = cudaGetLastError();
+  if (e != cudaSuccess) *err = "prep launch: ";
+  return e;
+}
+
+cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
+  cudaError_t e = cudaFuncSetAttribute(chunk_prep_chan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)prepc::SMEM_BYTES);
   if (e != cudaSuccess) {
-    *err = "prep launch: ";
+    *err = "cudaFuncSetAttribute: ";
+    return e;
+  }
+  CUtensorMap mq, mk, mv, mg;
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map(&mk, p.k, p.B, p.T, p.H, p.dk) ||
+      !make_map(&mv, p.v, p.B, p.T, p.H, p.dv) || !make_map_f32_rows(&mg, p.log_g, p.B, p.T, p.H, p.dk)) {
+    *err = "cuTensorMapEncodeTiled failed: ";
+    return cudaErrorInvalidValue;
+  }
+  PrepParams pp;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
+  pp.eps = p.eps; pp.scale = p.scale;
+  chunk_prep_chan_kernel<<<dim3(NC, p.H, p.B), NTHREADS, prepc::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *err = "prep launch: ";
+  return e;
+}
+
+template <bool CHAN>
+cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, cudaStream_t stream, std::string *err) {
+  cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<CHAN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)carry::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    *err = "cudaFuncSetAttribute: ";
     return e;
   }
   CarryParams cp;
   cp.T = p.T; cp.H = p.H; cp.dv = p.dv; cp.NC = NC;
-  cp.ws = static_cast<const uint8_t *>(ws); cp.s0 = p.s0; cp.s_final = p.s_final;
+  cp.rec_bytes = CHAN ? rec_bytes_chan(p.dv / 64) : rec_bytes(p.dv / 64);
+  cp.ws = ws; cp.s0 = p.s0; cp.s_final = p.s_final;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
+  chunk_carry_kernel<CHAN><<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
+}
+
+template <int VAR>
+cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
+  const int NC = (p.T + C - 1) / C;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  cudaError_t e;
+  if constexpr (VAR == kKDA) e = launch_prep_chan(p, NC, w, stream, err);
+  else e = launch_prep<VAR>(p, NC, w, stream, err);
+  if (e != cudaSuccess) return e;
+  return launch_carry<VAR == kKDA>(p, NC, w, stream, err);
 }
 
 }  // namespace
@@ -738,13 +1068,14 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
 
 bool gdr_split_supported(int variant, int dk, int dv) {
   using namespace gdr;
-  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA;
+  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA;
   return v && dk == 128 && (dv == 64 || dv == 128);
 }
 
-size_t gdr_split_workspace_bytes(int B, int T, int H, int dv) {
+size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   const size_t NC = (static_cast<size_t>(T) + 63) / 64;
-  return static_cast<size_t>(B) * H * NC * gdr::tc::rec_bytes(dv / 64);
+  const size_t rec = variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64) : gdr::tc::rec_bytes(dv / 64);
+  return static_cast<size_t>(B) * H * NC * rec;
 }
 
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
@@ -753,6 +1084,7 @@ cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t st
     case kDeltaNet: return tc::launch_split<kDeltaNet>(p, ws, stream, err);
     case kGatedDeltaNet: return tc::launch_split<kGatedDeltaNet>(p, ws, stream, err);
     case kKLA: return tc::launch_split<kKLA>(p, ws, stream, err);
+    case kKDA: return tc::launch_split<kKDA>(p, ws, stream, err);
     default: *err = "variant not covered: "; return cudaErrorInvalidValue;
   }
 }

@@ -13,11 +13,11 @@
 //     S_C = Diag(e^{gamma_C}) S0 + Kt^T E,  Kt[r][i] = beta_r k_r[i] e^{gamma_C[i] - gamma_r[i]}
 // The e^{gamma_t - gamma_r} factor is split around the chunk's middle token m:
 // [K o e^{gamma - gamma_m}; scale Q o e^{gamma - gamma_m}] (K o e^{gamma_m - gamma})^T.
-// Its factors span up to e^{|gamma_0 - gamma_63|}, beyond fp16's range, so
-// these two operands are bf16 split into hi + lo terms (three products,
-// ~16-bit precision); one bf16 rounding there alone leaves ~2.5% of the
-// output RMS.  MMA1 runs in two 64-channel halves so the split operands fit
-// in shared memory.  The channel log-decay tile (64 x 128 fp32) arrives by TMA
+// Its factors span up to e^{|gamma_0 - gamma_63|}, beyond fp16's range, and one
+// bf16 rounding there alone leaves ~2.5% of the output RMS, so these two
+// operands are tf32: fp32 range with an 11-bit significand like fp16's.
+// MMA1 runs in two 64-channel halves so the fp32 operands fit in shared
+// memory.  The channel log-decay tile (64 x 128 fp32) arrives by TMA
 // one chunk ahead and is scanned in place.  Everything after T follows the
 // scalar-decay kernel (fp16 carry operands, stacked [Qg; -W] S0, P E
 // accumulated onto the output rows); see chunk_tc.cu for the shared
@@ -54,10 +54,8 @@ constexpr uint32_t OFF_KT = 131072;     // fp16 Kt [Kb0 | Kb1]
 constexpr uint32_t OFF_ZT = 147456;     // bf16 [zero | T]
 constexpr uint32_t OFF_R = 163840;      // phase-shared region (60 KB), see below
 constexpr uint32_t OFF_P = OFF_R;                    // fp16 P (d .. j); rows 64-127 of [P; *] follow
-constexpr uint32_t OFF_XH = OFF_R + 8192;            // (c) bf16 hi [K o G; Q o G], 128 rows x 64 ch
-constexpr uint32_t OFF_XL = OFF_R + 24576;           // (c) bf16 lo
-constexpr uint32_t OFF_YH = OFF_R + 40960;           // (c) bf16 hi  K o G^-1, 64 rows x 64 ch
-constexpr uint32_t OFF_YL = OFF_R + 49152;           // (c) bf16 lo
+constexpr uint32_t OFF_XF = OFF_R + 8192;            // (c) tf32 [K o G; Q o G], 128 rows x 2 atoms of 32 ch
+constexpr uint32_t OFF_YF = OFF_R + 40960;           // (c) tf32 K o G^-1, 64 rows x 2 atoms of 32 ch
 constexpr uint32_t OFF_A = OFF_R + 8192;             // (d, e) fp32 A^T, 64 x LD
 constexpr uint32_t OFF_TF = OFF_R + 26624;           // (e) fp32 T, 64 x LD
 constexpr uint32_t OFF_KG = OFF_R + 45056;           // (e, f) bf16 K o e^{gamma} [Kb0 | Kb1]
@@ -68,7 +66,8 @@ constexpr uint32_t OFF_BAR = OFF_SC + 384 * 4;       // mbarriers + TMEM slot
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_KG % 1024 == 0 && OFF_E % 1024 == 0 && OFF_YH % 1024 == 0, "tile alignment");
+static_assert(OFF_KG % 1024 == 0 && OFF_E % 1024 == 0 && OFF_XF % 1024 == 0 && OFF_YF % 1024 == 0,
+              "tile alignment");
 
 constexpr uint32_t COL_G = 0;     // M128 x 64
 constexpr uint32_t COL_W = 64;    // M64 x 128
@@ -76,7 +75,7 @@ constexpr uint32_t COL_YE = 192;  // M128 x 64
 constexpr uint32_t COL_S = 256;   // M128 x 64
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t ID_G = idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_G = idesc_tf32(128, 64, false, false);
 constexpr uint32_t ID_W = idesc_bf16(64, 128, false, true);
 constexpr uint32_t ID_U = idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_YE = idesc_f16(128, 64, false, true);
@@ -91,9 +90,11 @@ struct Params {
   float scale;
 };
 
-__device__ __forceinline__ void split_bf16(float x, float &hi, float &lo) {
-  hi = __bfloat162float(__float2bfloat16_rn(x));
-  lo = x - hi;
+// Four bf16 values (8 bytes) to floats.
+__device__ __forceinline__ void unpack4(uint2 u, float *x) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
 }
 
 template <int VAR>
@@ -231,55 +232,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!mbar_wait(&bar_full[s], (c >> 1) & 1)) bad = 1;
     if (__syncthreads_or(bad)) break;
 
-    // ---- (c) MMA1 in two 64-channel halves: [K o G; Q o G] (K o G^-1)^T, hi/lo split;
+    // ---- (c) MMA1 in two 64-channel halves: [K o G; Q o G] (K o G^-1)^T in tf32;
     // also Kt = beta_r K o G_63 / G_r (fp16)
 #pragma unroll 1
     for (int hp = 0; hp < 2; ++hp) {
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int u = it * NTHREADS + tid;      // 512 units: (t, 8-channel chunk j)
-        const int t = u >> 3, j = u & 7;
-        const int ch0 = 64 * hp + 8 * j;
-        float kx[8], qx[8], g[8], g63[8];
-        unpack8(*reinterpret_cast<const uint4 *>(kq_ptr + hp * 16384 + sw128(t, j)), kx);
-        unpack8(*reinterpret_cast<const uint4 *>(kq_ptr + hp * 16384 + 8192 + sw128(t, j)), qx);
-        const float4 g0 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
-        const float4 g1 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0 + 4);
-        const float4 h0 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
-        const float4 h1 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0 + 4);
-        g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w; g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
-        g63[0] = h0.x; g63[1] = h0.y; g63[2] = h0.z; g63[3] = h0.w;
-        g63[4] = h1.x; g63[5] = h1.y; g63[6] = h1.z; g63[7] = h1.w;
+      for (int it = 0; it < 4; ++it) {
+        const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
+        const int t = u >> 4, j4 = u & 15;
+        const int ch0 = 64 * hp + 4 * j4;
+        const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);   // 4 bf16 values of the input tiles
+        float kx[4], qx[4];
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
+        const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
+        const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
         const float bt = sc_beta[t];
-        float kh[8], kl[8], qh[8], ql[8], ih[8], il[8], kt[8];
+        float kg[4], qg[4], ig[4], kt[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           const float inv = __frcp_rn(g[e]);
-          split_bf16(kx[e] * g[e], kh[e], kl[e]);
-          split_bf16(p.scale * qx[e] * g[e], qh[e], ql[e]);
-          split_bf16(kx[e] * inv, ih[e], il[e]);
+          kg[e] = tf32r(kx[e] * g[e]);
+          qg[e] = tf32r(p.scale * qx[e] * g[e]);
+          ig[e] = tf32r(kx[e] * inv);
           kt[e] = bt * kx[e] * (g63[e] * inv);
         }
-        st_chunk_bf16(sm + OFF_XH + sw128(t, j), kh);
-        st_chunk_bf16(sm + OFF_XL + sw128(t, j), kl);
-        st_chunk_bf16(sm + OFF_XH + sw128(64 + t, j), qh);
-        st_chunk_bf16(sm + OFF_XL + sw128(64 + t, j), ql);
-        st_chunk_bf16(sm + OFF_YH + sw128(t, j), ih);
-        st_chunk_bf16(sm + OFF_YL + sw128(t, j), il);
-        st_chunk_f16(sm + OFF_KT + hp * 8192 + sw128(t, j), kt);
+        // fp32 tiles: 32-channel atoms of 128-byte rows; 16-byte chunk j4 mod 8 of the row
+        const uint32_t xa = (j4 >> 3) * 16384, ya = (j4 >> 3) * 8192;
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(t, j4 & 7)) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(64 + t, j4 & 7)) =
+            make_float4(qg[0], qg[1], qg[2], qg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_YF + ya + sw128(t, j4 & 7)) = make_float4(ig[0], ig[1], ig[2], ig[3]);
+        *reinterpret_cast<uint2 *>(sm + OFF_KT + hp * 8192 + bf) =
+            make_uint2(pack_f16x2(kt[0], kt[1]), pack_f16x2(kt[2], kt[3]));
       }
       fence_async_smem();
       __syncthreads();
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t xh = smem_u32(sm + OFF_XH), xl = smem_u32(sm + OFF_XL);
-        const uint32_t yh = smem_u32(sm + OFF_YH), yl = smem_u32(sm + OFF_YL);
+        const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16(tmem + COL_G, sdesc(xh + kk * 32, 16, 1024), sdesc(yh + kk * 32, 16, 1024), ID_G, hp + kk > 0);
-          mma_bf16(tmem + COL_G, sdesc(xh + kk * 32, 16, 1024), sdesc(yl + kk * 32, 16, 1024), ID_G, 1);
-          mma_bf16(tmem + COL_G, sdesc(xl + kk * 32, 16, 1024), sdesc(yh + kk * 32, 16, 1024), ID_G, 1);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   sdesc(yf + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_G, hp + kk > 0);
         mma_commit(bar_mma);
       }
       if (!mbar_wait(bar_mma, mma_phase)) bad = 1;

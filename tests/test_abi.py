@@ -146,10 +146,13 @@ def test_workspace_sizes(L):
     assert L.gdr_forward_workspace_size(1, 1, 2, 65, 3, 128, 64, 65) == 2 * 3 * 2 * (57344 + 8192 + 16)
     assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 64) == 0   # one-kernel path
     assert L.gdr_forward_workspace_size(1, 0, 8, 2048, 8, 128, 128, 0) == 0    # fp32: per-token
-    assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 0    # KDA: one kernel
+    # KDA: the same record with Gamma_C a vector of 128 floats
+    assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 512)
+    assert L.gdr_forward_workspace_size(3, 1, 8, 2048, 8, 128, 128, 0) == 0    # GDN-2: per-token kernel
     assert L.gdr_forward_kernel_name(1, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
     assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == 2
-    assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_tc"
+    assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
+    assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 64).decode() == "chunk64_tc"
 
 
 def test_split_needs_workspace(L):
