@@ -51,32 +51,57 @@ __global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
     }
   }
 
-  for (int t = 0; t < p.T; ++t) {
+  // Inputs of one token as loaded (raw gates; derived values are formed at use).
+  struct TokenIn {
+    float kv[R], qv[R], lg[R], eb[R], ww[R], vv[8], beta;
+  };
+  auto load = [&](int t, TokenIn &d) {
     const size_t th = ((size_t)b * p.T + t) * p.H + h;
-    float kv[R], qv[R], g[R], ea[R], wc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      kv[r] = ld_io<IO>(k + th * DK + lane + 32 * r);
-      qv[r] = ld_io<IO>(q + th * DK + lane + 32 * r);
+      d.kv[r] = ld_io<IO>(k + th * DK + lane + 32 * r);
+      d.qv[r] = ld_io<IO>(q + th * DK + lane + 32 * r);
     }
-    float vv[8];
-    ld8<IO>(v + th * dv + c0, vv);
+    ld8<IO>(v + th * dv + c0, d.vv);
     if constexpr (scalar_decay(VAR)) {
-      const float gs = expf(__ldg(p.log_g + th));
+      const float lgs = __ldg(p.log_g + th);
 #pragma unroll
-      for (int r = 0; r < R; ++r) g[r] = gs;
+      for (int r = 0; r < R; ++r) d.lg[r] = lgs;
     } else if constexpr (channel_decay(VAR)) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) g[r] = expf(__ldg(p.log_g + th * DK + lane + 32 * r));
-    } else {
-#pragma unroll
-      for (int r = 0; r < R; ++r) g[r] = 1.f;
+      for (int r = 0; r < R; ++r) d.lg[r] = __ldg(p.log_g + th * DK + lane + 32 * r);
     }
     if constexpr (VAR == kGDN2) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        ea[r] = __ldg(p.erase_b + th * DK + lane + 32 * r) * kv[r];
-        wc[r] = __ldg(p.write_w + th * DK + lane + 32 * r) * kv[r];
+        d.eb[r] = __ldg(p.erase_b + th * DK + lane + 32 * r);
+        d.ww[r] = __ldg(p.write_w + th * DK + lane + 32 * r);
+      }
+    } else {
+      d.beta = __ldg(p.beta + th);
+    }
+  };
+
+  // Software pipeline over tokens: token t+1's loads are in flight while
+  // token t is computed, so each step waits for no memory latency.
+  TokenIn cur, nxt;
+  if (p.T > 0) load(0, cur);
+#pragma unroll 1
+  for (int t = 0; t < p.T; ++t) {
+    const size_t th = ((size_t)b * p.T + t) * p.H + h;
+    if (t + 1 < p.T) load(t + 1, nxt);
+    const float *kv = cur.kv, *qv = cur.qv, *vv = cur.vv;
+    float g[R], ea[R], wc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if constexpr (scalar_decay(VAR) || channel_decay(VAR)) g[r] = expf(cur.lg[r]);
+      else g[r] = 1.f;
+    }
+    if constexpr (VAR == kGDN2) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        ea[r] = cur.eb[r] * kv[r];
+        wc[r] = cur.ww[r] * kv[r];
       }
     }
 
@@ -115,7 +140,7 @@ __global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) out[c] = p.scale * (y[c] - s1 * x[c] + s2 * vv[c]);
     } else {
-      float step = __ldg(p.beta + th);                      // beta_t, or eta_t for KLA
+      float step = cur.beta;                                // beta_t, or eta_t for KLA
       if constexpr (VAR == kKLA) step = step / (s2 + p.eps);  // Kaczmarz step
       float e[8];
 #pragma unroll
@@ -131,6 +156,7 @@ __global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
       for (int c = 0; c < 8; ++c) out[c] = p.scale * fmaf(akq, e[c], y[c]);
     }
     if (lane == 0) st8<IO>(o + th * dv + c0, out);
+    cur = nxt;
   }
 
   if (p.s_final) {
