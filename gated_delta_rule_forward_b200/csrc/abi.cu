@@ -63,7 +63,7 @@ Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int d
   if (chunk == 65) {
     if (!sp) {
       *st = GDR_ERR_UNSUPPORTED;
-      *why = "chunk=65 two-kernel path needs bf16 I/O, dk = 128 and DeltaNet / Gated DeltaNet / KLA / KDA";
+      *why = "chunk=65 two-kernel path needs bf16 I/O and dk = 128";
       return Kernel::None;
     }
     if (ws < need) {

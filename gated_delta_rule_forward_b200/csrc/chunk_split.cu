@@ -66,6 +66,8 @@ __host__ __device__ constexpr uint32_t rec_sc(int ns) { return REC_U + 8192 * ns
 __host__ __device__ constexpr uint32_t rec_bytes(int ns) { return rec_sc(ns) + 16; }
 // channel decay: Gamma_C is a vector of d_k = 128 floats
 __host__ __device__ constexpr uint32_t rec_bytes_chan(int ns) { return rec_sc(ns) + 4 * 128; }
+// GDN-2: the channel-decay record, then (P^d V)^T (8 KB per 64 values) and (Dt^T V)^T (16 KB per 64 values)
+__host__ __device__ constexpr uint32_t rec_bytes_gdn2(int ns) { return rec_bytes_chan(ns) + 24576 * ns; }
 
 // ------------------------------------------------------------------ preparation kernel
 namespace prep {
@@ -669,6 +671,385 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ preparation kernel, GDN-2
+// GDN-2 ("Gated DeltaNet-2", technical core, read as in the header of gdr.h):
+// channel decay, erase vector a_t = b_t o k_t, write vector c_t = w_t o k_t.
+// With d_t = c_t - a_t the chunk form keeps the residual of the scalar
+// kernels (an exact rearrangement of the per-token recurrence):
+//     A = Gram(K, a), A^d = Gram(K, d) (strictly lower), P^a, P^d = Gram(scale Q, .) (lower),
+//     T = (I + A)^{-1},  R = T (I - A^d),  W = T (K o e^gamma),  U' = R V,  E = U' - W S0
+//     O = (scale Q o e^gamma) S0 + P^a E + P^d V
+//     S_C = e^{gamma_C} o S0 + At^T E + Dt^T V,   At, Dt rows a_r, d_r o e^{gamma_C - gamma_r}
+// where Gram(X, Y)_tr = sum_i x_t[i] y_r[i] e^{gamma_t[i] - gamma_r[i]}, factored
+// around the middle token as for KDA and computed as one tf32 product
+// [K o G; scale Q o G] [a o G^-1; d o G^-1]^T.  The record is the channel-decay
+// record (At in the Kt slot, P^a in the P slot) followed by the two terms
+// that do not involve the state, (P^d V)^T and (Dt^T V)^T, which the carry
+// adds to the output and to the state.
+namespace prepg {
+constexpr float SPAN_SAFE = 120.f;
+constexpr uint32_t OFF_KQ = 0;          // bf16 [Kb0 | Qb0 | Kb1 | Qb1] (TMA)
+constexpr uint32_t OFF_V = 32768;       // V boxes: bf16 (TMA), fp16 from (e) on
+constexpr uint32_t OFF_LG = 49152;      // fp32 [64][128]: log g (TMA), then G
+constexpr uint32_t OFF_R = 81920;       // phase-shared region
+constexpr uint32_t OFF_XF = OFF_R;              // (c) tf32 [K o G; Q o G], 2 atoms x 128 rows
+constexpr uint32_t OFF_YF = OFF_R + 32768;      // (c) tf32 [a o G^-1; d o G^-1], 2 atoms x 128 rows
+constexpr uint32_t OFF_A = OFF_R;               // (d, e) fp32 A^T
+constexpr uint32_t OFF_TF = OFF_R + 18432;      // (e) fp32 T
+constexpr uint32_t OFF_T = OFF_R + 36864;       // fp16 T, rows t
+constexpr uint32_t OFF_IAD = OFF_R + 45056;     // fp16 I - A^d, rows r (MN-major operand)
+constexpr uint32_t OFF_PD = OFF_R + 53248;      // fp16 P^d, rows t
+constexpr uint32_t OFF_RT = OFF_R + 61440;      // fp16 R, rows t
+constexpr uint32_t OFF_KG = OFF_R + 69632;      // (c..f) fp16 K o e^gamma [Kb0 | Kb1]
+constexpr uint32_t OFF_DT = OFF_R + 86016;      // (c..f) fp16 Dt [b0 | b1], rows r (MN-major operand)
+constexpr uint32_t OFF_SC = OFF_R + 102400;     // gamma_m [128], scratch [128]
+constexpr uint32_t OFF_BAR = OFF_SC + 256 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_TF + 64 * LD * 4 <= OFF_T && OFF_YF + 32768 <= OFF_KG, "phase region layout");
+static_assert((OFF_T | OFF_IAD | OFF_PD | OFF_RT | OFF_KG | OFF_DT | OFF_XF | OFF_YF) % 1024 == 0, "alignment");
+constexpr uint32_t COL_G = 0;     // (c, d) M128 x 128: [A | A^d ; P^a | P^d]
+constexpr uint32_t COL_SD = 0;    // (f, g) M128 x 128: (Dt^T V)^T
+constexpr uint32_t COL_R = 128;   // M64 x 64
+constexpr uint32_t COL_W = 192;   // M64 x 128
+constexpr uint32_t COL_U = 320;   // M128 x 64: U'^T
+constexpr uint32_t COL_OD = 384;  // M128 x 64: (P^d V)^T
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace prepg
+
+struct PrepG2Params {
+  int T, H, dv, NC;
+  const float *erase_b, *write_w;
+  uint8_t *ws;
+  float scale;
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    chunk_prep_gdn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                           const PrepG2Params p) {
+  using namespace prepg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + lane;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int NS = p.dv / 64;
+  const int t0 = c * C;
+
+  uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+  uint64_t *bar_lg = bar_in + 1;
+  uint64_t *bar_mma = bar_in + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
+  float *sc_gm = reinterpret_cast<float *>(sm + OFF_SC);     // [128] gamma_m (log2 units)
+  float *sc_tmp = sc_gm + 128;                               // [128]
+  float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
+  float *At = reinterpret_cast<float *>(sm + OFF_A);
+  float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
+  uint8_t *rec = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c) * rec_bytes_gdn2(NS);
+  uint8_t *rec_od = rec + rec_bytes_chan(NS);          // (P^d V)^T, rows v x 64 t fp16
+  uint8_t *rec_sd = rec_od + 8192 * NS;                // (Dt^T V)^T, rows v x 128 i fp16
+  uint8_t *kq_ptr = sm + OFF_KQ;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_in, 1);
+    mbar_init(bar_lg, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    mbar_expect_tx(bar_lg, 64 * DK * 4);
+    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, t0, b);
+    mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
+    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
+    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+  }
+  if (NS == 1) {   // d_v = 64: the transposed products read a 128-row V operand
+    for (int i = tid; i < 512; i += NTHREADS)
+      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  int bad = 0, range = 0;
+  uint32_t mma_phase = 0;
+
+  // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
+  if (!mbar_wait(bar_lg, 0)) bad = 1;
+  bad = __syncthreads_or(bad);
+  if (!bad) {
+    const int ch = tid & 127, hh = tid >> 7;
+    float run = 0.f;
+#pragma unroll 8
+    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+      run += Gr[t * DK + ch] * LOG2E;
+      Gr[t * DK + ch] = run;
+    }
+    if (hh == 0) sc_tmp[ch] = run;
+    __syncthreads();
+    const float gm = sc_tmp[ch];
+    if (hh == 0) sc_gm[ch] = gm;
+#pragma unroll 8
+    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+      float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
+      if (d > SPAN_SAFE || d < -SPAN_SAFE) {
+        range = 1;
+        d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
+      }
+      Gr[t * DK + ch] = ex2(d);
+    }
+  }
+  __syncthreads();
+  if (!bad && tid < DK)
+    reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * ex2(sc_gm[tid]);
+
+  // (b) inputs landed?
+  if (!mbar_wait(bar_in, 0)) bad = 1;
+  bad = __syncthreads_or(bad);
+  float qkmax = 0.f;
+
+  // (c) MMA1 in two 64-channel halves; the record's At and Qg; K o e^gamma and Dt for MMA2
+#pragma unroll 1
+  for (int hp = 0; hp < 2 && !bad; ++hp) {
+#pragma unroll 2
+    for (int it = 0; it < 4; ++it) {
+      const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
+      const int t = u >> 4, j4 = u & 15;
+      const int ch0 = 64 * hp + 4 * j4;
+      const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);
+      float kx[4], qx[4];
+      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+      float4 eb = make_float4(0.f, 0.f, 0.f, 0.f), wr = eb;
+      if (t0 + t < p.T) {
+        const size_t gi = ((static_cast<size_t>(b) * p.T + t0 + t) * p.H + h) * DK + ch0;
+        eb = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
+        wr = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
+      }
+      const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
+      const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
+      const float4 m4 = *reinterpret_cast<const float4 *>(sc_gm + ch0);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
+      const float em[4] = {ex2(m4.x), ex2(m4.y), ex2(m4.z), ex2(m4.w)};
+      const float ebv[4] = {eb.x, eb.y, eb.z, eb.w}, wrv[4] = {wr.x, wr.y, wr.z, wr.w};
+      float kg[4], qg[4], af[4], df[4], at[4], dt[4], qo[4], ke[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float inv = __frcp_rn(g[e]);
+        const float a = ebv[e] * kx[e], d = (wrv[e] - ebv[e]) * kx[e];
+        kg[e] = tf32r(kx[e] * g[e]);
+        qg[e] = tf32r(p.scale * qx[e] * g[e]);
+        af[e] = tf32r(a * inv);
+        df[e] = tf32r(d * inv);
+        at[e] = a * (g63[e] * inv);
+        dt[e] = d * (g63[e] * inv);
+        qo[e] = p.scale * qx[e] * g[e] * em[e];
+        ke[e] = kx[e] * g[e] * em[e];
+        qkmax = fmaxf(qkmax, fmaxf(fabsf(at[e]), fabsf(qo[e])));
+      }
+      const uint32_t xa = (j4 >> 3) * 16384;
+      const uint32_t sw = sw128(t, j4 & 7), sw64 = sw128(64 + t, j4 & 7);
+      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw64) = make_float4(qg[0], qg[1], qg[2], qg[3]);
+      *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw) = make_float4(af[0], af[1], af[2], af[3]);
+      *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw64) = make_float4(df[0], df[1], df[2], df[3]);
+      *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
+          make_uint2(pack_f16x2(at[0], at[1]), pack_f16x2(at[2], at[3]));
+      *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
+          make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
+      *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
+          make_uint2(pack_f16x2(ke[0], ke[1]), pack_f16x2(ke[2], ke[3]));
+      *reinterpret_cast<uint2 *>(sm + OFF_DT + hp * 8192 + bf) =
+          make_uint2(pack_f16x2(dt[0], dt[1]), pack_f16x2(dt[2], dt[3]));
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(yf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 128, false, false),
+                 hp + kk > 0);
+      mma_commit(bar_mma);
+    }
+    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    mma_phase ^= 1;
+    tc_fence_after();
+  }
+
+  // (d) rows t of K (lanes 0-63): A -> A^T scratch, I - A^d -> bf16 rows; rows t of Q
+  // (lanes 64-127): P^a -> fp16 record tile, P^d -> bf16 tile.  Column half `half`
+  // selects the a or the d block.
+  if (!bad) {
+    float g[64];
+    tmem_ld64(tmem + lane_base + COL_G + 64 * half, g);
+    const int t = row & 63;
+    if (quad < 2) {
+      if (half == 0) {
+#pragma unroll
+        for (int r = 0; r < 64; ++r) At[r * LD + t] = (r < t) ? tf32r(g[r]) : 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 64; ++r) g[r] = (r < t) ? -g[r] : (r == t ? 1.f : 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_IAD + sw128(t, j), g + 8 * j);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 64; ++r) g[r] = (r <= t) ? g[r] : 0.f;
+      if (half == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_chunk_f16(rec + REC_P + sw128(t, j), g + 8 * j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_PD + sw128(t, j), g + 8 * j);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // (e) T = (I + A)^{-1} as fp16 rows; then R = T (I - A^d).  The V tile turns
+  // fp16 in place (exact from bf16) so that every product of this kernel after
+  // MMA1 has fp16 operands: the GDN-2 terms pass more roundings into the state
+  // than the other variants' and bf16 there leaves ~2% of the state RMS.
+  solve_unit_lower_64(At, Tf, tid, warp, lane);
+  float tmax = 0.f;
+  for (int i = tid; i < NS * 512; i += NTHREADS) {
+    uint4 *chunk = reinterpret_cast<uint4 *>(sm + OFF_V) + i;
+    float x[8];
+    unpack8(*chunk, x);
+    st_chunk_f16(reinterpret_cast<uint8_t *>(chunk), x);
+  }
+  {
+    const int m = tid >> 2, n0 = (tid & 3) * 16;
+    float tv[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+      tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+      tmax = fmaxf(tmax, fabsf(tv[e]));
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) st_chunk_f16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
+  }
+  fence_async_smem();
+  __syncthreads();
+  if (!bad && tid == 0) {
+    tc_fence_after();
+    const uint32_t tt = smem_u32(sm + OFF_T), iad = smem_u32(sm + OFF_IAD);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + COL_R, sdesc(tt + kk * 32, 16, 1024), sdesc(iad + kk * 2048, 8192, 1024),
+               idesc_f16(64, 64, false, true), kk > 0);
+    mma_commit(bar_mma);
+  }
+  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+  bad = __syncthreads_or(bad);
+  mma_phase ^= 1;
+  tc_fence_after();
+  if (!bad) {   // R (M64 layout: rows 16 quad + lane, lane < 16) -> fp16 rows t
+    float w[32];
+    tmem_ld32(tmem + lane_base + COL_R + 32 * half, w);
+    if (lane < 16) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, fabsf(w[e]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_RT + sw128(quad * 16 + lane, 4 * half + j), w + 8 * j);
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  // (f) W = T (K o e^gamma); U'^T = V^T R^T; (P^d V)^T = V^T P^d^T; (Dt^T V)^T = V^T Dt
+  if (!bad && tid == 0) {
+    tc_fence_after();
+    const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
+    const uint32_t rt = smem_u32(sm + OFF_RT), pd = smem_u32(sm + OFF_PD), dtt = smem_u32(sm + OFF_DT);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t va = sdesc(vt + kk * 2048, 8192, 1024);
+      mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+               idesc_f16(64, 128, false, true), kk > 0);
+      mma_bf16(tmem + COL_U, va, sdesc(rt + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+      mma_bf16(tmem + COL_OD, va, sdesc(pd + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+      mma_bf16(tmem + COL_SD, va, sdesc(dtt + kk * 2048, 8192, 1024), idesc_f16(128, 128, true, true), kk > 0);
+    }
+    mma_commit(bar_mma);
+  }
+  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+  bad = __syncthreads_or(bad);
+  tc_fence_after();
+
+  // (g) -W (M64 layout), U'^T, (P^d V)^T and (Dt^T V)^T -> fp16 record tiles
+  float wmax = fmaxf(qkmax, tmax);
+  if (!bad) {
+    float w[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          wmax = fmaxf(wmax, fabsf(w[e]));
+          w[e] = -w[e];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+      }
+    }
+    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
+    if (row < p.dv) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+    }
+    tmem_ld32(tmem + lane_base + COL_OD + 32 * half, w);
+    if (row < p.dv) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f16(rec_od + row * 128 + half * 64 + 16 * j, w + 8 * j);
+    }
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      tmem_ld32(tmem + lane_base + COL_SD + 64 * half + 32 * part, w);
+      if (row < p.dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st_chunk_f16(rec_sd + row * 256 + half * 128 + part * 64 + 16 * j, w + 8 * j);
+      }
+    }
+  }
+  if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
+  if (range || wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ carry kernel
 // One CTA per (b, h) sweeps the chunks in order, warp-specialised: warp 16
 // issues the record copies and the MMAs; compute warp w (0-15) owns value
@@ -699,6 +1080,7 @@ constexpr uint32_t TMEM_COLS = 512;
 struct CarryParams {
   int T, H, dv, NC;
   uint32_t rec_bytes;    // bytes per record
+  uint32_t copy_bytes;   // leading bytes of a record that go through shared memory
   const uint8_t *ws;
   const float *s0;
   float *s_final;
@@ -719,9 +1101,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
   return true;
 }
 
-// CHAN: Gamma_C is a vector of d_k values (channel decay), else a scalar.
-template <bool CHAN>
+// MODE 0: scalar Gamma_C.  MODE 1: Gamma_C a vector of d_k values (channel
+// decay).  MODE 2: as 1, plus the record's (P^d V)^T and (Dt^T V)^T terms added
+// to the output and to the state (GDN-2); each compute thread loads its share
+// of them from the record one chunk ahead.
+template <int MODE>
 __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
+  constexpr bool CHAN = MODE >= 1;
   using namespace carry;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -776,8 +1162,8 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       const uint8_t *recs = p.ws + (static_cast<size_t>(b) * p.H + h) * NC * rb;
       auto issue_chunk = [&](int c) {
         const int s = c % NSTAGE;
-        mbar_expect_tx(&bar_full[s], rb);
-        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, rb, &bar_full[s]);
+        mbar_expect_tx(&bar_full[s], p.copy_bytes);
+        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, p.copy_bytes, &bar_full[s]);
         pend |= 1u << s;
       };
       auto wait_full = [&](int c) -> bool {
@@ -848,6 +1234,19 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       if (lane == 0) mbar_arrive(bar_sa);
     };
     store_state();
+    // MODE 2: this thread's (P^d V)^T (tokens 16 part ..) and (Dt^T V)^T (rows 32 part ..)
+    uint4 od_raw[2], sd_raw[4];
+    auto load_local = [&](int c) {
+      const uint8_t *r = p.ws + ((static_cast<size_t>(b) * p.H + h) * NC + c) * rb + p.copy_bytes;
+      const uint4 *od = reinterpret_cast<const uint4 *>(r + v * 128 + part * 32);
+      const uint4 *sd = reinterpret_cast<const uint4 *>(r + 8192 * NS + v * 256 + part * 64);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) od_raw[j] = has_v ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sd_raw[j] = has_v ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    if constexpr (MODE == 2)
+      if (NC > 0) load_local(0);
     for (int c = 0; c < NC; ++c) {
       uint8_t *st = sm + (c % NSTAGE) * STAGE;
       const uint32_t y = lrow + COL_Y + 128 * (c & 1);
@@ -896,6 +1295,18 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
         float d[32];
         tmem_ld32(lrow + COL_DS + 32 * part, d);
+        if constexpr (MODE == 2) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[j]);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __half22float2(hp[q2]);
+              d[8 * j + 2 * q2] += f.x;
+              d[8 * j + 2 * q2 + 1] += f.y;
+            }
+          }
+        }
 #pragma unroll
         for (int m = 0; m < 32; ++m) {
           S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d[m]);
@@ -913,6 +1324,19 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         float yo[16];
         tmem_ld16(y + 64 + 16 * part, yo);
         tmem_wait_ld();
+        if constexpr (MODE == 2) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&od_raw[j]);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __half22float2(hp[q2]);
+              yo[8 * j + 2 * q2] += f.x;
+              yo[8 * j + 2 * q2 + 1] += f.y;
+            }
+          }
+          if (c + 1 < NC) load_local(c + 1);
+        }
         if (has_v) {
           uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
 #pragma unroll
@@ -1009,6 +1433,28 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t s
   return e;
 }
 
+cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
+  cudaError_t e = cudaFuncSetAttribute(chunk_prep_gdn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)prepg::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    *err = "cudaFuncSetAttribute: ";
+    return e;
+  }
+  CUtensorMap mq, mk, mv, mg;
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map(&mk, p.k, p.B, p.T, p.H, p.dk) ||
+      !make_map(&mv, p.v, p.B, p.T, p.H, p.dv) || !make_map_f32_rows(&mg, p.log_g, p.B, p.T, p.H, p.dk)) {
+    *err = "cuTensorMapEncodeTiled failed: ";
+    return cudaErrorInvalidValue;
+  }
+  PrepG2Params pp;
+  pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.erase_b = p.erase_b; pp.write_w = p.write_w; pp.ws = ws; pp.scale = p.scale;
+  chunk_prep_gdn2_kernel<<<dim3(NC, p.H, p.B), NTHREADS, prepg::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *err = "prep launch: ";
+  return e;
+}
+
 cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_chan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prepc::SMEM_BYTES);
@@ -1032,9 +1478,9 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   return e;
 }
 
-template <bool CHAN>
+template <int MODE>
 cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, cudaStream_t stream, std::string *err) {
-  cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<CHAN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)carry::SMEM_BYTES);
   if (e != cudaSuccess) {
     *err = "cudaFuncSetAttribute: ";
@@ -1042,10 +1488,12 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, cudaStr
   }
   CarryParams cp;
   cp.T = p.T; cp.H = p.H; cp.dv = p.dv; cp.NC = NC;
-  cp.rec_bytes = CHAN ? rec_bytes_chan(p.dv / 64) : rec_bytes(p.dv / 64);
+  const int ns = p.dv / 64;
+  cp.rec_bytes = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
+  cp.copy_bytes = MODE == 0 ? rec_bytes(ns) : rec_bytes_chan(ns);
   cp.ws = ws; cp.s0 = p.s0; cp.s_final = p.s_final;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<CHAN><<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
+  chunk_carry_kernel<MODE><<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
@@ -1057,9 +1505,10 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   uint8_t *w = static_cast<uint8_t *>(ws);
   cudaError_t e;
   if constexpr (VAR == kKDA) e = launch_prep_chan(p, NC, w, stream, err);
+  else if constexpr (VAR == kGDN2) e = launch_prep_gdn2(p, NC, w, stream, err);
   else e = launch_prep<VAR>(p, NC, w, stream, err);
   if (e != cudaSuccess) return e;
-  return launch_carry<VAR == kKDA>(p, NC, w, stream, err);
+  return launch_carry<VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0>(p, NC, w, stream, err);
 }
 
 }  // namespace
@@ -1068,13 +1517,16 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
 
 bool gdr_split_supported(int variant, int dk, int dv) {
   using namespace gdr;
-  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA;
+  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA ||
+                 variant == kGDN2;
   return v && dk == 128 && (dv == 64 || dv == 128);
 }
 
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   const size_t NC = (static_cast<size_t>(T) + 63) / 64;
-  const size_t rec = variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64) : gdr::tc::rec_bytes(dv / 64);
+  const size_t rec = variant == gdr::kGDN2  ? gdr::tc::rec_bytes_gdn2(dv / 64)
+                     : variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64)
+                                            : gdr::tc::rec_bytes(dv / 64);
   return static_cast<size_t>(B) * H * NC * rec;
 }
 
@@ -1085,6 +1537,7 @@ cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t st
     case kGatedDeltaNet: return tc::launch_split<kGatedDeltaNet>(p, ws, stream, err);
     case kKLA: return tc::launch_split<kKLA>(p, ws, stream, err);
     case kKDA: return tc::launch_split<kKDA>(p, ws, stream, err);
+    case kGDN2: return tc::launch_split<kGDN2>(p, ws, stream, err);
     default: *err = "variant not covered: "; return cudaErrorInvalidValue;
   }
 }

@@ -148,7 +148,9 @@ def test_workspace_sizes(L):
     assert L.gdr_forward_workspace_size(1, 0, 8, 2048, 8, 128, 128, 0) == 0    # fp32: per-token
     # KDA: the same record with Gamma_C a vector of 128 floats
     assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 512)
-    assert L.gdr_forward_workspace_size(3, 1, 8, 2048, 8, 128, 128, 0) == 0    # GDN-2: per-token kernel
+    # GDN-2: the channel-decay record, then (P^d V)^T and (Dt^T V)^T (8 + 16 KB per 64 values)
+    assert L.gdr_forward_workspace_size(3, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 512 + 49152)
+    assert L.gdr_forward_kernel_name(3, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
     assert L.gdr_forward_kernel_name(1, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
     assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == 2
     assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
