@@ -97,11 +97,13 @@ typedef struct {
 
 /*
  * Bytes of device workspace gdr_forward_chunked uses for this problem and
- * `chunk` choice: B * H * ceil(T/64) records of 56 KB + 8 KB per 64 value
- * columns + 16 bytes for the two-kernel chunked path (chunk 0 or 65 with bf16 I/O,
- * dk = 128, DeltaNet / Gated DeltaNet / KLA), 0 otherwise.  The workspace is
- * caller-owned scratch, overwritten by every call; its contents are not
- * needed after the call completes on the stream.
+ * `chunk` choice: for the two-kernel chunked path (chunk 0 or 65 with bf16
+ * I/O and dk = 128) B * H * ceil(T/64) records of 56 KB + 8 KB per 64 value
+ * columns, plus 16 bytes (scalar decay: DeltaNet, Gated DeltaNet, KLA) or
+ * 512 bytes (channel decay: KDA), plus 24 KB per 64 value columns for GDN-2;
+ * 0 for every other path.  The workspace is caller-owned scratch, overwritten
+ * by every call; its contents are not needed after the call completes on
+ * the stream.
  */
 size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
                                   int dk, int dv, int chunk);
@@ -121,8 +123,8 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
  *      dk = 128;
  *   65 the two-kernel chunked path: a chunk-parallel preparation kernel (the
  *      S-independent products of every chunk, into the workspace) then the
- *      sequential carry kernel: DeltaNet, Gated DeltaNet, KLA with bf16 I/O,
- *      dk = 128; needs the workspace.
+ *      sequential carry kernel: all five variants with bf16 I/O and dk = 128;
+ *      needs the workspace.
  * A chunk value whose path does not cover the case returns GDR_ERR_UNSUPPORTED.
  * Shapes: B, T, H >= 0; dk in {64, 128}; dv in {64, 128}.  T = 0 copies
  * initial_state to final_state (or clears it); B * H = 0 does nothing.
@@ -144,14 +146,16 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
  * convenience.
  *
  * Arguments, layouts and results are those of gdr_forward_chunked.  It covers
- * DeltaNet, Gated DeltaNet and KLA with bf16 I/O, dk = 128, dv in {64, 128};
- * anything else returns GDR_ERR_UNSUPPORTED.
+ * the five variants with bf16 I/O, dk = 128, dv in {64, 128}; anything else
+ * returns GDR_ERR_UNSUPPORTED.
  *
  * The fixed scratch is a 32 MiB device array in the library's device image:
  * every GPU that loads the library holds it until the process exits.  A call
- * needs B * H * ceil(T / 64) records of 73744 bytes (dv = 128) or 65552 bytes
- * (dv = 64), i.e. B * H * ceil(T / 64) <= 455 (dv = 128) or <= 511 (dv = 64); larger
- * problems return GDR_ERR_UNSUPPORTED with the limit in gdr_last_error().
+ * needs B * H * ceil(T / 64) records of the size gdr_forward_workspace_size
+ * implies, so B * H * ceil(T / 64) may be at most 32 MiB over the record
+ * size: 455 at dv = 128 (511 at dv = 64) for DeltaNet, Gated DeltaNet and
+ * KLA, 451 (508) for KDA, 271 (370) for GDN-2.  Larger problems return
+ * GDR_ERR_UNSUPPORTED with the limit in gdr_last_error().
  * The first call on each device looks up the array's device address (and may
  * load the library's device code); make that first call before any stream
  * capture.  All calls share the array and each call rewrites what it uses
