@@ -1105,6 +1105,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
 // decay).  MODE 2: as 1, plus the record's (P^d V)^T and (Dt^T V)^T terms added
 // to the output and to the state (GDN-2); each compute thread loads its share
 // of them from the record one chunk ahead.
+// 17 warps: one SM sub-partition holds five of them, so 96 registers per thread.
 template <int MODE>
 __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
   constexpr bool CHAN = MODE >= 1;
@@ -1293,24 +1294,29 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       tc_fence_after();
       {
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
-        float d[32];
-        tmem_ld32(lrow + COL_DS + 32 * part, d);
-        if constexpr (MODE == 2) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[j]);
+        for (int hv = 0; hv < 2; ++hv) {   // two halves of 16 rows keep the register count down
+          float d[16];
+          tmem_ld16(lrow + COL_DS + 32 * part + 16 * hv, d);
+          tmem_wait_ld();
+          if constexpr (MODE == 2) {
 #pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              const float2 f = __half22float2(hp[q2]);
-              d[8 * j + 2 * q2] += f.x;
-              d[8 * j + 2 * q2 + 1] += f.y;
+            for (int j = 0; j < 2; ++j) {
+              const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[2 * hv + j]);
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const float2 f = __half22float2(hp[q2]);
+                d[8 * j + 2 * q2] += f.x;
+                d[8 * j + 2 * q2 + 1] += f.y;
+              }
             }
           }
-        }
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d[m]);
-          smax = fmaxf(smax, fabsf(S[m]));
+          for (int m = 0; m < 16; ++m) {
+            const int i = 16 * hv + m;
+            S[i] = fmaf(gcv[CHAN ? i : 0], S[i], d[m]);
+            smax = fmaxf(smax, fabsf(S[i]));
+          }
         }
         store_state();
       }

@@ -22,16 +22,16 @@ from gated_delta_rule_forward_b200.inputs import make_inputs, random_state
 from parity_util import assert_gpu_close, gate_kwargs, to_dev
 
 pytestmark = pytest.mark.gpu
-VARIANT_IDS = {"deltanet": 0, "gdn": 1, "kla": 4}
+VARIANT_IDS = {"deltanet": 0, "gdn": 1, "kda": 2, "gdn2": 3, "kla": 4}
 
 
 def call_noalloc(variant, d, S0, B, T, H, dv):
     o = torch.empty(B, T, H, dv, device="cuda", dtype=torch.bfloat16)
     S = torch.empty(B, H, 128, dv, device="cuda", dtype=torch.float32)
+    ptr = lambda name: None if d.get(name) is None else d[name].data_ptr()
     a = _lib.FwdArgs(q=d["q"].data_ptr(), k=d["k"].data_ptr(), v=d["v"].data_ptr(),
-                     beta=d["beta"].data_ptr(),
-                     log_g=None if d["log_g"] is None else d["log_g"].data_ptr(),
-                     erase_b=None, write_w=None, initial_state=S0.data_ptr(),
+                     beta=ptr("beta"), log_g=ptr("log_g"), erase_b=ptr("erase_b"),
+                     write_w=ptr("write_w"), initial_state=S0.data_ptr(),
                      final_state=S.data_ptr(), o=o.data_ptr())
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     st = _lib.lib().gdr_forward_chunked_noalloc(VARIANT_IDS[variant], 1, B, T, H, 128, dv, ctypes.byref(a),
@@ -40,7 +40,8 @@ def call_noalloc(variant, d, S0, B, T, H, dv):
     return o, S
 
 
-@pytest.mark.parametrize("variant,dv", [("gdn", 128), ("kla", 64), ("deltanet", 128)])
+@pytest.mark.parametrize("variant,dv", [("gdn", 128), ("kla", 64), ("deltanet", 128), ("kda", 128),
+                                        ("gdn2", 64)])
 def test_noalloc_matches_workspace_path_twice(variant, dv):
     B, T, H = 2, 333, 3                     # ragged tail; 2 * 3 * 6 = 36 records
     d = to_dev(make_inputs(variant, B, T, H, 128, dv, dtype=torch.bfloat16, seed=41))
