@@ -409,7 +409,7 @@ constexpr uint32_t OFF_KG = OFF_R + 49152;      // (c..f) bf16 K o e^gamma [Kb0 
 constexpr uint32_t OFF_A = OFF_R;               // (d, e) fp32 A^T, 64 x LD
 constexpr uint32_t OFF_TF = OFF_R + 18432;      // (e) fp32 T, 64 x LD
 constexpr uint32_t OFF_T = OFF_R + 36864;       // (e, f) bf16 T
-constexpr uint32_t OFF_SC = OFF_R + 65536;      // beta [64], gamma_m [128], scratch [128]
+constexpr uint32_t OFF_SC = OFF_R + 65536;      // beta [64], e^{gamma_m} [128], scratch [128]
 constexpr uint32_t OFF_BAR = OFF_SC + 320 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T && OFF_T + 8192 <= OFF_KG, "phase region layout");
@@ -445,8 +445,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t *bar_mma = bar_in + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);   // [64]
-  float *sc_gm = sc_beta + 64;                               // [128] gamma_m (log2 units)
-  float *sc_tmp = sc_gm + 128;                               // [128]
+  float *sc_em = sc_beta + 64;                               // [128] e^{gamma_m} per channel
+  float *sc_tmp = sc_em + 128;                               // [128]
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
     __syncthreads();
     const float gm = sc_tmp[ch];
-    if (hh == 0) sc_gm[ch] = gm;
+    if (hh == 0) sc_em[ch] = ex2(gm);
 #pragma unroll 8
     for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
       float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
@@ -512,8 +512,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   __syncthreads();
   // Gamma_C per channel into the record
-  if (!bad && tid < DK)
-    reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * ex2(sc_gm[tid]);
+  if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
 
   // (b) inputs landed?
   if (!mbar_wait(bar_in, 0)) bad = 1;
@@ -535,14 +534,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
       const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
       const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
-      const float4 m4 = *reinterpret_cast<const float4 *>(sc_gm + ch0);
+      const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
       const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
-      const float em[4] = {ex2(m4.x), ex2(m4.y), ex2(m4.z), ex2(m4.w)};
+      const float em[4] = {m4.x, m4.y, m4.z, m4.w};
       const float bt = sc_beta[t];
       float kg[4], qg[4], ig[4], kt[4], qo[4], ke[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float inv = __frcp_rn(g[e]);
+        const float inv = rcp_approx(g[e]);
         kg[e] = tf32r(kx[e] * g[e]);
         qg[e] = tf32r(p.scale * qx[e] * g[e]);
         ig[e] = tf32r(kx[e] * inv);
@@ -702,7 +701,7 @@ constexpr uint32_t OFF_PD = OFF_R + 53248;      // fp16 P^d, rows t
 constexpr uint32_t OFF_RT = OFF_R + 61440;      // fp16 R, rows t
 constexpr uint32_t OFF_KG = OFF_R + 69632;      // (c..f) fp16 K o e^gamma [Kb0 | Kb1]
 constexpr uint32_t OFF_DT = OFF_R + 86016;      // (c..f) fp16 Dt [b0 | b1], rows r (MN-major operand)
-constexpr uint32_t OFF_SC = OFF_R + 102400;     // gamma_m [128], scratch [128]
+constexpr uint32_t OFF_SC = OFF_R + 102400;     // e^{gamma_m} [128], scratch [128]
 constexpr uint32_t OFF_BAR = OFF_SC + 256 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -742,8 +741,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t *bar_lg = bar_in + 1;
   uint64_t *bar_mma = bar_in + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
-  float *sc_gm = reinterpret_cast<float *>(sm + OFF_SC);     // [128] gamma_m (log2 units)
-  float *sc_tmp = sc_gm + 128;                               // [128]
+  float *sc_em = reinterpret_cast<float *>(sm + OFF_SC);     // [128] e^{gamma_m} per channel
+  float *sc_tmp = sc_em + 128;                               // [128]
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
@@ -774,6 +773,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = tid; i < 512; i += NTHREADS)
       reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
+  // erase / write gates of the (t, 4-channel) units this thread builds in pass hp,
+  // loaded one pass ahead so that no pass waits for global memory
+  float4 ebs[2][4], wrs[2][4];
+  auto load_gates = [&](int hp) {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int t = (it * NTHREADS + tid) >> 4, ch0 = 64 * hp + 4 * (tid & 15);
+      ebs[hp][it] = wrs[hp][it] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t0 + t < p.T) {
+        const size_t gi = ((static_cast<size_t>(b) * p.T + t0 + t) * p.H + h) * DK + ch0;
+        ebs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
+        wrs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
+      }
+    }
+  };
+  load_gates(0);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -795,7 +810,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (hh == 0) sc_tmp[ch] = run;
     __syncthreads();
     const float gm = sc_tmp[ch];
-    if (hh == 0) sc_gm[ch] = gm;
+    if (hh == 0) sc_em[ch] = ex2(gm);
 #pragma unroll 8
     for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
       float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
@@ -807,8 +822,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
   __syncthreads();
-  if (!bad && tid < DK)
-    reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * ex2(sc_gm[tid]);
+  if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
 
   // (b) inputs landed?
   if (!mbar_wait(bar_in, 0)) bad = 1;
@@ -816,9 +830,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float qkmax = 0.f;
 
   // (c) MMA1 in two 64-channel halves; the record's At and Qg; K o e^gamma and Dt for MMA2
-#pragma unroll 1
-  for (int hp = 0; hp < 2 && !bad; ++hp) {
-#pragma unroll 2
+#pragma unroll
+  for (int hp = 0; hp < 2; ++hp) {
+    if (bad) break;
+    if (hp == 0) load_gates(1);
+#pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
       const int t = u >> 4, j4 = u & 15;
@@ -827,22 +843,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float kx[4], qx[4];
       unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
       unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
-      float4 eb = make_float4(0.f, 0.f, 0.f, 0.f), wr = eb;
-      if (t0 + t < p.T) {
-        const size_t gi = ((static_cast<size_t>(b) * p.T + t0 + t) * p.H + h) * DK + ch0;
-        eb = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
-        wr = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
-      }
+      const float4 eb = ebs[hp][it], wr = wrs[hp][it];
       const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
       const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
-      const float4 m4 = *reinterpret_cast<const float4 *>(sc_gm + ch0);
+      const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
       const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
-      const float em[4] = {ex2(m4.x), ex2(m4.y), ex2(m4.z), ex2(m4.w)};
+      const float em[4] = {m4.x, m4.y, m4.z, m4.w};
       const float ebv[4] = {eb.x, eb.y, eb.z, eb.w}, wrv[4] = {wr.x, wr.y, wr.z, wr.w};
       float kg[4], qg[4], af[4], df[4], at[4], dt[4], qo[4], ke[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float inv = __frcp_rn(g[e]);
+        const float inv = rcp_approx(g[e]);
         const float a = ebv[e] * kx[e], d = (wrv[e] - ebv[e]) * kx[e];
         kg[e] = tf32r(kx[e] * g[e]);
         qg[e] = tf32r(p.scale * qx[e] * g[e]);
@@ -1165,6 +1176,8 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         const int s = c % NSTAGE;
         mbar_expect_tx(&bar_full[s], p.copy_bytes);
         bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, p.copy_bytes, &bar_full[s]);
+        // MODE 2: the rest of the record, which the compute threads read themselves
+        if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
         pend |= 1u << s;
       };
       auto wait_full = [&](int c) -> bool {
