@@ -1088,13 +1088,26 @@ constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace carry
 
+// Segments: CTA (h, b, z) sweeps chunks [z seg_len, (z + 1) seg_len) of its
+// (b, h).  Its initial state is s0 + z s0_seg_stride (zeros if s0 is null, the
+// identity if CARRY_IDENTITY); it writes its final state to s_final +
+// z s_final_seg_stride (only the last segment if CARRY_LAST_FINAL).
+enum CarryFlags : int {
+  CARRY_IDENTITY = 1,     // start from S = I (d_v = 128): the segment's transition map
+  CARRY_NO_VALUES = 2,    // U' and GDN-2's state-free terms taken as zero
+  CARRY_NO_OUTPUT = 4,    // write no output rows
+  CARRY_LAST_FINAL = 8,   // only the last segment writes s_final
+};
+
 struct CarryParams {
   int T, H, dv, NC;
+  int seg_len, flags;
   uint32_t rec_bytes;    // bytes per record
   uint32_t copy_bytes;   // leading bytes of a record that go through shared memory
   const uint8_t *ws;
   const float *s0;
   float *s_final;
+  size_t s0_seg_stride, s_final_seg_stride;   // elements between segments' states
   __nv_bfloat16 *o;
 };
 
@@ -1125,7 +1138,9 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int NS = p.dv / 64, NC = p.NC;
+  const int c_first = blockIdx.z * p.seg_len;               // this CTA's first chunk
+  const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
+  const bool values = !(p.flags & CARRY_NO_VALUES);
 
   uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
   uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
@@ -1171,7 +1186,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   if (warp == NCOMPUTE) {
     // ---------------------------------------------------------------- issuer
     if (lane == 0) {
-      const uint8_t *recs = p.ws + (static_cast<size_t>(b) * p.H + h) * NC * rb;
+      const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
       auto issue_chunk = [&](int c) {
         const int s = c % NSTAGE;
         mbar_expect_tx(&bar_full[s], p.copy_bytes);
@@ -1235,7 +1250,10 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       const size_t base = ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
 #pragma unroll
       for (int k = 0; k < 32; ++k)
-        S[k] = (p.s0 != nullptr && has_v) ? __ldg(p.s0 + base + static_cast<size_t>(k) * p.dv) : 0.f;
+        S[k] = (p.flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
+               : (p.s0 != nullptr && has_v)
+                   ? __ldg(p.s0 + blockIdx.z * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv)
+                   : 0.f;
     }
     auto store_state = [&]() {
       uint32_t r[16];
@@ -1251,13 +1269,14 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     // MODE 2: this thread's (P^d V)^T (tokens 16 part ..) and (Dt^T V)^T (rows 32 part ..)
     uint4 od_raw[2], sd_raw[4];
     auto load_local = [&](int c) {
-      const uint8_t *r = p.ws + ((static_cast<size_t>(b) * p.H + h) * NC + c) * rb + p.copy_bytes;
+      const uint8_t *r = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first + c) * rb + p.copy_bytes;
       const uint4 *od = reinterpret_cast<const uint4 *>(r + v * 128 + part * 32);
       const uint4 *sd = reinterpret_cast<const uint4 *>(r + 8192 * NS + v * 256 + part * 64);
+      const bool on = has_v && values;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) od_raw[j] = has_v ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
+      for (int j = 0; j < 2; ++j) od_raw[j] = on ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sd_raw[j] = has_v ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+      for (int j = 0; j < 4; ++j) sd_raw[j] = on ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
     };
     if constexpr (MODE == 2)
       if (NC > 0) load_local(0);
@@ -1274,7 +1293,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         float e[16];
         tmem_ld16(y + 16 * part, e);
         tmem_wait_ld();
-        if (has_v) {
+        if (has_v && values) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const uint4 raw = *reinterpret_cast<const uint4 *>(st + REC_U + sw128(v, 2 * part + j));
@@ -1356,7 +1375,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           }
           if (c + 1 < NC) load_local(c + 1);
         }
-        if (has_v) {
+        if (has_v && !(p.flags & CARRY_NO_OUTPUT)) {
           uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
 #pragma unroll
           for (int m = 0; m < 16; ++m)
@@ -1365,7 +1384,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 #pragma unroll
           for (int it = 0; it < 2; ++it) {
             const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
-            const int t = c * C + 16 * part + tr;
+            const int t = (c_first + c) * C + 16 * part + tr;
             const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
             if (t < p.T)
               *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
@@ -1394,8 +1413,10 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     }
   } else if (warp < NCOMPUTE) {
     if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
-    if (p.s_final != nullptr && has_v) {
-      float *dst = p.s_final + ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+    const bool write_final = !(p.flags & CARRY_LAST_FINAL) || blockIdx.z + 1 == gridDim.z;
+    if (p.s_final != nullptr && has_v && write_final) {
+      float *dst = p.s_final + blockIdx.z * p.s_final_seg_stride +
+                   ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
 #pragma unroll
       for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
     }
@@ -1497,8 +1518,58 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   return e;
 }
 
+// Segment-start states: S_start[0] = s0 (zeros if null), S_start[g + 1] = M_g S_start[g] + D_g,
+// for one (b, h) and 16 value columns per CTA, in fp32.  M_g is the transition map of
+// segment g (the carry from the identity with the values taken as zero) and D_g its
+// end state from zero (both d_k x d_k / d_k x d_v, row-major).
+__global__ void __launch_bounds__(256) segment_chain_kernel(const float *s0, const float *M, const float *D,
+                                                            float *S_start, int G, int H, int dv) {
+  __shared__ float Sc[DK][16];
+  const int sl = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const size_t BH = static_cast<size_t>(gridDim.z) * H, bh = static_cast<size_t>(b) * H + h;
+  for (int e = tid; e < DK * 16; e += blockDim.x) {
+    const int i = e >> 4, j = e & 15;
+    const size_t at = (bh * DK + i) * dv + 16 * sl + j;
+    const float x = s0 != nullptr ? s0[at] : 0.f;
+    Sc[i][j] = x;
+    S_start[at] = x;
+  }
+  __syncthreads();
+  const int i = tid >> 1, j0 = 8 * (tid & 1);
+  for (int g = 0; g + 1 < G; ++g) {
+    const float *Mi = M + ((g * BH + bh) * DK + i) * DK;
+    const size_t at = ((g * BH + bh) * DK + i) * dv + 16 * sl + j0;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = D[at + j];
+    for (int k = 0; k < DK; k += 4) {
+      const float4 m = __ldg(reinterpret_cast<const float4 *>(Mi + k));
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        acc[j] = fmaf(m.x, Sc[k][j0 + j], fmaf(m.y, Sc[k + 1][j0 + j],
+                 fmaf(m.z, Sc[k + 2][j0 + j], fmaf(m.w, Sc[k + 3][j0 + j], acc[j]))));
+    }
+    __syncthreads();
+    const size_t out = (((g + 1) * BH + bh) * DK + i) * dv + 16 * sl + j0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      Sc[i][j0 + j] = acc[j];
+      S_start[out + j] = acc[j];
+    }
+    __syncthreads();
+  }
+}
+
+struct CarryLaunch {
+  int segments = 1, seg_len = 0, flags = 0;
+  const float *s0 = nullptr;
+  float *s_final = nullptr;
+  size_t s0_stride = 0, s_final_stride = 0;
+};
+
 template <int MODE>
-cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const CarryLaunch &l, cudaStream_t stream,
+                         std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)carry::SMEM_BYTES);
   if (e != cudaSuccess) {
@@ -1507,19 +1578,54 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, cudaStr
   }
   CarryParams cp;
   cp.T = p.T; cp.H = p.H; cp.dv = p.dv; cp.NC = NC;
+  cp.seg_len = l.seg_len; cp.flags = l.flags;
   const int ns = p.dv / 64;
   cp.rec_bytes = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
   cp.copy_bytes = MODE == 0 ? rec_bytes(ns) : rec_bytes_chan(ns);
-  cp.ws = ws; cp.s0 = p.s0; cp.s_final = p.s_final;
+  cp.ws = ws; cp.s0 = l.s0; cp.s_final = l.s_final;
+  cp.s0_seg_stride = l.s0_stride; cp.s_final_seg_stride = l.s_final_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<MODE><<<dim3(p.H, p.B), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
+  chunk_carry_kernel<MODE>
+      <<<dim3(p.H, p.B, l.segments), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
 }
 
+// Carry over segments when too few (b, h) sequences fill the machine: each of G
+// segments of a sequence gets its own CTA.  Phase 1 computes every segment's
+// affine map S_end = M_g S_start + D_g (two carries, from the identity with no
+// values and from zero); a chain kernel turns the maps into segment start
+// states; phase 2 runs every segment from its start with outputs.  The
+// sequential depth drops from NC chunks to about 2 NC / G.
+struct SegPlan {
+  int G = 1, L = 0;
+};
+SegPlan seg_plan(int B, int H, int dv, int NC) {
+  SegPlan sp;
+  sp.L = NC;
+  int dev = 0, sms = 0;
+  if (dv != 128 || NC < 64 || cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return sp;
+  }
+  const long long bh = static_cast<long long>(B) * H;
+  const int G = static_cast<int>(std::min<long long>(8, sms / (2 * bh) + 1));
+  if (G < 3) return sp;
+  sp.L = (NC + G - 1) / G;
+  sp.G = (NC + sp.L - 1) / sp.L;
+  return sp;
+}
+size_t seg_extra_floats(int B, int H, int dv, const SegPlan &sp) {
+  if (sp.G == 1) return 0;
+  const size_t bh = static_cast<size_t>(B) * H;
+  return (sp.G - 1) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.G * bh * DK * dv;
+}
+
 template <int VAR>
 cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
+  constexpr int MODE = VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0;
   const int NC = (p.T + C - 1) / C;
   uint8_t *w = static_cast<uint8_t *>(ws);
   cudaError_t e;
@@ -1527,7 +1633,44 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   else if constexpr (VAR == kGDN2) e = launch_prep_gdn2(p, NC, w, stream, err);
   else e = launch_prep<VAR>(p, NC, w, stream, err);
   if (e != cudaSuccess) return e;
-  return launch_carry<VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0>(p, NC, w, stream, err);
+  const SegPlan sp = seg_plan(p.B, p.H, p.dv, NC);
+  if (sp.G == 1) {
+    CarryLaunch l;
+    l.seg_len = NC;
+    l.s0 = p.s0;
+    l.s_final = p.s_final;
+    return launch_carry<MODE>(p, NC, w, l, stream, err);
+  }
+  const size_t bh = static_cast<size_t>(p.B) * p.H, ns = p.dv / 64;
+  const size_t rec = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
+  const size_t rec_total = (bh * NC * rec + 255) / 256 * 256;
+  float *Mb = reinterpret_cast<float *>(w + rec_total);
+  float *Db = Mb + (sp.G - 1) * bh * DK * DK;
+  float *Ss = Db + (sp.G - 1) * bh * DK * p.dv;
+  CarryLaunch m;   // phase 1: transition maps
+  m.segments = sp.G - 1; m.seg_len = sp.L;
+  m.flags = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
+  m.s_final = Mb; m.s_final_stride = bh * DK * DK;
+  e = launch_carry<MODE>(p, NC, w, m, stream, err);
+  if (e != cudaSuccess) return e;
+  CarryLaunch d;   // phase 1: end states from zero
+  d.segments = sp.G - 1; d.seg_len = sp.L;
+  d.flags = CARRY_NO_OUTPUT;
+  d.s_final = Db; d.s_final_stride = bh * DK * p.dv;
+  e = launch_carry<MODE>(p, NC, w, d, stream, err);
+  if (e != cudaSuccess) return e;
+  segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(p.s0, Mb, Db, Ss, sp.G, p.H, p.dv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *err = "segment chain launch: ";
+    return e;
+  }
+  CarryLaunch f;   // phase 2: every segment from its start, with outputs
+  f.segments = sp.G; f.seg_len = sp.L;
+  f.flags = CARRY_LAST_FINAL;
+  f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
+  f.s_final = p.s_final;
+  return launch_carry<MODE>(p, NC, w, f, stream, err);
 }
 
 }  // namespace
@@ -1546,7 +1689,15 @@ size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   const size_t rec = variant == gdr::kGDN2  ? gdr::tc::rec_bytes_gdn2(dv / 64)
                      : variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64)
                                             : gdr::tc::rec_bytes(dv / 64);
-  return static_cast<size_t>(B) * H * NC * rec;
+  const size_t records = static_cast<size_t>(B) * H * NC * rec;
+  const gdr::tc::SegPlan sp = gdr::tc::seg_plan(B, H, dv, static_cast<int>(NC));
+  if (sp.G == 1) return records;
+  return (records + 255) / 256 * 256 + 4 * gdr::tc::seg_extra_floats(B, H, dv, sp);
+}
+
+int gdr_split_launches(int B, int T, int H, int dv) {
+  const int NC = (T + 63) / 64;
+  return gdr::tc::seg_plan(B, H, dv, NC).G == 1 ? 2 : 5;
 }
 
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {

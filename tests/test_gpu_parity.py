@@ -142,6 +142,20 @@ def test_resume_split(variant, chunk):
     assert_gpu_close(Sb, S, "S")
 
 
+@pytest.mark.parametrize("variant", ["gdn", "kda", "kla", "gdn2"])
+def test_segmented_carry(variant):
+    """Few sequences, many chunks: the two-kernel path splits each sequence into
+    segments (transition maps, a chain of start states, then every segment from
+    its start).  B=1, H=2, T=4100 gives 65 chunks with a ragged tail; compared
+    element by element with the oracle, with an initial state."""
+    B, T, H = 1, 4100, 2
+    launches = gdr.forward_launches(variant, torch.bfloat16, B, T, H, 128, 128, 0)
+    assert launches == 5, f"expected the segmented carry (5 launches), got {launches}"
+    o, S, o_ref, S_ref = run_both(variant, B, T, H, 128, 128, torch.bfloat16, 0, seed=21)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
 def test_kla_is_gdn_with_kaczmarz_beta():
     """KLA = Gated DeltaNet with beta_t = eta_t / (||k_t||^2 + eps) ("Kaczmarz Linear
     Attention", implementation: only the diagonal coefficient matrix changes)."""
