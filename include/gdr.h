@@ -101,9 +101,12 @@ typedef struct {
  * I/O and dk = 128) B * H * ceil(T/64) records of 56 KB + 8 KB per 64 value
  * columns, plus 16 bytes (scalar decay: DeltaNet, Gated DeltaNet, KLA) or
  * 512 bytes (channel decay: KDA), plus 24 KB per 64 value columns for GDN-2;
- * 0 for every other path.  The workspace is caller-owned scratch, overwritten
- * by every call; its contents are not needed after the call completes on
- * the stream.
+ * 0 for every other path.  When few sequences of many chunks would leave
+ * most of the device idle (B * H small, dv = 128, T >= 4033), the carry runs
+ * in segments and the size adds their transition maps and start states
+ * (fp32, a few MB).  The workspace is caller-owned scratch, overwritten by
+ * every call; its contents are not needed after the call completes on the
+ * stream.
  */
 size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
                                   int dk, int dv, int chunk);
@@ -123,8 +126,9 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
  *      dk = 128;
  *   65 the two-kernel chunked path: a chunk-parallel preparation kernel (the
  *      S-independent products of every chunk, into the workspace) then the
- *      sequential carry kernel: all five variants with bf16 I/O and dk = 128;
- *      needs the workspace.
+ *      sequential carry kernel (for few long sequences: segment maps, a chain
+ *      of segment start states, then the segments in parallel): all five
+ *      variants with bf16 I/O and dk = 128; needs the workspace.
  * A chunk value whose path does not cover the case returns GDR_ERR_UNSUPPORTED.
  * Shapes: B, T, H >= 0; dk in {64, 128}; dv in {64, 128}.  T = 0 copies
  * initial_state to final_state (or clears it); B * H = 0 does nothing.
