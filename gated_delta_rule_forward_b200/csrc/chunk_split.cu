@@ -1266,20 +1266,24 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       if (lane == 0) mbar_arrive(bar_sa);
     };
     store_state();
-    // MODE 2: this thread's (P^d V)^T (tokens 16 part ..) and (Dt^T V)^T (rows 32 part ..)
+    // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
+    // each loaded from L2 (the issuer prefetches records there) just before the wait that
+    // precedes its use; short live ranges keep them out of local memory, where a pending
+    // load would stall its spill store
     uint4 od_raw[2], sd_raw[4];
-    auto load_local = [&](int c) {
-      const uint8_t *r = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first + c) * rb + p.copy_bytes;
-      const uint4 *od = reinterpret_cast<const uint4 *>(r + v * 128 + part * 32);
-      const uint4 *sd = reinterpret_cast<const uint4 *>(r + 8192 * NS + v * 256 + part * 64);
-      const bool on = has_v && values;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) od_raw[j] = on ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sd_raw[j] = on ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+    auto local_terms = [&](int c) {
+      return p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first + c) * rb + p.copy_bytes;
     };
-    if constexpr (MODE == 2)
-      if (NC > 0) load_local(0);
+    auto load_sd = [&](int c) {
+      const uint4 *sd = reinterpret_cast<const uint4 *>(local_terms(c) + 8192 * NS + v * 256 + part * 64);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sd_raw[j] = (has_v && values) ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto load_od = [&](int c) {
+      const uint4 *od = reinterpret_cast<const uint4 *>(local_terms(c) + v * 128 + part * 32);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
+    };
     for (int c = 0; c < NC; ++c) {
       uint8_t *st = sm + (c % NSTAGE) * STAGE;
       const uint32_t y = lrow + COL_Y + 128 * (c & 1);
@@ -1318,6 +1322,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_ea);
       }
+      if constexpr (MODE == 2) load_sd(c);
 
       // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row
       // for channel decay)
@@ -1351,6 +1356,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           }
         }
         store_state();
+        if constexpr (MODE == 2) load_od(c);
       }
 
       // output rows: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
@@ -1373,7 +1379,6 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
               yo[8 * j + 2 * q2 + 1] += f.y;
             }
           }
-          if (c + 1 < NC) load_local(c + 1);
         }
         if (has_v && !(p.flags & CARRY_NO_OUTPUT)) {
           uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
