@@ -436,232 +436,296 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int NS = p.dv / 64;
-  const int t0 = c * C;
+  const int total = p.NC * p.H * p.B;   // records, chunk index fastest
 
-  uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_lg = bar_in + 1;
-  uint64_t *bar_mma = bar_in + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
+  uint64_t *bar_kq = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // K, Q landed
+  uint64_t *bar_lg = bar_kq + 1;                                      // log g landed
+  uint64_t *bar_mma = bar_kq + 2;
+  uint64_t *bar_v = bar_kq + 3;                                       // V landed
+  uint64_t *bar_drain = bar_kq + 4;                                   // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_kq + 5);
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);   // [64]
   float *sc_em = sc_beta + 64;                               // [128] e^{gamma_m} per channel
   float *sc_tmp = sc_em + 128;                               // [128]
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
-  uint8_t *rec = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c) * rec_bytes_chan(NS);
   uint8_t *kq_ptr = sm + OFF_KQ;
+
+  // loads of record r (thread 0): log g and K, Q first, V once MMA2 no longer reads it
+  uint32_t issued = 0, landed = 0;   // thread 0: loads issued / seen landing (lg | kq << 8 | v << 16)
+  auto issue_kq_lg = [&](int r) {
+    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    mbar_expect_tx(bar_lg, 64 * DK * 4);
+    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, c * C, b);
+    mbar_expect_tx(bar_kq, 4 * 8192);
+    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_kq, 0, h, c * C, b);
+    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_kq, 0, h, c * C, b);
+    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_kq, 64, h, c * C, b);
+    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_kq, 64, h, c * C, b);
+    issued += 1u | (1u << 8);
+  };
+  auto issue_v = [&](int r) {
+    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    mbar_expect_tx(bar_v, NS * 8192);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_v, 64 * sl, h, c * C, b);
+    issued += 1u << 16;
+  };
+  auto load_beta = [&](int r) -> float {   // threads 0-63
+    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const int t = c * C + tid;
+    return (t < p.T) ? __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h) : 0.f;
+  };
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar_in, 1);
+    mbar_init(bar_kq, 1);
     mbar_init(bar_lg, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
-    mbar_expect_tx(bar_lg, 64 * DK * 4);
-    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, t0, b);
-    mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
-    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
-    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_g);
+    if (static_cast<int>(blockIdx.x) < total) {
+      issue_kq_lg(blockIdx.x);
+      issue_v(blockIdx.x);
+    }
   }
   if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
     for (int i = tid; i < 512; i += NTHREADS)
       reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
-  if (tid < 64) {
-    const int t = t0 + tid;
-    sc_beta[tid] = (t < p.T) ? __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h) : 0.f;
-  }
+  float bt_next = (tid < 64 && static_cast<int>(blockIdx.x) < total) ? load_beta(blockIdx.x) : 0.f;
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   int bad = 0, range = 0;
-
-  // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
-  if (!mbar_wait(bar_lg, 0)) bad = 1;
-  bad = __syncthreads_or(bad);
-  if (!bad) {
-    const int ch = tid & 127, hh = tid >> 7;
-    float run = 0.f;
-#pragma unroll 8
-    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-      run += Gr[t * DK + ch] * LOG2E;
-      Gr[t * DK + ch] = run;
-    }
-    if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
-    __syncthreads();
-    const float gm = sc_tmp[ch];
-    if (hh == 0) sc_em[ch] = ex2(gm);
-#pragma unroll 8
-    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-      float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
-      if (d > SPAN_SAFE || d < -SPAN_SAFE) {
-        range = 1;
-        d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
-      }
-      Gr[t * DK + ch] = ex2(d);
-    }
-  }
-  __syncthreads();
-  // Gamma_C per channel into the record
-  if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
-
-  // (b) inputs landed?
-  if (!mbar_wait(bar_in, 0)) bad = 1;
-  bad = __syncthreads_or(bad);
   uint32_t mma_phase = 0;
-  float qkmax = 0.f;
+  float wmax_all = 0.f;
 
-  // (c) MMA1 in two 64-channel halves; the record's Kt and Qg, and K o e^gamma for MMA2
-#pragma unroll 1
-  for (int hp = 0; hp < 2 && !bad; ++hp) {
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
-      const int t = u >> 4, j4 = u & 15;
-      const int ch0 = 64 * hp + 4 * j4;
-      const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);   // 4 values of a 16-bit tile row
-      float kx[4], qx[4];
-      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
-      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
-      const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
-      const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
-      const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
-      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
-      const float em[4] = {m4.x, m4.y, m4.z, m4.w};
-      const float bt = sc_beta[t];
-      float kg[4], qg[4], ig[4], kt[4], qo[4], ke[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float inv = rcp_approx(g[e]);
-        kg[e] = tf32r(kx[e] * g[e]);
-        qg[e] = tf32r(p.scale * qx[e] * g[e]);
-        ig[e] = tf32r(kx[e] * inv);
-        kt[e] = bt * kx[e] * (g63[e] * inv);
-        qo[e] = p.scale * qx[e] * g[e] * em[e];
-        ke[e] = kx[e] * g[e] * em[e];
-        qkmax = fmaxf(qkmax, fmaxf(fabsf(kt[e]), fabsf(qo[e])));
+  // Persistent over records (one CTA per SM): the next record's log g, K and Q
+  // are loaded once MMA1 has consumed this record's, its V once MMA2 has.
+  for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    const uint32_t ph = ((r - blockIdx.x) / gridDim.x) & 1;   // phase of the input barriers
+    uint8_t *rec = p.ws + static_cast<size_t>(r) * rec_bytes_chan(NS);
+    if (tid < 64) {
+      sc_beta[tid] = bt_next;
+      if (r + static_cast<int>(gridDim.x) < total) bt_next = load_beta(r + gridDim.x);
+    }
+    __syncthreads();
+
+    // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
+    if (!mbar_wait(bar_lg, ph)) bad = 1;
+    else if (tid == 0) landed += 1u;
+    bad = __syncthreads_or(bad);
+    if (!bad) {
+      const int ch = tid & 127, hh = tid >> 7;
+      float run = 0.f;
+#pragma unroll 8
+      for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+        run += Gr[t * DK + ch] * LOG2E;
+        Gr[t * DK + ch] = run;
       }
-      const uint32_t xa = (j4 >> 3) * 16384, ya = (j4 >> 3) * 8192;
-      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(t, j4 & 7)) = make_float4(kg[0], kg[1], kg[2], kg[3]);
-      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(64 + t, j4 & 7)) = make_float4(qg[0], qg[1], qg[2], qg[3]);
-      *reinterpret_cast<float4 *>(sm + OFF_YF + ya + sw128(t, j4 & 7)) = make_float4(ig[0], ig[1], ig[2], ig[3]);
-      *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
-          make_uint2(pack_f16x2(kt[0], kt[1]), pack_f16x2(kt[2], kt[3]));
-      *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
-          make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
-      *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
-          make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
+      if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
+      __syncthreads();
+      const float gm = sc_tmp[ch];
+      if (hh == 0) sc_em[ch] = ex2(gm);
+#pragma unroll 8
+      for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+        float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
+        if (d > SPAN_SAFE || d < -SPAN_SAFE) {
+          range = 1;
+          d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
+        }
+        Gr[t * DK + ch] = ex2(d);
+      }
+    }
+    __syncthreads();
+    // Gamma_C per channel into the record
+    if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
+
+    // (b) K and Q landed?
+    if (!mbar_wait(bar_kq, ph)) bad = 1;
+    else if (tid == 0) landed += 1u << 8;
+    bad = __syncthreads_or(bad);
+    float qkmax = 0.f;
+
+    // (c) MMA1 in two 64-channel halves; the record's Kt and Qg, and K o e^gamma for MMA2
+#pragma unroll 1
+    for (int hp = 0; hp < 2 && !bad; ++hp) {
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
+        const int t = u >> 4, j4 = u & 15;
+        const int ch0 = 64 * hp + 4 * j4;
+        const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);   // 4 values of a 16-bit tile row
+        float kx[4], qx[4];
+        unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+        unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
+        const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
+        const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
+        const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
+        const float em[4] = {m4.x, m4.y, m4.z, m4.w};
+        const float bt = sc_beta[t];
+        float kg[4], qg[4], ig[4], kt[4], qo[4], ke[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float inv = rcp_approx(g[e]);
+          kg[e] = tf32r(kx[e] * g[e]);
+          qg[e] = tf32r(p.scale * qx[e] * g[e]);
+          ig[e] = tf32r(kx[e] * inv);
+          kt[e] = bt * kx[e] * (g63[e] * inv);
+          qo[e] = p.scale * qx[e] * g[e] * em[e];
+          ke[e] = kx[e] * g[e] * em[e];
+          qkmax = fmaxf(qkmax, fmaxf(fabsf(kt[e]), fabsf(qo[e])));
+        }
+        const uint32_t xa = (j4 >> 3) * 16384, ya = (j4 >> 3) * 8192;
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(t, j4 & 7)) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw128(64 + t, j4 & 7)) = make_float4(qg[0], qg[1], qg[2], qg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_YF + ya + sw128(t, j4 & 7)) = make_float4(ig[0], ig[1], ig[2], ig[3]);
+        *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
+            make_uint2(pack_f16x2(kt[0], kt[1]), pack_f16x2(kt[2], kt[3]));
+        *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
+            make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
+        *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
+            make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   sdesc(yf + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 64, false, false),
+                   hp + kk > 0);
+        mma_commit(bar_mma);
+      }
+      if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+      bad = __syncthreads_or(bad);
+      mma_phase ^= 1;
+      tc_fence_after();
+    }
+
+    // log g, K and Q are consumed: the next record's are loaded from here on
+    if (!bad && tid == 0 && r + static_cast<int>(gridDim.x) < total) issue_kq_lg(r + gridDim.x);
+
+    // (d) A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
+    if (!bad) {
+      float g[32];
+      tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
+      const int t = row & 63;
+      const int r0 = 32 * half;
+      if (quad < 2) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * sc_beta[r0 + r]) : 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? g[r] * sc_beta[r0 + r] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // (e) T = (I + A)^{-1} as a bf16 tile
+    solve_unit_lower_64(At, Tf, tid, warp, lane);
+    {
+      const int m = tid >> 2, n0 = (tid & 3) * 16;
+      float tv[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0) {
+
+    // (f) MMA2: W = T (K o e^gamma) (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
+    if (!bad && tid == 0 && !mbar_wait(bar_v, ph)) bad = 1;
+    else if (!bad && tid == 0) landed += 1u << 16;
+    if (!bad && tid == 0) {
       tc_fence_after();
-      const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+      const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(yf + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 64, false, false),
-                 hp + kk > 0);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+                 idesc_bf16(64, 128, false, true), kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+                 idesc_bf16(128, 64, true, false), kk > 0);
       mma_commit(bar_mma);
     }
-    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
-  }
+    // V is consumed: the next record's is loaded during the epilogue
+    if (!bad && tid == 0 && r + static_cast<int>(gridDim.x) < total) issue_v(r + gridDim.x);
 
-  // (d) A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
-  if (!bad) {
-    float g[32];
-    tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
-    const int t = row & 63;
-    const int r0 = 32 * half;
-    if (quad < 2) {
+    // (g) -W (M64 layout) and U'^T -> fp16 record tiles
+    float wmax = qkmax;
+    if (!bad) {
+      float w[32];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * sc_beta[r0 + r]) : 0.f;
-    } else {
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+        if (lane < 16) {
 #pragma unroll
-      for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? g[r] * sc_beta[r0 + r] : 0.f;
+          for (int e = 0; e < 32; ++e) {
+            wmax = fmaxf(wmax, fabsf(w[e]));
+            w[e] = -w[e];
+          }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // (e) T = (I + A)^{-1} as a bf16 tile
-  solve_unit_lower_64(At, Tf, tid, warp, lane);
-  {
-    const int m = tid >> 2, n0 = (tid & 3) * 16;
-    float tv[16];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
-      tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
-    }
-#pragma unroll
-    for (int e = 0; e < 16; ++e) tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
-  }
-  fence_async_smem();
-  __syncthreads();
-
-  // (f) MMA2: W = T (K o e^gamma) (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
-  if (!bad && tid == 0) {
-    tc_fence_after();
-    const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
-               idesc_bf16(64, 128, false, true), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
-               idesc_bf16(128, 64, true, false), kk > 0);
-    mma_commit(bar_mma);
-  }
-  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
-  bad = __syncthreads_or(bad);
-  tc_fence_after();
-
-  // (g) -W (M64 layout) and U'^T -> fp16 record tiles
-  float wmax = qkmax;
-  if (!bad) {
-    float w[32];
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
-      if (lane < 16) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          wmax = fmaxf(wmax, fabsf(w[e]));
-          w[e] = -w[e];
+          for (int j = 0; j < 4; ++j)
+            st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
         }
+      }
+      tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
+      if (row < p.dv) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
       }
     }
-    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
-    if (row < p.dv) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+    wmax_all = fmaxf(wmax_all, wmax);
+    // tensor-memory reads done before the next record's MMA1
+    tc_fence_before();
+    __syncthreads();
+    if (bad) break;
+  }
+
+  if (bad && tid == 0) {
+    // a wait gave up: report it, then let the MMAs and loads in flight finish
+    // (each wait again bounded) before tensor memory is released
+    atomicOr(&g_gdr_split_error, 1);
+    mma_commit(bar_drain);
+    mbar_wait(bar_drain, 0);
+    uint64_t *bars[3] = {bar_lg, bar_kq, bar_v};
+    for (int i = 0; i < 3; ++i) {
+      const uint32_t n_issued = (issued >> (8 * i)) & 0xffu, n_landed = (landed >> (8 * i)) & 0xffu;
+      if (n_issued != n_landed) mbar_wait(bars[i], n_landed & 1u);
     }
   }
-  if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
-  if (range || wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
+  if (range || wmax_all > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1517,7 +1581,16 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
-  chunk_prep_chan_kernel<<<dim3(NC, p.H, p.B), NTHREADS, prepc::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) {
+    *err = "device query: ";
+    return e;
+  }
+  const long long records = static_cast<long long>(NC) * p.H * p.B;
+  const int grid = static_cast<int>(std::min<long long>(records, sms));   // one CTA per SM, persistent
+  chunk_prep_chan_kernel<<<grid, NTHREADS, prepc::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
