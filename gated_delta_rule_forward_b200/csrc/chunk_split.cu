@@ -1,6 +1,7 @@
-// Two-kernel chunked forward for the scalar-decay variants (DeltaNet, Gated
-// DeltaNet, KLA): a chunk-parallel preparation kernel and a sequential carry
-// kernel, with the per-chunk products passed through a workspace.
+// Two-kernel chunked forward for all five variants (DeltaNet, Gated DeltaNet,
+// KLA, KDA, Gated DeltaNet-2): chunk-parallel preparation kernels and a
+// sequential carry kernel, with the per-chunk products passed through a
+// workspace.
 //
 // The chunk algebra is the one of chunk_tc.cu ("Kaczmarz Linear Attention",
 // KLA update rule and implementation; "Gated DeltaNet-2", technical core):
@@ -8,16 +9,30 @@
 //     O = Diag(scale Gamma) Q S0 + P E,   S_C = Gamma_C S0 + K^T Diag(w) E.
 // Everything that does not depend on S0 -- A, P, the solve, W, U' and the
 // scaled copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K -- is the bulk of
-// the work and is independent across chunks.  The preparation kernel computes
-// it with one CTA per (batch, head, chunk) over the whole machine (two CTAs
-// per SM) instead of inside the sequential sweep.  The carry kernel then does
-// only what depends on the state, one CTA per (batch, head), in transposed
-// form so that the state is the tensor-memory operand of every product:
+// the work and is independent across chunks.  A preparation kernel computes
+// it per (batch, head, chunk) over the whole machine instead of inside the
+// sequential sweep; there is one for the scalar decays (DeltaNet, GDN, KLA),
+// one for the per-channel decay of KDA (Gamma_C a vector, the Gram product
+// in tf32 around the middle token) and one for GDN-2, whose separate erase
+// and write gates add two state-free terms (P^d V into the output and
+// D~^T V into the state) that its record carries precomputed.
+//
+// The carry kernel does only what depends on the state, one CTA per
+// (batch, head), in transposed form so that the state is the tensor-memory
+// operand of every product:
 //     Y_W = S0^T (-W)^T,  Y_Q = S0^T Qg^T,  E^T = U'^T + Y_W,
 //     dS^T = E^T Kt,  O^T = Y_Q + E^T P^T,  S_C^T = Gamma_C S0^T + dS^T.
 // Lane v of tensor memory is value column v; S^T and E^T are written there in
 // fp16 by the threads that own them and read by the MMAs from there, so the
 // sweep moves no operand through shared memory except the record itself.
+// Its template MODE picks the decay of the state update: a scalar Gamma_C,
+// a per-channel Gamma_C, or the per-channel one plus the GDN-2 terms.
+//
+// With few long sequences (B*H CTAs leave most SMs idle) the carry is
+// segmented: each sequence is cut into G segments, the chunk maps of every
+// segment (S -> M_g S + D_g, computed by two state-only passes of the carry
+// kernel) are chained by a small kernel into each segment's start state, and
+// a last pass runs all segments at once from their start states.
 //
 // Workspace record per (b, h, chunk).  The tiles the MMAs read are images of
 // the 128-byte-swizzled shared-memory layout, so the carry kernel bulk-copies
@@ -27,7 +42,8 @@
 //     REC_K   fp16 Kt, rows t, atoms [d_k 0-63 | 64-127] (read as the MN-major operand)  16 KB
 //     REC_P   fp16 P, rows t, columns r                            8 KB
 //     REC_U   fp16 U'^T, rows v, columns t (swizzled 16-byte chunks) 8 KB per 64 values
-//     REC_SC  fp32 Gamma_C, padded to 16 bytes
+//     REC_SC  fp32 Gamma_C: one value padded to 16 bytes, or d_k values
+//     GDN-2 only: the P^d V and D~^T V terms, 24 KB per 64 values
 #include <algorithm>
 #include <mutex>
 
@@ -210,7 +226,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), idesc_bf16(128, 64, false, false), kk > 0);
+        mma_ss(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), idesc_bf16(128, 64, false, false), kk > 0);
       }
       mma_commit(bar_mma);
     }
@@ -317,11 +333,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
+        mma_ss(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
                  idesc_bf16(64, 128, false, true), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+        mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
                  idesc_bf16(128, 64, true, false), kk > 0);
       mma_commit(bar_mma);
     }
@@ -419,12 +435,6 @@ constexpr uint32_t COL_W = 64;    // M64 x 128
 constexpr uint32_t COL_U = 192;   // M128 x 64: U'^T
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prepc
-
-__device__ __forceinline__ void unpack4_bf16(uint2 u, float *x) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_prep_chan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -568,8 +578,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int ch0 = 64 * hp + 4 * j4;
         const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);   // 4 values of a 16-bit tile row
         float kx[4], qx[4];
-        unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
-        unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
         const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
         const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
         const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
@@ -665,11 +675,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+        mma_ss(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
                  idesc_bf16(64, 128, false, true), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+        mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
                  idesc_bf16(128, 64, true, false), kk > 0);
       mma_commit(bar_mma);
     }
@@ -905,8 +915,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int ch0 = 64 * hp + 4 * j4;
       const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);
       float kx[4], qx[4];
-      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
-      unpack4_bf16(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+      unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+      unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
       const float4 eb = ebs[hp][it], wr = wrs[hp][it];
       const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
       const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
@@ -1029,7 +1039,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tt = smem_u32(sm + OFF_T), iad = smem_u32(sm + OFF_IAD);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + COL_R, sdesc(tt + kk * 32, 16, 1024), sdesc(iad + kk * 2048, 8192, 1024),
+      mma_ss(tmem + COL_R, sdesc(tt + kk * 32, 16, 1024), sdesc(iad + kk * 2048, 8192, 1024),
                idesc_f16(64, 64, false, true), kk > 0);
     mma_commit(bar_mma);
   }
@@ -1059,11 +1069,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const uint64_t va = sdesc(vt + kk * 2048, 8192, 1024);
-      mma_bf16(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+      mma_ss(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
                idesc_f16(64, 128, false, true), kk > 0);
-      mma_bf16(tmem + COL_U, va, sdesc(rt + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
-      mma_bf16(tmem + COL_OD, va, sdesc(pd + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
-      mma_bf16(tmem + COL_SD, va, sdesc(dtt + kk * 2048, 8192, 1024), idesc_f16(128, 128, true, true), kk > 0);
+      mma_ss(tmem + COL_U, va, sdesc(rt + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+      mma_ss(tmem + COL_OD, va, sdesc(pd + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+      mma_ss(tmem + COL_SD, va, sdesc(dtt + kk * 2048, 8192, 1024), idesc_f16(128, 128, true, true), kk > 0);
     }
     mma_commit(bar_mma);
   }

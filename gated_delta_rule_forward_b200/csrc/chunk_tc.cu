@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), ID_G, kk > 0);
+        mma_ss(tmem + COL_G, sdesc(a, 16, 1024), sdesc(a, 16, 1024), ID_G, kk > 0);
       }
       mma_commit(bar_mma);
     }
@@ -337,10 +337,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t tp = smem_u32(sm + OFF_TP), zt = smem_u32(sm + OFF_ZT);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024), ID_W, kk > 0);
+        mma_ss(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024), ID_W, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(zt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), ID_U, kk > 0);
+        mma_ss(tmem + COL_YE, sdesc(zt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), ID_U, kk > 0);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t qw = smem_u32(sm + OFF_QW);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+        mma_ss(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                  sdesc(s_tile + kk * 2048, 8192, 1024), ID_YE, 1);
       mma_commit(bar_mma);
     }
@@ -424,11 +424,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t et = smem_u32(sm + OFF_E), pt = smem_u32(sm + OFF_P);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_S, sdesc(k16 + kk * 2048, 8192, 1024), sdesc(ew + kk * 2048, 8192, 1024), ID_DS,
+        mma_ss(tmem + COL_S, sdesc(k16 + kk * 2048, 8192, 1024), sdesc(ew + kk * 2048, 8192, 1024), ID_DS,
                  kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_PE, 1);
+        mma_ss(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_PE, 1);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;

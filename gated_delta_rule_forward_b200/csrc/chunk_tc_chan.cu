@@ -90,12 +90,6 @@ struct Params {
   float scale;
 };
 
-// Four bf16 values (8 bytes) to floats.
-__device__ __forceinline__ void unpack4(uint2 u, float *x) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
 
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -337,11 +331,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t zt = smem_u32(sm + OFF_ZT), kg = smem_u32(sm + OFF_KG);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_W, sdesc(zt + 8192 + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024), ID_W,
+        mma_ss(tmem + COL_W, sdesc(zt + 8192 + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024), ID_W,
                  kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(zt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), ID_U, kk > 0);
+        mma_ss(tmem + COL_YE, sdesc(zt + kk * 32, 16, 1024), sdesc(vt + kk * 2048, 8192, 1024), ID_U, kk > 0);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
@@ -390,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t qw = smem_u32(sm + OFF_QW);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+        mma_ss(tmem + COL_YE, sdesc(qw + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                  sdesc(s_tile + kk * 2048, 8192, 1024), ID_YE, 1);
       mma_commit(bar_mma);
     }
@@ -418,11 +412,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t kt = smem_u32(sm + OFF_KT), et = smem_u32(sm + OFF_E), pt = smem_u32(sm + OFF_P);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_S, sdesc(kt + kk * 2048, 8192, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_DS,
+        mma_ss(tmem + COL_S, sdesc(kt + kk * 2048, 8192, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_DS,
                  kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_PE, 1);
+        mma_ss(tmem + COL_YE, sdesc(pt + kk * 32, 16, 1024), sdesc(et + kk * 2048, 8192, 1024), ID_PE, 1);
       mma_commit(bar_mma);
     }
     if (!mbar_wait(bar_mma, mma_phase)) bad = 1;

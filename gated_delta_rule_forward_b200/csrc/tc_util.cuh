@@ -203,8 +203,9 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
-// D[tmem] (+)= A * B, issued by one thread.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+// D[tmem] (+)= A * B with A and B in shared memory (kind::f16: both operands
+// bf16 or both fp16, as the instruction descriptor says), issued by one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -301,6 +302,13 @@ __device__ __forceinline__ void st_chunk_f16(uint8_t *addr, const float *x) {
   u.x = pack_f16x2(x[0], x[1]); u.y = pack_f16x2(x[2], x[3]);
   u.z = pack_f16x2(x[4], x[5]); u.w = pack_f16x2(x[6], x[7]);
   *reinterpret_cast<uint4 *>(addr) = u;
+}
+
+// Four bf16 values (8 bytes) to floats.
+__device__ __forceinline__ void unpack4(uint2 u, float *x) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float *x) {
