@@ -29,10 +29,10 @@
 // a per-channel Gamma_C, or the per-channel one plus the GDN-2 terms.
 //
 // With few long sequences (B*H CTAs leave most SMs idle) the carry is
-// segmented: each sequence is cut into G segments, the chunk maps of every
-// segment (S -> M_g S + D_g, computed by two state-only passes of the carry
+// segmented: each sequence is cut into G segments, the affine maps of the
+// segments (S -> M_g S + D_g, computed by one state-only launch of the carry
 // kernel) are chained by a small kernel into each segment's start state, and
-// a last pass runs all segments at once from their start states.
+// a last launch runs all segments at once from their start states.
 //
 // Workspace record per (b, h, chunk).  The tiles the MMAs read are images of
 // the 128-byte-swizzled shared-memory layout, so the carry kernel bulk-copies
@@ -1162,15 +1162,20 @@ constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace carry
 
-// Segments: CTA (h, b, z) sweeps chunks [z seg_len, (z + 1) seg_len) of its
-// (b, h).  Its initial state is s0 + z s0_seg_stride (zeros if s0 is null, the
-// identity if CARRY_IDENTITY); it writes its final state to s_final +
-// z s_final_seg_stride (only the last segment if CARRY_LAST_FINAL).
+// Segments: a launch holds up to two passes over segments of seg_len chunks.
+// CTA (h, b, z) with z < z_split belongs to pass A and sweeps segment z of its
+// (b, h): initial state s0 + z s0_seg_stride (zeros if s0 is null, or for
+// z > 0 under CARRY_S0_FIRST; the identity under CARRY_IDENTITY), final state
+// to s_final + z s_final_seg_stride (only the last segment under
+// CARRY_LAST_FINAL).  CTA z >= z_split belongs to pass B: segment
+// seg_first_b + (z - z_split) with flags_b, no initial state but the identity
+// or zeros, final state to s_final_b + (z - z_split) s_final_b_seg_stride.
 enum CarryFlags : int {
   CARRY_IDENTITY = 1,     // start from S = I (d_v = 128): the segment's transition map
   CARRY_NO_VALUES = 2,    // U' and GDN-2's state-free terms taken as zero
   CARRY_NO_OUTPUT = 4,    // write no output rows
   CARRY_LAST_FINAL = 8,   // only the last segment writes s_final
+  CARRY_S0_FIRST = 16,    // only segment 0 starts from s0, the others from zero
 };
 
 struct CarryParams {
@@ -1182,6 +1187,10 @@ struct CarryParams {
   const float *s0;
   float *s_final;
   size_t s0_seg_stride, s_final_seg_stride;   // elements between segments' states
+  int z_split;                                // CTAs z >= z_split run pass B
+  int seg_first_b, flags_b;
+  float *s_final_b;
+  size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
 };
 
@@ -1212,9 +1221,12 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int c_first = blockIdx.z * p.seg_len;               // this CTA's first chunk
+  const bool pass_b = static_cast<int>(blockIdx.z) >= p.z_split;
+  const int zi = pass_b ? blockIdx.z - p.z_split : blockIdx.z;      // index within the pass
+  const int flags = pass_b ? p.flags_b : p.flags;
+  const int c_first = (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
   const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
-  const bool values = !(p.flags & CARRY_NO_VALUES);
+  const bool values = !(flags & CARRY_NO_VALUES);
 
   uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
   uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
@@ -1322,12 +1334,11 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     // ---------------------------------------------------------------- compute warps
     {
       const size_t base = ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+      const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
 #pragma unroll
       for (int k = 0; k < 32; ++k)
-        S[k] = (p.flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
-               : (p.s0 != nullptr && has_v)
-                   ? __ldg(p.s0 + blockIdx.z * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv)
-                   : 0.f;
+        S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
+               : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
     }
     auto store_state = [&]() {
       uint32_t r[16];
@@ -1454,7 +1465,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
             }
           }
         }
-        if (has_v && !(p.flags & CARRY_NO_OUTPUT)) {
+        if (has_v && !(flags & CARRY_NO_OUTPUT)) {
           uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
 #pragma unroll
           for (int m = 0; m < 16; ++m)
@@ -1492,9 +1503,10 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     }
   } else if (warp < NCOMPUTE) {
     if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
-    const bool write_final = !(p.flags & CARRY_LAST_FINAL) || blockIdx.z + 1 == gridDim.z;
-    if (p.s_final != nullptr && has_v && write_final) {
-      float *dst = p.s_final + blockIdx.z * p.s_final_seg_stride +
+    const bool write_final = !(flags & CARRY_LAST_FINAL) || zi + 1 == p.z_split;
+    float *sf = pass_b ? p.s_final_b : p.s_final;
+    if (sf != nullptr && has_v && write_final) {
+      float *dst = sf + zi * (pass_b ? p.s_final_b_seg_stride : p.s_final_seg_stride) +
                    ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
 #pragma unroll
       for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
@@ -1606,10 +1618,12 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   return e;
 }
 
-// Segment-start states: S_start[0] = s0 (zeros if null), S_start[g + 1] = M_g S_start[g] + D_g,
-// for one (b, h) and 16 value columns per CTA, in fp32.  M_g is the transition map of
-// segment g (the carry from the identity with the values taken as zero) and D_g its
-// end state from zero (both d_k x d_k / d_k x d_v, row-major).
+// Segment-start states for one (b, h) and 16 value columns per CTA, in fp32:
+//     S_start[0] = s0 (zeros if null),  S_start[1] = D_0,
+//     S_start[g + 1] = M_g S_start[g] + D_g  (g = 1 .. G - 2).
+// D_0 is segment 0's end state from s0 itself; for g >= 1, M_g is the transition
+// map of segment g (the carry from the identity with the values taken as zero,
+// d_k x d_k, stored at index g - 1) and D_g its end state from zero (d_k x d_v).
 __global__ void __launch_bounds__(256) segment_chain_kernel(const float *s0, const float *M, const float *D,
                                                             float *S_start, int G, int H, int dv) {
   __shared__ float Sc[DK][16];
@@ -1625,12 +1639,12 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *s0, con
   __syncthreads();
   const int i = tid >> 1, j0 = 8 * (tid & 1);
   for (int g = 0; g + 1 < G; ++g) {
-    const float *Mi = M + ((g * BH + bh) * DK + i) * DK;
     const size_t at = ((g * BH + bh) * DK + i) * dv + 16 * sl + j0;
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = D[at + j];
-    for (int k = 0; k < DK; k += 4) {
+    const float *Mi = g > 0 ? M + (((g - 1) * BH + bh) * DK + i) * DK : nullptr;
+    for (int k = 0; g > 0 && k < DK; k += 4) {
       const float4 m = __ldg(reinterpret_cast<const float4 *>(Mi + k));
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -1653,6 +1667,10 @@ struct CarryLaunch {
   const float *s0 = nullptr;
   float *s_final = nullptr;
   size_t s0_stride = 0, s_final_stride = 0;
+  // optional pass B in the same launch
+  int segments_b = 0, seg_first_b = 0, flags_b = 0;
+  float *s_final_b = nullptr;
+  size_t s_final_b_stride = 0;
 };
 
 template <int MODE>
@@ -1672,20 +1690,26 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.copy_bytes = MODE == 0 ? rec_bytes(ns) : rec_bytes_chan(ns);
   cp.ws = ws; cp.s0 = l.s0; cp.s_final = l.s_final;
   cp.s0_seg_stride = l.s0_stride; cp.s_final_seg_stride = l.s_final_stride;
+  cp.z_split = l.segments;
+  cp.seg_first_b = l.seg_first_b; cp.flags_b = l.flags_b;
+  cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<MODE>
-      <<<dim3(p.H, p.B, l.segments), carry::NTHREADS_CARRY, carry::SMEM_BYTES, stream>>>(cp);
+  chunk_carry_kernel<MODE><<<dim3(p.H, p.B, l.segments + l.segments_b), carry::NTHREADS_CARRY,
+                             carry::SMEM_BYTES, stream>>>(cp);
   e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
 }
 
 // Carry over segments when too few (b, h) sequences fill the machine: each of G
-// segments of a sequence gets its own CTA.  Phase 1 computes every segment's
-// affine map S_end = M_g S_start + D_g (two carries, from the identity with no
-// values and from zero); a chain kernel turns the maps into segment start
-// states; phase 2 runs every segment from its start with outputs.  The
-// sequential depth drops from NC chunks to about 2 NC / G.
+// segments of a sequence gets its own CTA.  Phase 1, one launch, computes the
+// affine map S_end = M_g S_start + D_g of every segment but the last: D_g is
+// the end state from zero, except that segment 0 starts from s0 itself, so
+// D_0 is already S_start[1] and segment 0 needs no M; M_g (g >= 1) is the
+// carry from the identity with the values taken as zero.  That is 2G - 3
+// state-only CTAs per (b, h), all resident at once.  A chain kernel turns the
+// maps into segment start states; phase 2 runs every segment from its start
+// with outputs.  The sequential depth drops from NC chunks to about 2 NC / G.
 struct SegPlan {
   int G = 1, L = 0;
 };
@@ -1698,8 +1722,9 @@ SegPlan seg_plan(int B, int H, int dv, int NC) {
     cudaGetLastError();
     return sp;
   }
+  // phase 1 runs (2G - 3) bh CTAs, at most one per SM
   const long long bh = static_cast<long long>(B) * H;
-  const int G = static_cast<int>(std::min<long long>(8, sms / (2 * bh) + 1));
+  const int G = static_cast<int>(std::min<long long>(16, (sms / bh + 3) / 2));
   if (G < 3) return sp;
   sp.L = (NC + G - 1) / G;
   sp.G = (NC + sp.L - 1) / sp.L;
@@ -1708,7 +1733,7 @@ SegPlan seg_plan(int B, int H, int dv, int NC) {
 size_t seg_extra_floats(int B, int H, int dv, const SegPlan &sp) {
   if (sp.G == 1) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
-  return (sp.G - 1) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.G * bh * DK * dv;
+  return (sp.G - 2) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.G * bh * DK * dv;
 }
 
 template <int VAR>
@@ -1733,19 +1758,18 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   const size_t rec = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
   const size_t rec_total = (bh * NC * rec + 255) / 256 * 256;
   float *Mb = reinterpret_cast<float *>(w + rec_total);
-  float *Db = Mb + (sp.G - 1) * bh * DK * DK;
+  float *Db = Mb + (sp.G - 2) * bh * DK * DK;
   float *Ss = Db + (sp.G - 1) * bh * DK * p.dv;
-  CarryLaunch m;   // phase 1: transition maps
+  CarryLaunch m;   // phase 1, pass A: end states of segments 0 .. G-2 (segment 0 from s0, the rest from zero)
   m.segments = sp.G - 1; m.seg_len = sp.L;
-  m.flags = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
-  m.s_final = Mb; m.s_final_stride = bh * DK * DK;
+  m.flags = CARRY_NO_OUTPUT | CARRY_S0_FIRST;
+  m.s0 = p.s0;
+  m.s_final = Db; m.s_final_stride = bh * DK * p.dv;
+  // pass B: transition maps of segments 1 .. G-2
+  m.segments_b = sp.G - 2; m.seg_first_b = 1;
+  m.flags_b = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
+  m.s_final_b = Mb; m.s_final_b_stride = bh * DK * DK;
   e = launch_carry<MODE>(p, NC, w, m, stream, err);
-  if (e != cudaSuccess) return e;
-  CarryLaunch d;   // phase 1: end states from zero
-  d.segments = sp.G - 1; d.seg_len = sp.L;
-  d.flags = CARRY_NO_OUTPUT;
-  d.s_final = Db; d.s_final_stride = bh * DK * p.dv;
-  e = launch_carry<MODE>(p, NC, w, d, stream, err);
   if (e != cudaSuccess) return e;
   segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(p.s0, Mb, Db, Ss, sp.G, p.H, p.dv);
   e = cudaGetLastError();
@@ -1785,7 +1809,7 @@ size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
 
 int gdr_split_launches(int B, int T, int H, int dv) {
   const int NC = (T + 63) / 64;
-  return gdr::tc::seg_plan(B, H, dv, NC).G == 1 ? 2 : 5;
+  return gdr::tc::seg_plan(B, H, dv, NC).G == 1 ? 2 : 4;
 }
 
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {

@@ -145,13 +145,24 @@ def test_resume_split(variant, chunk):
 @pytest.mark.parametrize("variant", ["gdn", "kda", "kla", "gdn2"])
 def test_segmented_carry(variant):
     """Few sequences, many chunks: the two-kernel path splits each sequence into
-    segments (transition maps, a chain of start states, then every segment from
-    its start).  B=1, H=2, T=4100 gives 65 chunks with a ragged tail; compared
-    element by element with the oracle, with an initial state."""
+    segments (segment 0's end state and the other segments' affine maps in one
+    launch, a chain of start states, then every segment from its start).
+    B=1, H=2, T=4100 gives 65 chunks with a ragged tail (13 segments of 5);
+    compared element by element with the oracle, with an initial state."""
     B, T, H = 1, 4100, 2
     launches = gdr.forward_launches(variant, torch.bfloat16, B, T, H, 128, 128, 0)
-    assert launches == 5, f"expected the segmented carry (5 launches), got {launches}"
+    assert launches == 4, f"expected the segmented carry (4 launches), got {launches}"
     o, S, o_ref, S_ref = run_both(variant, B, T, H, 128, 128, torch.bfloat16, 0, seed=21)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
+def test_segmented_carry_no_initial_state():
+    """Segmented carry from a zero state, B=2 H=3 T=4480 (70 chunks, 12 segments
+    of 6): segment 0 then starts from zeros like every other segment's offset."""
+    B, T, H = 2, 4480, 3
+    assert gdr.forward_launches("gdn", torch.bfloat16, B, T, H, 128, 128, 0) == 4
+    o, S, o_ref, S_ref = run_both("gdn", B, T, H, 128, 128, torch.bfloat16, 0, seed=22, s0=False)
     assert_close(o, o_ref, torch.bfloat16, "o")
     assert_close(S, S_ref, torch.bfloat16, "S")
 
