@@ -183,6 +183,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   }
   float lg_next = 0.f, bt_next = 0.f;
   if (tid < 64 && static_cast<int>(blockIdx.x) < total) load_gates(blockIdx.x, lg_next, bt_next);
+  // every CTA of this persistent grid is resident from the start, so the carry
+  // kernel may launch now: its CTAs take SMs as preparation CTAs finish and
+  // wait for this grid to complete before they read a record
+  griddep_launch_dependents();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -513,6 +517,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   float bt_next = (tid < 64 && static_cast<int>(blockIdx.x) < total) ? load_beta(blockIdx.x) : 0.f;
+  griddep_launch_dependents();   // persistent grid: the carry may launch now (see chunk_prep_kernel)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -1298,6 +1303,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
                  kk > 0);
         mma_commit(bar_e);
       };
+      griddep_wait();   // the records are the preparation kernel's output
       for (int c = 0; c < NSTAGE && c < NC; ++c) issue_chunk(c);
       bool ok = wait_or_abort(bar_sa, 0, abort) && wait_full(0);
       if (ok) issue_y(0);
@@ -1351,6 +1357,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       if (lane == 0) mbar_arrive(bar_sa);
     };
     store_state();
+    griddep_wait();   // before any read of the records (MODE 2 reads some directly)
     // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
     // each loaded from L2 (the issuer prefetches records there) just before the wait that
     // precedes its use; short live ranges keep them out of local memory, where a pending
@@ -1673,9 +1680,13 @@ struct CarryLaunch {
   size_t s_final_b_stride = 0;
 };
 
+// `after_prep`: the launch follows the preparation kernel on the stream and may
+// overlap its tail (programmatic stream serialization).  The carry reads the
+// initial state before it waits for the preparation grid, so this is only for
+// an initial state that no kernel of this call writes.
 template <int MODE>
-cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const CarryLaunch &l, cudaStream_t stream,
-                         std::string *err) {
+cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const CarryLaunch &l, bool after_prep,
+                         cudaStream_t stream, std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)carry::SMEM_BYTES);
   if (e != cudaSuccess) {
@@ -1694,9 +1705,18 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.seg_first_b = l.seg_first_b; cp.flags_b = l.flags_b;
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  chunk_carry_kernel<MODE><<<dim3(p.H, p.B, l.segments + l.segments_b), carry::NTHREADS_CARRY,
-                             carry::SMEM_BYTES, stream>>>(cp);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.H, p.B, l.segments + l.segments_b);
+  cfg.blockDim = dim3(carry::NTHREADS_CARRY);
+  cfg.dynamicSmemBytes = carry::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_prep ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<MODE>, cp);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
 }
@@ -1752,7 +1772,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
     l.seg_len = NC;
     l.s0 = p.s0;
     l.s_final = p.s_final;
-    return launch_carry<MODE>(p, NC, w, l, stream, err);
+    return launch_carry<MODE>(p, NC, w, l, true, stream, err);
   }
   const size_t bh = static_cast<size_t>(p.B) * p.H, ns = p.dv / 64;
   const size_t rec = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
@@ -1769,7 +1789,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   m.segments_b = sp.G - 2; m.seg_first_b = 1;
   m.flags_b = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
   m.s_final_b = Mb; m.s_final_b_stride = bh * DK * DK;
-  e = launch_carry<MODE>(p, NC, w, m, stream, err);
+  e = launch_carry<MODE>(p, NC, w, m, true, stream, err);
   if (e != cudaSuccess) return e;
   segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(p.s0, Mb, Db, Ss, sp.G, p.H, p.dv);
   e = cudaGetLastError();
@@ -1782,7 +1802,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   f.flags = CARRY_LAST_FINAL;
   f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
   f.s_final = p.s_final;
-  return launch_carry<MODE>(p, NC, w, f, stream, err);
+  return launch_carry<MODE>(p, NC, w, f, false, stream, err);   // reads the chain kernel's states
 }
 
 }  // namespace
