@@ -147,7 +147,7 @@ int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, in
   if (kern == Kernel::None) return 0;
   if ((long)B * H == 0) return 0;
   if (T == 0) return 1;  // state copy or clear
-  if (kern == Kernel::Split) return gdr_split_launches(B, T, H, dv);
+  if (kern == Kernel::Split) return gdr_split_launches(variant, B, T, H, dv);
   return kern == Kernel::ChunkTC ? gdr_chunk_tc_launches(B, T, H, dk, dv) : 1;
 }
 

@@ -105,10 +105,23 @@ constexpr uint32_t TMEM_COLS = 256;
 
 struct PrepParams {
   int B, T, H, dv, NC;
+  int c0, ncr;   // the launch prepares chunks [c0, c0 + ncr) of every (b, h)
   const float *beta, *log_g;
   uint8_t *ws;
   float eps, scale;
 };
+
+// Launch-local record r (chunk fastest) -> batch, head, chunk.
+struct RecIdx {
+  int b, h, c;
+};
+__device__ __forceinline__ RecIdx rec_idx(const PrepParams &p, int r) {
+  const int bh = r / p.ncr;
+  return {bh / p.H, bh % p.H, p.c0 + (r - bh * p.ncr)};
+}
+__device__ __forceinline__ size_t rec_index(const PrepParams &p, const RecIdx &x) {
+  return (static_cast<size_t>(x.b) * p.H + x.h) * p.NC + x.c;
+}
 
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 2)
@@ -121,7 +134,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;
   const int NS = p.dv / 64;
-  const int total = p.NC * p.H * p.B;   // records, chunk index fastest
+  const int total = p.ncr * p.H * p.B;   // records of this launch, chunk index fastest
 
   uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
   uint64_t *bar_mma = bar_in + 1;
@@ -137,7 +150,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 
   // TMA loads of record r's K, Q and V (thread 0)
   auto issue_inputs = [&](int r) {
-    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const RecIdx x = rec_idx(p, r);
+    const int c = x.c, h = x.h, b = x.b;
     const int t0 = c * C;
     mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
     tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
@@ -148,7 +162,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   };
   // log decay and beta of token `tid` of record r (threads 0-63)
   auto load_gates = [&](int r, float &lg, float &bt) {
-    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const RecIdx x = rec_idx(p, r);
+    const int c = x.c, h = x.h, b = x.b;
     const int t = c * C + tid;
     lg = 0.f;
     bt = 0.f;
@@ -199,7 +214,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   // Persistent over records: the next record's loads are issued as soon as
   // MMA2 has consumed this record's inputs, and land during the epilogue.
   for (int r = blockIdx.x; r < total; r += gridDim.x) {
-    uint8_t *rec = p.ws + static_cast<size_t>(r) * rec_bytes(NS);
+    uint8_t *rec = p.ws + rec_index(p, rec_idx(p, r)) * rec_bytes(NS);
     // gates: beta_t, cumulative log2 decay, Gamma_t
     if (tid < 64) {
       float x = lg_next * LOG2E;
@@ -404,6 +419,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  // Launched as a programmatic dependent of a carry grid (the pipelined
+  // sweep), this grid completes only after that carry, so whatever is ordered
+  // after it is ordered after both.  Without such a launch this returns at once.
+  griddep_wait();
 }
 
 // ------------------------------------------------------------------ preparation kernel, channel decay
@@ -451,7 +470,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;
   const int NS = p.dv / 64;
-  const int total = p.NC * p.H * p.B;   // records, chunk index fastest
+  const int total = p.ncr * p.H * p.B;   // records of this launch, chunk index fastest
 
   uint64_t *bar_kq = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // K, Q landed
   uint64_t *bar_lg = bar_kq + 1;                                      // log g landed
@@ -470,7 +489,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // loads of record r (thread 0): log g and K, Q first, V once MMA2 no longer reads it
   uint32_t issued = 0, landed = 0;   // thread 0: loads issued / seen landing (lg | kq << 8 | v << 16)
   auto issue_kq_lg = [&](int r) {
-    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const RecIdx x = rec_idx(p, r);
+    const int c = x.c, h = x.h, b = x.b;
     mbar_expect_tx(bar_lg, 64 * DK * 4);
     tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, c * C, b);
     mbar_expect_tx(bar_kq, 4 * 8192);
@@ -481,13 +501,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     issued += 1u | (1u << 8);
   };
   auto issue_v = [&](int r) {
-    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const RecIdx x = rec_idx(p, r);
+    const int c = x.c, h = x.h, b = x.b;
     mbar_expect_tx(bar_v, NS * 8192);
     for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_v, 64 * sl, h, c * C, b);
     issued += 1u << 16;
   };
   auto load_beta = [&](int r) -> float {   // threads 0-63
-    const int c = r % p.NC, h = (r / p.NC) % p.H, b = r / (p.NC * p.H);
+    const RecIdx x = rec_idx(p, r);
+    const int c = x.c, h = x.h, b = x.b;
     const int t = c * C + tid;
     return (t < p.T) ? __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h) : 0.f;
   };
@@ -530,7 +552,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // are loaded once MMA1 has consumed this record's, its V once MMA2 has.
   for (int r = blockIdx.x; r < total; r += gridDim.x) {
     const uint32_t ph = ((r - blockIdx.x) / gridDim.x) & 1;   // phase of the input barriers
-    uint8_t *rec = p.ws + static_cast<size_t>(r) * rec_bytes_chan(NS);
+    uint8_t *rec = p.ws + rec_index(p, rec_idx(p, r)) * rec_bytes_chan(NS);
     if (tid < 64) {
       sc_beta[tid] = bt_next;
       if (r + static_cast<int>(gridDim.x) < total) bt_next = load_beta(r + gridDim.x);
@@ -747,6 +769,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  // Launched as a programmatic dependent of a carry grid (the pipelined
+  // sweep), this grid completes only after that carry, so whatever is ordered
+  // after it is ordered after both.  Without such a launch this returns at once.
+  griddep_wait();
 }
 
 // ------------------------------------------------------------------ preparation kernel, GDN-2
@@ -1167,7 +1193,8 @@ constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace carry
 
-// Segments: a launch holds up to two passes over segments of seg_len chunks.
+// Segments: a launch holds up to two passes over segments of seg_len chunks,
+// counted from chunk c_base.
 // CTA (h, b, z) with z < z_split belongs to pass A and sweeps segment z of its
 // (b, h): initial state s0 + z s0_seg_stride (zeros if s0 is null, or for
 // z > 0 under CARRY_S0_FIRST; the identity under CARRY_IDENTITY), final state
@@ -1192,6 +1219,8 @@ struct CarryParams {
   const float *s0;
   float *s_final;
   size_t s0_seg_stride, s_final_seg_stride;   // elements between segments' states
+  size_t s0_bh_stride, s_final_bh_stride;     // elements between (b, h) states (d_k d_v when packed)
+  int c_base;                                 // chunk of segment 0's start
   int z_split;                                // CTAs z >= z_split run pass B
   int seg_first_b, flags_b;
   float *s_final_b;
@@ -1229,7 +1258,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   const bool pass_b = static_cast<int>(blockIdx.z) >= p.z_split;
   const int zi = pass_b ? blockIdx.z - p.z_split : blockIdx.z;      // index within the pass
   const int flags = pass_b ? p.flags_b : p.flags;
-  const int c_first = (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
+  const int c_first = p.c_base + (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
   const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
   const bool values = !(flags & CARRY_NO_VALUES);
 
@@ -1264,6 +1293,9 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t rb = p.rec_bytes;
+  // every CTA of this grid holds its SM: a preparation grid launched as this
+  // grid's programmatic dependent (the pipelined sweep) may take the others
+  griddep_launch_dependents();
 
   // issuer's view of the record copies: stage has a copy in flight / phase parity to wait for
   uint32_t pend = 0, par = 0;
@@ -1338,8 +1370,9 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     }
   } else {
     // ---------------------------------------------------------------- compute warps
+    griddep_wait();   // the initial state and the records may be the previous grid's output
     {
-      const size_t base = ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+      const size_t base = (static_cast<size_t>(b) * p.H + h) * p.s0_bh_stride + static_cast<size_t>(32 * part) * p.dv + v;
       const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
 #pragma unroll
       for (int k = 0; k < 32; ++k)
@@ -1357,7 +1390,6 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       if (lane == 0) mbar_arrive(bar_sa);
     };
     store_state();
-    griddep_wait();   // before any read of the records (MODE 2 reads some directly)
     // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
     // each loaded from L2 (the issuer prefetches records there) just before the wait that
     // precedes its use; short live ranges keep them out of local memory, where a pending
@@ -1514,7 +1546,8 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     float *sf = pass_b ? p.s_final_b : p.s_final;
     if (sf != nullptr && has_v && write_final) {
       float *dst = sf + zi * (pass_b ? p.s_final_b_seg_stride : p.s_final_seg_stride) +
-                   ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+                   (static_cast<size_t>(b) * p.H + h) * (pass_b ? static_cast<size_t>(DK) * p.dv : p.s_final_bh_stride) +
+                   static_cast<size_t>(32 * part) * p.dv + v;
 #pragma unroll
       for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
     }
@@ -1527,8 +1560,33 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   }
 }
 
+// Chunk range of a preparation launch and the SMs its persistent grid is sized for.
+struct PrepRange {
+  int c0 = 0, ncr = 0;   // chunks [c0, c0 + ncr); ncr = 0: all
+  int sms = 0;           // 0: the whole device
+  bool after_carry = false;   // launched as the programmatic dependent of the carry before it
+};
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 template <int VAR>
-cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
+                        std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
   // all of the unified L1 as shared memory, so that two preparation CTAs fit on an SM
@@ -1547,9 +1605,10 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t s
   }
   PrepParams pp;
   pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
-  // persistent grid: as many CTAs as fit on the device at once, none idle
+  // persistent grid: as many CTAs as fit on the device (or on rg.sms SMs) at once, none idle
   int dev = 0, sms = 0, per_sm = 0;
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1563,10 +1622,11 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t s
   // resident at once (105 KB of shared memory and 128 x 256 registers each),
   // so the grid is sized for at least two.  A CTA that does not fit only
   // starts later; no CTA waits on another.
-  const long long records = static_cast<long long>(NC) * p.H * p.B;
+  if (rg.sms > 0) sms = std::min(sms, rg.sms);
+  const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
   const int grid = static_cast<int>(std::min<long long>(records, static_cast<long long>(std::max(per_sm, 2)) * sms));
-  chunk_prep_kernel<VAR><<<grid, NTHREADS, prep::SMEM_BYTES, stream>>>(mq, mk, mv, pp);
-  e = cudaGetLastError();
+  e = launch_maybe_pdl(chunk_prep_kernel<VAR>, dim3(grid), dim3(NTHREADS), prep::SMEM_BYTES, stream, rg.after_carry,
+                       mq, mk, mv, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
 }
@@ -1593,7 +1653,8 @@ cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   return e;
 }
 
-cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
+                             std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_chan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prepc::SMEM_BYTES);
   if (e != cudaSuccess) {
@@ -1608,6 +1669,7 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
   }
   PrepParams pp;
   pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
   int dev = 0, sms = 0;
@@ -1617,10 +1679,11 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
     *err = "device query: ";
     return e;
   }
-  const long long records = static_cast<long long>(NC) * p.H * p.B;
+  if (rg.sms > 0) sms = std::min(sms, rg.sms);
+  const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
   const int grid = static_cast<int>(std::min<long long>(records, sms));   // one CTA per SM, persistent
-  chunk_prep_chan_kernel<<<grid, NTHREADS, prepc::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
-  e = cudaGetLastError();
+  e = launch_maybe_pdl(chunk_prep_chan_kernel, dim3(grid), dim3(NTHREADS), prepc::SMEM_BYTES, stream,
+                       rg.after_carry, mq, mk, mv, mg, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
 }
@@ -1670,22 +1733,24 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *s0, con
 }
 
 struct CarryLaunch {
+  int c_base = 0;
   int segments = 1, seg_len = 0, flags = 0;
   const float *s0 = nullptr;
   float *s_final = nullptr;
   size_t s0_stride = 0, s_final_stride = 0;
+  size_t s0_bh_stride = 0, s_final_bh_stride = 0;   // 0: d_k d_v (packed [B, H, d_k, d_v])
   // optional pass B in the same launch
   int segments_b = 0, seg_first_b = 0, flags_b = 0;
   float *s_final_b = nullptr;
   size_t s_final_b_stride = 0;
 };
 
-// `after_prep`: the launch follows the preparation kernel on the stream and may
-// overlap its tail (programmatic stream serialization).  The carry reads the
-// initial state before it waits for the preparation grid, so this is only for
-// an initial state that no kernel of this call writes.
+// `pdl`: launched with programmatic stream serialization, so that its CTAs may
+// start (allocate, set up) while the grid before it on the stream finishes;
+// every thread waits for that grid's completion before it reads the initial
+// state or a record.
 template <int MODE>
-cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const CarryLaunch &l, bool after_prep,
+cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const CarryLaunch &l, bool pdl,
                          cudaStream_t stream, std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_carry_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)carry::SMEM_BYTES);
@@ -1701,22 +1766,15 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.copy_bytes = MODE == 0 ? rec_bytes(ns) : rec_bytes_chan(ns);
   cp.ws = ws; cp.s0 = l.s0; cp.s_final = l.s_final;
   cp.s0_seg_stride = l.s0_stride; cp.s_final_seg_stride = l.s_final_stride;
+  cp.c_base = l.c_base;
+  cp.s0_bh_stride = l.s0_bh_stride ? l.s0_bh_stride : static_cast<size_t>(DK) * p.dv;
+  cp.s_final_bh_stride = l.s_final_bh_stride ? l.s_final_bh_stride : static_cast<size_t>(DK) * p.dv;
   cp.z_split = l.segments;
   cp.seg_first_b = l.seg_first_b; cp.flags_b = l.flags_b;
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.H, p.B, l.segments + l.segments_b);
-  cfg.blockDim = dim3(carry::NTHREADS_CARRY);
-  cfg.dynamicSmemBytes = carry::SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = after_prep ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<MODE>, cp);
-  if (e == cudaSuccess) e = cudaGetLastError();
+  e = launch_maybe_pdl(chunk_carry_kernel<MODE>, dim3(p.H, p.B, l.segments + l.segments_b),
+                       dim3(carry::NTHREADS_CARRY), carry::SMEM_BYTES, stream, pdl, cp);
   if (e != cudaSuccess) *err = "carry launch: ";
   return e;
 }
@@ -1756,17 +1814,113 @@ size_t seg_extra_floats(int B, int H, int dv, const SegPlan &sp) {
   return (sp.G - 2) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.G * bh * DK * dv;
 }
 
+// Pipelined sweep.  The carry runs B*H CTAs, one per SM, and leaves the other
+// SMs idle; when enough are left, the sequences are cut at chunk c_split and
+// four grids run back to back on the caller's stream, each launched as the
+// programmatic dependent of the one before it:
+//     prep [0, c_split) on the whole device;
+//     carry [0, c_split), its CTAs taking SMs as the first preparation drains;
+//     prep [c_split, NC), launched once every carry CTA holds its SM and sized
+//         for the SMs the carry leaves; its last step waits for the carry grid;
+//     carry [c_split, NC) from the first carry's end states.
+// A grid waits only for the completion of the grid before it (griddepcontrol),
+// never on another's progress.  c_split minimises a cost model fitted to B200
+// measurements: a persistent preparation grid takes about P0 + P1 * (records
+// per CTA) us, a carry about C0 + C1 * (chunks) us; the plan is taken only where
+// the model expects at least 3% over the serial sweep.
+struct PipePlan {
+  int c_split = 0;   // 0: serial
+  int prep_sms = 0;  // SMs the second preparation grid is sized for
+};
+PipePlan pipe_plan(int variant, int B, int H, int NC) {
+  PipePlan pp;
+  if (variant == kGDN2 || NC < 4) return pp;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return pp;
+  }
+  const long long bh = static_cast<long long>(B) * H;
+  if (sms - bh < 16) return pp;
+  const bool chan = variant == kKDA;
+  const double slots = chan ? 1.0 : 2.0;                       // preparation CTAs per SM
+  const double P0 = chan ? 13.0 : 9.0, P1 = chan ? 10.8 : 8.2;  // us, us per record per CTA
+  const double C0 = chan ? 2.1 : 2.4, C1 = chan ? 1.85 : 1.69;  // us, us per chunk
+  auto prep = [&](double records, double ctas) { return P0 + P1 * records / ctas; };
+  const double serial = prep(double(NC) * bh, slots * sms) + C0 + C1 * NC;
+  double best = serial;
+  for (int cs = 1; cs < NC; ++cs) {
+    const double t = prep(double(cs) * bh, slots * sms) +
+                     std::max(C0 + C1 * cs, prep(double(NC - cs) * bh, slots * (sms - bh))) + C0 + C1 * (NC - cs) + 2.0;
+    if (t < best) {
+      best = t;
+      pp.c_split = cs;
+    }
+  }
+  if (best > 0.97 * serial) pp.c_split = 0;
+  pp.prep_sms = static_cast<int>(sms - bh);
+  return pp;
+}
+
+template <int VAR>
+cudaError_t launch_prep_any(const FwdProblem &p, int NC, uint8_t *w, const PrepRange &rg, cudaStream_t stream,
+                            std::string *err) {
+  if constexpr (VAR == kKDA) return launch_prep_chan(p, NC, w, rg, stream, err);
+  else if constexpr (VAR == kGDN2) return launch_prep_gdn2(p, NC, w, stream, err);
+  else return launch_prep<VAR>(p, NC, w, rg, stream, err);
+}
+
+template <int VAR>
+cudaError_t launch_pipelined(const FwdProblem &p, int NC, uint8_t *w, const PipePlan &pp, cudaStream_t stream,
+                             std::string *err) {
+  constexpr int MODE = VAR == kKDA ? 1 : 0;
+  static_assert(VAR != kGDN2, "GDN-2 preparation is not persistent");
+  const int cs = pp.c_split, ns = p.dv / 64;
+  const size_t rb = MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
+  // The first carry's end states go to each sequence's chunk-0 record, which
+  // that carry CTA has consumed by then and the second preparation never writes.
+  float *mid = reinterpret_cast<float *>(w);
+  const size_t mid_bh = static_cast<size_t>(NC) * rb / sizeof(float);
+  PrepRange r1;
+  r1.ncr = cs;
+  cudaError_t e = launch_prep_any<VAR>(p, NC, w, r1, stream, err);
+  if (e != cudaSuccess) return e;
+  CarryLaunch l1;
+  l1.seg_len = cs;
+  l1.s0 = p.s0;
+  l1.s_final = mid;
+  l1.s_final_bh_stride = mid_bh;
+  if ((e = launch_carry<MODE>(p, NC, w, l1, true, stream, err)) != cudaSuccess) return e;
+  PrepRange r2;
+  r2.c0 = cs;
+  r2.ncr = NC - cs;
+  r2.sms = pp.prep_sms;
+  r2.after_carry = true;
+  if ((e = launch_prep_any<VAR>(p, NC, w, r2, stream, err)) != cudaSuccess) return e;
+  CarryLaunch l2;
+  l2.c_base = cs;
+  l2.seg_len = NC - cs;
+  l2.s0 = mid;
+  l2.s0_bh_stride = mid_bh;
+  l2.s_final = p.s_final;
+  return launch_carry<MODE>(p, NC, w, l2, true, stream, err);
+}
+
 template <int VAR>
 cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
   constexpr int MODE = VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0;
   const int NC = (p.T + C - 1) / C;
   uint8_t *w = static_cast<uint8_t *>(ws);
-  cudaError_t e;
-  if constexpr (VAR == kKDA) e = launch_prep_chan(p, NC, w, stream, err);
-  else if constexpr (VAR == kGDN2) e = launch_prep_gdn2(p, NC, w, stream, err);
-  else e = launch_prep<VAR>(p, NC, w, stream, err);
-  if (e != cudaSuccess) return e;
   const SegPlan sp = seg_plan(p.B, p.H, p.dv, NC);
+  if constexpr (VAR != kGDN2) {
+    if (sp.G == 1) {
+      const PipePlan pp = pipe_plan(VAR, p.B, p.H, NC);
+      if (pp.c_split > 0) return launch_pipelined<VAR>(p, NC, w, pp, stream, err);
+    }
+  }
+  cudaError_t e = launch_prep_any<VAR>(p, NC, w, PrepRange(), stream, err);
+  if (e != cudaSuccess) return e;
   if (sp.G == 1) {
     CarryLaunch l;
     l.seg_len = NC;
@@ -1802,7 +1956,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   f.flags = CARRY_LAST_FINAL;
   f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
   f.s_final = p.s_final;
-  return launch_carry<MODE>(p, NC, w, f, false, stream, err);   // reads the chain kernel's states
+  return launch_carry<MODE>(p, NC, w, f, true, stream, err);
 }
 
 }  // namespace
@@ -1827,9 +1981,10 @@ size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   return (records + 255) / 256 * 256 + 4 * gdr::tc::seg_extra_floats(B, H, dv, sp);
 }
 
-int gdr_split_launches(int B, int T, int H, int dv) {
+int gdr_split_launches(int variant, int B, int T, int H, int dv) {
   const int NC = (T + 63) / 64;
-  return gdr::tc::seg_plan(B, H, dv, NC).G == 1 ? 2 : 4;
+  if (gdr::tc::seg_plan(B, H, dv, NC).G > 1) return 4;
+  return gdr::tc::pipe_plan(variant, B, H, NC).c_split > 0 ? 4 : 2;
 }
 
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {

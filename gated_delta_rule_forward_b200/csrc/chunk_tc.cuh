@@ -19,7 +19,7 @@ int gdr_read_chan_error();
 // Two-kernel path (chunk_split.cu): chunk-parallel preparation + sequential carry.
 bool gdr_split_supported(int variant, int dk, int dv);
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv);
-int gdr_split_launches(int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
+int gdr_split_launches(int variant, int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err);
 int gdr_read_split_error();
 // Fixed scratch of the no-allocation entry point (chunk_split.cu).

@@ -9,6 +9,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from gated_delta_rule_forward_b200 import _lib
 
@@ -152,7 +153,9 @@ def test_workspace_sizes(L):
     assert L.gdr_forward_workspace_size(3, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 512 + 49152)
     assert L.gdr_forward_kernel_name(3, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
     assert L.gdr_forward_kernel_name(1, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
-    assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == 2
+    # preparation + carry; with a device whose idle SMs pay for it, the pipelined
+    # sweep (two of each) -- without one, as here, the serial pair
+    assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == (4 if torch.cuda.is_available() else 2)
     assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
     assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 64).decode() == "chunk64_tc"
 

@@ -157,6 +157,34 @@ def test_segmented_carry(variant):
     assert_close(S, S_ref, torch.bfloat16, "S")
 
 
+@pytest.mark.parametrize("variant", ["gdn", "deltanet", "kla", "kda"])
+def test_pipelined_sweep(variant):
+    """B*H = 64 sequences leave most SMs idle beside the carry, so the two-kernel
+    path cuts the sweep in two: the second part's preparation runs beside the
+    first part's carry, and the second carry starts from the first one's states
+    (kept in the workspace).  24 chunks, the last one ragged; with an initial state."""
+    B, T, H = 4, 1531, 16
+    launches = gdr.forward_launches(variant, torch.bfloat16, B, T, H, 128, 128, 0)
+    assert launches == 4, f"expected the pipelined sweep (4 launches), got {launches}"
+    o, S, o_ref, S_ref = run_both(variant, B, T, H, 128, 128, torch.bfloat16, 0, seed=23)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
+def test_pipelined_sweep_no_states():
+    """The pipelined sweep with neither an initial nor a final state: the middle
+    states live in the workspace, so the output is unchanged."""
+    B, T, H = 4, 1531, 16
+    assert gdr.forward_launches("gdn", torch.bfloat16, B, T, H, 128, 128, 0) == 4
+    d = make_inputs("gdn", B, T, H, 128, 128, dtype=torch.bfloat16, seed=24)
+    dd = to_dev(d)
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant="gdn", **gate_kwargs(dd), output_final_state=False)
+    torch.cuda.synchronize()
+    assert S is None
+    o_ref, _ = oracle.forward("gdn", **d)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+
+
 def test_segmented_carry_no_initial_state():
     """Segmented carry from a zero state, B=2 H=3 T=4480 (70 chunks, 12 segments
     of 6): segment 0 then starts from zeros like every other segment's offset."""
