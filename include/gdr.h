@@ -126,9 +126,14 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
  *      dk = 128;
  *   65 the two-kernel chunked path: a chunk-parallel preparation kernel (the
  *      S-independent products of every chunk, into the workspace) then the
- *      sequential carry kernel (for few long sequences: segment maps, a chain
- *      of segment start states, then the segments in parallel): all five
- *      variants with bf16 I/O and dk = 128; needs the workspace.
+ *      sequential carry kernel: all five variants with bf16 I/O and dk = 128;
+ *      needs the workspace.  Where the carry's B * H CTAs leave SMs idle it
+ *      reschedules: for few long sequences, segment maps, a chain of segment
+ *      start states, then the segments in parallel; for a mid-size B * H
+ *      (DeltaNet, Gated DeltaNet, KLA, KDA), the sweep cut in two, with the
+ *      second part's preparation beside the first part's carry.  Its kernels
+ *      are chained on `stream` by programmatic dependent launch; the call
+ *      returns after enqueueing them, like every other path.
  * A chunk value whose path does not cover the case returns GDR_ERR_UNSUPPORTED.
  * Shapes: B, T, H >= 0; dk in {64, 128}; dv in {64, 128}.  T = 0 copies
  * initial_state to final_state (or clears it); B * H = 0 does nothing.
@@ -185,7 +190,10 @@ gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int d
 /*
  * Kernel launches one gdr_forward_chunked call with these arguments makes
  * (0 if the call would be rejected), and a short name of the kernel that runs
- * ("chunk64_tc", "token_f32io", "token_bf16io", ...).  Host-only, no GPU work.
+ * ("chunk64_split", "chunk64_tc", "token_f32io", "token_bf16io", ...).
+ * Host-only, no GPU work.  The two-kernel path makes 2 launches, or 4 when
+ * it reschedules (segmented or pipelined sweep); that choice reads the
+ * current device's SM count, and with no device present it is always 2.
  */
 int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk);
 const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv,
