@@ -107,6 +107,7 @@ struct PrepParams {
   int B, T, H, dv, NC;
   int c0, ncr;   // the launch prepares chunks [c0, c0 + ncr) of every (b, h)
   const float *beta, *log_g;
+  const float *erase_b, *write_w;   // GDN-2 only
   uint8_t *ws;
   float eps, scale;
 };
@@ -821,349 +822,410 @@ constexpr uint32_t COL_OD = 384;  // M128 x 64: (P^d V)^T
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace prepg
 
-struct PrepG2Params {
-  int T, H, dv, NC;
-  const float *erase_b, *write_w;
-  uint8_t *ws;
-  float scale;
-};
-
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_prep_gdn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                           const PrepG2Params p) {
+                           const PrepParams p) {
   using namespace prepg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int NS = p.dv / 64;
-  const int t0 = c * C;
+  const int total = p.ncr * p.H * p.B;   // records of this launch, chunk index fastest
 
-  uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_lg = bar_in + 1;
-  uint64_t *bar_mma = bar_in + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
+  uint64_t *bar_kq = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // K, Q landed
+  uint64_t *bar_lg = bar_kq + 1;                                      // log g landed
+  uint64_t *bar_mma = bar_kq + 2;
+  uint64_t *bar_v = bar_kq + 3;                                       // V landed
+  uint64_t *bar_drain = bar_kq + 4;                                   // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_kq + 5);
   float *sc_em = reinterpret_cast<float *>(sm + OFF_SC);     // [128] e^{gamma_m} per channel
   float *sc_tmp = sc_em + 128;                               // [128]
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
-  uint8_t *rec = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c) * rec_bytes_gdn2(NS);
-  uint8_t *rec_od = rec + rec_bytes_chan(NS);          // (P^d V)^T, rows v x 64 t fp16
-  uint8_t *rec_sd = rec_od + 8192 * NS;                // (Dt^T V)^T, rows v x 128 i fp16
   uint8_t *kq_ptr = sm + OFF_KQ;
+
+  // loads of record r (thread 0): log g and K, Q first, V once the last product no longer reads it
+  uint32_t issued = 0, landed = 0;   // thread 0: loads issued / seen landing (lg | kq << 8 | v << 16)
+  auto issue_kq_lg = [&](int r) {
+    const RecIdx x = rec_idx(p, r);
+    mbar_expect_tx(bar_lg, 64 * DK * 4);
+    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, x.h, x.c * C, x.b);
+    mbar_expect_tx(bar_kq, 4 * 8192);
+    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_kq, 0, x.h, x.c * C, x.b);
+    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_kq, 0, x.h, x.c * C, x.b);
+    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_kq, 64, x.h, x.c * C, x.b);
+    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_kq, 64, x.h, x.c * C, x.b);
+    issued += 1u | (1u << 8);
+  };
+  auto issue_v = [&](int r) {
+    const RecIdx x = rec_idx(p, r);
+    mbar_expect_tx(bar_v, NS * 8192);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_v, 64 * sl, x.h, x.c * C, x.b);
+    issued += 1u << 16;
+  };
+  // erase / write gates of the (t, 4-channel) units this thread builds in pass hp
+  // of record r, loaded one pass ahead so that no pass waits for global memory
+  float4 ebs[2][4], wrs[2][4];
+  auto load_gates = [&](int r, int hp) {
+    const RecIdx x = rec_idx(p, r);
+    const int t0 = x.c * C;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int t = (it * NTHREADS + tid) >> 4, ch0 = 64 * hp + 4 * (tid & 15);
+      ebs[hp][it] = wrs[hp][it] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t0 + t < p.T) {
+        const size_t gi = ((static_cast<size_t>(x.b) * p.T + t0 + t) * p.H + x.h) * DK + ch0;
+        ebs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
+        wrs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
+      }
+    }
+  };
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar_in, 1);
+    mbar_init(bar_kq, 1);
     mbar_init(bar_lg, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
-    mbar_expect_tx(bar_lg, 64 * DK * 4);
-    tma_load_4d(sm + OFF_LG, &tm_g, bar_lg, 0, h, t0, b);
-    mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
-    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
-    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_g);
+    if (static_cast<int>(blockIdx.x) < total) {
+      issue_kq_lg(blockIdx.x);
+      issue_v(blockIdx.x);
+    }
   }
   if (NS == 1) {   // d_v = 64: the transposed products read a 128-row V operand
     for (int i = tid; i < 512; i += NTHREADS)
       reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
-  // erase / write gates of the (t, 4-channel) units this thread builds in pass hp,
-  // loaded one pass ahead so that no pass waits for global memory
-  float4 ebs[2][4], wrs[2][4];
-  auto load_gates = [&](int hp) {
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int t = (it * NTHREADS + tid) >> 4, ch0 = 64 * hp + 4 * (tid & 15);
-      ebs[hp][it] = wrs[hp][it] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t0 + t < p.T) {
-        const size_t gi = ((static_cast<size_t>(b) * p.T + t0 + t) * p.H + h) * DK + ch0;
-        ebs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
-        wrs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
-      }
-    }
-  };
-  load_gates(0);
+  griddep_launch_dependents();   // persistent grid: the carry may launch now (see chunk_prep_kernel)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   int bad = 0, range = 0;
   uint32_t mma_phase = 0;
+  float wmax_all = 0.f;
 
-  // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
-  if (!mbar_wait(bar_lg, 0)) bad = 1;
-  bad = __syncthreads_or(bad);
-  if (!bad) {
-    const int ch = tid & 127, hh = tid >> 7;
-    float run = 0.f;
+  // Persistent over records (one CTA per SM): the next record's log g, K and Q
+  // are loaded once MMA1 has consumed this record's, its V once the last
+  // product has.
+  for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    const uint32_t ph = ((r - blockIdx.x) / gridDim.x) & 1;   // phase of the input barriers
+    uint8_t *rec = p.ws + rec_index(p, rec_idx(p, r)) * rec_bytes_gdn2(NS);
+    uint8_t *rec_od = rec + rec_bytes_chan(NS);          // (P^d V)^T, rows v x 64 t fp16
+    uint8_t *rec_sd = rec_od + 8192 * NS;                // (Dt^T V)^T, rows v x 128 i fp16
+    load_gates(r, 0);
+
+    // (a) per-channel cumulative log2 decay in place, then G = 2^(gamma - gamma_m), m = token 31
+    if (!mbar_wait(bar_lg, ph)) bad = 1;
+    else if (tid == 0) landed += 1u;
+    bad = __syncthreads_or(bad);
+    if (!bad) {
+      const int ch = tid & 127, hh = tid >> 7;
+      float run = 0.f;
 #pragma unroll 8
-    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-      run += Gr[t * DK + ch] * LOG2E;
-      Gr[t * DK + ch] = run;
+      for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+        run += Gr[t * DK + ch] * LOG2E;
+        Gr[t * DK + ch] = run;
+      }
+      if (hh == 0) sc_tmp[ch] = run;
+      __syncthreads();
+      const float gm = sc_tmp[ch];
+      if (hh == 0) sc_em[ch] = ex2(gm);
+#pragma unroll 8
+      for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
+        float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
+        if (d > SPAN_SAFE || d < -SPAN_SAFE) {
+          range = 1;
+          d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
+        }
+        Gr[t * DK + ch] = ex2(d);
+      }
     }
-    if (hh == 0) sc_tmp[ch] = run;
     __syncthreads();
-    const float gm = sc_tmp[ch];
-    if (hh == 0) sc_em[ch] = ex2(gm);
-#pragma unroll 8
-    for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-      float d = Gr[t * DK + ch] + (hh ? gm : 0.f) - gm;
-      if (d > SPAN_SAFE || d < -SPAN_SAFE) {
-        range = 1;
-        d = fminf(fmaxf(d, -SPAN_SAFE), SPAN_SAFE);
+    if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
+
+    // (b) K and Q landed?
+    if (!mbar_wait(bar_kq, ph)) bad = 1;
+    else if (tid == 0) landed += 1u << 8;
+    bad = __syncthreads_or(bad);
+    float qkmax = 0.f;
+
+    // (c) MMA1 in two 64-channel halves; the record's At and Qg; K o e^gamma and Dt for MMA2
+#pragma unroll
+    for (int hp = 0; hp < 2; ++hp) {
+      if (bad) break;
+      if (hp == 0) load_gates(r, 1);
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
+        const int t = u >> 4, j4 = u & 15;
+        const int ch0 = 64 * hp + 4 * j4;
+        const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);
+        float kx[4], qx[4];
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
+        unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        const float4 eb = ebs[hp][it], wr = wrs[hp][it];
+        const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
+        const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
+        const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
+        const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
+        const float em[4] = {m4.x, m4.y, m4.z, m4.w};
+        const float ebv[4] = {eb.x, eb.y, eb.z, eb.w}, wrv[4] = {wr.x, wr.y, wr.z, wr.w};
+        float kg[4], qg[4], af[4], df[4], at[4], dt[4], qo[4], ke[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float inv = rcp_approx(g[e]);
+          const float a = ebv[e] * kx[e], d = (wrv[e] - ebv[e]) * kx[e];
+          kg[e] = tf32r(kx[e] * g[e]);
+          qg[e] = tf32r(p.scale * qx[e] * g[e]);
+          af[e] = tf32r(a * inv);
+          df[e] = tf32r(d * inv);
+          at[e] = a * (g63[e] * inv);
+          dt[e] = d * (g63[e] * inv);
+          qo[e] = p.scale * qx[e] * g[e] * em[e];
+          ke[e] = kx[e] * g[e] * em[e];
+          qkmax = fmaxf(qkmax, fmaxf(fabsf(at[e]), fabsf(qo[e])));
+        }
+        const uint32_t xa = (j4 >> 3) * 16384;
+        const uint32_t sw = sw128(t, j4 & 7), sw64 = sw128(64 + t, j4 & 7);
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw64) = make_float4(qg[0], qg[1], qg[2], qg[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw) = make_float4(af[0], af[1], af[2], af[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw64) = make_float4(df[0], df[1], df[2], df[3]);
+        *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
+            make_uint2(pack_f16x2(at[0], at[1]), pack_f16x2(at[2], at[3]));
+        *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
+            make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
+        *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
+            make_uint2(pack_f16x2(ke[0], ke[1]), pack_f16x2(ke[2], ke[3]));
+        *reinterpret_cast<uint2 *>(sm + OFF_DT + hp * 8192 + bf) =
+            make_uint2(pack_f16x2(dt[0], dt[1]), pack_f16x2(dt[2], dt[3]));
       }
-      Gr[t * DK + ch] = ex2(d);
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   sdesc(yf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 128, false, false),
+                   hp + kk > 0);
+        mma_commit(bar_mma);
+      }
+      if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+      bad = __syncthreads_or(bad);
+      mma_phase ^= 1;
+      tc_fence_after();
     }
-  }
-  __syncthreads();
-  if (!bad && tid < DK) reinterpret_cast<float *>(rec + rec_sc(NS))[tid] = Gr[63 * DK + tid] * sc_em[tid];
 
-  // (b) inputs landed?
-  if (!mbar_wait(bar_in, 0)) bad = 1;
-  bad = __syncthreads_or(bad);
-  float qkmax = 0.f;
+    // log g, K and Q are consumed: the next record's are loaded from here on
+    if (!bad && tid == 0 && r + static_cast<int>(gridDim.x) < total) issue_kq_lg(r + gridDim.x);
 
-  // (c) MMA1 in two 64-channel halves; the record's At and Qg; K o e^gamma and Dt for MMA2
+    // (d) rows t of K (lanes 0-63): A -> A^T scratch, I - A^d -> fp16 rows; rows t of Q
+    // (lanes 64-127): P^a -> fp16 record tile, P^d -> fp16 tile.  Column half `half`
+    // selects the a or the d block.
+    if (!bad) {
+      float g[64];
+      tmem_ld64(tmem + lane_base + COL_G + 64 * half, g);
+      const int t = row & 63;
+      if (quad < 2) {
+        if (half == 0) {
 #pragma unroll
-  for (int hp = 0; hp < 2; ++hp) {
-    if (bad) break;
-    if (hp == 0) load_gates(1);
+          for (int r2 = 0; r2 < 64; ++r2) At[r2 * LD + t] = (r2 < t) ? tf32r(g[r2]) : 0.f;
+        } else {
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int u = it * NTHREADS + tid;      // 1024 units: (t, 4-channel group j4)
-      const int t = u >> 4, j4 = u & 15;
-      const int ch0 = 64 * hp + 4 * j4;
-      const uint32_t bf = sw128(t, j4 >> 1) + 8 * (j4 & 1);
-      float kx[4], qx[4];
-      unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
-      unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
-      const float4 eb = ebs[hp][it], wr = wrs[hp][it];
-      const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
-      const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
-      const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
-      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, g63[4] = {h4.x, h4.y, h4.z, h4.w};
-      const float em[4] = {m4.x, m4.y, m4.z, m4.w};
-      const float ebv[4] = {eb.x, eb.y, eb.z, eb.w}, wrv[4] = {wr.x, wr.y, wr.z, wr.w};
-      float kg[4], qg[4], af[4], df[4], at[4], dt[4], qo[4], ke[4];
+          for (int r2 = 0; r2 < 64; ++r2) g[r2] = (r2 < t) ? -g[r2] : (r2 == t ? 1.f : 0.f);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float inv = rcp_approx(g[e]);
-        const float a = ebv[e] * kx[e], d = (wrv[e] - ebv[e]) * kx[e];
-        kg[e] = tf32r(kx[e] * g[e]);
-        qg[e] = tf32r(p.scale * qx[e] * g[e]);
-        af[e] = tf32r(a * inv);
-        df[e] = tf32r(d * inv);
-        at[e] = a * (g63[e] * inv);
-        dt[e] = d * (g63[e] * inv);
-        qo[e] = p.scale * qx[e] * g[e] * em[e];
-        ke[e] = kx[e] * g[e] * em[e];
-        qkmax = fmaxf(qkmax, fmaxf(fabsf(at[e]), fabsf(qo[e])));
+          for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_IAD + sw128(t, j), g + 8 * j);
+        }
+      } else {
+#pragma unroll
+        for (int r2 = 0; r2 < 64; ++r2) g[r2] = (r2 <= t) ? g[r2] : 0.f;
+        if (half == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) st_chunk_f16(rec + REC_P + sw128(t, j), g + 8 * j);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_PD + sw128(t, j), g + 8 * j);
+        }
       }
-      const uint32_t xa = (j4 >> 3) * 16384;
-      const uint32_t sw = sw128(t, j4 & 7), sw64 = sw128(64 + t, j4 & 7);
-      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw) = make_float4(kg[0], kg[1], kg[2], kg[3]);
-      *reinterpret_cast<float4 *>(sm + OFF_XF + xa + sw64) = make_float4(qg[0], qg[1], qg[2], qg[3]);
-      *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw) = make_float4(af[0], af[1], af[2], af[3]);
-      *reinterpret_cast<float4 *>(sm + OFF_YF + xa + sw64) = make_float4(df[0], df[1], df[2], df[3]);
-      *reinterpret_cast<uint2 *>(rec + REC_K + hp * 8192 + bf) =
-          make_uint2(pack_f16x2(at[0], at[1]), pack_f16x2(at[2], at[3]));
-      *reinterpret_cast<uint2 *>(rec + REC_WQ + hp * 16384 + 8192 + bf) =
-          make_uint2(pack_f16x2(qo[0], qo[1]), pack_f16x2(qo[2], qo[3]));
-      *reinterpret_cast<uint2 *>(sm + OFF_KG + hp * 8192 + bf) =
-          make_uint2(pack_f16x2(ke[0], ke[1]), pack_f16x2(ke[2], ke[3]));
-      *reinterpret_cast<uint2 *>(sm + OFF_DT + hp * 8192 + bf) =
-          make_uint2(pack_f16x2(dt[0], dt[1]), pack_f16x2(dt[2], dt[3]));
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // (e) T = (I + A)^{-1} as fp16 rows; then R = T (I - A^d).  The V tile turns
+    // fp16 in place (exact from bf16) so that every product of this kernel after
+    // MMA1 has fp16 operands: the GDN-2 terms pass more roundings into the state
+    // than the other variants' and bf16 there leaves ~2% of the state RMS.
+    solve_unit_lower_64(At, Tf, tid, warp, lane);
+    float tmax = 0.f;
+    {
+      const int m = tid >> 2, n0 = (tid & 3) * 16;
+      float tv[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+        tmax = fmaxf(tmax, fabsf(tv[e]));
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) st_chunk_f16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0) {
+    if (!bad && tid == 0) {
       tc_fence_after();
-      const uint32_t xf = smem_u32(sm + OFF_XF), yf = smem_u32(sm + OFF_YF);
+      const uint32_t tt = smem_u32(sm + OFF_T), iad = smem_u32(sm + OFF_IAD);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_tf32(tmem + COL_G, sdesc(xf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(yf + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_tf32(128, 128, false, false),
-                 hp + kk > 0);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem + COL_R, sdesc(tt + kk * 32, 16, 1024), sdesc(iad + kk * 2048, 8192, 1024),
+               idesc_f16(64, 64, false, true), kk > 0);
       mma_commit(bar_mma);
     }
-    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+    // V landed? then to fp16 in place (the R product does not read it)
+    if (!bad && !mbar_wait(bar_v, ph)) bad = 1;
+    else if (!bad && tid == 0) landed += 1u << 16;
+    bad = __syncthreads_or(bad);
+    if (!bad) {
+      for (int i = tid; i < NS * 512; i += NTHREADS) {
+        uint4 *chunk = reinterpret_cast<uint4 *>(sm + OFF_V) + i;
+        float x[8];
+        unpack8(*chunk, x);
+        st_chunk_f16(reinterpret_cast<uint8_t *>(chunk), x);
+      }
+    }
+    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
-  }
-
-  // (d) rows t of K (lanes 0-63): A -> A^T scratch, I - A^d -> bf16 rows; rows t of Q
-  // (lanes 64-127): P^a -> fp16 record tile, P^d -> bf16 tile.  Column half `half`
-  // selects the a or the d block.
-  if (!bad) {
-    float g[64];
-    tmem_ld64(tmem + lane_base + COL_G + 64 * half, g);
-    const int t = row & 63;
-    if (quad < 2) {
-      if (half == 0) {
-#pragma unroll
-        for (int r = 0; r < 64; ++r) At[r * LD + t] = (r < t) ? tf32r(g[r]) : 0.f;
-      } else {
-#pragma unroll
-        for (int r = 0; r < 64; ++r) g[r] = (r < t) ? -g[r] : (r == t ? 1.f : 0.f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_IAD + sw128(t, j), g + 8 * j);
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 64; ++r) g[r] = (r <= t) ? g[r] : 0.f;
-      if (half == 0) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st_chunk_f16(rec + REC_P + sw128(t, j), g + 8 * j);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st_chunk_f16(sm + OFF_PD + sw128(t, j), g + 8 * j);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // (e) T = (I + A)^{-1} as fp16 rows; then R = T (I - A^d).  The V tile turns
-  // fp16 in place (exact from bf16) so that every product of this kernel after
-  // MMA1 has fp16 operands: the GDN-2 terms pass more roundings into the state
-  // than the other variants' and bf16 there leaves ~2% of the state RMS.
-  solve_unit_lower_64(At, Tf, tid, warp, lane);
-  float tmax = 0.f;
-  for (int i = tid; i < NS * 512; i += NTHREADS) {
-    uint4 *chunk = reinterpret_cast<uint4 *>(sm + OFF_V) + i;
-    float x[8];
-    unpack8(*chunk, x);
-    st_chunk_f16(reinterpret_cast<uint8_t *>(chunk), x);
-  }
-  {
-    const int m = tid >> 2, n0 = (tid & 3) * 16;
-    float tv[16];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
-      tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
-    }
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
-      tmax = fmaxf(tmax, fabsf(tv[e]));
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) st_chunk_f16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
-  }
-  fence_async_smem();
-  __syncthreads();
-  if (!bad && tid == 0) {
-    tc_fence_after();
-    const uint32_t tt = smem_u32(sm + OFF_T), iad = smem_u32(sm + OFF_IAD);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_ss(tmem + COL_R, sdesc(tt + kk * 32, 16, 1024), sdesc(iad + kk * 2048, 8192, 1024),
-               idesc_f16(64, 64, false, true), kk > 0);
-    mma_commit(bar_mma);
-  }
-  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
-  bad = __syncthreads_or(bad);
-  mma_phase ^= 1;
-  tc_fence_after();
-  if (!bad) {   // R (M64 layout: rows 16 quad + lane, lane < 16) -> fp16 rows t
-    float w[32];
-    tmem_ld32(tmem + lane_base + COL_R + 32 * half, w);
-    if (lane < 16) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, fabsf(w[e]));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_RT + sw128(quad * 16 + lane, 4 * half + j), w + 8 * j);
-    }
-  }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // (f) W = T (K o e^gamma); U'^T = V^T R^T; (P^d V)^T = V^T P^d^T; (Dt^T V)^T = V^T Dt
-  if (!bad && tid == 0) {
-    tc_fence_after();
-    const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
-    const uint32_t rt = smem_u32(sm + OFF_RT), pd = smem_u32(sm + OFF_PD), dtt = smem_u32(sm + OFF_DT);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint64_t va = sdesc(vt + kk * 2048, 8192, 1024);
-      mma_ss(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
-               idesc_f16(64, 128, false, true), kk > 0);
-      mma_ss(tmem + COL_U, va, sdesc(rt + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
-      mma_ss(tmem + COL_OD, va, sdesc(pd + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
-      mma_ss(tmem + COL_SD, va, sdesc(dtt + kk * 2048, 8192, 1024), idesc_f16(128, 128, true, true), kk > 0);
-    }
-    mma_commit(bar_mma);
-  }
-  if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
-  bad = __syncthreads_or(bad);
-  tc_fence_after();
-
-  // (g) -W (M64 layout), U'^T, (P^d V)^T and (Dt^T V)^T -> fp16 record tiles
-  float wmax = fmaxf(qkmax, tmax);
-  if (!bad) {
-    float w[32];
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+    if (!bad) {   // R (M64 layout: rows 16 quad + lane, lane < 16) -> fp16 rows t
+      float w[32];
+      tmem_ld32(tmem + lane_base + COL_R + 32 * half, w);
       if (lane < 16) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          wmax = fmaxf(wmax, fabsf(w[e]));
-          w[e] = -w[e];
-        }
+        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, fabsf(w[e]));
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        for (int j = 0; j < 4; ++j) st_chunk_f16(sm + OFF_RT + sw128(quad * 16 + lane, 4 * half + j), w + 8 * j);
       }
     }
-    tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
-    if (row < p.dv) {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // (f) W = T (K o e^gamma); U'^T = V^T R^T; (P^d V)^T = V^T P^d^T; (Dt^T V)^T = V^T Dt
+    if (!bad && tid == 0) {
+      tc_fence_after();
+      const uint32_t tt = smem_u32(sm + OFF_T), kg = smem_u32(sm + OFF_KG), vt = smem_u32(sm + OFF_V);
+      const uint32_t rt = smem_u32(sm + OFF_RT), pd = smem_u32(sm + OFF_PD), dtt = smem_u32(sm + OFF_DT);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t va = sdesc(vt + kk * 2048, 8192, 1024);
+        mma_ss(tmem + COL_W, sdesc(tt + kk * 32, 16, 1024), sdesc(kg + kk * 2048, 8192, 1024),
+               idesc_f16(64, 128, false, true), kk > 0);
+        mma_ss(tmem + COL_U, va, sdesc(rt + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+        mma_ss(tmem + COL_OD, va, sdesc(pd + kk * 32, 16, 1024), idesc_f16(128, 64, true, false), kk > 0);
+        mma_ss(tmem + COL_SD, va, sdesc(dtt + kk * 2048, 8192, 1024), idesc_f16(128, 128, true, true), kk > 0);
+      }
+      mma_commit(bar_mma);
     }
-    tmem_ld32(tmem + lane_base + COL_OD + 32 * half, w);
-    if (row < p.dv) {
+    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    mma_phase ^= 1;
+    tc_fence_after();
+    // V is consumed: the next record's is loaded during the epilogue
+    if (!bad && tid == 0 && r + static_cast<int>(gridDim.x) < total) issue_v(r + gridDim.x);
+
+    // (g) -W (M64 layout), U'^T, (P^d V)^T and (Dt^T V)^T -> fp16 record tiles
+    float wmax = fmaxf(qkmax, tmax);
+    if (!bad) {
+      float w[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
+        if (lane < 16) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f16(rec_od + row * 128 + half * 64 + 16 * j, w + 8 * j);
-    }
+          for (int e = 0; e < 32; ++e) {
+            wmax = fmaxf(wmax, fabsf(w[e]));
+            w[e] = -w[e];
+          }
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      tmem_ld32(tmem + lane_base + COL_SD + 64 * half + 32 * part, w);
+          for (int j = 0; j < 4; ++j)
+            st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
+        }
+      }
+      tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
       if (row < p.dv) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_chunk_f16(rec_sd + row * 256 + half * 128 + part * 64 + 16 * j, w + 8 * j);
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
+      }
+      tmem_ld32(tmem + lane_base + COL_OD + 32 * half, w);
+      if (row < p.dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_chunk_f16(rec_od + row * 128 + half * 64 + 16 * j, w + 8 * j);
+      }
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem + lane_base + COL_SD + 64 * half + 32 * part, w);
+        if (row < p.dv) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) wmax = fmaxf(wmax, fabsf(w[e]));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_chunk_f16(rec_sd + row * 256 + half * 128 + part * 64 + 16 * j, w + 8 * j);
+        }
       }
     }
+    wmax_all = fmaxf(wmax_all, wmax);
+    // tensor-memory reads done before the next record's MMA1
+    tc_fence_before();
+    __syncthreads();
+    if (bad) break;
   }
-  if (bad && tid == 0) atomicOr(&g_gdr_split_error, 1);
-  if (range || wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
+
+  if (bad && tid == 0) {
+    // a wait gave up: report it, then let the MMAs and loads in flight finish
+    // (each wait again bounded) before tensor memory is released
+    atomicOr(&g_gdr_split_error, 1);
+    mma_commit(bar_drain);
+    mbar_wait(bar_drain, 0);
+    uint64_t *bars[3] = {bar_lg, bar_kq, bar_v};
+    for (int i = 0; i < 3; ++i) {
+      const uint32_t n_issued = (issued >> (8 * i)) & 0xffu, n_landed = (landed >> (8 * i)) & 0xffu;
+      if (n_issued != n_landed) mbar_wait(bars[i], n_landed & 1u);
+    }
+  }
+  if (range || wmax_all > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  // programmatic dependent of a carry grid (the pipelined sweep): complete
+  // only after it (see chunk_prep_chan_kernel)
+  griddep_wait();
 }
 
 // ------------------------------------------------------------------ carry kernel
@@ -1631,7 +1693,8 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
   return e;
 }
 
-cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
+                             std::string *err) {
   cudaError_t e = cudaFuncSetAttribute(chunk_prep_gdn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prepg::SMEM_BYTES);
   if (e != cudaSuccess) {
@@ -1644,11 +1707,23 @@ cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, cudaStrea
     *err = "cuTensorMapEncodeTiled failed: ";
     return cudaErrorInvalidValue;
   }
-  PrepG2Params pp;
-  pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
-  pp.erase_b = p.erase_b; pp.write_w = p.write_w; pp.ws = ws; pp.scale = p.scale;
-  chunk_prep_gdn2_kernel<<<dim3(NC, p.H, p.B), NTHREADS, prepg::SMEM_BYTES, stream>>>(mq, mk, mv, mg, pp);
-  e = cudaGetLastError();
+  PrepParams pp;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
+  pp.beta = nullptr; pp.log_g = p.log_g; pp.erase_b = p.erase_b; pp.write_w = p.write_w; pp.ws = ws;
+  pp.eps = p.eps; pp.scale = p.scale;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) {
+    *err = "device query: ";
+    return e;
+  }
+  if (rg.sms > 0) sms = std::min(sms, rg.sms);
+  const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
+  const int grid = static_cast<int>(std::min<long long>(records, sms));   // one CTA per SM, persistent
+  e = launch_maybe_pdl(chunk_prep_gdn2_kernel, dim3(grid), dim3(NTHREADS), prepg::SMEM_BYTES, stream,
+                       rg.after_carry, mq, mk, mv, mg, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
 }
@@ -1834,7 +1909,7 @@ struct PipePlan {
 };
 PipePlan pipe_plan(int variant, int B, int H, int NC) {
   PipePlan pp;
-  if (variant == kGDN2 || NC < 4) return pp;
+  if (NC < 4) return pp;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -1843,10 +1918,13 @@ PipePlan pipe_plan(int variant, int B, int H, int NC) {
   }
   const long long bh = static_cast<long long>(B) * H;
   if (sms - bh < 16) return pp;
-  const bool chan = variant == kKDA;
-  const double slots = chan ? 1.0 : 2.0;                       // preparation CTAs per SM
-  const double P0 = chan ? 13.0 : 9.0, P1 = chan ? 10.8 : 8.2;  // us, us per record per CTA
-  const double C0 = chan ? 2.1 : 2.4, C1 = chan ? 1.85 : 1.69;  // us, us per chunk
+  // per variant family: scalar decay (two preparation CTAs per SM), KDA, GDN-2 (one each)
+  const int fam = variant == kGDN2 ? 2 : variant == kKDA ? 1 : 0;
+  const double slots = fam ? 1.0 : 2.0;                       // preparation CTAs per SM
+  const double P0 = fam ? 13.0 : 9.0;                         // us
+  const double P1 = fam == 2 ? 15.0 : fam ? 10.8 : 8.2;       // us per record per CTA
+  const double C0 = fam == 2 ? 2.5 : fam ? 2.1 : 2.4;         // us
+  const double C1 = fam == 2 ? 3.1 : fam ? 1.85 : 1.69;       // us per chunk
   auto prep = [&](double records, double ctas) { return P0 + P1 * records / ctas; };
   const double serial = prep(double(NC) * bh, slots * sms) + C0 + C1 * NC;
   double best = serial;
@@ -1867,17 +1945,16 @@ template <int VAR>
 cudaError_t launch_prep_any(const FwdProblem &p, int NC, uint8_t *w, const PrepRange &rg, cudaStream_t stream,
                             std::string *err) {
   if constexpr (VAR == kKDA) return launch_prep_chan(p, NC, w, rg, stream, err);
-  else if constexpr (VAR == kGDN2) return launch_prep_gdn2(p, NC, w, stream, err);
+  else if constexpr (VAR == kGDN2) return launch_prep_gdn2(p, NC, w, rg, stream, err);
   else return launch_prep<VAR>(p, NC, w, rg, stream, err);
 }
 
 template <int VAR>
 cudaError_t launch_pipelined(const FwdProblem &p, int NC, uint8_t *w, const PipePlan &pp, cudaStream_t stream,
                              std::string *err) {
-  constexpr int MODE = VAR == kKDA ? 1 : 0;
-  static_assert(VAR != kGDN2, "GDN-2 preparation is not persistent");
+  constexpr int MODE = VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0;
   const int cs = pp.c_split, ns = p.dv / 64;
-  const size_t rb = MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
+  const size_t rb = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
   // The first carry's end states go to each sequence's chunk-0 record, which
   // that carry CTA has consumed by then and the second preparation never writes.
   float *mid = reinterpret_cast<float *>(w);
@@ -1913,11 +1990,9 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std
   const int NC = (p.T + C - 1) / C;
   uint8_t *w = static_cast<uint8_t *>(ws);
   const SegPlan sp = seg_plan(p.B, p.H, p.dv, NC);
-  if constexpr (VAR != kGDN2) {
-    if (sp.G == 1) {
-      const PipePlan pp = pipe_plan(VAR, p.B, p.H, NC);
-      if (pp.c_split > 0) return launch_pipelined<VAR>(p, NC, w, pp, stream, err);
-    }
+  if (sp.G == 1) {
+    const PipePlan pp = pipe_plan(VAR, p.B, p.H, NC);
+    if (pp.c_split > 0) return launch_pipelined<VAR>(p, NC, w, pp, stream, err);
   }
   cudaError_t e = launch_prep_any<VAR>(p, NC, w, PrepRange(), stream, err);
   if (e != cudaSuccess) return e;

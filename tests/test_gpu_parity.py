@@ -157,7 +157,7 @@ def test_segmented_carry(variant):
     assert_close(S, S_ref, torch.bfloat16, "S")
 
 
-@pytest.mark.parametrize("variant", ["gdn", "deltanet", "kla", "kda"])
+@pytest.mark.parametrize("variant", ["gdn", "deltanet", "kla", "kda", "gdn2"])
 def test_pipelined_sweep(variant):
     """B*H = 64 sequences leave most SMs idle beside the carry, so the two-kernel
     path cuts the sweep in two: the second part's preparation runs beside the
