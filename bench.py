@@ -27,6 +27,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -70,12 +71,23 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
+def _code_only(text):
+    """Source text without // and /* */ comments or blank lines: what a
+    comment-only edit leaves unchanged (string literals hold no comment
+    markers in these sources)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_hash(kernel):
+    """Hash of the code (comments stripped) of a kernel's sources: keys the
+    recorded ncu traffic, so that a figure taken on other code is not used."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES.get(kernel, []) + ["gated_delta_rule_forward_b200/csrc/common.cuh"]:
         p = os.path.join(ROOT, rel)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(_code_only(open(p, encoding="utf-8").read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -28,11 +28,15 @@
 // Its template MODE picks the decay of the state update: a scalar Gamma_C,
 // a per-channel Gamma_C, or the per-channel one plus the GDN-2 terms.
 //
-// With few long sequences (B*H CTAs leave most SMs idle) the carry is
-// segmented: each sequence is cut into G segments, the affine maps of the
-// segments (S -> M_g S + D_g, computed by one state-only launch of the carry
-// kernel) are chained by a small kernel into each segment's start state, and
-// a last launch runs all segments at once from their start states.
+// The carry's B*H CTAs leave the rest of the device idle.  With few long
+// sequences the carry is segmented: each sequence is cut into G segments, the
+// affine maps of the segments (S -> M_g S + D_g, computed by one state-only
+// launch of the carry kernel) are chained by a small kernel into each
+// segment's start state, and a last launch runs all segments at once from
+// their start states.  Otherwise, where the idle SMs pay for it, the sweep is
+// pipelined: the chunks are cut in two, and the second part's preparation
+// runs on the SMs beside the first part's carry.  Consecutive grids are
+// chained by programmatic dependent launch (griddepcontrol).
 //
 // Workspace record per (b, h, chunk).  The tiles the MMAs read are images of
 // the 128-byte-swizzled shared-memory layout, so the carry kernel bulk-copies
