@@ -171,6 +171,17 @@ def test_pipelined_sweep(variant):
     assert_close(S, S_ref, torch.bfloat16, "S")
 
 
+@pytest.mark.parametrize("variant", ["gdn", "kda", "gdn2"])
+def test_pipelined_sweep_dv64(variant):
+    """The pipelined sweep at d_v = 64: the first carry's end states (32 KB per
+    sequence) in the chunk-0 records of the smaller dv = 64 record layout."""
+    B, T, H = 4, 1531, 16
+    assert gdr.forward_launches(variant, torch.bfloat16, B, T, H, 128, 64, 0) == 4
+    o, S, o_ref, S_ref = run_both(variant, B, T, H, 128, 64, torch.bfloat16, 0, seed=25)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
 def test_pipelined_sweep_no_states():
     """The pipelined sweep with neither an initial nor a final state: the middle
     states live in the workspace, so the output is unchanged."""
