@@ -81,7 +81,8 @@ def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=No
     contiguous.  Gates fp32: beta [B,T,H] (eta for KLA); log_g [B,T,H]
     (gdn, kla) or [B,T,H,dk] (kda, gdn2); erase_b / write_w [B,T,H,dk] (gdn2).
     initial_state: fp32 [B,H,dk,dv] or None.  Returns (o, final_state or None).
-    ``chunk``: 0 auto, 1 per-token kernel, 64 chunked tensor-core kernel.
+    ``chunk``: 0 auto, 1 per-token kernel, 64 one-kernel chunked path,
+    65 two-kernel chunked path (preparation + carry; workspace allocated here).
     """
     vid = variant_id(variant)
     if q.dim() != 4:
