@@ -66,6 +66,8 @@ def _load(mutant: int = 0) -> ctypes.CDLL:
             lib.oracle_decode_step.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp,
                                                dp, dp, d, d, i]
             lib.oracle_decode_step.restype = i
+            lib.oracle_backward.argtypes = [i, i, i, i, i, i] + [dp] * 18 + [d, d, i]
+            lib.oracle_backward.restype = i
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = i
             _libs[mutant] = lib
@@ -158,3 +160,41 @@ def decode_step(variant, q, k, v, state, beta=None, log_g=None, erase_b=None,
     if rc != 0:
         raise ValueError("oracle_decode_step rejected its arguments")
     return o, S
+
+
+def backward(variant, q, k, v, d_o, beta=None, log_g=None, erase_b=None, write_w=None,
+             initial_state=None, d_final=None, eps=1e-6, scale=1.0, threads=0, mutant=0):
+    """Gradients of <d_o, o> + <d_final, S_T> with respect to every input of
+    ``forward`` (reverse mode through the same fp64 recurrence).  Returns a dict
+    with keys q, k, v, beta, log_g, erase_b, write_w, initial_state (None for
+    inputs the variant does not take; ``beta`` is d/d eta for KLA)."""
+    q, k, v, d_o = _f64(q), _f64(k), _f64(v), _f64(d_o)
+    beta, log_g, erase_b, write_w = _f64(beta), _f64(log_g), _f64(erase_b), _f64(write_w)
+    initial_state, d_final = _f64(initial_state), _f64(d_final)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != (B, T, H, dk) or v.shape != (B, T, H, dv) or d_o.shape != (B, T, H, dv):
+        raise ValueError("q, k, v, d_o must be [B,T,H,dk], [B,T,H,dk], [B,T,H,dv], [B,T,H,dv]")
+    _check_gates(variant, beta, log_g, erase_b, write_w, (B, T, H), dk)
+    for name, st in (("initial_state", initial_state), ("d_final", d_final)):
+        if st is not None and st.shape != (B, H, dk, dv):
+            raise ValueError(f"{name} must be [B,H,dk,dv]")
+    if variant == "deltanet":
+        log_g = None
+    if variant == "gdn2":
+        beta = None
+    g = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v),
+         "beta": None if beta is None else np.zeros_like(beta),
+         "log_g": None if log_g is None else np.zeros_like(log_g),
+         "erase_b": None if variant != "gdn2" else np.zeros_like(erase_b),
+         "write_w": None if variant != "gdn2" else np.zeros_like(write_w),
+         "initial_state": np.zeros((B, H, dk, dv), np.float64)}
+    rc = _load(mutant).oracle_backward(
+        VARIANTS[variant], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_g),
+        _ptr(erase_b), _ptr(write_w), _ptr(initial_state), _ptr(d_o), _ptr(d_final),
+        _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["beta"]), _ptr(g["log_g"]),
+        _ptr(g["erase_b"]), _ptr(g["write_w"]), _ptr(g["initial_state"]),
+        float(eps), float(scale), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_backward rejected its arguments")
+    return g

@@ -48,9 +48,13 @@
  *   erase_b, write_w  [B, T, H, dk]   (GDN-2 only)
  *   state  [B, H, dk, dv]
  *
+ * oracle_backward gives the gradients of the same recurrence with respect to
+ * every input (reverse mode, the forward's steps taken backwards); it is pinned
+ * by finite differences of oracle_forward.
+ *
  * Mutants: building with -DORACLE_MUTANT=n plants one plausible mistake so
- * that the CPU tests can show that their pins catch it.  The default build
- * (no define) is the oracle.
+ * that the CPU tests can show that their pins catch it (1-7 in the forward,
+ * 8-10 in the backward).  The default build (no define) is the oracle.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -275,6 +279,217 @@ int oracle_decode_step(int variant, int N, int H, int dk, int dv,
                      write_w ? write_w + nh * dk : NULL,
                      eps, scale, o + nh * dv, x, work);
         free(x); free(work);
+    }
+    return 0;
+}
+
+/*
+ * Backward of the whole-sequence forward (reverse mode through the token
+ * recurrence, in the forward's own steps taken backwards).  Given the
+ * gradient of a loss with respect to the outputs, d_o [B,T,H,dv], and to the
+ * final state, d_final [B,H,dk,dv] (NULL: zero), it writes the gradient with
+ * respect to every input of oracle_forward:
+ *   dq, dk [B,T,H,dk]; dv [B,T,H,dv];
+ *   dbeta [B,T,H] (d/d beta_t, or d/d eta_t for KLA; not for GDN-2);
+ *   dlog_g [B,T,H] or [B,T,H,dk] (not for DeltaNet);
+ *   derase_b, dwrite_w [B,T,H,dk] (GDN-2 only);
+ *   dinitial_state [B,H,dk,dv] (may be NULL).
+ * Outputs a variant does not use may be NULL.  The states S_0 .. S_T of each
+ * (batch, head) are kept (T + 1 matrices of dk x dv doubles).
+ *
+ * Per token t, with dS the gradient with respect to S_t on entry:
+ *   o_t = S_t^T (scale q_t)    dS += scale q_t d_o_t^T,  dq_t = scale S_t d_o_t
+ *   S_t = S~ - a x^T + c v^T   da = -dS x,  dc = dS v,  dv_t = dS^T c,
+ *                              dx = -dS^T a,  dS~ = dS
+ *   x = S~^T k                 dS~ += k dx^T,  dk_t += S~ dx
+ *   S~ = Diag(g) S_{t-1}       d log g_i = g_i sum_j dS~_ij (S_{t-1})_ij (summed
+ *                              over i for a scalar decay),  dS_{t-1} = Diag(g) dS~
+ * then a, c back to their inputs: a = c = beta k (dbeta = k.(da + dc),
+ * dk += beta (da + dc)); for KLA beta = eta / (||k||^2 + eps) adds
+ * d eta = dbeta / (||k||^2 + eps) and dk -= 2 dbeta eta k / (||k||^2 + eps)^2;
+ * for GDN-2 a = b.k, c = w.k (db = da.k, dw = dc.k, dk += b.da + w.dc).
+ * Mutants 8-10 plant mistakes in these steps for the finite-difference pins.
+ */
+int oracle_backward(int variant, int B, int T, int H, int dk, int dv,
+                    const double *q, const double *k, const double *v,
+                    const double *beta, const double *log_g,
+                    const double *erase_b, const double *write_w,
+                    const double *initial_state, const double *d_o, const double *d_final,
+                    double *dq, double *dkey, double *dval, double *dbeta, double *dlog_g,
+                    double *derase_b, double *dwrite_w, double *dinitial_state,
+                    double eps, double scale, int nthreads)
+{
+    long bh;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0 || !d_o) return -1;
+    if (variant < OR_DELTANET || variant > OR_KLA) return -1;
+    if ((scalar_decay(variant) || channel_decay(variant)) && !log_g) return -1;
+    if (variant == OR_GDN2 && (!erase_b || !write_w)) return -1;
+    if (variant != OR_GDN2 && !beta) return -1;
+    if (!dq || !dkey || !dval) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < (long)B * H; ++bh) {
+        int b_ = (int)(bh / H), h = (int)(bh % H), t, i, j;
+        const size_t mat = (size_t)dk * dv;
+        double *Sall = (double *)malloc(sizeof(double) * mat * (size_t)(T + 1));
+        double *dS = (double *)malloc(sizeof(double) * mat);
+        double *St = (double *)malloc(sizeof(double) * mat);     /* S~ of token t */
+        double *x = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *work = (double *)malloc(sizeof(double) * (size_t)(dk > dv ? dk : dv));
+        double *obuf = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *a = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *c = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *da = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *dc = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *dx = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *g = (double *)malloc(sizeof(double) * (size_t)dk);
+
+        /* forward, keeping S_0 .. S_T */
+        if (initial_state)
+            memcpy(Sall, initial_state + bh * (long)mat, sizeof(double) * mat);
+        else
+            memset(Sall, 0, sizeof(double) * mat);
+        for (t = 0; t < T; ++t) {
+            long th = ((long)b_ * T + t) * H + h;
+            memcpy(Sall + (size_t)(t + 1) * mat, Sall + (size_t)t * mat, sizeof(double) * mat);
+            oracle_token(variant, dk, dv, Sall + (size_t)(t + 1) * mat, q + th * dk, k + th * dk, v + th * dv,
+                         beta ? beta[th] : 0.0, gate_ptr(variant, log_g, th, dk),
+                         erase_b ? erase_b + th * dk : NULL, write_w ? write_w + th * dk : NULL,
+                         eps, scale, obuf, x, work);
+        }
+
+        /* backward */
+        if (d_final)
+            memcpy(dS, d_final + bh * (long)mat, sizeof(double) * mat);
+        else
+            memset(dS, 0, sizeof(double) * mat);
+        for (t = T - 1; t >= 0; --t) {
+            long th = ((long)b_ * T + t) * H + h;
+            const double *qt = q + th * dk, *kt = k + th * dk, *vt = v + th * dv;
+            const double *dot = d_o + th * dv;
+            const double *Snew = Sall + (size_t)(t + 1) * mat, *Sprev = Sall + (size_t)t * mat;
+            const double *lg = gate_ptr(variant, log_g, th, dk);
+            double *dqt = dq + th * dk, *dkt = dkey + th * dk, *dvt = dval + th * dv;
+            double step = 0.0, nk = 0.0, dstep = 0.0;
+
+            /* readout o_t = S_t^T (scale q_t) */
+            for (i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                for (j = 0; j < dv; ++j) {
+                    acc += Snew[i * dv + j] * dot[j];
+                    dS[i * dv + j] += scale * qt[i] * dot[j];
+                }
+                dqt[i] = scale * acc;
+            }
+
+            /* recompute S~, x and the erase / write vectors a, c */
+            for (i = 0; i < dk; ++i)
+                g[i] = scalar_decay(variant) ? exp(lg[0]) : channel_decay(variant) ? exp(lg[i]) : 1.0;
+            for (i = 0; i < dk; ++i)
+                for (j = 0; j < dv; ++j) St[i * dv + j] = g[i] * Sprev[i * dv + j];
+            oracle_readout(dk, dv, St, kt, x);
+            if (variant == OR_GDN2) {
+                for (i = 0; i < dk; ++i) {
+                    a[i] = erase_b[th * dk + i] * kt[i];
+                    c[i] = write_w[th * dk + i] * kt[i];
+                }
+            } else {
+                step = beta[th];
+                if (variant == OR_KLA) {
+                    for (i = 0; i < dk; ++i) nk += kt[i] * kt[i];
+                    step = beta[th] / (nk + eps);
+                }
+                for (i = 0; i < dk; ++i) a[i] = c[i] = step * kt[i];
+            }
+
+            /* S_t = S~ - a x^T + c v^T */
+            for (i = 0; i < dk; ++i) {
+                double sa = 0.0, sc = 0.0;
+                for (j = 0; j < dv; ++j) {
+                    sa += dS[i * dv + j] * x[j];
+                    sc += dS[i * dv + j] * vt[j];
+                }
+                da[i] = -sa;
+                dc[i] = sc;
+            }
+            for (j = 0; j < dv; ++j) {
+                double sa = 0.0, sc = 0.0;
+                for (i = 0; i < dk; ++i) {
+                    sa += dS[i * dv + j] * a[i];
+                    sc += dS[i * dv + j] * c[i];
+                }
+#if ORACLE_MUTANT == 8
+                dx[j] = sa;                               /* mutant: sign of the erase term */
+#else
+                dx[j] = -sa;
+#endif
+                dvt[j] = sc;
+            }
+            /* dS now holds dS~; x = S~^T k adds k dx^T and gives dk its readout term */
+            for (i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                for (j = 0; j < dv; ++j) {
+                    acc += St[i * dv + j] * dx[j];
+                    dS[i * dv + j] += kt[i] * dx[j];
+                }
+#if ORACLE_MUTANT == 10
+                dkt[i] = 0.0;                             /* mutant: readout term of dk dropped */
+#else
+                dkt[i] = acc;
+#endif
+            }
+            /* S~ = Diag(g) S_{t-1} */
+            if (scalar_decay(variant) || channel_decay(variant)) {
+                double tot = 0.0;
+                for (i = 0; i < dk; ++i) {
+                    double acc = 0.0;
+                    for (j = 0; j < dv; ++j) acc += dS[i * dv + j] * Sprev[i * dv + j];
+                    if (channel_decay(variant)) {
+                        if (dlog_g) dlog_g[th * dk + i] = g[i] * acc;
+                    } else {
+                        tot += g[i] * acc;
+                    }
+                }
+                if (scalar_decay(variant) && dlog_g) dlog_g[th] = tot;
+            }
+            for (i = 0; i < dk; ++i)
+                for (j = 0; j < dv; ++j) {
+#if ORACLE_MUTANT == 9
+                    (void)0;                              /* mutant: decay not applied to dS */
+#else
+                    dS[i * dv + j] *= g[i];
+#endif
+                }
+
+            /* a, c back to k and the gates */
+            if (variant == OR_GDN2) {
+                for (i = 0; i < dk; ++i) {
+                    if (derase_b) derase_b[th * dk + i] = da[i] * kt[i];
+                    if (dwrite_w) dwrite_w[th * dk + i] = dc[i] * kt[i];
+                    dkt[i] += erase_b[th * dk + i] * da[i] + write_w[th * dk + i] * dc[i];
+                }
+            } else {
+                for (i = 0; i < dk; ++i) {
+                    dstep += kt[i] * (da[i] + dc[i]);
+                    dkt[i] += step * (da[i] + dc[i]);
+                }
+                if (variant == OR_KLA) {
+                    double den = nk + eps;
+                    if (dbeta) dbeta[th] = dstep / den;
+                    for (i = 0; i < dk; ++i) dkt[i] -= 2.0 * dstep * beta[th] * kt[i] / (den * den);
+                } else if (dbeta) {
+                    dbeta[th] = dstep;
+                }
+            }
+        }
+        if (dinitial_state) memcpy(dinitial_state + bh * (long)mat, dS, sizeof(double) * mat);
+        free(Sall); free(dS); free(St); free(x); free(work); free(obuf);
+        free(a); free(c); free(da); free(dc); free(dx); free(g);
     }
     return 0;
 }
