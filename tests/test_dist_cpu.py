@@ -65,3 +65,21 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(2.5, 1) == 2.5
     assert bench.job_throughput(10, 2, 4.0, 1) == pytest.approx(5000.0)
+
+
+def test_recorded_traffic_is_keyed_by_code_not_comments(tmp_path):
+    """bench.py uses a committed ncu traffic figure only for the code it was
+    taken on: a comment-only edit keeps the key, a code edit changes it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    code = "int f(int x) {\n  // one comment\n  return x + 1; /* another */\n}\n"
+    assert bench._code_only(code) == bench._code_only(code.replace("one comment", "reworded comment"))
+    assert bench._code_only(code) != bench._code_only(code.replace("x + 1", "x + 2"))
+    assert "comment" not in bench._code_only(code)
+    # every kernel named in the traffic table has a current key or is ignored
+    for line in open(os.path.join(ROOT, "profiles", "ncu_traffic.txt")):
+        f = line.split()
+        if line.startswith("#") or len(f) < 4:
+            continue
+        got = bench.recorded_traffic(f[0], f[1])
+        assert got is None or got == float(f[3])
