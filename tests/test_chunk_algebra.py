@@ -1,0 +1,134 @@
+"""The chunk-form equations, restated in float64 numpy, against the oracle.
+
+The CUDA path computes the forward in chunks (a chunk-parallel preparation and
+a sequential carry over chunks), and the planned backward does the same in
+reverse.  This CPU test pins both sets of equations, with a per-channel decay
+(KDA; a scalar decay and DeltaNet are its special cases), to the token-by-token
+oracle on a ragged sequence with an initial state and a q scale:
+
+forward, per chunk with the chunk-local cumulative log decay gamma (C x d_k):
+    A = tril(Diag(beta) (K o e^gamma)(K o e^-gamma)^T, -1),  T = (I + A)^-1
+    W = T Diag(beta) (K o e^gamma),  U' = T Diag(beta) V,  E = U' - W S0
+    P = tril(scale (Q o e^gamma)(K o e^-gamma)^T)
+    O = scale (Q o e^gamma) S0 + P E
+    S_C = Diag(e^gamma_C) S0 + Kt^T E,  Kt = K o e^(gamma_C - gamma)
+backward, chunks in reverse, dS the gradient of the chunk's end state:
+    dE = Kt dS + P^T dO
+    dS0 = Diag(e^gamma_C) dS + scale (Q o e^gamma)^T dO - W^T dE
+so the sequential part of the backward is the forward carry's mirror on the
+same per-chunk operands (Kt, P, Q o e^gamma, W); every other gradient is local
+to a chunk given S0, dS and dO.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_forward_b200.inputs import make_inputs
+
+C = 8
+
+
+def chunk_forward(q, k, v, beta, lg, s0, scale):
+    """One sequence: q, k [T, dk], v [T, dv], beta [T], lg [T, dk] (log decay)."""
+    T = k.shape[0]
+    o = np.zeros((T, v.shape[1]))
+    S = s0.copy()
+    saved = []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(T, c0 + C))
+        K, Q, V, b = k[sl], q[sl], v[sl], beta[sl]
+        gam = np.cumsum(lg[sl], axis=0)
+        Kg, Ki, Qg = K * np.exp(gam), K * np.exp(-gam), Q * np.exp(gam)
+        n = K.shape[0]
+        A = np.tril(b[:, None] * (Kg @ Ki.T), -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ (b[:, None] * Kg)
+        Up = Tm @ (b[:, None] * V)
+        E = Up - W @ S
+        P = np.tril(scale * (Qg @ Ki.T))
+        Kt = K * np.exp(gam[-1] - gam)
+        o[sl] = scale * Qg @ S + P @ E
+        saved.append(dict(sl=sl, S0=S.copy(), K=K, Q=Q, V=V, b=b, gam=gam, Kg=Kg, Ki=Ki, Qg=Qg,
+                          T=Tm, W=W, E=E, P=P, Kt=Kt))
+        S = np.exp(gam[-1])[:, None] * S + Kt.T @ E
+    return o, S, saved
+
+
+def chunk_backward(saved, dO, dS_final, scale):
+    T = saved[-1]["sl"].stop
+    dk, dv = saved[0]["K"].shape[1], saved[0]["V"].shape[1]
+    g = {"q": np.zeros((T, dk)), "k": np.zeros((T, dk)), "v": np.zeros((T, dv)),
+         "beta": np.zeros(T), "log_g": np.zeros((T, dk))}
+    dS = dS_final.copy()
+    for sv in reversed(saved):
+        sl, S0, K, Q, V, b, gam = (sv[x] for x in ("sl", "S0", "K", "Q", "V", "b", "gam"))
+        Kg, Ki, Qg, Tm, W, E, P, Kt = (sv[x] for x in ("Kg", "Ki", "Qg", "T", "W", "E", "P", "Kt"))
+        dOc = dO[sl]
+        gC = np.exp(gam[-1])
+        # the reverse carry: end-state gradient -> start-state gradient
+        dE = Kt @ dS + P.T @ dOc
+        dS0 = gC[:, None] * dS + scale * Qg.T @ dOc - W.T @ dE
+        # chunk-local gradients
+        dgam = np.zeros_like(gam)
+        dgam[-1] += np.sum(dS * S0, 1) * gC
+        dKt = E @ dS.T
+        dQg = scale * dOc @ S0.T
+        dP = np.tril(dOc @ E.T)
+        dW = -dE @ S0.T
+        tU, tW = Tm.T @ dE, Tm.T @ dW
+        dV = b[:, None] * tU
+        dKg = b[:, None] * tW
+        db = np.sum(V * tU, 1) + np.sum(Kg * tW, 1)
+        dT = dE @ (b[:, None] * V).T + dW @ (b[:, None] * Kg).T
+        dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+        db += np.sum(dA * (Kg @ Ki.T), 1)
+        M = b[:, None] * dA
+        dKg += M @ Ki
+        dKi = M.T @ Kg + scale * dP.T @ Qg
+        dQg += scale * dP @ Ki
+        fac = np.exp(gam[-1] - gam)
+        dK = dKt * fac + dKg * np.exp(gam) + dKi * np.exp(-gam)
+        dgam += -dKt * Kt + dKg * Kg - dKi * Ki + dQg * Qg
+        dgam[-1] += np.sum(dKt * Kt, 0)
+        g["q"][sl] = dQg * np.exp(gam)
+        g["k"][sl] = dK
+        g["v"][sl] = dV
+        g["beta"][sl] = db
+        g["log_g"][sl] = np.cumsum(dgam[::-1], axis=0)[::-1]
+        dS = dS0
+    g["initial_state"] = dS
+    return g
+
+
+@pytest.mark.parametrize("variant", ["deltanet", "gdn", "kda"])
+def test_chunk_equations_match_the_oracle(variant):
+    B, T, H, dk, dv, scale = 1, 29, 1, 6, 5, 0.7
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.float32, seed=7)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    rng = np.random.default_rng(7)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    dO = rng.standard_normal((B, T, H, dv))
+    dS = rng.standard_normal((B, H, dk, dv))
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=s0, scale=scale)
+    g_ref = oracle.backward(variant, d_o=dO, d_final=dS, initial_state=s0, scale=scale, **d)
+
+    if variant == "deltanet":
+        lg = np.zeros((T, dk))
+    elif variant == "gdn":
+        lg = np.repeat(d["log_g"][0, :, 0][:, None], dk, axis=1)
+    else:
+        lg = d["log_g"][0, :, 0]
+    o, S, saved = chunk_forward(d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0], d["beta"][0, :, 0],
+                                lg, s0[0, 0], scale)
+    np.testing.assert_allclose(o, o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref[0, 0], rtol=0, atol=1e-12)
+
+    g = chunk_backward(saved, dO[0, :, 0], dS[0, 0], scale)
+    for name in ("q", "k", "v", "beta"):
+        np.testing.assert_allclose(g[name], g_ref[name][0, :, 0], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(g["initial_state"], g_ref["initial_state"][0, 0], rtol=0, atol=1e-10)
+    if variant == "gdn":      # one decay per token: its gradient sums over the channels
+        np.testing.assert_allclose(g["log_g"].sum(1), g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
+    elif variant == "kda":
+        np.testing.assert_allclose(g["log_g"], g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
