@@ -132,3 +132,37 @@ def test_chunk_equations_match_the_oracle(variant):
         np.testing.assert_allclose(g["log_g"].sum(1), g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
     elif variant == "kda":
         np.testing.assert_allclose(g["log_g"], g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("variant", ["gdn", "kda"])
+def test_two_record_carry_step_matches_the_oracle(variant):
+    """One carry step over two records (c, c+1), from their single-chunk quantities
+    only, with G_c = Diag(e^gamma_C) of chunk c (the chunk's decay per channel):
+        M    = W_{c+1} Kt_c^T                     (cross term, local to the pair)
+        What = [W_c ; W_{c+1} G_c - M W_c],  Uhat = [U'_c ; U'_{c+1} - M U'_c]
+        [E_c ; E_{c+1}] = Uhat - What S
+        S''  = G_{c+1} G_c S + [Kt_c G_{c+1} ; Kt_{c+1}]^T [E_c ; E_{c+1}]
+        O_c  = Qg_c S + P_c E_c
+        O_c+1 = Qg_{c+1} G_c S + [Qg_{c+1} Kt_c^T , P_{c+1}] [E_c ; E_{c+1}]
+    (Qg = scale Q o e^gamma).  Half the sequential steps of the 64-token carry."""
+    B, T, H, dk, dv, scale = 1, 2 * C, 1, 6, 5, 0.7
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.float32, seed=9)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    rng = np.random.default_rng(9)
+    S = rng.standard_normal((dk, dv))
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=S[None, None], scale=scale)
+    lg = (np.repeat(d["log_g"][0, :, 0][:, None], dk, axis=1) if variant == "gdn" else d["log_g"][0, :, 0])
+    _, _, sv = chunk_forward(d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0], d["beta"][0, :, 0], lg, S, scale)
+    a, b = sv
+    ga, gb = np.exp(a["gam"][-1]), np.exp(b["gam"][-1])      # per-channel end decays
+    Upa, Upb = a["T"] @ (a["b"][:, None] * a["V"]), b["T"] @ (b["b"][:, None] * b["V"])
+    Qga, Qgb = scale * a["Qg"], scale * b["Qg"]
+    M = b["W"] @ a["Kt"].T
+    What = np.vstack([a["W"], b["W"] * ga[None, :] - M @ a["W"]])
+    Uhat = np.vstack([Upa, Upb - M @ Upa])
+    E = Uhat - What @ S
+    S2 = (gb * ga)[:, None] * S + np.vstack([a["Kt"] * gb[None, :], b["Kt"]]).T @ E
+    Oa = Qga @ S + a["P"] @ E[:C]
+    Ob = (Qgb * ga[None, :]) @ S + np.hstack([Qgb @ a["Kt"].T, b["P"]]) @ E
+    np.testing.assert_allclose(np.vstack([Oa, Ob]), o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S2, S_ref[0, 0], rtol=0, atol=1e-12)
