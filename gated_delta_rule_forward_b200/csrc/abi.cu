@@ -160,6 +160,16 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
   return "none";
 }
 
+gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms, int *segments,
+                              int *segment_chunks, int *split_chunk) {
+  if (!valid_variant(variant)) return fail(GDR_ERR_INVALID_ARG, "unknown variant");
+  if (!valid_dim(dv)) return fail(GDR_ERR_INVALID_ARG, "dv must be 64 or 128");
+  if (B < 0 || T < 0 || H < 0 || sms < 0) return fail(GDR_ERR_INVALID_ARG, "B, T, H and sms must be >= 0");
+  if (!segments || !segment_chunks || !split_chunk) return fail(GDR_ERR_INVALID_ARG, "output pointer is NULL");
+  gdr_split_plan(variant, B, T, H, dv, sms, segments, segment_chunks, split_chunk);
+  return GDR_OK;
+}
+
 gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                  const gdr_fwd_args_t *a, float eps, float scale, int chunk,
                                  void *workspace, size_t workspace_bytes, void *stream) {

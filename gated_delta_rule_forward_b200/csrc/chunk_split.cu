@@ -1870,22 +1870,31 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
 struct SegPlan {
   int G = 1, L = 0;
 };
-SegPlan seg_plan(int B, int H, int dv, int NC) {
-  SegPlan sp;
-  sp.L = NC;
+// SMs of the current device, 0 if there is none.
+int device_sms() {
   int dev = 0, sms = 0;
-  if (dv != 128 || NC < 64 || cudaGetDevice(&dev) != cudaSuccess ||
+  if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
-    return sp;
+    return 0;
   }
-  // phase 1 runs (2G - 3) bh CTAs, at most one per SM
+  return sms;
+}
+SegPlan seg_plan_for(int B, int H, int dv, int NC, int sms) {
+  SegPlan sp;
+  sp.L = NC;
   const long long bh = static_cast<long long>(B) * H;
+  if (dv != 128 || NC < 64 || bh <= 0 || sms <= 0) return sp;
+  // phase 1 runs (2G - 3) bh CTAs, at most one per SM
   const int G = static_cast<int>(std::min<long long>(16, (sms / bh + 3) / 2));
   if (G < 3) return sp;
   sp.L = (NC + G - 1) / G;
   sp.G = (NC + sp.L - 1) / sp.L;
   return sp;
+}
+SegPlan seg_plan(int B, int H, int dv, int NC) {
+  if (dv != 128 || NC < 64) return seg_plan_for(B, H, dv, NC, 0);
+  return seg_plan_for(B, H, dv, NC, device_sms());
 }
 size_t seg_extra_floats(int B, int H, int dv, const SegPlan &sp) {
   if (sp.G == 1) return 0;
@@ -1911,17 +1920,10 @@ struct PipePlan {
   int c_split = 0;   // 0: serial
   int prep_sms = 0;  // SMs the second preparation grid is sized for
 };
-PipePlan pipe_plan(int variant, int B, int H, int NC) {
+PipePlan pipe_plan_for(int variant, int B, int H, int NC, int sms) {
   PipePlan pp;
-  if (NC < 4) return pp;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return pp;
-  }
   const long long bh = static_cast<long long>(B) * H;
-  if (sms - bh < 16) return pp;
+  if (NC < 4 || bh <= 0 || sms - bh < 16) return pp;
   // per variant family: scalar decay (two preparation CTAs per SM), KDA, GDN-2 (one each)
   const int fam = variant == kGDN2 ? 2 : variant == kKDA ? 1 : 0;
   const double slots = fam ? 1.0 : 2.0;                       // preparation CTAs per SM
@@ -1943,6 +1945,10 @@ PipePlan pipe_plan(int variant, int B, int H, int NC) {
   if (best > 0.97 * serial) pp.c_split = 0;
   pp.prep_sms = static_cast<int>(sms - bh);
   return pp;
+}
+PipePlan pipe_plan(int variant, int B, int H, int NC) {
+  if (NC < 4) return PipePlan();
+  return pipe_plan_for(variant, B, H, NC, device_sms());
 }
 
 template <int VAR>
@@ -2058,6 +2064,15 @@ size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   const gdr::tc::SegPlan sp = gdr::tc::seg_plan(B, H, dv, static_cast<int>(NC));
   if (sp.G == 1) return records;
   return (records + 255) / 256 * 256 + 4 * gdr::tc::seg_extra_floats(B, H, dv, sp);
+}
+
+void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,
+                    int *split_chunk) {
+  const int NC = (T + 63) / 64;
+  const gdr::tc::SegPlan sp = gdr::tc::seg_plan_for(B, H, dv, NC, sms);
+  *segments = sp.G;
+  *segment_chunks = sp.L;
+  *split_chunk = sp.G == 1 ? gdr::tc::pipe_plan_for(variant, B, H, NC, sms).c_split : 0;
 }
 
 int gdr_split_launches(int variant, int B, int T, int H, int dv) {

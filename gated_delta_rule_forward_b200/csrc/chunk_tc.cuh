@@ -20,6 +20,9 @@ int gdr_read_chan_error();
 bool gdr_split_supported(int variant, int dk, int dv);
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv);
 int gdr_split_launches(int variant, int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
+// The two-kernel path's schedule on a device with `sms` SMs (no device query).
+void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,
+                    int *split_chunk);
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err);
 int gdr_read_split_error();
 // Fixed scratch of the no-allocation entry point (chunk_split.cu).

@@ -200,6 +200,24 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
                                     int chunk);
 
 /*
+ * How the two-kernel chunked path schedules B sequences of T tokens and H
+ * heads on a device with `sms` SMs (host-only; no device is queried, so it
+ * serves to inspect a plan for any device).  Writes
+ *   *segments        the carry's segments per sequence (1: not segmented),
+ *   *segment_chunks  64-token chunks per segment,
+ *   *split_chunk     the chunk where the pipelined sweep cuts each sequence
+ *                    (0: serial sweep; only when not segmented).
+ * Segmenting needs dv = 128, at least 64 chunks and floor(sms / (B * H))
+ * large enough for three segments; the pipelined sweep needs at least 16
+ * SMs beside the carry's B * H and is taken where its cost model expects a
+ * gain.  B * H = 0 plans one segment and no cut.  Returns
+ * GDR_ERR_INVALID_ARG for an unknown variant, dv not in {64, 128}, a
+ * negative size or a NULL output.
+ */
+gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms, int *segments,
+                              int *segment_chunks, int *split_chunk);
+
+/*
  * Synchronises `stream`, then reads and clears the library's device-side
  * error word.  Returns, since the previous call:
  *   GDR_ERR_TIMEOUT  a bounded wait inside a kernel (an mbarrier wait past its

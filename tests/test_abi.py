@@ -167,3 +167,43 @@ def test_split_needs_workspace(L):
                                  ctypes.c_void_p(FAKE), 1 << 20, None) == 4   # reaches the launch
     assert L.gdr_forward_chunked(1, 1, 2, 8, 2, 128, 128, ctypes.byref(a), 1e-6, 1.0, 65,
                                  ctypes.c_void_p(MISALIGNED), 1 << 20, None) == 3
+
+
+def _plan(L, variant, B, T, H, dv=128, sms=148):
+    g, lc, cs = ctypes.c_int(-1), ctypes.c_int(-1), ctypes.c_int(-1)
+    st = L.gdr_forward_plan(variant, B, T, H, dv, sms, ctypes.byref(g), ctypes.byref(lc), ctypes.byref(cs))
+    assert st == 0, L.gdr_last_error()
+    return g.value, lc.value, cs.value
+
+
+def test_two_kernel_schedule_on_a_148_sm_device(L):
+    """The schedules the benchmark workloads get on B200 (148 SMs), and the edge cases."""
+    assert _plan(L, 1, 8, 2048, 8) == (1, 32, 22)      # 350M GDN: pipelined, cut at chunk 22 of 32
+    assert _plan(L, 0, 8, 2048, 8) == (1, 32, 22)      # DeltaNet: the same kernels
+    assert _plan(L, 4, 4, 4096, 16) == (1, 64, 43)     # 1.3B KLA
+    assert _plan(L, 2, 4, 4096, 16) == (1, 64, 53)     # 1.3B KDA
+    assert _plan(L, 3, 4, 4096, 16) == (1, 64, 51)     # 1.3B GDN-2
+    assert _plan(L, 1, 1, 65536, 16) == (6, 171, 0)    # 64k: six segments of 171 chunks
+    assert _plan(L, 1, 1, 4100, 2) == (13, 5, 0)       # the segmented GPU test: 13 segments of 5
+    assert _plan(L, 1, 2, 4480, 3) == (12, 6, 0)       # and its other shape: 12 of 6
+    for v in range(5):                                  # the pipelined GPU tests (24 chunks)
+        assert _plan(L, v, 4, 1531, 16)[2] > 0
+        assert _plan(L, v, 4, 1531, 16, dv=64)[2] > 0
+    assert _plan(L, 1, 2, 130, 3) == (1, 3, 0)         # three chunks: serial
+    assert _plan(L, 1, 16, 2048, 16) == (1, 32, 0)     # B*H = 256 > SMs: serial
+    assert _plan(L, 1, 1, 65536, 16, dv=64)[0] == 1    # segmenting needs dv = 128
+    assert _plan(L, 1, 0, 5000, 8) == (1, 79, 0)       # no sequences: nothing to divide by
+    assert _plan(L, 1, 4, 4096, 16, sms=0) == (1, 64, 0)
+
+
+def test_two_kernel_schedule_rejects_bad_arguments(L):
+    g = ctypes.c_int()
+    assert L.gdr_forward_plan(9, 1, 64, 1, 128, 148, ctypes.byref(g), ctypes.byref(g), ctypes.byref(g)) == 1
+    assert L.gdr_forward_plan(1, 1, 64, 1, 96, 148, ctypes.byref(g), ctypes.byref(g), ctypes.byref(g)) == 1
+    assert L.gdr_forward_plan(1, -1, 64, 1, 128, 148, ctypes.byref(g), ctypes.byref(g), ctypes.byref(g)) == 1
+    assert L.gdr_forward_plan(1, 1, 64, 1, 128, 148, None, ctypes.byref(g), ctypes.byref(g)) == 1
+
+
+def test_empty_batch_workspace_query(L):
+    """B * H = 0 with a long T is a valid no-op call; its workspace query must not divide by B * H."""
+    assert L.gdr_forward_workspace_size(1, 1, 0, 5000, 8, 128, 128, 0) == 0
