@@ -17,7 +17,8 @@ backward, chunks in reverse, dS the gradient of the chunk's end state:
     dS0 = Diag(e^gamma_C) dS + scale (Q o e^gamma)^T dO - W^T dE
 so the sequential part of the backward is the forward carry's mirror on the
 same per-chunk operands (Kt, P, Q o e^gamma, W); every other gradient is local
-to a chunk given S0, dS and dO.
+to a chunk given S0, dS and dO.  GDN-2's chunk form (its own test below) and
+a carry step over two records (the 128-token step) are pinned the same way.
 """
 import numpy as np
 import pytest
@@ -166,3 +167,42 @@ def test_two_record_carry_step_matches_the_oracle(variant):
     Ob = (Qgb * ga[None, :]) @ S + np.hstack([Qgb @ a["Kt"].T, b["P"]]) @ E
     np.testing.assert_allclose(np.vstack([Oa, Ob]), o_ref[0, :, 0], rtol=0, atol=1e-12)
     np.testing.assert_allclose(S2, S_ref[0, 0], rtol=0, atol=1e-12)
+
+
+def test_gdn2_chunk_equations_match_the_oracle():
+    """GDN-2's chunk form, with a = b o k (erase) and d = (w - b) o k:
+        A = tril(Gram(K, a), -1),  A^d = tril(Gram(K, d), -1),  P^a, P^d = tril(Gram(scale Q, a or d))
+        T = (I + A)^-1,  W = T (K o e^gamma),  U' = T (I - A^d) V,  E = U' - W S0
+        O = scale (Q o e^gamma) S0 + P^a E + P^d V
+        S_C = Diag(e^gamma_C) S0 + (a o e^(gamma_C - gamma))^T E + (d o e^(gamma_C - gamma))^T V
+    where Gram(X, Y)_tr = sum_i x_t[i] y_r[i] e^(gamma_t[i] - gamma_r[i]): the residual
+    form of the other variants with the write split off ("Gated DeltaNet-2", technical
+    core, read as erase on the key side and write weighted per channel)."""
+    B, T, H, dk, dv, scale = 1, 29, 1, 6, 5, 0.7
+    d = make_inputs("gdn2", B, T, H, dk, dv, dtype=torch.float32, seed=11)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    S = np.random.default_rng(11).standard_normal((dk, dv))
+    o_ref, S_ref = oracle.forward("gdn2", **d, initial_state=S[None, None], scale=scale)
+    q, k, v = d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0]
+    lg, eb, ww = d["log_g"][0, :, 0], d["erase_b"][0, :, 0], d["write_w"][0, :, 0]
+    o = np.zeros((T, dv))
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(T, c0 + C))
+        K, Q, V = k[sl], scale * q[sl], v[sl]
+        gam = np.cumsum(lg[sl], axis=0)
+        a, dd = eb[sl] * K, (ww[sl] - eb[sl]) * K
+        n = K.shape[0]
+
+        def gram(X, Y):
+            return (X * np.exp(gam)) @ (Y * np.exp(-gam)).T
+
+        A, Ad = np.tril(gram(K, a), -1), np.tril(gram(K, dd), -1)
+        Pa, Pd = np.tril(gram(Q, a)), np.tril(gram(Q, dd))
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ (K * np.exp(gam))
+        E = Tm @ (np.eye(n) - Ad) @ V - W @ S
+        o[sl] = (Q * np.exp(gam)) @ S + Pa @ E + Pd @ V
+        fac = np.exp(gam[-1] - gam)
+        S = np.exp(gam[-1])[:, None] * S + (a * fac).T @ E + (dd * fac).T @ V
+    np.testing.assert_allclose(o, o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref[0, 0], rtol=0, atol=1e-12)
