@@ -7,8 +7,8 @@ package does not load the library; the first call does, and raises if the
 library is missing.
 """
 from .ops import (VARIANTS, decode_step, device_status, forward, forward_kernel_name,  # noqa: F401
-                  forward_launches)
+                  forward_launches, forward_plan)
 from ._lib import GdrError  # noqa: F401
 
-__all__ = ["forward", "decode_step", "device_status", "forward_launches", "forward_kernel_name", "VARIANTS",
-           "GdrError"]
+__all__ = ["forward", "decode_step", "device_status", "forward_launches", "forward_kernel_name", "forward_plan",
+           "VARIANTS", "GdrError"]

@@ -164,3 +164,13 @@ def forward_launches(variant, dtype, B, T, H, dk, dv, chunk=0) -> int:
 
 def forward_kernel_name(variant, dtype, B, T, H, dk, dv, chunk=0) -> str:
     return lib().gdr_forward_kernel_name(variant_id(variant), _DTYPES[dtype], B, T, H, dk, dv, chunk).decode()
+
+
+def forward_plan(variant, B, T, H, dv, sms) -> dict:
+    """How the two-kernel chunked path schedules this problem on a device with
+    ``sms`` SMs (host-only): segments per sequence, chunks per segment, and the
+    chunk where the pipelined sweep cuts each sequence (0: serial)."""
+    g, lc, cs = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    check(lib().gdr_forward_plan(variant_id(variant), B, T, H, dv, sms, ctypes.byref(g), ctypes.byref(lc),
+                                 ctypes.byref(cs)))
+    return {"segments": g.value, "segment_chunks": lc.value, "split_chunk": cs.value}

@@ -207,3 +207,11 @@ def test_two_kernel_schedule_rejects_bad_arguments(L):
 def test_empty_batch_workspace_query(L):
     """B * H = 0 with a long T is a valid no-op call; its workspace query must not divide by B * H."""
     assert L.gdr_forward_workspace_size(1, 1, 0, 5000, 8, 128, 128, 0) == 0
+
+
+def test_forward_plan_binding():
+    import gated_delta_rule_forward_b200 as gdr
+    assert gdr.forward_plan("gdn", 8, 2048, 8, 128, 148) == {"segments": 1, "segment_chunks": 32, "split_chunk": 22}
+    assert gdr.forward_plan("kla", 1, 65536, 16, 128, 148) == {"segments": 6, "segment_chunks": 171, "split_chunk": 0}
+    with pytest.raises(gdr.GdrError):
+        gdr.forward_plan("gdn", 8, 2048, 8, 96, 148)
