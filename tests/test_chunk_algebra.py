@@ -262,3 +262,49 @@ def test_fp16_carry_operands_fit_the_bf16_budget():
     bf16 = lambda x: torch.from_numpy(x).to(torch.bfloat16).double().numpy()
     assert run(f16) < 2e-2 / 2          # measured 6.4e-3
     assert run(bf16) > 2e-2             # measured 4.0e-2: bf16 operands break the budget
+
+
+def _round_tf32(x):
+    """Round to the tf32 format (8-bit exponent, 10 stored mantissa bits), to
+    nearest with ties to even, from the float32 bit pattern."""
+    u = np.asarray(x, np.float32).copy().view(np.uint32)
+    u = (u + np.uint32(0xFFF) + ((u >> np.uint32(13)) & np.uint32(1))) & np.uint32(0xFFFFE000)
+    return u.view(np.float32).astype(np.float64)
+
+
+def test_channel_decay_gram_needs_tf32_operands():
+    """KDA's Gram / attention product [K o G; Q o G](K o G^-1)^T, with the decay
+    factored around the chunk's middle token (G = e^(gamma - gamma_m)): with every
+    other product exact, tf32 operands keep a 2048-token sequence at d = 128 inside
+    the bf16 budget (2e-2 of RMS); bf16 operands, one rounding of G, do not."""
+    T, d, C64 = 2048, 128, 64
+    dd = make_inputs("kda", 1, T, 1, d, d, dtype=torch.bfloat16, seed=4)
+    dd = {k: (None if v is None else v.double().numpy()) for k, v in dd.items()}
+    o_ref, _ = oracle.forward("kda", **dd)
+    q, k, v, beta, lg = (dd[n][0, :, 0] for n in ("q", "k", "v", "beta", "log_g"))
+    assert _round_tf32(np.array([1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11]))[0] == 1.0   # tie to even
+    assert _round_tf32(np.array([1.0 + 3 * 2.0 ** -11]))[0] == 1.0 + 2.0 ** -9
+
+    def run(rnd):
+        S = np.zeros((d, d))
+        out = []
+        for c0 in range(0, T, C64):
+            sl = slice(c0, c0 + C64)
+            K, Q, V, b = k[sl], q[sl], v[sl], beta[sl]
+            gam = np.cumsum(lg[sl], axis=0)
+            G = np.exp(gam - gam[31])
+            GQ = rnd(np.vstack([K * G, Q * G])) @ rnd(K / G).T
+            A = np.tril(b[:, None] * GQ[:C64], -1)
+            P = np.tril(GQ[C64:])
+            Tm = np.linalg.inv(np.eye(C64) + A)
+            W = Tm @ (b[:, None] * K * np.exp(gam))
+            E = Tm @ (b[:, None] * V) - W @ S
+            out.append((Q * np.exp(gam)) @ S + P @ E)
+            S = np.exp(gam[-1])[:, None] * S + (K * np.exp(gam[-1] - gam)).T @ E
+        o = np.vstack(out)
+        return np.abs(o - o_ref[0, :, 0]).max() / np.sqrt(np.mean(o_ref[0, :, 0] ** 2))
+
+    bf16 = lambda x: torch.from_numpy(np.asarray(x, np.float64)).to(torch.bfloat16).double().numpy()
+    assert run(lambda x: x) < 1e-12          # the factored product is exact algebra
+    assert run(_round_tf32) < 2e-2 / 2       # measured 2.8e-3
+    assert run(bf16) > 2e-2                  # measured 3.4e-2
