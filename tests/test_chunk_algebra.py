@@ -308,3 +308,42 @@ def test_channel_decay_gram_needs_tf32_operands():
     assert run(lambda x: x) < 1e-12          # the factored product is exact algebra
     assert run(_round_tf32) < 2e-2 / 2       # measured 2.8e-3
     assert run(bf16) > 2e-2                  # measured 3.4e-2
+
+
+def test_gdn2_preparation_products_need_fp16_operands():
+    """GDN-2's preparation products after the Gram product (R = T (I - A^d), W,
+    U' = R V, P^d V, Dt^T V) pass more roundings into the state than the other
+    variants'.  With the carry operands in fp16 throughout, a 4096-token sequence
+    at d = 128 keeps its final state within a quarter of the bf16 budget
+    (2e-2 of RMS) when those products take fp16 operands.  With bf16 operands the
+    state error triples, to three quarters of the budget on this one sequence;
+    across the 64 sequences of the 1.3B layer it left the budget on the GPU."""
+    T, d, C64 = 4096, 128, 64
+    dd = make_inputs("gdn2", 1, T, 1, d, d, dtype=torch.bfloat16, seed=6)
+    dd = {k: (None if v is None else v.double().numpy()) for k, v in dd.items()}
+    o_ref, S_ref = oracle.forward("gdn2", **dd)
+    q, k, v, lg, eb, ww = (dd[n][0, :, 0] for n in ("q", "k", "v", "log_g", "erase_b", "write_w"))
+    f16 = lambda x: np.asarray(x).astype(np.float16).astype(np.float64)
+    f32 = lambda x: np.asarray(x).astype(np.float32).astype(np.float64)
+    bf16 = lambda x: torch.from_numpy(np.asarray(x, np.float64)).to(torch.bfloat16).double().numpy()
+
+    def state_error(rp):
+        S = np.zeros((d, d))
+        for c0 in range(0, T, C64):
+            sl = slice(c0, c0 + C64)
+            K, V = k[sl], v[sl]
+            gam = np.cumsum(lg[sl], axis=0)
+            a, dw = eb[sl] * K, (ww[sl] - eb[sl]) * K
+            Ad = np.tril((K * np.exp(gam)) @ (dw * np.exp(-gam)).T, -1)
+            Tm = np.linalg.inv(np.eye(C64) + np.tril((K * np.exp(gam)) @ (a * np.exp(-gam)).T, -1))
+            W = rp(Tm) @ rp(K * np.exp(gam))
+            Up = rp(rp(Tm) @ rp(np.eye(C64) - Ad)) @ rp(V)
+            fac = np.exp(gam[-1] - gam)
+            DtV = rp(dw * fac).T @ rp(V)
+            E = f32(f16(Up) - f16(W) @ f16(S))
+            S = f32(np.exp(gam[-1])[:, None] * S + f16(a * fac).T @ f16(E) + f16(DtV))
+        return np.abs(S - S_ref[0, 0]).max() / np.sqrt(np.mean(S_ref[0, 0] ** 2))
+
+    e16, eb16 = state_error(f16), state_error(bf16)
+    assert e16 < 2e-2 / 4                    # measured 4.9e-3
+    assert eb16 > 2.5 * e16                  # measured 1.5e-2
