@@ -33,3 +33,21 @@ def test_reference_arm_prints_one_contract_line():
 def test_warmup_below_three_is_rejected():
     r = _bench("--impl", "reference", "--workload", "gdn_decode_256x16", "--steps", "1", "--warmup", "1")
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    """Launched the way multi-GPU runs are (torchrun, two ranks, 127.0.0.1), rank 0
+    alone times the oracle and prints; the other rank exits 0 without work."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--gpus", "2", "--workload", "gdn_decode_256x16", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0
