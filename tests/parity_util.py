@@ -29,6 +29,14 @@ def max_rel(gpu, ref):
     return float(np.max(np.abs(gpu - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
+def elem_rel(gpu, ref):
+    """max |gpu - ref| / max(|ref|, 1e-6 max|ref|): the element-wise relative error,
+    floored where the reference is near zero (reported next to the fp32 bar)."""
+    gpu = gpu.detach().double().cpu().numpy() if hasattr(gpu, "detach") else np.asarray(gpu)
+    floor = 1e-6 * max(float(np.max(np.abs(ref))), 1e-30)
+    return float(np.max(np.abs(gpu - ref) / np.maximum(np.abs(ref), floor)))
+
+
 def rms_rel(gpu, ref):
     gpu = gpu.detach().double().cpu().numpy() if hasattr(gpu, "detach") else np.asarray(gpu)
     return float(np.max(np.abs(gpu - ref)) / max(np.sqrt(np.mean(ref * ref)), 1e-30))
@@ -49,7 +57,8 @@ def assert_close(gpu, ref, dtype, what=""):
     is an output stored in bf16; an fp32 tensor in a bf16 run is the state."""
     if dtype == torch.float32:
         err = max_rel(gpu, ref)
-        assert err <= F32_TOL, f"{what}: max|err|/max|ref| = {err:.3e} > {F32_TOL}"
+        assert err <= F32_TOL, (f"{what}: max|err|/max|ref| = {err:.3e} > {F32_TOL} "
+                                f"(element-wise, floored at 1e-6 max|ref|: {elem_rel(gpu, ref):.3e})")
     elif gpu.dtype == torch.bfloat16:
         err = bf16_out_rel(gpu, ref)
         assert err <= BF16_TOL, (f"{what}: max(|err| - 2^-8|ref|)/RMS(ref) = {err:.3e} > {BF16_TOL} "
