@@ -217,7 +217,7 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
   p.eps = eps; p.scale = scale;
   if (kern == Kernel::Split) {
     std::string err;
-    const cudaError_t e = gdr_launch_split(p, workspace, s, &err);
+    const cudaError_t e = gdr_launch_split(p, workspace, workspace_bytes, s, &err);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_split: " + err + cudaGetErrorString(e));
     return GDR_OK;
   }
@@ -238,14 +238,18 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
   if (!a) return fail(GDR_ERR_INVALID_ARG, "args is NULL");
   if (!split_ok(variant, dtype, dk, dv))
     return fail(GDR_ERR_UNSUPPORTED,
-                "the no-allocation entry point covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O and dk = 128");
-  const size_t need = gdr_split_workspace_bytes(variant, B, T, H, dv);
+                "the no-allocation entry point needs bf16 I/O, dk = 128 and dv in {64, 128} (all five variants)");
+  // The records must fit; the segmented carry's maps are optional (without
+  // room for them the call runs the unsegmented sweep).
+  const size_t rec = gdr_split_record_bytes(variant, dv);
+  const size_t records = (size_t)B * H * (((size_t)T + 63) / 64);
   const size_t have = gdr_split_fixed_scratch_bytes();
-  if (need > have)
+  if (records * rec > have)
     return fail(GDR_ERR_UNSUPPORTED,
-                "problem needs " + std::to_string(need) + " bytes of scratch but the fixed scratch holds " +
-                    std::to_string(have) + " (B * H * ceil(T / 64) must be at most " +
-                    std::to_string(have / (need / ((size_t)B * H * ((T + 63) / 64)))) + " for this dv)");
+                "problem needs " + std::to_string(records) + " records of " + std::to_string(rec) + " bytes (" +
+                    std::to_string(records * rec) + " bytes) but the fixed scratch holds " + std::to_string(have) +
+                    " bytes: B * H * ceil(T / 64) must be at most " + std::to_string(have / rec) +
+                    " for this variant and dv");
   if ((long)B * H == 0 || T == 0) return gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, a, eps, scale, 65,
                                                              nullptr, 0, stream);
   if (!a->q || !a->k || !a->v || !a->o) return fail(GDR_ERR_INVALID_ARG, "q, k, v and o are required");
@@ -259,9 +263,19 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
   if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be >= 0");
   if (injected_launch_fault()) return fail(GDR_ERR_CUDA, "injected launch failure (GDR_FAULT=launch)");
   void *scratch = nullptr;
-  const cudaError_t e = gdr_split_fixed_scratch(&scratch);
+  cudaError_t e = gdr_split_fixed_scratch(&scratch);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("fixed scratch lookup: ") + cudaGetErrorString(e));
-  return gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, a, eps, scale, 65, scratch, have, stream);
+  gdr::FwdProblem p;
+  p.variant = variant; p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
+  p.bf16_io = true;
+  p.q = a->q; p.k = a->k; p.v = a->v;
+  p.beta = a->beta; p.log_g = a->log_g; p.erase_b = a->erase_b; p.write_w = a->write_w;
+  p.s0 = a->initial_state; p.s_final = a->final_state; p.o = a->o;
+  p.eps = eps; p.scale = scale;
+  std::string err;
+  e = gdr_launch_split(p, scratch, have, static_cast<cudaStream_t>(stream), &err);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_split: " + err + cudaGetErrorString(e));
+  return GDR_OK;
 }
 
 gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv, const void *q, const void *k,

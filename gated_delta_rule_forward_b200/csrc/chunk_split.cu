@@ -1994,12 +1994,15 @@ cudaError_t launch_pipelined(const FwdProblem &p, int NC, uint8_t *w, const Pipe
   return launch_carry<MODE>(p, NC, w, l2, true, stream, err);
 }
 
+// `ws_bytes` is the workspace the call may use: a segmented plan whose maps do
+// not fit beside the records falls back to the unsegmented sweep.
 template <int VAR>
-cudaError_t launch_split(const FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
+cudaError_t launch_split(const FwdProblem &p, void *ws, size_t ws_bytes, cudaStream_t stream, std::string *err) {
   constexpr int MODE = VAR == kGDN2 ? 2 : VAR == kKDA ? 1 : 0;
   const int NC = (p.T + C - 1) / C;
   uint8_t *w = static_cast<uint8_t *>(ws);
-  const SegPlan sp = seg_plan(p.B, p.H, p.dv, NC);
+  SegPlan sp = seg_plan(p.B, p.H, p.dv, NC);
+  if (sp.G > 1 && gdr_split_workspace_bytes(VAR, p.B, p.T, p.H, p.dv) > ws_bytes) sp = SegPlan{1, NC};
   if (sp.G == 1) {
     const PipePlan pp = pipe_plan(VAR, p.B, p.H, NC);
     if (pp.c_split > 0) return launch_pipelined<VAR>(p, NC, w, pp, stream, err);
@@ -2055,12 +2058,15 @@ bool gdr_split_supported(int variant, int dk, int dv) {
   return v && dk == 128 && (dv == 64 || dv == 128);
 }
 
+size_t gdr_split_record_bytes(int variant, int dv) {
+  return variant == gdr::kGDN2  ? gdr::tc::rec_bytes_gdn2(dv / 64)
+         : variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64)
+                                : gdr::tc::rec_bytes(dv / 64);
+}
+
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
   const size_t NC = (static_cast<size_t>(T) + 63) / 64;
-  const size_t rec = variant == gdr::kGDN2  ? gdr::tc::rec_bytes_gdn2(dv / 64)
-                     : variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64)
-                                            : gdr::tc::rec_bytes(dv / 64);
-  const size_t records = static_cast<size_t>(B) * H * NC * rec;
+  const size_t records = static_cast<size_t>(B) * H * NC * gdr_split_record_bytes(variant, dv);
   const gdr::tc::SegPlan sp = gdr::tc::seg_plan(B, H, dv, static_cast<int>(NC));
   if (sp.G == 1) return records;
   return (records + 255) / 256 * 256 + 4 * gdr::tc::seg_extra_floats(B, H, dv, sp);
@@ -2081,14 +2087,15 @@ int gdr_split_launches(int variant, int B, int T, int H, int dv) {
   return gdr::tc::pipe_plan(variant, B, H, NC).c_split > 0 ? 4 : 2;
 }
 
-cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err) {
+cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, size_t ws_bytes, cudaStream_t stream,
+                             std::string *err) {
   using namespace gdr;
   switch (p.variant) {
-    case kDeltaNet: return tc::launch_split<kDeltaNet>(p, ws, stream, err);
-    case kGatedDeltaNet: return tc::launch_split<kGatedDeltaNet>(p, ws, stream, err);
-    case kKLA: return tc::launch_split<kKLA>(p, ws, stream, err);
-    case kKDA: return tc::launch_split<kKDA>(p, ws, stream, err);
-    case kGDN2: return tc::launch_split<kGDN2>(p, ws, stream, err);
+    case kDeltaNet: return tc::launch_split<kDeltaNet>(p, ws, ws_bytes, stream, err);
+    case kGatedDeltaNet: return tc::launch_split<kGatedDeltaNet>(p, ws, ws_bytes, stream, err);
+    case kKLA: return tc::launch_split<kKLA>(p, ws, ws_bytes, stream, err);
+    case kKDA: return tc::launch_split<kKDA>(p, ws, ws_bytes, stream, err);
+    case kGDN2: return tc::launch_split<kGDN2>(p, ws, ws_bytes, stream, err);
     default: *err = "variant not covered: "; return cudaErrorInvalidValue;
   }
 }

@@ -19,11 +19,14 @@ int gdr_read_chan_error();
 // Two-kernel path (chunk_split.cu): chunk-parallel preparation + sequential carry.
 bool gdr_split_supported(int variant, int dk, int dv);
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv);
+size_t gdr_split_record_bytes(int variant, int dv);   // bytes of one (b, h, chunk) record
 int gdr_split_launches(int variant, int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
 // The two-kernel path's schedule on a device with `sms` SMs (no device query).
 void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,
                     int *split_chunk);
-cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, cudaStream_t stream, std::string *err);
+// ws_bytes: the workspace at ws; a segmented plan that needs more runs unsegmented.
+cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, size_t ws_bytes, cudaStream_t stream,
+                             std::string *err);
 int gdr_read_split_error();
 // Fixed scratch of the no-allocation entry point (chunk_split.cu).
 size_t gdr_split_fixed_scratch_bytes();

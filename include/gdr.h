@@ -32,6 +32,9 @@
  * b_t = w_t = beta_t, as the page states it must.
  *
  * Conventions for every entry point:
+ *  - `variant`, `dtype` and the returned status are plain ints carrying the
+ *    values of gdr_variant_t, gdr_dtype_t and gdr_status_t below, so that the
+ *    ABI is the same for C callers and for foreign-function bindings.
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
  *    allocates no device memory, keeps no pointer after the call returns and
  *    never synchronises: work is enqueued on `stream` (a cudaStream_t passed as
@@ -160,26 +163,36 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
  *
  * The fixed scratch is a 32 MiB device array in the library's device image:
  * every GPU that loads the library holds it until the process exits.  A call
- * needs B * H * ceil(T / 64) records of the size gdr_forward_workspace_size
- * implies, so B * H * ceil(T / 64) may be at most 32 MiB over the record
- * size: 455 at dv = 128 (511 at dv = 64) for DeltaNet, Gated DeltaNet and
- * KLA, 451 (508) for KDA, 271 (370) for GDN-2.  Larger problems return
- * GDR_ERR_UNSUPPORTED with the limit in gdr_last_error().
- * The first call on each device looks up the array's device address (and may
- * load the library's device code); make that first call before any stream
- * capture.  All calls share the array and each call rewrites what it uses
- * before reading it, so nothing needs clearing; calls whose execution
- * overlaps on the GPU (different streams, or different host threads) race on
- * the array and must be serialised by the caller.
+ * needs B * H * ceil(T / 64) records (one per sequence, head and 64-token
+ * chunk), and they must fit in the array: at most 32 MiB / record bytes,
+ * i.e. 455 records at dv = 128 (511 at dv = 64) for DeltaNet, Gated DeltaNet
+ * and KLA, 451 (508) for KDA, 271 (370) for GDN-2.  Larger problems return
+ * GDR_ERR_UNSUPPORTED with the needed and available bytes and that limit in
+ * gdr_last_error().  For few long sequences gdr_forward_chunked runs the
+ * carry in segments, whose maps need room beside the records; where that room
+ * is not left in the array, this call runs the unsegmented sweep instead (the
+ * same results, a longer sequential carry).
+ * The array's device address is looked up for the CURRENT device, so the
+ * current device must be the device that owns `stream`.  The first call on
+ * each device does that lookup (and may load the library's device code);
+ * make that first call before any stream capture.  All calls share the array
+ * and each call rewrites what it uses before reading it, so nothing needs
+ * clearing; calls whose execution overlaps on the GPU (different streams, or
+ * different host threads) race on the array and must be serialised by the
+ * caller.
  */
 gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                          const gdr_fwd_args_t *args, float eps, float scale, void *stream);
 
 /*
- * One recurrent decode token for N independent sequences and H heads.
+ * One recurrent decode token for N independent sequences and H heads: the
+ * same per-token update as the forward ("Kaczmarz Linear Attention", KLA
+ * update rule: decay, residual at the key, erase and write; the GDN-2 form
+ * read as in the top comment), applied once to a state kept in device memory.
  * q, k [N,H,dk]; v, o [N,H,dv] (I/O dtype); beta [N,H]; log_g [N,H] or
  * [N,H,dk]; erase_b, write_w [N,H,dk]; state [N,H,dk,dv] fp32, read and
- * updated in place.  Gate roles as in gdr_fwd_args_t.
+ * updated in place.  Gate roles as in gdr_fwd_args_t.  One kernel launch;
+ * no workspace; validation and errors as for the forward.
  */
 gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv,
                              const void *q, const void *k, const void *v,
