@@ -1,0 +1,197 @@
+"""GPU parity on the method's own special cases, through every CUDA path.
+
+The seeded recipe of ``inputs.py`` draws well-conditioned inputs.  The cases
+below are the ones the pages single out, where the per-token recurrence has
+a known special behaviour, and where the chunked kernels' triangular solve,
+tf32 Gram operands and fp16 carry operands are stressed:
+
+* KLA with eta = 1, eps = 0 and q = k: each update is the exact projection
+  onto S^T k_t = v_t, so o_t = v_t ("Kaczmarz Linear Attention", theoretical
+  derivation and key properties);
+* KLA keys whose norms spread over three decades (the Kaczmarz step
+  eta / (||k||^2 + eps) then spans six), with and without the exact projection;
+* beta = 0, and GDN-2 with b = w = 0: the state only decays (a slow decay,
+  e^-0.035 per token on average, so that the decayed state stays inside fp32's
+  range); GDN-2 with only one of its two gates zero (write without erase,
+  erase without write);
+* one-hot keys and queries with beta = 1: the delta rule becomes a key ->
+  value table (DeltaNet; Gated DeltaNet with its decay on top);
+* strong decay: a scalar decay of up to e^-5 per token, and a channel-wise
+  decay at the chunked kernels' guard (e^-2.5 per token in every channel,
+  a span of 2^115 within one 64-token chunk around its middle token); beyond
+  the guard (e^-5 per token) the chunked kernels must report GDR_ERR_RANGE,
+  and the per-token kernel must still match.
+
+Every case runs chunk = 0 (automatic), 1 (per-token), 64 (one-kernel chunked,
+where it exists), 65 (two-kernel chunked) and the decode kernel (token by
+token from the same initial state), at T in {1, 63, 64, 65, 200}, and is
+compared element by element with the fp64 oracle under the tolerances of
+tests/parity_util.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_forward_b200 as gdr
+import oracle
+from gated_delta_rule_forward_b200.inputs import make_inputs, random_state
+from parity_util import assert_close, gate_kwargs, select, to_dev
+
+pytestmark = pytest.mark.gpu
+TS = [1, 63, 64, 65, 200]
+PATHS = [0, 1, 64, 65, "decode"]
+B, H = 2, 2
+
+
+def _gen(seed):
+    return torch.Generator().manual_seed(10_000 + int(seed))
+
+
+def case_inputs(case, T, seed=0):
+    """(variant, inputs dict (CPU), eps) for one special case."""
+    eps = 1e-6
+    if case == "kla_projection":                  # eta = 1, eps = 0, q = k
+        v = "kla"
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        d["beta"] = torch.ones_like(d["beta"])
+        d["q"] = d["k"].clone()
+        eps = 0.0
+    elif case in ("kla_key_decades", "kla_projection_decades"):
+        v = "kla"
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        norm = 10.0 ** (3.0 * torch.rand(B, T, H, generator=_gen(seed)) - 1.5)
+        k = d["k"].float()
+        k = k / k.norm(dim=-1, keepdim=True) * norm[..., None]
+        d["k"] = k.to(torch.bfloat16).contiguous()
+        if case == "kla_projection_decades":
+            d["beta"] = torch.ones_like(d["beta"])
+            d["q"] = d["k"].clone()
+            eps = 0.0
+    elif case in ("deltanet_beta0", "gdn_beta0", "kda_beta0", "kla_beta0"):
+        v = case.split("_")[0]
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        d["beta"] = torch.zeros_like(d["beta"])
+        if d["log_g"] is not None:                # a slow decay: S stays inside fp32's range
+            d["log_g"] = (0.05 * d["log_g"]).contiguous()
+    elif case in ("gdn2_b0_w0", "gdn2_b0", "gdn2_w0"):
+        v = "gdn2"
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        if case in ("gdn2_b0_w0", "gdn2_b0"):
+            d["erase_b"] = torch.zeros_like(d["erase_b"])
+        if case in ("gdn2_b0_w0", "gdn2_w0"):
+            d["write_w"] = torch.zeros_like(d["write_w"])
+        d["log_g"] = (0.05 * d["log_g"]).contiguous()
+    elif case in ("deltanet_one_hot", "gdn_one_hot"):
+        v = case.split("_")[0]
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        g = _gen(seed)
+        dk = d["k"].shape[-1]
+        jk = torch.randint(0, 16, (B, T, H), generator=g)      # 16 slots: keys repeat often
+        jq = torch.randint(0, 16, (B, T, H), generator=g)
+        d["k"] = torch.nn.functional.one_hot(jk, dk).to(torch.bfloat16).contiguous()
+        d["q"] = torch.nn.functional.one_hot(jq, dk).to(torch.bfloat16).contiguous()
+        d["beta"] = torch.ones_like(d["beta"])
+    elif case == "gdn_strong_decay":               # log alpha in [-5, 0]
+        v = "gdn"
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        d["log_g"] = (-5.0 * torch.rand(B, T, H, generator=_gen(seed))).contiguous()
+    elif case in ("kda_decay_at_guard", "gdn2_decay_at_guard"):
+        v = case.split("_")[0]
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        d["log_g"] = torch.full_like(d["log_g"], -2.5)
+    elif case in ("kda_decay_mixed", "gdn2_decay_mixed"):   # channels from e^-2.5 to 1 per token
+        v = case.split("_")[0]
+        d = make_inputs(v, B, T, H, dtype=torch.bfloat16, seed=seed)
+        d["log_g"] = (-2.5 * torch.rand(d["log_g"].shape, generator=_gen(seed))).contiguous()
+    else:
+        raise ValueError(case)
+    return v, d, eps
+
+
+CASES = ["kla_projection", "kla_key_decades", "kla_projection_decades",
+         "deltanet_beta0", "gdn_beta0", "kda_beta0", "kla_beta0",
+         "gdn2_b0_w0", "gdn2_b0", "gdn2_w0",
+         "deltanet_one_hot", "gdn_one_hot",
+         "gdn_strong_decay", "kda_decay_at_guard", "gdn2_decay_at_guard",
+         "kda_decay_mixed", "gdn2_decay_mixed"]
+
+
+def run_path(variant, d, S0, eps, path):
+    dd = to_dev(d)
+    if path == "decode":
+        state = S0.cuda().clone()
+        outs = []
+        for t in range(d["q"].shape[1]):
+            s = select(dd, t=t)
+            outs.append(gdr.decode_step(s["q"], s["k"], s["v"], state, variant=variant, eps=eps,
+                                        **gate_kwargs(s)))
+        torch.cuda.synchronize()
+        return torch.stack(outs, 1), state
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant=variant, **gate_kwargs(dd), eps=eps,
+                       initial_state=S0.cuda(), chunk=path)
+    torch.cuda.synchronize()
+    return o, S
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T", TS)
+@pytest.mark.parametrize("case", CASES)
+def test_special_case_against_oracle(case, T, path):
+    variant, d, eps = case_inputs(case, T, seed=T)
+    if path != "decode" and gdr.forward_kernel_name(variant, torch.bfloat16, B, T, H, 128, 128, path) == "none":
+        pytest.skip(f"chunk={path} has no kernel for {variant}")
+    S0 = random_state(B, H, 128, 128, 7 + T)
+    gdr.device_status()                           # no stale device-side flag
+    o, S = run_path(variant, d, S0, eps, path)
+    gdr.device_status()                           # no range or timeout fault in these cases
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=S0, eps=eps)
+    assert_close(o, o_ref, torch.bfloat16, f"{case} T={T} chunk={path} o")
+    assert_close(S, S_ref, torch.bfloat16, f"{case} T={T} chunk={path} S")
+    if case.startswith("kla_projection"):
+        # the exact projection reads back the value just written: o_t = v_t
+        assert_close(o, d["v"].double().numpy(), torch.bfloat16, f"{case} o = v")
+
+
+@pytest.mark.parametrize("T", [64, 200])
+@pytest.mark.parametrize("variant", ["kda", "gdn2"])
+def test_decay_beyond_the_guard_is_reported(variant, T):
+    """A channel-wise decay of e^-5 per token spans 2^230 within one chunk: the
+    chunked kernels cannot factor it in fp32 and must say so (GDR_ERR_RANGE,
+    after returning normally), and the per-token kernel still matches the oracle."""
+    d = make_inputs(variant, B, T, H, dtype=torch.bfloat16, seed=T)
+    d["log_g"] = torch.full_like(d["log_g"], -5.0)
+    S0 = random_state(B, H, 128, 128, 3)
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=S0)
+    gdr.device_status()
+    for path in (64, 65):
+        if gdr.forward_kernel_name(variant, torch.bfloat16, B, T, H, 128, 128, path) == "none":
+            continue
+        run_path(variant, d, S0, 1e-6, path)
+        with pytest.raises(gdr.GdrError) as e:
+            gdr.device_status()
+        assert e.value.status == 6, str(e.value)
+    o, S = run_path(variant, d, S0, 1e-6, 1)
+    gdr.device_status()
+    assert_close(o, o_ref, torch.bfloat16, "per-token o")
+    assert_close(S, S_ref, torch.bfloat16, "per-token S")
+
+
+def test_one_hot_table_readout():
+    """DeltaNet, one-hot keys, beta = 1, S0 = 0: the state is the table of the
+    last value written at each key, so a one-hot query e_j reads that value."""
+    T = 200
+    _, d, _ = case_inputs("deltanet_one_hot", T, seed=5)
+    dd = to_dev(d)
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant="deltanet", beta=dd["beta"])
+    torch.cuda.synchronize()
+    jk = d["k"].float().argmax(-1).numpy()
+    jq = d["q"].float().argmax(-1).numpy()
+    v = d["v"].float().numpy()
+    o = o.float().cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            last = {}
+            for t in range(T):
+                last[jk[b, t, h]] = v[b, t, h]
+                want = last.get(jq[b, t, h], np.zeros_like(v[b, t, h]))
+                np.testing.assert_allclose(o[b, t, h], want, rtol=2 ** -7, atol=1e-6)

@@ -279,3 +279,34 @@ def test_decode_head_dims(dkdv):
     o_ref, S_ref = oracle.decode_step("gdn2", d["q"], d["k"], d["v"], S0, **gate_kwargs(d))
     assert_close(o, o_ref, torch.bfloat16, "o")
     assert_close(state, S_ref, torch.bfloat16, "state")
+
+
+# ----------------------------------------------------------------- CLVR value routing
+@pytest.mark.parametrize("routing", ["target", "mixed", "output"])
+@pytest.mark.parametrize("variant", ["gdn", "deltanet"])
+def test_cross_layer_value_routing(variant, routing):
+    """Cross-layer value routing ("Linear Attention Architectures", the CLVR part):
+    a lower layer hands its write target to a higher layer, which writes it in
+    place of (or mixed with) its own value.  Only the value input changes, so the
+    kernels take the routed tensor as v: here the upper layer's v is the lower
+    layer's v ("target"), the mean of both ("mixed"), or the lower layer's output
+    ("output", the routed tensor produced on the GPU by the call before), and the
+    upper call is compared with the oracle fed the same routed values."""
+    B, T, H = 2, 333, 3
+    lower = make_inputs(variant, B, T, H, dtype=torch.bfloat16, seed=51)
+    upper = make_inputs(variant, B, T, H, dtype=torch.bfloat16, seed=52)
+    dl, du = to_dev(lower), to_dev(upper)
+    o_low, _ = gdr.forward(dl["q"], dl["k"], dl["v"], variant=variant, **gate_kwargs(dl))
+    if routing == "target":
+        v_routed = dl["v"]
+    elif routing == "mixed":
+        v_routed = (0.5 * (dl["v"].float() + du["v"].float())).to(torch.bfloat16).contiguous()
+    else:
+        v_routed = o_low
+    o, S = gdr.forward(du["q"], du["k"], v_routed, variant=variant, **gate_kwargs(du))
+    torch.cuda.synchronize()
+    ref_in = dict(upper)
+    ref_in["v"] = v_routed.cpu()
+    o_ref, S_ref = oracle.forward(variant, **ref_in)
+    assert_close(o, o_ref, torch.bfloat16, f"{routing} o")
+    assert_close(S, S_ref, torch.bfloat16, f"{routing} S")

@@ -3,7 +3,8 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import BF16_TOL, F32_TOL, assert_close, bf16_out_rel, elem_rel, max_rel, rms_rel
+from parity_util import (BF16_TOL, BULK_RMS, BULK_TOL, F32_TOL, assert_close, bf16_out_rel, bulk_rel, elem_rel,
+                          max_rel, rms_rel)
 
 
 def test_metrics_on_known_arrays():
@@ -28,3 +29,20 @@ def test_fp32_bar_fails_with_both_ratios_in_the_message():
     with pytest.raises(AssertionError, match="element-wise"):
         assert_close(gpu, ref, torch.float32, "o")
     assert F32_TOL == 1e-4 and BF16_TOL == 2e-2
+
+
+def test_bulk_metric_catches_an_error_the_rounding_allowance_forgives():
+    # a heavy tail (one element at 50 RMS) and an arithmetic error of 0.1 RMS on a bulk element
+    rng = np.random.default_rng(0)
+    ref = rng.standard_normal(4096)
+    ref[0] = 50.0 * np.sqrt(np.mean(ref * ref))
+    rms = np.sqrt(np.mean(ref * ref))
+    bad = ref.copy()
+    bad[1] = ref[1] + 0.1 * rms                        # |ref[1]| is well inside 4 RMS
+    bad_t = torch.from_numpy(bad).to(torch.bfloat16)
+    assert bulk_rel(bad_t, ref) > BULK_TOL
+    with pytest.raises(AssertionError):
+        assert_close(bad_t, ref, torch.bfloat16, "o")
+    # the exact result rounded to bf16 passes both metrics
+    ok = torch.from_numpy(ref).to(torch.bfloat16)
+    assert bulk_rel(ok, ref) <= BULK_RMS * 2 ** -8 + 1e-12
