@@ -54,8 +54,7 @@ METRIC = "gated-delta-rule layer tokens/s (fwd, decode) at 1 B200; % of bf16 TC 
 _CSRC = "gated_delta_rule_forward_b200/csrc/"
 _TC = [_CSRC + f for f in ("chunk_common.cuh", "tc_util.cuh", "tma_host.cuh")]
 KERNEL_SOURCES = {   # sources whose text keys a recorded ncu traffic figure
-    "chunk64_split": [_CSRC + "chunk_split.cu"] + _TC,
-    "chunk64_tc": [_CSRC + "chunk_tc.cu", _CSRC + "chunk_tc_chan.cu"] + _TC,
+    "chunk64_split": [_CSRC + "chunk_split.cu", _CSRC + "chunk_split.cuh"] + _TC,
     "token_bf16io": [_CSRC + "token_fwd.cu"],
     "token_f32io": [_CSRC + "token_fwd.cu"],
     "decode": [_CSRC + "decode.cu"],

@@ -8,7 +8,7 @@
 
 #include "common.cuh"
 #include "gdr.h"
-#include "chunk_tc.cuh"
+#include "chunk_split.cuh"
 
 namespace {
 
@@ -34,7 +34,7 @@ gdr_status_t check_cuda(cudaError_t e, const char *what) {
 bool valid_variant(int v) { return v >= GDR_DELTANET && v <= GDR_KLA; }
 bool valid_dim(int d) { return d == 64 || d == 128; }
 
-enum class Kernel { None, Token, ChunkTC, Split };
+enum class Kernel { None, Token, Split };
 
 bool split_ok(int variant, int dtype, int dk, int dv) {
   return dtype == GDR_BF16 && gdr_split_supported(variant, dk, dv);
@@ -42,28 +42,18 @@ bool split_ok(int variant, int dtype, int dk, int dv) {
 
 // Which kernel a forward call runs, or None with a status and reason.  `ws`
 // is the workspace the caller passes; the automatic choice takes the
-// two-kernel path only when the workspace is large enough for it.
+// chunked path only when the workspace is large enough for it.
 Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk, size_t ws,
                       gdr_status_t *st, std::string *why) {
   *st = GDR_OK;
-  const bool tc = dtype == GDR_BF16 && gdr_chunk_tc_supported(variant, dk, dv);
   const bool sp = split_ok(variant, dtype, dk, dv);
   const size_t need = sp ? gdr_split_workspace_bytes(variant, B, T, H, dv) : 0;
   if (chunk == 1) return Kernel::Token;
-  if (chunk == 0) {
-    if (sp && ws >= need) return Kernel::Split;
-    return tc ? Kernel::ChunkTC : Kernel::Token;
-  }
-  if (chunk == 64) {
-    if (tc) return Kernel::ChunkTC;
-    *st = GDR_ERR_UNSUPPORTED;
-    *why = "chunk=64 tensor-core kernel needs bf16 I/O and a supported (variant, dk, dv)";
-    return Kernel::None;
-  }
+  if (chunk == 0) return (sp && ws >= need) ? Kernel::Split : Kernel::Token;
   if (chunk == 65) {
     if (!sp) {
       *st = GDR_ERR_UNSUPPORTED;
-      *why = "chunk=65 two-kernel path needs bf16 I/O and dk = 128";
+      *why = "chunk=65 (the chunked path) needs bf16 I/O and dk = 128";
       return Kernel::None;
     }
     if (ws < need) {
@@ -73,8 +63,13 @@ Kernel select_forward(int variant, int dtype, int B, int T, int H, int dk, int d
     }
     return Kernel::Split;
   }
+  if (chunk == 64) {
+    *st = GDR_ERR_UNSUPPORTED;
+    *why = "chunk=64 (a one-kernel chunked path without workspace) is not built; use 0 (auto) or 65";
+    return Kernel::None;
+  }
   *st = GDR_ERR_INVALID_ARG;
-  *why = "chunk must be 0 (auto), 1 (per-token), 64 (chunked, one kernel) or 65 (chunked, two kernels)";
+  *why = "chunk must be 0 (auto), 1 (per-token) or 65 (chunked)";
   return Kernel::None;
 }
 
@@ -148,14 +143,13 @@ int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, in
   if ((long)B * H == 0) return 0;
   if (T == 0) return 1;  // state copy or clear
   if (kern == Kernel::Split) return gdr_split_launches(variant, B, T, H, dv);
-  return kern == Kernel::ChunkTC ? gdr_chunk_tc_launches(B, T, H, dk, dv) : 1;
+  return 1;
 }
 
 const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
   if (gdr_forward_launches(variant, dtype, B, T, H, dk, dv, chunk) == 0 && (long)B * H * T != 0) return "none";
   const Kernel kern = planned_kernel(variant, dtype, B, T, H, dk, dv, chunk);
   if (kern == Kernel::Split) return "chunk64_split";
-  if (kern == Kernel::ChunkTC) return "chunk64_tc";
   if (kern == Kernel::Token) return dtype == GDR_BF16 ? "token_bf16io" : "token_f32io";
   return "none";
 }
@@ -219,12 +213,6 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
     std::string err;
     const cudaError_t e = gdr_launch_split(p, workspace, workspace_bytes, s, &err);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_split: " + err + cudaGetErrorString(e));
-    return GDR_OK;
-  }
-  if (kern == Kernel::ChunkTC) {
-    std::string err;
-    const cudaError_t e = gdr_launch_chunk_tc(p, s, &err);
-    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_tc: " + err + cudaGetErrorString(e));
     return GDR_OK;
   }
   return check_cuda(gdr_launch_token_forward(p, s), "token_fwd launch");

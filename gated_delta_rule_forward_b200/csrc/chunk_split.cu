@@ -3,7 +3,7 @@
 // sequential carry kernel, with the per-chunk products passed through a
 // workspace.
 //
-// The chunk algebra is the one of chunk_tc.cu ("Kaczmarz Linear Attention",
+// The chunk algebra ("Kaczmarz Linear Attention",
 // KLA update rule and implementation; "Gated DeltaNet-2", technical core):
 //     T = (I + A)^{-1},  W = T Diag(Gamma) K,  U' = T V,  E = U' - W S0
 //     O = Diag(scale Gamma) Q S0 + P E,   S_C = Gamma_C S0 + K^T Diag(w) E.
@@ -52,7 +52,7 @@
 #include <mutex>
 
 #include "chunk_common.cuh"
-#include "chunk_tc.cuh"
+#include "chunk_split.cuh"
 #include "tc_util.cuh"
 #include "tma_host.cuh"
 
@@ -2100,8 +2100,9 @@ cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, size_t ws_bytes
   }
 }
 
-int gdr_read_split_error() {
+int gdr_read_device_error(cudaStream_t stream) {
   int h = 0, zero = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
   if (cudaMemcpyFromSymbol(&h, g_gdr_split_error, sizeof(int)) != cudaSuccess) return -1;
   if (h) cudaMemcpyToSymbol(g_gdr_split_error, &zero, sizeof(int));
   return h;

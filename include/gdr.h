@@ -100,7 +100,7 @@ typedef struct {
 
 /*
  * Bytes of device workspace gdr_forward_chunked uses for this problem and
- * `chunk` choice: for the two-kernel chunked path (chunk 0 or 65 with bf16
+ * `chunk` choice: for the chunked path (chunk 0 or 65 with bf16
  * I/O and dk = 128) B * H * ceil(T/64) records of 56 KB + 8 KB per 64 value
  * columns, plus 16 bytes (scalar decay: DeltaNet, Gated DeltaNet, KLA) or
  * 512 bytes (channel decay: KDA), plus 24 KB per 64 value columns for GDN-2;
@@ -117,26 +117,25 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
 /*
  * Whole-sequence forward of B sequences of T tokens and H heads.
  *
- * chunk selects the algorithm (all chunked paths use C = 64 tokens per chunk
- * and tcgen05 tensor cores with TMEM accumulators fed by TMA):
- *   0  automatic: the two-kernel chunked path when it covers the case and the
- *      workspace is at least gdr_forward_workspace_size() bytes, else the
- *      one-kernel chunked path where it exists, else the per-token kernel;
+ * chunk selects the algorithm:
+ *   0  automatic: the chunked path when it covers the case and the workspace
+ *      is at least gdr_forward_workspace_size() bytes, else the per-token
+ *      kernel;
  *   1  the per-token kernel (fp32 state in registers, exact fp32 arithmetic,
  *      any supported shape; the path used for fp32 I/O);
- *   64 the one-kernel chunked path (each CTA prepares and carries its chunks;
- *      no workspace): DeltaNet, Gated DeltaNet, KLA and KDA with bf16 I/O,
- *      dk = 128;
- *   65 the two-kernel chunked path: a chunk-parallel preparation kernel (the
+ *   65 the chunked path (C = 64 tokens per chunk, tcgen05 tensor cores with
+ *      TMEM accumulators fed by TMA): a chunk-parallel preparation kernel (the
  *      S-independent products of every chunk, into the workspace) then the
  *      sequential carry kernel: all five variants with bf16 I/O and dk = 128;
  *      needs the workspace.  Where the carry's B * H CTAs leave SMs idle it
  *      reschedules: for few long sequences, segment maps, a chain of segment
- *      start states, then the segments in parallel; for a mid-size B * H
- *      (DeltaNet, Gated DeltaNet, KLA, KDA), the sweep cut in two, with the
- *      second part's preparation beside the first part's carry.  Its kernels
- *      are chained on `stream` by programmatic dependent launch; the call
- *      returns after enqueueing them, like every other path.
+ *      start states, then the segments in parallel; for a mid-size B * H,
+ *      the sweep cut in two, with the second part's preparation beside the
+ *      first part's carry.  Its kernels are chained on `stream` by
+ *      programmatic dependent launch; the call returns after enqueueing them,
+ *      like every other path.
+ *   64 is reserved (a one-kernel chunked path without workspace, not built:
+ *      GDR_ERR_UNSUPPORTED).
  * A chunk value whose path does not cover the case returns GDR_ERR_UNSUPPORTED.
  * Shapes: B, T, H >= 0; dk in {64, 128}; dv in {64, 128}.  T = 0 copies
  * initial_state to final_state (or clears it); B * H = 0 does nothing.
@@ -151,7 +150,7 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
  * Forward for callers that cannot allocate device memory at call time: a
  * serving runtime whose device memory is planned up front and that forbids
  * allocation on its request path, or a host program that drives this
- * library without a device allocator of its own.  It runs the two-kernel
+ * library without a device allocator of its own.  It runs the
  * chunked path (chunk = 65 of gdr_forward_chunked) with the library's own
  * fixed scratch instead of a caller workspace, and allocates nothing.  The
  * pages have no counterpart to this entry point; it is a deployment
@@ -203,8 +202,8 @@ gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int d
 /*
  * Kernel launches one gdr_forward_chunked call with these arguments makes
  * (0 if the call would be rejected), and a short name of the kernel that runs
- * ("chunk64_split", "chunk64_tc", "token_f32io", "token_bf16io", ...).
- * Host-only, no GPU work.  The two-kernel path makes 2 launches, or 4 when
+ * ("chunk64_split", "token_f32io", "token_bf16io", or "none").
+ * Host-only, no GPU work.  The chunked path makes 2 launches, or 4 when
  * it reschedules (segmented or pipelined sweep); that choice reads the
  * current device's SM count, and with no device present it is always 2.
  */
@@ -213,7 +212,7 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
                                     int chunk);
 
 /*
- * How the two-kernel chunked path schedules B sequences of T tokens and H
+ * How the chunked path schedules B sequences of T tokens and H
  * heads on a device with `sms` SMs (host-only; no device is queried, so it
  * serves to inspect a plan for any device).  Writes
  *   *segments        the carry's segments per sequence (1: not segmented),

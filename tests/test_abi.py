@@ -115,8 +115,10 @@ def test_chunk_selection(L):
         for dt in (0, 1):
             assert L.gdr_forward_kernel_name(v, dt, 2, 100, 2, 64, 128, 1).decode().startswith("token")
             assert L.gdr_forward_launches(v, dt, 2, 100, 2, 64, 128, 1) == 1
-    # fp32 I/O never takes the tensor-core kernel
-    assert fwd(L, dtype=0, chunk=64) == 2
+    # fp32 I/O never takes the tensor-core kernel; chunk=64 (a one-kernel path) is not built
+    assert fwd(L, dtype=0, chunk=65) == 2
+    assert fwd(L, chunk=64) == 2
+    assert L.gdr_forward_kernel_name(1, 1, 8, 2048, 8, 128, 128, 64).decode() == "none"
     assert L.gdr_forward_kernel_name(1, 0, 8, 2048, 8, 128, 128, 0).decode() == "token_f32io"
     assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 7) == 0
 
@@ -145,7 +147,7 @@ def test_workspace_sizes(L):
     # P (8 KB), U'^T (8 KB per 64 value columns) and Gamma_C (16 bytes)
     assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 16)
     assert L.gdr_forward_workspace_size(1, 1, 2, 65, 3, 128, 64, 65) == 2 * 3 * 2 * (57344 + 8192 + 16)
-    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 64) == 0   # one-kernel path
+    assert L.gdr_forward_workspace_size(1, 1, 8, 2048, 8, 128, 128, 64) == 0   # not built
     assert L.gdr_forward_workspace_size(1, 0, 8, 2048, 8, 128, 128, 0) == 0    # fp32: per-token
     # KDA: the same record with Gamma_C a vector of 128 floats
     assert L.gdr_forward_workspace_size(2, 1, 8, 2048, 8, 128, 128, 0) == 8 * 8 * 32 * (57344 + 16384 + 512)
@@ -157,7 +159,6 @@ def test_workspace_sizes(L):
     # sweep (two of each) -- without one, as here, the serial pair
     assert L.gdr_forward_launches(1, 1, 8, 2048, 8, 128, 128, 0) == (4 if torch.cuda.is_available() else 2)
     assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 0).decode() == "chunk64_split"
-    assert L.gdr_forward_kernel_name(2, 1, 8, 2048, 8, 128, 128, 64).decode() == "chunk64_tc"
 
 
 def test_split_needs_workspace(L):
