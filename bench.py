@@ -6,11 +6,14 @@
 
 A step is one pass of the layer over one batch of synthetic input (seeded,
 recipe in gated_delta_rule_forward_b200/inputs.py).  The headline workload is
-the 350M-model layer shape: Gated DeltaNet forward, bf16 q/k/v/o, fp32 state,
-B=8 T=2048 H=8 dk=dv=128.  The line also carries the other workloads
-("also": DeltaNet on the same shape, KDA / KLA / GDN-2 at the 1.3B-model
-shape, the 65536-token forward and the 256 x 16 decode step), each with its
-own roofline.
+the largest single-GPU one, the long-context forward: Gated DeltaNet, bf16
+q/k/v/o, fp32 state, B=1 T=65536 H=16 dk=dv=128.  The line also carries the
+other workloads ("also": KLA on the same shape, the 350M-model layer (GDN and
+DeltaNet, B=8 T=2048 H=8), KDA / KLA / GDN-2 at the 1.3B-model shape, and
+the decode of 256 sequences x 16 heads: 1024 seeded steps from the
+long-context forward's final state, broadcast), each with its own roofline:
+achieved HBM bandwidth of the algorithmic bytes, and for the forwards also
+the tensor-core rate of the chunked algorithm's flops.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronisation on each side, CUDA events on the launching stream, max
@@ -49,7 +52,10 @@ WORKLOADS = {
     "kla_fwd_64k": ("kla", 1, 65536, 16, 128, 128),
     "gdn_decode_256x16": ("gdn", 256, None, 16, 128, 128),
 }
-DEFAULT = "gdn_fwd_350m"
+DEFAULT = "gdn_fwd_64k"
+DECODE_STEPS = 1024         # the decode chain after the long-context prefill
+DECODE_PREFILL = "gdn_fwd_64k"
+ORACLE_SAMPLE_TOKENS = 4096  # the oracle's timed sample of a long forward: its first tokens, every head
 METRIC = "gated-delta-rule layer tokens/s (fwd, decode) at 1 B200; % of bf16 TC / HBM roofline"
 _CSRC = "gated_delta_rule_forward_b200/csrc/"
 _TC = [_CSRC + f for f in ("chunk_common.cuh", "tc_util.cuh", "tma_host.cuh")]
@@ -119,6 +125,17 @@ def fwd_bytes(variant, B, T, H, dk, dv, io_bytes=2):
         b += 2 * th * dk * 4                           # erase and write gates
     b += B * H * dk * dv * 4                           # final state
     return b
+
+
+def fwd_flops(variant, B, T, H, dk, dv, C=64):
+    """Flops of the chunked algorithm per forward call (the tensor-core rate's
+    numerator): per token-head 2 C dk (K K^T) + 2 C dk (Q K^T) + 2 C dk (W) +
+    2 C dv (U') + 2 dk dv (W S) + 2 dk dv (Q S) + 2 C dv (P E) + 2 dk dv (K~^T E)
+    = 10 C d + 6 d^2 at dk = dv = d; GDN-2 adds the second Gram pair, R, and the
+    two state-free terms: 18 C d + 8 d^2."""
+    d = dk
+    per = (18 * C * d + 8 * d * d) if variant == "gdn2" else (10 * C * d + 6 * d * d)
+    return B * T * H * per
 
 
 def decode_bytes(variant, N, H, dk, dv, io_bytes=2):
@@ -259,7 +276,7 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
         "workload": name, "variant": variant, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
         "kernel": kernel, "launches_per_step": launches, "ms_per_step": total_ms / K,
         "launch_ms": launch_ms, "tokens_per_step": B * T, "wall": (t_wall0, t_wall1),
-        "alg_bytes": fwd_bytes(variant, B, T, H, dk, dv),
+        "alg_bytes": fwd_bytes(variant, B, T, H, dk, dv), "alg_flops": fwd_flops(variant, B, T, H, dk, dv),
     }
     res["value"] = job_throughput(B * T, K, total_ms, world)
     if e2e:
@@ -267,9 +284,9 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
     return res
 
 
-def streamed_e2e(pinned_sets, out_shape, call, K, W, world):
+def streamed_e2e(pinned_sets, out_specs, call, K, W, world):
     """K steps of (H2D of the step's inputs from pinned host memory, `call`, D2H
-    of its output into pinned host memory), double-buffered over three streams:
+    of its outputs into pinned host memory), double-buffered over three streams:
     step i+1's copy-in and step i-1's copy-out run while step i computes, as a
     stream of batches is served.  Every step's own copies are inside the timed
     region.  Returns the milliseconds of the K steps (max over ranks)."""
@@ -290,8 +307,8 @@ def streamed_e2e(pinned_sets, out_shape, call, K, W, world):
     bufs = [torch.empty(off, dtype=torch.uint8, device="cuda") for _ in range(2)]
     dev = [{k: bufs[j][o:o + torch.Size(sh).numel() * torch.empty(0, dtype=dt).element_size()].view(dt).view(sh)
             for k, (o, dt, sh) in layout.items()} for j in range(2)]
-    outs = [torch.empty(out_shape, device="cuda", dtype=torch.bfloat16) for _ in range(2)]
-    hosts = [torch.empty(out_shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    outs = [[torch.empty(sh, device="cuda", dtype=dt) for sh, dt in out_specs] for _ in range(2)]
+    hosts = [[torch.empty(sh, dtype=dt).pin_memory() for sh, dt in out_specs] for _ in range(2)]
     comp = torch.cuda.current_stream()
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
     in_ready = [torch.cuda.Event() for _ in range(2)]
@@ -311,7 +328,8 @@ def streamed_e2e(pinned_sets, out_shape, call, K, W, world):
         done[j].record(comp)
         cout.wait_event(done[j])
         with torch.cuda.stream(cout):
-            hosts[j].copy_(outs[j], non_blocking=True)
+            for h, o in zip(hosts[j], outs[j]):
+                h.copy_(o, non_blocking=True)
         out_free[j].record(cout)
 
     for i in range(W):
@@ -332,7 +350,7 @@ def streamed_e2e(pinned_sets, out_shape, call, K, W, world):
     return max_over_ranks(s.elapsed_time(e), world), off
 
 
-E2E_NOTE = ("one packed H2D of the step's inputs, the call, D2H of its output; double-buffered on three "
+E2E_NOTE = ("one packed H2D of the step's inputs, the call, D2H of its outputs; double-buffered on three "
             "streams (copies of neighbouring steps overlap)")
 
 
@@ -342,37 +360,58 @@ def forward_e2e(name, host, K, W, world):
     import gated_delta_rule_forward_b200 as gdr
     variant, B, T, H, dk, dv = WORKLOADS[name]
     pinned = {k: (None if v is None else v.pin_memory()) for k, v in host.items()}
-    d2h = B * T * H * dv * 2
+    shapes = [((B, T, H, dv), torch.bfloat16), ((B, H, dk, dv), torch.float32)]
+    d2h = B * T * H * dv * 2 + B * H * dk * dv * 4
 
-    def call(d, out):
-        gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), out=out, output_final_state=False)
+    def call(d, outs):
+        gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), out=outs[0], final_state=outs[1])
 
-    ms, h2d = streamed_e2e([pinned], (B, T, H, dv), call, K, W, world)
+    ms, h2d = streamed_e2e([pinned], shapes, call, K, W, world)
     return {"value": job_throughput(B * T, K, ms, world), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K, "schedule": E2E_NOTE}
 
 
-def run_decode_workload(name, K, W, world, e2e=False):
+def prefill_state(world_seed):
+    """Final state [1, H, dk, dv] of the long-context forward (the decode's prefill)."""
     import gated_delta_rule_forward_b200 as gdr
-    from gated_delta_rule_forward_b200.inputs import make_decode_inputs, random_state
+    from gated_delta_rule_forward_b200.inputs import make_inputs
+    variant, B, T, H, dk, dv = WORKLOADS[DECODE_PREFILL]
+    d = {k: (None if v is None else v.cuda())
+         for k, v in make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=world_seed).items()}
+    _, S = gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), chunk=0)
+    torch.cuda.synchronize()
+    return S
+
+
+def run_decode_workload(name, K, W, world, e2e=False, chain=True, seed=0):
+    """Decode of N sequences x H heads.  With `chain` (the long-context protocol):
+    the state starts as the long-context forward's final state broadcast to the N
+    sequences, and DECODE_STEPS steps with inputs seeded 1000 + s are timed as one
+    chain; otherwise K steps of that chain are timed."""
+    import gated_delta_rule_forward_b200 as gdr
+    from gated_delta_rule_forward_b200.inputs import make_decode_inputs
     variant, N, _, H, dk, dv = WORKLOADS[name]
+    n_steps = DECODE_STEPS if chain else K
+    n_inputs = min(n_steps, DECODE_STEPS)
     steps = [{k: (None if v is None else v.cuda()) for k, v in
-              make_decode_inputs(variant, N, H, s, dk, dv).items()} for s in range(4)]
-    state = random_state(N, H, dk, dv, 7).cuda()
+              make_decode_inputs(variant, N, H, s, dk, dv).items()} for s in range(n_inputs)]
+    start = prefill_state(seed).expand(N, H, dk, dv).contiguous()
+    state = start.clone()
     out = torch.empty(N, H, dv, device="cuda", dtype=torch.bfloat16)
 
     def step(i):
-        d = steps[i % 4]
+        d = steps[i % n_inputs]
         gdr.decode_step(d["q"], d["k"], d["v"], state, variant=variant, **gates(d), out=out)
 
     for i in range(W):
         step(i)
+    state.copy_(start)                  # the timed chain starts from the prefill state
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
     s.record()
-    for i in range(K):
+    for i in range(n_steps):
         step(i)
     e.record()
     torch.cuda.synchronize()
@@ -380,11 +419,14 @@ def run_decode_workload(name, K, W, world, e2e=False):
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
     res = {"workload": name, "variant": variant, "N": N, "H": H, "dk": dk, "dv": dv, "kernel": "decode",
-           "launches_per_step": 1, "ms_per_step": ms / K, "launch_ms": ms / K, "tokens_per_step": N,
-           "value": job_throughput(N, K, ms, world), "alg_bytes": decode_bytes(variant, N, H, dk, dv),
-           "wall": (t_wall0, t_wall1)}
+           "launches_per_step": 1, "steps_timed": n_steps, "ms_per_step": ms / n_steps,
+           "launch_ms": ms / n_steps, "tokens_per_step": N,
+           "value": job_throughput(N, n_steps, ms, world), "alg_bytes": decode_bytes(variant, N, H, dk, dv),
+           "wall": (t_wall0, t_wall1),
+           "protocol": (f"{n_steps} steps from the {DECODE_PREFILL} final state broadcast to {N} sequences, "
+                        "inputs seeded 1000 + step")}
     if e2e:
-        res["e2e"] = decode_e2e(name, steps, state, K, W, world)
+        res["e2e"] = decode_e2e(name, steps[:16], state, K, W, world)
     return res
 
 
@@ -397,10 +439,10 @@ def decode_e2e(name, dev_steps, state, K, W, world):
     pinned = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()} for d in dev_steps]
     d2h = N * H * dv * 2
 
-    def call(d, out):
-        gdr.decode_step(d["q"], d["k"], d["v"], state, variant=variant, **gates(d), out=out)
+    def call(d, outs):
+        gdr.decode_step(d["q"], d["k"], d["v"], state, variant=variant, **gates(d), out=outs[0])
 
-    ms, h2d = streamed_e2e(pinned, (N, H, dv), call, K, W, world)
+    ms, h2d = streamed_e2e(pinned, [((N, H, dv), torch.bfloat16)], call, K, W, world)
     return {"value": job_throughput(N, K, ms, world), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K, "schedule": E2E_NOTE}
 
@@ -415,6 +457,17 @@ def roofline(res, peaks):
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
             "peak_source": peaks["source"], "alg_bytes_per_launch": res["alg_bytes"],
             "launches_timed": res["launches_per_step"]}
+
+
+def roofline_tensor(res, peaks):
+    """The chunked algorithm's flops (fwd_flops) over the call's event-timed
+    duration, against the measured dense bf16 tensor peak (the carry's fp16 and
+    the channel-decay Gram product's tf32 operands run on the same units; tf32
+    at half the bf16 rate, which this figure does not discount)."""
+    achieved = res["alg_flops"] / (res["launch_ms"] / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4), "peak_source": peaks["source"],
+            "alg_flops_per_launch": res["alg_flops"]}
 
 
 def cpu_baseline(name):
@@ -432,15 +485,17 @@ def cpu_baseline(name):
         dt = time.perf_counter() - t0
         return {"value": passes * B / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
                 "sample": f"{passes} decode step(s) of all {B} sequences x {H} heads, fp64, {dt:.2f} s wall"}
-    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+    Ts = min(T, ORACLE_SAMPLE_TOKENS)
+    d = make_inputs(variant, B, Ts, H, dk, dv, dtype=torch.bfloat16, seed=0)
     oracle.forward(variant, **{k: (None if v is None else v[:, :64]) for k, v in d.items()})  # build/load
     passes, t0 = 0, time.perf_counter()
     while passes == 0 or time.perf_counter() - t0 < 2.0:     # >= 2 s wall on all host cores
         oracle.forward(variant, **d)
         passes += 1
     dt = time.perf_counter() - t0
-    return {"value": passes * B * T / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{passes} pass(es) of the whole workload ({B} x {T} tokens x {H} heads), fp64, "
+    what = "the whole workload" if Ts == T else f"the first {Ts} of its {T} tokens"
+    return {"value": passes * B * Ts / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{passes} pass(es) of {what} ({B} sequence(s) x {Ts} tokens x {H} heads), fp64, "
                       f"{dt:.2f} s wall"}
 
 
@@ -455,7 +510,8 @@ def native(args):
     sampler.start()
     t0 = time.time()
     if WORKLOADS[args.workload][2] is None:
-        main = run_decode_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e)
+        main = run_decode_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e,
+                                   chain=False, seed=rank)
     else:
         main = run_forward_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e,
                                     seed=rank)   # each rank its own sequences
@@ -466,9 +522,11 @@ def native(args):
             if name == args.workload:
                 continue
             k = max(3, args.steps // 4) if "64k" in name else args.steps
-            r = (run_decode_workload(name, k, args.warmup, world) if WORKLOADS[name][2] is None
-                 else run_forward_workload(name, k, args.warmup, world))
+            r = (run_decode_workload(name, k, args.warmup, world, chain=True, seed=rank)
+                 if WORKLOADS[name][2] is None else run_forward_workload(name, k, args.warmup, world, seed=rank))
             r["roofline"] = roofline(r, peaks)
+            if "alg_flops" in r:
+                r["roofline_tensor"] = roofline_tensor(r, peaks)
             r["unit"] = "tokens/s"
             r.pop("wall", None)
             also.append(r)
@@ -492,6 +550,7 @@ def native(args):
                    "state": "fp32", "parallelism": f"dp{world}",
                    "l2": "inputs > L2; two input sets rotated between steps"},
         "roofline": roofline(main, peaks),
+        "roofline_tensor": roofline_tensor(main, peaks) if "alg_flops" in main else None,
         "cpu_baseline": cpu,
         "e2e": main.get("e2e"),
         "gpu_launches": main["launches_per_step"] * args.steps,
@@ -516,11 +575,13 @@ def reference(args):
         run = lambda: oracle.decode_step(variant, d["q"], d["k"], d["v"], S, **gates(d))
         tokens = B
         sample = f"one decode step of all {B} sequences x {H} heads per step, fp64"
-    else:           # forward: one of the B sequences per step
-        d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+    else:           # forward: one of the B sequences per step (its first tokens if it is long)
+        Ts = min(T, ORACLE_SAMPLE_TOKENS)
+        d = make_inputs(variant, 1, Ts, H, dk, dv, dtype=torch.bfloat16, seed=0)
         run = lambda: oracle.forward(variant, **d)
-        tokens = T
-        sample = f"1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
+        tokens = Ts
+        sample = (f"1 of {B} sequences x {T} tokens x {H} heads per step, fp64" if Ts == T else
+                  f"the first {Ts} of the {T} tokens of 1 of {B} sequence(s) x {H} heads per step, fp64")
     for _ in range(args.warmup):
         run()
     t0 = time.perf_counter()

@@ -97,8 +97,8 @@ constexpr uint32_t OFF_A = 49152;       // fp32 A^T, 64 x LD
 constexpr uint32_t OFF_TF = OFF_A + 64 * LD * 4;
 constexpr uint32_t OFF_T = 86016;       // bf16 T
 constexpr uint32_t OFF_TP = 94208;      // bf16 T Diag(Gamma)
-constexpr uint32_t OFF_SC = 102400;     // scalars: 5 x 64 floats
-constexpr uint32_t OFF_BAR = OFF_SC + 5 * 64 * 4;
+constexpr uint32_t OFF_SC = 102400;     // scalars: 6 x 64 floats
+constexpr uint32_t OFF_BAR = OFF_SC + 6 * 64 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T, "layout");
 constexpr uint32_t COL_G = 0;     // M128 x 64 (dead before W)
@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   float *sc_wf = sc_g2 + 64;
   float *sc_G = sc_wf + 64;
   float *sc_tmp = sc_G + 64;
+  float *sc_rk = sc_tmp + 64;   // 1 / ||k_t||
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
 
@@ -259,20 +260,31 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     mma_phase ^= 1;
     tc_fence_after();
 
-    // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile
+    // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile.
+    // The chunk algebra runs on unit keys: with khat_t = k_t / ||k_t||,
+    // beta'_t = beta_t ||k_t||^2 and v'_t = v_t / ||k_t||, the update
+    // S~ + beta_t k_t (v_t - S~^T k_t)^T equals S~ + beta'_t khat_t (v'_t - S~^T khat_t)^T,
+    // so the Gram entries are bounded by beta' and a spread of key norms does
+    // not amplify the fp16 rounding of U' and W S0 (E = U' - W S0 then carries
+    // v / ||k||, and K~, P absorb the other factor).  ||k_t||^2 is the diagonal
+    // of K K^T; the column coefficient c_r = beta'_r / ||k_r|| (beta_r ||k_r||, or
+    // eta_r ||k_r|| / (||k_r||^2 + eps) for KLA's Kaczmarz step) replaces beta_r.
     if (!bad) {
       float g[32];
       tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
       const int t = row & 63;
       const int r0 = 32 * half;
-      if constexpr (VAR == kKLA) {
-        if (quad < 2 && (t >> 5) == half) {
-          float kk = 0.f;
+      if (quad < 2 && (t >> 5) == half) {
+        float kk = 0.f;
 #pragma unroll
-          for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
-          const float eta = sc_beta[t];
-          sc_beta[t] = (eta == 0.f) ? 0.f : eta / (kk + p.eps);   // Kaczmarz step
-        }
+        for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
+        const float rk = kk > 0.f ? rsqrtf(kk) : 0.f;
+        const float bt = sc_beta[t];
+        float c;
+        if constexpr (VAR == kKLA) c = (bt == 0.f) ? 0.f : bt * (kk * rk) / (kk + p.eps);   // Kaczmarz step
+        else c = bt * (kk * rk);
+        sc_beta[t] = c;
+        sc_rk[t] = rk;
       }
       __syncthreads();
       const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
@@ -296,8 +308,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int r = 0; r < 32; ++r) fac[r] = sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]);
       }
       if (quad < 2) {
+        const float rkt = sc_rk[t];
 #pragma unroll
-        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(g[r] * fac[r]) : 0.f;
+        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(rkt * g[r] * fac[r]) : 0.f;
       } else {
 #pragma unroll
         for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
@@ -308,7 +321,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tc_fence_before();
     __syncthreads();
 
-    // T = (I + A)^{-1}; T and T Diag(Gamma) as bf16 tiles
+    // T = (I + A)^{-1}; T Diag(1/||k||) (for U' = T V') and T Diag(Gamma / ||k||)
+    // (for W = T Diag(Gamma) Khat) as bf16 tiles
     solve_unit_lower_64(At, Tf, tid, warp, lane);
     {
       const int m = tid >> 2, n0 = (tid & 3) * 16;
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+        tv[e] = (n0 + e <= m) ? tv[e] * sc_rk[n0 + e] : 0.f;
         tg[e] = tv[e] * sc_G[n0 + e];
       }
 #pragma unroll
