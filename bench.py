@@ -11,7 +11,9 @@ q/k/v/o, fp32 state, B=1 T=65536 H=16 dk=dv=128.  The line also carries the
 other workloads ("also": KLA on the same shape, the 350M-model layer (GDN and
 DeltaNet, B=8 T=2048 H=8), KDA / KLA / GDN-2 at the 1.3B-model shape, and
 the decode of 256 sequences x 16 heads: 1024 seeded steps from the
-long-context forward's final state, broadcast), each with its own roofline:
+long-context forward's final state, broadcast, and the 350M layer fed raw
+projections and logits, the kernels applying the input transforms), each
+with its own roofline:
 achieved HBM bandwidth of the algorithmic bytes, and for the forwards also
 the tensor-core rate of the chunked algorithm's flops.
 
@@ -51,7 +53,9 @@ WORKLOADS = {
     "gdn_fwd_64k": ("gdn", 1, 65536, 16, 128, 128),
     "kla_fwd_64k": ("kla", 1, 65536, 16, 128, 128),
     "gdn_decode_256x16": ("gdn", 256, None, 16, 128, 128),
+    "gdn_fwd_350m_raw": ("gdn", 8, 2048, 8, 128, 128),
 }
+RAW_WORKLOADS = {"gdn_fwd_350m_raw"}   # raw projections and logits in; the kernels apply the transforms
 DEFAULT = "gdn_fwd_64k"
 DECODE_STEPS = 1024         # the decode chain after the long-context prefill
 DECODE_PREFILL = "gdn_fwd_64k"
@@ -226,9 +230,10 @@ def job_throughput(units_per_rank_step, steps, ms_max, world):
 # ----------------------------------------------------------------------------- native arm
 def make_device_sets(name, seed):
     """Two device-resident input sets of a forward workload (and the host copy)."""
-    from gated_delta_rule_forward_b200.inputs import make_inputs
+    from gated_delta_rule_forward_b200.inputs import make_inputs, make_raw_inputs
     variant, B, T, H, dk, dv = WORKLOADS[name]
-    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=seed)
+    make = make_raw_inputs if name in RAW_WORKLOADS else make_inputs
+    d = make(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=seed)
     dev = {k: (None if v is None else v.cuda()) for k, v in d.items()}
     # second set: the same tensors rolled along the head axis (distinct values and addresses)
     dev2 = {k: (None if v is None else torch.roll(v, 1, dims=-2 if v.dim() == 4 else -1).contiguous())
@@ -249,10 +254,12 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
     kernel = gdr.forward_kernel_name(variant, torch.bfloat16, B, T, H, dk, dv, 0)
     launches = gdr.forward_launches(variant, torch.bfloat16, B, T, H, dk, dv, 0)
 
+    raw = name in RAW_WORKLOADS
+
     def step(i):
         d = sets[i % 2]
         gdr.forward(d["q"], d["k"], d["v"], variant=variant, **gates(d), out=outs[i % 2],
-                    final_state=finals[i % 2], chunk=0)
+                    final_state=finals[i % 2], chunk=0, raw_inputs=raw)
 
     for i in range(W):
         step(i)
@@ -273,7 +280,7 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
     total_ms = max_over_ranks(total_ms, world)
     launch_ms = sum(per) / K                  # one kernel per step: its average duration
     res = {
-        "workload": name, "variant": variant, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+        "workload": name, "variant": variant, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "raw_inputs": raw,
         "kernel": kernel, "launches_per_step": launches, "ms_per_step": total_ms / K,
         "launch_ms": launch_ms, "tokens_per_step": B * T, "wall": (t_wall0, t_wall1),
         "alg_bytes": fwd_bytes(variant, B, T, H, dk, dv), "alg_flops": fwd_flops(variant, B, T, H, dk, dv),

@@ -32,6 +32,13 @@ gdr_status_t check_cuda(cudaError_t e, const char *what) {
 }
 
 bool valid_variant(int v) { return v >= GDR_DELTANET && v <= GDR_KLA; }
+
+// The raw-input flag may be OR'ed into a variant: returns it and strips it.
+bool take_raw(int &variant) {
+  const bool raw = (variant & GDR_RAW_INPUTS) != 0;
+  variant &= ~GDR_RAW_INPUTS;
+  return raw;
+}
 bool valid_dim(int d) { return d == 64 || d == 128; }
 
 enum class Kernel { None, Token, Split };
@@ -122,6 +129,7 @@ gdr_status_t gdr_device_status(void *stream) {
 }
 
 size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  take_raw(variant);
   if (!valid_variant(variant) || !valid_dim(dk) || !valid_dim(dv) || B <= 0 || T <= 0 || H <= 0) return 0;
   if ((chunk == 0 || chunk == 65) && split_ok(variant, dtype, dk, dv)) return gdr_split_workspace_bytes(variant, B, T, H, dv);
   return 0;
@@ -129,6 +137,7 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H, i
 
 // The kernel a call with a workspace of gdr_forward_workspace_size() bytes runs.
 static Kernel planned_kernel(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  take_raw(variant);
   gdr_status_t st;
   std::string why;
   const size_t ws = gdr_forward_workspace_size(variant, dtype, B, T, H, dk, dv, chunk);
@@ -136,6 +145,7 @@ static Kernel planned_kernel(int variant, int dtype, int B, int T, int H, int dk
 }
 
 int gdr_forward_launches(int variant, int dtype, int B, int T, int H, int dk, int dv, int chunk) {
+  take_raw(variant);
   if (!valid_variant(variant) || (dtype != 0 && dtype != 1) || !valid_dim(dk) || !valid_dim(dv)) return 0;
   if (B < 0 || T < 0 || H < 0) return 0;
   const Kernel kern = planned_kernel(variant, dtype, B, T, H, dk, dv, chunk);
@@ -156,6 +166,7 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
 
 gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms, int *segments,
                               int *segment_chunks, int *split_chunk) {
+  take_raw(variant);
   if (!valid_variant(variant)) return fail(GDR_ERR_INVALID_ARG, "unknown variant");
   if (!valid_dim(dv)) return fail(GDR_ERR_INVALID_ARG, "dv must be 64 or 128");
   if (B < 0 || T < 0 || H < 0 || sms < 0) return fail(GDR_ERR_INVALID_ARG, "B, T, H and sms must be >= 0");
@@ -167,6 +178,7 @@ gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms,
 gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                  const gdr_fwd_args_t *a, float eps, float scale, int chunk,
                                  void *workspace, size_t workspace_bytes, void *stream) {
+  const bool raw = take_raw(variant);
   gdr_status_t st = validate_common(variant, dtype, dk, dv);
   if (st != GDR_OK) return st;
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
@@ -205,6 +217,7 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
   gdr::FwdProblem p;
   p.variant = variant; p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
   p.bf16_io = dtype == GDR_BF16;
+  p.raw = raw;
   p.q = a->q; p.k = a->k; p.v = a->v;
   p.beta = a->beta; p.log_g = a->log_g; p.erase_b = a->erase_b; p.write_w = a->write_w;
   p.s0 = a->initial_state; p.s_final = a->final_state; p.o = a->o;
@@ -220,6 +233,8 @@ gdr_status_t gdr_forward_chunked(int variant, int dtype, int B, int T, int H, in
 
 gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, int H, int dk, int dv,
                                          const gdr_fwd_args_t *a, float eps, float scale, void *stream) {
+  const int variant_arg = variant;
+  const bool raw = take_raw(variant);
   gdr_status_t st = validate_common(variant, dtype, dk, dv);
   if (st != GDR_OK) return st;
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
@@ -238,7 +253,7 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
                     std::to_string(records * rec) + " bytes) but the fixed scratch holds " + std::to_string(have) +
                     " bytes: B * H * ceil(T / 64) must be at most " + std::to_string(have / rec) +
                     " for this variant and dv");
-  if ((long)B * H == 0 || T == 0) return gdr_forward_chunked(variant, dtype, B, T, H, dk, dv, a, eps, scale, 65,
+  if ((long)B * H == 0 || T == 0) return gdr_forward_chunked(variant_arg, dtype, B, T, H, dk, dv, a, eps, scale, 65,
                                                              nullptr, 0, stream);
   if (!a->q || !a->k || !a->v || !a->o) return fail(GDR_ERR_INVALID_ARG, "q, k, v and o are required");
   const void *io[4] = {a->q, a->k, a->v, a->o};
@@ -256,6 +271,7 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
   gdr::FwdProblem p;
   p.variant = variant; p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
   p.bf16_io = true;
+  p.raw = raw;
   p.q = a->q; p.k = a->k; p.v = a->v;
   p.beta = a->beta; p.log_g = a->log_g; p.erase_b = a->erase_b; p.write_w = a->write_w;
   p.s0 = a->initial_state; p.s_final = a->final_state; p.o = a->o;
@@ -269,6 +285,7 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
 gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int dv, const void *q, const void *k,
                              const void *v, const float *beta, const float *log_g, const float *erase_b,
                              const float *write_w, float *state, void *o, float eps, float scale, void *stream) {
+  const bool raw = take_raw(variant);
   gdr_status_t st = validate_common(variant, dtype, dk, dv);
   if (st != GDR_OK) return st;
   if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "N and H must be >= 0");
@@ -284,6 +301,7 @@ gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int d
   gdr::DecodeProblem p;
   p.variant = variant; p.N = N; p.H = H; p.dk = dk; p.dv = dv;
   p.bf16_io = dtype == GDR_BF16;
+  p.raw = raw;
   p.q = q; p.k = k; p.v = v;
   p.beta = beta; p.log_g = log_g; p.erase_b = erase_b; p.write_w = write_w;
   p.state = state; p.o = o; p.eps = eps; p.scale = scale;

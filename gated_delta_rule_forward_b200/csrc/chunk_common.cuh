@@ -1,6 +1,7 @@
 // Shared pieces of the chunked tensor-core kernels.
 #pragma once
 
+#include "common.cuh"
 #include "tc_util.cuh"
 
 namespace gdr {
@@ -10,6 +11,26 @@ constexpr int LD = 72;   // row stride (floats) of A^T and T scratch: conflict-f
 
 // Round to tf32 and keep as float: the solve stores its operands pre-rounded.
 __device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
+
+// Raw-input mode: 1 / ||row|| (floored as raw_inv_norm does) of the 64 rows of
+// a bf16 tile stored as two 64-element atoms of 128-byte swizzled rows (atom 1
+// at atom0 + atom_stride), into out[0..63].  256 threads, four per row; every
+// thread of the block must call it.
+__device__ __forceinline__ void tile_row_inv_norms(const uint8_t *atom0, uint32_t atom_stride, float *out, int tid) {
+  const int row = tid >> 2, qtr = tid & 3;
+  const uint8_t *a = atom0 + (qtr >> 1) * atom_stride;
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float x[8];
+    unpack8(*reinterpret_cast<const uint4 *>(a + sw128(row, 4 * (qtr & 1) + j)), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  if (qtr == 0) out[row] = raw_inv_norm(ss);
+}
 
 // T = (I + A)^{-1} for a strictly lower-triangular 64 x 64 A (C = 64), 16x16-blocked.
 // At[r * LD + t] holds A[t][r] pre-rounded to tf32 (written by the caller); the

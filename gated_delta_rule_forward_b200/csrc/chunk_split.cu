@@ -49,6 +49,8 @@
 //     REC_SC  fp32 Gamma_C: one value padded to 16 bytes, or d_k values
 //     GDN-2 only: the P^d V and D~^T V terms, 24 KB per 64 values
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "chunk_common.cuh"
@@ -97,8 +99,8 @@ constexpr uint32_t OFF_A = 49152;       // fp32 A^T, 64 x LD
 constexpr uint32_t OFF_TF = OFF_A + 64 * LD * 4;
 constexpr uint32_t OFF_T = 86016;       // bf16 T
 constexpr uint32_t OFF_TP = 94208;      // bf16 T Diag(Gamma)
-constexpr uint32_t OFF_SC = 102400;     // scalars: 6 x 64 floats
-constexpr uint32_t OFF_BAR = OFF_SC + 6 * 64 * 4;
+constexpr uint32_t OFF_SC = 102400;     // scalars: 8 x 64 floats
+constexpr uint32_t OFF_BAR = OFF_SC + 8 * 64 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T, "layout");
 constexpr uint32_t COL_G = 0;     // M128 x 64 (dead before W)
@@ -109,6 +111,7 @@ constexpr uint32_t TMEM_COLS = 256;
 
 struct PrepParams {
   int B, T, H, dv, NC;
+  bool raw;      // raw-input mode: unit q (and k), gates from their logits
   int c0, ncr;   // the launch prepares chunks [c0, c0 + ncr) of every (b, h)
   const float *beta, *log_g;
   const float *erase_b, *write_w;   // GDN-2 only
@@ -141,30 +144,47 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int NS = p.dv / 64;
   const int total = p.ncr * p.H * p.B;   // records of this launch, chunk index fastest
 
-  uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_mma = bar_in + 1;
-  uint64_t *bar_drain = bar_in + 2;     // error path only
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 3);
+  uint64_t *bar_q = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // Q landed
+  uint64_t *bar_k = bar_q + 1;          // K landed
+  uint64_t *bar_v = bar_q + 2;          // V landed
+  uint64_t *bar_mma = bar_q + 3;        // MMA1, then W
+  uint64_t *bar_u = bar_q + 4;          // U'^T
+  uint64_t *bar_drain = bar_q + 5;      // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_q + 6);
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);
   float *sc_g2 = sc_beta + 64;
   float *sc_wf = sc_g2 + 64;
   float *sc_G = sc_wf + 64;
   float *sc_tmp = sc_G + 64;
   float *sc_rk = sc_tmp + 64;   // 1 / ||k_t||
+  float *sc_vk = sc_rk + 64;    // 1 / ||k_t|| of the keys the recurrence sees (1 for keys normalised here)
+  float *sc_qn = sc_vk + 64;    // raw-input mode: 1 / ||q_t||
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
 
-  // TMA loads of record r's K, Q and V (thread 0)
-  auto issue_inputs = [&](int r) {
+  // TMA loads of record r's Q, K and V (thread 0), each on its own barrier so
+  // that each is issued as soon as the previous record no longer reads it:
+  // Q after the Qg conversion, K after W, V after U'.
+  uint32_t issued = 0, landed = 0;   // thread 0: loads issued / seen landing (q | k << 8 | v << 16)
+  auto issue_q = [&](int r) {
     const RecIdx x = rec_idx(p, r);
-    const int c = x.c, h = x.h, b = x.b;
-    const int t0 = c * C;
-    mbar_expect_tx(bar_in, 4 * 8192 + NS * 8192);
-    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_in, 0, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_in, 64, h, t0, b);
-    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_in, 64, h, t0, b);
-    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_in, 64 * sl, h, t0, b);
+    mbar_expect_tx(bar_q, 2 * 8192);
+    tma_load_4d(sm + OFF_KQ + 8192, &tm_q, bar_q, 0, x.h, x.c * C, x.b);
+    tma_load_4d(sm + OFF_KQ + 24576, &tm_q, bar_q, 64, x.h, x.c * C, x.b);
+    issued += 1u;
+  };
+  auto issue_k = [&](int r) {
+    const RecIdx x = rec_idx(p, r);
+    mbar_expect_tx(bar_k, 2 * 8192);
+    tma_load_4d(sm + OFF_KQ + 0, &tm_k, bar_k, 0, x.h, x.c * C, x.b);
+    tma_load_4d(sm + OFF_KQ + 16384, &tm_k, bar_k, 64, x.h, x.c * C, x.b);
+    issued += 1u << 8;
+  };
+  auto issue_v = [&](int r) {
+    const RecIdx x = rec_idx(p, r);
+    mbar_expect_tx(bar_v, NS * 8192);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_v, 64 * sl, x.h, x.c * C, x.b);
+    issued += 1u << 16;
   };
   // log decay and beta of token `tid` of record r (threads 0-63)
   auto load_gates = [&](int r, float &lg, float &bt) {
@@ -177,6 +197,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const size_t th = (static_cast<size_t>(b) * p.T + t) * p.H + h;
       if constexpr (scalar_decay(VAR)) lg = __ldg(p.log_g + th);
       bt = __ldg(p.beta + th);
+      if (p.raw) {
+        if constexpr (scalar_decay(VAR)) lg = raw_log_decay(lg);
+        bt = raw_gate(bt);
+      }
     }
   };
 
@@ -184,18 +208,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
-  bool in_flight = false;   // thread 0: a record's loads are outstanding on bar_in
   if (tid == 0) {
-    mbar_init(bar_in, 1);
+    mbar_init(bar_q, 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_u, 1);
     mbar_init(bar_drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     if (static_cast<int>(blockIdx.x) < total) {
-      issue_inputs(blockIdx.x);
-      in_flight = true;
+      issue_q(blockIdx.x);
+      issue_k(blockIdx.x);
+      issue_v(blockIdx.x);
     }
   }
   if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
@@ -213,13 +240,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   const uint32_t kq = smem_u32(sm + OFF_KQ);
-  uint32_t mma_phase = 0, in_phase = 0;
+  uint32_t mma_phase = 0;
   int bad = 0;
   float wmax = 0.f;
 
-  // Persistent over records: the next record's loads are issued as soon as
-  // MMA2 has consumed this record's inputs, and land during the epilogue.
+  // Persistent over records: each of the next record's loads is issued as soon
+  // as this record no longer reads its buffer.
   for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    const uint32_t ph = ((r - blockIdx.x) / gridDim.x) & 1;   // phase of the input and U' barriers
+    const bool more = r + static_cast<int>(gridDim.x) < total;
     uint8_t *rec = p.ws + rec_index(p, rec_idx(p, r)) * rec_bytes(NS);
     // gates: beta_t, cumulative log2 decay, Gamma_t
     if (tid < 64) {
@@ -239,11 +268,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       sc_g2[tid] = g2;
       sc_G[tid] = ex2(g2);
     }
-    if (!mbar_wait(bar_in, in_phase)) bad = 1;
+    if (!mbar_wait(bar_q, ph) || !mbar_wait(bar_k, ph)) bad = 1;
+    else if (tid == 0) landed += 1u | (1u << 8);
     bad = __syncthreads_or(bad);
     if (bad) break;
-    in_phase ^= 1;
-    if (tid == 0) in_flight = false;
+    if (p.raw) tile_row_inv_norms(sm + OFF_KQ + 8192, 16384, sc_qn, tid);   // read after MMA1's barrier
 
     // MMA1: [K;Q] K^T
     if (!bad && tid == 0) {
@@ -280,11 +309,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
         const float rk = kk > 0.f ? rsqrtf(kk) : 0.f;
         const float bt = sc_beta[t];
-        float c;
-        if constexpr (VAR == kKLA) c = (bt == 0.f) ? 0.f : bt * (kk * rk) / (kk + p.eps);   // Kaczmarz step
-        else c = bt * (kk * rk);
+        float c, vk = rk;
+        if constexpr (VAR == kKLA) {
+          c = (bt == 0.f) ? 0.f : bt * (kk * rk) / (kk + p.eps);   // Kaczmarz step
+        } else if (p.raw) {   // the recurrence sees the unit key k / ||k||: beta' = beta, v' = v
+          c = bt * rk;
+          vk = 1.f;
+        } else {
+          c = bt * (kk * rk);
+        }
         sc_beta[t] = c;
         sc_rk[t] = rk;
+        sc_vk[t] = vk;
       }
       __syncthreads();
       const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
@@ -312,8 +348,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
         for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(rkt * g[r] * fac[r]) : 0.f;
       } else {
+        const float qs = p.raw ? p.scale * sc_qn[t] : p.scale;
 #pragma unroll
-        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? p.scale * g[r] * fac[r] : 0.f;
+        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? qs * g[r] * fac[r] : 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
       }
@@ -321,28 +358,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tc_fence_before();
     __syncthreads();
 
-    // T = (I + A)^{-1}; T Diag(1/||k||) (for U' = T V') and T Diag(Gamma / ||k||)
-    // (for W = T Diag(Gamma) Khat) as bf16 tiles
-    solve_unit_lower_64(At, Tf, tid, warp, lane);
-    {
-      const int m = tid >> 2, n0 = (tid & 3) * 16;
-      float tv[16], tg[16];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
-        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        tv[e] = (n0 + e <= m) ? tv[e] * sc_rk[n0 + e] : 0.f;
-        tg[e] = tv[e] * sc_G[n0 + e];
-      }
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
-        st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
-      }
-    }
     // Gamma_C, and the fp16 copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K
     // (2048 sixteen-byte chunks in the swizzled image of the bf16 tiles)
     if (tid == 0) *reinterpret_cast<float4 *>(rec + rec_sc(NS)) = make_float4(sc_G[63], 0.f, 0.f, 0.f);
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint32_t off = sw128(r, j);
       float x[8];
       unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KQ + kb * 16384 + isq * 8192 + off), x);
-      const float f = isq ? p.scale * sc_G[r] : sc_wf[r];
+      const float f = isq ? p.scale * sc_G[r] * (p.raw ? sc_qn[r] : 1.f) : sc_wf[r];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         x[e] *= f;
@@ -362,38 +377,71 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       st_chunk_f16(rec + (isq ? REC_WQ + kb * 16384 + 8192 : REC_K + kb * 8192) + off, x);
     }
+    // Q is consumed: the next record's Q lands during the solve
+    __syncthreads();
+    if (tid == 0 && more) issue_q(r + gridDim.x);
+
+    // T = (I + A)^{-1}; T Diag(1/||k||) (for U' = T V'; the keys the recurrence
+    // sees) and T Diag(Gamma / ||k||) (for W = T Diag(Gamma) Khat) as bf16 tiles
+    solve_unit_lower_64(At, Tf, tid, warp, lane);
+    {
+      const int m = tid >> 2, n0 = (tid & 3) * 16;
+      float tv[16], tg[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = *reinterpret_cast<const float4 *>(Tf + m * LD + n0 + 4 * q4);
+        tv[4 * q4 + 0] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float te = (n0 + e <= m) ? tv[e] : 0.f;
+        tv[e] = te * sc_vk[n0 + e];
+        tg[e] = te * sc_G[n0 + e] * sc_rk[n0 + e];
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        st_chunk_bf16(sm + OFF_T + sw128(m, 2 * (tid & 3) + j), tv + 8 * j);
+        st_chunk_bf16(sm + OFF_TP + sw128(m, 2 * (tid & 3) + j), tg + 8 * j);
+      }
+    }
     fence_async_smem();
     __syncthreads();
 
-    // MMA2: W = T Diag(Gamma) K (M64 N128); U'^T = V^T T^T (M128 over d_v, N64)
+    // MMA2: W = T Diag(Gamma) K (M64 N128), then U'^T = V^T T^T (M128 over d_v,
+    // N64) on its own barrier, so that the W epilogue runs beside the U' product
     if (!bad && tid == 0) {
-      tc_fence_after();
-      const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
+      if (!mbar_wait(bar_v, ph)) {
+        bad = 1;
+      } else {
+        landed += 1u << 16;
+        tc_fence_after();
+        const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
                  idesc_bf16(64, 128, false, true), kk > 0);
+        mma_commit(bar_mma);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
                  idesc_bf16(128, 64, true, false), kk > 0);
-      mma_commit(bar_mma);
+        mma_commit(bar_u);
+      }
     }
-    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    bad = __syncthreads_or(bad);
+    if (bad) break;
+    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
+    if (bad) break;
     tc_fence_after();
-
-    // this record's inputs are consumed: start the next record's loads
-    if (!bad && r + static_cast<int>(gridDim.x) < total && tid == 0) {
-      issue_inputs(r + gridDim.x);
-      in_flight = true;
-    }
+    // K is consumed: the next record's K lands during the epilogues
+    if (tid == 0 && more) issue_k(r + gridDim.x);
 
     // -W (M64 layout: rows 16 quad + lane, lane < 16; column half `half` is d_k
-    // atom `half`) and U'^T (lane v = value column, columns t) -> fp16 record tiles
+    // atom `half`) -> fp16 record tile
     wmax = fmaxf(wmax, qkmax);
-    if (!bad) {
+    {
       float w[32];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
@@ -409,6 +457,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
         }
       }
+    }
+    // U'^T (lane v = value column, columns t) -> fp16 record tile
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_u, ph))) bad = 1;
+    if (!bad) {
+      tc_fence_after();
+      if (tid == 0 && more) issue_v(r + gridDim.x);   // V is consumed
+      float w[32];
       tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
       if (row < p.dv) {
 #pragma unroll
@@ -419,7 +474,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     }
     // tensor-memory reads done before the next record's MMA1
     tc_fence_before();
-    __syncthreads();
+    bad = __syncthreads_or(bad);
     if (bad) break;
   }
 
@@ -429,7 +484,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     atomicOr(&g_gdr_split_error, 1);
     mma_commit(bar_drain);
     mbar_wait(bar_drain, 0);
-    if (in_flight) mbar_wait(bar_in, in_phase);
+    uint64_t *bars[3] = {bar_q, bar_k, bar_v};
+    for (int i = 0; i < 3; ++i) {
+      const uint32_t n_issued = (issued >> (8 * i)) & 0xffu, n_landed = (landed >> (8 * i)) & 0xffu;
+      if (n_issued != n_landed) mbar_wait(bars[i], n_landed & 1u);
+    }
   }
   if (wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
   tc_fence_before();
@@ -467,8 +526,8 @@ constexpr uint32_t OFF_KG = OFF_R + 49152;      // (c..f) bf16 K o e^gamma [Kb0 
 constexpr uint32_t OFF_A = OFF_R;               // (d, e) fp32 A^T, 64 x LD
 constexpr uint32_t OFF_TF = OFF_R + 18432;      // (e) fp32 T, 64 x LD
 constexpr uint32_t OFF_T = OFF_R + 36864;       // (e, f) bf16 T
-constexpr uint32_t OFF_SC = OFF_R + 65536;      // beta [64], e^{gamma_m} [128], scratch [128]
-constexpr uint32_t OFF_BAR = OFF_SC + 320 * 4;
+constexpr uint32_t OFF_SC = OFF_R + 65536;      // beta [64], e^{gamma_m} [128], scratch [128], 1/||k|| [64], 1/||q|| [64]
+constexpr uint32_t OFF_BAR = OFF_SC + 448 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T && OFF_T + 8192 <= OFF_KG, "phase region layout");
 static_assert(OFF_XF % 1024 == 0 && OFF_YF % 1024 == 0 && OFF_KG % 1024 == 0 && OFF_T % 1024 == 0, "alignment");
@@ -500,6 +559,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);   // [64]
   float *sc_em = sc_beta + 64;                               // [128] e^{gamma_m} per channel
   float *sc_tmp = sc_em + 128;                               // [128]
+  float *sc_kn = sc_tmp + 128;                               // [64] raw-input mode: 1 / ||k_t||
+  float *sc_qn = sc_kn + 64;                                 // [64] raw-input mode: 1 / ||q_t||
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
@@ -530,7 +591,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const RecIdx x = rec_idx(p, r);
     const int c = x.c, h = x.h, b = x.b;
     const int t = c * C + tid;
-    return (t < p.T) ? __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h) : 0.f;
+    if (t >= p.T) return 0.f;
+    const float bt = __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h);
+    return p.raw ? raw_gate(bt) : bt;
   };
 
   if (warp == 0) {
@@ -587,7 +650,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float run = 0.f;
 #pragma unroll 8
       for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-        run += Gr[t * DK + ch] * LOG2E;
+        run += (p.raw ? raw_log_decay(Gr[t * DK + ch]) : Gr[t * DK + ch]) * LOG2E;
         Gr[t * DK + ch] = run;
       }
       if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
@@ -612,6 +675,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!mbar_wait(bar_kq, ph)) bad = 1;
     else if (tid == 0) landed += 1u << 8;
     bad = __syncthreads_or(bad);
+    if (p.raw && !bad) {   // unit q and k
+      tile_row_inv_norms(kq_ptr, 16384, sc_kn, tid);
+      tile_row_inv_norms(kq_ptr + 8192, 16384, sc_qn, tid);
+      __syncthreads();
+    }
     float qkmax = 0.f;
 
     // (c) MMA1 in two 64-channel halves; the record's Kt and Qg, and K o e^gamma for MMA2
@@ -626,6 +694,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float kx[4], qx[4];
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        if (p.raw) {
+          const float kn = sc_kn[t], qn = sc_qn[t];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kx[e] *= kn;
+            qx[e] *= qn;
+          }
+        }
         const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
         const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
         const float4 m4 = *reinterpret_cast<const float4 *>(sc_em + ch0);
@@ -825,8 +901,8 @@ constexpr uint32_t OFF_PD = OFF_R + 53248;      // fp16 P^d, rows t
 constexpr uint32_t OFF_RT = OFF_R + 61440;      // fp16 R, rows t
 constexpr uint32_t OFF_KG = OFF_R + 69632;      // (c..f) fp16 K o e^gamma [Kb0 | Kb1]
 constexpr uint32_t OFF_DT = OFF_R + 86016;      // (c..f) fp16 Dt [b0 | b1], rows r (MN-major operand)
-constexpr uint32_t OFF_SC = OFF_R + 102400;     // e^{gamma_m} [128], scratch [128]
-constexpr uint32_t OFF_BAR = OFF_SC + 256 * 4;
+constexpr uint32_t OFF_SC = OFF_R + 102400;     // e^{gamma_m} [128], scratch [128], 1/||k|| [64], 1/||q|| [64]
+constexpr uint32_t OFF_BAR = OFF_SC + 384 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_TF + 64 * LD * 4 <= OFF_T && OFF_YF + 32768 <= OFF_KG, "phase region layout");
@@ -861,6 +937,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_kq + 5);
   float *sc_em = reinterpret_cast<float *>(sm + OFF_SC);     // [128] e^{gamma_m} per channel
   float *sc_tmp = sc_em + 128;                               // [128]
+  float *sc_kn = sc_tmp + 128;                               // [64] raw-input mode: 1 / ||k_t||
+  float *sc_qn = sc_kn + 64;                                 // [64] raw-input mode: 1 / ||q_t||
   float *Gr = reinterpret_cast<float *>(sm + OFF_LG);        // [64][128]
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
@@ -899,6 +977,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const size_t gi = ((static_cast<size_t>(x.b) * p.T + t0 + t) * p.H + x.h) * DK + ch0;
         ebs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
         wrs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
+        if (p.raw) {
+          float4 &e4 = ebs[hp][it], &w4 = wrs[hp][it];
+          e4 = make_float4(raw_gate(e4.x), raw_gate(e4.y), raw_gate(e4.z), raw_gate(e4.w));
+          w4 = make_float4(raw_gate(w4.x), raw_gate(w4.y), raw_gate(w4.z), raw_gate(w4.w));
+        }
       }
     }
   };
@@ -955,7 +1038,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float run = 0.f;
 #pragma unroll 8
       for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-        run += Gr[t * DK + ch] * LOG2E;
+        run += (p.raw ? raw_log_decay(Gr[t * DK + ch]) : Gr[t * DK + ch]) * LOG2E;
         Gr[t * DK + ch] = run;
       }
       if (hh == 0) sc_tmp[ch] = run;
@@ -979,6 +1062,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!mbar_wait(bar_kq, ph)) bad = 1;
     else if (tid == 0) landed += 1u << 8;
     bad = __syncthreads_or(bad);
+    if (p.raw && !bad) {   // unit q and k
+      tile_row_inv_norms(kq_ptr, 16384, sc_kn, tid);
+      tile_row_inv_norms(kq_ptr + 8192, 16384, sc_qn, tid);
+      __syncthreads();
+    }
     float qkmax = 0.f;
 
     // (c) MMA1 in two 64-channel halves; the record's At and Qg; K o e^gamma and Dt for MMA2
@@ -995,6 +1083,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float kx[4], qx[4];
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
+        if (p.raw) {
+          const float kn = sc_kn[t], qn = sc_qn[t];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kx[e] *= kn;
+            qx[e] *= qn;
+          }
+        }
         const float4 eb = ebs[hp][it], wr = wrs[hp][it];
         const float4 g4 = *reinterpret_cast<const float4 *>(Gr + t * DK + ch0);
         const float4 h4 = *reinterpret_cast<const float4 *>(Gr + 63 * DK + ch0);
@@ -1262,15 +1358,18 @@ constexpr int NSTAGE = 3;
 constexpr int NCOMPUTE = 16;
 constexpr int NTHREADS_CARRY = (NCOMPUTE + 1) * 32;
 constexpr uint32_t STAGE = 74752;        // record image (<= 74240 bytes), 1 KB aligned
+constexpr uint32_t PART_A = REC_P;       // [-W; Qg] and Kt: the operands of Y and dS
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(STAGE % 1024 == 0 && STAGE >= rec_bytes(2) && STAGE >= rec_bytes_chan(2), "stage layout");
+static_assert(PART_A % 16 == 0 && (REC_U - REC_P) % 16 == 0, "bulk copies move 16-byte multiples");
 constexpr uint32_t COL_Y = 0;      // 2 x 128: [(-W S0)^T | (Qg S0)^T + (P E)^T], [v][t]
 constexpr uint32_t COL_DS = 256;   // 128: dS^T, [v][i]
 constexpr uint32_t COL_SA = 384;   // 64: fp16 S^T, d_k packed two per column (MMA operand)
-constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column (MMA operand)
+constexpr uint32_t COL_EA = 448;   // 2 x 32: fp16 E^T, tokens packed two per column (MMA operand), by chunk parity
 constexpr uint32_t TMEM_COLS = 512;
+constexpr long long WAIT_LIMIT = 1ll << 31;   // cycles, about a second
 }  // namespace carry
 
 // Segments: a launch holds up to two passes over segments of seg_len chunks,
@@ -1306,15 +1405,18 @@ struct CarryParams {
   float *s_final_b;
   size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
+  long long wait_limit;   // cycles a wait may spin before the kernel gives up
+  int fault_chunk;        // >= 0: CTA (0, 0, 0) never copies that chunk's operands (host fault injection)
 };
 
-// Bounded wait that also gives up once another warp has raised `abort`.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort) {
+// Bounded wait: gives up after `limit` cycles (raising `abort`) or once another
+// thread has raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort, long long limit) {
   if (mbar_try_wait(bar, phase)) return true;
   const long long start = clock64();
   while (!mbar_try_wait(bar, phase)) {
     if (*abort) return false;
-    if (clock64() - start > (1ll << 31)) {
+    if (clock64() - start > limit) {
       *abort = 1;
       return false;
     }
@@ -1322,10 +1424,45 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
   return true;
 }
 
+// Barrier of the NTHREADS_CARRY threads (named barrier 1) that returns whether
+// any of them passed `bad`: every thread then takes the same branch.
+__device__ __forceinline__ bool carry_barrier_or(bool bad) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(bad ? 1u : 0u), "n"(carry::NTHREADS_CARRY)
+      : "memory");
+  return r != 0;
+}
+
 // MODE 0: scalar Gamma_C.  MODE 1: Gamma_C a vector of d_k values (channel
 // decay).  MODE 2: as 1, plus the record's (P^d V)^T and (Dt^T V)^T terms added
 // to the output and to the state (GDN-2); each compute thread loads its share
-// of them from the record one chunk ahead.
+// of them from the record (the issuer prefetches it into L2).
+//
+// 16 compute warps (thread v of warp (quad, part) owns value column v = 32 quad
+// + lane, d_k rows 32 part .. 32 part + 31 of S^T in fp32 registers, and tokens
+// 16 part .. 16 part + 15 of E^T and of the output) and one issuer warp.  Per
+// chunk c the compute warps hand over to the issuer through two barriers
+// (named barrier 1 with an OR reduction, so that a failed wait ends the sweep
+// for every warp at the same point), and the issuer's MMAs complete on
+// mbarriers the compute warps wait for:
+//     wait Y(c);  E^T = U'^T + Y_W -> tensor memory (fp16, two buffers by
+//     chunk parity, so that the second P half of chunk c-1 may still read its own) | barrier B1
+//     issuer: dS^T = E^T Kt,  first half of Y_Q += E^T P^T
+//     output rows of chunk c-1;  wait dS(c);  S^T = Gamma_C S^T + dS^T  | barrier B2
+//     issuer: copies of the next records,  Y(c+1) = S^T [-W; Qg]^T,
+//             second half of Y_Q(c) += E^T P^T
+// The P product is split around Y(c+1) so that it fills the tensor pipe while
+// the compute warps work instead of delaying the products on the state's
+// critical path.  A record is copied in two parts: [-W; Qg] and Kt (read only
+// by Y and dS) as soon as the stage's chunk has finished dS, three chunks
+// ahead; P, U'^T and Gamma_C once that chunk's last P half and output rows are
+// done, two chunks ahead.
 // 17 warps: one SM sub-partition holds five of them, so 96 registers per thread.
 template <int MODE>
 __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
@@ -1341,30 +1478,30 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   const int c_first = p.c_base + (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
   const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
   const bool values = !(flags & CARRY_NO_VALUES);
+  const long long limit = p.wait_limit;
+  const int fault_chunk = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.fault_chunk : -1;
 
-  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
-  uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
-  uint64_t *bar_s = bar_e + 1;            // dS^T(c) done
-  uint64_t *bar_o = bar_e + 2;            // E^T P^T (c) done
-  uint64_t *bar_ea = bar_e + 3;           // E^T(c) in tensor memory (16 warps)
-  uint64_t *bar_sa = bar_e + 4;           // S^T in tensor memory (16 warps)
-  uint64_t *bar_done = bar_e + 5;         // chunk c's Y read and stage released (16 warps)
-  uint64_t *bar_drain = bar_e + 6;        // error path only
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 7);
-  volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 8);
+  uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] part A landed
+  uint64_t *bar_b = bar_a + NSTAGE;       // [NSTAGE] part B landed
+  uint64_t *bar_e = bar_b + NSTAGE;       // Y(c) done
+  uint64_t *bar_s = bar_e + 1;            // dS^T(c) (and the first P half) done
+  uint64_t *bar_o = bar_e + 2;            // Y_Q(c) complete (second P half done)
+  uint64_t *bar_drain = bar_e + 3;        // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 4);
+  volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 5);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < NSTAGE; ++i) mbar_init(&bar_full[i], 1);
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&bar_a[i], 1);
+      mbar_init(&bar_b[i], 1);
+    }
     mbar_init(bar_e, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
-    mbar_init(bar_ea, NCOMPUTE);
-    mbar_init(bar_sa, NCOMPUTE);
-    mbar_init(bar_done, NCOMPUTE);
     mbar_init(bar_drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -1373,133 +1510,163 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t rb = p.rec_bytes;
+  const uint32_t part_b = p.copy_bytes - PART_A;
   // every CTA of this grid holds its SM: a preparation grid launched as this
   // grid's programmatic dependent (the pipelined sweep) may take the others
   griddep_launch_dependents();
 
-  // issuer's view of the record copies: stage has a copy in flight / phase parity to wait for
+  const bool issuer = warp == NCOMPUTE;
+  const bool leader = issuer && lane == 0;
+  // issuer's view of the record copies: (part, stage) has a copy in flight, and
+  // the phase parity each part's barrier completes next
   uint32_t pend = 0, par = 0;
   float smax = 0.f;
   float S[32];
   const int quad = warp & 3, part = (warp >> 2) & 3;
   const int v = quad * 32 + lane;
-  const bool has_v = quad * 32 < p.dv;   // warp-uniform (d_v is 64 or 128)
+  const bool has_v = !issuer && quad * 32 < p.dv;   // warp-uniform (d_v is 64 or 128)
   const uint32_t lrow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
 
-  if (warp == NCOMPUTE) {
-    // ---------------------------------------------------------------- issuer
-    if (lane == 0) {
-      const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
-      auto issue_chunk = [&](int c) {
-        const int s = c % NSTAGE;
-        mbar_expect_tx(&bar_full[s], p.copy_bytes);
-        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, p.copy_bytes, &bar_full[s]);
-        // MODE 2: the rest of the record, which the compute threads read themselves
-        if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
-        pend |= 1u << s;
-      };
-      auto wait_full = [&](int c) -> bool {
-        const int s = c % NSTAGE;
-        if (!wait_or_abort(&bar_full[s], (c / NSTAGE) & 1, abort)) return false;
-        pend &= ~(1u << s);
-        par ^= 1u << s;
-        return true;
-      };
-      auto issue_y = [&](int c) {   // Y(c) = S^T [-W; Qg]^T
-        tc_fence_after();
-        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
+  auto copy_a = [&](int c) {   // leader: [-W; Qg] and Kt of chunk c
+    const int s = c % NSTAGE;
+    if (c == fault_chunk) return;   // injected fault: no copy and no expected bytes
+    mbar_expect_tx(&bar_a[s], PART_A);
+    bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, PART_A, &bar_a[s]);
+    pend |= 1u << s;
+  };
+  auto copy_b = [&](int c) {   // leader: P, U'^T and Gamma_C of chunk c (and the GDN-2 terms into L2)
+    const int s = c % NSTAGE;
+    mbar_expect_tx(&bar_b[s], part_b);
+    bulk_load(sm + s * STAGE + PART_A, recs + static_cast<size_t>(c) * rb + PART_A, part_b, &bar_b[s]);
+    if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
+    pend |= 1u << (NSTAGE + s);
+  };
+  // leader: wait for part A of chunk c, then Y(c) = S^T [-W; Qg]^T
+  auto issue_y = [&](int c) -> bool {
+    const int s = c % NSTAGE;
+    if (!wait_or_abort(&bar_a[s], (c / NSTAGE) & 1, abort, limit)) return false;
+    pend &= ~(1u << s);
+    par ^= 1u << s;
+    tc_fence_after();
+    const uint32_t st = smem_u32(sm + s * STAGE);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
-                 sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
-                 kk > 0);
-        mma_commit(bar_e);
-      };
-      griddep_wait();   // the records are the preparation kernel's output
-      for (int c = 0; c < NSTAGE && c < NC; ++c) issue_chunk(c);
-      bool ok = wait_or_abort(bar_sa, 0, abort) && wait_full(0);
-      if (ok) issue_y(0);
-      // Waits follow the order in which the compute warps arrive (done(c-1)
-      // before E(c) before S(c)), so no barrier can complete a phase the
-      // issuer has not waited for yet.
-      for (int c = 0; ok && c < NC; ++c) {
-        // chunk c-1 fully consumed: its stage takes record c+2
-        if (c >= 1) {
-          if (!(ok = wait_or_abort(bar_done, (c - 1) & 1, abort))) break;
-          if (c + 2 < NC) issue_chunk(c + 2);
-        }
-        // dS^T = E^T Kt ; Y_Q += E^T P^T
-        if (!(ok = wait_or_abort(bar_ea, c & 1, abort))) break;
-        tc_fence_after();
-        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
+             sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
+             kk > 0);
+    mma_commit(bar_e);
+    return true;
+  };
+  // leader: Y_Q(c) += E^T P^T over tokens 32 h2 .. 32 h2 + 31 of chunk c
+  auto issue_p = [&](int c, int h2) {
+    const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + COL_DS, tmem + COL_EA + 8 * kk, sdesc(st + REC_K + kk * 2048, 8192, 1024),
-                 idesc_f16(128, 128, false, true), kk > 0);
-        mma_commit(bar_s);
+    for (int kk = 2 * h2; kk < 2 * h2 + 2; ++kk)
+      mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 32 * (c & 1) + 8 * kk,
+             sdesc(st + REC_P + kk * 32, 16, 1024),
+             idesc_f16(128, 64, false, false), 1);
+  };
+  // leader: wait for part B of chunk c (its U'^T and Gamma_C are read by the compute warps)
+  auto note_b = [&](int c) {
+    const int s = c % NSTAGE;
+    pend &= ~(1u << (NSTAGE + s));
+    par ^= 1u << (NSTAGE + s);
+  };
+
+  // ---------------------------------------------------------------- set-up
+  griddep_wait();   // the initial state and the records may be the previous grid's output
+  if (leader) {
+    for (int c = 0; c < NSTAGE && c < NC; ++c) copy_a(c);
+    for (int c = 0; c < NSTAGE - 1 && c < NC; ++c) copy_b(c);
+  }
+  auto store_state = [&]() {
+    uint32_t r[16];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 8 * kk, sdesc(st + REC_P + kk * 32, 16, 1024),
-                 idesc_f16(128, 64, false, false), 1);
-        mma_commit(bar_o);
-        if (c + 1 < NC) {
-          if (!(ok = wait_or_abort(bar_sa, (c + 1) & 1, abort) && wait_full(c + 1))) break;
-          issue_y(c + 1);
+    for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
+    tmem_st16(lrow + COL_SA + 16 * part, r);
+    tmem_wait_st();
+  };
+  if (!issuer) {
+    const size_t base = (static_cast<size_t>(b) * p.H + h) * p.s0_bh_stride + static_cast<size_t>(32 * part) * p.dv + v;
+    const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
+             : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
+    store_state();
+  }
+  tc_fence_before();
+  bool bad = carry_barrier_or(false);
+  if (leader && NC > 0 && !issue_y(0)) bad = true;
+
+  // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
+  // loaded from L2 shortly before their use
+  uint4 od_raw[2], sd_raw[4];
+  auto local_terms = [&](int c) { return recs + static_cast<size_t>(c) * rb + p.copy_bytes; };
+  auto load_sd = [&](int c) {
+    const uint4 *sd = reinterpret_cast<const uint4 *>(local_terms(c) + 8192 * NS + v * 256 + part * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sd_raw[j] = (has_v && values) ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  auto load_od = [&](int c) {
+    const uint4 *od = reinterpret_cast<const uint4 *>(local_terms(c) + v * 128 + part * 32);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  // output rows of chunk c: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
+  // through this warp's 1 KB of the stage's (consumed) U'^T tile into 16-byte stores
+  auto output_rows = [&](int c) -> bool {
+    const bool ok = __all_sync(0xffffffffu, wait_or_abort(bar_o, c & 1, abort, limit));
+    if (!ok) return false;
+    tc_fence_after();
+    float yo[16];
+    tmem_ld16(lrow + COL_Y + 128 * (c & 1) + 64 + 16 * part, yo);
+    tmem_wait_ld();
+    if constexpr (MODE == 2) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const __half2 *hp = reinterpret_cast<const __half2 *>(&od_raw[j]);
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+          const float2 f = __half22float2(hp[q2]);
+          yo[8 * j + 2 * q2] += f.x;
+          yo[8 * j + 2 * q2 + 1] += f.y;
         }
       }
     }
-  } else {
-    // ---------------------------------------------------------------- compute warps
-    griddep_wait();   // the initial state and the records may be the previous grid's output
-    {
-      const size_t base = (static_cast<size_t>(b) * p.H + h) * p.s0_bh_stride + static_cast<size_t>(32 * part) * p.dv + v;
-      const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
+    if (has_v && !(flags & CARRY_NO_OUTPUT)) {
+      uint8_t *tile = sm + (c % NSTAGE) * STAGE + REC_U + (quad * 4 + part) * 1024;
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
-               : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
-    }
-    auto store_state = [&]() {
-      uint32_t r[16];
-#pragma unroll
-      for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
-      tmem_st16(lrow + COL_SA + 16 * part, r);
-      tmem_wait_st();
-      tc_fence_before();
+      for (int m = 0; m < 16; ++m)
+        *reinterpret_cast<__nv_bfloat16 *>(tile + m * 64 + lane * 2) = __float2bfloat16_rn(yo[m]);
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sa);
-    };
-    store_state();
-    // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
-    // each loaded from L2 (the issuer prefetches records there) just before the wait that
-    // precedes its use; short live ranges keep them out of local memory, where a pending
-    // load would stall its spill store
-    uint4 od_raw[2], sd_raw[4];
-    auto local_terms = [&](int c) {
-      return p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first + c) * rb + p.copy_bytes;
-    };
-    auto load_sd = [&](int c) {
-      const uint4 *sd = reinterpret_cast<const uint4 *>(local_terms(c) + 8192 * NS + v * 256 + part * 64);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sd_raw[j] = (has_v && values) ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
-    };
-    auto load_od = [&](int c) {
-      const uint4 *od = reinterpret_cast<const uint4 *>(local_terms(c) + v * 128 + part * 32);
-#pragma unroll
-      for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
-    };
-    for (int c = 0; c < NC; ++c) {
-      uint8_t *st = sm + (c % NSTAGE) * STAGE;
-      const uint32_t y = lrow + COL_Y + 128 * (c & 1);
+      for (int it = 0; it < 2; ++it) {
+        const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
+        const int t = (c_first + c) * C + 16 * part + tr;
+        const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
+        if (t < p.T)
+          *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
+                                     8 * piece) = val;
+      }
+      fence_async_smem();   // the next copy into this stage is an async-proxy write
+    }
+    return true;
+  };
 
+  // ---------------------------------------------------------------- sweep
+  for (int c = 0; c < NC; ++c) {
+    const int s = c % NSTAGE;
+    uint8_t *st = sm + s * STAGE;
+    if (!issuer) {
       // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15
-      bool ok = wait_or_abort(&bar_full[c % NSTAGE], (c / NSTAGE) & 1, abort) &&
-                wait_or_abort(bar_e, c & 1, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      {
+      bad = !__all_sync(0xffffffffu, wait_or_abort(&bar_b[s], (c / NSTAGE) & 1, abort, limit) &&
+                                         wait_or_abort(bar_e, c & 1, abort, limit));
+      if (!bad) {
+        tc_fence_after();
         float e[16];
-        tmem_ld16(y + 16 * part, e);
+        tmem_ld16(lrow + COL_Y + 128 * (c & 1) + 16 * part, e);
         tmem_wait_ld();
         if (has_v && values) {
 #pragma unroll
@@ -1520,20 +1687,34 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           smax = fmaxf(smax, fmaxf(fabsf(e[2 * m]), fabsf(e[2 * m + 1])));
           r[m] = pack_f16x2(e[2 * m], e[2 * m + 1]);
         }
-        tmem_st8(lrow + COL_EA + 8 * part, r);
+        tmem_st8(lrow + COL_EA + 32 * (c & 1) + 8 * part, r);
         tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ea);
+        if constexpr (MODE == 2) load_sd(c);
       }
-      if constexpr (MODE == 2) load_sd(c);
+    }
+    tc_fence_before();
+    bad = carry_barrier_or(bad);   // B1: E^T(c) in tensor memory
+    if (bad) break;
 
-      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row
-      // for channel decay)
-      ok = wait_or_abort(bar_s, c & 1, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
+    if (leader) {
+      note_b(c);   // every compute warp observed part B of chunk c before B1
+      // dS^T = E^T Kt ; first half of Y_Q(c) += E^T P^T
       tc_fence_after();
-      {
+      const uint32_t sa = smem_u32(st);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tmem + COL_DS, tmem + COL_EA + 32 * (c & 1) + 8 * kk, sdesc(sa + REC_K + kk * 2048, 8192, 1024),
+               idesc_f16(128, 128, false, true), kk > 0);
+      mma_commit(bar_s);
+      issue_p(c, 0);
+    }
+    if (!issuer) {
+      // output rows of the previous chunk while dS(c) runs
+      if (c >= 1 && !output_rows(c - 1)) bad = true;
+      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row for channel decay)
+      if (!bad) bad = !__all_sync(0xffffffffu, wait_or_abort(bar_s, c & 1, abort, limit));
+      if (!bad) {
+        tc_fence_after();
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
 #pragma unroll
         for (int hv = 0; hv < 2; ++hv) {   // two halves of 16 rows keep the register count down
@@ -1562,65 +1743,37 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         store_state();
         if constexpr (MODE == 2) load_od(c);
       }
+    }
+    tc_fence_before();
+    bad = carry_barrier_or(bad);   // B2: S^T in tensor memory; chunk c-1 fully consumed
+    if (bad) break;
 
-      // output rows: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
-      // through this warp's 1 KB of the stage's (now unused) U'^T tile into 16-byte stores
-      ok = wait_or_abort(bar_o, c & 1, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      {
-        float yo[16];
-        tmem_ld16(y + 64 + 16 * part, yo);
-        tmem_wait_ld();
-        if constexpr (MODE == 2) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const __half2 *hp = reinterpret_cast<const __half2 *>(&od_raw[j]);
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              const float2 f = __half22float2(hp[q2]);
-              yo[8 * j + 2 * q2] += f.x;
-              yo[8 * j + 2 * q2 + 1] += f.y;
-            }
-          }
-        }
-        if (has_v && !(flags & CARRY_NO_OUTPUT)) {
-          uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            *reinterpret_cast<__nv_bfloat16 *>(tile + m * 64 + lane * 2) = __float2bfloat16_rn(yo[m]);
-          __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 2; ++it) {
-            const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
-            const int t = (c_first + c) * C + 16 * part + tr;
-            const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
-            if (t < p.T)
-              *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
-                                         8 * piece) = val;
-          }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_done);
-      }
+    if (leader) {
+      // stage (c+2) % NSTAGE held chunk c-1, whose P and output rows are done;
+      // stage c % NSTAGE's part A is consumed (Y(c) and dS(c) are done)
+      if (c + 2 < NC) copy_b(c + 2);
+      if (c + NSTAGE < NC) copy_a(c + NSTAGE);
+      if (c + 1 < NC && !issue_y(c + 1)) bad = true;   // raises `abort`; every warp stops at B1
+      issue_p(c, 1);
+      mma_commit(bar_o);
     }
   }
+  // output rows of the last chunk
+  if (!bad && !issuer && NC > 0 && !output_rows(NC - 1)) bad = true;
 
   __syncthreads();
   const bool failed = *abort != 0;
   if (failed) {
     // a wait gave up: report it, then let the MMAs and copies in flight
     // finish (each wait again bounded) before tensor memory is released
-    if (warp == NCOMPUTE && lane == 0) {
+    if (leader) {
       atomicOr(&g_gdr_split_error, 1);
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0);
-      for (int s = 0; s < NSTAGE; ++s)
-        if (pend >> s & 1u) mbar_wait(&bar_full[s], par >> s & 1u);
+      for (int i = 0; i < 2 * NSTAGE; ++i)
+        if (pend >> i & 1u) mbar_wait(i < NSTAGE ? &bar_a[i] : &bar_b[i - NSTAGE], par >> i & 1u);
     }
-  } else if (warp < NCOMPUTE) {
+  } else if (!issuer) {
     if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
     const bool write_final = !(flags & CARRY_LAST_FINAL) || zi + 1 == p.z_split;
     float *sf = pass_b ? p.s_final_b : p.s_final;
@@ -1684,7 +1837,7 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
     return cudaErrorInvalidValue;
   }
   PrepParams pp;
-  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC; pp.raw = p.raw;
   pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
@@ -1726,7 +1879,7 @@ cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, const Pre
     return cudaErrorInvalidValue;
   }
   PrepParams pp;
-  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC; pp.raw = p.raw;
   pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
   pp.beta = nullptr; pp.log_g = p.log_g; pp.erase_b = p.erase_b; pp.write_w = p.write_w; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
@@ -1761,7 +1914,7 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, const Pre
     return cudaErrorInvalidValue;
   }
   PrepParams pp;
-  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC;
+  pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC; pp.raw = p.raw;
   pp.c0 = rg.c0; pp.ncr = rg.ncr > 0 ? rg.ncr : NC;
   pp.beta = p.beta; pp.log_g = p.log_g; pp.ws = ws;
   pp.eps = p.eps; pp.scale = p.scale;
@@ -1866,6 +2019,12 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.seg_first_b = l.seg_first_b; cp.flags_b = l.flags_b;
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
+  // GDR_FAULT=wait (host-side fault injection for the failure-path tests): CTA
+  // (0, 0, 0) never copies chunk 1's operands, and waits give up after 2^20 cycles.
+  const char *fault = std::getenv("GDR_FAULT");
+  const bool inject = fault != nullptr && std::strcmp(fault, "wait") == 0;
+  cp.wait_limit = inject ? (1ll << 20) : carry::WAIT_LIMIT;
+  cp.fault_chunk = inject ? 1 : -1;
   e = launch_maybe_pdl(chunk_carry_kernel<MODE>, dim3(p.H, p.B, l.segments + l.segments_b),
                        dim3(carry::NTHREADS_CARRY), carry::SMEM_BYTES, stream, pdl, cp);
   if (e != cudaSuccess) *err = "carry launch: ";

@@ -13,10 +13,12 @@ enum Variant : int { kDeltaNet = 0, kGatedDeltaNet = 1, kKDA = 2, kGDN2 = 3, kKL
 __host__ __device__ constexpr bool scalar_decay(int v) { return v == kGatedDeltaNet || v == kKLA; }
 __host__ __device__ constexpr bool channel_decay(int v) { return v == kKDA || v == kGDN2; }
 
-// Problem description handed from the ABI layer to the launchers.
+// Problem description handed from the ABI layer to the launchers.  `raw`:
+// q, k, beta and the gates arrive as raw projections and logits, and the
+// kernels apply the input transforms on their load paths (see raw_* below).
 struct FwdProblem {
   int variant, B, T, H, dk, dv;
-  bool bf16_io;
+  bool bf16_io, raw;
   const void *q, *k, *v;
   const float *beta, *log_g, *erase_b, *write_w;
   const float *s0;
@@ -27,7 +29,7 @@ struct FwdProblem {
 
 struct DecodeProblem {
   int variant, N, H, dk, dv;
-  bool bf16_io;
+  bool bf16_io, raw;
   const void *q, *k, *v;
   const float *beta, *log_g, *erase_b, *write_w;
   float *state;
@@ -80,6 +82,15 @@ template <> __device__ __forceinline__ void st8<__nv_bfloat16>(__nv_bfloat16 *p,
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
   *reinterpret_cast<uint4 *>(p) = u;
 }
+
+// Input transforms of the raw-input mode (the parameterisation the workloads
+// use): a decay logit x gives log g = -softplus(x) (so g = sigmoid(-x) in
+// (0, 1)); beta / eta and the GDN-2 erase and write gates are sigmoid of their
+// logits; q and k are scaled to unit L2 norm (KLA's keys are not: its step
+// eta / (||k||^2 + eps) carries their norm), with the norm floored at 1e-6.
+__device__ __forceinline__ float raw_log_decay(float x) { return -(fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)))); }
+__device__ __forceinline__ float raw_gate(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float raw_inv_norm(float sumsq) { return 1.f / fmaxf(sqrtf(sumsq), 1e-6f); }
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll

@@ -13,7 +13,9 @@
 //   - the update S = S~ - a x^T + c v^T is written straight from registers
 //     (in place) and o = scale * (y - (a.q) x + (c.q) v).
 // Recurrence as in "Kaczmarz Linear Attention" (KLA update rule) and the
-// erase/write reading of "Gated DeltaNet-2" (technical core).
+// erase/write reading of "Gated DeltaNet-2" (technical core).  In the raw-input
+// mode q and k are scaled to unit norm and the gates taken from their logits
+// on the load path (a few hundred bytes beside the 128 KB state stream).
 #include "common.cuh"
 
 namespace gdr {
@@ -46,16 +48,33 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeP
   const IO *q = static_cast<const IO *>(p.q) + nh * DK;
   const IO *k = static_cast<const IO *>(p.k) + nh * DK;
   const IO *v = static_cast<const IO *>(p.v) + nh * DV;
+  const bool raw = p.raw;
+  __shared__ float inv_qk[2];
+  if (raw && tid < 64) {   // raw-input mode: warp 0 sums q^2, warp 1 k^2
+    const IO *x = tid < 32 ? q : k;
+    float ss = 0.f;
+    for (int i = tid & 31; i < DK; i += 32) {
+      const float e = ld_io<IO>(x + i);
+      ss = fmaf(e, e, ss);
+    }
+    ss = warp_sum(ss);
+    if ((tid & 31) == 0) inv_qk[tid >> 5] = (tid >= 32 && VAR == kKLA) ? 1.f : raw_inv_norm(ss);
+  }
+  if (raw) __syncthreads();
   if (tid < DK) {
-    const float kk = ld_io<IO>(k + tid);
+    const float kk = ld_io<IO>(k + tid) * (raw ? inv_qk[1] : 1.f);
     kf[tid] = kk;
-    qf[tid] = ld_io<IO>(q + tid);
-    if constexpr (scalar_decay(VAR)) gf[tid] = expf(__ldg(p.log_g + nh));
-    else if constexpr (channel_decay(VAR)) gf[tid] = expf(__ldg(p.log_g + nh * DK + tid));
-    else gf[tid] = 1.f;
+    qf[tid] = ld_io<IO>(q + tid) * (raw ? inv_qk[0] : 1.f);
+    if constexpr (scalar_decay(VAR) || channel_decay(VAR)) {
+      const float lg = __ldg(p.log_g + (scalar_decay(VAR) ? nh : nh * DK + tid));
+      gf[tid] = expf(raw ? raw_log_decay(lg) : lg);
+    } else {
+      gf[tid] = 1.f;
+    }
     if constexpr (VAR == kGDN2) {
-      af[tid] = __ldg(p.erase_b + nh * DK + tid) * kk;
-      cf[tid] = __ldg(p.write_w + nh * DK + tid) * kk;
+      const float eb = __ldg(p.erase_b + nh * DK + tid), ww = __ldg(p.write_w + nh * DK + tid);
+      af[tid] = (raw ? raw_gate(eb) : eb) * kk;
+      cf[tid] = (raw ? raw_gate(ww) : ww) * kk;
     }
   }
   if (tid < DV) vf[tid] = ld_io<IO>(v + tid);
@@ -79,6 +98,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeP
   float step = 0.f;
   if constexpr (VAR != kGDN2) {
     step = __ldg(p.beta + nh);                        // beta, or eta for KLA
+    if (raw) step = raw_gate(step);
     if constexpr (VAR == kKLA) step = step / (s2 + p.eps);
   }
 

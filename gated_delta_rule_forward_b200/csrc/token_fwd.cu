@@ -13,7 +13,8 @@
 //
 // This kernel serves fp32 I/O (where the 1e-4 relative bar rules out bf16
 // tensor-core operands), chunk == 1 requests, and shapes the chunked kernel
-// does not cover.  Columns are independent, so the slicing is exact.
+// does not cover.  Columns are independent, so the slicing is exact.  In the
+// raw-input mode each token's q, k and gates are transformed as they are used.
 #include "common.cuh"
 
 namespace gdr {
@@ -81,6 +82,28 @@ __global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
       d.beta = __ldg(p.beta + th);
     }
   };
+  // raw-input mode: unit q (and k, except KLA's), gates from their logits
+  auto transform = [&](TokenIn &d) {
+    float qq = 0.f, kk = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      qq = fmaf(d.qv[r], d.qv[r], qq);
+      kk = fmaf(d.kv[r], d.kv[r], kk);
+    }
+    const float rq = raw_inv_norm(warp_sum(qq));
+    const float rk = VAR == kKLA ? 1.f : raw_inv_norm(warp_sum(kk));
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      d.qv[r] *= rq;
+      d.kv[r] *= rk;
+      if constexpr (scalar_decay(VAR) || channel_decay(VAR)) d.lg[r] = raw_log_decay(d.lg[r]);
+      if constexpr (VAR == kGDN2) {
+        d.eb[r] = raw_gate(d.eb[r]);
+        d.ww[r] = raw_gate(d.ww[r]);
+      }
+    }
+    if constexpr (VAR != kGDN2) d.beta = raw_gate(d.beta);
+  };
 
   // Software pipeline over tokens: token t+1's loads are in flight while
   // token t is computed, so each step waits for no memory latency.
@@ -90,6 +113,7 @@ __global__ void __launch_bounds__(128) token_fwd_kernel(const FwdProblem p) {
   for (int t = 0; t < p.T; ++t) {
     const size_t th = ((size_t)b * p.T + t) * p.H + h;
     if (t + 1 < p.T) load(t + 1, nxt);
+    if (p.raw) transform(cur);
     const float *kv = cur.kv, *qv = cur.qv, *vv = cur.vv;
     float g[R], ea[R], wc[R];
 #pragma unroll

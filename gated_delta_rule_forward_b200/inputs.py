@@ -80,6 +80,55 @@ def make_inputs(variant: str, B: int, T: int, H: int, dk: int = 128, dv: int = 1
     }
 
 
+def make_raw_inputs(variant: str, B: int, T: int, H: int, dk: int = 128, dv: int = 128,
+                    dtype: torch.dtype = torch.bfloat16, seed: int = 0) -> dict:
+    """The same draws as make_inputs, before the transforms: q and k as drawn
+    (KLA's k already scaled by 1/sqrt(dk) and the key scale, since that is its
+    key), v, and the logits of beta (eta), of the decay and of the GDN-2 gates.
+    q, k, v in the I/O dtype, the logits fp32.  For the raw-input mode."""
+    if variant not in VARIANT_NAMES:
+        raise ValueError(f"unknown variant {variant!r}")
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn(B, T, H, dk, generator=g)
+    k = torch.randn(B, T, H, dk, generator=g)
+    v = torch.randn(B, T, H, dv, generator=g)
+    beta_logit = torch.randn(B, T, H, generator=g)
+    channel = variant in CHANNEL_DECAY
+    decay_logit = torch.randn(*((B, T, H, dk) if channel else (B, T, H)), generator=g)
+    erase_logit = write_logit = None
+    if variant == "gdn2":
+        erase_logit = torch.randn(B, T, H, dk, generator=g)
+        write_logit = torch.randn(B, T, H, dk, generator=g)
+    if variant == "kla":
+        key_scale = torch.exp(0.5 * torch.randn(B, T, H, generator=g))
+        k = k / (dk ** 0.5) * key_scale[..., None]
+    return {
+        "q": q.to(dtype).contiguous(), "k": k.to(dtype).contiguous(), "v": v.to(dtype).contiguous(),
+        "beta": None if variant == "gdn2" else beta_logit.contiguous(),
+        "log_g": None if variant == "deltanet" else decay_logit.contiguous(),
+        "erase_b": None if erase_logit is None else erase_logit.contiguous(),
+        "write_w": None if write_logit is None else write_logit.contiguous(),
+    }
+
+
+def transform_raw(variant: str, raw: dict) -> dict:
+    """The input transforms applied to raw inputs, in float64 on the exact
+    values passed (the I/O-dtype q, k, v up-cast): unit q, unit k except KLA's,
+    sigmoid of beta / eta and of the GDN-2 gates, log_g = -softplus.  What the
+    raw-input mode of the kernels is compared against."""
+    f = lambda x: None if x is None else x.double()
+    q, k = f(raw["q"]), f(raw["k"])
+    q = q / q.norm(dim=-1, keepdim=True).clamp_min(1e-6)
+    if variant != "kla":
+        k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-6)
+    sig = lambda x: None if x is None else torch.sigmoid(x.double())
+    return {
+        "q": q, "k": k, "v": f(raw["v"]), "beta": sig(raw["beta"]),
+        "log_g": None if raw["log_g"] is None else -F.softplus(raw["log_g"].double()),
+        "erase_b": sig(raw["erase_b"]), "write_w": sig(raw["write_w"]),
+    }
+
+
 def make_decode_inputs(variant: str, N: int, H: int, step: int, dk: int = 128, dv: int = 128,
                        dtype: torch.dtype = torch.bfloat16, base_seed: int = 1000) -> dict:
     """Inputs of decode step ``step`` for N sequences (seed base_seed + step); [N,H,...]."""

@@ -14,6 +14,7 @@ import torch
 from ._lib import FwdArgs, check, lib
 
 VARIANTS = {"deltanet": 0, "gdn": 1, "kda": 2, "gdn2": 3, "kla": 4}
+RAW_INPUTS = 0x100   # GDR_RAW_INPUTS (include/gdr.h)
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 CHANNEL_DECAY = ("kda", "gdn2")
 
@@ -74,15 +75,17 @@ def _stream(stream, device):
 
 def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=None,
             initial_state=None, output_final_state=True, eps=1e-6, scale=1.0, chunk=0,
-            out=None, final_state=None, stream=None):
+            out=None, final_state=None, stream=None, raw_inputs=False):
     """Gated delta-rule forward over whole sequences.
 
     q, k: [B,T,H,dk]; v: [B,T,H,dv]; bf16 or fp32 (all the same), CUDA,
     contiguous.  Gates fp32: beta [B,T,H] (eta for KLA); log_g [B,T,H]
     (gdn, kla) or [B,T,H,dk] (kda, gdn2); erase_b / write_w [B,T,H,dk] (gdn2).
     initial_state: fp32 [B,H,dk,dv] or None.  Returns (o, final_state or None).
-    ``chunk``: 0 auto, 1 per-token kernel, 64 one-kernel chunked path,
-    65 two-kernel chunked path (preparation + carry; workspace allocated here).
+    ``chunk``: 0 auto, 1 per-token kernel, 65 chunked path (preparation +
+    carry; workspace allocated here).  ``raw_inputs``: q, k, beta and the gates
+    are raw projections and logits; the kernels normalise q and k (not KLA's k)
+    and apply sigmoid / -softplus themselves (GDR_RAW_INPUTS).
     """
     vid = variant_id(variant)
     if q.dim() != 4:
@@ -118,17 +121,19 @@ def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=No
                 o=out.data_ptr())
     L = lib()
     dt = _DTYPES[q.dtype]
-    ws = L.gdr_forward_workspace_size(vid, dt, B, T, H, dk, dv, chunk)
+    vflag = vid | (RAW_INPUTS if raw_inputs else 0)
+    ws = L.gdr_forward_workspace_size(vflag, dt, B, T, H, dk, dv, chunk)
     workspace = torch.empty(ws, device=dev, dtype=torch.uint8) if ws else None
-    check(L.gdr_forward_chunked(vid, dt, B, T, H, dk, dv, ctypes.byref(a), float(eps), float(scale),
+    check(L.gdr_forward_chunked(vflag, dt, B, T, H, dk, dv, ctypes.byref(a), float(eps), float(scale),
                                 int(chunk), _ptr(workspace), ws, _stream(stream, dev)))
     return out, final_state
 
 
 def decode_step(q, k, v, state, *, variant, beta=None, log_g=None, erase_b=None, write_w=None,
-                eps=1e-6, scale=1.0, out=None, stream=None):
+                eps=1e-6, scale=1.0, out=None, stream=None, raw_inputs=False):
     """One decode token for N sequences: q, k [N,H,dk]; v [N,H,dv]; state fp32
-    [N,H,dk,dv] updated in place.  Returns o [N,H,dv]."""
+    [N,H,dk,dv] updated in place.  Returns o [N,H,dv].  ``raw_inputs`` as for
+    forward()."""
     vid = variant_id(variant)
     N, H, dk = q.shape
     dv = v.shape[-1]
@@ -145,7 +150,8 @@ def decode_step(q, k, v, state, *, variant, beta=None, log_g=None, erase_b=None,
         out = torch.empty(N, H, dv, device=dev, dtype=q.dtype)
     else:
         _need(out, "out", (N, H, dv), q.dtype, dev)
-    check(lib().gdr_decode_step(vid, _DTYPES[q.dtype], N, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+    check(lib().gdr_decode_step(vid | (RAW_INPUTS if raw_inputs else 0), _DTYPES[q.dtype], N, H, dk, dv,
+                                _ptr(q), _ptr(k), _ptr(v),
                                 _ptr(beta), _ptr(log_g), _ptr(erase_b), _ptr(write_w), _ptr(state),
                                 _ptr(out), float(eps), float(scale), _stream(stream, dev)))
     return out

@@ -34,7 +34,8 @@
  * Conventions for every entry point:
  *  - `variant`, `dtype` and the returned status are plain ints carrying the
  *    values of gdr_variant_t, gdr_dtype_t and gdr_status_t below, so that the
- *    ABI is the same for C callers and for foreign-function bindings.
+ *    ABI is the same for C callers and for foreign-function bindings; `variant`
+ *    may carry the GDR_RAW_INPUTS flag.  `stream` is a cudaStream_t.
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
  *    allocates no device memory, keeps no pointer after the call returns and
  *    never synchronises: work is enqueued on `stream` (a cudaStream_t passed as
@@ -68,6 +69,23 @@ typedef enum {
     GDR_GDN2 = 3,
     GDR_KLA = 4
 } gdr_variant_t;
+
+/*
+ * Raw-input mode: OR this flag into `variant` (of any entry point) to pass q,
+ * k, beta and the gates as raw projections and logits; the kernels then apply
+ * the input transforms on their load paths instead of the caller doing a
+ * separate elementwise pass:
+ *   q <- q / max(||q||, 1e-6) and k <- k / max(||k||, 1e-6) per (token, head)
+ *        (KLA's keys are left as they are: its Kaczmarz step
+ *        eta / (||k||^2 + eps) already carries their norm);
+ *   beta (eta for KLA), erase_b, write_w <- sigmoid of the value passed;
+ *   log_g <- -softplus of the value passed, so that g = sigmoid(-x) in (0, 1).
+ * These are the key normalisation and gate activations of the pages' layers
+ * ("Kaczmarz Linear Attention", KLA update rule: beta_t = eta_t/(||k_t||^2 +
+ * eps) with eta a gate; ablations: keys normalised), applied to the raw
+ * activations.  Shapes, dtypes and layouts are unchanged.
+ */
+#define GDR_RAW_INPUTS 0x100
 
 typedef enum {
     GDR_F32 = 0,   /* q, k, v, o in fp32 */

@@ -216,3 +216,17 @@ def test_forward_plan_binding():
     assert gdr.forward_plan("kla", 1, 65536, 16, 128, 148) == {"segments": 6, "segment_chunks": 171, "split_chunk": 0}
     with pytest.raises(gdr.GdrError):
         gdr.forward_plan("gdn", 8, 2048, 8, 96, 148)
+
+
+def test_raw_input_flag_is_accepted_everywhere(L):
+    RAW = 0x100                                      # GDR_RAW_INPUTS
+    for v in range(5):
+        assert fwd(L, variant=v | RAW, a=args()) == 4                 # validated, reaches the launch
+        assert L.gdr_forward_kernel_name(v | RAW, 1, 8, 2048, 8, 128, 128, 0).decode() == \
+            L.gdr_forward_kernel_name(v, 1, 8, 2048, 8, 128, 128, 0).decode()
+        assert L.gdr_forward_workspace_size(v | RAW, 1, 8, 2048, 8, 128, 128, 0) == \
+            L.gdr_forward_workspace_size(v, 1, 8, 2048, 8, 128, 128, 0)
+    assert fwd(L, variant=5 | RAW) == 1                               # the flag does not hide a bad variant
+    i = ctypes.c_void_p
+    assert L.gdr_decode_step(1 | RAW, 1, 4, 2, 128, 128, i(FAKE), i(FAKE), i(FAKE), i(FAKE), i(FAKE), None,
+                             None, i(FAKE), i(FAKE), 1e-6, 1.0, None) == 4

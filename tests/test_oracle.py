@@ -357,3 +357,19 @@ def test_mutants_are_caught(mutant):
         except AssertionError:
             failures += 1
     assert failures > 0, f"no pin caught mutant {mutant}: {MUTANTS[mutant]}"
+
+
+def test_raw_inputs_follow_the_recipe():
+    """inputs.make_raw_inputs draws what make_inputs draws, and transform_raw
+    applies the recipe's transforms: the two agree up to the I/O rounding."""
+    import torch
+
+    from gated_delta_rule_forward_b200.inputs import make_inputs, make_raw_inputs, transform_raw
+    for variant in ("deltanet", "gdn", "kda", "gdn2", "kla"):
+        ref = make_inputs(variant, 2, 9, 3, 128, 64, dtype=torch.float32, seed=5)
+        got = transform_raw(variant, make_raw_inputs(variant, 2, 9, 3, 128, 64, dtype=torch.float32, seed=5))
+        for name, x in ref.items():
+            if x is None:
+                assert got[name] is None, name
+                continue
+            assert torch.allclose(got[name].float(), x, rtol=1e-5, atol=1e-6), (variant, name)
