@@ -131,7 +131,7 @@ __device__ __forceinline__ size_t rec_index(const PrepParams &p, const RecIdx &x
   return (static_cast<size_t>(x.b) * p.H + x.h) * p.NC + x.c;
 }
 
-template <int VAR>
+template <int VAR, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 2)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrepParams p) {
@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   float *sc_wf = sc_g2 + 64;
   float *sc_G = sc_wf + 64;
   float *sc_tmp = sc_G + 64;
-  float *sc_rk = sc_tmp + 64;   // 1 / ||k_t||
-  float *sc_vk = sc_rk + 64;    // 1 / ||k_t|| of the keys the recurrence sees (1 for keys normalised here)
-  float *sc_qn = sc_vk + 64;    // raw-input mode: 1 / ||q_t||
+  float *sc_rk = sc_tmp + 64;   // raw-input mode: 1 / ||k_t|| (keys normalised here), else 1
+  float *sc_qn = sc_rk + 64;    // raw-input mode: 1 / ||q_t||
+  float *sc_scan = sc_qn + 64;  // per-warp prefix sums of the log decay
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
 
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const size_t th = (static_cast<size_t>(b) * p.T + t) * p.H + h;
       if constexpr (scalar_decay(VAR)) lg = __ldg(p.log_g + th);
       bt = __ldg(p.beta + th);
-      if (p.raw) {
+      if constexpr (RAW) {
         if constexpr (scalar_decay(VAR)) lg = raw_log_decay(lg);
         bt = raw_gate(bt);
       }
@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     for (int i = tid; i < 512; i += NTHREADS)
       reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
+  if (tid < 64) sc_rk[tid] = 1.f;   // rewritten per record only where keys are normalised here
   float lg_next = 0.f, bt_next = 0.f;
   if (tid < 64 && static_cast<int>(blockIdx.x) < total) load_gates(blockIdx.x, lg_next, bt_next);
   // every CTA of this persistent grid is resident from the start, so the carry
@@ -250,7 +251,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const uint32_t ph = ((r - blockIdx.x) / gridDim.x) & 1;   // phase of the input and U' barriers
     const bool more = r + static_cast<int>(gridDim.x) < total;
     uint8_t *rec = p.ws + rec_index(p, rec_idx(p, r)) * rec_bytes(NS);
-    // gates: beta_t, cumulative log2 decay, Gamma_t
+    // gates (warps 0 and 1, meeting at a 64-thread barrier): beta_t, cumulative
+    // log2 decay, Gamma_t; and, where beta is the column coefficient (no
+    // Kaczmarz step, no keys normalised here), the column factors of A, P, Kt
+    constexpr bool diag_pass = VAR == kKLA || RAW;   // the coefficient needs ||k_t||^2 from MMA1
     if (tid < 64) {
       float x = lg_next * LOG2E;
 #pragma unroll
@@ -258,21 +262,24 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         const float y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
-      sc_tmp[tid] = x;
+      sc_scan[tid] = x;
       sc_beta[tid] = bt_next;
-      if (r + static_cast<int>(gridDim.x) < total) load_gates(r + gridDim.x, lg_next, bt_next);
-    }
-    __syncthreads();
-    if (tid < 64) {
-      const float g2 = sc_tmp[tid] + (tid >= 32 ? sc_tmp[31] : 0.f);
+      if (more) load_gates(r + gridDim.x, lg_next, bt_next);
+      named_bar_sync(2, 64);
+      const float g2 = sc_scan[tid] + (tid >= 32 ? sc_scan[31] : 0.f);
       sc_g2[tid] = g2;
       sc_G[tid] = ex2(g2);
+      if constexpr (!diag_pass) {
+        named_bar_sync(2, 64);
+        sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - g2);
+        sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - g2);
+      }
     }
     if (!mbar_wait(bar_q, ph) || !mbar_wait(bar_k, ph)) bad = 1;
     else if (tid == 0) landed += 1u | (1u << 8);
     bad = __syncthreads_or(bad);
     if (bad) break;
-    if (p.raw) tile_row_inv_norms(sm + OFF_KQ + 8192, 16384, sc_qn, tid);   // read after MMA1's barrier
+    if constexpr (RAW) tile_row_inv_norms(sm + OFF_KQ + 8192, 16384, sc_qn, tid);   // read after MMA1's barrier
 
     // MMA1: [K;Q] K^T
     if (!bad && tid == 0) {
@@ -284,51 +291,45 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       mma_commit(bar_mma);
     }
-    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
 
-    // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile.
-    // The chunk algebra runs on unit keys: with khat_t = k_t / ||k_t||,
-    // beta'_t = beta_t ||k_t||^2 and v'_t = v_t / ||k_t||, the update
-    // S~ + beta_t k_t (v_t - S~^T k_t)^T equals S~ + beta'_t khat_t (v'_t - S~^T khat_t)^T,
-    // so the Gram entries are bounded by beta' and a spread of key norms does
-    // not amplify the fp16 rounding of U' and W S0 (E = U' - W S0 then carries
-    // v / ||k||, and K~, P absorb the other factor).  ||k_t||^2 is the diagonal
-    // of K K^T; the column coefficient c_r = beta'_r / ||k_r|| (beta_r ||k_r||, or
-    // eta_r ||k_r|| / (||k_r||^2 + eps) for KLA's Kaczmarz step) replaces beta_r.
+    // A (lanes 0-63) -> A^T scratch; P (lanes 64-127) -> fp16 record tile.  The
+    // column coefficient c_r is beta_r, or for KLA the Kaczmarz step
+    // eta_r / (||k_r||^2 + eps), ||k_r||^2 being the diagonal of K K^T.  In the
+    // raw-input mode the recurrence sees the unit keys khat = k / ||k|| (not
+    // for KLA): the Gram entries of the raw keys are scaled by 1/||k_t|| (row
+    // factor rk_t) and 1/||k_r|| (in c_r = beta_r / ||k_r||), and W and Kt take
+    // the same factors, so no separate normalisation pass is needed.
     if (!bad) {
       float g[32];
       tmem_ld32(tmem + lane_base + COL_G + 32 * half, g);
       const int t = row & 63;
       const int r0 = 32 * half;
-      if (quad < 2 && (t >> 5) == half) {
-        float kk = 0.f;
+      if constexpr (diag_pass) {
+        if (quad < 2 && (t >> 5) == half) {
+          float kk = 0.f;
 #pragma unroll
-        for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
-        const float rk = kk > 0.f ? rsqrtf(kk) : 0.f;
-        const float bt = sc_beta[t];
-        float c, vk = rk;
-        if constexpr (VAR == kKLA) {
-          c = (bt == 0.f) ? 0.f : bt * (kk * rk) / (kk + p.eps);   // Kaczmarz step
-        } else if (p.raw) {   // the recurrence sees the unit key k / ||k||: beta' = beta, v' = v
-          c = bt * rk;
-          vk = 1.f;
-        } else {
-          c = bt * (kk * rk);
+          for (int r = 0; r < 32; ++r) kk = (r0 + r == t) ? g[r] : kk;
+          const float bt = sc_beta[t];
+          if constexpr (VAR == kKLA) {
+            sc_beta[t] = (bt == 0.f) ? 0.f : bt / (kk + p.eps);   // Kaczmarz step
+          } else {
+            const float rk = kk > 0.f ? rsqrtf(kk) : 0.f;
+            sc_beta[t] = bt * rk;
+            sc_rk[t] = rk;
+          }
         }
-        sc_beta[t] = c;
-        sc_rk[t] = rk;
-        sc_vk[t] = vk;
+        __syncthreads();
+        if (tid < 64) {
+          sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - sc_g2[tid]);
+          sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - sc_g2[tid]);
+        }
+        __syncthreads();
       }
-      __syncthreads();
       const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
-      if (tid < 64) {
-        sc_wf[tid] = sc_beta[tid] * ex2(sc_g2[63] - sc_g2[tid]);
-        sc_tmp[tid] = sc_beta[tid] * ex2(sc_g2[tid & 32] - sc_g2[tid]);
-      }
-      __syncthreads();
       const float g2t = sc_g2[t];
       const float rowf = (t >= r0) ? ex2(g2t - sc_g2[r0]) : 0.f;
       float fac[32];
@@ -348,15 +349,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
         for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(rkt * g[r] * fac[r]) : 0.f;
       } else {
-        const float qs = p.raw ? p.scale * sc_qn[t] : p.scale;
+        const float qs = RAW ? p.scale * sc_qn[t] : p.scale;
 #pragma unroll
         for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? qs * g[r] * fac[r] : 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
       }
     }
-    tc_fence_before();
-    __syncthreads();
+    tc_fence_before();   // the tensor-memory reads above, ordered by the barrier after the conversion
 
     // Gamma_C, and the fp16 copies Qg = Diag(scale Gamma) Q and Kt = Diag(w) K
     // (2048 sixteen-byte chunks in the swizzled image of the bf16 tiles)
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint32_t off = sw128(r, j);
       float x[8];
       unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KQ + kb * 16384 + isq * 8192 + off), x);
-      const float f = isq ? p.scale * sc_G[r] * (p.raw ? sc_qn[r] : 1.f) : sc_wf[r];
+      const float f = isq ? p.scale * sc_G[r] * (RAW ? sc_qn[r] : 1.f) : sc_wf[r];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         x[e] *= f;
@@ -381,8 +381,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncthreads();
     if (tid == 0 && more) issue_q(r + gridDim.x);
 
-    // T = (I + A)^{-1}; T Diag(1/||k||) (for U' = T V'; the keys the recurrence
-    // sees) and T Diag(Gamma / ||k||) (for W = T Diag(Gamma) Khat) as bf16 tiles
+    // T = (I + A)^{-1}; T (for U' = T V) and T Diag(Gamma rk) (for W = T Diag(Gamma) K,
+    // the keys normalised in the raw-input mode) as bf16 tiles
     solve_unit_lower_64(At, Tf, tid, warp, lane);
     {
       const int m = tid >> 2, n0 = (tid & 3) * 16;
@@ -394,9 +394,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float te = (n0 + e <= m) ? tv[e] : 0.f;
-        tv[e] = te * sc_vk[n0 + e];
-        tg[e] = te * sc_G[n0 + e] * sc_rk[n0 + e];
+        tv[e] = (n0 + e <= m) ? tv[e] : 0.f;
+        tg[e] = tv[e] * sc_G[n0 + e] * sc_rk[n0 + e];
       }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -408,8 +407,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncthreads();
 
     // MMA2: W = T Diag(Gamma) K (M64 N128), then U'^T = V^T T^T (M128 over d_v,
-    // N64) on its own barrier, so that the W epilogue runs beside the U' product
-    if (!bad && tid == 0) {
+    // N64) on its own barrier, so that the W epilogue runs beside the U' product.
+    // (If thread 0's wait for V gave up, nothing is issued and every thread's
+    // wait for W gives up too.)
+    if (tid == 0) {
       if (!mbar_wait(bar_v, ph)) {
         bad = 1;
       } else {
@@ -428,9 +429,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         mma_commit(bar_u);
       }
     }
-    bad = __syncthreads_or(bad);
-    if (bad) break;
-    if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     if (bad) break;
@@ -459,7 +458,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
     }
     // U'^T (lane v = value column, columns t) -> fp16 record tile
-    if (!__all_sync(0xffffffffu, mbar_wait(bar_u, ph))) bad = 1;
+    if (tid == 0 && !mbar_wait(bar_u, ph)) bad = 1;   // one waiter; the rest sleep in the barrier
+    tc_fence_before();
+    bad = __syncthreads_or(bad);
     if (!bad) {
       tc_fence_after();
       if (tid == 0 && more) issue_v(r + gridDim.x);   // V is consumed
@@ -537,6 +538,7 @@ constexpr uint32_t COL_U = 192;   // M128 x 64: U'^T
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prepc
 
+template <bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_prep_chan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -593,7 +595,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int t = c * C + tid;
     if (t >= p.T) return 0.f;
     const float bt = __ldg(p.beta + (static_cast<size_t>(b) * p.T + t) * p.H + h);
-    return p.raw ? raw_gate(bt) : bt;
+    return RAW ? raw_gate(bt) : bt;
   };
 
   if (warp == 0) {
@@ -647,10 +649,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bad = __syncthreads_or(bad);
     if (!bad) {
       const int ch = tid & 127, hh = tid >> 7;
+      const int valid = p.T - rec_idx(p, r).c * C;   // tokens of this chunk inside the sequence
       float run = 0.f;
 #pragma unroll 8
       for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-        run += (p.raw ? raw_log_decay(Gr[t * DK + ch]) : Gr[t * DK + ch]) * LOG2E;
+        // raw-input mode: -softplus of the logit; past the sequence's end the
+        // padding decays nothing (a zero logit would decay by one half)
+        const float lg = Gr[t * DK + ch];
+        run += (RAW ? (t < valid ? raw_log_decay(lg) : 0.f) : lg) * LOG2E;
         Gr[t * DK + ch] = run;
       }
       if (hh == 0) sc_tmp[ch] = run;   // gamma at token 31
@@ -675,7 +681,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!mbar_wait(bar_kq, ph)) bad = 1;
     else if (tid == 0) landed += 1u << 8;
     bad = __syncthreads_or(bad);
-    if (p.raw && !bad) {   // unit q and k
+    if (RAW && !bad) {   // unit q and k
       tile_row_inv_norms(kq_ptr, 16384, sc_kn, tid);
       tile_row_inv_norms(kq_ptr + 8192, 16384, sc_qn, tid);
       __syncthreads();
@@ -694,7 +700,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float kx[4], qx[4];
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
-        if (p.raw) {
+        if constexpr (RAW) {
           const float kn = sc_kn[t], qn = sc_qn[t];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -743,7 +749,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    hp + kk > 0);
         mma_commit(bar_mma);
       }
-      if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+      if (tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
       bad = __syncthreads_or(bad);
       mma_phase ^= 1;
       tc_fence_after();
@@ -805,7 +811,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  idesc_bf16(128, 64, true, false), kk > 0);
       mma_commit(bar_mma);
     }
-    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
@@ -916,6 +922,7 @@ constexpr uint32_t COL_OD = 384;  // M128 x 64: (P^d V)^T
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace prepg
 
+template <bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_prep_gdn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -977,7 +984,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const size_t gi = ((static_cast<size_t>(x.b) * p.T + t0 + t) * p.H + x.h) * DK + ch0;
         ebs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.erase_b + gi));
         wrs[hp][it] = __ldg(reinterpret_cast<const float4 *>(p.write_w + gi));
-        if (p.raw) {
+        if constexpr (RAW) {
           float4 &e4 = ebs[hp][it], &w4 = wrs[hp][it];
           e4 = make_float4(raw_gate(e4.x), raw_gate(e4.y), raw_gate(e4.z), raw_gate(e4.w));
           w4 = make_float4(raw_gate(w4.x), raw_gate(w4.y), raw_gate(w4.z), raw_gate(w4.w));
@@ -1035,10 +1042,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bad = __syncthreads_or(bad);
     if (!bad) {
       const int ch = tid & 127, hh = tid >> 7;
+      const int valid = p.T - rec_idx(p, r).c * C;   // tokens of this chunk inside the sequence
       float run = 0.f;
 #pragma unroll 8
       for (int t = 32 * hh; t < 32 * hh + 32; ++t) {
-        run += (p.raw ? raw_log_decay(Gr[t * DK + ch]) : Gr[t * DK + ch]) * LOG2E;
+        // raw-input mode: -softplus of the logit; past the sequence's end the
+        // padding decays nothing (a zero logit would decay by one half)
+        const float lg = Gr[t * DK + ch];
+        run += (RAW ? (t < valid ? raw_log_decay(lg) : 0.f) : lg) * LOG2E;
         Gr[t * DK + ch] = run;
       }
       if (hh == 0) sc_tmp[ch] = run;
@@ -1062,7 +1073,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!mbar_wait(bar_kq, ph)) bad = 1;
     else if (tid == 0) landed += 1u << 8;
     bad = __syncthreads_or(bad);
-    if (p.raw && !bad) {   // unit q and k
+    if (RAW && !bad) {   // unit q and k
       tile_row_inv_norms(kq_ptr, 16384, sc_kn, tid);
       tile_row_inv_norms(kq_ptr + 8192, 16384, sc_qn, tid);
       __syncthreads();
@@ -1083,7 +1094,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float kx[4], qx[4];
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + bf), kx);
         unpack4(*reinterpret_cast<const uint2 *>(kq_ptr + hp * 16384 + 8192 + bf), qx);
-        if (p.raw) {
+        if constexpr (RAW) {
           const float kn = sc_kn[t], qn = sc_qn[t];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1140,7 +1151,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    hp + kk > 0);
         mma_commit(bar_mma);
       }
-      if (!mbar_wait(bar_mma, mma_phase)) bad = 1;
+      if (tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
       bad = __syncthreads_or(bad);
       mma_phase ^= 1;
       tc_fence_after();
@@ -1226,7 +1237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         st_chunk_f16(reinterpret_cast<uint8_t *>(chunk), x);
       }
     }
-    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
@@ -1260,7 +1271,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       mma_commit(bar_mma);
     }
-    if (!bad && !mbar_wait(bar_mma, mma_phase)) bad = 1;
+    if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
     bad = __syncthreads_or(bad);
     mma_phase ^= 1;
     tc_fence_after();
@@ -1358,16 +1369,14 @@ constexpr int NSTAGE = 3;
 constexpr int NCOMPUTE = 16;
 constexpr int NTHREADS_CARRY = (NCOMPUTE + 1) * 32;
 constexpr uint32_t STAGE = 74752;        // record image (<= 74240 bytes), 1 KB aligned
-constexpr uint32_t PART_A = REC_P;       // [-W; Qg] and Kt: the operands of Y and dS
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(STAGE % 1024 == 0 && STAGE >= rec_bytes(2) && STAGE >= rec_bytes_chan(2), "stage layout");
-static_assert(PART_A % 16 == 0 && (REC_U - REC_P) % 16 == 0, "bulk copies move 16-byte multiples");
 constexpr uint32_t COL_Y = 0;      // 2 x 128: [(-W S0)^T | (Qg S0)^T + (P E)^T], [v][t]
 constexpr uint32_t COL_DS = 256;   // 128: dS^T, [v][i]
 constexpr uint32_t COL_SA = 384;   // 64: fp16 S^T, d_k packed two per column (MMA operand)
-constexpr uint32_t COL_EA = 448;   // 2 x 32: fp16 E^T, tokens packed two per column (MMA operand), by chunk parity
+constexpr uint32_t COL_EA = 448;   // 32: fp16 E^T, tokens packed two per column (MMA operand)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 1ll << 31;   // cycles, about a second
 }  // namespace carry
@@ -1387,6 +1396,7 @@ enum CarryFlags : int {
   CARRY_NO_OUTPUT = 4,    // write no output rows
   CARRY_LAST_FINAL = 8,   // only the last segment writes s_final
   CARRY_S0_FIRST = 16,    // only segment 0 starts from s0, the others from zero
+  CARRY_FAULT_MISSING_COPY = 32,   // host fault injection (see the issuer's prologue)
 };
 
 struct CarryParams {
@@ -1405,18 +1415,28 @@ struct CarryParams {
   float *s_final_b;
   size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
-  long long wait_limit;   // cycles a wait may spin before the kernel gives up
-  int fault_chunk;        // >= 0: CTA (0, 0, 0) never copies that chunk's operands (host fault injection)
 };
 
-// Bounded wait: gives up after `limit` cycles (raising `abort`) or once another
-// thread has raised `abort`.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort, long long limit) {
+// max |x_i| over 16 values as a tree (four levels instead of a chain of 16).
+__device__ __forceinline__ float max_abs16(const float *x) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1]));
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
+
+// Bounded wait: gives up after carry::WAIT_LIMIT cycles (raising `abort`) or
+// once another warp has raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort) {
   if (mbar_try_wait(bar, phase)) return true;
   const long long start = clock64();
   while (!mbar_try_wait(bar, phase)) {
     if (*abort) return false;
-    if (clock64() - start > limit) {
+    if (clock64() - start > carry::WAIT_LIMIT) {
       *abort = 1;
       return false;
     }
@@ -1424,45 +1444,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
   return true;
 }
 
-// Barrier of the NTHREADS_CARRY threads (named barrier 1) that returns whether
-// any of them passed `bad`: every thread then takes the same branch.
-__device__ __forceinline__ bool carry_barrier_or(bool bad) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(bad ? 1u : 0u), "n"(carry::NTHREADS_CARRY)
-      : "memory");
-  return r != 0;
-}
-
 // MODE 0: scalar Gamma_C.  MODE 1: Gamma_C a vector of d_k values (channel
 // decay).  MODE 2: as 1, plus the record's (P^d V)^T and (Dt^T V)^T terms added
 // to the output and to the state (GDN-2); each compute thread loads its share
-// of them from the record (the issuer prefetches it into L2).
-//
-// 16 compute warps (thread v of warp (quad, part) owns value column v = 32 quad
-// + lane, d_k rows 32 part .. 32 part + 31 of S^T in fp32 registers, and tokens
-// 16 part .. 16 part + 15 of E^T and of the output) and one issuer warp.  Per
-// chunk c the compute warps hand over to the issuer through two barriers
-// (named barrier 1 with an OR reduction, so that a failed wait ends the sweep
-// for every warp at the same point), and the issuer's MMAs complete on
-// mbarriers the compute warps wait for:
-//     wait Y(c);  E^T = U'^T + Y_W -> tensor memory (fp16, two buffers by
-//     chunk parity, so that the second P half of chunk c-1 may still read its own) | barrier B1
-//     issuer: dS^T = E^T Kt,  first half of Y_Q += E^T P^T
-//     output rows of chunk c-1;  wait dS(c);  S^T = Gamma_C S^T + dS^T  | barrier B2
-//     issuer: copies of the next records,  Y(c+1) = S^T [-W; Qg]^T,
-//             second half of Y_Q(c) += E^T P^T
-// The P product is split around Y(c+1) so that it fills the tensor pipe while
-// the compute warps work instead of delaying the products on the state's
-// critical path.  A record is copied in two parts: [-W; Qg] and Kt (read only
-// by Y and dS) as soon as the stage's chunk has finished dS, three chunks
-// ahead; P, U'^T and Gamma_C once that chunk's last P half and output rows are
-// done, two chunks ahead.
+// of them from the record one chunk ahead.
 // 17 warps: one SM sub-partition holds five of them, so 96 registers per thread.
 template <int MODE>
 __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(const CarryParams p) {
@@ -1478,30 +1463,30 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   const int c_first = p.c_base + (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
   const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
   const bool values = !(flags & CARRY_NO_VALUES);
-  const long long limit = p.wait_limit;
-  const int fault_chunk = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.fault_chunk : -1;
 
-  uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] part A landed
-  uint64_t *bar_b = bar_a + NSTAGE;       // [NSTAGE] part B landed
-  uint64_t *bar_e = bar_b + NSTAGE;       // Y(c) done
-  uint64_t *bar_s = bar_e + 1;            // dS^T(c) (and the first P half) done
-  uint64_t *bar_o = bar_e + 2;            // Y_Q(c) complete (second P half done)
-  uint64_t *bar_drain = bar_e + 3;        // error path only
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 4);
-  volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 5);
+  uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
+  uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
+  uint64_t *bar_s = bar_e + 1;            // dS^T(c) done
+  uint64_t *bar_o = bar_e + 2;            // E^T P^T (c) done
+  uint64_t *bar_ea = bar_e + 3;           // E^T(c) in tensor memory (16 warps)
+  uint64_t *bar_sa = bar_e + 4;           // S^T in tensor memory (16 warps)
+  uint64_t *bar_done = bar_e + 5;         // chunk c's Y read and stage released (16 warps)
+  uint64_t *bar_drain = bar_e + 6;        // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 7);
+  volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 8);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < NSTAGE; ++i) {
-      mbar_init(&bar_a[i], 1);
-      mbar_init(&bar_b[i], 1);
-    }
+    for (int i = 0; i < NSTAGE; ++i) mbar_init(&bar_full[i], 1);
     mbar_init(bar_e, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_ea, NCOMPUTE);
+    mbar_init(bar_sa, NCOMPUTE);
+    mbar_init(bar_done, NCOMPUTE);
     mbar_init(bar_drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -1510,270 +1495,259 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t rb = p.rec_bytes;
-  const uint32_t part_b = p.copy_bytes - PART_A;
   // every CTA of this grid holds its SM: a preparation grid launched as this
   // grid's programmatic dependent (the pipelined sweep) may take the others
   griddep_launch_dependents();
 
-  const bool issuer = warp == NCOMPUTE;
-  const bool leader = issuer && lane == 0;
-  // issuer's view of the record copies: (part, stage) has a copy in flight, and
-  // the phase parity each part's barrier completes next
+  // issuer's view of the record copies: stage has a copy in flight / phase parity to wait for
   uint32_t pend = 0, par = 0;
   float smax = 0.f;
   float S[32];
   const int quad = warp & 3, part = (warp >> 2) & 3;
   const int v = quad * 32 + lane;
-  const bool has_v = !issuer && quad * 32 < p.dv;   // warp-uniform (d_v is 64 or 128)
+  const bool has_v = quad * 32 < p.dv;   // warp-uniform (d_v is 64 or 128)
   const uint32_t lrow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-  const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
 
-  auto copy_a = [&](int c) {   // leader: [-W; Qg] and Kt of chunk c
-    const int s = c % NSTAGE;
-    if (c == fault_chunk) return;   // injected fault: no copy and no expected bytes
-    mbar_expect_tx(&bar_a[s], PART_A);
-    bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, PART_A, &bar_a[s]);
-    pend |= 1u << s;
-  };
-  auto copy_b = [&](int c) {   // leader: P, U'^T and Gamma_C of chunk c (and the GDN-2 terms into L2)
-    const int s = c % NSTAGE;
-    mbar_expect_tx(&bar_b[s], part_b);
-    bulk_load(sm + s * STAGE + PART_A, recs + static_cast<size_t>(c) * rb + PART_A, part_b, &bar_b[s]);
-    if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
-    pend |= 1u << (NSTAGE + s);
-  };
-  // leader: wait for part A of chunk c, then Y(c) = S^T [-W; Qg]^T
-  auto issue_y = [&](int c) -> bool {
-    const int s = c % NSTAGE;
-    if (!wait_or_abort(&bar_a[s], (c / NSTAGE) & 1, abort, limit)) return false;
-    pend &= ~(1u << s);
-    par ^= 1u << s;
-    tc_fence_after();
-    const uint32_t st = smem_u32(sm + s * STAGE);
+  if (warp == NCOMPUTE) {
+    // ---------------------------------------------------------------- issuer
+    if (lane == 0) {
+      const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
+      auto issue_chunk = [&](int c) {
+        const int s = c % NSTAGE;
+        mbar_expect_tx(&bar_full[s], p.copy_bytes);
+        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, p.copy_bytes, &bar_full[s]);
+        // MODE 2: the rest of the record, which the compute threads read themselves
+        if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
+        pend |= 1u << s;
+      };
+      auto wait_full = [&](int c) -> bool {
+        const int s = c % NSTAGE;
+        if (!wait_or_abort(&bar_full[s], (c / NSTAGE) & 1, abort)) return false;
+        pend &= ~(1u << s);
+        par ^= 1u << s;
+        return true;
+      };
+      auto issue_y = [&](int c) {   // Y(c) = S^T [-W; Qg]^T
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
-             sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
-             kk > 0);
-    mma_commit(bar_e);
-    return true;
-  };
-  // leader: Y_Q(c) += E^T P^T over tokens 32 h2 .. 32 h2 + 31 of chunk c
-  auto issue_p = [&](int c, int h2) {
-    const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
+                 sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
+                 kk > 0);
+        mma_commit(bar_e);
+      };
+      griddep_wait();   // the records are the preparation kernel's output
+      // CARRY_FAULT_MISSING_COPY (host fault injection): CTA (0, 0, 0) never copies
+      // record 1 nor expects its bytes, so the waits for it give up after their limit
+      const bool inject = (flags & CARRY_FAULT_MISSING_COPY) && (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
+      for (int c = 0; c < NSTAGE && c < NC; ++c)
+        if (!(inject && c == 1)) issue_chunk(c);
+      bool ok = wait_or_abort(bar_sa, 0, abort) && wait_full(0);
+      if (ok) issue_y(0);
+      // Waits follow the order in which the compute warps arrive (done(c-1)
+      // before E(c) before S(c)), so no barrier can complete a phase the
+      // issuer has not waited for yet.
+      for (int c = 0; ok && c < NC; ++c) {
+        // chunk c-1 fully consumed: its stage takes record c+2
+        if (c >= 1) {
+          if (!(ok = wait_or_abort(bar_done, (c - 1) & 1, abort))) break;
+          if (c + 2 < NC) issue_chunk(c + 2);
+        }
+        // dS^T = E^T Kt ; Y_Q += E^T P^T
+        if (!(ok = wait_or_abort(bar_ea, c & 1, abort))) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
 #pragma unroll
-    for (int kk = 2 * h2; kk < 2 * h2 + 2; ++kk)
-      mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 32 * (c & 1) + 8 * kk,
-             sdesc(st + REC_P + kk * 32, 16, 1024),
-             idesc_f16(128, 64, false, false), 1);
-  };
-  // leader: wait for part B of chunk c (its U'^T and Gamma_C are read by the compute warps)
-  auto note_b = [&](int c) {
-    const int s = c % NSTAGE;
-    pend &= ~(1u << (NSTAGE + s));
-    par ^= 1u << (NSTAGE + s);
-  };
-
-  // ---------------------------------------------------------------- set-up
-  griddep_wait();   // the initial state and the records may be the previous grid's output
-  if (leader) {
-    for (int c = 0; c < NSTAGE && c < NC; ++c) copy_a(c);
-    for (int c = 0; c < NSTAGE - 1 && c < NC; ++c) copy_b(c);
-  }
-  auto store_state = [&]() {
-    uint32_t r[16];
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + COL_DS, tmem + COL_EA + 8 * kk, sdesc(st + REC_K + kk * 2048, 8192, 1024),
+                 idesc_f16(128, 128, false, true), kk > 0);
+        mma_commit(bar_s);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
-    tmem_st16(lrow + COL_SA + 16 * part, r);
-    tmem_wait_st();
-  };
-  if (!issuer) {
-    const size_t base = (static_cast<size_t>(b) * p.H + h) * p.s0_bh_stride + static_cast<size_t>(32 * part) * p.dv + v;
-    const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
-             : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
-    store_state();
-  }
-  tc_fence_before();
-  bool bad = carry_barrier_or(false);
-  if (leader && NC > 0 && !issue_y(0)) bad = true;
-
-  // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
-  // loaded from L2 shortly before their use
-  uint4 od_raw[2], sd_raw[4];
-  auto local_terms = [&](int c) { return recs + static_cast<size_t>(c) * rb + p.copy_bytes; };
-  auto load_sd = [&](int c) {
-    const uint4 *sd = reinterpret_cast<const uint4 *>(local_terms(c) + 8192 * NS + v * 256 + part * 64);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) sd_raw[j] = (has_v && values) ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  auto load_od = [&](int c) {
-    const uint4 *od = reinterpret_cast<const uint4 *>(local_terms(c) + v * 128 + part * 32);
-#pragma unroll
-    for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  // output rows of chunk c: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
-  // through this warp's 1 KB of the stage's (consumed) U'^T tile into 16-byte stores
-  auto output_rows = [&](int c) -> bool {
-    const bool ok = __all_sync(0xffffffffu, wait_or_abort(bar_o, c & 1, abort, limit));
-    if (!ok) return false;
-    tc_fence_after();
-    float yo[16];
-    tmem_ld16(lrow + COL_Y + 128 * (c & 1) + 64 + 16 * part, yo);
-    tmem_wait_ld();
-    if constexpr (MODE == 2) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const __half2 *hp = reinterpret_cast<const __half2 *>(&od_raw[j]);
-#pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
-          const float2 f = __half22float2(hp[q2]);
-          yo[8 * j + 2 * q2] += f.x;
-          yo[8 * j + 2 * q2 + 1] += f.y;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 8 * kk, sdesc(st + REC_P + kk * 32, 16, 1024),
+                 idesc_f16(128, 64, false, false), 1);
+        mma_commit(bar_o);
+        if (c + 1 < NC) {
+          if (!(ok = wait_or_abort(bar_sa, (c + 1) & 1, abort) && wait_full(c + 1))) break;
+          issue_y(c + 1);
         }
       }
     }
-    if (has_v && !(flags & CARRY_NO_OUTPUT)) {
-      uint8_t *tile = sm + (c % NSTAGE) * STAGE + REC_U + (quad * 4 + part) * 1024;
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    griddep_wait();   // the initial state and the records may be the previous grid's output
+    {
+      const size_t base = (static_cast<size_t>(b) * p.H + h) * p.s0_bh_stride + static_cast<size_t>(32 * part) * p.dv + v;
+      const bool from_s0 = !pass_b && p.s0 != nullptr && has_v && (zi == 0 || !(flags & CARRY_S0_FIRST));
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
-        *reinterpret_cast<__nv_bfloat16 *>(tile + m * 64 + lane * 2) = __float2bfloat16_rn(yo[m]);
-      __syncwarp();
-#pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
-        const int t = (c_first + c) * C + 16 * part + tr;
-        const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
-        if (t < p.T)
-          *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
-                                     8 * piece) = val;
-      }
-      fence_async_smem();   // the next copy into this stage is an async-proxy write
+      for (int k = 0; k < 32; ++k)
+        S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
+               : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
     }
-    return true;
-  };
+    auto store_state = [&]() {
+      uint32_t r[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
+      tmem_st16(lrow + COL_SA + 16 * part, r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sa);
+    };
+    store_state();
+    // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
+    // each loaded from L2 (the issuer prefetches records there) just before the wait that
+    // precedes its use; short live ranges keep them out of local memory, where a pending
+    // load would stall its spill store
+    uint4 od_raw[2], sd_raw[4];
+    auto local_terms = [&](int c) {
+      return p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first + c) * rb + p.copy_bytes;
+    };
+    auto load_sd = [&](int c) {
+      const uint4 *sd = reinterpret_cast<const uint4 *>(local_terms(c) + 8192 * NS + v * 256 + part * 64);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sd_raw[j] = (has_v && values) ? __ldg(sd + j) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto load_od = [&](int c) {
+      const uint4 *od = reinterpret_cast<const uint4 *>(local_terms(c) + v * 128 + part * 32);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    for (int c = 0; c < NC; ++c) {
+      uint8_t *st = sm + (c % NSTAGE) * STAGE;
+      const uint32_t y = lrow + COL_Y + 128 * (c & 1);
 
-  // ---------------------------------------------------------------- sweep
-  for (int c = 0; c < NC; ++c) {
-    const int s = c % NSTAGE;
-    uint8_t *st = sm + s * STAGE;
-    if (!issuer) {
-      // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15
-      bad = !__all_sync(0xffffffffu, wait_or_abort(&bar_b[s], (c / NSTAGE) & 1, abort, limit) &&
-                                         wait_or_abort(bar_e, c & 1, abort, limit));
-      if (!bad) {
-        tc_fence_after();
+      // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15; U'^T is read from the
+      // stage before Y(c) is waited for
+      bool ok = wait_or_abort(&bar_full[c % NSTAGE], (c / NSTAGE) & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      uint4 u_raw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+      if (has_v && values) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) u_raw[j] = *reinterpret_cast<const uint4 *>(st + REC_U + sw128(v, 2 * part + j));
+      }
+      ok = wait_or_abort(bar_e, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
         float e[16];
-        tmem_ld16(lrow + COL_Y + 128 * (c & 1) + 16 * part, e);
+        tmem_ld16(y + 16 * part, e);
         tmem_wait_ld();
-        if (has_v && values) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(st + REC_U + sw128(v, 2 * part + j));
-            const __half2 *hp = reinterpret_cast<const __half2 *>(&raw);
+        for (int j = 0; j < 2; ++j) {
+          const __half2 *hp = reinterpret_cast<const __half2 *>(&u_raw[j]);
 #pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              const float2 f = __half22float2(hp[q2]);
-              e[8 * j + 2 * q2] += f.x;
-              e[8 * j + 2 * q2 + 1] += f.y;
-            }
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 f = __half22float2(hp[q2]);
+            e[8 * j + 2 * q2] += f.x;
+            e[8 * j + 2 * q2 + 1] += f.y;
           }
         }
         uint32_t r[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          smax = fmaxf(smax, fmaxf(fabsf(e[2 * m]), fabsf(e[2 * m + 1])));
-          r[m] = pack_f16x2(e[2 * m], e[2 * m + 1]);
-        }
-        tmem_st8(lrow + COL_EA + 32 * (c & 1) + 8 * part, r);
+        for (int m = 0; m < 8; ++m) r[m] = pack_f16x2(e[2 * m], e[2 * m + 1]);
+        tmem_st8(lrow + COL_EA + 8 * part, r);
         tmem_wait_st();
-        if constexpr (MODE == 2) load_sd(c);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ea);
+        smax = fmaxf(smax, max_abs16(e));   // the range check, after the hand-off
       }
-    }
-    tc_fence_before();
-    bad = carry_barrier_or(bad);   // B1: E^T(c) in tensor memory
-    if (bad) break;
+      if constexpr (MODE == 2) load_sd(c);
 
-    if (leader) {
-      note_b(c);   // every compute warp observed part B of chunk c before B1
-      // dS^T = E^T Kt ; first half of Y_Q(c) += E^T P^T
+      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row
+      // for channel decay)
+      ok = wait_or_abort(bar_s, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const uint32_t sa = smem_u32(st);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tmem + COL_DS, tmem + COL_EA + 32 * (c & 1) + 8 * kk, sdesc(sa + REC_K + kk * 2048, 8192, 1024),
-               idesc_f16(128, 128, false, true), kk > 0);
-      mma_commit(bar_s);
-      issue_p(c, 0);
-    }
-    if (!issuer) {
-      // output rows of the previous chunk while dS(c) runs
-      if (c >= 1 && !output_rows(c - 1)) bad = true;
-      // S^T = Gamma_C S^T + dS^T, d_k rows 32 part .. 32 part + 31 (Gamma_C per row for channel decay)
-      if (!bad) bad = !__all_sync(0xffffffffu, wait_or_abort(bar_s, c & 1, abort, limit));
-      if (!bad) {
-        tc_fence_after();
+      {
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
+        float d0[16], d1[16];
+        tmem_ld16(lrow + COL_DS + 32 * part, d0);
+        tmem_ld16(lrow + COL_DS + 32 * part + 16, d1);
+        tmem_wait_ld();
+        if constexpr (MODE == 2) {
 #pragma unroll
-        for (int hv = 0; hv < 2; ++hv) {   // two halves of 16 rows keep the register count down
-          float d[16];
-          tmem_ld16(lrow + COL_DS + 32 * part + 16 * hv, d);
-          tmem_wait_ld();
-          if constexpr (MODE == 2) {
+          for (int j = 0; j < 4; ++j) {
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[j]);
+            float *d = j < 2 ? d0 : d1;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[2 * hv + j]);
-#pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                const float2 f = __half22float2(hp[q2]);
-                d[8 * j + 2 * q2] += f.x;
-                d[8 * j + 2 * q2 + 1] += f.y;
-              }
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __half22float2(hp[q2]);
+              d[8 * (j & 1) + 2 * q2] += f.x;
+              d[8 * (j & 1) + 2 * q2 + 1] += f.y;
             }
           }
+        }
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int i = 16 * hv + m;
-            S[i] = fmaf(gcv[CHAN ? i : 0], S[i], d[m]);
-            smax = fmaxf(smax, fabsf(S[i]));
-          }
+        for (int m = 0; m < 16; ++m) {
+          S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d0[m]);
+          S[16 + m] = fmaf(gcv[CHAN ? 16 + m : 0], S[16 + m], d1[m]);
         }
         store_state();
+        smax = fmaxf(smax, fmaxf(max_abs16(S), max_abs16(S + 16)));   // after the hand-off
         if constexpr (MODE == 2) load_od(c);
       }
-    }
-    tc_fence_before();
-    bad = carry_barrier_or(bad);   // B2: S^T in tensor memory; chunk c-1 fully consumed
-    if (bad) break;
 
-    if (leader) {
-      // stage (c+2) % NSTAGE held chunk c-1, whose P and output rows are done;
-      // stage c % NSTAGE's part A is consumed (Y(c) and dS(c) are done)
-      if (c + 2 < NC) copy_b(c + 2);
-      if (c + NSTAGE < NC) copy_a(c + NSTAGE);
-      if (c + 1 < NC && !issue_y(c + 1)) bad = true;   // raises `abort`; every warp stops at B1
-      issue_p(c, 1);
-      mma_commit(bar_o);
+      // output rows: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
+      // through this warp's 1 KB of the stage's (now unused) U'^T tile into 16-byte stores
+      ok = wait_or_abort(bar_o, c & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
+        float yo[16];
+        tmem_ld16(y + 64 + 16 * part, yo);
+        tmem_wait_ld();
+        if constexpr (MODE == 2) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const __half2 *hp = reinterpret_cast<const __half2 *>(&od_raw[j]);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __half22float2(hp[q2]);
+              yo[8 * j + 2 * q2] += f.x;
+              yo[8 * j + 2 * q2 + 1] += f.y;
+            }
+          }
+        }
+        if (has_v && !(flags & CARRY_NO_OUTPUT)) {
+          uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            *reinterpret_cast<__nv_bfloat16 *>(tile + m * 64 + lane * 2) = __float2bfloat16_rn(yo[m]);
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const int q = it * 32 + lane, tr = q >> 2, piece = q & 3;
+            const int t = (c_first + c) * C + 16 * part + tr;
+            const uint4 val = *reinterpret_cast<const uint4 *>(tile + tr * 64 + piece * 16);
+            if (t < p.T)
+              *reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * p.dv + 32 * quad +
+                                         8 * piece) = val;
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_done);
+      }
     }
   }
-  // output rows of the last chunk
-  if (!bad && !issuer && NC > 0 && !output_rows(NC - 1)) bad = true;
 
   __syncthreads();
   const bool failed = *abort != 0;
   if (failed) {
     // a wait gave up: report it, then let the MMAs and copies in flight
     // finish (each wait again bounded) before tensor memory is released
-    if (leader) {
+    if (warp == NCOMPUTE && lane == 0) {
       atomicOr(&g_gdr_split_error, 1);
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0);
-      for (int i = 0; i < 2 * NSTAGE; ++i)
-        if (pend >> i & 1u) mbar_wait(i < NSTAGE ? &bar_a[i] : &bar_b[i - NSTAGE], par >> i & 1u);
+      for (int s = 0; s < NSTAGE; ++s)
+        if (pend >> s & 1u) mbar_wait(&bar_full[s], par >> s & 1u);
     }
-  } else if (!issuer) {
+  } else if (warp < NCOMPUTE) {
     if (smax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
     const bool write_final = !(flags & CARRY_LAST_FINAL) || zi + 1 == p.z_split;
     float *sf = pass_b ? p.s_final_b : p.s_final;
@@ -1820,11 +1794,12 @@ cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 template <int VAR>
 cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
                         std::string *err) {
-  cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.raw ? chunk_prep_kernel<VAR, true> : chunk_prep_kernel<VAR, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
   // all of the unified L1 as shared memory, so that two preparation CTAs fit on an SM
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_prep_kernel<VAR>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) {
     *err = "cudaFuncSetAttribute: ";
@@ -1846,7 +1821,7 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_prep_kernel<VAR>, NTHREADS, prep::SMEM_BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTHREADS, prep::SMEM_BYTES);
   if (e != cudaSuccess) {
     *err = "occupancy query: ";
     return e;
@@ -1858,7 +1833,7 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
   if (rg.sms > 0) sms = std::min(sms, rg.sms);
   const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
   const int grid = static_cast<int>(std::min<long long>(records, static_cast<long long>(std::max(per_sm, 2)) * sms));
-  e = launch_maybe_pdl(chunk_prep_kernel<VAR>, dim3(grid), dim3(NTHREADS), prep::SMEM_BYTES, stream, rg.after_carry,
+  e = launch_maybe_pdl(kern, dim3(grid), dim3(NTHREADS), prep::SMEM_BYTES, stream, rg.after_carry,
                        mq, mk, mv, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
@@ -1866,7 +1841,8 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
 
 cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
                              std::string *err) {
-  cudaError_t e = cudaFuncSetAttribute(chunk_prep_gdn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.raw ? chunk_prep_gdn2_kernel<true> : chunk_prep_gdn2_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prepg::SMEM_BYTES);
   if (e != cudaSuccess) {
     *err = "cudaFuncSetAttribute: ";
@@ -1893,7 +1869,7 @@ cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, const Pre
   if (rg.sms > 0) sms = std::min(sms, rg.sms);
   const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
   const int grid = static_cast<int>(std::min<long long>(records, sms));   // one CTA per SM, persistent
-  e = launch_maybe_pdl(chunk_prep_gdn2_kernel, dim3(grid), dim3(NTHREADS), prepg::SMEM_BYTES, stream,
+  e = launch_maybe_pdl(kern, dim3(grid), dim3(NTHREADS), prepg::SMEM_BYTES, stream,
                        rg.after_carry, mq, mk, mv, mg, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
@@ -1901,7 +1877,8 @@ cudaError_t launch_prep_gdn2(const FwdProblem &p, int NC, uint8_t *ws, const Pre
 
 cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, const PrepRange &rg, cudaStream_t stream,
                              std::string *err) {
-  cudaError_t e = cudaFuncSetAttribute(chunk_prep_chan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.raw ? chunk_prep_chan_kernel<true> : chunk_prep_chan_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prepc::SMEM_BYTES);
   if (e != cudaSuccess) {
     *err = "cudaFuncSetAttribute: ";
@@ -1928,7 +1905,7 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, const Pre
   if (rg.sms > 0) sms = std::min(sms, rg.sms);
   const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
   const int grid = static_cast<int>(std::min<long long>(records, sms));   // one CTA per SM, persistent
-  e = launch_maybe_pdl(chunk_prep_chan_kernel, dim3(grid), dim3(NTHREADS), prepc::SMEM_BYTES, stream,
+  e = launch_maybe_pdl(kern, dim3(grid), dim3(NTHREADS), prepc::SMEM_BYTES, stream,
                        rg.after_carry, mq, mk, mv, mg, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
   return e;
@@ -2020,11 +1997,13 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
   // GDR_FAULT=wait (host-side fault injection for the failure-path tests): CTA
-  // (0, 0, 0) never copies chunk 1's operands, and waits give up after 2^20 cycles.
+  // (0, 0, 0) never copies chunk 1's record, so its waits give up after their
+  // limit (about a second).
   const char *fault = std::getenv("GDR_FAULT");
-  const bool inject = fault != nullptr && std::strcmp(fault, "wait") == 0;
-  cp.wait_limit = inject ? (1ll << 20) : carry::WAIT_LIMIT;
-  cp.fault_chunk = inject ? 1 : -1;
+  if (fault != nullptr && std::strcmp(fault, "wait") == 0) {
+    cp.flags |= CARRY_FAULT_MISSING_COPY;
+    cp.flags_b |= CARRY_FAULT_MISSING_COPY;
+  }
   e = launch_maybe_pdl(chunk_carry_kernel<MODE>, dim3(p.H, p.B, l.segments + l.segments_b),
                        dim3(carry::NTHREADS_CARRY), carry::SMEM_BYTES, stream, pdl, cp);
   if (e != cudaSuccess) *err = "carry launch: ";

@@ -8,9 +8,9 @@ gdr_device_status() reads after synchronising the stream:
   scaled by 1e5.
 * GDR_ERR_TIMEOUT: a bounded wait inside a kernel gave up.  Made here by
   host-side fault injection (GDR_FAULT=wait): the carry kernel's first CTA
-  never issues the copy of one record (nor expects its bytes), and its waits
-  give up after 2^20 cycles instead of about a second; the kernel then drains
-  its own MMAs and copies, frees its tensor memory and returns.
+  never issues the copy of one record (nor expects its bytes), so its waits
+  give up after their limit (about a second); the kernel then drains its own
+  MMAs and copies, frees its tensor memory and returns.
 
 In both cases the kernel returns normally, the status is reported once (the
 word is cleared when read), and the next call on the same context computes
