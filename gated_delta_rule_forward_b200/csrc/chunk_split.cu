@@ -1663,27 +1663,35 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       tc_fence_after();
       {
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
-        float d0[16], d1[16];
-        tmem_ld16(lrow + COL_DS + 32 * part, d0);
-        tmem_ld16(lrow + COL_DS + 32 * part + 16, d1);
-        tmem_wait_ld();
-        if constexpr (MODE == 2) {
+        if constexpr (MODE < 2) {   // both halves of dS^T in one wait
+          float d0[16], d1[16];
+          tmem_ld16(lrow + COL_DS + 32 * part, d0);
+          tmem_ld16(lrow + COL_DS + 32 * part + 16, d1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[j]);
-            float *d = j < 2 ? d0 : d1;
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              const float2 f = __half22float2(hp[q2]);
-              d[8 * (j & 1) + 2 * q2] += f.x;
-              d[8 * (j & 1) + 2 * q2 + 1] += f.y;
-            }
+          for (int m = 0; m < 16; ++m) {
+            S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d0[m]);
+            S[16 + m] = fmaf(gcv[CHAN ? 16 + m : 0], S[16 + m], d1[m]);
           }
-        }
+        } else {   // GDN-2: two halves of 16 rows keep its extra terms in registers
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d0[m]);
-          S[16 + m] = fmaf(gcv[CHAN ? 16 + m : 0], S[16 + m], d1[m]);
+          for (int hv = 0; hv < 2; ++hv) {
+            float d[16];
+            tmem_ld16(lrow + COL_DS + 32 * part + 16 * hv, d);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const __half2 *hp = reinterpret_cast<const __half2 *>(&sd_raw[2 * hv + j]);
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const float2 f = __half22float2(hp[q2]);
+                d[8 * j + 2 * q2] += f.x;
+                d[8 * j + 2 * q2 + 1] += f.y;
+              }
+            }
+#pragma unroll
+            for (int m = 0; m < 16; ++m) S[16 * hv + m] = fmaf(gcv[16 * hv + m], S[16 * hv + m], d[m]);
+          }
         }
         store_state();
         smax = fmaxf(smax, fmaxf(max_abs16(S), max_abs16(S + 16)));   // after the hand-off
