@@ -92,21 +92,31 @@ __host__ __device__ constexpr uint32_t rec_bytes_chan(int ns) { return rec_sc(ns
 __host__ __device__ constexpr uint32_t rec_bytes_gdn2(int ns) { return rec_bytes_chan(ns) + 24576 * ns; }
 
 // ------------------------------------------------------------------ preparation kernel
+// Three CTAs share an SM (72 KB of shared memory, 128 tensor-memory columns
+// and at most 80 registers a thread each), so buffers are reused by phase:
+//   Q slots: Q, then (once the Qg conversion has read it) this record's V;
+//   A^T scratch: A for the solve, then the bf16 tiles T and T Diag(Gamma rk);
+//   T scratch: fp32 T from the solve, then the staging image of -W, which a
+//   bulk copy writes to the record.
 namespace prep {
-constexpr uint32_t OFF_KQ = 0;          // bf16 [Kb0 | Qb0 | Kb1 | Qb1] (TMA)
-constexpr uint32_t OFF_V = 32768;       // bf16 V, one 8 KB box per value slice (TMA)
-constexpr uint32_t OFF_A = 49152;       // fp32 A^T, 64 x LD
-constexpr uint32_t OFF_TF = OFF_A + 64 * LD * 4;
-constexpr uint32_t OFF_T = 86016;       // bf16 T
-constexpr uint32_t OFF_TP = 94208;      // bf16 T Diag(Gamma)
-constexpr uint32_t OFF_SC = 102400;     // scalars: 8 x 64 floats
+constexpr int CTAS_PER_SM = 3;
+constexpr uint32_t OFF_KQ = 0;          // bf16 [Kb0 | Qb0 | Kb1 | Qb1] (TMA); V lands in the Q slots
+constexpr uint32_t OFF_V = OFF_KQ + 8192;   // V slice sl at OFF_V + 16384 sl (the Q slots)
+constexpr uint32_t OFF_A = 32768;       // fp32 A^T, 64 x LD
+constexpr uint32_t OFF_T = OFF_A;       // after the solve: bf16 T
+constexpr uint32_t OFF_TP = OFF_A + 8192;   // after the solve: bf16 T Diag(Gamma rk)
+constexpr uint32_t OFF_TF = OFF_A + 64 * LD * 4;   // fp32 T, 64 x LD
+constexpr uint32_t OFF_WS = OFF_TF;     // after the T tiles: fp16 -W image [atom 0 | atom 1], 16 KB
+constexpr uint32_t OFF_SC = OFF_TF + 64 * LD * 4;   // scalars: 8 x 64 floats
 constexpr uint32_t OFF_BAR = OFF_SC + 8 * 64 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
-static_assert(OFF_TF + 64 * LD * 4 <= OFF_T, "layout");
-constexpr uint32_t COL_G = 0;     // M128 x 64 (dead before W)
-constexpr uint32_t COL_W = 0;     // M64 x 128
-constexpr uint32_t COL_U = 128;   // M128 x 64: U'^T
-constexpr uint32_t TMEM_COLS = 256;
+static_assert(OFF_TP + 8192 <= OFF_TF && 16384 <= 64 * LD * 4, "phase reuse");
+static_assert(OFF_A % 1024 == 0 && OFF_TP % 1024 == 0 && OFF_WS % 1024 == 0, "tile alignment");
+static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 233472, "three CTAs per SM");
+constexpr uint32_t COL_G = 0;     // M128 x 64: [K; Q] K^T (dead before W)
+constexpr uint32_t COL_W = 0;     // M128 x 64: W^T (lane = d_k channel, columns t)
+constexpr uint32_t COL_U = 64;    // M128 x 64: U'^T (lane = value column, columns t)
+constexpr uint32_t TMEM_COLS = 128;
 }  // namespace prep
 
 struct PrepParams {
@@ -132,7 +142,7 @@ __device__ __forceinline__ size_t rec_index(const PrepParams &p, const RecIdx &x
 }
 
 template <int VAR, bool RAW>
-__global__ void __launch_bounds__(NTHREADS, 2)
+__global__ void __launch_bounds__(NTHREADS, prep::CTAS_PER_SM)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrepParams p) {
   using namespace prep;
@@ -147,10 +157,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   uint64_t *bar_q = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // Q landed
   uint64_t *bar_k = bar_q + 1;          // K landed
   uint64_t *bar_v = bar_q + 2;          // V landed
-  uint64_t *bar_mma = bar_q + 3;        // MMA1, then W
-  uint64_t *bar_u = bar_q + 4;          // U'^T
-  uint64_t *bar_drain = bar_q + 5;      // error path only
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_q + 6);
+  uint64_t *bar_mma = bar_q + 3;        // MMA1, then MMA2 (W^T and U'^T)
+  uint64_t *bar_drain = bar_q + 4;      // error path only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_q + 5);
   float *sc_beta = reinterpret_cast<float *>(sm + OFF_SC);
   float *sc_g2 = sc_beta + 64;
   float *sc_wf = sc_g2 + 64;
@@ -162,9 +171,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   float *At = reinterpret_cast<float *>(sm + OFF_A);
   float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
 
-  // TMA loads of record r's Q, K and V (thread 0), each on its own barrier so
-  // that each is issued as soon as the previous record no longer reads it:
-  // Q after the Qg conversion, K after W, V after U'.
+  // TMA loads of record r's Q, K and V (thread 0), each on its own barrier:
+  // the next record's Q and K once MMA2 has read this record's K and V (V sits
+  // in the Q slots), this record's V once its Qg conversion has read Q.
   uint32_t issued = 0, landed = 0;   // thread 0: loads issued / seen landing (q | k << 8 | v << 16)
   auto issue_q = [&](int r) {
     const RecIdx x = rec_idx(p, r);
@@ -183,7 +192,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   auto issue_v = [&](int r) {
     const RecIdx x = rec_idx(p, r);
     mbar_expect_tx(bar_v, NS * 8192);
-    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 8192, &tm_v, bar_v, 64 * sl, x.h, x.c * C, x.b);
+    for (int sl = 0; sl < NS; ++sl) tma_load_4d(sm + OFF_V + sl * 16384, &tm_v, bar_v, 64 * sl, x.h, x.c * C, x.b);
     issued += 1u << 16;
   };
   // log decay and beta of token `tid` of record r (threads 0-63)
@@ -213,7 +222,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
-    mbar_init(bar_u, 1);
     mbar_init(bar_drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q);
@@ -222,12 +230,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (static_cast<int>(blockIdx.x) < total) {
       issue_q(blockIdx.x);
       issue_k(blockIdx.x);
-      issue_v(blockIdx.x);
     }
-  }
-  if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
-    for (int i = tid; i < 512; i += NTHREADS)
-      reinterpret_cast<uint4 *>(sm + OFF_V + 8192)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (tid < 64) sc_rk[tid] = 1.f;   // rewritten per record only where keys are normalised here
   float lg_next = 0.f, bt_next = 0.f;
@@ -331,30 +334,24 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       const bool fast = sc_g2[0] - sc_g2[63] < 120.f;
       const float g2t = sc_g2[t];
+      // column factor of entry (t, r0 + r): c_r Gamma_t / Gamma_r, factored
+      // through the block's first column where the decay range allows it
       const float rowf = (t >= r0) ? ex2(g2t - sc_g2[r0]) : 0.f;
-      float fac[32];
-      if (fast) {
+      auto emit = [&](auto fac) {
+        if (quad < 2) {
+          const float rkt = sc_rk[t];
 #pragma unroll
-        for (int r4 = 0; r4 < 32; r4 += 4) {
-          const float4 cb = *reinterpret_cast<const float4 *>(sc_tmp + r0 + r4);
-          fac[r4 + 0] = cb.x * rowf; fac[r4 + 1] = cb.y * rowf;
-          fac[r4 + 2] = cb.z * rowf; fac[r4 + 3] = cb.w * rowf;
+          for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(rkt * g[r] * fac(r)) : 0.f;
+        } else {
+          const float qs = RAW ? p.scale * sc_qn[t] : p.scale;
+#pragma unroll
+          for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? qs * g[r] * fac(r) : 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
         }
-      } else {
-#pragma unroll
-        for (int r = 0; r < 32; ++r) fac[r] = sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]);
-      }
-      if (quad < 2) {
-        const float rkt = sc_rk[t];
-#pragma unroll
-        for (int r = 0; r < 32; ++r) At[(r0 + r) * LD + t] = (r0 + r < t) ? tf32r(rkt * g[r] * fac[r]) : 0.f;
-      } else {
-        const float qs = RAW ? p.scale * sc_qn[t] : p.scale;
-#pragma unroll
-        for (int r = 0; r < 32; ++r) g[r] = (r0 + r <= t) ? qs * g[r] * fac[r] : 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_P + sw128(t, 4 * half + j), g + 8 * j);
-      }
+      };
+      if (fast) emit([&](int r) { return sc_tmp[r0 + r] * rowf; });
+      else emit([&](int r) { return sc_beta[r0 + r] * ex2(g2t - sc_g2[r0 + r]); });
     }
     tc_fence_before();   // the tensor-memory reads above, ordered by the barrier after the conversion
 
@@ -377,9 +374,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       st_chunk_f16(rec + (isq ? REC_WQ + kb * 16384 + 8192 : REC_K + kb * 8192) + off, x);
     }
-    // Q is consumed: the next record's Q lands during the solve
+    // Q is consumed: this record's V lands in its slots during the solve.  The
+    // previous record's -W bulk copy must have read the T scratch before the
+    // solve writes it.
+    if (tid == 0) bulk_wait_read();
     __syncthreads();
-    if (tid == 0 && more) issue_q(r + gridDim.x);
+    if (tid == 0) issue_v(r);
+    if (NS == 1) {   // d_v = 64: the transposed U' product reads a 128-row V operand
+      for (int i = tid; i < 512; i += NTHREADS)
+        reinterpret_cast<uint4 *>(sm + OFF_V + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
 
     // T = (I + A)^{-1}; T (for U' = T V) and T Diag(Gamma rk) (for W = T Diag(Gamma) K,
     // the keys normalised in the raw-input mode) as bf16 tiles
@@ -406,10 +410,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     fence_async_smem();
     __syncthreads();
 
-    // MMA2: W = T Diag(Gamma) K (M64 N128), then U'^T = V^T T^T (M128 over d_v,
-    // N64) on its own barrier, so that the W epilogue runs beside the U' product.
-    // (If thread 0's wait for V gave up, nothing is issued and every thread's
-    // wait for W gives up too.)
+    // MMA2: W^T = K^T (T Diag(Gamma rk))^T (M128 over d_k, N64) and U'^T = V^T T^T
+    // (M128 over d_v, N64), both with the d_k / d_v operand MN-major
     if (tid == 0) {
       if (!mbar_wait(bar_v, ph)) {
         bad = 1;
@@ -419,14 +421,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         const uint32_t tp = smem_u32(sm + OFF_TP), tt = smem_u32(sm + OFF_T), vt = smem_u32(sm + OFF_V);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + COL_W, sdesc(tp + kk * 32, 16, 1024), sdesc(kq + kk * 2048, 16384, 1024),
-                 idesc_bf16(64, 128, false, true), kk > 0);
-        mma_commit(bar_mma);
+          mma_ss(tmem + COL_W, sdesc(kq + kk * 2048, 16384, 1024), sdesc(tp + kk * 32, 16, 1024),
+                 idesc_bf16(128, 64, true, false), kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 8192, 1024), sdesc(tt + kk * 32, 16, 1024),
+          mma_ss(tmem + COL_U, sdesc(vt + kk * 2048, 16384, 1024), sdesc(tt + kk * 32, 16, 1024),
                  idesc_bf16(128, 64, true, false), kk > 0);
-        mma_commit(bar_u);
+        mma_commit(bar_mma);
       }
     }
     if (!bad && tid == 0 && !mbar_wait(bar_mma, mma_phase)) bad = 1;   // one waiter; the rest sleep in the barrier
@@ -434,37 +435,25 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     mma_phase ^= 1;
     if (bad) break;
     tc_fence_after();
-    // K is consumed: the next record's K lands during the epilogues
-    if (tid == 0 && more) issue_k(r + gridDim.x);
+    // K and V (in the Q slots) are consumed: the next record's Q and K land during the epilogues
+    if (tid == 0 && more) {
+      issue_q(r + gridDim.x);
+      issue_k(r + gridDim.x);
+    }
 
-    // -W (M64 layout: rows 16 quad + lane, lane < 16; column half `half` is d_k
-    // atom `half`) -> fp16 record tile
+    // -W^T (lane = d_k channel i, tokens 32 half ..) -> the staging image of the
+    // record's -W tile (rows t, 64-channel atoms, 128-byte swizzle); U'^T (lane v =
+    // value column, columns t) -> fp16 record tile
     wmax = fmaxf(wmax, qkmax);
     {
       float w[32];
+      tmem_ld32(tmem + lane_base + COL_W + 32 * half, w);
+      uint8_t *ws = sm + OFF_WS + (row >> 6) * 8192 + (row & 7) * 2;
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tmem + lane_base + COL_W + 64 * half + 32 * part, w);
-        if (lane < 16) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            wmax = fmaxf(wmax, fabsf(w[e]));
-            w[e] = -w[e];
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_chunk_f16(rec + REC_WQ + half * 16384 + sw128(quad * 16 + lane, 4 * part + j), w + 8 * j);
-        }
+      for (int e = 0; e < 32; ++e) {
+        wmax = fmaxf(wmax, fabsf(w[e]));
+        *reinterpret_cast<__half *>(ws + sw128(32 * half + e, (row & 63) >> 3)) = __float2half_rn(-w[e]);
       }
-    }
-    // U'^T (lane v = value column, columns t) -> fp16 record tile
-    if (tid == 0 && !mbar_wait(bar_u, ph)) bad = 1;   // one waiter; the rest sleep in the barrier
-    tc_fence_before();
-    bad = __syncthreads_or(bad);
-    if (!bad) {
-      tc_fence_after();
-      if (tid == 0 && more) issue_v(r + gridDim.x);   // V is consumed
-      float w[32];
       tmem_ld32(tmem + lane_base + COL_U + 32 * half, w);
       if (row < p.dv) {
 #pragma unroll
@@ -473,10 +462,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int j = 0; j < 4; ++j) st_chunk_f16(rec + REC_U + sw128(row, 4 * half + j), w + 8 * j);
       }
     }
-    // tensor-memory reads done before the next record's MMA1
+    // tensor-memory reads done before the next record's MMA1; the -W image to the record
+    fence_async_smem();
     tc_fence_before();
     bad = __syncthreads_or(bad);
     if (bad) break;
+    if (tid == 0) {
+      bulk_store(rec + REC_WQ, sm + OFF_WS, 8192);
+      bulk_store(rec + REC_WQ + 16384, sm + OFF_WS + 8192, 8192);
+      bulk_commit();
+    }
   }
 
   if (bad && tid == 0) {
@@ -491,6 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       if (n_issued != n_landed) mbar_wait(bars[i], n_landed & 1u);
     }
   }
+  if (tid == 0) bulk_wait_all();   // the last record's -W copy
   if (wmax > F16_SAFE) atomicOr(&g_gdr_split_error, 2);
   tc_fence_before();
   __syncthreads();
@@ -1805,7 +1801,7 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
   auto kern = p.raw ? chunk_prep_kernel<VAR, true> : chunk_prep_kernel<VAR, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
-  // all of the unified L1 as shared memory, so that two preparation CTAs fit on an SM
+  // all of the unified L1 as shared memory, so that three preparation CTAs fit on an SM
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
@@ -1834,13 +1830,14 @@ cudaError_t launch_prep(const FwdProblem &p, int NC, uint8_t *ws, const PrepRang
     *err = "occupancy query: ";
     return e;
   }
-  // The occupancy query reports one CTA per SM for this kernel, yet two are
-  // resident at once (105 KB of shared memory and 128 x 256 registers each),
-  // so the grid is sized for at least two.  A CTA that does not fit only
-  // starts later; no CTA waits on another.
+  // The occupancy query may report fewer CTAs per SM than are resident once
+  // the carveout applies (72 KB of shared memory and 80 x 256 registers each),
+  // so the grid is sized for at least prep::CTAS_PER_SM.  A CTA that does not
+  // fit only starts later; no CTA waits on another.
   if (rg.sms > 0) sms = std::min(sms, rg.sms);
   const long long records = static_cast<long long>(pp.ncr) * p.H * p.B;
-  const int grid = static_cast<int>(std::min<long long>(records, static_cast<long long>(std::max(per_sm, 2)) * sms));
+  const int grid = static_cast<int>(
+      std::min<long long>(records, static_cast<long long>(std::max(per_sm, prep::CTAS_PER_SM)) * sms));
   e = launch_maybe_pdl(kern, dim3(grid), dim3(NTHREADS), prep::SMEM_BYTES, stream, rg.after_carry,
                        mq, mk, mv, pp);
   if (e != cudaSuccess) *err = "prep launch: ";
@@ -2084,13 +2081,13 @@ PipePlan pipe_plan_for(int variant, int B, int H, int NC, int sms) {
   PipePlan pp;
   const long long bh = static_cast<long long>(B) * H;
   if (NC < 4 || bh <= 0 || sms - bh < 16) return pp;
-  // per variant family: scalar decay (two preparation CTAs per SM), KDA, GDN-2 (one each)
+  // per variant family: scalar decay (three preparation CTAs per SM), KDA, GDN-2 (one each)
   const int fam = variant == kGDN2 ? 2 : variant == kKDA ? 1 : 0;
-  const double slots = fam ? 1.0 : 2.0;                       // preparation CTAs per SM
+  const double slots = fam ? 1.0 : 3.0;                       // preparation CTAs per SM
   const double P0 = fam ? 13.0 : 9.0;                         // us
-  const double P1 = fam == 2 ? 15.0 : fam ? 10.8 : 8.2;       // us per record per CTA
+  const double P1 = fam == 2 ? 15.0 : fam ? 10.8 : 11.5;      // us per record per CTA
   const double C0 = fam == 2 ? 2.5 : fam ? 2.1 : 2.4;         // us
-  const double C1 = fam == 2 ? 3.1 : fam ? 1.85 : 1.69;       // us per chunk
+  const double C1 = fam == 2 ? 3.1 : fam ? 1.85 : 2.1;        // us per chunk
   auto prep = [&](double records, double ctas) { return P0 + P1 * records / ctas; };
   const double serial = prep(double(NC) * bh, slots * sms) + C0 + C1 * NC;
   double best = serial;

@@ -68,6 +68,20 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Plain (untiled) bulk copy shared -> global, tracked by the issuing thread's
+// bulk-async group; both addresses 16-byte aligned, size a multiple of 16 bytes.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the issuing thread's committed bulk copies have finished reading
+// shared memory (the source may then be overwritten).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until they have completed (their writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Bulk prefetch of global memory into L2 (no shared memory, no completion to wait for).
 // Address 16-byte aligned, size a multiple of 16 bytes.
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {

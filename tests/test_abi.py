@@ -179,9 +179,9 @@ def _plan(L, variant, B, T, H, dv=128, sms=148):
 
 def test_two_kernel_schedule_on_a_148_sm_device(L):
     """The schedules the benchmark workloads get on B200 (148 SMs), and the edge cases."""
-    assert _plan(L, 1, 8, 2048, 8) == (1, 32, 22)      # 350M GDN: pipelined, cut at chunk 22 of 32
-    assert _plan(L, 0, 8, 2048, 8) == (1, 32, 22)      # DeltaNet: the same kernels
-    assert _plan(L, 4, 4, 4096, 16) == (1, 64, 43)     # 1.3B KLA
+    assert _plan(L, 1, 8, 2048, 8) == (1, 32, 20)      # 350M GDN: pipelined, cut at chunk 20 of 32
+    assert _plan(L, 0, 8, 2048, 8) == (1, 32, 20)      # DeltaNet: the same kernels
+    assert _plan(L, 4, 4, 4096, 16) == (1, 64, 39)     # 1.3B KLA
     assert _plan(L, 2, 4, 4096, 16) == (1, 64, 53)     # 1.3B KDA
     assert _plan(L, 3, 4, 4096, 16) == (1, 64, 51)     # 1.3B GDN-2
     assert _plan(L, 1, 1, 65536, 16) == (6, 171, 0)    # 64k: six segments of 171 chunks
@@ -212,7 +212,7 @@ def test_empty_batch_workspace_query(L):
 
 def test_forward_plan_binding():
     import gated_delta_rule_forward_b200 as gdr
-    assert gdr.forward_plan("gdn", 8, 2048, 8, 128, 148) == {"segments": 1, "segment_chunks": 32, "split_chunk": 22}
+    assert gdr.forward_plan("gdn", 8, 2048, 8, 128, 148) == {"segments": 1, "segment_chunks": 32, "split_chunk": 20}
     assert gdr.forward_plan("kla", 1, 65536, 16, 128, 148) == {"segments": 6, "segment_chunks": 171, "split_chunk": 0}
     with pytest.raises(gdr.GdrError):
         gdr.forward_plan("gdn", 8, 2048, 8, 96, 148)
