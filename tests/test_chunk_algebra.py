@@ -347,3 +347,117 @@ def test_gdn2_preparation_products_need_fp16_operands():
     e16, eb16 = state_error(f16), state_error(bf16)
     assert e16 < 2e-2 / 4                    # measured 4.9e-3
     assert eb16 > 2.5 * e16                  # measured 1.5e-2
+
+
+def scalar_backward_as_built(q, k, v, beta, lg, s0, dO, dS_final, scale):
+    """The scalar-decay backward in the form the CUDA path computes it (one
+    sequence; q, k [T, dk], v [T, dv], beta and lg [T]).  Three passes:
+
+    1. the forward carry, keeping each chunk's start state S0_c;
+    2. the reverse carry, run as a forward carry over the chunks in reverse with
+       the state X = dS (gradient of the chunk's end state) and per chunk
+           Y = Kt X (the forward's -W S0 slot),  dE = R + Y with R = P^T dO,
+           X <- Gamma_C X + F + (-W)^T dE  with F = Qg^T dO (scale included),
+       the forward carry's steps with Kt in the -W operand, -W in the Kt operand,
+       R in the U' slot and F as the extra state term;
+    3. per chunk, from S0_c, dS_c, dE_c and the inputs, with D_tr = e^(g_t - g_r)
+       (r <= t, g the chunk-local cumulative log decay), e = e^g, f = e^(g_C - g):
+           G = K K^T, A = tril(Diag(beta) (D o G), -1), T = (I + A)^-1
+           E = T Diag(beta) V - T Diag(beta e) K S0
+           dk  = Diag(f) E dS^T + Diag(beta e) T^T dW + N1 K + N1^T K + N2^T Q
+           dq  = scale Diag(e) dO S0^T + N2 K
+           dv  = Diag(beta) T^T dE
+           dW  = -dE S0^T,  dP = tril(dO E^T),  N2 = scale (dP o D)
+           dT  = dE V^T Diag(beta) + dW K^T Diag(beta e)
+           dA  = tril(-T^T dT T^T, -1),  N1 = Diag(beta) (dA o D)
+           dbeta = rowsum(V o T^T dE) + rowsum(Diag(e) K o T^T dW) + rowsum(dA o D o G)
+           dg_t  = sum_i [dq o Q + (Diag(beta e) T^T dW + N1 K) o K - Diag(f) E dS^T o K
+                          - (N1^T K + N2^T Q) o K]_ti,  plus at the chunk's last token
+                   sum(Diag(f) E dS^T o K) + e^(g_C) sum(dS o S0)
+           dlog_g_t = sum_{s >= t in the chunk} dg_s."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    chunks = [slice(c0, min(T, c0 + C)) for c0 in range(0, T, C)]
+    # 1. forward carry with chunk-start states
+    S, S0s, per = s0.copy(), [], []
+    for sl in chunks:
+        K, Q, V, b = k[sl], q[sl], v[sl], beta[sl]
+        n = K.shape[0]
+        g = np.cumsum(lg[sl])
+        D = np.tril(np.exp(g[:, None] - g[None, :]))
+        e, f = np.exp(g), np.exp(g[-1] - g)
+        A = np.tril(b[:, None] * D * (K @ K.T), -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ ((b * e)[:, None] * K)
+        Up = Tm @ (b[:, None] * V)
+        P = scale * D * (Q @ K.T)
+        Qg = scale * e[:, None] * Q
+        Kt = f[:, None] * K
+        S0s.append(S.copy())
+        per.append(dict(K=K, Q=Q, V=V, b=b, g=g, D=D, e=e, f=f, T=Tm, W=W, P=P, Qg=Qg, Kt=Kt))
+        S = np.exp(g[-1]) * S + Kt.T @ (Up - W @ S)
+    # 2. reverse carry
+    X, dSs, dEs = dS_final.copy(), [None] * len(chunks), [None] * len(chunks)
+    for c in reversed(range(len(chunks))):
+        r, dOc = per[c], dO[chunks[c]]
+        dSs[c] = X.copy()
+        dE = r["P"].T @ dOc + r["Kt"] @ X
+        dEs[c] = dE
+        X = np.exp(r["g"][-1]) * X + r["Qg"].T @ dOc + (-r["W"]).T @ dE
+    g_all = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v),
+             "beta": np.zeros(T), "log_g": np.zeros(T), "initial_state": X}
+    # 3. chunk-local gradients
+    for c, sl in enumerate(chunks):
+        r, S0, dS, dE, dOc = per[c], S0s[c], dSs[c], dEs[c], dO[sl]
+        K, Q, V, b, D, e, f, Tm = (r[x] for x in ("K", "Q", "V", "b", "D", "e", "f", "T"))
+        n = K.shape[0]
+        E = Tm @ (b[:, None] * V) - Tm @ ((b * e)[:, None] * K) @ S0
+        X1 = f[:, None] * (E @ dS.T)
+        dW = -dE @ S0.T
+        tU, tW = Tm.T @ dE, Tm.T @ dW
+        dP = np.tril(dOc @ E.T)
+        dT = (dE @ V.T) * b[None, :] + (dW @ K.T) * (b * e)[None, :]
+        dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+        G = K @ K.T
+        N1 = b[:, None] * dA * D
+        N2 = scale * dP * D
+        Y1 = (b * e)[:, None] * tW + N1 @ K
+        Y2 = N1.T @ K + N2.T @ Q
+        dq = scale * e[:, None] * (dOc @ S0.T) + N2 @ K
+        g_all["q"][sl] = dq
+        g_all["k"][sl] = X1 + Y1 + Y2
+        g_all["v"][sl] = b[:, None] * tU
+        g_all["beta"][sl] = (np.sum(V * tU, 1) + e * np.sum(K * tW, 1) + np.sum(dA * D * G, 1))
+        dg = np.sum(dq * Q + (Y1 - X1 - Y2) * K, 1)
+        dg[n - 1] += np.sum(X1 * K) + np.exp(r["g"][-1]) * np.sum(dS * S0)
+        g_all["log_g"][sl] = np.cumsum(dg[::-1])[::-1]
+    return g_all
+
+
+@pytest.mark.parametrize("variant", ["deltanet", "gdn", "kla"])
+def test_scalar_backward_as_built_matches_the_oracle(variant):
+    B, T, H, dk, dv, scale = 1, 29, 1, 6, 5, 0.7
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.float32, seed=11)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    rng = np.random.default_rng(11)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    dO = rng.standard_normal((B, T, H, dv))
+    dS = rng.standard_normal((B, H, dk, dv))
+    eps = 1e-6
+    g_ref = oracle.backward(variant, d_o=dO, d_final=dS, initial_state=s0, scale=scale, eps=eps, **d)
+    q, k, v = d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0]
+    lg = np.zeros(T) if variant == "deltanet" else d["log_g"][0, :, 0]
+    beta = d["beta"][0, :, 0]
+    if variant == "kla":                       # the Kaczmarz step from eta and ||k||^2
+        nk = np.sum(k * k, 1)
+        beta = beta / (nk + eps)
+    g = scalar_backward_as_built(q, k, v, beta, lg, s0[0, 0], dO[0, :, 0], dS[0, 0], scale)
+    if variant == "kla":                       # chain rule through beta = eta / (||k||^2 + eps)
+        dbeta = g["beta"]
+        g["beta"] = dbeta / (nk + eps)
+        g["k"] = g["k"] - (2 * dbeta * beta / (nk + eps))[:, None] * k
+    for name in ("q", "k", "v", "beta"):
+        np.testing.assert_allclose(g[name], g_ref[name][0, :, 0], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(g["initial_state"], g_ref["initial_state"][0, 0], rtol=0, atol=1e-10)
+    if variant != "deltanet":
+        np.testing.assert_allclose(g["log_g"], g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
