@@ -16,7 +16,7 @@ EXPORTS = (
     "gdr_forward_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
     "gdr_forward_launches", "gdr_forward_kernel_name", "gdr_status_string",
     "gdr_last_error", "gdr_version", "gdr_device_status", "gdr_forward_chunked_noalloc",
-    "gdr_forward_plan",
+    "gdr_forward_plan", "gdr_backward_workspace_size", "gdr_backward",
 )
 
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_ALIGNMENT",
@@ -27,6 +27,11 @@ class FwdArgs(ctypes.Structure):
     """Mirror of gdr_fwd_args_t (include/gdr.h)."""
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "q", "k", "v", "beta", "log_g", "erase_b", "write_w", "initial_state", "final_state", "o")]
+
+
+class BwdGrads(ctypes.Structure):
+    """Mirror of gdr_bwd_grads_t (include/gdr.h)."""
+    _fields_ = [(name, ctypes.c_void_p) for name in ("dq", "dk", "dv", "dbeta", "dlog_g", "d_initial_state")]
 
 
 _lock = threading.Lock()
@@ -65,6 +70,11 @@ def lib() -> ctypes.CDLL:
             L.gdr_device_status.restype = i
             L.gdr_version.argtypes = []
             L.gdr_version.restype = i
+            L.gdr_backward_workspace_size.argtypes = [i] * 7
+            L.gdr_backward_workspace_size.restype = sz
+            L.gdr_backward.argtypes = ([i] * 7 + [ctypes.POINTER(FwdArgs), vp, vp, ctypes.POINTER(BwdGrads), f, f,
+                                                 vp, sz, vp])
+            L.gdr_backward.restype = i
             _lib = L
         return _lib
 

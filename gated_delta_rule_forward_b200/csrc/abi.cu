@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "gdr.h"
+#include "chunk_bwd.cuh"
 #include "chunk_split.cuh"
 
 namespace {
@@ -121,8 +122,10 @@ const char *gdr_status_string(gdr_status_t s) {
 const char *gdr_last_error(void) { return g_last_error.c_str(); }
 
 gdr_status_t gdr_device_status(void *stream) {
-  const int e = gdr_read_device_error(static_cast<cudaStream_t>(stream));
-  if (e < 0) return fail(GDR_ERR_CUDA, "synchronisation or symbol read failed");
+  const int ef = gdr_read_device_error(static_cast<cudaStream_t>(stream));
+  const int eb = gdr_bwd_read_device_error(static_cast<cudaStream_t>(stream));
+  if (ef < 0 || eb < 0) return fail(GDR_ERR_CUDA, "synchronisation or symbol read failed");
+  const int e = ef | eb;
   if (e & 1) return fail(GDR_ERR_TIMEOUT, "a bounded device-side wait gave up");
   if (e & 2) return fail(GDR_ERR_RANGE, "a chunked-kernel operand left its representable range");
   return GDR_OK;
@@ -279,6 +282,67 @@ gdr_status_t gdr_forward_chunked_noalloc(int variant, int dtype, int B, int T, i
   std::string err;
   e = gdr_launch_split(p, scratch, have, static_cast<cudaStream_t>(stream), &err);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "chunk64_split: " + err + cudaGetErrorString(e));
+  return GDR_OK;
+}
+
+size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv) {
+  if (variant & GDR_RAW_INPUTS) return 0;
+  if (!gdr_bwd_supported(variant, dtype == GDR_BF16, dk, dv) || B <= 0 || T <= 0 || H <= 0) return 0;
+  return gdr_bwd_workspace_bytes(variant, B, T, H, dv);
+}
+
+gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, int dv, const gdr_fwd_args_t *a,
+                          const void *d_o, const float *d_final, const gdr_bwd_grads_t *g, float eps, float scale,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+  if (variant & GDR_RAW_INPUTS) return fail(GDR_ERR_UNSUPPORTED, "the backward takes transformed inputs (no GDR_RAW_INPUTS)");
+  gdr_status_t st = validate_common(variant, dtype, dk, dv);
+  if (st != GDR_OK) return st;
+  if (!gdr_bwd_supported(variant, dtype == GDR_BF16, dk, dv))
+    return fail(GDR_ERR_UNSUPPORTED,
+                "the backward covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O, dk = 128 and dv in {64, 128}");
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
+  if (!a || !g) return fail(GDR_ERR_INVALID_ARG, "args and grads are required");
+  if ((long)B * H == 0) return GDR_OK;
+  if ((a->initial_state && !aligned16(a->initial_state)) || (d_final && !aligned16(d_final)) ||
+      (g->d_initial_state && !aligned16(g->d_initial_state)))
+    return fail(GDR_ERR_ALIGNMENT, "state pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {   // no tokens: the initial state's gradient is the final state's
+    if (!g->d_initial_state) return GDR_OK;
+    const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+    if (d_final)
+      return check_cuda(cudaMemcpyAsync(g->d_initial_state, d_final, bytes, cudaMemcpyDeviceToDevice, s),
+                        "state gradient copy");
+    return check_cuda(cudaMemsetAsync(g->d_initial_state, 0, bytes, s), "state gradient clear");
+  }
+  if (!a->q || !a->k || !a->v || !d_o || !g->dq || !g->dk || !g->dv || !g->dbeta)
+    return fail(GDR_ERR_INVALID_ARG, "q, k, v, d_o, dq, dk, dv and dbeta are required");
+  if (variant != GDR_DELTANET && !g->dlog_g) return fail(GDR_ERR_INVALID_ARG, "dlog_g is required for this variant");
+  const void *ptrs[9] = {a->q, a->k, a->v, d_o, g->dq, g->dk, g->dv, g->dbeta, g->dlog_g};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  st = validate_gates(variant, a->beta, a->log_g, a->erase_b, a->write_w);
+  if (st != GDR_OK) return st;
+  if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be >= 0");
+  if (!workspace || !aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "a 16-byte aligned workspace is required");
+  if (workspace_bytes < gdr_bwd_workspace_bytes(variant, B, T, H, dv))
+    return fail(GDR_ERR_INVALID_ARG, "the workspace must be at least gdr_backward_workspace_size() bytes");
+  if (injected_launch_fault()) return fail(GDR_ERR_CUDA, "injected launch failure (GDR_FAULT=launch)");
+  gdr::BwdProblem p;
+  p.f.variant = variant; p.f.B = B; p.f.T = T; p.f.H = H; p.f.dk = dk; p.f.dv = dv;
+  p.f.bf16_io = true;
+  p.f.raw = false;
+  p.f.q = a->q; p.f.k = a->k; p.f.v = a->v;
+  p.f.beta = a->beta; p.f.log_g = a->log_g; p.f.erase_b = nullptr; p.f.write_w = nullptr;
+  p.f.s0 = a->initial_state; p.f.s_final = nullptr; p.f.o = nullptr;
+  p.f.eps = eps; p.f.scale = scale;
+  p.d_o = d_o; p.d_final = d_final;
+  p.dq = g->dq; p.dk = g->dk; p.dv = g->dv;
+  p.dbeta = g->dbeta; p.dlog_g = variant == GDR_DELTANET ? nullptr : g->dlog_g;
+  p.d_s0 = g->d_initial_state;
+  std::string err;
+  const cudaError_t e = gdr_launch_backward(p, workspace, workspace_bytes, s, &err);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "backward: " + err + cudaGetErrorString(e));
   return GDR_OK;
 }
 

@@ -1,0 +1,915 @@
+// Chunk-parallel kernels of the chunked backward for the scalar-decay variants
+// (DeltaNet, Gated DeltaNet, KLA).  "Gated DeltaNet-2" (technical core) asks
+// for a gate-aware backward that keeps the chunkwise structure; this one
+// reverses the forward's chunk algebra ("Kaczmarz Linear Attention", KLA
+// update rule and implementation):
+//     forward, per chunk:  E = U' - W S0,  O = Qg S0 + P E,  S_C = Gamma_C S0 + Kt^T E
+//     backward, dS the gradient of the chunk's end state:
+//         dE  = Kt dS + P^T dO
+//         dS0 = Gamma_C dS + Qg^T dO - W^T dE
+// The recurrence in dS is the forward carry's own form with the operands
+// exchanged (Kt where -W was, -W where Kt was, R = P^T dO where U' was and
+// F = Qg^T dO as an extra state term), so it runs on the forward's carry
+// kernel over "reverse records" that bwd_rev_prep_kernel builds here from the
+// forward's records, with the chunks in reverse order.  Every other gradient
+// is local to a chunk given its start state S0 and dS; bwd_local_kernel
+// computes them per chunk, dE included (the records carry beta in P and Kt,
+// so the carry's own residual is Diag(beta) dE, which cannot be divided
+// back where beta vanishes).  With g the chunk-local cumulative log decay,
+// D_tr = e^(g_t - g_r) for r <= t, e = e^g and f = e^(g_C - g):
+//     dE = Diag(f) K dS + P^T dO,  P = scale tril(D o Q K^T)
+//     G = K K^T,  A = tril(Diag(beta) (D o G), -1),  T = (I + A)^-1
+//     E = T Diag(beta) V - T Diag(beta e) K S0,  dW = -dE S0^T,  dP = tril(dO E^T)
+//     dT = dE V^T Diag(beta) + dW K^T Diag(beta e),  dA = tril(-T^T dT T^T, -1)
+//     N1 = Diag(beta) (dA o D),  N2 = scale (dP o D)
+//     dk = Diag(f) E dS^T + Diag(beta e) T^T dW + N1 K + N1^T K + N2^T Q
+//     dq = scale Diag(e) dO S0^T + N2 K,   dv = Diag(beta) T^T dE
+//     dbeta = rowsum(V o T^T dE) + e o rowsum(K o T^T dW) + rowsum(dA o D o G)
+//     dg_t = sum_i [dq o Q + (Diag(beta e) T^T dW + N1 K - Diag(f) E dS^T - N1^T K - N2^T Q) o K]_ti
+//            (+ sum(Diag(f) E dS^T o K) + e^(g_C) sum(dS o S0) at the chunk's last token)
+//     dlog_g_t = sum of dg_s over the chunk's tokens s >= t
+// and for KLA, beta = eta / (||k||^2 + eps): d eta = dbeta / (||k||^2 + eps),
+// dk -= 2 dbeta beta / (||k||^2 + eps) k.  Decay enters only through D, e and
+// f, all at most 1, so no factor overflows however strong the decay.
+//
+// The reverse carry's fp16 operands need the gradients near unit scale: dO and
+// the final-state gradient are scaled by a power of two s (max |.| to [0.5, 1)),
+// and the local kernel and the initial-state gradient divide it out again.
+#include <algorithm>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "chunk_bwd.cuh"
+#include "chunk_common.cuh"
+#include "chunk_record.cuh"
+
+// Device-side error word of this file (bit 1: a reverse-record operand beyond
+// the fp16 range).
+__device__ int g_gdr_bwd_error = 0;
+
+namespace gdr {
+namespace tc {
+namespace {
+
+constexpr int NT = 256;
+constexpr float F16_SAFE_BWD = 60000.f;
+constexpr float LOG2E_BWD = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- SIMT products
+// A matrix operand: element (r, c) is p[r * ld + c], or p[c * ld + r] for TR.
+// GLOBAL operands are read through the read-only cache.
+template <typename E, bool TR, bool GLOBAL = false>
+struct Mat {
+  using elem = E;
+  static constexpr bool kTr = TR;
+  static constexpr bool kGlobal = GLOBAL;
+  const E *p;
+  int ld;
+};
+
+template <typename E, bool G>
+__device__ __forceinline__ void ld4(const E *p, float (&x)[4]);
+template <>
+__device__ __forceinline__ void ld4<float, false>(const float *p, float (&x)[4]) {
+  const float4 v = *reinterpret_cast<const float4 *>(p);
+  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void ld4<float, true>(const float *p, float (&x)[4]) {
+  const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void ld4<__nv_bfloat16, false>(const __nv_bfloat16 *p, float (&x)[4]) {
+  unpack4(*reinterpret_cast<const uint2 *>(p), x);
+}
+template <typename E, bool G>
+__device__ __forceinline__ float ld1(const E *p);
+template <>
+__device__ __forceinline__ float ld1<float, false>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld1<float, true>(const float *p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld1<__nv_bfloat16, false>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+// acc[i][j] (+/-)= sum_{k < K} A(r0 + i, k) ks[k] B(k, c0 + 16 j): a thread's
+// MR x NR tile of rows r0 .. r0 + MR - 1 and columns c0, c0 + 16, ...  (ks, a
+// per-k factor in shared memory, may be null).  K is a multiple of 4, and r0
+// of 4 where A is TR.
+template <int MR, int NR, bool NEG, typename MA, typename MB>
+__device__ __forceinline__ void mm(float (&acc)[MR][NR], const MA a, const MB b, int K, int r0, int c0,
+                                   const float *ks = nullptr) {
+  using EA = typename MA::elem;
+  using EB = typename MB::elem;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 4) {
+    float af[MR][4], bf[4][NR];
+    if constexpr (!MA::kTr) {
+#pragma unroll
+      for (int i = 0; i < MR; ++i) ld4<EA, MA::kGlobal>(a.p + (r0 + i) * a.ld + k0, af[i]);
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int i4 = 0; i4 < MR; i4 += 4) {
+          float x[4];
+          ld4<EA, MA::kGlobal>(a.p + (k0 + kk) * a.ld + r0 + i4, x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) af[i4 + e][kk] = x[e];
+        }
+    }
+    if constexpr (!MB::kTr) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int j = 0; j < NR; ++j) bf[kk][j] = ld1<EB, MB::kGlobal>(b.p + (k0 + kk) * b.ld + c0 + 16 * j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NR; ++j) {
+        float x[4];
+        ld4<EB, MB::kGlobal>(b.p + (c0 + 16 * j) * b.ld + k0, x);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) bf[kk][j] = x[kk];
+      }
+    }
+    if (ks != nullptr) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const float f = ks[k0 + kk];
+#pragma unroll
+        for (int j = 0; j < NR; ++j) bf[kk][j] *= f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MR; ++i)
+#pragma unroll
+      for (int j = 0; j < NR; ++j)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) acc[i][j] = fmaf(NEG ? -af[i][kk] : af[i][kk], bf[kk][j], acc[i][j]);
+  }
+}
+
+template <int MR, int NR>
+__device__ __forceinline__ void zero(float (&acc)[MR][NR]) {
+#pragma unroll
+  for (int i = 0; i < MR; ++i)
+#pragma unroll
+    for (int j = 0; j < NR; ++j) acc[i][j] = 0.f;
+}
+
+// Sum over the 16 lanes of a half warp (the column groups of one row group).
+__device__ __forceinline__ float half_warp_sum(float x) {
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// The power of two s with s * max|gradient| in [0.5, 1) (1 when the maximum is
+// zero or not finite).
+__device__ __forceinline__ float grad_scale(const uint32_t *absmax) {
+  const float m = __uint_as_float(*absmax);
+  if (!(m > 0.f) || !(m < 3.0e38f)) return 1.f;
+  int ex;
+  frexpf(m, &ex);
+  ex = max(-120, min(120, ex));
+  return ldexpf(1.f, -ex);
+}
+
+// ---------------------------------------------------------------- gradient scale
+__global__ void bwd_absmax_kernel(const __nv_bfloat16 *d_o, size_t n_o, const float *d_final, size_t n_f,
+                                  uint32_t *out) {
+  float m = 0.f;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_o; i += stride)
+    m = fmaxf(m, fabsf(__bfloat162float(d_o[i])));
+  if (d_final != nullptr)
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_f; i += stride)
+      m = fmaxf(m, fabsf(__ldg(d_final + i)));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));   // non-negative floats order as integers
+}
+
+__global__ void bwd_scale_state_kernel(const float *d_final, size_t n, const uint32_t *absmax, float *x0) {
+  const float s = grad_scale(absmax);
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    x0[i] = d_final != nullptr ? s * __ldg(d_final + i) : 0.f;
+}
+
+__global__ void bwd_unscale_kernel(const float *xf, size_t n, const uint32_t *absmax, float *d_s0) {
+  const float inv = 1.f / grad_scale(absmax);
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    d_s0[i] = __ldg(xf + i) * inv;
+}
+
+// ---------------------------------------------------------------- reverse records
+struct RevPrepParams {
+  int T, H, NC;
+  uint32_t rb_f, rb_r;   // bytes of a forward record / a reverse record
+  bool chan;             // Gamma_C stored as d_k values in the forward record
+  const __nv_bfloat16 *d_o;
+  const uint8_t *fwd;
+  uint8_t *rev;
+  const uint32_t *absmax;
+};
+
+// One CTA per forward record (b, h, c); it writes reverse record (b, h, NC-1-c)
+// in the channel-decay + GDN-2 record format the carry's third mode reads:
+//     -W slot of REC_WQ <- Kt (the Qg slot cleared),  REC_K <- -W,
+//     U' slot <- R^T = (s dO)^T P,  Gamma_C as d_k values,
+//     the output term cleared,  the state term <- F^T = (s dO)^T Qg.
+template <int DV>
+__global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams p) {
+  constexpr int NS = DV / 64;
+  constexpr int LDO = DV + 4, LDP = C + 4, LDQ = DK + 4;
+  extern __shared__ float4 smem_rev[];
+  float *sO = reinterpret_cast<float *>(smem_rev);   // [C][LDO] s dO, rows t
+  float *sP = sO + C * LDO;                          // [C][LDP] P, rows t
+  float *sQ = sP + C * LDP;                          // [C][LDQ] Qg, rows t
+  const int tid = threadIdx.x;
+  const int r = blockIdx.x;
+  const int bh = r / p.NC, c = r - bh * p.NC;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const uint8_t *src = p.fwd + static_cast<size_t>(r) * p.rb_f;
+  uint8_t *dst = p.rev + (static_cast<size_t>(bh) * p.NC + (p.NC - 1 - c)) * p.rb_r;
+  const float s = grad_scale(p.absmax);
+
+  for (int i = tid; i < C * DV / 8; i += NT) {
+    const int t = i / (DV / 8), v8 = (i % (DV / 8)) * 8;
+    const int tg = c * C + t;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (tg < p.T)
+      unpack8(__ldg(reinterpret_cast<const uint4 *>(p.d_o + ((static_cast<size_t>(b) * p.T + tg) * p.H + h) * DV + v8)),
+              x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sO[t * LDO + v8 + e] = s * x[e];
+  }
+  for (int i = tid; i < C * C / 8; i += NT) {
+    const int t = i >> 3, j = i & 7;
+    const uint4 u = *reinterpret_cast<const uint4 *>(src + REC_P + sw128(t, j));
+    const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(hp[e]);
+      sP[t * LDP + 8 * j + 2 * e] = f.x;
+      sP[t * LDP + 8 * j + 2 * e + 1] = f.y;
+    }
+  }
+  for (int i = tid; i < C * DK / 8; i += NT) {
+    const int t = i >> 4, a = (i >> 3) & 1, j = i & 7;
+    const uint4 u = *reinterpret_cast<const uint4 *>(src + REC_WQ + a * 16384 + 8192 + sw128(t, j));
+    const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(hp[e]);
+      sQ[t * LDQ + 64 * a + 8 * j + 2 * e] = f.x;
+      sQ[t * LDQ + 64 * a + 8 * j + 2 * e + 1] = f.y;
+    }
+  }
+  // tile copies and cleared slots (16-byte units)
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < 1024; i += NT) {
+    const int a = i >> 9, j = i & 511;
+    *reinterpret_cast<uint4 *>(dst + REC_WQ + a * 16384 + 16 * j) =
+        *reinterpret_cast<const uint4 *>(src + REC_K + a * 8192 + 16 * j);
+    *reinterpret_cast<uint4 *>(dst + REC_WQ + a * 16384 + 8192 + 16 * j) = z;
+    *reinterpret_cast<uint4 *>(dst + REC_K + a * 8192 + 16 * j) =
+        *reinterpret_cast<const uint4 *>(src + REC_WQ + a * 16384 + 16 * j);
+  }
+  for (int i = tid; i < 512; i += NT) *reinterpret_cast<uint4 *>(dst + REC_P + 16 * i) = z;
+  for (int i = tid; i < 512 * NS; i += NT) *reinterpret_cast<uint4 *>(dst + rec_bytes_chan(NS) + 16 * i) = z;
+  if (tid < DK) {
+    const float *g = reinterpret_cast<const float *>(src + rec_sc(NS));
+    reinterpret_cast<float *>(dst + rec_sc(NS))[tid] = p.chan ? g[tid] : g[0];
+  }
+  __syncthreads();
+
+  const int rg = tid >> 4, cg = tid & 15;
+  constexpr int MR = DV / 16;
+  float vmax = 0.f;
+  {   // R^T [v][t] into the U' slot (rows v, 128-byte swizzled)
+    float acc[MR][4];
+    zero(acc);
+    mm<MR, 4, false>(acc, Mat<float, true>{sO, LDO}, Mat<float, false>{sP, LDP}, C, MR * rg, cg);
+#pragma unroll
+    for (int i = 0; i < MR; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = MR * rg + i, t = cg + 16 * j;
+        vmax = fmaxf(vmax, fabsf(acc[i][j]));
+        *reinterpret_cast<__half *>(dst + REC_U + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(acc[i][j]);
+      }
+  }
+  {   // F^T [v][i] after the output term, unswizzled rows of d_k values
+    float acc[MR][8];
+    zero(acc);
+    mm<MR, 8, false>(acc, Mat<float, true>{sO, LDO}, Mat<float, false>{sQ, LDQ}, C, MR * rg, cg);
+    __half *f = reinterpret_cast<__half *>(dst + rec_bytes_chan(NS) + 8192 * NS);
+#pragma unroll
+    for (int i = 0; i < MR; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        vmax = fmaxf(vmax, fabsf(acc[i][j]));
+        f[(MR * rg + i) * DK + cg + 16 * j] = __float2half_rn(acc[i][j]);
+      }
+  }
+  if (vmax > F16_SAFE_BWD) atomicOr(&g_gdr_bwd_error, 2);
+}
+
+// ---------------------------------------------------------------- chunk-local gradients
+struct LocalParams {
+  int T, H, NC;
+  bool decay, kla;
+  float eps, scale;
+  const __nv_bfloat16 *q, *k, *v, *d_o;
+  const float *beta, *log_g;
+  const float *s0s, *dss;   // chunk start states and end-state gradients (the latter in reverse chunk order)
+  const uint32_t *absmax;
+  __nv_bfloat16 *dq, *dk, *dv;
+  float *dbeta, *dlog_g;
+};
+
+template <int DV>
+struct LocalSmem {
+  static constexpr int LDB = DK + 8;    // bf16 rows of K, Q
+  static constexpr int LDBV = DV + 8;   // bf16 rows of V, dO
+  static constexpr int LDF = DV + 4;    // fp32 rows of dE, E
+  static constexpr int LDW = DK + 4;    // fp32 rows of W
+  static constexpr int LDC = C + 4;     // fp32 rows of C-wide tiles (dW^T, X, dP)
+  static constexpr size_t K = 0;
+  static constexpr size_t Q = K + C * LDB * 2;
+  static constexpr size_t V = Q + C * LDB * 2;
+  static constexpr size_t O = V + C * LDBV * 2;
+  static constexpr size_t DE = O + C * LDBV * 2;
+  static constexpr size_t E = DE + C * LDF * 4;
+  static constexpr size_t W = E + static_cast<size_t>(std::max(C * LDF, C * LDC)) * 4;
+  static constexpr size_t A = W + static_cast<size_t>(std::max(C * LDW, DK * LDC)) * 4;
+  static constexpr size_t TT = A + C * LD * 4;
+  static constexpr size_t P = TT + C * LD * 4;
+  static constexpr size_t SC = P + C * LDC * 4;
+  static constexpr size_t BYTES = SC + (9 * C + 4) * 4;
+};
+
+// One CTA per chunk (b, h, c).
+template <int DV>
+__global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
+  using L = LocalSmem<DV>;
+  constexpr int LDB = L::LDB, LDBV = L::LDBV, LDF = L::LDF, LDW = L::LDW, LDC = L::LDC;
+  constexpr int NRV = DV / 16, NRK = DK / 16;
+  extern __shared__ float4 smem_loc[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>(smem_loc);
+  __nv_bfloat16 *sK = reinterpret_cast<__nv_bfloat16 *>(sm + L::K);
+  __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(sm + L::Q);
+  __nv_bfloat16 *sV = reinterpret_cast<__nv_bfloat16 *>(sm + L::V);
+  __nv_bfloat16 *sO = reinterpret_cast<__nv_bfloat16 *>(sm + L::O);
+  float *sdE = reinterpret_cast<float *>(sm + L::DE);
+  float *sE = reinterpret_cast<float *>(sm + L::E);    // E, later X = dT T^T
+  float *sW = reinterpret_cast<float *>(sm + L::W);    // W, later dW^T
+  float *sA = reinterpret_cast<float *>(sm + L::A);    // A^T for the solve, later dT, dA, N1
+  float *sT = reinterpret_cast<float *>(sm + L::TT);   // T
+  float *sP = reinterpret_cast<float *>(sm + L::P);    // dP, later N2
+  float *sbeta = reinterpret_cast<float *>(sm + L::SC);
+  float *sbe = sbeta + C;     // beta e
+  float *see = sbe + C;       // e
+  float *sff = see + C;       // f
+  float *sscan = sff + C;     // per-warp scan of the log2 decay
+  float *sG = sscan + C;      // cumulative log2 decay
+  float *sdb = sG + C;        // dbeta
+  float *sdg = sdb + C;       // dg
+  float *snk = sdg + C;       // ||k||^2
+  float *sred = snk + C;      // [0] sum X1 o K, [1] sum dS o S0
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = tid >> 4, cg = tid & 15;
+  const int bh = blockIdx.x / p.NC, c = blockIdx.x - bh * p.NC;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int t0 = c * C, n = min(C, p.T - t0);
+  const float s = grad_scale(p.absmax), inv_s = 1.f / s;
+  const size_t rc = static_cast<size_t>(bh) * p.NC + (p.NC - 1 - c);   // reverse-order index of this chunk
+  const float *S0 = p.s0s + static_cast<size_t>(blockIdx.x) * DK * DV;
+  const float *dS = p.dss + rc * DK * DV;
+  auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
+
+  // ---- inputs: bf16 tiles (zero past T)
+  for (int i = tid; i < C * DK / 8; i += NT) {
+    const int t = i / (DK / 8), j = i % (DK / 8);
+    uint4 uq = make_uint4(0u, 0u, 0u, 0u), uk = uq;
+    if (t < n) {
+      uq = __ldg(reinterpret_cast<const uint4 *>(p.q + row(t) * DK) + j);
+      uk = __ldg(reinterpret_cast<const uint4 *>(p.k + row(t) * DK) + j);
+    }
+    *reinterpret_cast<uint4 *>(sQ + t * LDB + 8 * j) = uq;
+    *reinterpret_cast<uint4 *>(sK + t * LDB + 8 * j) = uk;
+  }
+  for (int i = tid; i < C * DV / 8; i += NT) {
+    const int t = i / (DV / 8), j = i % (DV / 8);
+    uint4 uv = make_uint4(0u, 0u, 0u, 0u), uo = uv;
+    if (t < n) {
+      uv = __ldg(reinterpret_cast<const uint4 *>(p.v + row(t) * DV) + j);
+      uo = __ldg(reinterpret_cast<const uint4 *>(p.d_o + row(t) * DV) + j);
+    }
+    *reinterpret_cast<uint4 *>(sV + t * LDBV + 8 * j) = uv;
+    *reinterpret_cast<uint4 *>(sO + t * LDBV + 8 * j) = uo;
+  }
+  if (tid < C) {
+    sdb[tid] = 0.f;
+    sdg[tid] = 0.f;
+  }
+  if (tid < 4) sred[tid] = 0.f;
+  __syncthreads();
+
+  // ---- token scalars (threads 0-63): beta (KLA: eta / (||k||^2 + eps)), the
+  // cumulative log2 decay, e and f
+  if (tid < C) {
+    const int t = tid;
+    float bt = 0.f, lg = 0.f, nk = 0.f;
+    for (int i = 0; i < DK; ++i) {
+      const float x = __bfloat162float(sK[t * LDB + i]);
+      nk = fmaf(x, x, nk);
+    }
+    if (t < n) {
+      bt = __ldg(p.beta + row(t));
+      if (p.decay) lg = __ldg(p.log_g + row(t));
+    }
+    if (p.kla) bt = bt / (nk + p.eps);
+    snk[t] = nk;
+    sbeta[t] = bt;
+    float x = lg * LOG2E_BWD;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    sscan[t] = x;
+  }
+  __syncthreads();
+  if (tid < C) {
+    const int t = tid;
+    sG[t] = sscan[t] + (t >= 32 ? sscan[31] : 0.f);
+  }
+  __syncthreads();
+  if (tid < C) {
+    const int t = tid;
+    const float e = ex2(sG[t]);
+    see[t] = e;
+    sff[t] = ex2(sG[n - 1] - sG[t]);
+    sbe[t] = sbeta[t] * e;
+  }
+  __syncthreads();
+
+  // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
+  {
+    float g[4][4];
+    zero(g);
+    mm<4, 4, false>(g, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * rg + i, r = cg + 16 * j;
+        const float a = r < t ? sbeta[t] * ex2(sG[t] - sG[r]) * g[i][j] : 0.f;
+        sA[r * LD + t] = tf32r(a);
+      }
+  }
+  __syncthreads();
+  solve_unit_lower_64(sA, sT, tid, warp, lane);   // ends with a barrier
+  for (int i = tid; i < C * C; i += NT) {
+    const int m = i / C, j = i % C;
+    if (j > m) sT[m * LD + j] = 0.f;
+  }
+  __syncthreads();
+
+  // ---- U' = T Diag(beta) V and W = T Diag(beta e) K; E = U' - W S0
+  float ue[4][NRV];
+  zero(ue);
+  mm<4, NRV, false>(ue, Mat<float, false>{sT, LD}, Mat<__nv_bfloat16, false>{sV, LDBV}, C, 4 * rg, cg, sbeta);
+  {
+    float w[4][NRK];
+    zero(w);
+    mm<4, NRK, false>(w, Mat<float, false>{sT, LD}, Mat<__nv_bfloat16, false>{sK, LDB}, C, 4 * rg, cg, sbe);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NRK; ++j) sW[(4 * rg + i) * LDW + cg + 16 * j] = w[i][j];
+  }
+  __syncthreads();
+  mm<4, NRV, true>(ue, Mat<float, false>{sW, LDW}, Mat<float, false, true>{S0, DV}, DK, 4 * rg, cg);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NRV; ++j) sE[(4 * rg + i) * LDF + cg + 16 * j] = ue[i][j];
+  // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
+  // reverse carry's own dE is Diag(beta) dE (its records carry beta in P and Kt), so it is
+  // recomputed here rather than divided by beta.
+  {
+    float gq[4][4];
+    zero(gq);
+    mm<4, 4, false>(gq, Mat<__nv_bfloat16, false>{sQ, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * rg + i, r = cg + 16 * j;
+        sP[t * LDC + r] = r <= t ? p.scale * ex2(sG[t] - sG[r]) * gq[i][j] : 0.f;
+      }
+  }
+  __syncthreads();
+  {
+    float acc[4][NRV];
+    zero(acc);
+    mm<4, NRV, false>(acc, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<float, false, true>{dS, DV}, DK, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float f = sff[4 * rg + i] * inv_s;
+#pragma unroll
+      for (int j = 0; j < NRV; ++j) acc[i][j] *= f;
+    }
+    mm<4, NRV, false>(acc, Mat<float, true>{sP, LDC}, Mat<__nv_bfloat16, false>{sO, LDBV}, C, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NRV; ++j) sdE[(4 * rg + i) * LDF + cg + 16 * j] = acc[i][j];
+  }
+  __syncthreads();
+
+  // ---- dk^T (rows i = 8 rg .., columns t = cg + 16 j) starts as (Diag(f) E dS^T)^T / s
+  float dkT[8][4];
+  float dgp[4] = {0.f, 0.f, 0.f, 0.f};   // this thread's share of dg_t, t = cg + 16 j
+  float x1k = 0.f;
+  zero(dkT);
+  mm<8, 4, false>(dkT, Mat<float, false, true>{dS, DV}, Mat<float, true>{sE, LDF}, DV, 8 * rg, cg);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int t = cg + 16 * j;
+    const float ft = sff[t] * inv_s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dkT[i][j] *= ft;
+      const float x = dkT[i][j] * __bfloat162float(sK[t * LDB + 8 * rg + i]);
+      x1k += x;
+      dgp[j] -= x;
+    }
+  }
+  // ---- dP = tril(dO E^T)
+  {
+    float acc[4][4];
+    zero(acc);
+    mm<4, 4, false>(acc, Mat<__nv_bfloat16, false>{sO, LDBV}, Mat<float, true>{sE, LDF}, DV, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * rg + i, r = cg + 16 * j;
+        sP[t * LDC + r] = r <= t ? acc[i][j] : 0.f;
+      }
+  }
+  // ---- dW^T = -S0 dE^T  (d_k x C, over W, which E = U' - W S0 has finished reading)
+  {
+    float acc[8][4];
+    zero(acc);
+    mm<8, 4, true>(acc, Mat<float, false, true>{S0, DV}, Mat<float, true>{sdE, LDF}, DV, 8 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sW[(8 * rg + i) * LDC + cg + 16 * j] = acc[i][j];
+  }
+  __syncthreads();
+
+  // ---- dv = Diag(beta) T^T dE;  dbeta += rowsum(V o T^T dE)
+  {
+    float acc[4][NRV];
+    zero(acc);
+    mm<4, NRV, false>(acc, Mat<float, true>{sT, LD}, Mat<float, false>{sdE, LDF}, C, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = 4 * rg + i;
+      const float bt = sbeta[t];
+      float part = 0.f;
+#pragma unroll
+      for (int j = 0; j < NRV; ++j) {
+        const int v = cg + 16 * j;
+        part = fmaf(__bfloat162float(sV[t * LDBV + v]), acc[i][j], part);
+        if (t < n) p.dv[row(t) * DV + v] = __float2bfloat16_rn(bt * acc[i][j]);
+      }
+      part = half_warp_sum(part);
+      if (cg == 0) atomicAdd(&sdb[t], part);
+    }
+  }
+  // ---- (T^T dW)^T = dW^T T:  dk += Diag(beta e) T^T dW;  dbeta += e o rowsum(K o T^T dW)
+  {
+    float acc[8][4];
+    zero(acc);
+    mm<8, 4, false>(acc, Mat<float, false>{sW, LDC}, Mat<float, false>{sT, LD}, C, 8 * rg, cg);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = cg + 16 * j;
+      const float bet = sbe[t], et = see[t];
+      float dbp = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float kv = __bfloat162float(sK[t * LDB + 8 * rg + i]);
+        const float y = bet * acc[i][j];
+        dkT[i][j] += y;
+        dgp[j] = fmaf(y, kv, dgp[j]);
+        dbp = fmaf(et * kv, acc[i][j], dbp);
+      }
+      dbp += __shfl_xor_sync(0xffffffffu, dbp, 16);
+      if (lane < 16) atomicAdd(&sdb[t], dbp);
+    }
+  }
+  // ---- dT = dE V^T Diag(beta) + dW K^T Diag(beta e)  (over A^T, dead since the solve)
+  {
+    float a1[4][4], a2[4][4];
+    zero(a1);
+    zero(a2);
+    mm<4, 4, false>(a1, Mat<float, false>{sdE, LDF}, Mat<__nv_bfloat16, true>{sV, LDBV}, DV, 4 * rg, cg);
+    mm<4, 4, false>(a2, Mat<float, true>{sW, LDC}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * rg + i, r = cg + 16 * j;
+        sA[t * LD + r] = sbeta[r] * a1[i][j] + sbe[r] * a2[i][j];
+      }
+  }
+  __syncthreads();
+  // ---- X = dT T^T (over E), then dA = tril(-T^T X, -1) (over dT)
+  {
+    float acc[4][4];
+    zero(acc);
+    mm<4, 4, false>(acc, Mat<float, false>{sA, LD}, Mat<float, true>{sT, LD}, C, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sE[(4 * rg + i) * LDC + cg + 16 * j] = acc[i][j];
+  }
+  __syncthreads();
+  {
+    float acc[4][4];
+    zero(acc);
+    mm<4, 4, true>(acc, Mat<float, true>{sT, LD}, Mat<float, false>{sE, LDC}, C, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * rg + i, r = cg + 16 * j;
+        sA[t * LD + r] = r < t ? acc[i][j] : 0.f;
+      }
+  }
+  __syncthreads();
+  // ---- G = K K^T again: dbeta += rowsum(dA o D o G); N1 = Diag(beta) (dA o D), N2 = scale (dP o D)
+  {
+    float g[4][4];
+    zero(g);
+    mm<4, 4, false>(g, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = 4 * rg + i;
+      float part = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = cg + 16 * j;
+        const float d = r <= t ? ex2(sG[t] - sG[r]) : 0.f;
+        const float da = sA[t * LD + r];
+        part = fmaf(da * d, g[i][j], part);
+        sA[t * LD + r] = sbeta[t] * da * d;
+        sP[t * LDC + r] = p.scale * sP[t * LDC + r] * d;
+      }
+      part = half_warp_sum(part);
+      if (cg == 0) atomicAdd(&sdb[t], part);
+    }
+  }
+  __syncthreads();
+  // ---- dk += N1 K + N1^T K + N2^T Q   (as K^T N1^T, K^T N1, Q^T N2)
+  {
+    float acc[8][4];
+    zero(acc);
+    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, true>{sA, LD}, C, 8 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dkT[i][j] += acc[i][j];
+        dgp[j] = fmaf(acc[i][j], __bfloat162float(sK[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
+      }
+    zero(acc);
+    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, false>{sA, LD}, C, 8 * rg, cg);
+    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sQ, LDB}, Mat<float, false>{sP, LDC}, C, 8 * rg, cg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dkT[i][j] += acc[i][j];
+        dgp[j] = fmaf(-acc[i][j], __bfloat162float(sK[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
+      }
+  }
+  // ---- dq = scale Diag(e) dO S0^T + N2 K
+  float dqT[8][4];
+  zero(dqT);
+  mm<8, 4, false>(dqT, Mat<float, false, true>{S0, DV}, Mat<__nv_bfloat16, true>{sO, LDBV}, DV, 8 * rg, cg);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float f = p.scale * see[cg + 16 * j];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dqT[i][j] *= f;
+  }
+  mm<8, 4, false>(dqT, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, true>{sP, LDC}, C, 8 * rg, cg);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      dgp[j] = fmaf(dqT[i][j], __bfloat162float(sQ[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
+
+  // ---- reductions: dg_t over the row groups; sum(X1 o K); sum(dS o S0)
+  {
+    float ss = 0.f;
+    const float4 *a = reinterpret_cast<const float4 *>(dS), *bb = reinterpret_cast<const float4 *>(S0);
+    for (int i = tid; i < DK * DV / 4; i += NT) {
+      const float4 x = __ldg(a + i), y = __ldg(bb + i);
+      ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      x1k += __shfl_xor_sync(0xffffffffu, x1k, o);
+    }
+    if (lane == 0) {
+      atomicAdd(&sred[0], x1k);
+      atomicAdd(&sred[1], ss);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = dgp[j] + __shfl_xor_sync(0xffffffffu, dgp[j], 16);
+      if (lane < 16) atomicAdd(&sdg[cg + 16 * j], x);
+    }
+  }
+  __syncthreads();
+
+  // ---- KLA: beta = eta / (||k||^2 + eps) adds -2 dbeta beta / (||k||^2 + eps) k to dk
+  if (p.kla) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = cg + 16 * j;
+      const float w = -2.f * sdb[t] * sbeta[t] / (snk[t] + p.eps);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dkT[i][j] = fmaf(w, __bfloat162float(sK[t * LDB + 8 * rg + i]), dkT[i][j]);
+    }
+  }
+  // ---- dq, dk: eight consecutive d_k values per (thread, token)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int t = cg + 16 * j;
+    if (t < n) {
+      float xk[8], xq[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        xk[i] = dkT[i][j];
+        xq[i] = dqT[i][j];
+      }
+      st_chunk_bf16(reinterpret_cast<uint8_t *>(p.dk + row(t) * DK + 8 * rg), xk);
+      st_chunk_bf16(reinterpret_cast<uint8_t *>(p.dq + row(t) * DK + 8 * rg), xq);
+    }
+  }
+  // ---- dbeta (d eta for KLA) and dlog_g = suffix sums of dg over the chunk's tokens
+  if (tid < C) {
+    const int t = tid;
+    if (t < n) p.dbeta[row(t)] = p.kla ? sdb[t] / (snk[t] + p.eps) : sdb[t];
+    if (p.decay && p.dlog_g != nullptr) {
+      float x = 0.f;
+      if (t < n) x = sdg[t] + (t == n - 1 ? sred[0] + ex2(sG[n - 1]) * sred[1] * inv_s : 0.f);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+      }
+      sscan[t] = x;   // suffix sums within each warp
+    }
+  }
+  __syncthreads();
+  if (tid < C && p.decay && p.dlog_g != nullptr) {
+    const int t = tid;
+    const float x = sscan[t] + (t < 32 ? sscan[32] : 0.f);
+    if (t < n) p.dlog_g[row(t)] = x;
+  }
+}
+
+int grid_for(size_t n) { return static_cast<int>(std::min<size_t>((n + 255) / 256, 4096)); }
+
+}  // namespace
+}  // namespace tc
+
+BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
+  using namespace tc;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t NC = (static_cast<size_t>(T) + C - 1) / C, bh = static_cast<size_t>(B) * H, ns = dv / 64;
+  const size_t rb_f = variant == kKDA ? rec_bytes_chan(static_cast<int>(ns)) : rec_bytes(static_cast<int>(ns));
+  BwdLayout L;
+  L.fwd_rec = 0;
+  L.rev_rec = up(bh * NC * rb_f);
+  L.s0s = L.rev_rec + up(bh * NC * rec_bytes_gdn2(static_cast<int>(ns)));
+  L.dss = L.s0s + up(bh * NC * DK * dv * 4);
+  L.x0 = L.dss + up(bh * NC * DK * dv * 4);
+  L.xf = L.x0 + up(bh * DK * dv * 4);
+  L.absmax = L.xf + up(bh * DK * dv * 4);
+  L.total = L.absmax + 256;
+  return L;
+}
+
+}  // namespace gdr
+
+bool gdr_bwd_supported(int variant, int dtype_bf16, int dk, int dv) {
+  using namespace gdr;
+  return (variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA) && dtype_bf16 && dk == 128 &&
+         (dv == 64 || dv == 128);
+}
+
+size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv) {
+  return gdr::bwd_layout(variant, B, T, H, dv).total;
+}
+
+cudaError_t gdr_bwd_launch_scale(const gdr::BwdProblem &p, uint32_t *absmax, float *x0, cudaStream_t s) {
+  using namespace gdr::tc;
+  const gdr::FwdProblem &f = p.f;
+  cudaError_t e = cudaMemsetAsync(absmax, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  const size_t n_o = static_cast<size_t>(f.B) * f.T * f.H * f.dv, n_s = static_cast<size_t>(f.B) * f.H * f.dk * f.dv;
+  bwd_absmax_kernel<<<grid_for(std::max(n_o, n_s)), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(p.d_o), n_o,
+                                                                  p.d_final, n_s, absmax);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_scale_state_kernel<<<grid_for(n_s), 256, 0, s>>>(p.d_final, n_s, absmax, x0);
+  return cudaGetLastError();
+}
+
+cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd_rec, uint8_t *rev_rec,
+                                    const uint32_t *absmax, cudaStream_t s) {
+  using namespace gdr::tc;
+  const gdr::FwdProblem &f = p.f;
+  RevPrepParams rp;
+  rp.T = f.T; rp.H = f.H; rp.NC = (f.T + C - 1) / C;
+  const int ns = f.dv / 64;
+  rp.chan = f.variant == gdr::kKDA;
+  rp.rb_f = rp.chan ? rec_bytes_chan(ns) : rec_bytes(ns);
+  rp.rb_r = rec_bytes_gdn2(ns);
+  rp.d_o = static_cast<const __nv_bfloat16 *>(p.d_o);
+  rp.fwd = fwd_rec; rp.rev = rev_rec; rp.absmax = absmax;
+  const int grid = f.B * f.H * rp.NC;
+  auto run = [&](auto kern, int dv) {
+    const size_t smem = (static_cast<size_t>(C) * (dv + 4) + C * (C + 4) + C * (DK + 4)) * 4;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NT, smem, s>>>(rp);
+    return cudaGetLastError();
+  };
+  return f.dv == 128 ? run(bwd_rev_prep_kernel<128>, 128) : run(bwd_rev_prep_kernel<64>, 64);
+}
+
+cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const float *s0s, const float *dss,
+                                 const uint32_t *absmax, cudaStream_t s) {
+  using namespace gdr::tc;
+  const gdr::FwdProblem &f = p.f;
+  LocalParams lp;
+  lp.T = f.T; lp.H = f.H; lp.NC = (f.T + C - 1) / C;
+  lp.decay = f.variant != gdr::kDeltaNet;
+  lp.kla = f.variant == gdr::kKLA;
+  lp.eps = f.eps; lp.scale = f.scale;
+  lp.q = static_cast<const __nv_bfloat16 *>(f.q);
+  lp.k = static_cast<const __nv_bfloat16 *>(f.k);
+  lp.v = static_cast<const __nv_bfloat16 *>(f.v);
+  lp.d_o = static_cast<const __nv_bfloat16 *>(p.d_o);
+  lp.beta = f.beta; lp.log_g = f.log_g;
+  lp.s0s = s0s; lp.dss = dss; lp.absmax = absmax;
+  lp.dq = static_cast<__nv_bfloat16 *>(p.dq);
+  lp.dk = static_cast<__nv_bfloat16 *>(p.dk);
+  lp.dv = static_cast<__nv_bfloat16 *>(p.dv);
+  lp.dbeta = p.dbeta; lp.dlog_g = p.dlog_g;
+  const int grid = f.B * f.H * lp.NC;
+  auto run = [&](auto kern, size_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NT, smem, s>>>(lp);
+    return cudaGetLastError();
+  };
+  return f.dv == 128 ? run(bwd_local_kernel<128>, LocalSmem<128>::BYTES)
+                     : run(bwd_local_kernel<64>, LocalSmem<64>::BYTES);
+}
+
+cudaError_t gdr_bwd_launch_unscale(const gdr::BwdProblem &p, const float *xf, const uint32_t *absmax,
+                                   cudaStream_t s) {
+  using namespace gdr::tc;
+  if (p.d_s0 == nullptr) return cudaSuccess;
+  const size_t n = static_cast<size_t>(p.f.B) * p.f.H * p.f.dk * p.f.dv;
+  bwd_unscale_kernel<<<grid_for(n), 256, 0, s>>>(xf, n, absmax, p.d_s0);
+  return cudaGetLastError();
+}
+
+int gdr_bwd_read_device_error(cudaStream_t s) {
+  if (cudaStreamSynchronize(s) != cudaSuccess) return -1;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gdr_bwd_error, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_gdr_bwd_error, &z, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}

@@ -53,7 +53,9 @@
 #include <cstring>
 #include <mutex>
 
+#include "chunk_bwd.cuh"
 #include "chunk_common.cuh"
+#include "chunk_record.cuh"
 #include "chunk_split.cuh"
 #include "tc_util.cuh"
 #include "tma_host.cuh"
@@ -74,22 +76,10 @@ namespace gdr {
 namespace tc {
 namespace {
 
-constexpr int C = 64;
-constexpr int DK = 128;
 constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float F16_SAFE = 60000.f;
 
-constexpr uint32_t REC_WQ = 0;
-constexpr uint32_t REC_K = 32768;
-constexpr uint32_t REC_P = 49152;
-constexpr uint32_t REC_U = 57344;
-__host__ __device__ constexpr uint32_t rec_sc(int ns) { return REC_U + 8192 * ns; }
-__host__ __device__ constexpr uint32_t rec_bytes(int ns) { return rec_sc(ns) + 16; }
-// channel decay: Gamma_C is a vector of d_k = 128 floats
-__host__ __device__ constexpr uint32_t rec_bytes_chan(int ns) { return rec_sc(ns) + 4 * 128; }
-// GDN-2: the channel-decay record, then (P^d V)^T (8 KB per 64 values) and (Dt^T V)^T (16 KB per 64 values)
-__host__ __device__ constexpr uint32_t rec_bytes_gdn2(int ns) { return rec_bytes_chan(ns) + 24576 * ns; }
 
 // ------------------------------------------------------------------ preparation kernel
 // Three CTAs share an SM (72 KB of shared memory, 128 tensor-memory columns
@@ -1393,6 +1383,7 @@ enum CarryFlags : int {
   CARRY_LAST_FINAL = 8,   // only the last segment writes s_final
   CARRY_S0_FIRST = 16,    // only segment 0 starts from s0, the others from zero
   CARRY_FAULT_MISSING_COPY = 32,   // host fault injection (see the issuer's prologue)
+  CARRY_WRITE_STATES = 64,   // write every chunk's start state to `states` (fp32 [B,H,NC,d_k,d_v])
 };
 
 struct CarryParams {
@@ -1411,6 +1402,7 @@ struct CarryParams {
   float *s_final_b;
   size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
+  float *states;   // CARRY_WRITE_STATES output, indexed by (b, h, chunk)
 };
 
 // max |x_i| over 16 values as a tree (four levels instead of a chain of 16).
@@ -1610,9 +1602,15 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 #pragma unroll
       for (int j = 0; j < 2; ++j) od_raw[j] = (has_v && values) ? __ldg(od + j) : make_uint4(0u, 0u, 0u, 0u);
     };
+    const size_t chunk0 = (static_cast<size_t>(b) * p.H + h) * p.NC + c_first;   // this CTA's first chunk, all (b, h)
     for (int c = 0; c < NC; ++c) {
       uint8_t *st = sm + (c % NSTAGE) * STAGE;
       const uint32_t y = lrow + COL_Y + 128 * (c & 1);
+      if ((flags & CARRY_WRITE_STATES) && has_v) {   // S (fp32) at the chunk's start: rows 32 part .., column v
+        float *dst = p.states + ((chunk0 + c) * DK + 32 * part) * p.dv + v;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
+      }
 
       // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15; U'^T is read from the
       // stage before Y(c) is waited for
@@ -1971,6 +1969,7 @@ struct CarryLaunch {
   int segments_b = 0, seg_first_b = 0, flags_b = 0;
   float *s_final_b = nullptr;
   size_t s_final_b_stride = 0;
+  float *states = nullptr;   // CARRY_WRITE_STATES output
 };
 
 // `pdl`: launched with programmatic stream serialization, so that its CTAs may
@@ -2001,6 +2000,7 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.seg_first_b = l.seg_first_b; cp.flags_b = l.flags_b;
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
+  cp.states = l.states;
   // GDR_FAULT=wait (host-side fault injection for the failure-path tests): CTA
   // (0, 0, 0) never copies chunk 1's record, so its waits give up after their
   // limit (about a second).
@@ -2204,9 +2204,71 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, size_t ws_bytes, cudaStr
   return launch_carry<MODE>(p, NC, w, f, true, stream, err);
 }
 
+// The backward's steps on the stream (each the programmatic dependent of the
+// one before where the kernel supports it): the forward's records; a carry
+// that keeps every chunk's start state (no outputs); the gradient scale and
+// the reverse records; the reverse carry (third carry mode, over the reverse
+// records) keeping every chunk's end-state gradient; the chunk-local
+// gradients; the initial state's gradient.  Both carries run unsegmented.
+template <int VAR>
+cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t stream, std::string *err) {
+  constexpr int MODE = VAR == kKDA ? 1 : 0;
+  const FwdProblem &p = bp.f;
+  const int NC = (p.T + C - 1) / C;
+  const BwdLayout L = bwd_layout(VAR, p.B, p.T, p.H, p.dv);
+  float *s0s = reinterpret_cast<float *>(w + L.s0s), *dss = reinterpret_cast<float *>(w + L.dss);
+  float *x0 = reinterpret_cast<float *>(w + L.x0), *xf = reinterpret_cast<float *>(w + L.xf);
+  uint32_t *absmax = reinterpret_cast<uint32_t *>(w + L.absmax);
+  cudaError_t e = launch_prep_any<VAR>(p, NC, w + L.fwd_rec, PrepRange(), stream, err);
+  if (e != cudaSuccess) return e;
+  CarryLaunch lf;
+  lf.seg_len = NC;
+  lf.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
+  lf.s0 = p.s0;
+  lf.states = s0s;
+  if ((e = launch_carry<MODE>(p, NC, w + L.fwd_rec, lf, true, stream, err)) != cudaSuccess) return e;
+  if ((e = gdr_bwd_launch_scale(bp, absmax, x0, stream)) != cudaSuccess) {
+    *err = "gradient scale: ";
+    return e;
+  }
+  if ((e = gdr_bwd_launch_rev_prep(bp, w + L.fwd_rec, w + L.rev_rec, absmax, stream)) != cudaSuccess) {
+    *err = "reverse records: ";
+    return e;
+  }
+  CarryLaunch lr;
+  lr.seg_len = NC;
+  lr.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
+  lr.s0 = x0;
+  lr.s_final = xf;
+  lr.states = dss;
+  if ((e = launch_carry<2>(p, NC, w + L.rev_rec, lr, true, stream, err)) != cudaSuccess) return e;
+  if ((e = gdr_bwd_launch_local(bp, s0s, dss, absmax, stream)) != cudaSuccess) {
+    *err = "local gradients: ";
+    return e;
+  }
+  if ((e = gdr_bwd_launch_unscale(bp, xf, absmax, stream)) != cudaSuccess) *err = "initial-state gradient: ";
+  return e;
+}
+
 }  // namespace
 }  // namespace tc
 }  // namespace gdr
+
+cudaError_t gdr_launch_backward(const gdr::BwdProblem &p, void *ws, size_t ws_bytes, cudaStream_t stream,
+                                std::string *err) {
+  using namespace gdr;
+  if (ws_bytes < bwd_layout(p.f.variant, p.f.B, p.f.T, p.f.H, p.f.dv).total) {
+    *err = "workspace smaller than gdr_backward_workspace_size(): ";
+    return cudaErrorInvalidValue;
+  }
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  switch (p.f.variant) {
+    case kDeltaNet: return tc::launch_backward<kDeltaNet>(p, w, stream, err);
+    case kGatedDeltaNet: return tc::launch_backward<kGatedDeltaNet>(p, w, stream, err);
+    case kKLA: return tc::launch_backward<kKLA>(p, w, stream, err);
+    default: *err = "variant not covered by the backward: "; return cudaErrorInvalidValue;
+  }
+}
 
 bool gdr_split_supported(int variant, int dk, int dv) {
   using namespace gdr;

@@ -140,3 +140,10 @@ def random_state(B: int, H: int, dk: int, dv: int, seed: int, scale: float = 0.5
     """A seeded fp32 state [B,H,dk,dv] (for initial-state and decode tests)."""
     g = torch.Generator().manual_seed(int(seed))
     return (scale * torch.randn(B, H, dk, dv, generator=g)).contiguous()
+
+
+def random_output_grad(B: int, T: int, H: int, dv: int, seed: int, dtype: torch.dtype = torch.bfloat16,
+                       scale: float = 1.0) -> torch.Tensor:
+    """A seeded gradient of the outputs d_o [B,T,H,dv] ~ scale * N(0, 1) (for the backward)."""
+    g = torch.Generator().manual_seed(int(seed))
+    return (scale * torch.randn(B, T, H, dv, generator=g)).to(dtype).contiguous()

@@ -11,7 +11,7 @@ import ctypes
 
 import torch
 
-from ._lib import FwdArgs, check, lib
+from ._lib import BwdGrads, FwdArgs, check, lib
 
 VARIANTS = {"deltanet": 0, "gdn": 1, "kda": 2, "gdn2": 3, "kla": 4}
 RAW_INPUTS = 0x100   # GDR_RAW_INPUTS (include/gdr.h)
@@ -127,6 +127,53 @@ def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=No
     check(L.gdr_forward_chunked(vflag, dt, B, T, H, dk, dv, ctypes.byref(a), float(eps), float(scale),
                                 int(chunk), _ptr(workspace), ws, _stream(stream, dev)))
     return out, final_state
+
+
+def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, initial_state=None, d_final_state=None,
+             eps=1e-6, scale=1.0, stream=None):
+    """Gradients of <d_o, o> + <d_final_state, S_T> for the forward over the
+    same inputs: the chunked backward (DeltaNet, Gated DeltaNet, KLA; bf16
+    q, k, v, d_o with dk = 128, dv 64 or 128; gates fp32 as for forward()).
+    Returns a dict with dq, dk, dv (bf16), beta (d beta, or d eta for KLA),
+    log_g (None for DeltaNet) and initial_state (fp32 [B,H,dk,dv]; the
+    gradient of the initial state, zero-initial-state runs included)."""
+    vid = variant_id(variant)
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    if q.dtype not in _DTYPES:
+        raise ValueError("q, k, v must be bf16 or fp32")
+    _need(k, "k", (B, T, H, dk), q.dtype, dev)
+    _need(v, "v", (B, T, H, dv), q.dtype, dev)
+    _need(d_o, "d_o", (B, T, H, dv), q.dtype, dev)
+    beta, log_g, _, _ = _gates(vid, (B, T, H), dk, dev, beta, log_g, None, None)
+    f32 = torch.float32
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), f32, dev)
+    if d_final_state is not None:
+        _need(d_final_state, "d_final_state", (B, H, dk, dv), f32, dev)
+    g = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+         "beta": torch.empty(B, T, H, device=dev, dtype=f32),
+         "log_g": None if log_g is None else torch.empty(B, T, H, device=dev, dtype=f32),
+         "initial_state": torch.empty(B, H, dk, dv, device=dev, dtype=f32)}
+    a = FwdArgs(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), beta=beta.data_ptr(),
+                log_g=None if log_g is None else log_g.data_ptr(),
+                initial_state=None if initial_state is None else initial_state.data_ptr())
+    gr = BwdGrads(dq=g["q"].data_ptr(), dk=g["k"].data_ptr(), dv=g["v"].data_ptr(), dbeta=g["beta"].data_ptr(),
+                  dlog_g=None if g["log_g"] is None else g["log_g"].data_ptr(),
+                  d_initial_state=g["initial_state"].data_ptr())
+    L = lib()
+    dt = _DTYPES[q.dtype]
+    ws = L.gdr_backward_workspace_size(vid, dt, B, T, H, dk, dv)
+    workspace = torch.empty(max(ws, 16), device=dev, dtype=torch.uint8)
+    check(L.gdr_backward(vid, dt, B, T, H, dk, dv, ctypes.byref(a), _ptr(d_o),
+                         _ptr(d_final_state), ctypes.byref(gr), float(eps), float(scale),
+                         _ptr(workspace), ws, _stream(stream, dev)))
+    return g
 
 
 def decode_step(q, k, v, state, *, variant, beta=None, log_g=None, erase_b=None, write_w=None,

@@ -217,6 +217,57 @@ gdr_status_t gdr_decode_step(int variant, int dtype, int N, int H, int dk, int d
                              const float *erase_b, const float *write_w,
                              float *state, void *o, float eps, float scale, void *stream);
 
+/* Backward-call gradients (outputs, caller-owned device memory).  Unused entries are NULL. */
+typedef struct {
+    void *dq;                 /* [B,T,H,dk] I/O dtype */
+    void *dk;                 /* [B,T,H,dk] I/O dtype */
+    void *dv;                 /* [B,T,H,dv] I/O dtype */
+    float *dbeta;             /* [B,T,H]: d beta, or d eta for KLA */
+    float *dlog_g;            /* [B,T,H] (GDN, KLA); DeltaNet: unused */
+    float *d_initial_state;   /* [B,H,dk,dv], or NULL when not wanted */
+} gdr_bwd_grads_t;
+
+/*
+ * Bytes of device workspace gdr_backward needs (0 for a case it does not
+ * cover): the forward's records, the reverse carry's records (B * H *
+ * ceil(T/64) of each), every chunk's start state and end-state gradient
+ * (fp32, dk * dv each), plus two states.
+ */
+size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv);
+
+/*
+ * Gradients of  <d_o, o> + <d_final_state, S_T>  with respect to the
+ * forward's inputs, for the forward that `args` describes (its o and
+ * final_state are not used): the gate-aware backward that keeps the
+ * chunkwise structure ("Gated DeltaNet-2: Decoupling Erase and Write in
+ * Linear Attention", technical core), for the scalar-decay variants DeltaNet,
+ * Gated DeltaNet and KLA with bf16 I/O, dk = 128 and dv in {64, 128}.  With S
+ * the state and dS its gradient, per 64-token chunk:
+ *     forward   E = U' - W S0,  O = Qg S0 + P E,  S_C = Gamma_C S0 + Kt^T E
+ *     backward  dE = Kt dS + P^T dO,  dS0 = Gamma_C dS + Qg^T dO - W^T dE
+ * ("Kaczmarz Linear Attention", KLA update rule and implementation: the
+ * chunkwise solver of Gated DeltaNet with KLA's diagonal step).  It re-runs
+ * the forward's chunk products and carry (keeping every chunk's start state),
+ * runs the dS recurrence through the same carry kernel over the chunks in
+ * reverse, then computes every chunk's q, k, v and gate gradients in
+ * parallel.  KLA's d eta includes the path through its Kaczmarz step
+ * eta / (||k||^2 + eps).  d_o [B,T,H,dv] in the I/O dtype (required);
+ * d_final_state [B,H,dk,dv] fp32 or NULL (zero).  The tensor-core carries use
+ * fp16 operands with fp32 accumulation, like the forward's chunked path: the
+ * gradients match an exact backward to about 1e-3 of their RMS; the
+ * gradients are rescaled internally by a power of two so that d_o's range
+ * does not matter.  workspace: at least gdr_backward_workspace_size() bytes,
+ * 16-byte aligned, overwritten.  The raw-input mode (GDR_RAW_INPUTS), KDA,
+ * GDN-2, fp32 I/O and dk = 64 return GDR_ERR_UNSUPPORTED.  T = 0 gives
+ * d_initial_state = d_final_state.  Validation and errors as for the
+ * forward; a reverse-record operand beyond the fp16 range is reported as
+ * GDR_ERR_RANGE by gdr_device_status().
+ */
+gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, int dv,
+                          const gdr_fwd_args_t *args, const void *d_o, const float *d_final_state,
+                          const gdr_bwd_grads_t *grads, float eps, float scale,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /*
  * Kernel launches one gdr_forward_chunked call with these arguments makes
  * (0 if the call would be rejected), and a short name of the kernel that runs
@@ -256,8 +307,10 @@ gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms,
  *   GDR_ERR_RANGE    a chunked-kernel operand left its range: an fp16 carry
  *                    operand (state, residual, W) above 6e4 in magnitude, or a
  *                    channel-wise decay spanning more than 2^120 within one
- *                    64-token chunk; the results of that call are unreliable
- *                    and chunk=1 (per-token fp32) is the safe path;
+ *                    64-token chunk, or (backward) a reverse-carry operand
+ *                    above 6e4; the results of that call are unreliable
+ *                    and, for the forward, chunk=1 (per-token fp32) is the
+ *                    safe path;
  *   GDR_ERR_CUDA     the synchronisation failed;
  *   GDR_OK           otherwise.
  */

@@ -230,3 +230,44 @@ def test_raw_input_flag_is_accepted_everywhere(L):
     i = ctypes.c_void_p
     assert L.gdr_decode_step(1 | RAW, 1, 4, 2, 128, 128, i(FAKE), i(FAKE), i(FAKE), i(FAKE), i(FAKE), None,
                              None, i(FAKE), i(FAKE), 1e-6, 1.0, None) == 4
+
+
+def bwd_call(L, variant=1, dtype=1, B=2, T=130, H=3, dk=128, dv=128, ws=None, d_o=FAKE, grads=None, a=None,
+             eps=1e-6):
+    a = a or args(initial_state=FAKE)
+    g = grads or _lib.BwdGrads(dq=FAKE, dk=FAKE, dv=FAKE, dbeta=FAKE, dlog_g=FAKE, d_initial_state=FAKE)
+    need = L.gdr_backward_workspace_size(variant, dtype, B, T, H, dk, dv)
+    return L.gdr_backward(variant, dtype, B, T, H, dk, dv, ctypes.byref(a), d_o, FAKE, ctypes.byref(g),
+                          eps, 1.0, FAKE, need if ws is None else ws, None)
+
+
+def test_backward_validation(L):
+    assert bwd_call(L) == 4                                  # valid: reaches the (injected) launch failure
+    for v in (0, 1, 4):
+        assert bwd_call(L, variant=v) == 4
+    assert bwd_call(L, variant=2) == 2 and bwd_call(L, variant=3) == 2     # KDA, GDN-2: unsupported
+    assert bwd_call(L, variant=1 | 0x100) == 2                               # raw inputs: unsupported
+    assert bwd_call(L, dtype=0) == 2 and bwd_call(L, dk=64) == 2             # fp32 I/O, dk = 64
+    assert bwd_call(L, dv=96) == 2
+    assert bwd_call(L, variant=9) == 1 and bwd_call(L, T=-1) == 1
+    assert bwd_call(L, ws=16) == 1                                           # workspace too small
+    assert bwd_call(L, d_o=None) == 1
+    assert bwd_call(L, d_o=MISALIGNED) == 3
+    g = _lib.BwdGrads(dq=FAKE, dk=FAKE, dv=FAKE, dbeta=FAKE, dlog_g=None, d_initial_state=None)
+    assert bwd_call(L, grads=g) == 1                                         # GDN needs dlog_g
+    assert bwd_call(L, variant=0, grads=g) == 4                              # DeltaNet does not
+    assert bwd_call(L, a=args(log_g=None, initial_state=FAKE)) == 1          # GDN needs log_g
+    assert bwd_call(L, eps=-1.0) == 1
+    assert bwd_call(L, B=0) == 0                                             # empty batch: nothing to do
+
+
+def test_backward_workspace_sizes(L):
+    # forward records + reverse records + two fp32 states per chunk + two states
+    B, T, H, NC, bh = 8, 2048, 8, 32, 64
+    rec, rev = 57344 + 8192 * 2 + 16, 57344 + 8192 * 2 + 512 + 24576 * 2
+    up = lambda x: (x + 255) // 256 * 256
+    want = up(bh * NC * rec) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
+    assert L.gdr_backward_workspace_size(1, 1, B, T, H, 128, 128) == want
+    assert L.gdr_backward_workspace_size(2, 1, B, T, H, 128, 128) == 0       # KDA
+    assert L.gdr_backward_workspace_size(1, 0, B, T, H, 128, 128) == 0       # fp32 I/O
+    assert L.gdr_backward_workspace_size(1, 1, B, 0, H, 128, 128) == 0

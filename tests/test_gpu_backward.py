@@ -1,0 +1,130 @@
+"""GPU parity of the chunked backward (DeltaNet, Gated DeltaNet, KLA) against
+the fp64 reverse-mode oracle, through the C ABI.
+
+The backward re-runs the forward's chunk products and carry, runs the
+end-state-gradient recurrence on the forward's carry kernel over the chunks in
+reverse, and computes each chunk's gradients in fp32.  Its carries use fp16
+operands with fp32 accumulation, as the forward's chunked path does, so the
+bar is the forward's (tests/parity_util.py): bf16 gradients (dq, dk, dv)
+within 2e-2 of RMS beyond their own bf16 rounding (and 3.56e-2 plain on the
+bulk), fp32 gradients (d beta / d eta, d log_g, the initial state's) within
+2e-2 of RMS.  The oracle sees the bf16-rounded inputs up-cast exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_forward_b200 as gdr
+import oracle
+from gated_delta_rule_forward_b200.inputs import make_inputs, random_output_grad, random_state
+from parity_util import assert_close, select, to_dev
+
+pytestmark = pytest.mark.gpu
+VARS = ["deltanet", "gdn", "kla"]
+
+
+def run_backward(variant, B, T, H, dv=128, seed=0, s0=True, d_final=True, do_scale=1.0, scale=None, edit=None):
+    dk = 128
+    scale = dk ** -0.5 if scale is None else scale
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=seed)
+    if edit is not None:
+        edit(d)
+    S0 = random_state(B, H, dk, dv, seed + 1) if s0 else None
+    dS = random_state(B, H, dk, dv, seed + 2, scale=1.0) if d_final else None
+    dO = random_output_grad(B, T, H, dv, seed + 3, scale=do_scale)
+    dd = to_dev(d)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, beta=dd["beta"], log_g=dd["log_g"],
+                     initial_state=None if S0 is None else S0.cuda(),
+                     d_final_state=None if dS is None else dS.cuda(), scale=scale)
+    gdr.device_status()
+    ref = oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"],
+                          initial_state=S0, d_final=dS, scale=scale)
+    return g, ref
+
+
+def check_grads(g, ref, variant, what=""):
+    for name in ("q", "k", "v"):
+        assert_close(g[name], ref[name], torch.bfloat16, f"{what} d{name}")
+    assert_close(g["beta"], ref["beta"], torch.bfloat16, f"{what} d{'eta' if variant == 'kla' else 'beta'}")
+    if variant != "deltanet":
+        assert_close(g["log_g"], ref["log_g"], torch.bfloat16, f"{what} dlog_g")
+    assert_close(g["initial_state"], ref["initial_state"], torch.bfloat16, f"{what} d initial state")
+
+
+@pytest.mark.parametrize("dv", [128, 64])
+@pytest.mark.parametrize("variant", VARS)
+def test_backward_small_ragged(variant, dv):
+    """Four chunks, the last one ragged (200 = 3 x 64 + 8), with an initial
+    state and a final-state gradient."""
+    g, ref = run_backward(variant, 2, 200, 3, dv=dv, seed=21)
+    check_grads(g, ref, variant)
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 65, 128])
+def test_backward_short_sequences(T):
+    """One partial chunk, one full chunk, one token past a chunk boundary."""
+    g, ref = run_backward("gdn", 1, T, 2, seed=22)
+    check_grads(g, ref, "gdn", f"T={T}")
+
+
+def test_backward_without_states():
+    """No initial state and no final-state gradient: the initial state's
+    gradient is still returned (that of a zero initial state)."""
+    g, ref = run_backward("gdn", 2, 150, 2, seed=23, s0=False, d_final=False)
+    check_grads(g, ref, "gdn")
+
+
+def test_backward_zero_length():
+    """T = 0: no token gradients; the initial state's gradient is the final state's."""
+    dS = random_state(1, 2, 128, 128, 5).cuda()
+    z = torch.empty(1, 0, 2, 128, device="cuda", dtype=torch.bfloat16)
+    beta = torch.empty(1, 0, 2, device="cuda")
+    g = gdr.backward(z, z, z, z, variant="gdn", beta=beta, log_g=beta, d_final_state=dS)
+    torch.cuda.synchronize()
+    assert torch.equal(g["initial_state"], dS)
+
+
+@pytest.mark.parametrize("do_scale", [1e-6, 1e4])
+def test_backward_gradient_magnitudes(do_scale):
+    """Output gradients far from unit scale: the internal power-of-two rescaling
+    keeps the fp16 operands of the reverse carry in range."""
+    g, ref = run_backward("kla", 2, 160, 2, seed=24, d_final=False, do_scale=do_scale)
+    check_grads(g, ref, "kla", f"d_o x {do_scale:g}")
+
+
+def test_backward_strong_decay():
+    """A decay logit scaled by 6 (log g down to about -20 per token): decay
+    enters only through factors at most 1, so nothing overflows."""
+    def edit(d):
+        d["log_g"] = (d["log_g"] * 6.0).contiguous()
+    g, ref = run_backward("gdn", 1, 192, 2, seed=25, edit=edit)
+    check_grads(g, ref, "gdn", "strong decay")
+
+
+@pytest.mark.parametrize("variant", ["gdn", "kla"])
+def test_backward_350m_layer_sampled(variant):
+    """The 350M layer (B=8, T=2048, H=8, full size, in the launch configuration of
+    a training step), checked against the oracle on two of its sequences."""
+    B, T, H = 8, 2048, 8
+    dk = dv = 128
+    scale = dk ** -0.5
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=26)
+    dO = random_output_grad(B, T, H, dv, 27)
+    dd = to_dev(d)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, beta=dd["beta"], log_g=dd["log_g"],
+                     scale=scale)
+    gdr.device_status()
+    for b in (0, B - 1):
+        s = select(d, b=slice(b, b + 1))
+        ref = oracle.backward(variant, s["q"], s["k"], s["v"], dO[b:b + 1], beta=s["beta"], log_g=s["log_g"],
+                              scale=scale)
+        gb = {k: (None if x is None else x[b:b + 1]) for k, x in g.items()}
+        check_grads(gb, ref, variant, f"sequence {b}")
+
+
+def test_backward_rejects_uncovered_cases():
+    d = to_dev(make_inputs("kda", 1, 64, 1))
+    dO = torch.zeros(1, 64, 1, 128, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(gdr.GdrError) as e:
+        gdr.backward(d["q"], d["k"], d["v"], dO, variant="kda", beta=d["beta"], log_g=d["log_g"])
+    assert e.value.status == 2   # GDR_ERR_UNSUPPORTED
