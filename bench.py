@@ -11,9 +11,9 @@ q/k/v/o, fp32 state, B=1 T=65536 H=16 dk=dv=128.  The line also carries the
 other workloads ("also": KLA on the same shape, the 350M-model layer (GDN and
 DeltaNet, B=8 T=2048 H=8), KDA / KLA / GDN-2 at the 1.3B-model shape, and
 the decode of 256 sequences x 16 heads: 1024 seeded steps from the
-long-context forward's final state, broadcast, and the 350M layer fed raw
-projections and logits, the kernels applying the input transforms), each
-with its own roofline:
+long-context forward's final state, broadcast, the 350M layer fed raw
+projections and logits, the kernels applying the input transforms, and the
+350M layer's chunked backward), each with its own roofline:
 achieved HBM bandwidth of the algorithmic bytes, and for the forwards also
 the tensor-core rate of the chunked algorithm's flops.
 
@@ -54,7 +54,9 @@ WORKLOADS = {
     "kla_fwd_64k": ("kla", 1, 65536, 16, 128, 128),
     "gdn_decode_256x16": ("gdn", 256, None, 16, 128, 128),
     "gdn_fwd_350m_raw": ("gdn", 8, 2048, 8, 128, 128),
+    "gdn_bwd_350m": ("gdn", 8, 2048, 8, 128, 128),
 }
+BWD_WORKLOADS = {"gdn_bwd_350m"}   # the chunked backward (gradients of o and the final state)
 RAW_WORKLOADS = {"gdn_fwd_350m_raw"}   # raw projections and logits in; the kernels apply the transforms
 DEFAULT = "gdn_fwd_64k"
 DECODE_STEPS = 1024         # the decode chain after the long-context prefill
@@ -68,6 +70,7 @@ KERNEL_SOURCES = {   # sources whose text keys a recorded ncu traffic figure
     "token_bf16io": [_CSRC + "token_fwd.cu"],
     "token_f32io": [_CSRC + "token_fwd.cu"],
     "decode": [_CSRC + "decode.cu"],
+    "chunk64_backward": [_CSRC + "chunk_bwd.cu", _CSRC + "chunk_bwd.cuh", _CSRC + "chunk_split.cu"] + _TC,
 }
 
 
@@ -140,6 +143,19 @@ def fwd_flops(variant, B, T, H, dk, dv, C=64):
     d = dk
     per = (18 * C * d + 8 * d * d) if variant == "gdn2" else (10 * C * d + 6 * d * d)
     return B * T * H * per
+
+
+def bwd_bytes(variant, B, T, H, dk, dv, io_bytes=2):
+    """Algorithmic HBM bytes of one backward call: q, k, v, d_o and the gates
+    read once; dq, dk, dv, the gate gradients and the initial state's gradient
+    written once (no initial state, no final-state gradient)."""
+    th = B * T * H
+    b = th * (2 * dk + 2 * dv) * io_bytes + th * (2 * dk + dv) * io_bytes
+    b += th * 4 * 2                                    # beta in, d beta out
+    if variant in ("gdn", "kla"):
+        b += th * 4 * 2                                # log decay in, its gradient out
+    b += B * H * dk * dv * 4                           # initial state's gradient
+    return b
 
 
 def decode_bytes(variant, N, H, dk, dv, io_bytes=2):
@@ -288,6 +304,44 @@ def run_forward_workload(name, K, W, world, e2e=False, seed=0):
     res["value"] = job_throughput(B * T, K, total_ms, world)
     if e2e:
         res["e2e"] = forward_e2e(name, host, K, W, world)
+    return res
+
+
+def run_backward_workload(name, K, W, world, seed=0):
+    """The chunked backward of a forward workload: the gradients of <d_o, o> with
+    respect to every input (the forward's products and carry re-run inside)."""
+    import gated_delta_rule_forward_b200 as gdr
+    from gated_delta_rule_forward_b200.inputs import random_output_grad
+    variant, B, T, H, dk, dv = WORKLOADS[name]
+    sets, _ = make_device_sets(name, seed)
+    grads = [random_output_grad(B, T, H, dv, seed + 11 + j).cuda() for j in range(2)]
+
+    def step(i):
+        d = sets[i % 2]
+        gdr.backward(d["q"], d["k"], d["v"], grads[i % 2], variant=variant, beta=d["beta"], log_g=d["log_g"],
+                     scale=dk ** -0.5)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_wall0 = time.time()
+    for i in range(K):
+        starts[i].record()
+        step(i)
+        ends[i].record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), world)
+    res = {"workload": name, "variant": variant, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+           "kernel": "chunk64_backward", "launches_per_step": 9, "ms_per_step": total_ms / K,
+           "launch_ms": sum(per) / K, "tokens_per_step": B * T, "wall": (t_wall0, t_wall1),
+           "alg_bytes": bwd_bytes(variant, B, T, H, dk, dv)}
+    res["value"] = job_throughput(B * T, K, total_ms, world)
     return res
 
 
@@ -529,8 +583,12 @@ def native(args):
             if name == args.workload:
                 continue
             k = max(3, args.steps // 4) if "64k" in name else args.steps
-            r = (run_decode_workload(name, k, args.warmup, world, chain=True, seed=rank)
-                 if WORKLOADS[name][2] is None else run_forward_workload(name, k, args.warmup, world, seed=rank))
+            if name in BWD_WORKLOADS:
+                r = run_backward_workload(name, max(3, args.steps // 4), args.warmup, world, seed=rank)
+            elif WORKLOADS[name][2] is None:
+                r = run_decode_workload(name, k, args.warmup, world, chain=True, seed=rank)
+            else:
+                r = run_forward_workload(name, k, args.warmup, world, seed=rank)
             r["roofline"] = roofline(r, peaks)
             if "alg_flops" in r:
                 r["roofline_tensor"] = roofline_tensor(r, peaks)
@@ -616,7 +674,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT, choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT, choices=[w for w in WORKLOADS if w not in BWD_WORKLOADS])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-also", action="store_true", help="only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")

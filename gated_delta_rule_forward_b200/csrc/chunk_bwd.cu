@@ -36,6 +36,7 @@
 // the final-state gradient are scaled by a power of two s (max |.| to [0.5, 1)),
 // and the local kernel and the initial-state gradient divide it out again.
 #include <algorithm>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -55,7 +56,14 @@ constexpr int NT = 256;
 constexpr float F16_SAFE_BWD = 60000.f;
 constexpr float LOG2E_BWD = 1.4426950408889634f;
 
-// ---------------------------------------------------------------- SIMT products
+// ---------------------------------------------------------------- warp-tile products
+// The products run on the tensor cores through the warp-level tf32 MMA
+// (m16n8k8, fp32 accumulation): a CTA's eight warps tile an M x N product
+// (M, N in {64, 128}) into 16-row tiles, each warp covering 16 rows and N * RT
+// / 64 columns, RT = M / 16 row tiles.  Operands come from shared or global
+// memory through views that may transpose them, so every product of the
+// chunk algebra is written as it reads.
+//
 // A matrix operand: element (r, c) is p[r * ld + c], or p[c * ld + r] for TR.
 // GLOBAL operands are read through the read-only cache.
 template <typename E, bool TR, bool GLOBAL = false>
@@ -68,22 +76,6 @@ struct Mat {
 };
 
 template <typename E, bool G>
-__device__ __forceinline__ void ld4(const E *p, float (&x)[4]);
-template <>
-__device__ __forceinline__ void ld4<float, false>(const float *p, float (&x)[4]) {
-  const float4 v = *reinterpret_cast<const float4 *>(p);
-  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void ld4<float, true>(const float *p, float (&x)[4]) {
-  const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
-  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void ld4<__nv_bfloat16, false>(const __nv_bfloat16 *p, float (&x)[4]) {
-  unpack4(*reinterpret_cast<const uint2 *>(p), x);
-}
-template <typename E, bool G>
 __device__ __forceinline__ float ld1(const E *p);
 template <>
 __device__ __forceinline__ float ld1<float, false>(const float *p) { return *p; }
@@ -92,76 +84,95 @@ __device__ __forceinline__ float ld1<float, true>(const float *p) { return __ldg
 template <>
 __device__ __forceinline__ float ld1<__nv_bfloat16, false>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
-// acc[i][j] (+/-)= sum_{k < K} A(r0 + i, k) ks[k] B(k, c0 + 16 j): a thread's
-// MR x NR tile of rows r0 .. r0 + MR - 1 and columns c0, c0 + 16, ...  (ks, a
-// per-k factor in shared memory, may be null).  K is a multiple of 4, and r0
-// of 4 where A is TR.
-template <int MR, int NR, bool NEG, typename MA, typename MB>
-__device__ __forceinline__ void mm(float (&acc)[MR][NR], const MA a, const MB b, int K, int r0, int c0,
-                                   const float *ks = nullptr) {
-  using EA = typename MA::elem;
-  using EB = typename MB::elem;
-#pragma unroll 2
-  for (int k0 = 0; k0 < K; k0 += 4) {
-    float af[MR][4], bf[4][NR];
-    if constexpr (!MA::kTr) {
+template <typename V>
+__device__ __forceinline__ float at(const V &m, int r, int c) {
+  return ld1<typename V::elem, V::kGlobal>(m.p + (V::kTr ? c * m.ld + r : r * m.ld + c));
+}
+// The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N product.
+template <int M, int N>
+struct Tiling {
+  static constexpr int RT = M / 16;          // row tiles
+  static constexpr int CH = 8 / RT;          // column parts
+  static constexpr int NT = N / 8 / CH;      // 8-column MMA tiles per warp
+  static __device__ __forceinline__ int m0(int w) { return 16 * (w % RT); }
+  static __device__ __forceinline__ int n0(int w) { return (w / RT) * (N / CH); }
+};
+
+// acc (+/-)= A(m0.., k) ks[k] B(k, n0..) over k < K (a multiple of 8); ks, a
+// per-k factor in shared memory, may be null.  acc[j] is the m16n8 fragment of
+// columns n0 + 8 j .. n0 + 8 j + 7: {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}
+// with g = lane / 4, t = lane % 4.  PRECISE: each fp32 operand is split into
+// two tf32 parts, x = hi + lo, and the product taken as a_hi b_hi + a_lo b_hi +
+// a_hi b_lo (three-pass tf32: about fp32 accuracy; a bf16 operand is exact in
+// tf32 and has no lo part, so its products take two passes).  Otherwise one
+// tf32 pass (for results that are stored in fp16 anyway).
+template <typename V>
+__device__ __forceinline__ void split(const V &m, int r, int c, float scale, uint32_t &hi, uint32_t &lo) {
+  const float x = at(m, r, c) * scale;
+  hi = std::is_same<typename V::elem, __nv_bfloat16>::value && scale == 1.f ? __float_as_uint(x) : to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+template <int NT, bool NEG, typename MA, typename MB, bool PRECISE = true>
+__device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b, int K, int m0, int n0, int lane,
+                                    const float *ks = nullptr) {
+  constexpr bool a_exact = !PRECISE || std::is_same<typename MA::elem, __nv_bfloat16>::value;
+  const bool b_exact = !PRECISE || (std::is_same<typename MB::elem, __nv_bfloat16>::value && ks == nullptr);
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[4], al[4];
+    split(a, m0 + g, k0 + t, 1.f, ah[0], al[0]);
+    split(a, m0 + g + 8, k0 + t, 1.f, ah[1], al[1]);
+    split(a, m0 + g, k0 + t + 4, 1.f, ah[2], al[2]);
+    split(a, m0 + g + 8, k0 + t + 4, 1.f, ah[3], al[3]);
+    if (NEG) {
 #pragma unroll
-      for (int i = 0; i < MR; ++i) ld4<EA, MA::kGlobal>(a.p + (r0 + i) * a.ld + k0, af[i]);
-    } else {
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int i4 = 0; i4 < MR; i4 += 4) {
-          float x[4];
-          ld4<EA, MA::kGlobal>(a.p + (k0 + kk) * a.ld + r0 + i4, x);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) af[i4 + e][kk] = x[e];
-        }
-    }
-    if constexpr (!MB::kTr) {
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int j = 0; j < NR; ++j) bf[kk][j] = ld1<EB, MB::kGlobal>(b.p + (k0 + kk) * b.ld + c0 + 16 * j);
-    } else {
-#pragma unroll
-      for (int j = 0; j < NR; ++j) {
-        float x[4];
-        ld4<EB, MB::kGlobal>(b.p + (c0 + 16 * j) * b.ld + k0, x);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) bf[kk][j] = x[kk];
+      for (int e = 0; e < 4; ++e) {
+        ah[e] ^= 0x80000000u;
+        al[e] ^= 0x80000000u;
       }
     }
-    if (ks != nullptr) {
+    const float s0 = ks != nullptr ? ks[k0 + t] : 1.f, s1 = ks != nullptr ? ks[k0 + t + 4] : 1.f;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const float f = ks[k0 + kk];
-#pragma unroll
-        for (int j = 0; j < NR; ++j) bf[kk][j] *= f;
-      }
+    for (int j = 0; j < NT; ++j) {
+      uint32_t bh0, bl0, bh1, bl1;
+      split(b, k0 + t, n0 + 8 * j + g, s0, bh0, bl0);
+      split(b, k0 + t + 4, n0 + 8 * j + g, s1, bh1, bl1);
+      if (!b_exact) mma_tf32_16x8x8(acc[j], ah, bl0, bl1);
+      if (!a_exact) mma_tf32_16x8x8(acc[j], al, bh0, bh1);
+      mma_tf32_16x8x8(acc[j], ah, bh0, bh1);
     }
-#pragma unroll
-    for (int i = 0; i < MR; ++i)
-#pragma unroll
-      for (int j = 0; j < NR; ++j)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) acc[i][j] = fmaf(NEG ? -af[i][kk] : af[i][kk], bf[kk][j], acc[i][j]);
   }
 }
 
-template <int MR, int NR>
-__device__ __forceinline__ void zero(float (&acc)[MR][NR]) {
+// f(row, col, value) for each accumulator element of a warp tile.
+template <int NT, typename F>
+__device__ __forceinline__ void each(float (&acc)[NT][4], int m0, int n0, int lane, F f) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int i = 0; i < MR; ++i)
+  for (int j = 0; j < NT; ++j)
 #pragma unroll
-    for (int j = 0; j < NR; ++j) acc[i][j] = 0.f;
+    for (int e = 0; e < 4; ++e) f(m0 + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[j][e]);
 }
 
-// Sum over the 16 lanes of a half warp (the column groups of one row group).
-__device__ __forceinline__ float half_warp_sum(float x) {
+template <int NT>
+__device__ __forceinline__ void zero(float (&acc)[NT][4]) {
 #pragma unroll
-  for (int o = 8; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+}
+
+// Sums over the lanes of a quad (the four lanes that share a row of a fragment)
+// and over the eight quads (the lanes that share a column).
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+__device__ __forceinline__ float column_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  x += __shfl_xor_sync(0xffffffffu, x, 8);
+  return x + __shfl_xor_sync(0xffffffffu, x, 16);
 }
 
 // The power of two s with s * max|gradient| in [0.5, 1) (1 when the maximum is
@@ -180,8 +191,13 @@ __global__ void bwd_absmax_kernel(const __nv_bfloat16 *d_o, size_t n_o, const fl
                                   uint32_t *out) {
   float m = 0.f;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_o; i += stride)
-    m = fmaxf(m, fabsf(__bfloat162float(d_o[i])));
+  const uint4 *o8 = reinterpret_cast<const uint4 *>(d_o);   // n_o is a multiple of 8 (d_v is)
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_o / 8; i += stride) {
+    float x[8];
+    unpack8(__ldg(o8 + i), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[e]));
+  }
   if (d_final != nullptr)
     for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_f; i += stride)
       m = fmaxf(m, fabsf(__ldg(d_final + i)));
@@ -286,34 +302,32 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
   }
   __syncthreads();
 
-  const int rg = tid >> 4, cg = tid & 15;
-  constexpr int MR = DV / 16;
+  const int warp = tid >> 5, lane = tid & 31;
   float vmax = 0.f;
   {   // R^T [v][t] into the U' slot (rows v, 128-byte swizzled)
-    float acc[MR][4];
+    using TL = Tiling<DV, C>;
+    float acc[TL::NT][4];
     zero(acc);
-    mm<MR, 4, false>(acc, Mat<float, true>{sO, LDO}, Mat<float, false>{sP, LDP}, C, MR * rg, cg);
-#pragma unroll
-    for (int i = 0; i < MR; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int v = MR * rg + i, t = cg + 16 * j;
-        vmax = fmaxf(vmax, fabsf(acc[i][j]));
-        *reinterpret_cast<__half *>(dst + REC_U + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(acc[i][j]);
-      }
+    const int m0 = TL::m0(warp), n0 = TL::n0(warp);
+    wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
+                                                                   Mat<float, false>{sP, LDP}, C, m0, n0, lane);
+    each(acc, m0, n0, lane, [&](int v, int t, float &x) {
+      vmax = fmaxf(vmax, fabsf(x));
+      *reinterpret_cast<__half *>(dst + REC_U + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(x);
+    });
   }
   {   // F^T [v][i] after the output term, unswizzled rows of d_k values
-    float acc[MR][8];
+    using TL = Tiling<DV, DK>;
+    float acc[TL::NT][4];
     zero(acc);
-    mm<MR, 8, false>(acc, Mat<float, true>{sO, LDO}, Mat<float, false>{sQ, LDQ}, C, MR * rg, cg);
+    const int m0 = TL::m0(warp), n0 = TL::n0(warp);
+    wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
+                                                                   Mat<float, false>{sQ, LDQ}, C, m0, n0, lane);
     __half *f = reinterpret_cast<__half *>(dst + rec_bytes_chan(NS) + 8192 * NS);
-#pragma unroll
-    for (int i = 0; i < MR; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        vmax = fmaxf(vmax, fabsf(acc[i][j]));
-        f[(MR * rg + i) * DK + cg + 16 * j] = __float2half_rn(acc[i][j]);
-      }
+    each(acc, m0, n0, lane, [&](int v, int i, float &x) {
+      vmax = fmaxf(vmax, fabsf(x));
+      f[v * DK + i] = __float2half_rn(x);
+    });
   }
   if (vmax > F16_SAFE_BWD) atomicOr(&g_gdr_bwd_error, 2);
 }
@@ -381,7 +395,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   float *snk = sdg + C;       // ||k||^2
   float *sred = snk + C;      // [0] sum X1 o K, [1] sum dS o S0
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = tid >> 4, cg = tid & 15;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x / p.NC, c = blockIdx.x - bh * p.NC;
   const int b = bh / p.H, h = bh - b * p.H;
   const int t0 = c * C, n = min(C, p.T - t0);
@@ -458,19 +472,28 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   }
   __syncthreads();
 
+  using CC = Tiling<C, C>;     // C x C products
+  using CV = Tiling<C, DV>;    // C x d_v
+  using CK = Tiling<C, DK>;    // C x d_k
+  using KC = Tiling<DK, C>;    // d_k x C (the transposed gradient tiles)
+  const int mc = CC::m0(warp), nc = CC::n0(warp);
+  const int mv = CV::m0(warp), nv = CV::n0(warp);
+  const int mk = CK::m0(warp), nk = CK::n0(warp);
+  const int mt = KC::m0(warp), nt = KC::n0(warp);
+  using BK = Mat<__nv_bfloat16, false>;   // a bf16 tile as stored
+  using BKT = Mat<__nv_bfloat16, true>;   // ... transposed
+  using F = Mat<float, false>;
+  using FT = Mat<float, true>;
+  using FG = Mat<float, false, true>;     // a global fp32 matrix (S0, dS)
+
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
-    float g[4][4];
+    float g[CC::NT][4];
     zero(g);
-    mm<4, 4, false>(g, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = 4 * rg + i, r = cg + 16 * j;
-        const float a = r < t ? sbeta[t] * ex2(sG[t] - sG[r]) * g[i][j] : 0.f;
-        sA[r * LD + t] = tf32r(a);
-      }
+    wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    each(g, mc, nc, lane, [&](int t, int r, float &x) {
+      sA[r * LD + t] = tf32r(r < t ? sbeta[t] * ex2(sG[t] - sG[r]) * x : 0.f);
+    });
   }
   __syncthreads();
   solve_unit_lower_64(sA, sT, tid, warp, lane);   // ends with a barrier
@@ -481,247 +504,204 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   __syncthreads();
 
   // ---- U' = T Diag(beta) V and W = T Diag(beta e) K; E = U' - W S0
-  float ue[4][NRV];
+  float ue[CV::NT][4];
   zero(ue);
-  mm<4, NRV, false>(ue, Mat<float, false>{sT, LD}, Mat<__nv_bfloat16, false>{sV, LDBV}, C, 4 * rg, cg, sbeta);
+  wmm<CV::NT, false>(ue, F{sT, LD}, BK{sV, LDBV}, C, mv, nv, lane, sbeta);
   {
-    float w[4][NRK];
+    float w[CK::NT][4];
     zero(w);
-    mm<4, NRK, false>(w, Mat<float, false>{sT, LD}, Mat<__nv_bfloat16, false>{sK, LDB}, C, 4 * rg, cg, sbe);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NRK; ++j) sW[(4 * rg + i) * LDW + cg + 16 * j] = w[i][j];
+    wmm<CK::NT, false>(w, F{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
+    each(w, mk, nk, lane, [&](int t, int i, float &x) { sW[t * LDW + i] = x; });
   }
   __syncthreads();
-  mm<4, NRV, true>(ue, Mat<float, false>{sW, LDW}, Mat<float, false, true>{S0, DV}, DK, 4 * rg, cg);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NRV; ++j) sE[(4 * rg + i) * LDF + cg + 16 * j] = ue[i][j];
+  wmm<CV::NT, true>(ue, F{sW, LDW}, FG{S0, DV}, DK, mv, nv, lane);
+  each(ue, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
   // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
   // reverse carry's own dE is Diag(beta) dE (its records carry beta in P and Kt), so it is
   // recomputed here rather than divided by beta.
   {
-    float gq[4][4];
+    float gq[CC::NT][4];
     zero(gq);
-    mm<4, 4, false>(gq, Mat<__nv_bfloat16, false>{sQ, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = 4 * rg + i, r = cg + 16 * j;
-        sP[t * LDC + r] = r <= t ? p.scale * ex2(sG[t] - sG[r]) * gq[i][j] : 0.f;
-      }
+    wmm<CC::NT, false>(gq, BK{sQ, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    each(gq, mc, nc, lane, [&](int t, int r, float &x) {
+      sP[t * LDC + r] = r <= t ? p.scale * ex2(sG[t] - sG[r]) * x : 0.f;
+    });
   }
   __syncthreads();
   {
-    float acc[4][NRV];
+    float acc[CV::NT][4];
     zero(acc);
-    mm<4, NRV, false>(acc, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<float, false, true>{dS, DV}, DK, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float f = sff[4 * rg + i] * inv_s;
-#pragma unroll
-      for (int j = 0; j < NRV; ++j) acc[i][j] *= f;
-    }
-    mm<4, NRV, false>(acc, Mat<float, true>{sP, LDC}, Mat<__nv_bfloat16, false>{sO, LDBV}, C, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NRV; ++j) sdE[(4 * rg + i) * LDF + cg + 16 * j] = acc[i][j];
+    wmm<CV::NT, false>(acc, BK{sK, LDB}, FG{dS, DV}, DK, mv, nv, lane);
+    each(acc, mv, nv, lane, [&](int t, int, float &x) { x *= sff[t] * inv_s; });
+    wmm<CV::NT, false>(acc, FT{sP, LDC}, BK{sO, LDBV}, C, mv, nv, lane);
+    each(acc, mv, nv, lane, [&](int t, int v, float &x) { sdE[t * LDF + v] = x; });
   }
   __syncthreads();
 
-  // ---- dk^T (rows i = 8 rg .., columns t = cg + 16 j) starts as (Diag(f) E dS^T)^T / s
-  float dkT[8][4];
-  float dgp[4] = {0.f, 0.f, 0.f, 0.f};   // this thread's share of dg_t, t = cg + 16 j
+  // ---- dk^T (d_k x C tiles) starts as (Diag(f) E dS^T)^T / s
+  float dkT[KC::NT][4];
+  float dgp[KC::NT][2];   // this thread's column sums toward dg_t (columns n0 + 8 j + 2 t + e)
   float x1k = 0.f;
   zero(dkT);
-  mm<8, 4, false>(dkT, Mat<float, false, true>{dS, DV}, Mat<float, true>{sE, LDF}, DV, 8 * rg, cg);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int t = cg + 16 * j;
-    const float ft = sff[t] * inv_s;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      dkT[i][j] *= ft;
-      const float x = dkT[i][j] * __bfloat162float(sK[t * LDB + 8 * rg + i]);
-      x1k += x;
-      dgp[j] -= x;
-    }
-  }
+  for (int j = 0; j < KC::NT; ++j) dgp[j][0] = dgp[j][1] = 0.f;
+  auto add_dg = [&](int col, float x) {   // col of the warp tile -> its dgp slot
+    dgp[(col - nt) >> 3][col & 1] += x;
+  };
+  wmm<KC::NT, false>(dkT, FG{dS, DV}, FT{sE, LDF}, DV, mt, nt, lane);
+  each(dkT, mt, nt, lane, [&](int i, int t, float &x) {
+    x *= sff[t] * inv_s;
+    const float y = x * __bfloat162float(sK[t * LDB + i]);
+    x1k += y;
+    add_dg(t, -y);
+  });
   // ---- dP = tril(dO E^T)
   {
-    float acc[4][4];
+    float acc[CC::NT][4];
     zero(acc);
-    mm<4, 4, false>(acc, Mat<__nv_bfloat16, false>{sO, LDBV}, Mat<float, true>{sE, LDF}, DV, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = 4 * rg + i, r = cg + 16 * j;
-        sP[t * LDC + r] = r <= t ? acc[i][j] : 0.f;
-      }
+    wmm<CC::NT, false>(acc, BK{sO, LDBV}, FT{sE, LDF}, DV, mc, nc, lane);
+    each(acc, mc, nc, lane, [&](int t, int r, float &x) { sP[t * LDC + r] = r <= t ? x : 0.f; });
   }
   // ---- dW^T = -S0 dE^T  (d_k x C, over W, which E = U' - W S0 has finished reading)
   {
-    float acc[8][4];
+    float acc[KC::NT][4];
     zero(acc);
-    mm<8, 4, true>(acc, Mat<float, false, true>{S0, DV}, Mat<float, true>{sdE, LDF}, DV, 8 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sW[(8 * rg + i) * LDC + cg + 16 * j] = acc[i][j];
+    wmm<KC::NT, true>(acc, FG{S0, DV}, FT{sdE, LDF}, DV, mt, nt, lane);
+    each(acc, mt, nt, lane, [&](int i, int t, float &x) { sW[i * LDC + t] = x; });
   }
   __syncthreads();
 
   // ---- dv = Diag(beta) T^T dE;  dbeta += rowsum(V o T^T dE)
   {
-    float acc[4][NRV];
+    float acc[CV::NT][4];
     zero(acc);
-    mm<4, NRV, false>(acc, Mat<float, true>{sT, LD}, Mat<float, false>{sdE, LDF}, C, 4 * rg, cg);
+    wmm<CV::NT, false>(acc, FT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
+    float part[2] = {0.f, 0.f};   // rows g and g + 8 of the tile
+    each(acc, mv, nv, lane, [&](int t, int v, float &x) {
+      part[(t - mv) >> 3] = fmaf(__bfloat162float(sV[t * LDBV + v]), x, part[(t - mv) >> 3]);
+      x *= sbeta[t];
+    });
+    const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = 4 * rg + i;
-      const float bt = sbeta[t];
-      float part = 0.f;
+    for (int j = 0; j < CV::NT; ++j)
 #pragma unroll
-      for (int j = 0; j < NRV; ++j) {
-        const int v = cg + 16 * j;
-        part = fmaf(__bfloat162float(sV[t * LDBV + v]), acc[i][j], part);
-        if (t < n) p.dv[row(t) * DV + v] = __float2bfloat16_rn(bt * acc[i][j]);
+      for (int h2 = 0; h2 < 2; ++h2) {   // two adjacent values per store
+        const int t = mv + g + 8 * h2, v = nv + 8 * j + 2 * tq;
+        if (t < n)
+          *reinterpret_cast<uint32_t *>(p.dv + row(t) * DV + v) = pack_bf16x2(acc[j][2 * h2], acc[j][2 * h2 + 1]);
       }
-      part = half_warp_sum(part);
-      if (cg == 0) atomicAdd(&sdb[t], part);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float s2 = quad_sum(part[h2]);
+      if (tq == 0) atomicAdd(&sdb[mv + g + 8 * h2], s2);
     }
   }
   // ---- (T^T dW)^T = dW^T T:  dk += Diag(beta e) T^T dW;  dbeta += e o rowsum(K o T^T dW)
   {
-    float acc[8][4];
+    float acc[KC::NT][4];
     zero(acc);
-    mm<8, 4, false>(acc, Mat<float, false>{sW, LDC}, Mat<float, false>{sT, LD}, C, 8 * rg, cg);
+    wmm<KC::NT, false>(acc, F{sW, LDC}, F{sT, LD}, C, mt, nt, lane);
+    float dbp[KC::NT][2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int t = cg + 16 * j;
-      const float bet = sbe[t], et = see[t];
-      float dbp = 0.f;
+    for (int j = 0; j < KC::NT; ++j) dbp[j][0] = dbp[j][1] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float kv = __bfloat162float(sK[t * LDB + 8 * rg + i]);
-        const float y = bet * acc[i][j];
-        dkT[i][j] += y;
-        dgp[j] = fmaf(y, kv, dgp[j]);
-        dbp = fmaf(et * kv, acc[i][j], dbp);
+    for (int j = 0; j < KC::NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = mt + (lane >> 2) + 8 * (e >> 1), t = nt + 8 * j + 2 * (lane & 3) + (e & 1);
+        const float kv = __bfloat162float(sK[t * LDB + i]);
+        const float y = sbe[t] * acc[j][e];
+        dkT[j][e] += y;
+        dgp[j][e & 1] = fmaf(y, kv, dgp[j][e & 1]);
+        dbp[j][e & 1] = fmaf(see[t] * kv, acc[j][e], dbp[j][e & 1]);
       }
-      dbp += __shfl_xor_sync(0xffffffffu, dbp, 16);
-      if (lane < 16) atomicAdd(&sdb[t], dbp);
-    }
+#pragma unroll
+    for (int j = 0; j < KC::NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float s2 = column_sum(dbp[j][e]);
+        if (lane < 4) atomicAdd(&sdb[nt + 8 * j + 2 * lane + e], s2);
+      }
   }
   // ---- dT = dE V^T Diag(beta) + dW K^T Diag(beta e)  (over A^T, dead since the solve)
   {
-    float a1[4][4], a2[4][4];
+    float a1[CC::NT][4], a2[CC::NT][4];
     zero(a1);
     zero(a2);
-    mm<4, 4, false>(a1, Mat<float, false>{sdE, LDF}, Mat<__nv_bfloat16, true>{sV, LDBV}, DV, 4 * rg, cg);
-    mm<4, 4, false>(a2, Mat<float, true>{sW, LDC}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+    wmm<CC::NT, false>(a1, F{sdE, LDF}, BKT{sV, LDBV}, DV, mc, nc, lane);
+    wmm<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < CC::NT; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = 4 * rg + i, r = cg + 16 * j;
-        sA[t * LD + r] = sbeta[r] * a1[i][j] + sbe[r] * a2[i][j];
+      for (int e = 0; e < 4; ++e) {
+        const int t = mc + (lane >> 2) + 8 * (e >> 1), r = nc + 8 * j + 2 * (lane & 3) + (e & 1);
+        sA[t * LD + r] = sbeta[r] * a1[j][e] + sbe[r] * a2[j][e];
       }
   }
   __syncthreads();
   // ---- X = dT T^T (over E), then dA = tril(-T^T X, -1) (over dT)
   {
-    float acc[4][4];
+    float acc[CC::NT][4];
     zero(acc);
-    mm<4, 4, false>(acc, Mat<float, false>{sA, LD}, Mat<float, true>{sT, LD}, C, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sE[(4 * rg + i) * LDC + cg + 16 * j] = acc[i][j];
+    wmm<CC::NT, false>(acc, F{sA, LD}, FT{sT, LD}, C, mc, nc, lane);
+    each(acc, mc, nc, lane, [&](int t, int r, float &x) { sE[t * LDC + r] = x; });
   }
   __syncthreads();
   {
-    float acc[4][4];
+    float acc[CC::NT][4];
     zero(acc);
-    mm<4, 4, true>(acc, Mat<float, true>{sT, LD}, Mat<float, false>{sE, LDC}, C, 4 * rg, cg);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = 4 * rg + i, r = cg + 16 * j;
-        sA[t * LD + r] = r < t ? acc[i][j] : 0.f;
-      }
+    wmm<CC::NT, true>(acc, FT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    each(acc, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = r < t ? x : 0.f; });
   }
   __syncthreads();
   // ---- G = K K^T again: dbeta += rowsum(dA o D o G); N1 = Diag(beta) (dA o D), N2 = scale (dP o D)
   {
-    float g[4][4];
+    float g[CC::NT][4];
     zero(g);
-    mm<4, 4, false>(g, Mat<__nv_bfloat16, false>{sK, LDB}, Mat<__nv_bfloat16, true>{sK, LDB}, DK, 4 * rg, cg);
+    wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    float part[2] = {0.f, 0.f};
+    each(g, mc, nc, lane, [&](int t, int r, float &x) {
+      const float d = r <= t ? ex2(sG[t] - sG[r]) : 0.f;
+      const float da = sA[t * LD + r];
+      part[(t - mc) >> 3] = fmaf(da * d, x, part[(t - mc) >> 3]);
+      sA[t * LD + r] = sbeta[t] * da * d;
+      sP[t * LDC + r] = p.scale * sP[t * LDC + r] * d;
+    });
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = 4 * rg + i;
-      float part = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = cg + 16 * j;
-        const float d = r <= t ? ex2(sG[t] - sG[r]) : 0.f;
-        const float da = sA[t * LD + r];
-        part = fmaf(da * d, g[i][j], part);
-        sA[t * LD + r] = sbeta[t] * da * d;
-        sP[t * LDC + r] = p.scale * sP[t * LDC + r] * d;
-      }
-      part = half_warp_sum(part);
-      if (cg == 0) atomicAdd(&sdb[t], part);
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float s2 = quad_sum(part[h2]);
+      if ((lane & 3) == 0) atomicAdd(&sdb[mc + (lane >> 2) + 8 * h2], s2);
     }
   }
   __syncthreads();
   // ---- dk += N1 K + N1^T K + N2^T Q   (as K^T N1^T, K^T N1, Q^T N2)
   {
-    float acc[8][4];
+    float acc[KC::NT][4];
     zero(acc);
-    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, true>{sA, LD}, C, 8 * rg, cg);
+    wmm<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
+    each(acc, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, x * __bfloat162float(sK[t * LDB + i])); });
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int j = 0; j < KC::NT; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        dkT[i][j] += acc[i][j];
-        dgp[j] = fmaf(acc[i][j], __bfloat162float(sK[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
-      }
+      for (int e = 0; e < 4; ++e) dkT[j][e] += acc[j][e];
     zero(acc);
-    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, false>{sA, LD}, C, 8 * rg, cg);
-    mm<8, 4, false>(acc, Mat<__nv_bfloat16, true>{sQ, LDB}, Mat<float, false>{sP, LDC}, C, 8 * rg, cg);
+    wmm<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
+    wmm<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
+    each(acc, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, -x * __bfloat162float(sK[t * LDB + i])); });
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int j = 0; j < KC::NT; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        dkT[i][j] += acc[i][j];
-        dgp[j] = fmaf(-acc[i][j], __bfloat162float(sK[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
-      }
+      for (int e = 0; e < 4; ++e) dkT[j][e] += acc[j][e];
   }
   // ---- dq = scale Diag(e) dO S0^T + N2 K
-  float dqT[8][4];
+  float dqT[KC::NT][4];
   zero(dqT);
-  mm<8, 4, false>(dqT, Mat<float, false, true>{S0, DV}, Mat<__nv_bfloat16, true>{sO, LDBV}, DV, 8 * rg, cg);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float f = p.scale * see[cg + 16 * j];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dqT[i][j] *= f;
-  }
-  mm<8, 4, false>(dqT, Mat<__nv_bfloat16, true>{sK, LDB}, Mat<float, true>{sP, LDC}, C, 8 * rg, cg);
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      dgp[j] = fmaf(dqT[i][j], __bfloat162float(sQ[(cg + 16 * j) * LDB + 8 * rg + i]), dgp[j]);
+  wmm<KC::NT, false>(dqT, FG{S0, DV}, BKT{sO, LDBV}, DV, mt, nt, lane);
+  each(dqT, mt, nt, lane, [&](int, int t, float &x) { x *= p.scale * see[t]; });
+  wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
+  each(dqT, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, x * __bfloat162float(sQ[t * LDB + i])); });
 
-  // ---- reductions: dg_t over the row groups; sum(X1 o K); sum(dS o S0)
+  // ---- reductions: dg_t over the rows; sum(X1 o K); sum(dS o S0)
   {
     float ss = 0.f;
     const float4 *a = reinterpret_cast<const float4 *>(dS), *bb = reinterpret_cast<const float4 *>(S0);
@@ -739,36 +719,30 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
       atomicAdd(&sred[1], ss);
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float x = dgp[j] + __shfl_xor_sync(0xffffffffu, dgp[j], 16);
-      if (lane < 16) atomicAdd(&sdg[cg + 16 * j], x);
-    }
+    for (int j = 0; j < KC::NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float s2 = column_sum(dgp[j][e]);
+        if (lane < 4) atomicAdd(&sdg[nt + 8 * j + 2 * lane + e], s2);
+      }
   }
   __syncthreads();
 
-  // ---- KLA: beta = eta / (||k||^2 + eps) adds -2 dbeta beta / (||k||^2 + eps) k to dk
-  if (p.kla) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int t = cg + 16 * j;
-      const float w = -2.f * sdb[t] * sbeta[t] / (snk[t] + p.eps);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) dkT[i][j] = fmaf(w, __bfloat162float(sK[t * LDB + 8 * rg + i]), dkT[i][j]);
-    }
-  }
-  // ---- dq, dk: eight consecutive d_k values per (thread, token)
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int t = cg + 16 * j;
+  // ---- KLA: beta = eta / (||k||^2 + eps) adds -2 dbeta beta / (||k||^2 + eps) k to dk;
+  // then dk and dq through bf16 tiles (over W and E, both dead) for row-contiguous stores
+  __nv_bfloat16 *stk = reinterpret_cast<__nv_bfloat16 *>(sE);
+  __nv_bfloat16 *stq = reinterpret_cast<__nv_bfloat16 *>(sW);
+  each(dkT, mt, nt, lane, [&](int i, int t, float &x) {
+    if (p.kla) x = fmaf(-2.f * sdb[t] * sbeta[t] / (snk[t] + p.eps), __bfloat162float(sK[t * LDB + i]), x);
+    stk[t * LDB + i] = __float2bfloat16_rn(x);
+  });
+  each(dqT, mt, nt, lane, [&](int i, int t, float &x) { stq[t * LDB + i] = __float2bfloat16_rn(x); });
+  __syncthreads();
+  for (int i = tid; i < C * DK / 8; i += NT) {
+    const int t = i / (DK / 8), j = i % (DK / 8);
     if (t < n) {
-      float xk[8], xq[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        xk[i] = dkT[i][j];
-        xq[i] = dqT[i][j];
-      }
-      st_chunk_bf16(reinterpret_cast<uint8_t *>(p.dk + row(t) * DK + 8 * rg), xk);
-      st_chunk_bf16(reinterpret_cast<uint8_t *>(p.dq + row(t) * DK + 8 * rg), xq);
+      reinterpret_cast<uint4 *>(p.dk + row(t) * DK)[j] = *reinterpret_cast<const uint4 *>(stk + t * LDB + 8 * j);
+      reinterpret_cast<uint4 *>(p.dq + row(t) * DK)[j] = *reinterpret_cast<const uint4 *>(stq + t * LDB + 8 * j);
     }
   }
   // ---- dbeta (d eta for KLA) and dlog_g = suffix sums of dg over the chunk's tokens
