@@ -66,7 +66,7 @@ METRIC = "gated-delta-rule layer tokens/s (fwd, decode) at 1 B200; % of bf16 TC 
 _CSRC = "gated_delta_rule_forward_b200/csrc/"
 _TC = [_CSRC + f for f in ("chunk_common.cuh", "tc_util.cuh", "tma_host.cuh")]
 KERNEL_SOURCES = {   # sources whose text keys a recorded ncu traffic figure
-    "chunk64_split": [_CSRC + "chunk_split.cu", _CSRC + "chunk_split.cuh"] + _TC,
+    "chunk64_split": [_CSRC + "chunk_split.cu", _CSRC + "chunk_split.cuh", _CSRC + "chunk_record.cuh"] + _TC,
     "token_bf16io": [_CSRC + "token_fwd.cu"],
     "token_f32io": [_CSRC + "token_fwd.cu"],
     "decode": [_CSRC + "decode.cu"],
@@ -546,6 +546,18 @@ def cpu_baseline(name):
         dt = time.perf_counter() - t0
         return {"value": passes * B / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
                 "sample": f"{passes} decode step(s) of all {B} sequences x {H} heads, fp64, {dt:.2f} s wall"}
+    if name in BWD_WORKLOADS:   # backward: one sequence's gradients per pass
+        from gated_delta_rule_forward_b200.inputs import random_output_grad
+        d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+        dO = random_output_grad(1, T, H, dv, 1)
+        passes, t0 = 0, time.perf_counter()
+        while passes == 0 or time.perf_counter() - t0 < 2.0:
+            oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"], scale=dk ** -0.5)
+            passes += 1
+        dt = time.perf_counter() - t0
+        return {"value": passes * T / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                "sample": f"{passes} backward pass(es) of 1 of {B} sequences x {T} tokens x {H} heads, fp64, "
+                          f"{dt:.2f} s wall"}
     Ts = min(T, ORACLE_SAMPLE_TOKENS)
     d = make_inputs(variant, B, Ts, H, dk, dv, dtype=torch.bfloat16, seed=0)
     oracle.forward(variant, **{k: (None if v is None else v[:, :64]) for k, v in d.items()})  # build/load
@@ -570,7 +582,9 @@ def native(args):
     sampler = ClockSampler(local)
     sampler.start()
     t0 = time.time()
-    if WORKLOADS[args.workload][2] is None:
+    if args.workload in BWD_WORKLOADS:
+        main = run_backward_workload(args.workload, args.steps, args.warmup, world, seed=rank)
+    elif WORKLOADS[args.workload][2] is None:
         main = run_decode_workload(args.workload, args.steps, args.warmup, world, e2e=not args.no_e2e,
                                    chain=False, seed=rank)
     else:
@@ -640,6 +654,14 @@ def reference(args):
         run = lambda: oracle.decode_step(variant, d["q"], d["k"], d["v"], S, **gates(d))
         tokens = B
         sample = f"one decode step of all {B} sequences x {H} heads per step, fp64"
+    elif args.workload in BWD_WORKLOADS:   # backward: one of the B sequences' gradients per step
+        from gated_delta_rule_forward_b200.inputs import random_output_grad
+        d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
+        dO = random_output_grad(1, T, H, dv, 1)
+        run = lambda: oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"],
+                                      scale=dk ** -0.5)
+        tokens = T
+        sample = f"the backward of 1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
     else:           # forward: one of the B sequences per step (its first tokens if it is long)
         Ts = min(T, ORACLE_SAMPLE_TOKENS)
         d = make_inputs(variant, 1, Ts, H, dk, dv, dtype=torch.bfloat16, seed=0)
@@ -674,7 +696,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT, choices=[w for w in WORKLOADS if w not in BWD_WORKLOADS])
+    ap.add_argument("--workload", default=DEFAULT, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-also", action="store_true", help="only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
