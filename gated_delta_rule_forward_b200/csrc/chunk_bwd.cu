@@ -59,8 +59,8 @@ constexpr float LOG2E_BWD = 1.4426950408889634f;
 // ---------------------------------------------------------------- warp-tile products
 // The products run on the tensor cores through the warp-level tf32 MMA
 // (m16n8k8, fp32 accumulation): a CTA's eight warps tile an M x N product
-// (M, N in {64, 128}) into 16-row tiles, each warp covering 16 rows and N * RT
-// / 64 columns, RT = M / 16 row tiles.  Operands come from shared or global
+// (M, N in {64, 128}) into 16-row tiles, each of W warps covering 16 rows and
+// N * RT / (8 W) columns, RT = M / 16 row tiles.  Operands come from shared or global
 // memory through views that may transpose them, so every product of the
 // chunk algebra is written as it reads.
 //
@@ -88,12 +88,14 @@ template <typename V>
 __device__ __forceinline__ float at(const V &m, int r, int c) {
   return ld1<typename V::elem, V::kGlobal>(m.p + (V::kTr ? c * m.ld + r : r * m.ld + c));
 }
-// The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N product.
-template <int M, int N>
+// The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N
+// product shared by W warps.
+template <int M, int N, int W = 8>
 struct Tiling {
   static constexpr int RT = M / 16;          // row tiles
-  static constexpr int CH = 8 / RT;          // column parts
+  static constexpr int CH = W / RT;          // column parts
   static constexpr int NT = N / 8 / CH;      // 8-column MMA tiles per warp
+  static_assert(CH >= 1 && NT >= 1, "tiling");
   static __device__ __forceinline__ int m0(int w) { return 16 * (w % RT); }
   static __device__ __forceinline__ int n0(int w) { return (w / RT) * (N / CH); }
 };
@@ -118,7 +120,7 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b,
   constexpr bool a_exact = !PRECISE || std::is_same<typename MA::elem, __nv_bfloat16>::value;
   const bool b_exact = !PRECISE || (std::is_same<typename MB::elem, __nv_bfloat16>::value && ks == nullptr);
   const int g = lane >> 2, t = lane & 3;
-#pragma unroll 1
+#pragma unroll 2
   for (int k0 = 0; k0 < K; k0 += 8) {
     uint32_t ah[4], al[4];
     split(a, m0 + g, k0 + t, 1.f, ah[0], al[0]);
@@ -145,7 +147,9 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b,
   }
 }
 
-// f(row, col, value) for each accumulator element of a warp tile.
+// f(row, col, value) for each accumulator element of a warp tile; each_je
+// also passes the fragment indices (j, e), compile-time constants after
+// unrolling, for per-column register arrays.
 template <int NT, typename F>
 __device__ __forceinline__ void each(float (&acc)[NT][4], int m0, int n0, int lane, F f) {
   const int g = lane >> 2, t = lane & 3;
@@ -153,6 +157,14 @@ __device__ __forceinline__ void each(float (&acc)[NT][4], int m0, int n0, int la
   for (int j = 0; j < NT; ++j)
 #pragma unroll
     for (int e = 0; e < 4; ++e) f(m0 + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[j][e]);
+}
+template <int NT, typename F>
+__device__ __forceinline__ void each_je(float (&acc)[NT][4], int m0, int n0, int lane, F f) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f(j, e, m0 + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[j][e]);
 }
 
 template <int NT>
@@ -304,31 +316,43 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
 
   const int warp = tid >> 5, lane = tid & 31;
   float vmax = 0.f;
-  {   // R^T [v][t] into the U' slot (rows v, 128-byte swizzled)
+  // Both products are staged in shared memory as the record's byte images and
+  // written with 16-byte stores: R^T over P's tile once R is done, F^T over
+  // dO's tile once F is done.
+  uint8_t *stage_r = reinterpret_cast<uint8_t *>(sP);
+  __half *stage_f = reinterpret_cast<__half *>(sO);
+  {   // R^T [v][t]: the U' slot's rows v, 128-byte swizzled
     using TL = Tiling<DV, C>;
     float acc[TL::NT][4];
     zero(acc);
     const int m0 = TL::m0(warp), n0 = TL::n0(warp);
     wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
                                                                    Mat<float, false>{sP, LDP}, C, m0, n0, lane);
+    __syncthreads();   // every warp has read P
     each(acc, m0, n0, lane, [&](int v, int t, float &x) {
       vmax = fmaxf(vmax, fabsf(x));
-      *reinterpret_cast<__half *>(dst + REC_U + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(x);
+      *reinterpret_cast<__half *>(stage_r + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(x);
     });
   }
-  {   // F^T [v][i] after the output term, unswizzled rows of d_k values
+  {   // F^T [v][i]: unswizzled rows of d_k values after the output term
     using TL = Tiling<DV, DK>;
     float acc[TL::NT][4];
     zero(acc);
     const int m0 = TL::m0(warp), n0 = TL::n0(warp);
     wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
                                                                    Mat<float, false>{sQ, LDQ}, C, m0, n0, lane);
-    __half *f = reinterpret_cast<__half *>(dst + rec_bytes_chan(NS) + 8192 * NS);
+    __syncthreads();   // every warp has read dO
     each(acc, m0, n0, lane, [&](int v, int i, float &x) {
       vmax = fmaxf(vmax, fabsf(x));
-      f[v * DK + i] = __float2half_rn(x);
+      stage_f[v * DK + i] = __float2half_rn(x);
     });
   }
+  __syncthreads();
+  for (int i = tid; i < DV * 128 / 16; i += NT)
+    *reinterpret_cast<uint4 *>(dst + REC_U + 16 * i) = *reinterpret_cast<const uint4 *>(stage_r + 16 * i);
+  for (int i = tid; i < DV * DK * 2 / 16; i += NT)
+    *reinterpret_cast<uint4 *>(dst + rec_bytes_chan(NS) + 8192 * NS + 16 * i) =
+        *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(stage_f) + 16 * i);
   if (vmax > F16_SAFE_BWD) atomicOr(&g_gdr_bwd_error, 2);
 }
 
@@ -366,9 +390,12 @@ struct LocalSmem {
   static constexpr size_t BYTES = SC + (9 * C + 4) * 4;
 };
 
-// One CTA per chunk (b, h, c).
+// One CTA of NTL threads per chunk (b, h, c): sixteen warps share each
+// product, so that the chunk's chain of small dependent products runs with
+// twice the warps in flight of an eight-warp CTA (one CTA fits an SM).
+constexpr int NTL = 512;
 template <int DV>
-__global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
+__global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) {
   using L = LocalSmem<DV>;
   constexpr int LDB = L::LDB, LDBV = L::LDBV, LDF = L::LDF, LDW = L::LDW, LDC = L::LDC;
   constexpr int NRV = DV / 16, NRK = DK / 16;
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
 
   // ---- inputs: bf16 tiles (zero past T)
-  for (int i = tid; i < C * DK / 8; i += NT) {
+  for (int i = tid; i < C * DK / 8; i += NTL) {
     const int t = i / (DK / 8), j = i % (DK / 8);
     uint4 uq = make_uint4(0u, 0u, 0u, 0u), uk = uq;
     if (t < n) {
@@ -416,7 +443,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
     *reinterpret_cast<uint4 *>(sQ + t * LDB + 8 * j) = uq;
     *reinterpret_cast<uint4 *>(sK + t * LDB + 8 * j) = uk;
   }
-  for (int i = tid; i < C * DV / 8; i += NT) {
+  for (int i = tid; i < C * DV / 8; i += NTL) {
     const int t = i / (DV / 8), j = i % (DV / 8);
     uint4 uv = make_uint4(0u, 0u, 0u, 0u), uo = uv;
     if (t < n) {
@@ -472,10 +499,11 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   }
   __syncthreads();
 
-  using CC = Tiling<C, C>;     // C x C products
-  using CV = Tiling<C, DV>;    // C x d_v
-  using CK = Tiling<C, DK>;    // C x d_k
-  using KC = Tiling<DK, C>;    // d_k x C (the transposed gradient tiles)
+  constexpr int LW = NTL / 32;
+  using CC = Tiling<C, C, LW>;     // C x C products
+  using CV = Tiling<C, DV, LW>;    // C x d_v
+  using CK = Tiling<C, DK, LW>;    // C x d_k
+  using KC = Tiling<DK, C, LW>;    // d_k x C (the transposed gradient tiles)
   const int mc = CC::m0(warp), nc = CC::n0(warp);
   const int mv = CV::m0(warp), nv = CV::n0(warp);
   const int mk = CK::m0(warp), nk = CK::n0(warp);
@@ -497,7 +525,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   }
   __syncthreads();
   solve_unit_lower_64(sA, sT, tid, warp, lane);   // ends with a barrier
-  for (int i = tid; i < C * C; i += NT) {
+  for (int i = tid; i < C * C; i += NTL) {
     const int m = i / C, j = i % C;
     if (j > m) sT[m * LD + j] = 0.f;
   }
@@ -545,15 +573,12 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   zero(dkT);
 #pragma unroll
   for (int j = 0; j < KC::NT; ++j) dgp[j][0] = dgp[j][1] = 0.f;
-  auto add_dg = [&](int col, float x) {   // col of the warp tile -> its dgp slot
-    dgp[(col - nt) >> 3][col & 1] += x;
-  };
   wmm<KC::NT, false>(dkT, FG{dS, DV}, FT{sE, LDF}, DV, mt, nt, lane);
-  each(dkT, mt, nt, lane, [&](int i, int t, float &x) {
+  each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
     x *= sff[t] * inv_s;
     const float y = x * __bfloat162float(sK[t * LDB + i]);
     x1k += y;
-    add_dg(t, -y);
+    dgp[j][e & 1] -= y;
   });
   // ---- dP = tril(dO E^T)
   {
@@ -577,8 +602,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
     zero(acc);
     wmm<CV::NT, false>(acc, FT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
     float part[2] = {0.f, 0.f};   // rows g and g + 8 of the tile
-    each(acc, mv, nv, lane, [&](int t, int v, float &x) {
-      part[(t - mv) >> 3] = fmaf(__bfloat162float(sV[t * LDBV + v]), x, part[(t - mv) >> 3]);
+    each_je(acc, mv, nv, lane, [&](int, int e, int t, int v, float &x) {
+      part[e >> 1] = fmaf(__bfloat162float(sV[t * LDBV + v]), x, part[e >> 1]);
       x *= sbeta[t];
     });
     const int g = lane >> 2, tq = lane & 3;
@@ -660,10 +685,10 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
     zero(g);
     wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
     float part[2] = {0.f, 0.f};
-    each(g, mc, nc, lane, [&](int t, int r, float &x) {
+    each_je(g, mc, nc, lane, [&](int, int e, int t, int r, float &x) {
       const float d = r <= t ? ex2(sG[t] - sG[r]) : 0.f;
       const float da = sA[t * LD + r];
-      part[(t - mc) >> 3] = fmaf(da * d, x, part[(t - mc) >> 3]);
+      part[e >> 1] = fmaf(da * d, x, part[e >> 1]);
       sA[t * LD + r] = sbeta[t] * da * d;
       sP[t * LDC + r] = p.scale * sP[t * LDC + r] * d;
     });
@@ -679,7 +704,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
     float acc[KC::NT][4];
     zero(acc);
     wmm<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
-    each(acc, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, x * __bfloat162float(sK[t * LDB + i])); });
+    each_je(acc, mt, nt, lane,
+            [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] += x * __bfloat162float(sK[t * LDB + i]); });
 #pragma unroll
     for (int j = 0; j < KC::NT; ++j)
 #pragma unroll
@@ -687,7 +713,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
     zero(acc);
     wmm<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
     wmm<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
-    each(acc, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, -x * __bfloat162float(sK[t * LDB + i])); });
+    each_je(acc, mt, nt, lane,
+            [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] -= x * __bfloat162float(sK[t * LDB + i]); });
 #pragma unroll
     for (int j = 0; j < KC::NT; ++j)
 #pragma unroll
@@ -699,13 +726,14 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   wmm<KC::NT, false>(dqT, FG{S0, DV}, BKT{sO, LDBV}, DV, mt, nt, lane);
   each(dqT, mt, nt, lane, [&](int, int t, float &x) { x *= p.scale * see[t]; });
   wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
-  each(dqT, mt, nt, lane, [&](int i, int t, float &x) { add_dg(t, x * __bfloat162float(sQ[t * LDB + i])); });
+  each_je(dqT, mt, nt, lane,
+          [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] += x * __bfloat162float(sQ[t * LDB + i]); });
 
   // ---- reductions: dg_t over the rows; sum(X1 o K); sum(dS o S0)
   {
     float ss = 0.f;
     const float4 *a = reinterpret_cast<const float4 *>(dS), *bb = reinterpret_cast<const float4 *>(S0);
-    for (int i = tid; i < DK * DV / 4; i += NT) {
+    for (int i = tid; i < DK * DV / 4; i += NTL) {
       const float4 x = __ldg(a + i), y = __ldg(bb + i);
       ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
     }
@@ -738,7 +766,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_local_kernel(const LocalParams p) {
   });
   each(dqT, mt, nt, lane, [&](int i, int t, float &x) { stq[t * LDB + i] = __float2bfloat16_rn(x); });
   __syncthreads();
-  for (int i = tid; i < C * DK / 8; i += NT) {
+  for (int i = tid; i < C * DK / 8; i += NTL) {
     const int t = i / (DK / 8), j = i % (DK / 8);
     if (t < n) {
       reinterpret_cast<uint4 *>(p.dk + row(t) * DK)[j] = *reinterpret_cast<const uint4 *>(stk + t * LDB + 8 * j);
@@ -861,7 +889,7 @@ cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const float *s0s, con
   auto run = [&](auto kern, size_t smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, NT, smem, s>>>(lp);
+    kern<<<grid, NTL, smem, s>>>(lp);
     return cudaGetLastError();
   };
   return f.dv == 128 ? run(bwd_local_kernel<128>, LocalSmem<128>::BYTES)

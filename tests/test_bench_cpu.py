@@ -51,3 +51,12 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0
+
+
+def test_reference_arm_times_the_oracle_backward():
+    """The backward workload's reference arm times the oracle's reverse mode on one sequence per step."""
+    r = _bench("--impl", "reference", "--workload", "gdn_bwd_350m", "--steps", "1", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"]["workload"] == "gdn_bwd_350m" and d["value"] > 0
+    assert "backward" in d["cpu_baseline"]["sample"]
