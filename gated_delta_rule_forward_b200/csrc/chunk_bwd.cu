@@ -65,12 +65,14 @@ constexpr float LOG2E_BWD = 1.4426950408889634f;
 // chunk algebra is written as it reads.
 //
 // A matrix operand: element (r, c) is p[r * ld + c], or p[c * ld + r] for TR.
-// GLOBAL operands are read through the read-only cache.
-template <typename E, bool TR, bool GLOBAL = false>
+// GLOBAL operands are read through the read-only cache; an EXACT fp32 operand
+// holds tf32 values already (the solve's T), so it needs no second tf32 part.
+template <typename E, bool TR, bool GLOBAL = false, bool EXACT = false>
 struct Mat {
   using elem = E;
   static constexpr bool kTr = TR;
   static constexpr bool kGlobal = GLOBAL;
+  static constexpr bool kExact = EXACT || std::is_same<E, __nv_bfloat16>::value;
   const E *p;
   int ld;
 };
@@ -111,14 +113,14 @@ struct Tiling {
 template <typename V>
 __device__ __forceinline__ void split(const V &m, int r, int c, float scale, uint32_t &hi, uint32_t &lo) {
   const float x = at(m, r, c) * scale;
-  hi = std::is_same<typename V::elem, __nv_bfloat16>::value && scale == 1.f ? __float_as_uint(x) : to_tf32(x);
+  hi = V::kExact && scale == 1.f ? __float_as_uint(x) : to_tf32(x);
   lo = to_tf32(x - __uint_as_float(hi));
 }
 template <int NT, bool NEG, typename MA, typename MB, bool PRECISE = true>
 __device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b, int K, int m0, int n0, int lane,
                                     const float *ks = nullptr) {
-  constexpr bool a_exact = !PRECISE || std::is_same<typename MA::elem, __nv_bfloat16>::value;
-  const bool b_exact = !PRECISE || (std::is_same<typename MB::elem, __nv_bfloat16>::value && ks == nullptr);
+  constexpr bool a_exact = !PRECISE || MA::kExact;
+  const bool b_exact = !PRECISE || (MB::kExact && ks == nullptr);
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll 2
   for (int k0 = 0; k0 < K; k0 += 8) {
@@ -513,6 +515,8 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   using F = Mat<float, false>;
   using FT = Mat<float, true>;
   using FG = Mat<float, false, true>;     // a global fp32 matrix (S0, dS)
+  using TX = Mat<float, false, false, true>;   // T (tf32 values from the solve)
+  using TXT = Mat<float, true, false, true>;   // ... transposed
 
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
@@ -534,11 +538,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // ---- U' = T Diag(beta) V and W = T Diag(beta e) K; E = U' - W S0
   float ue[CV::NT][4];
   zero(ue);
-  wmm<CV::NT, false>(ue, F{sT, LD}, BK{sV, LDBV}, C, mv, nv, lane, sbeta);
+  wmm<CV::NT, false>(ue, TX{sT, LD}, BK{sV, LDBV}, C, mv, nv, lane, sbeta);
   {
     float w[CK::NT][4];
     zero(w);
-    wmm<CK::NT, false>(w, F{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
+    wmm<CK::NT, false>(w, TX{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
     each(w, mk, nk, lane, [&](int t, int i, float &x) { sW[t * LDW + i] = x; });
   }
   __syncthreads();
@@ -600,7 +604,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[CV::NT][4];
     zero(acc);
-    wmm<CV::NT, false>(acc, FT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
+    wmm<CV::NT, false>(acc, TXT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
     float part[2] = {0.f, 0.f};   // rows g and g + 8 of the tile
     each_je(acc, mv, nv, lane, [&](int, int e, int t, int v, float &x) {
       part[e >> 1] = fmaf(__bfloat162float(sV[t * LDBV + v]), x, part[e >> 1]);
@@ -625,7 +629,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[KC::NT][4];
     zero(acc);
-    wmm<KC::NT, false>(acc, F{sW, LDC}, F{sT, LD}, C, mt, nt, lane);
+    wmm<KC::NT, false>(acc, F{sW, LDC}, TX{sT, LD}, C, mt, nt, lane);
     float dbp[KC::NT][2];
 #pragma unroll
     for (int j = 0; j < KC::NT; ++j) dbp[j][0] = dbp[j][1] = 0.f;
@@ -668,14 +672,14 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm<CC::NT, false>(acc, F{sA, LD}, FT{sT, LD}, C, mc, nc, lane);
+    wmm<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sE[t * LDC + r] = x; });
   }
   __syncthreads();
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm<CC::NT, true>(acc, FT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    wmm<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = r < t ? x : 0.f; });
   }
   __syncthreads();
