@@ -137,15 +137,24 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b,
       }
     }
     const float s0 = ks != nullptr ? ks[k0 + t] : 1.f, s1 = ks != nullptr ? ks[k0 + t + 4] : 1.f;
+    // all B fragments first, then the passes as three sweeps over the tiles, so
+    // that consecutive MMAs accumulate into different fragments
+    uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      uint32_t bh0, bl0, bh1, bl1;
-      split(b, k0 + t, n0 + 8 * j + g, s0, bh0, bl0);
-      split(b, k0 + t + 4, n0 + 8 * j + g, s1, bh1, bl1);
-      if (!b_exact) mma_tf32_16x8x8(acc[j], ah, bl0, bl1);
-      if (!a_exact) mma_tf32_16x8x8(acc[j], al, bh0, bh1);
-      mma_tf32_16x8x8(acc[j], ah, bh0, bh1);
+      split(b, k0 + t, n0 + 8 * j + g, s0, bh[j][0], bl[j][0]);
+      split(b, k0 + t + 4, n0 + 8 * j + g, s1, bh[j][1], bl[j][1]);
     }
+    if (!b_exact) {
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_tf32_16x8x8(acc[j], ah, bl[j][0], bl[j][1]);
+    }
+    if (!a_exact) {
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_tf32_16x8x8(acc[j], al, bh[j][0], bh[j][1]);
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) mma_tf32_16x8x8(acc[j], ah, bh[j][0], bh[j][1]);
   }
 }
 
