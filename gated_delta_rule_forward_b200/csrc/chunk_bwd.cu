@@ -387,18 +387,22 @@ struct LocalSmem {
   static constexpr int LDF = DV + 4;    // fp32 rows of dE, E
   static constexpr int LDW = DK + 4;    // fp32 rows of W
   static constexpr int LDC = C + 4;     // fp32 rows of C-wide tiles (dW^T, X, dP)
+  static constexpr int LDH = 66;        // fp32 rows of a 64-column half of S0 or dS
   static constexpr size_t K = 0;
   static constexpr size_t Q = K + C * LDB * 2;
   static constexpr size_t V = Q + C * LDB * 2;
   static constexpr size_t O = V + C * LDBV * 2;
-  static constexpr size_t DE = O + C * LDBV * 2;
-  static constexpr size_t E = DE + C * LDF * 4;
+  static constexpr size_t E = O + C * LDBV * 2;
   static constexpr size_t W = E + static_cast<size_t>(std::max(C * LDF, C * LDC)) * 4;
-  static constexpr size_t A = W + static_cast<size_t>(std::max(C * LDW, DK * LDC)) * 4;
-  static constexpr size_t TT = A + C * LD * 4;
-  static constexpr size_t P = TT + C * LD * 4;
+  static constexpr size_t TT = W + static_cast<size_t>(std::max(C * LDW, DK * LDC)) * 4;
+  static constexpr size_t DE = TT + C * LD * 4;   // DE, A and P are contiguous: S0's staging before dE and P exist
+  static constexpr size_t A = DE + C * LDF * 4;
+  static constexpr size_t P = A + C * LD * 4;
   static constexpr size_t SC = P + C * LDC * 4;
   static constexpr size_t BYTES = SC + (9 * C + 4) * 4;
+  static_assert(A + C * LD * 4 + C * LDC * 4 - DE >= static_cast<size_t>(DK) * LDF * 4, "S0 staging over dE, A, P");
+  static_assert(std::max(C * LDW, DK * LDC) >= DK * LDH, "a half of dS over W");
+  static constexpr bool kS0HalvesOverE = std::max(C * LDF, C * LDC) >= DK * LDH;   // d_v = 128
 };
 
 // One CTA of NTL threads per chunk (b, h, c): sixteen warps share each
@@ -554,9 +558,21 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     wmm<CK::NT, false>(w, TX{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
     each(w, mk, nk, lane, [&](int t, int i, float &x) { sW[t * LDW + i] = x; });
   }
+  // S0 through shared memory (over dE, A and P, none of which holds data yet):
+  // E = U' - W S0 and dq's first part, scale Diag(e) dO S0^T
+  float *sS = reinterpret_cast<float *>(sm + L::DE);
+  for (int i = tid; i < DK * DV / 4; i += NTL) {
+    const int r = i / (DV / 4), c4 = i % (DV / 4);
+    *reinterpret_cast<float4 *>(sS + r * LDF + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(S0) + i);
+  }
   __syncthreads();
-  wmm<CV::NT, true>(ue, F{sW, LDW}, FG{S0, DV}, DK, mv, nv, lane);
+  wmm<CV::NT, true>(ue, F{sW, LDW}, F{sS, LDF}, DK, mv, nv, lane);
   each(ue, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
+  float dqT[KC::NT][4];
+  zero(dqT);
+  wmm<KC::NT, false>(dqT, F{sS, LDF}, BKT{sO, LDBV}, DV, mt, nt, lane);
+  each(dqT, mt, nt, lane, [&](int, int t, float &x) { x *= p.scale * see[t]; });
+  __syncthreads();   // S0's staging is read: P may overwrite it
   // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
   // reverse carry's own dE is Diag(beta) dE (its records carry beta in P and Kt), so it is
   // recomputed here rather than divided by beta.
@@ -569,24 +585,36 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     });
   }
   __syncthreads();
-  {
-    float acc[CV::NT][4];
-    zero(acc);
-    wmm<CV::NT, false>(acc, BK{sK, LDB}, FG{dS, DV}, DK, mv, nv, lane);
-    each(acc, mv, nv, lane, [&](int t, int, float &x) { x *= sff[t] * inv_s; });
-    wmm<CV::NT, false>(acc, FT{sP, LDC}, BK{sO, LDBV}, C, mv, nv, lane);
-    each(acc, mv, nv, lane, [&](int t, int v, float &x) { sdE[t * LDF + v] = x; });
-  }
-  __syncthreads();
-
-  // ---- dk^T (d_k x C tiles) starts as (Diag(f) E dS^T)^T / s
+  // ---- with dS through shared memory in 64-column halves (over W, which E has
+  // finished reading): dE's columns of the half, and dk^T's first part
+  // (Diag(f) E dS^T)^T / s accumulated over the halves
   float dkT[KC::NT][4];
   float dgp[KC::NT][2];   // this thread's column sums toward dg_t (columns n0 + 8 j + 2 t + e)
   float x1k = 0.f;
   zero(dkT);
 #pragma unroll
   for (int j = 0; j < KC::NT; ++j) dgp[j][0] = dgp[j][1] = 0.f;
-  wmm<KC::NT, false>(dkT, FG{dS, DV}, FT{sE, LDF}, DV, mt, nt, lane);
+  {
+    using CH = Tiling<C, 64, LW>;
+    const int mh = CH::m0(warp), nh = CH::n0(warp);
+    float *sH = reinterpret_cast<float *>(sm + L::W);
+    for (int h = 0; h < DV / 64; ++h) {
+      for (int i = tid; i < DK * 32; i += NTL) {   // float2 pairs of the half
+        const int r = i >> 5, c2 = i & 31;
+        *reinterpret_cast<float2 *>(sH + r * L::LDH + 2 * c2) =
+            __ldg(reinterpret_cast<const float2 *>(dS + r * DV + 64 * h) + c2);
+      }
+      __syncthreads();
+      float acc[CH::NT][4];
+      zero(acc);
+      wmm<CH::NT, false>(acc, BK{sK, LDB}, F{sH, L::LDH}, DK, mh, nh, lane);
+      each(acc, mh, nh, lane, [&](int t, int, float &x) { x *= sff[t] * inv_s; });
+      wmm<CH::NT, false>(acc, FT{sP, LDC}, BK{sO + 64 * h, LDBV}, C, mh, nh, lane);
+      each(acc, mh, nh, lane, [&](int t, int v, float &x) { sdE[t * LDF + 64 * h + v] = x; });
+      wmm<KC::NT, false>(dkT, F{sH, L::LDH}, FT{sE + 64 * h, LDF}, 64, mt, nt, lane);
+      __syncthreads();   // the half is read before the next one lands
+    }
+  }
   each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
     x *= sff[t] * inv_s;
     const float y = x * __bfloat162float(sK[t * LDB + i]);
@@ -600,11 +628,27 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     wmm<CC::NT, false>(acc, BK{sO, LDBV}, FT{sE, LDF}, DV, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sP[t * LDC + r] = r <= t ? x : 0.f; });
   }
-  // ---- dW^T = -S0 dE^T  (d_k x C, over W, which E = U' - W S0 has finished reading)
+  // ---- dW^T = -S0 dE^T  (d_k x C, over W); at d_v = 128 with S0 through shared
+  // memory in halves, over E once dP has read it
   {
     float acc[KC::NT][4];
     zero(acc);
-    wmm<KC::NT, true>(acc, FG{S0, DV}, FT{sdE, LDF}, DV, mt, nt, lane);
+    if constexpr (L::kS0HalvesOverE) {
+      __syncthreads();   // dP has read E
+      float *sH = reinterpret_cast<float *>(sm + L::E);
+      for (int h = 0; h < DV / 64; ++h) {
+        for (int i = tid; i < DK * 32; i += NTL) {
+          const int r = i >> 5, c2 = i & 31;
+          *reinterpret_cast<float2 *>(sH + r * L::LDH + 2 * c2) =
+              __ldg(reinterpret_cast<const float2 *>(S0 + r * DV + 64 * h) + c2);
+        }
+        __syncthreads();
+        wmm<KC::NT, true>(acc, F{sH, L::LDH}, FT{sdE + 64 * h, LDF}, 64, mt, nt, lane);
+        __syncthreads();
+      }
+    } else {
+      wmm<KC::NT, true>(acc, FG{S0, DV}, FT{sdE, LDF}, DV, mt, nt, lane);
+    }
     each(acc, mt, nt, lane, [&](int i, int t, float &x) { sW[i * LDC + t] = x; });
   }
   __syncthreads();
@@ -733,11 +777,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
 #pragma unroll
       for (int e = 0; e < 4; ++e) dkT[j][e] += acc[j][e];
   }
-  // ---- dq = scale Diag(e) dO S0^T + N2 K
-  float dqT[KC::NT][4];
-  zero(dqT);
-  wmm<KC::NT, false>(dqT, FG{S0, DV}, BKT{sO, LDBV}, DV, mt, nt, lane);
-  each(dqT, mt, nt, lane, [&](int, int t, float &x) { x *= p.scale * see[t]; });
+  // ---- dq += N2 K
   wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
   each_je(dqT, mt, nt, lane,
           [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] += x * __bfloat162float(sQ[t * LDB + i]); });
