@@ -128,3 +128,23 @@ def test_backward_rejects_uncovered_cases():
     with pytest.raises(gdr.GdrError) as e:
         gdr.backward(d["q"], d["k"], d["v"], dO, variant="kda", beta=d["beta"], log_g=d["log_g"])
     assert e.value.status == 2   # GDR_ERR_UNSUPPORTED
+
+
+def test_backward_long_context_sampled():
+    """The 65536-token sequence (B=1, H=16): 1024 chunks through both carries,
+    checked against the oracle on two of its heads."""
+    B, T, H = 1, 65536, 16
+    scale = 128 ** -0.5
+    d = make_inputs("gdn", B, T, H, dtype=torch.bfloat16, seed=28)
+    dO = random_output_grad(B, T, H, 128, 29)
+    dd = to_dev(d)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant="gdn", beta=dd["beta"], log_g=dd["log_g"],
+                     scale=scale)
+    gdr.device_status()
+    for h in (0, H - 1):
+        s = select(d, h=slice(h, h + 1))
+        ref = oracle.backward("gdn", s["q"], s["k"], s["v"], dO[:, :, h:h + 1], beta=s["beta"], log_g=s["log_g"],
+                              scale=scale)
+        gh = {k: (None if x is None else (x[:, h:h + 1] if k == "initial_state" else x[:, :, h:h + 1]))
+              for k, x in g.items()}
+        check_grads(gh, ref, "gdn", f"head {h}")
