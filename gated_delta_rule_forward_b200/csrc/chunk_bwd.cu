@@ -43,6 +43,7 @@
 #include "chunk_bwd.cuh"
 #include "chunk_common.cuh"
 #include "chunk_record.cuh"
+#include "chunk_split.cuh"
 
 // Device-side error word of this file (bit 1: a reverse-record operand beyond
 // the fp16 range).
@@ -866,7 +867,9 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
   L.dss = L.s0s + up(bh * NC * DK * dv * 4);
   L.x0 = L.dss + up(bh * NC * DK * dv * 4);
   L.xf = L.x0 + up(bh * DK * dv * 4);
-  L.absmax = L.xf + up(bh * DK * dv * 4);
+  L.maps = L.xf + up(bh * DK * dv * 4);
+  L.maps_bytes = gdr_split_segment_bytes(B, T, H, dv);
+  L.absmax = L.maps + up(L.maps_bytes);
   L.total = L.absmax + 256;
   return L;
 }

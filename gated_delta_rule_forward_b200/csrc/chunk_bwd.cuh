@@ -26,6 +26,7 @@ struct BwdLayout {
   size_t s0s;       // fp32 start state of every chunk        [B,H,NC,dk,dv]
   size_t dss;       // fp32 end-state gradient, reverse order [B,H,NC,dk,dv]
   size_t x0, xf;    // reverse carry's start (scaled d_final) and end (scaled d_s0) [B,H,dk,dv]
+  size_t maps, maps_bytes;   // the segmented carries' maps and start states (0 bytes: unsegmented)
   size_t absmax;    // the gradients' magnitude (one fp32 word)
   size_t total;
 };

@@ -2151,6 +2151,45 @@ cudaError_t launch_pipelined(const FwdProblem &p, int NC, uint8_t *w, const Pipe
   return launch_carry<MODE>(p, NC, w, l2, true, stream, err);
 }
 
+// The carry over segments (few long sequences, sp.G > 1) on the records at
+// `records`, with the segment maps, offsets and start states at `maps`
+// (seg_extra_floats floats): phase 1, the chain of start states, then phase 2,
+// every segment from its start state with flags2 added (the forward: none, so
+// with outputs; the backward's carries: no outputs, chunk states kept).
+template <int MODE>
+cudaError_t launch_segmented(const FwdProblem &p, int NC, const SegPlan &sp, const uint8_t *records, uint8_t *maps,
+                             const float *s0, float *s_final, int flags2, float *states, cudaStream_t stream,
+                             std::string *err) {
+  const size_t bh = static_cast<size_t>(p.B) * p.H;
+  float *Mb = reinterpret_cast<float *>(maps);
+  float *Db = Mb + (sp.G - 2) * bh * DK * DK;
+  float *Ss = Db + (sp.G - 1) * bh * DK * p.dv;
+  CarryLaunch m;   // phase 1, pass A: end states of segments 0 .. G-2 (segment 0 from s0, the rest from zero)
+  m.segments = sp.G - 1; m.seg_len = sp.L;
+  m.flags = CARRY_NO_OUTPUT | CARRY_S0_FIRST;
+  m.s0 = s0;
+  m.s_final = Db; m.s_final_stride = bh * DK * p.dv;
+  // pass B: transition maps of segments 1 .. G-2
+  m.segments_b = sp.G - 2; m.seg_first_b = 1;
+  m.flags_b = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
+  m.s_final_b = Mb; m.s_final_b_stride = bh * DK * DK;
+  cudaError_t e = launch_carry<MODE>(p, NC, records, m, true, stream, err);
+  if (e != cudaSuccess) return e;
+  segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(s0, Mb, Db, Ss, sp.G, p.H, p.dv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *err = "segment chain launch: ";
+    return e;
+  }
+  CarryLaunch f;   // phase 2: every segment from its start
+  f.segments = sp.G; f.seg_len = sp.L;
+  f.flags = CARRY_LAST_FINAL | flags2;
+  f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
+  f.s_final = s_final;
+  f.states = states;
+  return launch_carry<MODE>(p, NC, records, f, true, stream, err);
+}
+
 // `ws_bytes` is the workspace the call may use: a segmented plan whose maps do
 // not fit beside the records falls back to the unsegmented sweep.
 template <int VAR>
@@ -2176,32 +2215,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, size_t ws_bytes, cudaStr
   const size_t bh = static_cast<size_t>(p.B) * p.H, ns = p.dv / 64;
   const size_t rec = MODE == 2 ? rec_bytes_gdn2(ns) : MODE == 1 ? rec_bytes_chan(ns) : rec_bytes(ns);
   const size_t rec_total = (bh * NC * rec + 255) / 256 * 256;
-  float *Mb = reinterpret_cast<float *>(w + rec_total);
-  float *Db = Mb + (sp.G - 2) * bh * DK * DK;
-  float *Ss = Db + (sp.G - 1) * bh * DK * p.dv;
-  CarryLaunch m;   // phase 1, pass A: end states of segments 0 .. G-2 (segment 0 from s0, the rest from zero)
-  m.segments = sp.G - 1; m.seg_len = sp.L;
-  m.flags = CARRY_NO_OUTPUT | CARRY_S0_FIRST;
-  m.s0 = p.s0;
-  m.s_final = Db; m.s_final_stride = bh * DK * p.dv;
-  // pass B: transition maps of segments 1 .. G-2
-  m.segments_b = sp.G - 2; m.seg_first_b = 1;
-  m.flags_b = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
-  m.s_final_b = Mb; m.s_final_b_stride = bh * DK * DK;
-  e = launch_carry<MODE>(p, NC, w, m, true, stream, err);
-  if (e != cudaSuccess) return e;
-  segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(p.s0, Mb, Db, Ss, sp.G, p.H, p.dv);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    *err = "segment chain launch: ";
-    return e;
-  }
-  CarryLaunch f;   // phase 2: every segment from its start, with outputs
-  f.segments = sp.G; f.seg_len = sp.L;
-  f.flags = CARRY_LAST_FINAL;
-  f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
-  f.s_final = p.s_final;
-  return launch_carry<MODE>(p, NC, w, f, true, stream, err);
+  return launch_segmented<MODE>(p, NC, sp, w, w + rec_total, p.s0, p.s_final, 0, nullptr, stream, err);
 }
 
 // The backward's steps on the stream (each the programmatic dependent of the
@@ -2209,7 +2223,8 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, size_t ws_bytes, cudaStr
 // that keeps every chunk's start state (no outputs); the gradient scale and
 // the reverse records; the reverse carry (third carry mode, over the reverse
 // records) keeping every chunk's end-state gradient; the chunk-local
-// gradients; the initial state's gradient.  Both carries run unsegmented.
+// gradients; the initial state's gradient.  Both carries run segmented where
+// the forward's would (few long sequences).
 template <int VAR>
 cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t stream, std::string *err) {
   constexpr int MODE = VAR == kKDA ? 1 : 0;
@@ -2219,14 +2234,21 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
   float *s0s = reinterpret_cast<float *>(w + L.s0s), *dss = reinterpret_cast<float *>(w + L.dss);
   float *x0 = reinterpret_cast<float *>(w + L.x0), *xf = reinterpret_cast<float *>(w + L.xf);
   uint32_t *absmax = reinterpret_cast<uint32_t *>(w + L.absmax);
+  const SegPlan sp = L.maps_bytes > 0 ? seg_plan(p.B, p.H, p.dv, NC) : SegPlan{1, NC};
   cudaError_t e = launch_prep_any<VAR>(p, NC, w + L.fwd_rec, PrepRange(), stream, err);
   if (e != cudaSuccess) return e;
-  CarryLaunch lf;
-  lf.seg_len = NC;
-  lf.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
-  lf.s0 = p.s0;
-  lf.states = s0s;
-  if ((e = launch_carry<MODE>(p, NC, w + L.fwd_rec, lf, true, stream, err)) != cudaSuccess) return e;
+  if (sp.G > 1) {
+    e = launch_segmented<MODE>(p, NC, sp, w + L.fwd_rec, w + L.maps, p.s0, nullptr,
+                               CARRY_NO_OUTPUT | CARRY_WRITE_STATES, s0s, stream, err);
+  } else {
+    CarryLaunch lf;
+    lf.seg_len = NC;
+    lf.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
+    lf.s0 = p.s0;
+    lf.states = s0s;
+    e = launch_carry<MODE>(p, NC, w + L.fwd_rec, lf, true, stream, err);
+  }
+  if (e != cudaSuccess) return e;
   if ((e = gdr_bwd_launch_scale(bp, absmax, x0, stream)) != cudaSuccess) {
     *err = "gradient scale: ";
     return e;
@@ -2235,13 +2257,19 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
     *err = "reverse records: ";
     return e;
   }
-  CarryLaunch lr;
-  lr.seg_len = NC;
-  lr.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
-  lr.s0 = x0;
-  lr.s_final = xf;
-  lr.states = dss;
-  if ((e = launch_carry<2>(p, NC, w + L.rev_rec, lr, true, stream, err)) != cudaSuccess) return e;
+  if (sp.G > 1) {
+    e = launch_segmented<2>(p, NC, sp, w + L.rev_rec, w + L.maps, x0, xf, CARRY_NO_OUTPUT | CARRY_WRITE_STATES,
+                            dss, stream, err);
+  } else {
+    CarryLaunch lr;
+    lr.seg_len = NC;
+    lr.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
+    lr.s0 = x0;
+    lr.s_final = xf;
+    lr.states = dss;
+    e = launch_carry<2>(p, NC, w + L.rev_rec, lr, true, stream, err);
+  }
+  if (e != cudaSuccess) return e;
   if ((e = gdr_bwd_launch_local(bp, s0s, dss, absmax, stream)) != cudaSuccess) {
     *err = "local gradients: ";
     return e;
@@ -2281,6 +2309,12 @@ size_t gdr_split_record_bytes(int variant, int dv) {
   return variant == gdr::kGDN2  ? gdr::tc::rec_bytes_gdn2(dv / 64)
          : variant == gdr::kKDA ? gdr::tc::rec_bytes_chan(dv / 64)
                                 : gdr::tc::rec_bytes(dv / 64);
+}
+
+size_t gdr_split_segment_bytes(int B, int T, int H, int dv) {
+  const int NC = (T + 63) / 64;
+  const gdr::tc::SegPlan sp = gdr::tc::seg_plan(B, H, dv, NC);
+  return sp.G == 1 ? 0 : 4 * gdr::tc::seg_extra_floats(B, H, dv, sp);
 }
 
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {

@@ -12,6 +12,8 @@ int gdr_read_device_error(cudaStream_t stream);
 bool gdr_split_supported(int variant, int dk, int dv);
 size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv);
 size_t gdr_split_record_bytes(int variant, int dv);   // bytes of one (b, h, chunk) record
+// Bytes of the segmented carry's maps, offsets and start states on the current device (0 when not segmented).
+size_t gdr_split_segment_bytes(int B, int T, int H, int dv);
 int gdr_split_launches(int variant, int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
 // The two-kernel path's schedule on a device with `sms` SMs (no device query).
 void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,

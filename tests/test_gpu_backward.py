@@ -148,3 +148,12 @@ def test_backward_long_context_sampled():
         gh = {k: (None if x is None else (x[:, h:h + 1] if k == "initial_state" else x[:, :, h:h + 1]))
               for k, x in g.items()}
         check_grads(gh, ref, "gdn", f"head {h}")
+
+
+@pytest.mark.parametrize("variant", ["gdn", "kla"])
+def test_backward_segmented(variant):
+    """Few long sequences (B*H = 2, 65 chunks): both carries run in segments (13
+    of 5 chunks) from an initial state and a final-state gradient."""
+    assert gdr.forward_plan(variant, 1, 4100, 2, 128, 148)["segments"] == 13
+    g, ref = run_backward(variant, 1, 4100, 2, seed=30)
+    check_grads(g, ref, variant)
