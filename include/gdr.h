@@ -231,7 +231,10 @@ typedef struct {
  * Bytes of device workspace gdr_backward needs (0 for a case it does not
  * cover): the forward's records, the reverse carry's records (B * H *
  * ceil(T/64) of each), every chunk's start state and end-state gradient
- * (fp32, dk * dv each), plus two states.
+ * (fp32, dk * dv each), plus two states; for few long sequences (where the
+ * forward's carry runs in segments) also the segment maps and start states
+ * its two carries share.  The segmenting reads the current device's SM
+ * count, so query the size on the device that runs the call.
  */
 size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, int dk, int dv);
 
@@ -249,7 +252,8 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * chunkwise solver of Gated DeltaNet with KLA's diagonal step).  It re-runs
  * the forward's chunk products and carry (keeping every chunk's start state),
  * runs the dS recurrence through the same carry kernel over the chunks in
- * reverse, then computes every chunk's q, k, v and gate gradients in
+ * reverse (both carries in segments for few long sequences, as the
+ * forward's), then computes every chunk's q, k, v and gate gradients in
  * parallel.  KLA's d eta includes the path through its Kaczmarz step
  * eta / (||k||^2 + eps).  d_o [B,T,H,dv] in the I/O dtype (required);
  * d_final_state [B,H,dk,dv] fp32 or NULL (zero).  The tensor-core carries use
