@@ -1346,7 +1346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // quarter w / 4 of its d_k range (fp32 registers), of E^T's tokens and of the
 // output tokens.  The two sides hand over through mbarriers only:
 //     issuer:  Y(c) = S^T [-W; Qg]^T -> bar_e      compute: E^T(c) -> bar_ea
-//              dS^T(c), Y_Q += E^T P^T -> bar_s/o           S^T(c) -> bar_sa
+//              dS^T(c), Y_Q += E^T P^T -> bar_s/o           S^T(c) -> bar_sa, bar_sa1
 //              record c+2 (after bar_done of c-1)           output rows (c) -> bar_done
 // Y is double-buffered so Y(c+1) runs while the output rows of c are written;
 // records arrive by bulk copy two chunks ahead of their use.
@@ -1457,11 +1457,12 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   uint64_t *bar_s = bar_e + 1;            // dS^T(c) done
   uint64_t *bar_o = bar_e + 2;            // E^T P^T (c) done
   uint64_t *bar_ea = bar_e + 3;           // E^T(c) in tensor memory (16 warps)
-  uint64_t *bar_sa = bar_e + 4;           // S^T in tensor memory (16 warps)
+  uint64_t *bar_sa = bar_e + 4;           // S^T (scalar decay), or its first half-rows, in tensor memory (16 warps)
   uint64_t *bar_done = bar_e + 5;         // chunk c's Y read and stage released (16 warps)
   uint64_t *bar_drain = bar_e + 6;        // error path only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_e + 7);
   volatile int *abort = reinterpret_cast<volatile int *>(bar_e + 8);
+  uint64_t *bar_sa1 = bar_e + 9;          // S^T's second half-rows in tensor memory (16 warps)
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -1474,6 +1475,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     mbar_init(bar_o, 1);
     mbar_init(bar_ea, NCOMPUTE);
     mbar_init(bar_sa, NCOMPUTE);
+    mbar_init(bar_sa1, NCOMPUTE);
     mbar_init(bar_done, NCOMPUTE);
     mbar_init(bar_drain, 1);
     *abort = 0;
@@ -1515,15 +1517,38 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         par ^= 1u << s;
         return true;
       };
-      auto issue_y = [&](int c) {   // Y(c) = S^T [-W; Qg]^T
-        tc_fence_after();
+      // Y(c) = S^T [-W; Qg]^T over d_k in 16-row steps.  With channel decay (a
+      // longer S update) the even steps (each compute warp's first 16 rows) go as
+      // soon as those are stored and the odd ones after the rest; with a scalar
+      // decay the state is handed off whole (the second hand-off costs more than
+      // it saves there).
+      auto issue_y = [&](int c) -> bool {
         const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
+        if constexpr (MODE == 0) {
+          if (!wait_or_abort(bar_sa, c & 1, abort)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
-                 sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idesc_f16(128, 128, false, false),
-                 kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
+                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   idesc_f16(128, 128, false, false), kk > 0);
+          mma_commit(bar_e);
+          return true;
+        }
+#pragma unroll
+        for (int odd = 0; odd < 2; ++odd) {
+          if (!wait_or_abort(odd ? bar_sa1 : bar_sa, c & 1, abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const int kk = 2 * k2 + odd;
+            mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
+                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   idesc_f16(128, 128, false, false), kk > 0);
+          }
+        }
         mma_commit(bar_e);
+        return true;
       };
       griddep_wait();   // the records are the preparation kernel's output
       // CARRY_FAULT_MISSING_COPY (host fault injection): CTA (0, 0, 0) never copies
@@ -1531,8 +1556,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       const bool inject = (flags & CARRY_FAULT_MISSING_COPY) && (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
       for (int c = 0; c < NSTAGE && c < NC; ++c)
         if (!(inject && c == 1)) issue_chunk(c);
-      bool ok = wait_or_abort(bar_sa, 0, abort) && wait_full(0);
-      if (ok) issue_y(0);
+      bool ok = wait_full(0) && issue_y(0);
       // Waits follow the order in which the compute warps arrive (done(c-1)
       // before E(c) before S(c)), so no barrier can complete a phase the
       // issuer has not waited for yet.
@@ -1557,8 +1581,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
                  idesc_f16(128, 64, false, false), 1);
         mma_commit(bar_o);
         if (c + 1 < NC) {
-          if (!(ok = wait_or_abort(bar_sa, (c + 1) & 1, abort) && wait_full(c + 1))) break;
-          issue_y(c + 1);
+          if (!(ok = wait_full(c + 1) && issue_y(c + 1))) break;
         }
       }
     }
@@ -1573,7 +1596,20 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
         S[k] = (flags & CARRY_IDENTITY) ? (32 * part + k == v ? 1.f : 0.f)
                : from_s0 ? __ldg(p.s0 + zi * p.s0_seg_stride + base + static_cast<size_t>(k) * p.dv) : 0.f;
     }
-    auto store_state = [&]() {
+    // S^T rows 32 part + 16 hv .. + 15 as fp16 pairs into columns 16 part + 8 hv ..
+    // (the Y product's K-step 2 part + hv), then that half's hand-off
+    auto store_half = [&](int hv) {
+      uint32_t r[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) r[m] = pack_f16x2(S[16 * hv + 2 * m], S[16 * hv + 2 * m + 1]);
+      tmem_st8(lrow + COL_SA + 16 * part + 8 * hv, r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(hv ? bar_sa1 : bar_sa);
+    };
+    // scalar decay: S^T's 32 rows in one store and one hand-off
+    auto store_whole = [&]() {
       uint32_t r[16];
 #pragma unroll
       for (int m = 0; m < 16; ++m) r[m] = pack_f16x2(S[2 * m], S[2 * m + 1]);
@@ -1583,7 +1619,12 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_sa);
     };
-    store_state();
+    if constexpr (MODE == 0) {
+      store_whole();
+    } else {
+      store_half(0);
+      store_half(1);
+    }
     // MODE 2: this thread's (Dt^T V)^T (rows 32 part ..) and (P^d V)^T (tokens 16 part ..),
     // each loaded from L2 (the issuer prefetches records there) just before the wait that
     // precedes its use; short live ranges keep them out of local memory, where a pending
@@ -1657,15 +1698,27 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       tc_fence_after();
       {
         const float *gcv = reinterpret_cast<const float *>(st + rec_sc(NS)) + (CHAN ? 32 * part : 0);
-        if constexpr (MODE < 2) {   // both halves of dS^T in one wait
+        if constexpr (MODE == 0) {   // both halves of dS^T in one wait, one hand-off
           float d0[16], d1[16];
           tmem_ld16(lrow + COL_DS + 32 * part, d0);
           tmem_ld16(lrow + COL_DS + 32 * part + 16, d1);
           tmem_wait_ld();
+          const float gc = gcv[0];
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            S[m] = fmaf(gcv[CHAN ? m : 0], S[m], d0[m]);
-            S[16 + m] = fmaf(gcv[CHAN ? 16 + m : 0], S[16 + m], d1[m]);
+            S[m] = fmaf(gc, S[m], d0[m]);
+            S[16 + m] = fmaf(gc, S[16 + m], d1[m]);
+          }
+          store_whole();
+        } else if constexpr (MODE == 1) {   // channel decay: half by half (registers)
+#pragma unroll
+          for (int hv = 0; hv < 2; ++hv) {
+            float d[16];
+            tmem_ld16(lrow + COL_DS + 32 * part + 16 * hv, d);
+            tmem_wait_ld();
+#pragma unroll
+            for (int m = 0; m < 16; ++m) S[16 * hv + m] = fmaf(gcv[16 * hv + m], S[16 * hv + m], d[m]);
+            store_half(hv);
           }
         } else {   // GDN-2: two halves of 16 rows keep its extra terms in registers
 #pragma unroll
@@ -1686,8 +1739,9 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 #pragma unroll
             for (int m = 0; m < 16; ++m) S[16 * hv + m] = fmaf(gcv[16 * hv + m], S[16 * hv + m], d[m]);
           }
+          store_half(0);
+          store_half(1);
         }
-        store_state();
         smax = fmaxf(smax, fmaxf(max_abs16(S), max_abs16(S + 16)));   // after the hand-off
         if constexpr (MODE == 2) load_od(c);
       }
