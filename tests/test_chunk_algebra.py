@@ -461,3 +461,103 @@ def test_scalar_backward_as_built_matches_the_oracle(variant):
     np.testing.assert_allclose(g["initial_state"], g_ref["initial_state"][0, 0], rtol=0, atol=1e-10)
     if variant != "deltanet":
         np.testing.assert_allclose(g["log_g"], g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
+
+
+def channel_local_as_built(K, Q, V, b, lg, S0, dS, dO, scale):
+    """KDA's chunk-local gradients in the form the CUDA path computes them (one
+    chunk, lg [n, dk] the per-channel log decay, S0 the chunk's start state, dS
+    its end-state gradient).  With g the chunk-local cumulative log decay per
+    channel and a middle token m, the decay enters only through per-element
+    factors on the K and Q operands and on the results:
+        a = e^(g - g_m), bb = e^(g_m - g) (K o a)(K o bb)^T = the decayed Gram,
+        e = e^g, f = e^(g_C - g) (both at most 1)
+        A = tril(Diag(beta) (K o a)(K o bb)^T, -1),  T = (I + A)^-1
+        W = T Diag(beta) (K o e),  E = T Diag(beta) V - W S0
+        P = scale tril((Q o a)(K o bb)^T),  dE = (K o f) dS + P^T dO
+        dW = -dE S0^T,  dP = tril(dO E^T),  dT = dE V^T Diag(beta) + dW (K o e)^T Diag(beta)
+        dA = tril(-T^T dT T^T, -1),  N1 = Diag(beta) dA,  N2 = scale dP
+        dk = f o E dS^T + e o Diag(beta) T^T dW + a o N1 (K o bb) + bb o N1^T (K o a) + bb o N2^T (Q o a)
+        dq = e o scale dO S0^T + a o N2 (K o bb),  dv = Diag(beta) T^T dE
+        dbeta = rowsum(V o T^T dE) + rowsum((K o e) o T^T dW) + rowsum(dA o (K o a)(K o bb)^T)
+        dg = dq o Q + (e o Diag(beta) T^T dW + a o N1 (K o bb) - f o E dS^T
+             - bb o N1^T (K o a) - bb o N2^T (Q o a)) o K,
+             plus at the chunk's last token colsum(f o E dS^T o K) + e^(g_C) o rowsum(dS o S0)
+        dlog_g_t = sum over s >= t of dg_s (per channel)."""
+    n = K.shape[0]
+    g = np.cumsum(lg, axis=0)
+    m = (n - 1) // 2
+    a, bb = np.exp(g - g[m]), np.exp(g[m] - g)
+    e, f = np.exp(g), np.exp(g[-1] - g)
+    Ka, Kb, Qa, Ke, Kf = K * a, K * bb, Q * a, K * e, K * f
+    Gd = Ka @ Kb.T
+    A = np.tril(b[:, None] * Gd, -1)
+    Tm = np.linalg.inv(np.eye(n) + A)
+    W = Tm @ (b[:, None] * Ke)
+    E = Tm @ (b[:, None] * V) - W @ S0
+    P = np.tril(scale * (Qa @ Kb.T))
+    dE = Kf @ dS + P.T @ dO
+    dW = -dE @ S0.T
+    dP = np.tril(dO @ E.T)
+    dT = (dE @ V.T) * b[None, :] + (dW @ Ke.T) * b[None, :]
+    dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+    N1 = b[:, None] * dA
+    N2 = scale * dP
+    tU, tW = Tm.T @ dE, Tm.T @ dW
+    X1 = f * (E @ dS.T)
+    Y1 = e * (b[:, None] * tW) + a * (N1 @ Kb)
+    Y2 = bb * (N1.T @ Ka) + bb * (N2.T @ Qa)
+    dq = e * (scale * dO @ S0.T) + a * (N2 @ Kb)
+    dk = X1 + Y1 + Y2
+    dv = b[:, None] * tU
+    dbeta = np.sum(V * tU, 1) + np.sum(Ke * tW, 1) + np.sum(dA * Gd, 1)
+    dg = dq * Q + (Y1 - X1 - Y2) * K
+    dg[n - 1] += np.sum(X1 * K, 0) + np.exp(g[-1]) * np.sum(dS * S0, 1)
+    return dq, dk, dv, dbeta, np.cumsum(dg[::-1], axis=0)[::-1]
+
+
+def test_channel_backward_as_built_matches_the_oracle():
+    """KDA: the forward and reverse carries in chunk form (as for the scalar
+    decay, with Gamma_C a vector) and the channel-resolved local gradients,
+    against the reverse-mode oracle."""
+    B, T, H, dk, dv, scale = 1, 29, 1, 6, 5, 0.7
+    d = make_inputs("kda", B, T, H, dk, dv, dtype=torch.float32, seed=13)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    rng = np.random.default_rng(13)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    dO = rng.standard_normal((B, T, H, dv))
+    dSf = rng.standard_normal((B, H, dk, dv))
+    g_ref = oracle.backward("kda", d_o=dO, d_final=dSf, initial_state=s0, scale=scale, **d)
+    q, k, v, beta, lg = (d[x][0, :, 0] for x in ("q", "k", "v", "beta", "log_g"))
+    dOn = dO[0, :, 0]
+    chunks = [slice(c0, min(T, c0 + C)) for c0 in range(0, T, C)]
+    # forward carry: chunk start states
+    S, S0s = s0[0, 0].copy(), []
+    for sl in chunks:
+        K, V, bt = k[sl], v[sl], beta[sl]
+        gam = np.cumsum(lg[sl], axis=0)
+        n = K.shape[0]
+        A = np.tril(bt[:, None] * ((K * np.exp(gam)) @ (K * np.exp(-gam)).T), -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        E = Tm @ (bt[:, None] * V) - Tm @ (bt[:, None] * K * np.exp(gam)) @ S
+        S0s.append(S.copy())
+        S = np.exp(gam[-1])[:, None] * S + (K * np.exp(gam[-1] - gam)).T @ E
+    # reverse carry: end-state gradients
+    X, dSs = dSf[0, 0].copy(), [None] * len(chunks)
+    for c in reversed(range(len(chunks))):
+        sl = chunks[c]
+        K, Q, bt = k[sl], q[sl], beta[sl]
+        gam = np.cumsum(lg[sl], axis=0)
+        n = K.shape[0]
+        dSs[c] = X.copy()
+        A = np.tril(bt[:, None] * ((K * np.exp(gam)) @ (K * np.exp(-gam)).T), -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ (bt[:, None] * K * np.exp(gam))
+        P = np.tril(scale * ((Q * np.exp(gam)) @ (K * np.exp(-gam)).T))
+        dE = (K * np.exp(gam[-1] - gam)) @ X + P.T @ dOn[sl]
+        X = np.exp(gam[-1])[:, None] * X + scale * (Q * np.exp(gam)).T @ dOn[sl] - W.T @ dE
+    np.testing.assert_allclose(X, g_ref["initial_state"][0, 0], rtol=0, atol=1e-10)
+    for c, sl in enumerate(chunks):
+        dq, dkk, dvv, db, dlg = channel_local_as_built(k[sl], q[sl], v[sl], beta[sl], lg[sl], S0s[c], dSs[c],
+                                                       dOn[sl], scale)
+        for name, x in (("q", dq), ("k", dkk), ("v", dvv), ("beta", db), ("log_g", dlg)):
+            np.testing.assert_allclose(x, g_ref[name][0, sl, 0], rtol=0, atol=1e-10, err_msg=name)
