@@ -299,7 +299,7 @@ gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, i
   if (st != GDR_OK) return st;
   if (!gdr_bwd_supported(variant, dtype == GDR_BF16, dk, dv))
     return fail(GDR_ERR_UNSUPPORTED,
-                "the backward covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O, dk = 128 and dv in {64, 128}");
+                "the backward covers DeltaNet, Gated DeltaNet, KDA and KLA with bf16 I/O, dk = 128 and dv in {64, 128}");
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
   if (!a || !g) return fail(GDR_ERR_INVALID_ARG, "args and grads are required");
   if ((long)B * H == 0) return GDR_OK;

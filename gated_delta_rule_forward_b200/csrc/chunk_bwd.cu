@@ -1,5 +1,5 @@
-// Chunk-parallel kernels of the chunked backward for the scalar-decay variants
-// (DeltaNet, Gated DeltaNet, KLA).  "Gated DeltaNet-2" (technical core) asks
+// Chunk-parallel kernels of the chunked backward for DeltaNet, Gated DeltaNet,
+// KDA and KLA.  "Gated DeltaNet-2" (technical core) asks
 // for a gate-aware backward that keeps the chunkwise structure; this one
 // reverses the forward's chunk algebra ("Kaczmarz Linear Attention", KLA
 // update rule and implementation):
@@ -91,6 +91,51 @@ template <typename V>
 __device__ __forceinline__ float at(const V &m, int r, int c) {
   return ld1<typename V::elem, V::kGlobal>(m.p + (V::kTr ? c * m.ld + r : r * m.ld + c));
 }
+// Channel decay (KDA): a bf16 tile of K or Q scaled element by element by
+// 2^(sg (gamma[t][i] - ref[i])), gamma the chunk-local cumulative log2 decay per
+// token t and channel i (an fp32 tile of row stride LDG in shared memory) and
+// ref a per-channel vector.  Element (r, c) is the (token, channel) one, or the
+// (channel, token) one for TR; a GLOBAL tile has token rows ld apart and reads
+// zero past the chunk's n tokens.
+constexpr int LDG = DK + 4;
+template <bool TR, bool GLOBAL = false>
+struct Fac {
+  using elem = float;
+  static constexpr bool kTr = TR;
+  static constexpr bool kGlobal = GLOBAL;
+  static constexpr bool kExact = false;
+  const __nv_bfloat16 *x;
+  int ld, n;
+  const float *g, *ref;
+  float sg;
+};
+template <bool TR, bool GLOBAL>
+__device__ __forceinline__ float at(const Fac<TR, GLOBAL> &m, int r, int c) {
+  const int t = TR ? c : r, i = TR ? r : c;
+  float x;
+  if constexpr (GLOBAL) {
+    x = t < m.n ? __bfloat162float(__ldg(m.x + t * m.ld + i)) : 0.f;
+  } else {
+    x = __bfloat162float(m.x[t * m.ld + i]);
+  }
+  return x * ex2(m.sg * (m.g[t * LDG + i] - m.ref[i]));
+}
+// A bf16 tile in global memory with token rows ld apart, zero past the chunk's n tokens.
+template <bool TR>
+struct GB {
+  using elem = __nv_bfloat16;
+  static constexpr bool kTr = TR;
+  static constexpr bool kGlobal = true;
+  static constexpr bool kExact = true;
+  const __nv_bfloat16 *x;
+  int ld, n;
+};
+template <bool TR>
+__device__ __forceinline__ float at(const GB<TR> &m, int r, int c) {
+  const int t = TR ? c : r, j = TR ? r : c;
+  return t < m.n ? __bfloat162float(__ldg(m.x + t * m.ld + j)) : 0.f;
+}
+
 // The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N
 // product shared by W warps.
 template <int M, int N, int W = 8>
@@ -374,15 +419,18 @@ struct LocalParams {
   bool decay, kla;
   float eps, scale;
   const __nv_bfloat16 *q, *k, *v, *d_o;
-  const float *beta, *log_g;
+  const float *beta, *log_g;   // log_g [B,T,H], or [B,T,H,d_k] with channel decay
   const float *s0s, *dss;   // chunk start states and end-state gradients (the latter in reverse chunk order)
   const uint32_t *absmax;
   __nv_bfloat16 *dq, *dk, *dv;
-  float *dbeta, *dlog_g;
+  float *dbeta, *dlog_g;    // dlog_g laid out as log_g
 };
 
-template <int DV>
+// CHAN: channel decay, with the decay tile after the scalars; at d_v = 128 Q and
+// V are then read from global memory (through the read-only cache) to make room.
+template <int DV, bool CHAN>
 struct LocalSmem {
+  static constexpr bool kQVGlobal = CHAN && DV == 128;
   static constexpr int LDB = DK + 8;    // bf16 rows of K, Q
   static constexpr int LDBV = DV + 8;   // bf16 rows of V, dO
   static constexpr int LDF = DV + 4;    // fp32 rows of dE, E
@@ -391,8 +439,8 @@ struct LocalSmem {
   static constexpr int LDH = 66;        // fp32 rows of a 64-column half of S0 or dS
   static constexpr size_t K = 0;
   static constexpr size_t Q = K + C * LDB * 2;
-  static constexpr size_t V = Q + C * LDB * 2;
-  static constexpr size_t O = V + C * LDBV * 2;
+  static constexpr size_t V = Q + (kQVGlobal ? 0 : C * LDB * 2);
+  static constexpr size_t O = V + (kQVGlobal ? 0 : C * LDBV * 2);
   static constexpr size_t E = O + C * LDBV * 2;
   static constexpr size_t W = E + static_cast<size_t>(std::max(C * LDF, C * LDC)) * 4;
   static constexpr size_t TT = W + static_cast<size_t>(std::max(C * LDW, DK * LDC)) * 4;
@@ -400,7 +448,9 @@ struct LocalSmem {
   static constexpr size_t A = DE + C * LDF * 4;
   static constexpr size_t P = A + C * LD * 4;
   static constexpr size_t SC = P + C * LDC * 4;
-  static constexpr size_t BYTES = SC + (9 * C + 4) * 4;
+  static constexpr size_t GAM = SC + (9 * C + 4 + (CHAN ? 5 * DK : 0)) * 4;   // [C][LDG] gamma
+  static constexpr size_t BYTES = GAM + (CHAN ? C * LDG * 4 : 0);
+  static_assert(BYTES <= 232448 && GAM % 16 == 0, "shared memory");
   static_assert(A + C * LD * 4 + C * LDC * 4 - DE >= static_cast<size_t>(DK) * LDF * 4, "S0 staging over dE, A, P");
   static_assert(std::max(C * LDW, DK * LDC) >= DK * LDH, "a half of dS over W");
   static constexpr bool kS0HalvesOverE = std::max(C * LDF, C * LDC) >= DK * LDH;   // d_v = 128
@@ -409,12 +459,29 @@ struct LocalSmem {
 // One CTA of NTL threads per chunk (b, h, c): sixteen warps share each
 // product, so that the chunk's chain of small dependent products runs with
 // twice the warps in flight of an eight-warp CTA (one CTA fits an SM).
+//
+// With channel decay (CHAN, KDA: "Gated DeltaNet-2", what is new) the decay
+// enters the products element by element.  With gamma the chunk-local
+// cumulative log decay per token and channel, factored around token m = 31 as
+// the forward's preparation factors it (whose range check bounds every factor
+// by 2^120), a = e^(gamma - gamma_m), b = e^(gamma_m - gamma), e = e^gamma and
+// f = e^(gamma_C - gamma), all (token x channel):
+//     G~ = (K o a)(K o b)^T,  A = tril(Diag(beta) G~, -1),  P = scale tril((Q o a)(K o b)^T)
+//     W = T Diag(beta) (K o e),  dE = (K o f) dS + P^T dO,  dT = (dE V^T + dW (K o e)^T) Diag(beta)
+//     N1 = Diag(beta) dA,  N2 = scale dP
+//     X1 = f o (E dS^T),  Y1 = e o (Diag(beta) T^T dW) + a o (N1 (K o b)),
+//     Y2 = b o (N1^T (K o a) + N2^T (Q o a))
+//     dk = X1 + Y1 + Y2,  dq = scale e o (dO S0^T) + a o (N2 (K o b))
+//     dbeta = rowsum(V o T^T dE) + rowsum((K o e) o T^T dW) + rowsum(dA o G~)
+//     dg = dq o Q + (Y1 - X1 - Y2) o K, plus sum_t (X1 o K)_t + e^(gamma_C) o rowsum(dS o S0)
+//     at the chunk's last token; dlog_g = per-channel suffix sums of dg over the chunk.
 constexpr int NTL = 512;
-template <int DV>
+template <int DV, bool CHAN>
 __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) {
-  using L = LocalSmem<DV>;
+  using L = LocalSmem<DV, CHAN>;
+  constexpr bool QVG = L::kQVGlobal;
   constexpr int LDB = L::LDB, LDBV = L::LDBV, LDF = L::LDF, LDW = L::LDW, LDC = L::LDC;
-  constexpr int NRV = DV / 16, NRK = DK / 16;
+  static_assert(NTL == 4 * DK, "the channel scans run four 16-token parts per channel");
   extern __shared__ float4 smem_loc[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(smem_loc);
   __nv_bfloat16 *sK = reinterpret_cast<__nv_bfloat16 *>(sm + L::K);
@@ -437,6 +504,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   float *sdg = sdb + C;       // dg
   float *snk = sdg + C;       // ||k||^2
   float *sred = snk + C;      // [0] sum X1 o K, [1] sum dS o S0
+  // channel decay: gamma_m, gamma_C, zeros, and per channel sum_t X1 o K and sum_v dS o S0
+  float *sgm = sred + 4, *sgC = sgm + DK, *szero = sgC + DK, *sx1k = szero + DK, *sss = sx1k + DK;
+  float *sgam = reinterpret_cast<float *>(sm + L::GAM);   // [C][LDG] cumulative log2 decay
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x / p.NC, c = blockIdx.x - bh * p.NC;
@@ -453,21 +523,29 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     const int t = i / (DK / 8), j = i % (DK / 8);
     uint4 uq = make_uint4(0u, 0u, 0u, 0u), uk = uq;
     if (t < n) {
-      uq = __ldg(reinterpret_cast<const uint4 *>(p.q + row(t) * DK) + j);
+      if constexpr (!QVG) uq = __ldg(reinterpret_cast<const uint4 *>(p.q + row(t) * DK) + j);
       uk = __ldg(reinterpret_cast<const uint4 *>(p.k + row(t) * DK) + j);
     }
-    *reinterpret_cast<uint4 *>(sQ + t * LDB + 8 * j) = uq;
+    if constexpr (!QVG) *reinterpret_cast<uint4 *>(sQ + t * LDB + 8 * j) = uq;
     *reinterpret_cast<uint4 *>(sK + t * LDB + 8 * j) = uk;
   }
   for (int i = tid; i < C * DV / 8; i += NTL) {
     const int t = i / (DV / 8), j = i % (DV / 8);
     uint4 uv = make_uint4(0u, 0u, 0u, 0u), uo = uv;
     if (t < n) {
-      uv = __ldg(reinterpret_cast<const uint4 *>(p.v + row(t) * DV) + j);
+      if constexpr (!QVG) uv = __ldg(reinterpret_cast<const uint4 *>(p.v + row(t) * DV) + j);
       uo = __ldg(reinterpret_cast<const uint4 *>(p.d_o + row(t) * DV) + j);
     }
-    *reinterpret_cast<uint4 *>(sV + t * LDBV + 8 * j) = uv;
+    if constexpr (!QVG) *reinterpret_cast<uint4 *>(sV + t * LDBV + 8 * j) = uv;
     *reinterpret_cast<uint4 *>(sO + t * LDBV + 8 * j) = uo;
+  }
+  if constexpr (CHAN) {   // log g per channel (zero past T: no decay)
+    for (int i = tid; i < C * DK / 4; i += NTL) {
+      const int t = i / (DK / 4), j = i % (DK / 4);
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < n) x = __ldg(reinterpret_cast<const float4 *>(p.log_g + row(t) * DK) + j);
+      *reinterpret_cast<float4 *>(sgam + t * LDG + 4 * j) = x;
+    }
   }
   if (tid < C) {
     sdb[tid] = 0.f;
@@ -487,7 +565,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     }
     if (t < n) {
       bt = __ldg(p.beta + row(t));
-      if (p.decay) lg = __ldg(p.log_g + row(t));
+      if (!CHAN && p.decay) lg = __ldg(p.log_g + row(t));
     }
     if (p.kla) bt = bt / (nk + p.eps);
     snk[t] = nk;
@@ -514,6 +592,28 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     sbe[t] = sbeta[t] * e;
   }
   __syncthreads();
+  if constexpr (CHAN) {   // gamma: per-channel prefix sums in log2 units, four 16-token parts
+    const int i = tid % DK, part = tid / DK;
+    float *stot = sdE;   // part totals (dE holds nothing yet)
+    float run = 0.f;
+    for (int t = 16 * part; t < 16 * part + 16; ++t) {
+      run = fmaf(sgam[t * LDG + i], LOG2E_BWD, run);
+      sgam[t * LDG + i] = run;
+    }
+    stot[part * DK + i] = run;
+    __syncthreads();
+    float off = 0.f;
+    for (int q = 0; q < part; ++q) off += stot[q * DK + i];
+    for (int t = 16 * part; t < 16 * part + 16; ++t) sgam[t * LDG + i] += off;
+    __syncthreads();
+    if (tid < DK) {
+      sgm[tid] = sgam[31 * LDG + tid];
+      sgC[tid] = sgam[(n - 1) * LDG + tid];
+      szero[tid] = 0.f;
+      sx1k[tid] = 0.f;
+    }
+    __syncthreads();
+  }
 
   constexpr int LW = NTL / 32;
   using CC = Tiling<C, C, LW>;     // C x C products
@@ -531,14 +631,46 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   using FG = Mat<float, false, true>;     // a global fp32 matrix (S0, dS)
   using TX = Mat<float, false, false, true>;   // T (tf32 values from the solve)
   using TXT = Mat<float, true, false, true>;   // ... transposed
+  // channel decay: K o 2^(sg (gamma - ref)) and Q o a, V as stored or read from global memory
+  auto kfac = [&](const float *ref, float sg) { return Fac<false>{sK, LDB, C, sgam, ref, sg}; };
+  auto kfacT = [&](const float *ref, float sg) { return Fac<true>{sK, LDB, C, sgam, ref, sg}; };
+  auto qa = [&]() {
+    if constexpr (QVG) return Fac<false, true>{p.q + row(0) * DK, p.H * DK, n, sgam, sgm, 1.f};
+    else return Fac<false>{sQ, LDB, C, sgam, sgm, 1.f};
+  };
+  auto qaT = [&]() {
+    if constexpr (QVG) return Fac<true, true>{p.q + row(0) * DK, p.H * DK, n, sgam, sgm, 1.f};
+    else return Fac<true>{sQ, LDB, C, sgam, sgm, 1.f};
+  };
+  auto vm = [&]() {
+    if constexpr (QVG) return GB<false>{p.v + row(0) * DV, p.H * DV, n};
+    else return BK{sV, LDBV};
+  };
+  auto vmT = [&]() {
+    if constexpr (QVG) return GB<true>{p.v + row(0) * DV, p.H * DV, n};
+    else return BKT{sV, LDBV};
+  };
+  auto qat = [&](int t, int i) {
+    if constexpr (QVG) return t < n ? __bfloat162float(__ldg(p.q + row(t) * DK + i)) : 0.f;
+    else return __bfloat162float(sQ[t * LDB + i]);
+  };
+  auto vat = [&](int t, int v) {
+    if constexpr (QVG) return t < n ? __bfloat162float(__ldg(p.v + row(t) * DV + v)) : 0.f;
+    else return __bfloat162float(sV[t * LDBV + v]);
+  };
 
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
     float g[CC::NT][4];
     zero(g);
-    wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    if constexpr (CHAN) {
+      wmm<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    }
     each(g, mc, nc, lane, [&](int t, int r, float &x) {
-      sA[r * LD + t] = tf32r(r < t ? sbeta[t] * ex2(sG[t] - sG[r]) * x : 0.f);
+      const float d = CHAN ? 1.f : ex2(sG[t] - sG[r]);
+      sA[r * LD + t] = tf32r(r < t ? sbeta[t] * d * x : 0.f);
     });
   }
   __syncthreads();
@@ -552,11 +684,15 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // ---- U' = T Diag(beta) V and W = T Diag(beta e) K; E = U' - W S0
   float ue[CV::NT][4];
   zero(ue);
-  wmm<CV::NT, false>(ue, TX{sT, LD}, BK{sV, LDBV}, C, mv, nv, lane, sbeta);
+  wmm<CV::NT, false>(ue, TX{sT, LD}, vm(), C, mv, nv, lane, sbeta);
   {
     float w[CK::NT][4];
     zero(w);
-    wmm<CK::NT, false>(w, TX{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
+    if constexpr (CHAN) {
+      wmm<CK::NT, false>(w, TX{sT, LD}, kfac(szero, 1.f), C, mk, nk, lane, sbeta);
+    } else {
+      wmm<CK::NT, false>(w, TX{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
+    }
     each(w, mk, nk, lane, [&](int t, int i, float &x) { sW[t * LDW + i] = x; });
   }
   // S0 through shared memory (over dE, A and P, none of which holds data yet):
@@ -572,7 +708,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   float dqT[KC::NT][4];
   zero(dqT);
   wmm<KC::NT, false>(dqT, F{sS, LDF}, BKT{sO, LDBV}, DV, mt, nt, lane);
-  each(dqT, mt, nt, lane, [&](int, int t, float &x) { x *= p.scale * see[t]; });
+  each(dqT, mt, nt, lane, [&](int i, int t, float &x) { x *= p.scale * (CHAN ? ex2(sgam[t * LDG + i]) : see[t]); });
   __syncthreads();   // S0's staging is read: P may overwrite it
   // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
   // reverse carry's own dE is Diag(beta) dE (its records carry beta in P and Kt), so it is
@@ -580,9 +716,13 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float gq[CC::NT][4];
     zero(gq);
-    wmm<CC::NT, false>(gq, BK{sQ, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    if constexpr (CHAN) {
+      wmm<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(gq, BK{sQ, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    }
     each(gq, mc, nc, lane, [&](int t, int r, float &x) {
-      sP[t * LDC + r] = r <= t ? p.scale * ex2(sG[t] - sG[r]) * x : 0.f;
+      sP[t * LDC + r] = r <= t ? p.scale * (CHAN ? 1.f : ex2(sG[t] - sG[r])) * x : 0.f;
     });
   }
   __syncthreads();
@@ -590,11 +730,20 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // finished reading): dE's columns of the half, and dk^T's first part
   // (Diag(f) E dS^T)^T / s accumulated over the halves
   float dkT[KC::NT][4];
-  float dgp[KC::NT][2];   // this thread's column sums toward dg_t (columns n0 + 8 j + 2 t + e)
+  float dgp[KC::NT][2];   // scalar decay: this thread's column sums toward dg_t (columns n0 + 8 j + 2 t + e)
+  float dgT[KC::NT][4];   // channel decay: dg^T, the tile of dkT
   float x1k = 0.f;
   zero(dkT);
+  zero(dgT);
 #pragma unroll
   for (int j = 0; j < KC::NT; ++j) dgp[j][0] = dgp[j][1] = 0.f;
+  auto add_dg = [&](int j, int e, float y) {
+    if constexpr (CHAN) {
+      dgT[j][e] += y;
+    } else {
+      dgp[j][e & 1] += y;
+    }
+  };
   {
     using CH = Tiling<C, 64, LW>;
     const int mh = CH::m0(warp), nh = CH::n0(warp);
@@ -608,20 +757,39 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       __syncthreads();
       float acc[CH::NT][4];
       zero(acc);
-      wmm<CH::NT, false>(acc, BK{sK, LDB}, F{sH, L::LDH}, DK, mh, nh, lane);
-      each(acc, mh, nh, lane, [&](int t, int, float &x) { x *= sff[t] * inv_s; });
+      if constexpr (CHAN) {
+        wmm<CH::NT, false>(acc, kfac(sgC, -1.f), F{sH, L::LDH}, DK, mh, nh, lane);
+        each(acc, mh, nh, lane, [&](int, int, float &x) { x *= inv_s; });
+      } else {
+        wmm<CH::NT, false>(acc, BK{sK, LDB}, F{sH, L::LDH}, DK, mh, nh, lane);
+        each(acc, mh, nh, lane, [&](int t, int, float &x) { x *= sff[t] * inv_s; });
+      }
       wmm<CH::NT, false>(acc, FT{sP, LDC}, BK{sO + 64 * h, LDBV}, C, mh, nh, lane);
       each(acc, mh, nh, lane, [&](int t, int v, float &x) { sdE[t * LDF + 64 * h + v] = x; });
       wmm<KC::NT, false>(dkT, F{sH, L::LDH}, FT{sE + 64 * h, LDF}, 64, mt, nt, lane);
       __syncthreads();   // the half is read before the next one lands
     }
   }
-  each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
-    x *= sff[t] * inv_s;
-    const float y = x * __bfloat162float(sK[t * LDB + i]);
-    x1k += y;
-    dgp[j][e & 1] -= y;
-  });
+  {
+    float x1r[2] = {0.f, 0.f};   // channel decay: rows mt + g, mt + g + 8 of sum_t X1 o K
+    each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+      x *= (CHAN ? ex2(sgC[i] - sgam[t * LDG + i]) : sff[t]) * inv_s;
+      const float y = x * __bfloat162float(sK[t * LDB + i]);
+      if constexpr (CHAN) {
+        x1r[e >> 1] += y;
+      } else {
+        x1k += y;
+      }
+      add_dg(j, e, -y);
+    });
+    if constexpr (CHAN) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float s2 = quad_sum(x1r[h2]);
+        if ((lane & 3) == 0) atomicAdd(&sx1k[mt + (lane >> 2) + 8 * h2], s2);
+      }
+    }
+  }
   // ---- dP = tril(dO E^T)
   {
     float acc[CC::NT][4];
@@ -661,7 +829,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     wmm<CV::NT, false>(acc, TXT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
     float part[2] = {0.f, 0.f};   // rows g and g + 8 of the tile
     each_je(acc, mv, nv, lane, [&](int, int e, int t, int v, float &x) {
-      part[e >> 1] = fmaf(__bfloat162float(sV[t * LDBV + v]), x, part[e >> 1]);
+      part[e >> 1] = fmaf(vat(t, v), x, part[e >> 1]);
       x *= sbeta[t];
     });
     const int g = lane >> 2, tq = lane & 3;
@@ -693,10 +861,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       for (int e = 0; e < 4; ++e) {
         const int i = mt + (lane >> 2) + 8 * (e >> 1), t = nt + 8 * j + 2 * (lane & 3) + (e & 1);
         const float kv = __bfloat162float(sK[t * LDB + i]);
-        const float y = sbe[t] * acc[j][e];
+        const float et = CHAN ? ex2(sgam[t * LDG + i]) : see[t];
+        const float y = (CHAN ? sbeta[t] * et : sbe[t]) * acc[j][e];
         dkT[j][e] += y;
-        dgp[j][e & 1] = fmaf(y, kv, dgp[j][e & 1]);
-        dbp[j][e & 1] = fmaf(see[t] * kv, acc[j][e], dbp[j][e & 1]);
+        add_dg(j, e, y * kv);
+        dbp[j][e & 1] = fmaf(et * kv, acc[j][e], dbp[j][e & 1]);
       }
 #pragma unroll
     for (int j = 0; j < KC::NT; ++j)
@@ -711,14 +880,18 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     float a1[CC::NT][4], a2[CC::NT][4];
     zero(a1);
     zero(a2);
-    wmm<CC::NT, false>(a1, F{sdE, LDF}, BKT{sV, LDBV}, DV, mc, nc, lane);
-    wmm<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
+    wmm<CC::NT, false>(a1, F{sdE, LDF}, vmT(), DV, mc, nc, lane);
+    if constexpr (CHAN) {
+      wmm<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
+    }
 #pragma unroll
     for (int j = 0; j < CC::NT; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int t = mc + (lane >> 2) + 8 * (e >> 1), r = nc + 8 * j + 2 * (lane & 3) + (e & 1);
-        sA[t * LD + r] = sbeta[r] * a1[j][e] + sbe[r] * a2[j][e];
+        sA[t * LD + r] = CHAN ? sbeta[r] * (a1[j][e] + a2[j][e]) : sbeta[r] * a1[j][e] + sbe[r] * a2[j][e];
       }
   }
   __syncthreads();
@@ -741,12 +914,17 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float g[CC::NT][4];
     zero(g);
-    wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    if constexpr (CHAN) {
+      wmm<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
+    }
     float part[2] = {0.f, 0.f};
     each_je(g, mc, nc, lane, [&](int, int e, int t, int r, float &x) {
-      const float d = r <= t ? ex2(sG[t] - sG[r]) : 0.f;
+      const float d = r <= t ? (CHAN ? 1.f : ex2(sG[t] - sG[r])) : 0.f;
       const float da = sA[t * LD + r];
-      part[e >> 1] = fmaf(da * d, x, part[e >> 1]);
+      // dA is strictly lower; above the diagonal the factored Gram may overflow (0 inf = NaN)
+      if (r < t) part[e >> 1] = fmaf(da * d, x, part[e >> 1]);
       sA[t * LD + r] = sbeta[t] * da * d;
       sP[t * LDC + r] = p.scale * sP[t * LDC + r] * d;
     });
@@ -761,52 +939,78 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[KC::NT][4];
     zero(acc);
-    wmm<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
-    each_je(acc, mt, nt, lane,
-            [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] += x * __bfloat162float(sK[t * LDB + i]); });
-#pragma unroll
-    for (int j = 0; j < KC::NT; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dkT[j][e] += acc[j][e];
+    if constexpr (CHAN) {
+      wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
+    } else {
+      wmm<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
+    }
+    each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+      if constexpr (CHAN) x *= ex2(sgam[t * LDG + i] - sgm[i]);
+      add_dg(j, e, x * __bfloat162float(sK[t * LDB + i]));
+      dkT[j][e] += x;
+    });
     zero(acc);
-    wmm<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
-    wmm<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
-    each_je(acc, mt, nt, lane,
-            [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] -= x * __bfloat162float(sK[t * LDB + i]); });
-#pragma unroll
-    for (int j = 0; j < KC::NT; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dkT[j][e] += acc[j][e];
+    if constexpr (CHAN) {
+      wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, qaT(), F{sP, LDC}, C, mt, nt, lane);
+    } else {
+      wmm<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
+    }
+    each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+      if constexpr (CHAN) x *= ex2(sgm[i] - sgam[t * LDG + i]);
+      add_dg(j, e, -x * __bfloat162float(sK[t * LDB + i]));
+      dkT[j][e] += x;
+    });
   }
   // ---- dq += N2 K
-  wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
-  each_je(dqT, mt, nt, lane,
-          [&](int j, int e, int i, int t, float &x) { dgp[j][e & 1] += x * __bfloat162float(sQ[t * LDB + i]); });
+  if constexpr (CHAN) {
+    float acc[KC::NT][4];
+    zero(acc);
+    wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+    each_je(acc, mt, nt, lane,
+            [&](int j, int e, int i, int t, float &x) { dqT[j][e] += x * ex2(sgam[t * LDG + i] - sgm[i]); });
+  } else {
+    wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
+  }
+  each_je(dqT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) { add_dg(j, e, x * qat(t, i)); });
 
   // ---- reductions: dg_t over the rows; sum(X1 o K); sum(dS o S0)
   {
-    float ss = 0.f;
     const float4 *a = reinterpret_cast<const float4 *>(dS), *bb = reinterpret_cast<const float4 *>(S0);
-    for (int i = tid; i < DK * DV / 4; i += NTL) {
-      const float4 x = __ldg(a + i), y = __ldg(bb + i);
-      ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
-    }
+    if constexpr (CHAN) {   // per state row: DV / 4 lanes a row, every thread the same number of rows
+      constexpr int GL = DV / 4;
+      static_assert((DK * DV / 4) % NTL == 0 && 32 % GL == 0, "row groups");
+      for (int i = tid; i < DK * DV / 4; i += NTL) {
+        const float4 x = __ldg(a + i), y = __ldg(bb + i);
+        float ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      x1k += __shfl_xor_sync(0xffffffffu, x1k, o);
-    }
-    if (lane == 0) {
-      atomicAdd(&sred[0], x1k);
-      atomicAdd(&sred[1], ss);
-    }
-#pragma unroll
-    for (int j = 0; j < KC::NT; ++j)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float s2 = column_sum(dgp[j][e]);
-        if (lane < 4) atomicAdd(&sdg[nt + 8 * j + 2 * lane + e], s2);
+        for (int o = GL / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane % GL == 0) sss[i / GL] = ss;
       }
+    } else {
+      float ss = 0.f;
+      for (int i = tid; i < DK * DV / 4; i += NTL) {
+        const float4 x = __ldg(a + i), y = __ldg(bb + i);
+        ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        x1k += __shfl_xor_sync(0xffffffffu, x1k, o);
+      }
+      if (lane == 0) {
+        atomicAdd(&sred[0], x1k);
+        atomicAdd(&sred[1], ss);
+      }
+#pragma unroll
+      for (int j = 0; j < KC::NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float s2 = column_sum(dgp[j][e]);
+          if (lane < 4) atomicAdd(&sdg[nt + 8 * j + 2 * lane + e], s2);
+        }
+    }
   }
   __syncthreads();
 
@@ -819,6 +1023,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     stk[t * LDB + i] = __float2bfloat16_rn(x);
   });
   each(dqT, mt, nt, lane, [&](int i, int t, float &x) { stq[t * LDB + i] = __float2bfloat16_rn(x); });
+  if constexpr (CHAN) {   // dg over the decay tile, which nothing reads any more
+    each(dgT, mt, nt, lane, [&](int i, int t, float &x) { sgam[t * LDG + i] = x; });
+  }
   __syncthreads();
   for (int i = tid; i < C * DK / 8; i += NTL) {
     const int t = i / (DK / 8), j = i % (DK / 8);
@@ -831,7 +1038,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   if (tid < C) {
     const int t = tid;
     if (t < n) p.dbeta[row(t)] = p.kla ? sdb[t] / (snk[t] + p.eps) : sdb[t];
-    if (p.decay && p.dlog_g != nullptr) {
+    if (!CHAN && p.decay && p.dlog_g != nullptr) {
       float x = 0.f;
       if (t < n) x = sdg[t] + (t == n - 1 ? sred[0] + ex2(sG[n - 1]) * sred[1] * inv_s : 0.f);
 #pragma unroll
@@ -843,10 +1050,28 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     }
   }
   __syncthreads();
-  if (tid < C && p.decay && p.dlog_g != nullptr) {
+  if (!CHAN && tid < C && p.decay && p.dlog_g != nullptr) {
     const int t = tid;
     const float x = sscan[t] + (t < 32 ? sscan[32] : 0.f);
     if (t < n) p.dlog_g[row(t)] = x;
+  }
+  if constexpr (CHAN) {   // per-channel suffix sums of dg, four 16-token parts per channel
+    if (p.dlog_g != nullptr) {
+      const int i = tid % DK, part = tid / DK;
+      float *stot = sdE;   // part totals (dE is dead)
+      float run = 0.f;
+      for (int t = 16 * part + 15; t >= 16 * part; --t) {
+        float x = t < n ? sgam[t * LDG + i] : 0.f;
+        if (t == n - 1) x += sx1k[i] + ex2(sgC[i]) * sss[i] * inv_s;
+        run += x;
+        sgam[t * LDG + i] = run;
+      }
+      stot[part * DK + i] = run;
+      __syncthreads();
+      float off = 0.f;
+      for (int q = part + 1; q < NTL / DK; ++q) off += stot[q * DK + i];
+      for (int t = 16 * part; t < 16 * part + 16 && t < n; ++t) p.dlog_g[row(t) * DK + i] = sgam[t * LDG + i] + off;
+    }
   }
 }
 
@@ -878,8 +1103,8 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
 
 bool gdr_bwd_supported(int variant, int dtype_bf16, int dk, int dv) {
   using namespace gdr;
-  return (variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA) && dtype_bf16 && dk == 128 &&
-         (dv == 64 || dv == 128);
+  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA;
+  return v && dtype_bf16 && dk == 128 && (dv == 64 || dv == 128);
 }
 
 size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv) {
@@ -948,8 +1173,11 @@ cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const float *s0s, con
     kern<<<grid, NTL, smem, s>>>(lp);
     return cudaGetLastError();
   };
-  return f.dv == 128 ? run(bwd_local_kernel<128>, LocalSmem<128>::BYTES)
-                     : run(bwd_local_kernel<64>, LocalSmem<64>::BYTES);
+  if (f.variant == gdr::kKDA)
+    return f.dv == 128 ? run(bwd_local_kernel<128, true>, LocalSmem<128, true>::BYTES)
+                       : run(bwd_local_kernel<64, true>, LocalSmem<64, true>::BYTES);
+  return f.dv == 128 ? run(bwd_local_kernel<128, false>, LocalSmem<128, false>::BYTES)
+                     : run(bwd_local_kernel<64, false>, LocalSmem<64, false>::BYTES);
 }
 
 cudaError_t gdr_bwd_launch_unscale(const gdr::BwdProblem &p, const float *xf, const uint32_t *absmax,

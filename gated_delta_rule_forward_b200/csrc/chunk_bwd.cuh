@@ -1,5 +1,5 @@
-// Chunked backward of the scalar-decay variants (DeltaNet, Gated DeltaNet,
-// KLA): its chunk-parallel kernels (chunk_bwd.cu) and the orchestration over
+// Chunked backward of DeltaNet, Gated DeltaNet, KDA and KLA: its
+// chunk-parallel kernels (chunk_bwd.cu) and the orchestration over
 // the forward's preparation and carry kernels (chunk_split.cu).
 #pragma once
 #include <cstdint>
@@ -15,7 +15,7 @@ struct BwdProblem {
   const float *d_final;    // [B,H,dk,dv] gradient of the final state, or null (zero)
   void *dq, *dk, *dv;      // [B,T,H,dk], [B,T,H,dk], [B,T,H,dv] I/O dtype
   float *dbeta;            // [B,T,H]: d beta, or d eta for KLA
-  float *dlog_g;           // [B,T,H] (GDN, KLA); null for DeltaNet
+  float *dlog_g;           // [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA); null for DeltaNet
   float *d_s0;             // [B,H,dk,dv] gradient of the initial state, or null
 };
 
@@ -34,8 +34,8 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv);
 
 }  // namespace gdr
 
-// The backward covers DeltaNet, Gated DeltaNet and KLA with bf16 I/O, dk = 128
-// and dv in {64, 128}.
+// The backward covers DeltaNet, Gated DeltaNet, KDA and KLA with bf16 I/O,
+// dk = 128 and dv in {64, 128}.
 bool gdr_bwd_supported(int variant, int dtype_bf16, int dk, int dv);
 size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv);
 

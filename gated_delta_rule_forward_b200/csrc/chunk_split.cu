@@ -2348,6 +2348,7 @@ cudaError_t gdr_launch_backward(const gdr::BwdProblem &p, void *ws, size_t ws_by
     case kDeltaNet: return tc::launch_backward<kDeltaNet>(p, w, stream, err);
     case kGatedDeltaNet: return tc::launch_backward<kGatedDeltaNet>(p, w, stream, err);
     case kKLA: return tc::launch_backward<kKLA>(p, w, stream, err);
+    case kKDA: return tc::launch_backward<kKDA>(p, w, stream, err);
     default: *err = "variant not covered by the backward: "; return cudaErrorInvalidValue;
   }
 }

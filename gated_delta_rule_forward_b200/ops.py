@@ -132,10 +132,10 @@ def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=No
 def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, initial_state=None, d_final_state=None,
              eps=1e-6, scale=1.0, stream=None):
     """Gradients of <d_o, o> + <d_final_state, S_T> for the forward over the
-    same inputs: the chunked backward (DeltaNet, Gated DeltaNet, KLA; bf16
-    q, k, v, d_o with dk = 128, dv 64 or 128; gates fp32 as for forward()).
-    Returns a dict with dq, dk, dv (bf16), beta (d beta, or d eta for KLA),
-    log_g (None for DeltaNet) and initial_state (fp32 [B,H,dk,dv]; the
+    same inputs: the chunked backward (DeltaNet, Gated DeltaNet, KDA, KLA;
+    bf16 q, k, v, d_o with dk = 128, dv 64 or 128; gates fp32 as for
+    forward()).  Returns a dict with dq, dk, dv (bf16), beta (d beta, or d eta
+    for KLA), log_g (shaped as log_g; None for DeltaNet) and initial_state (fp32 [B,H,dk,dv]; the
     gradient of the initial state, zero-initial-state runs included)."""
     vid = variant_id(variant)
     if q.dim() != 4:
@@ -158,7 +158,7 @@ def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, initial_state=None
         _need(d_final_state, "d_final_state", (B, H, dk, dv), f32, dev)
     g = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
          "beta": torch.empty(B, T, H, device=dev, dtype=f32),
-         "log_g": None if log_g is None else torch.empty(B, T, H, device=dev, dtype=f32),
+         "log_g": None if log_g is None else torch.empty(log_g.shape, device=dev, dtype=f32),
          "initial_state": torch.empty(B, H, dk, dv, device=dev, dtype=f32)}
     a = FwdArgs(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), beta=beta.data_ptr(),
                 log_g=None if log_g is None else log_g.data_ptr(),

@@ -223,7 +223,7 @@ typedef struct {
     void *dk;                 /* [B,T,H,dk] I/O dtype */
     void *dv;                 /* [B,T,H,dv] I/O dtype */
     float *dbeta;             /* [B,T,H]: d beta, or d eta for KLA */
-    float *dlog_g;            /* [B,T,H] (GDN, KLA); DeltaNet: unused */
+    float *dlog_g;            /* [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA); DeltaNet: unused */
     float *d_initial_state;   /* [B,H,dk,dv], or NULL when not wanted */
 } gdr_bwd_grads_t;
 
@@ -243,8 +243,8 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * forward's inputs, for the forward that `args` describes (its o and
  * final_state are not used): the gate-aware backward that keeps the
  * chunkwise structure ("Gated DeltaNet-2: Decoupling Erase and Write in
- * Linear Attention", technical core), for the scalar-decay variants DeltaNet,
- * Gated DeltaNet and KLA with bf16 I/O, dk = 128 and dv in {64, 128}.  With S
+ * Linear Attention", technical core), for DeltaNet, Gated DeltaNet, KDA and
+ * KLA with bf16 I/O, dk = 128 and dv in {64, 128}.  With S
  * the state and dS its gradient, per 64-token chunk:
  *     forward   E = U' - W S0,  O = Qg S0 + P E,  S_C = Gamma_C S0 + Kt^T E
  *     backward  dE = Kt dS + P^T dO,  dS0 = Gamma_C dS + Qg^T dO - W^T dE
@@ -254,14 +254,17 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * runs the dS recurrence through the same carry kernel over the chunks in
  * reverse (both carries in segments for few long sequences, as the
  * forward's), then computes every chunk's q, k, v and gate gradients in
- * parallel.  KLA's d eta includes the path through its Kaczmarz step
+ * parallel; for KDA the chunk products take the channel decay element by
+ * element, factored around the chunk's middle token as the forward's are
+ * (so the forward's GDR_ERR_RANGE check covers them too), and dlog_g is per
+ * channel.  KLA's d eta includes the path through its Kaczmarz step
  * eta / (||k||^2 + eps).  d_o [B,T,H,dv] in the I/O dtype (required);
  * d_final_state [B,H,dk,dv] fp32 or NULL (zero).  The tensor-core carries use
  * fp16 operands with fp32 accumulation, like the forward's chunked path: the
  * gradients match an exact backward to about 1e-3 of their RMS; the
  * gradients are rescaled internally by a power of two so that d_o's range
  * does not matter.  workspace: at least gdr_backward_workspace_size() bytes,
- * 16-byte aligned, overwritten.  The raw-input mode (GDR_RAW_INPUTS), KDA,
+ * 16-byte aligned, overwritten.  The raw-input mode (GDR_RAW_INPUTS),
  * GDN-2, fp32 I/O and dk = 64 return GDR_ERR_UNSUPPORTED.  T = 0 gives
  * d_initial_state = d_final_state.  Validation and errors as for the
  * forward; a reverse-record operand beyond the fp16 range is reported as

@@ -243,9 +243,9 @@ def bwd_call(L, variant=1, dtype=1, B=2, T=130, H=3, dk=128, dv=128, ws=None, d_
 
 def test_backward_validation(L):
     assert bwd_call(L) == 4                                  # valid: reaches the (injected) launch failure
-    for v in (0, 1, 4):
+    for v in (0, 1, 2, 4):
         assert bwd_call(L, variant=v) == 4
-    assert bwd_call(L, variant=2) == 2 and bwd_call(L, variant=3) == 2     # KDA, GDN-2: unsupported
+    assert bwd_call(L, variant=3) == 2                                       # GDN-2: unsupported
     assert bwd_call(L, variant=1 | 0x100) == 2                               # raw inputs: unsupported
     assert bwd_call(L, dtype=0) == 2 and bwd_call(L, dk=64) == 2             # fp32 I/O, dk = 64
     assert bwd_call(L, dv=96) == 2
@@ -268,6 +268,9 @@ def test_backward_workspace_sizes(L):
     up = lambda x: (x + 255) // 256 * 256
     want = up(bh * NC * rec) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
     assert L.gdr_backward_workspace_size(1, 1, B, T, H, 128, 128) == want
-    assert L.gdr_backward_workspace_size(2, 1, B, T, H, 128, 128) == 0       # KDA
+    rec_kda = rec + 512 - 16                                                 # Gamma_C as 128 floats
+    want_kda = up(bh * NC * rec_kda) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
+    assert L.gdr_backward_workspace_size(2, 1, B, T, H, 128, 128) == want_kda
+    assert L.gdr_backward_workspace_size(3, 1, B, T, H, 128, 128) == 0       # GDN-2
     assert L.gdr_backward_workspace_size(1, 0, B, T, H, 128, 128) == 0       # fp32 I/O
     assert L.gdr_backward_workspace_size(1, 1, B, 0, H, 128, 128) == 0

@@ -1,5 +1,5 @@
-"""GPU parity of the chunked backward (DeltaNet, Gated DeltaNet, KLA) against
-the fp64 reverse-mode oracle, through the C ABI.
+"""GPU parity of the chunked backward (DeltaNet, Gated DeltaNet, KDA, KLA)
+against the fp64 reverse-mode oracle, through the C ABI.
 
 The backward re-runs the forward's chunk products and carry, runs the
 end-state-gradient recurrence on the forward's carry kernel over the chunks in
@@ -20,7 +20,7 @@ from gated_delta_rule_forward_b200.inputs import make_inputs, random_output_grad
 from parity_util import assert_close, select, to_dev
 
 pytestmark = pytest.mark.gpu
-VARS = ["deltanet", "gdn", "kla"]
+VARS = ["deltanet", "gdn", "kda", "kla"]
 
 
 def run_backward(variant, B, T, H, dv=128, seed=0, s0=True, d_final=True, do_scale=1.0, scale=None, edit=None):
@@ -67,6 +67,15 @@ def test_backward_short_sequences(T):
     check_grads(g, ref, "gdn", f"T={T}")
 
 
+@pytest.mark.parametrize("T", [1, 20, 37, 65])
+def test_backward_short_sequences_channel_decay(T):
+    """KDA's chunk products factor the decay around token 31 of a chunk, or
+    around the last token of a shorter one: chunks of 1, 20 and 37 tokens and
+    a 1-token tail."""
+    g, ref = run_backward("kda", 1, T, 2, seed=31)
+    check_grads(g, ref, "kda", f"T={T}")
+
+
 def test_backward_without_states():
     """No initial state and no final-state gradient: the initial state's
     gradient is still returned (that of a zero initial state)."""
@@ -101,7 +110,43 @@ def test_backward_strong_decay():
     check_grads(g, ref, "gdn", "strong decay")
 
 
-@pytest.mark.parametrize("variant", ["gdn", "kla"])
+def chunk_span_log2(log_g):
+    """Largest |gamma_t - gamma_31| within a 64-token chunk (log2 units), gamma the
+    chunk-local cumulative log decay of each channel (zero-padded past T)."""
+    B, T, H, dk = log_g.shape
+    NC = (T + 63) // 64
+    pad = np.zeros((B, NC * 64, H, dk))
+    pad[:, :T] = log_g.double().numpy()
+    g = np.cumsum(pad.reshape(B, NC, 64, H, dk), axis=2)
+    return float(np.abs(g - g[:, :, 31:32]).max() / np.log(2.0))
+
+
+def test_backward_strong_channel_decay():
+    """KDA with its decay doubled: factors up to 2^102 within a chunk, inside
+    the forward's factoring range (2^120)."""
+    def edit(d):
+        d["log_g"] = (d["log_g"] * 2.0).contiguous()
+        span = chunk_span_log2(d["log_g"])
+        assert 90.0 < span < 120.0, span
+    g, ref = run_backward("kda", 1, 192, 2, seed=25, edit=edit)
+    check_grads(g, ref, "kda", "strong channel decay")
+
+
+def test_backward_decay_beyond_the_guard_is_reported():
+    """KDA with a decay of e^-5 per token on every channel spans 2^230 within
+    a chunk: the backward returns normally and reports GDR_ERR_RANGE."""
+    d = to_dev(make_inputs("kda", 1, 130, 2, seed=32))
+    d["log_g"] = torch.full_like(d["log_g"], -5.0)
+    dO = random_output_grad(1, 130, 2, 128, 33).cuda()
+    gdr.device_status()
+    gdr.backward(d["q"], d["k"], d["v"], dO, variant="kda", beta=d["beta"], log_g=d["log_g"])
+    with pytest.raises(gdr.GdrError) as e:
+        gdr.device_status()
+    assert e.value.status == 6, str(e.value)
+    gdr.device_status()   # the flag is cleared once read
+
+
+@pytest.mark.parametrize("variant", ["gdn", "kla", "kda"])
 def test_backward_350m_layer_sampled(variant):
     """The 350M layer (B=8, T=2048, H=8, full size, in the launch configuration of
     a training step), checked against the oracle on two of its sequences."""
@@ -123,10 +168,11 @@ def test_backward_350m_layer_sampled(variant):
 
 
 def test_backward_rejects_uncovered_cases():
-    d = to_dev(make_inputs("kda", 1, 64, 1))
-    dO = torch.zeros(1, 64, 1, 128, device="cuda", dtype=torch.bfloat16)
+    """fp32 I/O is not covered by the backward (GDR_ERR_UNSUPPORTED)."""
+    d = to_dev(make_inputs("gdn", 1, 64, 1, dtype=torch.float32))
+    dO = torch.zeros(1, 64, 1, 128, device="cuda", dtype=torch.float32)
     with pytest.raises(gdr.GdrError) as e:
-        gdr.backward(d["q"], d["k"], d["v"], dO, variant="kda", beta=d["beta"], log_g=d["log_g"])
+        gdr.backward(d["q"], d["k"], d["v"], dO, variant="gdn", beta=d["beta"], log_g=d["log_g"])
     assert e.value.status == 2   # GDR_ERR_UNSUPPORTED
 
 
@@ -150,7 +196,7 @@ def test_backward_long_context_sampled():
         check_grads(gh, ref, "gdn", f"head {h}")
 
 
-@pytest.mark.parametrize("variant", ["gdn", "kla"])
+@pytest.mark.parametrize("variant", ["gdn", "kla", "kda"])
 def test_backward_segmented(variant):
     """Few long sequences (B*H = 2, 65 chunks): both carries run in segments (13
     of 5 chunks) from an initial state and a final-state gradient."""
