@@ -55,8 +55,9 @@ WORKLOADS = {
     "gdn_decode_256x16": ("gdn", 256, None, 16, 128, 128),
     "gdn_fwd_350m_raw": ("gdn", 8, 2048, 8, 128, 128),
     "gdn_bwd_350m": ("gdn", 8, 2048, 8, 128, 128),
+    "kda_bwd_1p3b": ("kda", 4, 4096, 16, 128, 128),
 }
-BWD_WORKLOADS = {"gdn_bwd_350m"}   # the chunked backward (gradients of o and the final state)
+BWD_WORKLOADS = {"gdn_bwd_350m", "kda_bwd_1p3b"}   # the chunked backward (gradients of o and the final state)
 RAW_WORKLOADS = {"gdn_fwd_350m_raw"}   # raw projections and logits in; the kernels apply the transforms
 DEFAULT = "gdn_fwd_64k"
 DECODE_STEPS = 1024         # the decode chain after the long-context prefill

@@ -1451,6 +1451,9 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
   const int c_first = p.c_base + (pass_b ? p.seg_first_b + zi : zi) * p.seg_len;   // this CTA's first chunk
   const int NS = p.dv / 64, NC = min(p.seg_len, p.NC - c_first);   // chunks of this CTA
   const bool values = !(flags & CARRY_NO_VALUES);
+  // A carry without outputs copies only -W, Kt, U' (unless NO_VALUES) and the decay of
+  // each record, and takes neither Qg's half of the Y product nor E^T P^T.
+  const bool lite = (flags & CARRY_NO_OUTPUT) != 0;
 
   uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);   // [NSTAGE] records landed
   uint64_t *bar_e = bar_full + NSTAGE;    // Y(c) done
@@ -1504,10 +1507,25 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       const uint8_t *recs = p.ws + ((static_cast<size_t>(b) * p.H + h) * p.NC + c_first) * rb;
       auto issue_chunk = [&](int c) {
         const int s = c % NSTAGE;
-        mbar_expect_tx(&bar_full[s], p.copy_bytes);
-        bulk_load(sm + s * STAGE, recs + static_cast<size_t>(c) * rb, p.copy_bytes, &bar_full[s]);
+        const uint8_t *src = recs + static_cast<size_t>(c) * rb;
+        uint8_t *dst = sm + s * STAGE;
+        if (lite) {   // -W's two atoms, Kt, then U' (unless NO_VALUES) and the decay
+          const uint32_t tail = values ? REC_U : rec_sc(NS);
+          mbar_expect_tx(&bar_full[s], 32768 + (p.copy_bytes - tail));
+          bulk_load(dst + REC_WQ, src + REC_WQ, 8192, &bar_full[s]);
+          bulk_load(dst + REC_WQ + 16384, src + REC_WQ + 16384, 8192, &bar_full[s]);
+          bulk_load(dst + REC_K, src + REC_K, 16384, &bar_full[s]);
+          bulk_load(dst + tail, src + tail, p.copy_bytes - tail, &bar_full[s]);
+        } else {
+          mbar_expect_tx(&bar_full[s], p.copy_bytes);
+          bulk_load(dst, src, p.copy_bytes, &bar_full[s]);
+        }
         // MODE 2: the rest of the record, which the compute threads read themselves
-        if constexpr (MODE == 2) prefetch_l2(recs + static_cast<size_t>(c) * rb + p.copy_bytes, rb - p.copy_bytes);
+        // (without outputs, its state term only)
+        if constexpr (MODE == 2) {
+          const uint32_t skip = lite ? 8192u * NS : 0u;
+          prefetch_l2(src + p.copy_bytes + skip, rb - p.copy_bytes - skip);
+        }
         pend |= 1u << s;
       };
       auto wait_full = [&](int c) -> bool {
@@ -1522,6 +1540,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       // soon as those are stored and the odd ones after the rest; with a scalar
       // decay the state is handed off whole (the second hand-off costs more than
       // it saves there).
+      const uint32_t id_y = lite ? idesc_f16(128, 64, false, false) : idesc_f16(128, 128, false, false);
       auto issue_y = [&](int c) -> bool {
         const uint32_t st = smem_u32(sm + (c % NSTAGE) * STAGE);
         if constexpr (MODE == 0) {
@@ -1530,8 +1549,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
-                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   idesc_f16(128, 128, false, false), kk > 0);
+                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_y, kk > 0);
           mma_commit(bar_e);
           return true;
         }
@@ -1543,8 +1561,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           for (int k2 = 0; k2 < 4; ++k2) {
             const int kk = 2 * k2 + odd;
             mma_ts(tmem + COL_Y + 128 * (c & 1), tmem + COL_SA + 8 * kk,
-                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   idesc_f16(128, 128, false, false), kk > 0);
+                   sdesc(st + REC_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_y, kk > 0);
           }
         }
         mma_commit(bar_e);
@@ -1575,11 +1592,13 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           mma_ts(tmem + COL_DS, tmem + COL_EA + 8 * kk, sdesc(st + REC_K + kk * 2048, 8192, 1024),
                  idesc_f16(128, 128, false, true), kk > 0);
         mma_commit(bar_s);
+        if (!lite) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 8 * kk, sdesc(st + REC_P + kk * 32, 16, 1024),
-                 idesc_f16(128, 64, false, false), 1);
-        mma_commit(bar_o);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + COL_Y + 128 * (c & 1) + 64, tmem + COL_EA + 8 * kk, sdesc(st + REC_P + kk * 32, 16, 1024),
+                   idesc_f16(128, 64, false, false), 1);
+          mma_commit(bar_o);
+        }
         if (c + 1 < NC) {
           if (!(ok = wait_full(c + 1) && issue_y(c + 1))) break;
         }
@@ -1743,15 +1762,21 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           store_half(1);
         }
         smax = fmaxf(smax, fmaxf(max_abs16(S), max_abs16(S + 16)));   // after the hand-off
-        if constexpr (MODE == 2) load_od(c);
+        if constexpr (MODE == 2) {
+          if (!lite) load_od(c);
+        }
       }
 
       // output rows: tokens 16 part .. 16 part + 15 of value columns 32 quad .., transposed
-      // through this warp's 1 KB of the stage's (now unused) U'^T tile into 16-byte stores
-      ok = wait_or_abort(bar_o, c & 1, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      {
+      // through this warp's 1 KB of the stage's (now unused) U'^T tile into 16-byte stores.
+      // Without outputs the stage is released once the S update is done: every MMA that
+      // reads it completed before bar_s.
+      if (!lite) {
+        ok = wait_or_abort(bar_o, c & 1, abort);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+      }
+      if (!lite) {
         float yo[16];
         tmem_ld16(y + 64 + 16 * part, yo);
         tmem_wait_ld();
@@ -1767,7 +1792,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
             }
           }
         }
-        if (has_v && !(flags & CARRY_NO_OUTPUT)) {
+        if (has_v) {
           uint8_t *tile = st + REC_U + (quad * 4 + part) * 1024;
 #pragma unroll
           for (int m = 0; m < 16; ++m)
@@ -1783,11 +1808,11 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
                                          8 * piece) = val;
           }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_done);
       }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_done);
     }
   }
 
