@@ -302,9 +302,11 @@ struct RevPrepParams {
 
 // One CTA per forward record (b, h, c); it writes reverse record (b, h, NC-1-c)
 // in the channel-decay + GDN-2 record format the carry's third mode reads:
-//     -W slot of REC_WQ <- Kt (the Qg slot cleared),  REC_K <- -W,
+//     -W slot of REC_WQ <- Kt,  REC_K <- -W,
 //     U' slot <- R^T = (s dO)^T P,  Gamma_C as d_k values,
-//     the output term cleared,  the state term <- F^T = (s dO)^T Qg.
+//     the state term <- F^T = (s dO)^T Qg.
+// The Qg slots, P and the output term stay unwritten: the reverse carry runs
+// without outputs and reads none of them.
 template <int DV>
 __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams p) {
   constexpr int NS = DV / 64;
@@ -353,18 +355,14 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
       sQ[t * LDQ + 64 * a + 8 * j + 2 * e + 1] = f.y;
     }
   }
-  // tile copies and cleared slots (16-byte units)
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  // tile copies (16-byte units)
   for (int i = tid; i < 1024; i += NT) {
     const int a = i >> 9, j = i & 511;
     *reinterpret_cast<uint4 *>(dst + REC_WQ + a * 16384 + 16 * j) =
         *reinterpret_cast<const uint4 *>(src + REC_K + a * 8192 + 16 * j);
-    *reinterpret_cast<uint4 *>(dst + REC_WQ + a * 16384 + 8192 + 16 * j) = z;
     *reinterpret_cast<uint4 *>(dst + REC_K + a * 8192 + 16 * j) =
         *reinterpret_cast<const uint4 *>(src + REC_WQ + a * 16384 + 16 * j);
   }
-  for (int i = tid; i < 512; i += NT) *reinterpret_cast<uint4 *>(dst + REC_P + 16 * i) = z;
-  for (int i = tid; i < 512 * NS; i += NT) *reinterpret_cast<uint4 *>(dst + rec_bytes_chan(NS) + 16 * i) = z;
   if (tid < DK) {
     const float *g = reinterpret_cast<const float *>(src + rec_sc(NS));
     reinterpret_cast<float *>(dst + rec_sc(NS))[tid] = p.chan ? g[tid] : g[0];
