@@ -1578,10 +1578,11 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
       // before E(c) before S(c)), so no barrier can complete a phase the
       // issuer has not waited for yet.
       for (int c = 0; ok && c < NC; ++c) {
-        // chunk c-1 fully consumed: its stage takes record c+2
+        // chunk c-1 fully consumed: its stage takes record c+2 (without outputs, whose
+        // record takes four copies, they are issued after the dS product, off its path)
         if (c >= 1) {
           if (!(ok = wait_or_abort(bar_done, (c - 1) & 1, abort))) break;
-          if (c + 2 < NC) issue_chunk(c + 2);
+          if (!lite && c + 2 < NC) issue_chunk(c + 2);
         }
         // dS^T = E^T Kt ; Y_Q += E^T P^T
         if (!(ok = wait_or_abort(bar_ea, c & 1, abort))) break;
@@ -1592,6 +1593,7 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
           mma_ts(tmem + COL_DS, tmem + COL_EA + 8 * kk, sdesc(st + REC_K + kk * 2048, 8192, 1024),
                  idesc_f16(128, 128, false, true), kk > 0);
         mma_commit(bar_s);
+        if (lite && c >= 1 && c + 2 < NC) issue_chunk(c + 2);
         if (!lite) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
