@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
 
   // ---- inputs: bf16 tiles (zero past T)
+#pragma unroll
   for (int i = tid; i < C * DK / 8; i += NTL) {
     const int t = i / (DK / 8), j = i % (DK / 8);
     uint4 uq = make_uint4(0u, 0u, 0u, 0u), uk = uq;
@@ -527,6 +528,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     if constexpr (!QVG) *reinterpret_cast<uint4 *>(sQ + t * LDB + 8 * j) = uq;
     *reinterpret_cast<uint4 *>(sK + t * LDB + 8 * j) = uk;
   }
+#pragma unroll
   for (int i = tid; i < C * DV / 8; i += NTL) {
     const int t = i / (DV / 8), j = i % (DV / 8);
     uint4 uv = make_uint4(0u, 0u, 0u, 0u), uo = uv;
@@ -538,6 +540,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     *reinterpret_cast<uint4 *>(sO + t * LDBV + 8 * j) = uo;
   }
   if constexpr (CHAN) {   // log g per channel (zero past T: no decay)
+#pragma unroll
     for (int i = tid; i < C * DK / 4; i += NTL) {
       const int t = i / (DK / 4), j = i % (DK / 4);
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -696,6 +699,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // S0 through shared memory (over dE, A and P, none of which holds data yet):
   // E = U' - W S0 and dq's first part, scale Diag(e) dO S0^T
   float *sS = reinterpret_cast<float *>(sm + L::DE);
+#pragma unroll
   for (int i = tid; i < DK * DV / 4; i += NTL) {
     const int r = i / (DV / 4), c4 = i % (DV / 4);
     *reinterpret_cast<float4 *>(sS + r * LDF + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(S0) + i);
@@ -747,6 +751,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     const int mh = CH::m0(warp), nh = CH::n0(warp);
     float *sH = reinterpret_cast<float *>(sm + L::W);
     for (int h = 0; h < DV / 64; ++h) {
+#pragma unroll
       for (int i = tid; i < DK * 32; i += NTL) {   // float2 pairs of the half
         const int r = i >> 5, c2 = i & 31;
         *reinterpret_cast<float2 *>(sH + r * L::LDH + 2 * c2) =
@@ -804,6 +809,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       __syncthreads();   // dP has read E
       float *sH = reinterpret_cast<float *>(sm + L::E);
       for (int h = 0; h < DV / 64; ++h) {
+#pragma unroll
         for (int i = tid; i < DK * 32; i += NTL) {
           const int r = i >> 5, c2 = i & 31;
           *reinterpret_cast<float2 *>(sH + r * L::LDH + 2 * c2) =
@@ -979,6 +985,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     if constexpr (CHAN) {   // per state row: DV / 4 lanes a row, every thread the same number of rows
       constexpr int GL = DV / 4;
       static_assert((DK * DV / 4) % NTL == 0 && 32 % GL == 0, "row groups");
+#pragma unroll 4
       for (int i = tid; i < DK * DV / 4; i += NTL) {
         const float4 x = __ldg(a + i), y = __ldg(bb + i);
         float ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
@@ -988,6 +995,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       }
     } else {
       float ss = 0.f;
+#pragma unroll
       for (int i = tid; i < DK * DV / 4; i += NTL) {
         const float4 x = __ldg(a + i), y = __ldg(bb + i);
         ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
