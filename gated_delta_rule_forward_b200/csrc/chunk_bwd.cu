@@ -204,6 +204,14 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], const MA a, const MB b,
   }
 }
 
+// One tf32 pass, for the products whose rounding the gradients absorb (see
+// bwd_local_kernel).
+template <int NT, bool NEG, typename MA, typename MB>
+__device__ __forceinline__ void wmm1(float (&acc)[NT][4], const MA a, const MB b, int K, int m0, int n0, int lane,
+                                     const float *ks = nullptr) {
+  wmm<NT, NEG, MA, MB, false>(acc, a, b, K, m0, n0, lane, ks);
+}
+
 // f(row, col, value) for each accumulator element of a warp tile; each_je
 // also passes the fragment indices (j, e), compile-time constants after
 // unrolling, for per-column register arrays.
@@ -473,6 +481,15 @@ struct LocalSmem {
 //     dbeta = rowsum(V o T^T dE) + rowsum((K o e) o T^T dW) + rowsum(dA o G~)
 //     dg = dq o Q + (Y1 - X1 - Y2) o K, plus sum_t (X1 o K)_t + e^(gamma_C) o rowsum(dS o S0)
 //     at the chunk's last token; dlog_g = per-channel suffix sums of dg over the chunk.
+//
+// Precision: fp32 operands are split into two tf32 parts (wmm) except in the
+// products that take one pass (wmm1): dT, X = dT T^T and dA; KDA's factored
+// Gram and P products; and, with scalar decay, the dk and dq products with N1
+// and N2.  Measured against the fp64 oracle (the 350M layer and small ragged
+// and strong-decay cases of every variant), this moved no gradient past 5e-3
+// of its RMS (d log g 6.0e-3 -> 5.8e-3, dk 2.3e-3 -> 4.8e-3); one pass for
+// E, dW or the dE, U', W products moved d log g to 1.5-2.9e-2, and KDA's dk
+// products at one pass 2.6e-2.
 constexpr int NTL = 512;
 template <int DV, bool CHAN>
 __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) {
@@ -665,7 +682,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     float g[CC::NT][4];
     zero(g);
     if constexpr (CHAN) {
-      wmm<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
+      wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
     }
@@ -719,7 +736,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     float gq[CC::NT][4];
     zero(gq);
     if constexpr (CHAN) {
-      wmm<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
+      wmm1<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(gq, BK{sQ, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
     }
@@ -884,11 +901,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     float a1[CC::NT][4], a2[CC::NT][4];
     zero(a1);
     zero(a2);
-    wmm<CC::NT, false>(a1, F{sdE, LDF}, vmT(), DV, mc, nc, lane);
+    wmm1<CC::NT, false>(a1, F{sdE, LDF}, vmT(), DV, mc, nc, lane);
     if constexpr (CHAN) {
-      wmm<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
+      wmm1<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
     } else {
-      wmm<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
+      wmm1<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
     }
 #pragma unroll
     for (int j = 0; j < CC::NT; ++j)
@@ -903,14 +920,14 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
+    wmm1<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sE[t * LDC + r] = x; });
   }
   __syncthreads();
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    wmm1<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = r < t ? x : 0.f; });
   }
   __syncthreads();
@@ -919,7 +936,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     float g[CC::NT][4];
     zero(g);
     if constexpr (CHAN) {
-      wmm<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
+      wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
     }
@@ -946,7 +963,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     if constexpr (CHAN) {
       wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
     } else {
-      wmm<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
+      wmm1<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
     }
     each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
       if constexpr (CHAN) x *= ex2(sgam[t * LDG + i] - sgm[i]);
@@ -958,8 +975,8 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
       wmm<KC::NT, false>(acc, qaT(), F{sP, LDC}, C, mt, nt, lane);
     } else {
-      wmm<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
-      wmm<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
+      wmm1<KC::NT, false>(acc, BKT{sK, LDB}, F{sA, LD}, C, mt, nt, lane);
+      wmm1<KC::NT, false>(acc, BKT{sQ, LDB}, F{sP, LDC}, C, mt, nt, lane);
     }
     each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
       if constexpr (CHAN) x *= ex2(sgm[i] - sgam[t * LDG + i]);
@@ -975,7 +992,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     each_je(acc, mt, nt, lane,
             [&](int j, int e, int i, int t, float &x) { dqT[j][e] += x * ex2(sgam[t * LDG + i] - sgm[i]); });
   } else {
-    wmm<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
+    wmm1<KC::NT, false>(dqT, BKT{sK, LDB}, FT{sP, LDC}, C, mt, nt, lane);
   }
   each_je(dqT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) { add_dg(j, e, x * qat(t, i)); });
 
