@@ -280,7 +280,16 @@ __global__ void bwd_absmax_kernel(const __nv_bfloat16 *d_o, size_t n_o, const fl
       m = fmaxf(m, fabsf(__ldg(d_final + i)));
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));   // non-negative floats order as integers
+  // one atomic per block (not per warp): thousands of atomics on one word serialise
+  __shared__ float wmax[32];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? wmax[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) atomicMax(out, __float_as_uint(m));   // non-negative floats order as integers
+  }
 }
 
 __global__ void bwd_scale_state_kernel(const float *d_final, size_t n, const uint32_t *absmax, float *x0) {
@@ -1140,8 +1149,10 @@ cudaError_t gdr_bwd_launch_scale(const gdr::BwdProblem &p, uint32_t *absmax, flo
   cudaError_t e = cudaMemsetAsync(absmax, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   const size_t n_o = static_cast<size_t>(f.B) * f.T * f.H * f.dv, n_s = static_cast<size_t>(f.B) * f.H * f.dk * f.dv;
-  bwd_absmax_kernel<<<grid_for(std::max(n_o, n_s)), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(p.d_o), n_o,
-                                                                  p.d_final, n_s, absmax);
+  // a grid-stride sweep of 16-byte loads (d_o) and floats (d_final), one atomic per block
+  const int grid = static_cast<int>(std::min<size_t>((std::max(n_o / 8, n_s) + 255) / 256, 1024));
+  bwd_absmax_kernel<<<std::max(grid, 1), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(p.d_o), n_o, p.d_final,
+                                                      n_s, absmax);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_scale_state_kernel<<<grid_for(n_s), 256, 0, s>>>(p.d_final, n_s, absmax, x0);
   return cudaGetLastError();
