@@ -73,7 +73,7 @@ struct Mat {
   using elem = E;
   static constexpr bool kTr = TR;
   static constexpr bool kGlobal = GLOBAL;
-  static constexpr bool kExact = EXACT || std::is_same<E, __nv_bfloat16>::value;
+  static constexpr bool kExact = EXACT || std::is_same<E, __nv_bfloat16>::value || std::is_same<E, __half>::value;
   const E *p;
   int ld;
 };
@@ -86,6 +86,8 @@ template <>
 __device__ __forceinline__ float ld1<float, true>(const float *p) { return __ldg(p); }
 template <>
 __device__ __forceinline__ float ld1<__nv_bfloat16, false>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+template <>
+__device__ __forceinline__ float ld1<__half, false>(const __half *p) { return __half2float(*p); }
 
 template <typename V>
 __device__ __forceinline__ float at(const V &m, int r, int c) {
@@ -324,14 +326,20 @@ struct RevPrepParams {
 //     the state term <- F^T = (s dO)^T Qg.
 // The Qg slots, P and the output term stay unwritten: the reverse carry runs
 // without outputs and reads none of them.
+//
+// Every operand is exact in 16 bits (s dO in bf16, s a power of two; P and Qg
+// are the record's fp16), so the tiles stay 16-bit in shared memory (44 KB at
+// d_v = 128, three CTAs per SM) and one tf32 pass is exact per product; F^T is
+// taken in two 64-column halves, and both products go from the fragments
+// straight to the record.
 template <int DV>
-__global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams p) {
+__global__ void __launch_bounds__(NT, 3) bwd_rev_prep_kernel(const RevPrepParams p) {
   constexpr int NS = DV / 64;
-  constexpr int LDO = DV + 4, LDP = C + 4, LDQ = DK + 4;
+  constexpr int LDO = DV + 8, LDP = C + 8, LDQ = DK + 8;   // 16-bit rows, 16 bytes of padding
   extern __shared__ float4 smem_rev[];
-  float *sO = reinterpret_cast<float *>(smem_rev);   // [C][LDO] s dO, rows t
-  float *sP = sO + C * LDO;                          // [C][LDP] P, rows t
-  float *sQ = sP + C * LDP;                          // [C][LDQ] Qg, rows t
+  __nv_bfloat16 *sO = reinterpret_cast<__nv_bfloat16 *>(smem_rev);   // [C][LDO] s dO, rows t
+  __half *sP = reinterpret_cast<__half *>(sO + C * LDO);               // [C][LDP] P, rows t
+  __half *sQ = sP + C * LDP;                                           // [C][LDQ] Qg, rows t
   const int tid = threadIdx.x;
   const int r = blockIdx.x;
   const int bh = r / p.NC, c = r - bh * p.NC;
@@ -340,6 +348,7 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
   uint8_t *dst = p.rev + (static_cast<size_t>(bh) * p.NC + (p.NC - 1 - c)) * p.rb_r;
   const float s = grad_scale(p.absmax);
 
+#pragma unroll
   for (int i = tid; i < C * DV / 8; i += NT) {
     const int t = i / (DV / 8), v8 = (i % (DV / 8)) * 8;
     const int tg = c * C + t;
@@ -348,29 +357,19 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
       unpack8(__ldg(reinterpret_cast<const uint4 *>(p.d_o + ((static_cast<size_t>(b) * p.T + tg) * p.H + h) * DV + v8)),
               x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sO[t * LDO + v8 + e] = s * x[e];
+    for (int e = 0; e < 8; ++e) x[e] *= s;
+    st_chunk_bf16(reinterpret_cast<uint8_t *>(sO + t * LDO + v8), x);
   }
-  for (int i = tid; i < C * C / 8; i += NT) {
+#pragma unroll
+  for (int i = tid; i < C * C / 8; i += NT) {   // P: the record's swizzled rows, 16 bytes at a time
     const int t = i >> 3, j = i & 7;
-    const uint4 u = *reinterpret_cast<const uint4 *>(src + REC_P + sw128(t, j));
-    const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(hp[e]);
-      sP[t * LDP + 8 * j + 2 * e] = f.x;
-      sP[t * LDP + 8 * j + 2 * e + 1] = f.y;
-    }
+    *reinterpret_cast<uint4 *>(sP + t * LDP + 8 * j) = *reinterpret_cast<const uint4 *>(src + REC_P + sw128(t, j));
   }
-  for (int i = tid; i < C * DK / 8; i += NT) {
-    const int t = i >> 4, a = (i >> 3) & 1, j = i & 7;
-    const uint4 u = *reinterpret_cast<const uint4 *>(src + REC_WQ + a * 16384 + 8192 + sw128(t, j));
-    const __half2 *hp = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(hp[e]);
-      sQ[t * LDQ + 64 * a + 8 * j + 2 * e] = f.x;
-      sQ[t * LDQ + 64 * a + 8 * j + 2 * e + 1] = f.y;
-    }
+  for (int i = tid; i < C * DK / 8; i += NT) {   // Qg: two 64-channel atoms
+    const int t = i >> 4, a = (i >> 3) & 1, j = i & 7;
+    *reinterpret_cast<uint4 *>(sQ + t * LDQ + 64 * a + 8 * j) =
+        *reinterpret_cast<const uint4 *>(src + REC_WQ + a * 16384 + 8192 + sw128(t, j));
   }
   // tile copies (16-byte units)
   for (int i = tid; i < 1024; i += NT) {
@@ -388,43 +387,42 @@ __global__ void __launch_bounds__(NT, 2) bwd_rev_prep_kernel(const RevPrepParams
 
   const int warp = tid >> 5, lane = tid & 31;
   float vmax = 0.f;
-  // Both products are staged in shared memory as the record's byte images and
-  // written with 16-byte stores: R^T over P's tile once R is done, F^T over
-  // dO's tile once F is done.
-  uint8_t *stage_r = reinterpret_cast<uint8_t *>(sP);
-  __half *stage_f = reinterpret_cast<__half *>(sO);
+  using TL = Tiling<DV, 64>;
+  const int m0 = TL::m0(warp), n0 = TL::n0(warp);
+  using OT = Mat<__nv_bfloat16, true>;
+  using HM = Mat<__half, false>;
   {   // R^T [v][t]: the U' slot's rows v, 128-byte swizzled
-    using TL = Tiling<DV, C>;
     float acc[TL::NT][4];
     zero(acc);
-    const int m0 = TL::m0(warp), n0 = TL::n0(warp);
-    wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
-                                                                   Mat<float, false>{sP, LDP}, C, m0, n0, lane);
-    __syncthreads();   // every warp has read P
-    each(acc, m0, n0, lane, [&](int v, int t, float &x) {
-      vmax = fmaxf(vmax, fabsf(x));
-      *reinterpret_cast<__half *>(stage_r + sw128(v, t >> 3) + (t & 7) * 2) = __float2half_rn(x);
-    });
+    wmm<TL::NT, false, OT, HM, false>(acc, OT{sO, LDO}, HM{sP, LDP}, C, m0, n0, lane);
+    const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int j = 0; j < TL::NT; ++j)
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {   // two adjacent tokens per 4-byte store
+        const int v = m0 + g + 8 * h2, t = n0 + 8 * j + 2 * tq;
+        const float x0 = acc[j][2 * h2], x1 = acc[j][2 * h2 + 1];
+        vmax = fmaxf(vmax, fmaxf(fabsf(x0), fabsf(x1)));
+        *reinterpret_cast<uint32_t *>(dst + REC_U + sw128(v, t >> 3) + (t & 7) * 2) = pack_f16x2(x0, x1);
+      }
   }
-  {   // F^T [v][i]: unswizzled rows of d_k values after the output term
-    using TL = Tiling<DV, DK>;
+  uint8_t *fdst = dst + rec_bytes_chan(NS) + 8192 * NS;   // F^T [v][i]: unswizzled rows of d_k values
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
     float acc[TL::NT][4];
     zero(acc);
-    const int m0 = TL::m0(warp), n0 = TL::n0(warp);
-    wmm<TL::NT, false, Mat<float, true>, Mat<float, false>, false>(acc, Mat<float, true>{sO, LDO},
-                                                                   Mat<float, false>{sQ, LDQ}, C, m0, n0, lane);
-    __syncthreads();   // every warp has read dO
-    each(acc, m0, n0, lane, [&](int v, int i, float &x) {
-      vmax = fmaxf(vmax, fabsf(x));
-      stage_f[v * DK + i] = __float2half_rn(x);
-    });
+    wmm<TL::NT, false, OT, HM, false>(acc, OT{sO, LDO}, HM{sQ + 64 * hh, LDQ}, C, m0, n0, lane);
+    const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int j = 0; j < TL::NT; ++j)
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int v = m0 + g + 8 * h2, i = 64 * hh + n0 + 8 * j + 2 * tq;
+        const float x0 = acc[j][2 * h2], x1 = acc[j][2 * h2 + 1];
+        vmax = fmaxf(vmax, fmaxf(fabsf(x0), fabsf(x1)));
+        *reinterpret_cast<uint32_t *>(fdst + (v * DK + i) * 2) = pack_f16x2(x0, x1);
+      }
   }
-  __syncthreads();
-  for (int i = tid; i < DV * 128 / 16; i += NT)
-    *reinterpret_cast<uint4 *>(dst + REC_U + 16 * i) = *reinterpret_cast<const uint4 *>(stage_r + 16 * i);
-  for (int i = tid; i < DV * DK * 2 / 16; i += NT)
-    *reinterpret_cast<uint4 *>(dst + rec_bytes_chan(NS) + 8192 * NS + 16 * i) =
-        *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(stage_f) + 16 * i);
   if (vmax > F16_SAFE_BWD) atomicOr(&g_gdr_bwd_error, 2);
 }
 
@@ -1172,7 +1170,7 @@ cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd
   rp.fwd = fwd_rec; rp.rev = rev_rec; rp.absmax = absmax;
   const int grid = f.B * f.H * rp.NC;
   auto run = [&](auto kern, int dv) {
-    const size_t smem = (static_cast<size_t>(C) * (dv + 4) + C * (C + 4) + C * (DK + 4)) * 4;
+    const size_t smem = (static_cast<size_t>(C) * (dv + 8) + C * (C + 8) + C * (DK + 8)) * 2;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<grid, NT, smem, s>>>(rp);
