@@ -433,7 +433,9 @@ struct LocalParams {
   float eps, scale;
   const __nv_bfloat16 *q, *k, *v, *d_o;
   const float *beta, *log_g;   // log_g [B,T,H], or [B,T,H,d_k] with channel decay
-  const float *s0s, *dss;   // chunk start states and end-state gradients (the latter in reverse chunk order)
+  const void *s0s;          // chunk start states: fp16 as the forward carry's MMAs take them
+                            // (scalar decay), fp32 (channel decay)
+  const float *dss;         // (scaled) end-state gradients in reverse chunk order
   const uint32_t *absmax;
   __nv_bfloat16 *dq, *dk, *dv;
   float *dbeta, *dlog_g;    // dlog_g laid out as log_g
@@ -449,7 +451,9 @@ struct LocalSmem {
   static constexpr int LDF = DV + 4;    // fp32 rows of dE, E
   static constexpr int LDW = DK + 4;    // fp32 rows of W
   static constexpr int LDC = C + 4;     // fp32 rows of C-wide tiles (dW^T, X, dP)
-  static constexpr int LDH = 66;        // fp32 rows of a 64-column half of S0 or dS
+  static constexpr int LDS = DV + 8;    // fp16 rows of S0 (over dE, A, P)
+  static constexpr int LDSE = DV + 4;   // fp16 rows of S0's second staging (over E)
+  static constexpr int LDH = 66;        // fp32 rows of a 64-column half of dS (over W) or of S0 (over E)
   static constexpr size_t K = 0;
   static constexpr size_t Q = K + C * LDB * 2;
   static constexpr size_t V = Q + (kQVGlobal ? 0 : C * LDB * 2);
@@ -466,7 +470,8 @@ struct LocalSmem {
   static_assert(BYTES <= 232448 && GAM % 16 == 0, "shared memory");
   static_assert(A + C * LD * 4 + C * LDC * 4 - DE >= static_cast<size_t>(DK) * LDF * 4, "S0 staging over dE, A, P");
   static_assert(std::max(C * LDW, DK * LDC) >= DK * LDH, "a half of dS over W");
-  static constexpr bool kS0HalvesOverE = std::max(C * LDF, C * LDC) >= DK * LDH;   // d_v = 128
+  static_assert(std::max(C * LDF, C * LDC) * 4 >= DK * LDSE * 2, "S0 (fp16) over E");
+  static constexpr bool kS0HalvesOverE = std::max(C * LDF, C * LDC) >= DK * LDH;   // fp32 S0: d_v = 128
 };
 
 // One CTA of NTL threads per chunk (b, h, c): sixteen warps share each
@@ -536,7 +541,10 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   const int t0 = c * C, n = min(C, p.T - t0);
   const float s = grad_scale(p.absmax), inv_s = 1.f / s;
   const size_t rc = static_cast<size_t>(bh) * p.NC + (p.NC - 1 - c);   // reverse-order index of this chunk
-  const float *S0 = p.s0s + static_cast<size_t>(blockIdx.x) * DK * DV;
+  // S0 in fp16 with scalar decay; in fp32 with channel decay, whose d log g its fp16
+  // rounding would move to ~2e-2 of RMS on long sequences
+  using S0E = std::conditional_t<CHAN, float, __half>;
+  const S0E *S0 = static_cast<const S0E *>(p.s0s) + static_cast<size_t>(blockIdx.x) * DK * DV;
   const float *dS = p.dss + rc * DK * DV;
   auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
 
@@ -653,7 +661,8 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   using BKT = Mat<__nv_bfloat16, true>;   // ... transposed
   using F = Mat<float, false>;
   using FT = Mat<float, true>;
-  using FG = Mat<float, false, true>;     // a global fp32 matrix (S0, dS)
+  using HS = Mat<__half, false>;          // an fp16 tile (S0)
+  using FG = Mat<float, false, true>;     // a global fp32 matrix (S0)
   using TX = Mat<float, false, false, true>;   // T (tf32 values from the solve)
   using TXT = Mat<float, true, false, true>;   // ... transposed
   // channel decay: K o 2^(sg (gamma - ref)) and Q o a, V as stored or read from global memory
@@ -722,18 +731,32 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   }
   // S0 through shared memory (over dE, A and P, none of which holds data yet):
   // E = U' - W S0 and dq's first part, scale Diag(e) dO S0^T
-  float *sS = reinterpret_cast<float *>(sm + L::DE);
-#pragma unroll
-  for (int i = tid; i < DK * DV / 4; i += NTL) {
-    const int r = i / (DV / 4), c4 = i % (DV / 4);
-    *reinterpret_cast<float4 *>(sS + r * LDF + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(S0) + i);
-  }
-  __syncthreads();
-  wmm<CV::NT, true>(ue, F{sW, LDW}, F{sS, LDF}, DK, mv, nv, lane);
-  each(ue, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
   float dqT[KC::NT][4];
-  zero(dqT);
-  wmm<KC::NT, false>(dqT, F{sS, LDF}, BKT{sO, LDBV}, DV, mt, nt, lane);
+  if constexpr (CHAN) {
+    float *sS = reinterpret_cast<float *>(sm + L::DE);
+#pragma unroll
+    for (int i = tid; i < DK * DV / 4; i += NTL) {
+      const int r = i / (DV / 4), c4 = i % (DV / 4);
+      *reinterpret_cast<float4 *>(sS + r * LDF + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(S0) + i);
+    }
+    __syncthreads();
+    wmm<CV::NT, true>(ue, F{sW, LDW}, F{sS, LDF}, DK, mv, nv, lane);
+    each(ue, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
+    zero(dqT);
+    wmm<KC::NT, false>(dqT, F{sS, LDF}, BKT{sO, LDBV}, DV, mt, nt, lane);
+  } else {
+    __half *sS = reinterpret_cast<__half *>(sm + L::DE);
+#pragma unroll
+    for (int i = tid; i < DK * DV / 8; i += NTL) {
+      const int r = i / (DV / 8), c8 = i % (DV / 8);
+      *reinterpret_cast<uint4 *>(sS + r * L::LDS + 8 * c8) = __ldg(reinterpret_cast<const uint4 *>(S0) + i);
+    }
+    __syncthreads();
+    wmm<CV::NT, true>(ue, F{sW, LDW}, HS{sS, L::LDS}, DK, mv, nv, lane);
+    each(ue, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
+    zero(dqT);
+    wmm<KC::NT, false>(dqT, HS{sS, L::LDS}, BKT{sO, LDBV}, DV, mt, nt, lane);
+  }
   each(dqT, mt, nt, lane, [&](int i, int t, float &x) { x *= p.scale * (CHAN ? ex2(sgam[t * LDG + i]) : see[t]); });
   __syncthreads();   // S0's staging is read: P may overwrite it
   // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
@@ -794,7 +817,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       wmm<CH::NT, false>(acc, FT{sP, LDC}, BK{sO + 64 * h, LDBV}, C, mh, nh, lane);
       each(acc, mh, nh, lane, [&](int t, int v, float &x) { sdE[t * LDF + 64 * h + v] = x; });
       wmm<KC::NT, false>(dkT, F{sH, L::LDH}, FT{sE + 64 * h, LDF}, 64, mt, nt, lane);
-      __syncthreads();   // the half is read before the next one lands
+      __syncthreads();   // the half is read before the next one (or dW^T) lands over it
     }
   }
   {
@@ -824,12 +847,24 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     wmm<CC::NT, false>(acc, BK{sO, LDBV}, FT{sE, LDF}, DV, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sP[t * LDC + r] = r <= t ? x : 0.f; });
   }
-  // ---- dW^T = -S0 dE^T  (d_k x C, over W); at d_v = 128 with S0 through shared
-  // memory in halves, over E once dP has read it
+  // ---- dW^T = -S0 dE^T  (d_k x C, over W), S0 through shared memory again, over
+  // E once dP has read it (fp32 S0: in halves at d_v = 128, else from global memory)
   {
     float acc[KC::NT][4];
     zero(acc);
-    if constexpr (L::kS0HalvesOverE) {
+    if constexpr (!CHAN) {
+      __syncthreads();   // dP has read E
+      __half *sH = reinterpret_cast<__half *>(sm + L::E);
+#pragma unroll
+      for (int i = tid; i < DK * DV / 8; i += NTL) {
+        const int r = i / (DV / 8), c8 = i % (DV / 8);
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(S0) + i);   // rows of LDSE halves: 8-byte aligned
+        *reinterpret_cast<uint2 *>(sH + r * L::LDSE + 8 * c8) = make_uint2(u.x, u.y);
+        *reinterpret_cast<uint2 *>(sH + r * L::LDSE + 8 * c8 + 4) = make_uint2(u.z, u.w);
+      }
+      __syncthreads();
+      wmm<KC::NT, true>(acc, HS{sH, L::LDSE}, FT{sdE, LDF}, DV, mt, nt, lane);
+    } else if constexpr (L::kS0HalvesOverE) {
       __syncthreads();   // dP has read E
       float *sH = reinterpret_cast<float *>(sm + L::E);
       for (int h = 0; h < DV / 64; ++h) {
@@ -844,7 +879,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
         __syncthreads();
       }
     } else {
-      wmm<KC::NT, true>(acc, FG{S0, DV}, FT{sdE, LDF}, DV, mt, nt, lane);
+      wmm<KC::NT, true>(acc, FG{reinterpret_cast<const float *>(S0), DV}, FT{sdE, LDF}, DV, mt, nt, lane);
     }
     each(acc, mt, nt, lane, [&](int i, int t, float &x) { sW[i * LDC + t] = x; });
   }
@@ -1005,8 +1040,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
 
   // ---- reductions: dg_t over the rows; sum(X1 o K); sum(dS o S0)
   {
-    const float4 *a = reinterpret_cast<const float4 *>(dS), *bb = reinterpret_cast<const float4 *>(S0);
-    if constexpr (CHAN) {   // per state row: DV / 4 lanes a row, every thread the same number of rows
+    const float4 *a = reinterpret_cast<const float4 *>(dS);
+    if constexpr (CHAN) {   // per state row (fp32 S0): DV / 4 lanes a row, every thread the same number of rows
+      const float4 *bb = reinterpret_cast<const float4 *>(S0);
       constexpr int GL = DV / 4;
       static_assert((DK * DV / 4) % NTL == 0 && 32 % GL == 0, "row groups");
 #pragma unroll 4
@@ -1017,12 +1053,18 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
         for (int o = GL / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (lane % GL == 0) sss[i / GL] = ss;
       }
-    } else {
+    } else {   // fp16 S0: eight products at a time
+      const uint4 *bb = reinterpret_cast<const uint4 *>(S0);
       float ss = 0.f;
 #pragma unroll
-      for (int i = tid; i < DK * DV / 4; i += NTL) {
-        const float4 x = __ldg(a + i), y = __ldg(bb + i);
-        ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
+      for (int i = tid; i < DK * DV / 8; i += NTL) {
+        const float4 x0 = __ldg(a + 2 * i), x1 = __ldg(a + 2 * i + 1);
+        const uint4 w = __ldg(bb + i);
+        const __half2 *y = reinterpret_cast<const __half2 *>(&w);
+        const float2 y0 = __half22float2(y[0]), y1 = __half22float2(y[1]), y2 = __half22float2(y[2]),
+                     y3 = __half22float2(y[3]);
+        ss = fmaf(x0.x, y0.x, fmaf(x0.y, y0.y, fmaf(x0.z, y1.x, fmaf(x0.w, y1.y, ss))));
+        ss = fmaf(x1.x, y2.x, fmaf(x1.y, y2.y, fmaf(x1.z, y3.x, fmaf(x1.w, y3.y, ss))));
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) {
@@ -1119,7 +1161,7 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
   L.fwd_rec = 0;
   L.rev_rec = up(bh * NC * rb_f);
   L.s0s = L.rev_rec + up(bh * NC * rec_bytes_gdn2(static_cast<int>(ns)));
-  L.dss = L.s0s + up(bh * NC * DK * dv * 4);
+  L.dss = L.s0s + up(bh * NC * DK * dv * (variant == kKDA ? 4 : 2));   // S0: fp32 with channel decay
   L.x0 = L.dss + up(bh * NC * DK * dv * 4);
   L.xf = L.x0 + up(bh * DK * dv * 4);
   L.maps = L.xf + up(bh * DK * dv * 4);
@@ -1179,7 +1221,7 @@ cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd
   return f.dv == 128 ? run(bwd_rev_prep_kernel<128>, 128) : run(bwd_rev_prep_kernel<64>, 64);
 }
 
-cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const float *s0s, const float *dss,
+cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, const float *dss,
                                  const uint32_t *absmax, cudaStream_t s) {
   using namespace gdr::tc;
   const gdr::FwdProblem &f = p.f;

@@ -4,6 +4,7 @@
 #pragma once
 #include <cstdint>
 #include <string>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -23,8 +24,8 @@ struct BwdProblem {
 struct BwdLayout {
   size_t fwd_rec;   // the forward's per-chunk records
   size_t rev_rec;   // the reverse carry's records, chunks in reverse order
-  size_t s0s;       // fp32 start state of every chunk        [B,H,NC,dk,dv]
-  size_t dss;       // fp32 end-state gradient, reverse order [B,H,NC,dk,dv]
+  size_t s0s;       // start state of every chunk   [B,H,NC,dk,dv] fp16 (KDA: fp32)
+  size_t dss;       // end-state gradient (scaled), reverse chunk order [B,H,NC,dk,dv] fp32
   size_t x0, xf;    // reverse carry's start (scaled d_final) and end (scaled d_s0) [B,H,dk,dv]
   size_t maps, maps_bytes;   // the segmented carries' maps and start states (0 bytes: unsegmented)
   size_t absmax;    // the gradients' magnitude (one fp32 word)
@@ -44,7 +45,7 @@ size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv);
 cudaError_t gdr_bwd_launch_scale(const gdr::BwdProblem &p, uint32_t *absmax, float *x0, cudaStream_t s);
 cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd_rec, uint8_t *rev_rec,
                                     const uint32_t *absmax, cudaStream_t s);
-cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const float *s0s, const float *dss,
+cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, const float *dss,
                                   const uint32_t *absmax, cudaStream_t s);
 cudaError_t gdr_bwd_launch_unscale(const gdr::BwdProblem &p, const float *xf, const uint32_t *absmax,
                                    cudaStream_t s);

@@ -1383,7 +1383,8 @@ enum CarryFlags : int {
   CARRY_LAST_FINAL = 8,   // only the last segment writes s_final
   CARRY_S0_FIRST = 16,    // only segment 0 starts from s0, the others from zero
   CARRY_FAULT_MISSING_COPY = 32,   // host fault injection (see the issuer's prologue)
-  CARRY_WRITE_STATES = 64,   // write every chunk's start state to `states` (fp32 [B,H,NC,d_k,d_v])
+  CARRY_WRITE_STATES = 64,   // write every chunk's start state to `states` ([B,H,NC,d_k,d_v], fp32)
+  CARRY_STATES_F16 = 128,    // ... in fp16 instead: the state as this kernel's MMAs take it
 };
 
 struct CarryParams {
@@ -1402,7 +1403,7 @@ struct CarryParams {
   float *s_final_b;
   size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
-  float *states;   // CARRY_WRITE_STATES output, indexed by (b, h, chunk)
+  void *states;    // CARRY_WRITE_STATES output, indexed by (b, h, chunk)
 };
 
 // max |x_i| over 16 values as a tree (four levels instead of a chain of 16).
@@ -1668,10 +1669,17 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
     for (int c = 0; c < NC; ++c) {
       uint8_t *st = sm + (c % NSTAGE) * STAGE;
       const uint32_t y = lrow + COL_Y + 128 * (c & 1);
-      if ((flags & CARRY_WRITE_STATES) && has_v) {   // S (fp32) at the chunk's start: rows 32 part .., column v
-        float *dst = p.states + ((chunk0 + c) * DK + 32 * part) * p.dv + v;
+      if ((flags & CARRY_WRITE_STATES) && has_v) {   // S at the chunk's start: rows 32 part .., column v
+        const size_t at = ((chunk0 + c) * DK + 32 * part) * p.dv + v;
+        if (flags & CARRY_STATES_F16) {
+          __half *dst = static_cast<__half *>(p.states) + at;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
+          for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = __float2half_rn(S[k]);
+        } else {
+          float *dst = static_cast<float *>(p.states) + at;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
+        }
       }
 
       // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15; U'^T is read from the
@@ -2050,7 +2058,7 @@ struct CarryLaunch {
   int segments_b = 0, seg_first_b = 0, flags_b = 0;
   float *s_final_b = nullptr;
   size_t s_final_b_stride = 0;
-  float *states = nullptr;   // CARRY_WRITE_STATES output
+  void *states = nullptr;    // CARRY_WRITE_STATES output
 };
 
 // `pdl`: launched with programmatic stream serialization, so that its CTAs may
@@ -2239,7 +2247,7 @@ cudaError_t launch_pipelined(const FwdProblem &p, int NC, uint8_t *w, const Pipe
 // with outputs; the backward's carries: no outputs, chunk states kept).
 template <int MODE>
 cudaError_t launch_segmented(const FwdProblem &p, int NC, const SegPlan &sp, const uint8_t *records, uint8_t *maps,
-                             const float *s0, float *s_final, int flags2, float *states, cudaStream_t stream,
+                             const float *s0, float *s_final, int flags2, void *states, cudaStream_t stream,
                              std::string *err) {
   const size_t bh = static_cast<size_t>(p.B) * p.H;
   float *Mb = reinterpret_cast<float *>(maps);
@@ -2312,7 +2320,12 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
   const FwdProblem &p = bp.f;
   const int NC = (p.T + C - 1) / C;
   const BwdLayout L = bwd_layout(VAR, p.B, p.T, p.H, p.dv);
-  float *s0s = reinterpret_cast<float *>(w + L.s0s), *dss = reinterpret_cast<float *>(w + L.dss);
+  // chunk start states in fp16 (the forward carry's own operand) for scalar decay, in fp32 for
+  // channel decay; the reverse carry's states, whose fp16 rounding the gate gradients do not
+  // absorb, in fp32
+  void *s0s = w + L.s0s;
+  float *dss = reinterpret_cast<float *>(w + L.dss);
+  const int s0_f16 = MODE == 1 ? 0 : CARRY_STATES_F16;
   float *x0 = reinterpret_cast<float *>(w + L.x0), *xf = reinterpret_cast<float *>(w + L.xf);
   uint32_t *absmax = reinterpret_cast<uint32_t *>(w + L.absmax);
   const SegPlan sp = L.maps_bytes > 0 ? seg_plan(p.B, p.H, p.dv, NC) : SegPlan{1, NC};
@@ -2320,11 +2333,11 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
   if (e != cudaSuccess) return e;
   if (sp.G > 1) {
     e = launch_segmented<MODE>(p, NC, sp, w + L.fwd_rec, w + L.maps, p.s0, nullptr,
-                               CARRY_NO_OUTPUT | CARRY_WRITE_STATES, s0s, stream, err);
+                               CARRY_NO_OUTPUT | CARRY_WRITE_STATES | s0_f16, s0s, stream, err);
   } else {
     CarryLaunch lf;
     lf.seg_len = NC;
-    lf.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES;
+    lf.flags = CARRY_NO_OUTPUT | CARRY_WRITE_STATES | s0_f16;
     lf.s0 = p.s0;
     lf.states = s0s;
     e = launch_carry<MODE>(p, NC, w + L.fwd_rec, lf, true, stream, err);

@@ -230,8 +230,8 @@ typedef struct {
 /*
  * Bytes of device workspace gdr_backward needs (0 for a case it does not
  * cover): the forward's records, the reverse carry's records (B * H *
- * ceil(T/64) of each), every chunk's start state and end-state gradient
- * (fp32, dk * dv each), plus two states; for few long sequences (where the
+ * ceil(T/64) of each), every chunk's start state (dk * dv, fp16; fp32 for
+ * KDA) and end-state gradient (dk * dv, fp32), plus two states; for few long sequences (where the
  * forward's carry runs in segments) also the segment maps and start states
  * its two carries share.  The segmenting reads the current device's SM
  * count, so query the size on the device that runs the call.

@@ -266,7 +266,9 @@ def test_backward_workspace_sizes(L):
     B, T, H, NC, bh = 8, 2048, 8, 32, 64
     rec, rev = 57344 + 8192 * 2 + 16, 57344 + 8192 * 2 + 512 + 24576 * 2
     up = lambda x: (x + 255) // 256 * 256
-    want = up(bh * NC * rec) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
+    # chunk start states in fp16 (fp32 for KDA), end-state gradients in fp32
+    want = up(bh * NC * rec) + up(bh * NC * rev) + up(bh * NC * 128 * 128 * 2) + up(bh * NC * 128 * 128 * 4) + \
+        2 * up(bh * 128 * 128 * 4) + 256
     assert L.gdr_backward_workspace_size(1, 1, B, T, H, 128, 128) == want
     rec_kda = rec + 512 - 16                                                 # Gamma_C as 128 floats
     want_kda = up(bh * NC * rec_kda) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
