@@ -565,3 +565,115 @@ def test_channel_backward_as_built_matches_the_oracle(T):
                                                        dOn[sl], scale)
         for name, x in (("q", dq), ("k", dkk), ("v", dvv), ("beta", db), ("log_g", dlg)):
             np.testing.assert_allclose(x, g_ref[name][0, sl, 0], rtol=0, atol=1e-10, err_msg=name)
+
+
+def gdn2_local_as_built(K, Q, V, eb, ww, lg, S0, dS, dO, scale):
+    """GDN-2's chunk-local gradients in the form a chunk-parallel kernel computes
+    them (one chunk; eb, ww, lg [n, dk] the erase gate, write gate and log decay;
+    S0 the chunk's start state, dS its end-state gradient).  With a = eb o k,
+    d = (ww - eb) o k, the factors a_ = e^(g - g_m), bb = e^(g_m - g), e = e^g,
+    f = e^(g_C - g) (middle token m as for KDA), and the factored operands
+    Ka = K o a_, Qa = Q o a_, Ab = a o bb, Db = d o bb, Ke = K o e, Af = a o f,
+    Df = d o f:
+        A = tril(Ka Ab^T, -1),  A^d = tril(Ka Db^T, -1),  T = (I + A)^-1
+        Y = V - A^d V,  W = T Ke,  E = T Y - W S0
+        P^a = scale tril(Qa Ab^T),  P^d = scale tril(Qa Db^T)
+        dE = Af dS + P^a^T dO,  dW = -dE S0^T,  tU = T^T dE,  tW = T^T dW
+        dT = dE Y^T + dW Ke^T,  dA = tril(-T^T dT T^T, -1),  dA^d = -tril(tU V^T, -1)
+        N2a = scale tril(dO E^T),  N2d = scale tril(dO V^T)
+        dv = tU - A^d^T tU + P^d^T dO + Df dS
+        dKa = dA Ab + dA^d Db,  dAb = dA^T Ka + N2a^T Qa,  dDb = dA^d^T Ka + N2d^T Qa
+        dQa = N2a Ab + N2d Db,  dKe = tW,  dQe = scale dO S0^T,  dAf = E dS^T,  dDf = V dS^T
+        dq = a_ o dQa + e o dQe,  da = bb o dAb + f o dAf,  dd = bb o dDb + f o dDf
+        dk = a_ o dKa + e o dKe + eb o da + (ww - eb) o dd
+        d eb = k o (da - dd),  d ww = k o dd
+        dg = dKa o Ka + dQa o Qa - dAb o Ab - dDb o Db + dKe o Ke + dQe o (Q o e)
+             - dAf o Af - dDf o Df, plus colsum(dAf o Af + dDf o Df) + e^(g_C) o rowsum(dS o S0)
+             at the chunk's last token; d log g = per-channel suffix sums of dg."""
+    n = K.shape[0]
+    g = np.cumsum(lg, axis=0)
+    m = min(C // 2 - 1, n - 1)
+    a_, bb = np.exp(g - g[m]), np.exp(g[m] - g)
+    e, f = np.exp(g), np.exp(g[-1] - g)
+    a, d = eb * K, (ww - eb) * K
+    Ka, Qa, Ab, Db, Ke, Af, Df = K * a_, Q * a_, a * bb, d * bb, K * e, a * f, d * f
+    A = np.tril(Ka @ Ab.T, -1)
+    Ad = np.tril(Ka @ Db.T, -1)
+    Tm = np.linalg.inv(np.eye(n) + A)
+    Y = V - Ad @ V
+    W = Tm @ Ke
+    E = Tm @ Y - W @ S0
+    Pa = scale * np.tril(Qa @ Ab.T)
+    Pd = scale * np.tril(Qa @ Db.T)
+    dE = Af @ dS + Pa.T @ dO
+    dW = -dE @ S0.T
+    tU, tW = Tm.T @ dE, Tm.T @ dW
+    dT = dE @ Y.T + dW @ Ke.T
+    dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+    dAd = -np.tril(tU @ V.T, -1)
+    N2a, N2d = scale * np.tril(dO @ E.T), scale * np.tril(dO @ V.T)
+    dv = tU - Ad.T @ tU + Pd.T @ dO + Df @ dS
+    dKa = dA @ Ab + dAd @ Db
+    dAb = dA.T @ Ka + N2a.T @ Qa
+    dDb = dAd.T @ Ka + N2d.T @ Qa
+    dQa = N2a @ Ab + N2d @ Db
+    dKe, dQe, dAf, dDf = tW, scale * dO @ S0.T, E @ dS.T, V @ dS.T
+    dq = a_ * dQa + e * dQe
+    da, dd = bb * dAb + f * dAf, bb * dDb + f * dDf
+    dk = a_ * dKa + e * dKe + eb * da + (ww - eb) * dd
+    deb, dww = K * (da - dd), K * dd
+    dg = (dKa * Ka + dQa * Qa - dAb * Ab - dDb * Db + dKe * Ke + dQe * (Q * e) - dAf * Af - dDf * Df)
+    dg[n - 1] += np.sum(dAf * Af + dDf * Df, 0) + np.exp(g[-1]) * np.sum(dS * S0, 1)
+    return dq, dk, dv, deb, dww, np.cumsum(dg[::-1], axis=0)[::-1]
+
+
+@pytest.mark.parametrize("T", [27, 29])
+def test_gdn2_backward_as_built_matches_the_oracle(T):
+    """GDN-2: the forward carry in chunk form (E the residual, the record's Ã = a o f),
+    the reverse carry dE = Ã dS + P^a^T dO, dS0 = Diag(e^g_C) dS + scale (Q o e)^T dO - W^T dE
+    (the state-free terms P^d V and D̃^T V do not enter it), and the chunk-local
+    gradients above, against the reverse-mode oracle."""
+    B, H, dk, dv, scale = 1, 1, 6, 5, 0.7
+    d = make_inputs("gdn2", B, T, H, dk, dv, dtype=torch.float32, seed=17)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    rng = np.random.default_rng(17)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    dO = rng.standard_normal((B, T, H, dv))
+    dSf = rng.standard_normal((B, H, dk, dv))
+    g_ref = oracle.backward("gdn2", d_o=dO, d_final=dSf, initial_state=s0, scale=scale, **d)
+    q, k, v, lg, eb, ww = (d[x][0, :, 0] for x in ("q", "k", "v", "log_g", "erase_b", "write_w"))
+    dOn = dO[0, :, 0]
+    chunks = [slice(c0, min(T, c0 + C)) for c0 in range(0, T, C)]
+
+    def chunk_ops(sl):
+        K, Q = k[sl], q[sl]
+        gam = np.cumsum(lg[sl], axis=0)
+        a, dd = eb[sl] * K, (ww[sl] - eb[sl]) * K
+        n = K.shape[0]
+        G = lambda X, Y: (X * np.exp(gam)) @ (Y * np.exp(-gam)).T
+        A, Ad = np.tril(G(K, a), -1), np.tril(G(K, dd), -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ (K * np.exp(gam))
+        Pa = scale * np.tril(G(Q, a))
+        fac = np.exp(gam[-1] - gam)
+        return gam, a, dd, Ad, Tm, W, Pa, fac
+
+    S, S0s = s0[0, 0].copy(), []
+    for sl in chunks:   # forward carry: chunk start states
+        gam, a, dd, Ad, Tm, W, Pa, fac = chunk_ops(sl)
+        E = Tm @ (v[sl] - Ad @ v[sl]) - W @ S
+        S0s.append(S.copy())
+        S = np.exp(gam[-1])[:, None] * S + (a * fac).T @ E + (dd * fac).T @ v[sl]
+    X, dSs = dSf[0, 0].copy(), [None] * len(chunks)
+    for c in reversed(range(len(chunks))):   # reverse carry: end-state gradients
+        sl = chunks[c]
+        gam, a, dd, Ad, Tm, W, Pa, fac = chunk_ops(sl)
+        dSs[c] = X.copy()
+        dE = (a * fac) @ X + Pa.T @ dOn[sl]
+        X = np.exp(gam[-1])[:, None] * X + scale * (q[sl] * np.exp(gam)).T @ dOn[sl] - W.T @ dE
+    np.testing.assert_allclose(X, g_ref["initial_state"][0, 0], rtol=0, atol=1e-10)
+    names = ("q", "k", "v", "erase_b", "write_w", "log_g")
+    for c, sl in enumerate(chunks):
+        got = gdn2_local_as_built(k[sl], q[sl], v[sl], eb[sl], ww[sl], lg[sl], S0s[c], dSs[c], dOn[sl], scale)
+        for name, x in zip(names, got):
+            np.testing.assert_allclose(x, g_ref[name][0, sl, 0], rtol=0, atol=1e-10, err_msg=f"{name} chunk {c}")
