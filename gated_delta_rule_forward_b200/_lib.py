@@ -31,7 +31,8 @@ class FwdArgs(ctypes.Structure):
 
 class BwdGrads(ctypes.Structure):
     """Mirror of gdr_bwd_grads_t (include/gdr.h)."""
-    _fields_ = [(name, ctypes.c_void_p) for name in ("dq", "dk", "dv", "dbeta", "dlog_g", "d_initial_state")]
+    _fields_ = [(name, ctypes.c_void_p) for name in ("dq", "dk", "dv", "dbeta", "dlog_g", "d_initial_state",
+                                                      "d_erase_b", "d_write_w")]
 
 
 _lock = threading.Lock()

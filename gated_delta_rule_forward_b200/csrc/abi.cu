@@ -299,7 +299,7 @@ gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, i
   if (st != GDR_OK) return st;
   if (!gdr_bwd_supported(variant, dtype == GDR_BF16, dk, dv))
     return fail(GDR_ERR_UNSUPPORTED,
-                "the backward covers DeltaNet, Gated DeltaNet, KDA and KLA with bf16 I/O, dk = 128 and dv in {64, 128}");
+                "the backward needs bf16 I/O, dk = 128 and dv in {64, 128}");
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "B, T and H must be >= 0");
   if (!a || !g) return fail(GDR_ERR_INVALID_ARG, "args and grads are required");
   if ((long)B * H == 0) return GDR_OK;
@@ -315,10 +315,14 @@ gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, i
                         "state gradient copy");
     return check_cuda(cudaMemsetAsync(g->d_initial_state, 0, bytes, s), "state gradient clear");
   }
-  if (!a->q || !a->k || !a->v || !d_o || !g->dq || !g->dk || !g->dv || !g->dbeta)
-    return fail(GDR_ERR_INVALID_ARG, "q, k, v, d_o, dq, dk, dv and dbeta are required");
+  if (!a->q || !a->k || !a->v || !d_o || !g->dq || !g->dk || !g->dv)
+    return fail(GDR_ERR_INVALID_ARG, "q, k, v, d_o, dq, dk and dv are required");
+  if (variant != GDR_GDN2 && !g->dbeta) return fail(GDR_ERR_INVALID_ARG, "dbeta is required for this variant");
+  if (variant == GDR_GDN2 && (!g->d_erase_b || !g->d_write_w))
+    return fail(GDR_ERR_INVALID_ARG, "GDN-2 needs d_erase_b and d_write_w");
   if (variant != GDR_DELTANET && !g->dlog_g) return fail(GDR_ERR_INVALID_ARG, "dlog_g is required for this variant");
-  const void *ptrs[9] = {a->q, a->k, a->v, d_o, g->dq, g->dk, g->dv, g->dbeta, g->dlog_g};
+  const void *ptrs[11] = {a->q, a->k, a->v, d_o, g->dq, g->dk, g->dv, g->dbeta, g->dlog_g, g->d_erase_b,
+                          g->d_write_w};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return fail(GDR_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
   st = validate_gates(variant, a->beta, a->log_g, a->erase_b, a->write_w);
@@ -333,13 +337,17 @@ gdr_status_t gdr_backward(int variant, int dtype, int B, int T, int H, int dk, i
   p.f.bf16_io = true;
   p.f.raw = false;
   p.f.q = a->q; p.f.k = a->k; p.f.v = a->v;
-  p.f.beta = a->beta; p.f.log_g = a->log_g; p.f.erase_b = nullptr; p.f.write_w = nullptr;
+  p.f.beta = a->beta; p.f.log_g = a->log_g;
+  p.f.erase_b = variant == GDR_GDN2 ? a->erase_b : nullptr;
+  p.f.write_w = variant == GDR_GDN2 ? a->write_w : nullptr;
   p.f.s0 = a->initial_state; p.f.s_final = nullptr; p.f.o = nullptr;
   p.f.eps = eps; p.f.scale = scale;
   p.d_o = d_o; p.d_final = d_final;
   p.dq = g->dq; p.dk = g->dk; p.dv = g->dv;
   p.dbeta = g->dbeta; p.dlog_g = variant == GDR_DELTANET ? nullptr : g->dlog_g;
   p.d_s0 = g->d_initial_state;
+  p.d_erase = variant == GDR_GDN2 ? g->d_erase_b : nullptr;
+  p.d_write = variant == GDR_GDN2 ? g->d_write_w : nullptr;
   std::string err;
   const cudaError_t e = gdr_launch_backward(p, workspace, workspace_bytes, s, &err);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "backward: " + err + cudaGetErrorString(e));

@@ -138,6 +138,31 @@ __device__ __forceinline__ float at(const GB<TR> &m, int r, int c) {
   return t < m.n ? __bfloat162float(__ldg(m.x + t * m.ld + j)) : 0.f;
 }
 
+// GDN-2: a factored key tile times a gate per (token, channel) read from global
+// memory, K o gate o 2^(sg (gamma - ref)), gate = the erase gate b (GM 1) or
+// w - b (GM 2); zero past the chunk's n tokens.
+template <bool TR, int GM>
+struct FacG {
+  using elem = float;
+  static constexpr bool kTr = TR;
+  static constexpr bool kGlobal = false;
+  static constexpr bool kExact = false;
+  const __nv_bfloat16 *x;
+  int ld, n;
+  const float *g, *ref;
+  float sg;
+  const float *eb, *ww;
+  int gld;
+};
+template <bool TR, int GM>
+__device__ __forceinline__ float at(const FacG<TR, GM> &m, int r, int c) {
+  const int t = TR ? c : r, i = TR ? r : c;
+  if (t >= m.n) return 0.f;
+  float gt = __ldg(m.eb + t * m.gld + i);
+  if (GM == 2) gt = __ldg(m.ww + t * m.gld + i) - gt;
+  return __bfloat162float(m.x[t * m.ld + i]) * gt * ex2(m.sg * (m.g[t * LDG + i] - m.ref[i]));
+}
+
 // The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N
 // product shared by W warps.
 template <int M, int N, int W = 8>
@@ -439,6 +464,12 @@ struct LocalParams {
   const uint32_t *absmax;
   __nv_bfloat16 *dq, *dk, *dv;
   float *dbeta, *dlog_g;    // dlog_g laid out as log_g
+  // GDN-2: the gates, their gradients, and per-chunk scratch in the forward and
+  // reverse records' slots (dead once the reverse carry has run)
+  const float *erase_b, *write_w;
+  float *d_erase, *d_write;
+  uint8_t *scr_f, *scr_r;
+  uint32_t rb_f, rb_r;
 };
 
 // CHAN: channel decay, with the decay tile after the scalars; at d_v = 128 Q and
@@ -502,9 +533,27 @@ struct LocalSmem {
 // of its RMS (d log g 6.0e-3 -> 5.8e-3, dk 2.3e-3 -> 4.8e-3); one pass for
 // E, dW or the dE, U', W products moved d log g to 1.5-2.9e-2, and KDA's dk
 // products at one pass 2.6e-2.
+//
+// GDN-2 (G2, with CHAN) has erase and write gates in place of beta: with
+// a = b o k, d = (w - b) o k and the factors above (a_ for the middle-token
+// factor a), the chunk's forward is A = tril((K o a_)(a o b)^T, -1), A^d likewise
+// with d, T = (I + A)^-1, Zt = I - A^d, E = T Zt V - W S0 with W = T (K o e),
+// P^a, P^d = scale tril((Q o a_)(a or d o b)^T), and
+//     dE = (a o f) dS + P^a^T dO,  tU = T^T dE,  dv = Zt^T tU + P^d^T dO + (d o f) dS
+//     dT = dE V^T Zt^T + dW (K o e)^T,  dA = tril(-T^T dT T^T, -1),  dA^d = -tril(tU V^T, -1)
+//     dk = a_ o (dA (a o b) + dA^d (d o b)) + e o T^T dW + b o da + (w - b) o dd
+//     da = b o (dA^T (K o a_) + N2a^T (Q o a_)) + f o (E dS^T)
+//     dd = b o (dA^d^T (K o a_) + N2d^T (Q o a_)) + f o (V dS^T)
+//     dq = scale e o (dO S0^T) + a_ o (N2a (a o b) + N2d (d o b))
+//     d erase = k o (da - dd),  d write = k o dd,  N2a = scale tril(dO E^T), N2d = scale tril(dO V^T)
+//     dg = dq o Q + (a_ o dKa + e o T^T dW) o K - da o a - dd o d, plus the f parts of
+//     da o a + dd o d summed over the chunk and e^(gamma_C) o rowsum(dS o S0) at its last token.
+// I - A^d, P^d, dA^d, da, dd and the (d o f) dS term go through global scratch: this
+// chunk's slots of the forward and reverse records, which nothing reads any more.
 constexpr int NTL = 512;
-template <int DV, bool CHAN>
+template <int DV, bool CHAN, bool G2 = false>
 __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) {
+  static_assert(CHAN || !G2, "GDN-2 has channel decay");
   using L = LocalSmem<DV, CHAN>;
   constexpr bool QVG = L::kQVGlobal;
   constexpr int LDB = L::LDB, LDBV = L::LDBV, LDF = L::LDF, LDW = L::LDW, LDC = L::LDC;
@@ -547,6 +596,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   const S0E *S0 = static_cast<const S0E *>(p.s0s) + static_cast<size_t>(blockIdx.x) * DK * DV;
   const float *dS = p.dss + rc * DK * DV;
   auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
+  // GDN-2 scratch: [I - A^d | P^d | dA^d] (C x C each) and [da | dd] (C x d_k), (d o f) dS (C x d_v)
+  float *scZ = reinterpret_cast<float *>(p.scr_f + static_cast<size_t>(blockIdx.x) * p.rb_f);
+  float *scPd = scZ + C * C, *scAd = scPd + C * C;
+  float *scDa = reinterpret_cast<float *>(p.scr_r + rc * p.rb_r);
+  float *scDd = scDa + C * DK, *scDv = scDd + C * DK;
 
   // ---- inputs: bf16 tiles (zero past T)
 #pragma unroll
@@ -597,7 +651,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       nk = fmaf(x, x, nk);
     }
     if (t < n) {
-      bt = __ldg(p.beta + row(t));
+      if constexpr (!G2) bt = __ldg(p.beta + row(t));
       if (!CHAN && p.decay) lg = __ldg(p.log_g + row(t));
     }
     if (p.kla) bt = bt / (nk + p.eps);
@@ -692,19 +746,33 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     if constexpr (QVG) return t < n ? __bfloat162float(__ldg(p.v + row(t) * DV + v)) : 0.f;
     else return __bfloat162float(sV[t * LDBV + v]);
   };
+  auto vmTh = [&](int h0) {   // columns h0 .. of V, transposed
+    if constexpr (QVG) return GB<true>{p.v + row(0) * DV + h0, p.H * DV, n};
+    else return BKT{sV + h0, LDBV};
+  };
+  // GDN-2: the gated key tiles (a o 2^.., d o 2^..) and the gates themselves
+  const float *ebp = G2 ? p.erase_b + row(0) * DK : nullptr, *wwp = G2 ? p.write_w + row(0) * DK : nullptr;
+  const int gld = p.H * DK;
+  auto afacT = [&](const float *ref, float sg) { return FacG<true, 1>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
+  auto dfacT = [&](const float *ref, float sg) { return FacG<true, 2>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
+  auto afac = [&](const float *ref, float sg) { return FacG<false, 1>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
+  auto dfac = [&](const float *ref, float sg) { return FacG<false, 2>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
+  auto gate = [&](const float *gp, int t, int i) { return t < n ? __ldg(gp + t * gld + i) : 0.f; };
 
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
     float g[CC::NT][4];
     zero(g);
-    if constexpr (CHAN) {
+    if constexpr (G2) {
+      wmm<CC::NT, false>(g, kfac(sgm, 1.f), afacT(sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
     }
     each(g, mc, nc, lane, [&](int t, int r, float &x) {
       const float d = CHAN ? 1.f : ex2(sG[t] - sG[r]);
-      sA[r * LD + t] = tf32r(r < t ? sbeta[t] * d * x : 0.f);
+      sA[r * LD + t] = tf32r(r < t ? (G2 ? 1.f : sbeta[t]) * d * x : 0.f);
     });
   }
   __syncthreads();
@@ -715,14 +783,35 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   }
   __syncthreads();
 
-  // ---- U' = T Diag(beta) V and W = T Diag(beta e) K; E = U' - W S0
+  if constexpr (G2) {   // Zt = I - tril((K o a_)(d o b)^T, -1) to scratch, then R = T Zt (over P)
+    {
+      float g[CC::NT][4];
+      zero(g);
+      wmm<CC::NT, false>(g, kfac(sgm, 1.f), dfacT(sgm, -1.f), DK, mc, nc, lane);
+      each(g, mc, nc, lane,
+           [&](int t, int r, float &x) { scZ[t * C + r] = r == t ? 1.f : (r < t ? -x : 0.f); });
+    }
+    __syncthreads();
+    float acc[CC::NT][4];
+    zero(acc);
+    wmm<CC::NT, false>(acc, TX{sT, LD}, F{scZ, C}, C, mc, nc, lane);
+    each(acc, mc, nc, lane, [&](int t, int r, float &x) { sP[t * LDC + r] = x; });
+    __syncthreads();
+  }
+  // ---- U' = T Diag(beta) V (GDN-2: T Zt V) and W = T Diag(beta e) K; E = U' - W S0
   float ue[CV::NT][4];
   zero(ue);
-  wmm<CV::NT, false>(ue, TX{sT, LD}, vm(), C, mv, nv, lane, sbeta);
+  if constexpr (G2) {
+    wmm<CV::NT, false>(ue, F{sP, LDC}, vm(), C, mv, nv, lane);
+  } else {
+    wmm<CV::NT, false>(ue, TX{sT, LD}, vm(), C, mv, nv, lane, sbeta);
+  }
   {
     float w[CK::NT][4];
     zero(w);
-    if constexpr (CHAN) {
+    if constexpr (G2) {
+      wmm<CK::NT, false>(w, TX{sT, LD}, kfac(szero, 1.f), C, mk, nk, lane);
+    } else if constexpr (CHAN) {
       wmm<CK::NT, false>(w, TX{sT, LD}, kfac(szero, 1.f), C, mk, nk, lane, sbeta);
     } else {
       wmm<CK::NT, false>(w, TX{sT, LD}, BK{sK, LDB}, C, mk, nk, lane, sbe);
@@ -732,6 +821,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // S0 through shared memory (over dE, A and P, none of which holds data yet):
   // E = U' - W S0 and dq's first part, scale Diag(e) dO S0^T
   float dqT[KC::NT][4];
+  if constexpr (G2) __syncthreads();   // R (over P) is read before S0 lands over it
   if constexpr (CHAN) {
     float *sS = reinterpret_cast<float *>(sm + L::DE);
 #pragma unroll
@@ -765,7 +855,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float gq[CC::NT][4];
     zero(gq);
-    if constexpr (CHAN) {
+    if constexpr (G2) {
+      wmm<CC::NT, false>(gq, qa(), afacT(sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(gq, BK{sQ, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
@@ -773,6 +865,12 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     each(gq, mc, nc, lane, [&](int t, int r, float &x) {
       sP[t * LDC + r] = r <= t ? p.scale * (CHAN ? 1.f : ex2(sG[t] - sG[r])) * x : 0.f;
     });
+  }
+  if constexpr (G2) {   // P^d to scratch
+    float gq[CC::NT][4];
+    zero(gq);
+    wmm<CC::NT, false>(gq, qa(), dfacT(sgm, -1.f), DK, mc, nc, lane);
+    each(gq, mc, nc, lane, [&](int t, int r, float &x) { scPd[t * C + r] = r <= t ? p.scale * x : 0.f; });
   }
   __syncthreads();
   // ---- with dS through shared memory in 64-column halves (over W, which E has
@@ -807,7 +905,10 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       __syncthreads();
       float acc[CH::NT][4];
       zero(acc);
-      if constexpr (CHAN) {
+      if constexpr (G2) {
+        wmm<CH::NT, false>(acc, afac(sgC, -1.f), F{sH, L::LDH}, DK, mh, nh, lane);
+        each(acc, mh, nh, lane, [&](int, int, float &x) { x *= inv_s; });
+      } else if constexpr (CHAN) {
         wmm<CH::NT, false>(acc, kfac(sgC, -1.f), F{sH, L::LDH}, DK, mh, nh, lane);
         each(acc, mh, nh, lane, [&](int, int, float &x) { x *= inv_s; });
       } else {
@@ -817,10 +918,33 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       wmm<CH::NT, false>(acc, FT{sP, LDC}, BK{sO + 64 * h, LDBV}, C, mh, nh, lane);
       each(acc, mh, nh, lane, [&](int t, int v, float &x) { sdE[t * LDF + 64 * h + v] = x; });
       wmm<KC::NT, false>(dkT, F{sH, L::LDH}, FT{sE + 64 * h, LDF}, 64, mt, nt, lane);
+      if constexpr (G2) {   // V dS^T (in dgT, still zero) and (d o f) dS / s to scratch
+        wmm<KC::NT, false>(dgT, F{sH, L::LDH}, vmTh(64 * h), 64, mt, nt, lane);
+        zero(acc);
+        wmm<CH::NT, false>(acc, dfac(sgC, -1.f), F{sH, L::LDH}, DK, mh, nh, lane);
+        each(acc, mh, nh, lane, [&](int t, int v, float &x) { scDv[t * DV + 64 * h + v] = x * inv_s; });
+      }
       __syncthreads();   // the half is read before the next one (or dW^T) lands over it
     }
   }
-  {
+  if constexpr (G2) {   // f o E dS^T and f o V dS^T start da and dd; their sum with a, d for the last token
+    float x1r[2] = {0.f, 0.f};
+    each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+      const float f = ex2(sgC[i] - sgam[t * LDG + i]) * inv_s;
+      const float da = x * f, dd = dgT[j][e] * f;
+      scDa[t * DK + i] = da;
+      scDd[t * DK + i] = dd;
+      const float kv = __bfloat162float(sK[t * LDB + i]), eb = gate(ebp, t, i), ww = gate(wwp, t, i);
+      x1r[e >> 1] += (da * eb + dd * (ww - eb)) * kv;
+      x = 0.f;
+      dgT[j][e] = 0.f;
+    });
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float s2 = quad_sum(x1r[h2]);
+      if ((lane & 3) == 0) atomicAdd(&sx1k[mt + (lane >> 2) + 8 * h2], s2);
+    }
+  } else {
     float x1r[2] = {0.f, 0.f};   // channel decay: rows mt + g, mt + g + 8 of sum_t X1 o K
     each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
       x *= (CHAN ? ex2(sgC[i] - sgam[t * LDG + i]) : sff[t]) * inv_s;
@@ -886,7 +1010,39 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   __syncthreads();
 
   // ---- dv = Diag(beta) T^T dE;  dbeta += rowsum(V o T^T dE)
-  {
+  // (GDN-2: tU = T^T dE over E, dv = Zt^T tU + P^d^T dO + (d o f) dS, dA^d = -tril(tU V^T, -1))
+  if constexpr (G2) {
+    {
+      float acc[CV::NT][4];
+      zero(acc);
+      wmm<CV::NT, false>(acc, TXT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
+      each(acc, mv, nv, lane, [&](int t, int v, float &x) { sE[t * LDF + v] = x; });
+    }
+    __syncthreads();
+    {
+      float acc[CV::NT][4];
+      zero(acc);
+      wmm<CV::NT, false>(acc, FT{scZ, C}, F{sE, LDF}, C, mv, nv, lane);
+      wmm<CV::NT, false>(acc, FT{scPd, C}, BK{sO, LDBV}, C, mv, nv, lane);
+      each(acc, mv, nv, lane, [&](int t, int v, float &x) { x += scDv[t * DV + v]; });
+      const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+      for (int j = 0; j < CV::NT; ++j)
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int t = mv + g + 8 * h2, v = nv + 8 * j + 2 * tq;
+          if (t < n)
+            *reinterpret_cast<uint32_t *>(p.dv + row(t) * DV + v) =
+                pack_bf16x2(acc[j][2 * h2], acc[j][2 * h2 + 1]);
+        }
+    }
+    {
+      float acc[CC::NT][4];
+      zero(acc);
+      wmm<CC::NT, true>(acc, F{sE, LDF}, vmT(), DV, mc, nc, lane);
+      each(acc, mc, nc, lane, [&](int t, int r, float &x) { scAd[t * C + r] = r < t ? x : 0.f; });
+    }
+  } else {
     float acc[CV::NT][4];
     zero(acc);
     wmm<CV::NT, false>(acc, TXT{sT, LD}, F{sdE, LDF}, C, mv, nv, lane);
@@ -925,21 +1081,38 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
         const int i = mt + (lane >> 2) + 8 * (e >> 1), t = nt + 8 * j + 2 * (lane & 3) + (e & 1);
         const float kv = __bfloat162float(sK[t * LDB + i]);
         const float et = CHAN ? ex2(sgam[t * LDG + i]) : see[t];
-        const float y = (CHAN ? sbeta[t] * et : sbe[t]) * acc[j][e];
+        const float y = (G2 ? et : CHAN ? sbeta[t] * et : sbe[t]) * acc[j][e];
         dkT[j][e] += y;
         add_dg(j, e, y * kv);
         dbp[j][e & 1] = fmaf(et * kv, acc[j][e], dbp[j][e & 1]);
       }
+    if constexpr (!G2) {
 #pragma unroll
-    for (int j = 0; j < KC::NT; ++j)
+      for (int j = 0; j < KC::NT; ++j)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float s2 = column_sum(dbp[j][e]);
-        if (lane < 4) atomicAdd(&sdb[nt + 8 * j + 2 * lane + e], s2);
-      }
+        for (int e = 0; e < 2; ++e) {
+          const float s2 = column_sum(dbp[j][e]);
+          if (lane < 4) atomicAdd(&sdb[nt + 8 * j + 2 * lane + e], s2);
+        }
+    }
   }
-  // ---- dT = dE V^T Diag(beta) + dW K^T Diag(beta e)  (over A^T, dead since the solve)
-  {
+  // ---- dT = dE V^T Diag(beta) + dW K^T Diag(beta e)  (over A^T, dead since the solve;
+  // GDN-2: dE V^T Zt^T + dW (K o e)^T)
+  if constexpr (G2) {
+    float a2[CC::NT][4];
+    {   // (full precision: d erase is the small difference of two gradients built from these)
+      float a1[CC::NT][4];
+      zero(a1);
+      wmm<CC::NT, false>(a1, F{sdE, LDF}, vmT(), DV, mc, nc, lane);
+      each(a1, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = x; });
+    }
+    zero(a2);
+    wmm<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
+    __syncthreads();
+    wmm<CC::NT, false>(a2, F{sA, LD}, FT{scZ, C}, C, mc, nc, lane);
+    __syncthreads();
+    each(a2, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = x; });
+  } else {
     float a1[CC::NT][4], a2[CC::NT][4];
     zero(a1);
     zero(a2);
@@ -962,19 +1135,37 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm1<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
+    if constexpr (G2) {
+      wmm<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
+    } else {
+      wmm1<CC::NT, false>(acc, F{sA, LD}, TXT{sT, LD}, C, mc, nc, lane);
+    }
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sE[t * LDC + r] = x; });
   }
   __syncthreads();
   {
     float acc[CC::NT][4];
     zero(acc);
-    wmm1<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    if constexpr (G2) {
+      wmm<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    } else {
+      wmm1<CC::NT, true>(acc, TXT{sT, LD}, F{sE, LDC}, C, mc, nc, lane);
+    }
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = r < t ? x : 0.f; });
   }
   __syncthreads();
   // ---- G = K K^T again: dbeta += rowsum(dA o D o G); N1 = Diag(beta) (dA o D), N2 = scale (dP o D)
-  {
+  // (GDN-2: N1 = dA; N2a = scale dP in place, N2d = scale tril(dO V^T) over T, dead since dA)
+  if constexpr (G2) {
+    for (int i = tid; i < C * C; i += NTL) {
+      const int t = i / C, r = i % C;
+      sP[t * LDC + r] *= p.scale;
+    }
+    float acc[CC::NT][4];
+    zero(acc);
+    wmm<CC::NT, false>(acc, BK{sO, LDBV}, vmT(), DV, mc, nc, lane);
+    each(acc, mc, nc, lane, [&](int t, int r, float &x) { sT[t * LD + r] = r <= t ? p.scale * x : 0.f; });
+  } else {
     float g[CC::NT][4];
     zero(g);
     if constexpr (CHAN) {
@@ -999,7 +1190,51 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   }
   __syncthreads();
   // ---- dk += N1 K + N1^T K + N2^T Q   (as K^T N1^T, K^T N1, Q^T N2)
-  {
+  if constexpr (G2) {
+    {   // dKa = dA (a o b) + dA^d (d o b): dk += a_ o dKa, dg += dKa o Ka
+      float acc[KC::NT][4];
+      zero(acc);
+      wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{scAd, C}, C, mt, nt, lane);
+      each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+        x *= ex2(sgam[t * LDG + i] - sgm[i]);
+        add_dg(j, e, x * __bfloat162float(sK[t * LDB + i]));
+        dkT[j][e] += x;
+      });
+    }
+    {   // da += b o (dA^T Ka + N2a^T Qa),  dd += b o (dA^d^T Ka + N2d^T Qa)
+      float acc[KC::NT][4];
+      zero(acc);
+      wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, qaT(), F{sP, LDC}, C, mt, nt, lane);
+      each(acc, mt, nt, lane,
+           [&](int i, int t, float &x) { scDa[t * DK + i] += x * ex2(sgm[i] - sgam[t * LDG + i]); });
+      zero(acc);
+      wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{scAd, C}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, qaT(), F{sT, LD}, C, mt, nt, lane);
+      each(acc, mt, nt, lane,
+           [&](int i, int t, float &x) { scDd[t * DK + i] += x * ex2(sgm[i] - sgam[t * LDG + i]); });
+    }
+    {   // dq += a_ o (N2a (a o b) + N2d (d o b))
+      float acc[KC::NT][4];
+      zero(acc);
+      wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{sT, LD}, C, mt, nt, lane);
+      each_je(acc, mt, nt, lane,
+              [&](int j, int e, int i, int t, float &x) { dqT[j][e] += x * ex2(sgam[t * LDG + i] - sgm[i]); });
+    }
+    // the gates' gradients; dk += b o da + (w - b) o dd;  dg -= da o a + dd o d
+    each_je(dkT, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
+      const float da = scDa[t * DK + i], dd = scDd[t * DK + i];
+      const float kv = __bfloat162float(sK[t * LDB + i]), eb = gate(ebp, t, i), ww = gate(wwp, t, i);
+      x += eb * da + (ww - eb) * dd;
+      add_dg(j, e, -(da * eb + dd * (ww - eb)) * kv);
+      if (t < n) {
+        p.d_erase[row(t) * DK + i] = kv * (da - dd);
+        p.d_write[row(t) * DK + i] = kv * dd;
+      }
+    });
+  } else {
     float acc[KC::NT][4];
     zero(acc);
     if constexpr (CHAN) {
@@ -1026,8 +1261,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       dkT[j][e] += x;
     });
   }
-  // ---- dq += N2 K
-  if constexpr (CHAN) {
+  // ---- dq += N2 K (GDN-2: above)
+  if constexpr (G2) {
+  } else if constexpr (CHAN) {
     float acc[KC::NT][4];
     zero(acc);
     wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
@@ -1109,7 +1345,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   // ---- dbeta (d eta for KLA) and dlog_g = suffix sums of dg over the chunk's tokens
   if (tid < C) {
     const int t = tid;
-    if (t < n) p.dbeta[row(t)] = p.kla ? sdb[t] / (snk[t] + p.eps) : sdb[t];
+    if (!G2 && t < n) p.dbeta[row(t)] = p.kla ? sdb[t] / (snk[t] + p.eps) : sdb[t];
     if (!CHAN && p.decay && p.dlog_g != nullptr) {
       float x = 0.f;
       if (t < n) x = sdg[t] + (t == n - 1 ? sred[0] + ex2(sG[n - 1]) * sred[1] * inv_s : 0.f);
@@ -1156,12 +1392,15 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
   using namespace tc;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t NC = (static_cast<size_t>(T) + C - 1) / C, bh = static_cast<size_t>(B) * H, ns = dv / 64;
-  const size_t rb_f = variant == kKDA ? rec_bytes_chan(static_cast<int>(ns)) : rec_bytes(static_cast<int>(ns));
+  const size_t rb_f = variant == kGDN2 ? rec_bytes_gdn2(static_cast<int>(ns))
+                      : variant == kKDA ? rec_bytes_chan(static_cast<int>(ns))
+                                        : rec_bytes(static_cast<int>(ns));
   BwdLayout L;
   L.fwd_rec = 0;
   L.rev_rec = up(bh * NC * rb_f);
   L.s0s = L.rev_rec + up(bh * NC * rec_bytes_gdn2(static_cast<int>(ns)));
-  L.dss = L.s0s + up(bh * NC * DK * dv * (variant == kKDA ? 4 : 2));   // S0: fp32 with channel decay
+  const bool chan = variant == kKDA || variant == kGDN2;
+  L.dss = L.s0s + up(bh * NC * DK * dv * (chan ? 4 : 2));   // S0: fp32 with channel decay
   L.x0 = L.dss + up(bh * NC * DK * dv * 4);
   L.xf = L.x0 + up(bh * DK * dv * 4);
   L.maps = L.xf + up(bh * DK * dv * 4);
@@ -1175,7 +1414,8 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv) {
 
 bool gdr_bwd_supported(int variant, int dtype_bf16, int dk, int dv) {
   using namespace gdr;
-  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA;
+  const bool v = variant == kDeltaNet || variant == kGatedDeltaNet || variant == kKLA || variant == kKDA ||
+                 variant == kGDN2;
   return v && dtype_bf16 && dk == 128 && (dv == 64 || dv == 128);
 }
 
@@ -1205,8 +1445,8 @@ cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd
   RevPrepParams rp;
   rp.T = f.T; rp.H = f.H; rp.NC = (f.T + C - 1) / C;
   const int ns = f.dv / 64;
-  rp.chan = f.variant == gdr::kKDA;
-  rp.rb_f = rp.chan ? rec_bytes_chan(ns) : rec_bytes(ns);
+  rp.chan = f.variant == gdr::kKDA || f.variant == gdr::kGDN2;
+  rp.rb_f = f.variant == gdr::kGDN2 ? rec_bytes_gdn2(ns) : rp.chan ? rec_bytes_chan(ns) : rec_bytes(ns);
   rp.rb_r = rec_bytes_gdn2(ns);
   rp.d_o = static_cast<const __nv_bfloat16 *>(p.d_o);
   rp.fwd = fwd_rec; rp.rev = rev_rec; rp.absmax = absmax;
@@ -1222,7 +1462,7 @@ cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd
 }
 
 cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, const float *dss,
-                                 const uint32_t *absmax, cudaStream_t s) {
+                                 const uint32_t *absmax, uint8_t *fwd_rec, uint8_t *rev_rec, cudaStream_t s) {
   using namespace gdr::tc;
   const gdr::FwdProblem &f = p.f;
   LocalParams lp;
@@ -1240,6 +1480,10 @@ cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, cons
   lp.dk = static_cast<__nv_bfloat16 *>(p.dk);
   lp.dv = static_cast<__nv_bfloat16 *>(p.dv);
   lp.dbeta = p.dbeta; lp.dlog_g = p.dlog_g;
+  lp.erase_b = f.erase_b; lp.write_w = f.write_w;
+  lp.d_erase = p.d_erase; lp.d_write = p.d_write;
+  lp.scr_f = fwd_rec; lp.scr_r = rev_rec;
+  lp.rb_f = rec_bytes_gdn2(f.dv / 64); lp.rb_r = rec_bytes_gdn2(f.dv / 64);
   const int grid = f.B * f.H * lp.NC;
   auto run = [&](auto kern, size_t smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1247,6 +1491,9 @@ cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, cons
     kern<<<grid, NTL, smem, s>>>(lp);
     return cudaGetLastError();
   };
+  if (f.variant == gdr::kGDN2)
+    return f.dv == 128 ? run(bwd_local_kernel<128, true, true>, LocalSmem<128, true>::BYTES)
+                       : run(bwd_local_kernel<64, true, true>, LocalSmem<64, true>::BYTES);
   if (f.variant == gdr::kKDA)
     return f.dv == 128 ? run(bwd_local_kernel<128, true>, LocalSmem<128, true>::BYTES)
                        : run(bwd_local_kernel<64, true>, LocalSmem<64, true>::BYTES);

@@ -1,5 +1,4 @@
-// Chunked backward of DeltaNet, Gated DeltaNet, KDA and KLA: its
-// chunk-parallel kernels (chunk_bwd.cu) and the orchestration over
+// Chunked backward of the five variants: its chunk-parallel kernels (chunk_bwd.cu) and the orchestration over
 // the forward's preparation and carry kernels (chunk_split.cu).
 #pragma once
 #include <cstdint>
@@ -18,6 +17,7 @@ struct BwdProblem {
   float *dbeta;            // [B,T,H]: d beta, or d eta for KLA
   float *dlog_g;           // [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA); null for DeltaNet
   float *d_s0;             // [B,H,dk,dv] gradient of the initial state, or null
+  float *d_erase, *d_write;   // [B,T,H,dk] GDN-2's erase and write gate gradients
 };
 
 // Byte offsets of the backward's workspace regions (each 256-byte aligned).
@@ -35,8 +35,8 @@ BwdLayout bwd_layout(int variant, int B, int T, int H, int dv);
 
 }  // namespace gdr
 
-// The backward covers DeltaNet, Gated DeltaNet, KDA and KLA with bf16 I/O,
-// dk = 128 and dv in {64, 128}.
+// The backward covers all five variants with bf16 I/O, dk = 128 and dv in
+// {64, 128}.
 bool gdr_bwd_supported(int variant, int dtype_bf16, int dk, int dv);
 size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv);
 
@@ -45,8 +45,10 @@ size_t gdr_bwd_workspace_bytes(int variant, int B, int T, int H, int dv);
 cudaError_t gdr_bwd_launch_scale(const gdr::BwdProblem &p, uint32_t *absmax, float *x0, cudaStream_t s);
 cudaError_t gdr_bwd_launch_rev_prep(const gdr::BwdProblem &p, const uint8_t *fwd_rec, uint8_t *rev_rec,
                                     const uint32_t *absmax, cudaStream_t s);
+// GDN-2 uses each chunk's slots of the forward and reverse records (dead by
+// then) as scratch.
 cudaError_t gdr_bwd_launch_local(const gdr::BwdProblem &p, const void *s0s, const float *dss,
-                                  const uint32_t *absmax, cudaStream_t s);
+                                  const uint32_t *absmax, uint8_t *fwd_rec, uint8_t *rev_rec, cudaStream_t s);
 cudaError_t gdr_bwd_launch_unscale(const gdr::BwdProblem &p, const float *xf, const uint32_t *absmax,
                                    cudaStream_t s);
 // Read and clear this file's device error word (bit 1: an fp16 operand of the

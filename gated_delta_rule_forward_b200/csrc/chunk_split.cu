@@ -2316,7 +2316,7 @@ cudaError_t launch_split(const FwdProblem &p, void *ws, size_t ws_bytes, cudaStr
 // the forward's would (few long sequences).
 template <int VAR>
 cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t stream, std::string *err) {
-  constexpr int MODE = VAR == kKDA ? 1 : 0;
+  constexpr int MODE = VAR == kKDA ? 1 : VAR == kGDN2 ? 2 : 0;
   const FwdProblem &p = bp.f;
   const int NC = (p.T + C - 1) / C;
   const BwdLayout L = bwd_layout(VAR, p.B, p.T, p.H, p.dv);
@@ -2325,7 +2325,7 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
   // absorb, in fp32
   void *s0s = w + L.s0s;
   float *dss = reinterpret_cast<float *>(w + L.dss);
-  const int s0_f16 = MODE == 1 ? 0 : CARRY_STATES_F16;
+  const int s0_f16 = MODE == 0 ? CARRY_STATES_F16 : 0;
   float *x0 = reinterpret_cast<float *>(w + L.x0), *xf = reinterpret_cast<float *>(w + L.xf);
   uint32_t *absmax = reinterpret_cast<uint32_t *>(w + L.absmax);
   const SegPlan sp = L.maps_bytes > 0 ? seg_plan(p.B, p.H, p.dv, NC) : SegPlan{1, NC};
@@ -2364,7 +2364,7 @@ cudaError_t launch_backward(const BwdProblem &bp, uint8_t *w, cudaStream_t strea
     e = launch_carry<2>(p, NC, w + L.rev_rec, lr, true, stream, err);
   }
   if (e != cudaSuccess) return e;
-  if ((e = gdr_bwd_launch_local(bp, s0s, dss, absmax, stream)) != cudaSuccess) {
+  if ((e = gdr_bwd_launch_local(bp, s0s, dss, absmax, w + L.fwd_rec, w + L.rev_rec, stream)) != cudaSuccess) {
     *err = "local gradients: ";
     return e;
   }
@@ -2389,6 +2389,7 @@ cudaError_t gdr_launch_backward(const gdr::BwdProblem &p, void *ws, size_t ws_by
     case kGatedDeltaNet: return tc::launch_backward<kGatedDeltaNet>(p, w, stream, err);
     case kKLA: return tc::launch_backward<kKLA>(p, w, stream, err);
     case kKDA: return tc::launch_backward<kKDA>(p, w, stream, err);
+    case kGDN2: return tc::launch_backward<kGDN2>(p, w, stream, err);
     default: *err = "variant not covered by the backward: "; return cudaErrorInvalidValue;
   }
 }

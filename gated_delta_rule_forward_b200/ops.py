@@ -129,13 +129,14 @@ def forward(q, k, v, *, variant, beta=None, log_g=None, erase_b=None, write_w=No
     return out, final_state
 
 
-def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, initial_state=None, d_final_state=None,
-             eps=1e-6, scale=1.0, stream=None):
+def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, erase_b=None, write_w=None, initial_state=None,
+             d_final_state=None, eps=1e-6, scale=1.0, stream=None):
     """Gradients of <d_o, o> + <d_final_state, S_T> for the forward over the
-    same inputs: the chunked backward (DeltaNet, Gated DeltaNet, KDA, KLA;
-    bf16 q, k, v, d_o with dk = 128, dv 64 or 128; gates fp32 as for
-    forward()).  Returns a dict with dq, dk, dv (bf16), beta (d beta, or d eta
-    for KLA), log_g (shaped as log_g; None for DeltaNet) and initial_state (fp32 [B,H,dk,dv]; the
+    same inputs: the chunked backward (all five variants; bf16 q, k, v, d_o
+    with dk = 128, dv 64 or 128; gates fp32 as for forward()).  Returns a dict
+    keyed by the inputs: q, k, v (bf16), beta (d beta, or d eta for KLA; None
+    for GDN-2), log_g (shaped as log_g; None for DeltaNet), erase_b and
+    write_w (GDN-2, else None) and initial_state (fp32 [B,H,dk,dv]; the
     gradient of the initial state, zero-initial-state runs included)."""
     vid = variant_id(variant)
     if q.dim() != 4:
@@ -150,22 +151,24 @@ def backward(q, k, v, d_o, *, variant, beta=None, log_g=None, initial_state=None
     _need(k, "k", (B, T, H, dk), q.dtype, dev)
     _need(v, "v", (B, T, H, dv), q.dtype, dev)
     _need(d_o, "d_o", (B, T, H, dv), q.dtype, dev)
-    beta, log_g, _, _ = _gates(vid, (B, T, H), dk, dev, beta, log_g, None, None)
+    beta, log_g, erase_b, write_w = _gates(vid, (B, T, H), dk, dev, beta, log_g, erase_b, write_w)
     f32 = torch.float32
     if initial_state is not None:
         _need(initial_state, "initial_state", (B, H, dk, dv), f32, dev)
     if d_final_state is not None:
         _need(d_final_state, "d_final_state", (B, H, dk, dv), f32, dev)
     g = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
-         "beta": torch.empty(B, T, H, device=dev, dtype=f32),
+         "beta": None if beta is None else torch.empty(B, T, H, device=dev, dtype=f32),
          "log_g": None if log_g is None else torch.empty(log_g.shape, device=dev, dtype=f32),
+         "erase_b": None if erase_b is None else torch.empty_like(erase_b),
+         "write_w": None if write_w is None else torch.empty_like(write_w),
          "initial_state": torch.empty(B, H, dk, dv, device=dev, dtype=f32)}
-    a = FwdArgs(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), beta=beta.data_ptr(),
-                log_g=None if log_g is None else log_g.data_ptr(),
-                initial_state=None if initial_state is None else initial_state.data_ptr())
-    gr = BwdGrads(dq=g["q"].data_ptr(), dk=g["k"].data_ptr(), dv=g["v"].data_ptr(), dbeta=g["beta"].data_ptr(),
-                  dlog_g=None if g["log_g"] is None else g["log_g"].data_ptr(),
-                  d_initial_state=g["initial_state"].data_ptr())
+    opt = lambda x: None if x is None else x.data_ptr()
+    a = FwdArgs(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), beta=opt(beta), log_g=opt(log_g),
+                erase_b=opt(erase_b), write_w=opt(write_w), initial_state=opt(initial_state))
+    gr = BwdGrads(dq=g["q"].data_ptr(), dk=g["k"].data_ptr(), dv=g["v"].data_ptr(), dbeta=opt(g["beta"]),
+                  dlog_g=opt(g["log_g"]), d_initial_state=g["initial_state"].data_ptr(),
+                  d_erase_b=opt(g["erase_b"]), d_write_w=opt(g["write_w"]))
     L = lib()
     dt = _DTYPES[q.dtype]
     ws = L.gdr_backward_workspace_size(vid, dt, B, T, H, dk, dv)

@@ -222,9 +222,11 @@ typedef struct {
     void *dq;                 /* [B,T,H,dk] I/O dtype */
     void *dk;                 /* [B,T,H,dk] I/O dtype */
     void *dv;                 /* [B,T,H,dv] I/O dtype */
-    float *dbeta;             /* [B,T,H]: d beta, or d eta for KLA */
-    float *dlog_g;            /* [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA); DeltaNet: unused */
+    float *dbeta;             /* [B,T,H]: d beta, or d eta for KLA; GDN-2: unused */
+    float *dlog_g;            /* [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA, GDN-2); DeltaNet: unused */
     float *d_initial_state;   /* [B,H,dk,dv], or NULL when not wanted */
+    float *d_erase_b;         /* [B,T,H,dk], GDN-2 only */
+    float *d_write_w;         /* [B,T,H,dk], GDN-2 only */
 } gdr_bwd_grads_t;
 
 /*
@@ -243,8 +245,8 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * forward's inputs, for the forward that `args` describes (its o and
  * final_state are not used): the gate-aware backward that keeps the
  * chunkwise structure ("Gated DeltaNet-2: Decoupling Erase and Write in
- * Linear Attention", technical core), for DeltaNet, Gated DeltaNet, KDA and
- * KLA with bf16 I/O, dk = 128 and dv in {64, 128}.  With S
+ * Linear Attention", technical core), for all five variants with bf16 I/O,
+ * dk = 128 and dv in {64, 128}.  With S
  * the state and dS its gradient, per 64-token chunk:
  *     forward   E = U' - W S0,  O = Qg S0 + P E,  S_C = Gamma_C S0 + Kt^T E
  *     backward  dE = Kt dS + P^T dO,  dS0 = Gamma_C dS + Qg^T dO - W^T dE
@@ -264,8 +266,10 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * gradients match an exact backward to about 1e-3 of their RMS; the
  * gradients are rescaled internally by a power of two so that d_o's range
  * does not matter.  workspace: at least gdr_backward_workspace_size() bytes,
- * 16-byte aligned, overwritten.  The raw-input mode (GDR_RAW_INPUTS),
- * GDN-2, fp32 I/O and dk = 64 return GDR_ERR_UNSUPPORTED.  T = 0 gives
+ * 16-byte aligned, overwritten.  For GDN-2 the records' state-free terms
+ * (P^d V, D~^T V) do not enter the dS recurrence, and the chunk-local kernel
+ * also returns d erase_b and d write_w.  The raw-input mode (GDR_RAW_INPUTS),
+ * fp32 I/O and dk = 64 return GDR_ERR_UNSUPPORTED.  T = 0 gives
  * d_initial_state = d_final_state.  Validation and errors as for the
  * forward; a reverse-record operand beyond the fp16 range is reported as
  * GDR_ERR_RANGE by gdr_device_status().

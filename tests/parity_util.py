@@ -17,6 +17,16 @@ Tolerances (written here once, used by every parity test):
         the arithmetic budget plus the largest bf16 rounding such an element
         can have.  It is reported beside the first metric so that the
         rounding allowance cannot hide an error on the bulk of the output.
+  * GDN-2's gate gradients (d erase_b, d write_w; fp32) in the backward, per
+    64-token chunk: max|gpu - ref| <= 2e-2 * RMS(ref) + 2^-10 * max|ref| over
+    the chunk.  The gradients inherit the relative error of the chunk states
+    that the carries hold with fp16 operands (unit roundoff 2^-11; 2^-10 allows
+    twice that) in proportion to the size of the terms a chunk's gradients
+    are built from.  d erase_b is k times a difference of two such terms, which
+    the final-state gradient dominates at the sequence's last tokens: under a
+    random unit-scale d_final the last chunk's largest elements reach ~270
+    RMS, and every element of that chunk carries an error of ~2^-11 of them.
+    In every other chunk the allowance is a few 1e-3 RMS.
 """
 import numpy as np
 import torch
@@ -88,6 +98,23 @@ def assert_close(gpu, ref, dtype, what=""):
     else:
         err = rms_rel(gpu, ref)
         assert err <= BF16_TOL, f"{what}: max|err|/RMS(ref) = {err:.3e} > {BF16_TOL}"
+    return err
+
+
+CARRY_ROUND = 2.0 ** -10
+
+
+def assert_close_gate_grad(gpu, ref, what="", chunk=64):
+    """GDN-2's fp32 gate gradients [B,T,H,dk] (see module docstring): per chunk,
+    max(|err|) - 2^-10 max|ref| <= 2e-2 RMS(ref)."""
+    gpu = gpu.detach().double().cpu().numpy() if hasattr(gpu, "detach") else np.asarray(gpu)
+    rms = max(np.sqrt(np.mean(ref * ref)), 1e-30)
+    err, T = 0.0, ref.shape[1]
+    for c0 in range(0, T, chunk):
+        e = np.abs(gpu[:, c0:c0 + chunk] - ref[:, c0:c0 + chunk]).max()
+        err = max(err, (e - CARRY_ROUND * np.abs(ref[:, c0:c0 + chunk]).max()) / rms)
+    assert err <= BF16_TOL, (f"{what}: max over chunks of (max|err| - 2^-10 max|ref|)/RMS(ref) = {err:.3e} > "
+                             f"{BF16_TOL} (plain max|err|/RMS = {rms_rel(gpu, ref):.3e})")
     return err
 
 

@@ -245,7 +245,12 @@ def test_backward_validation(L):
     assert bwd_call(L) == 4                                  # valid: reaches the (injected) launch failure
     for v in (0, 1, 2, 4):
         assert bwd_call(L, variant=v) == 4
-    assert bwd_call(L, variant=3) == 2                                       # GDN-2: unsupported
+    assert bwd_call(L, variant=3) == 1                                       # GDN-2 needs its gate gradients
+    g2 = _lib.BwdGrads(dq=FAKE, dk=FAKE, dv=FAKE, dbeta=None, dlog_g=FAKE, d_initial_state=FAKE,
+                       d_erase_b=FAKE, d_write_w=FAKE)
+    a2 = args(beta=None, erase_b=FAKE, write_w=FAKE, initial_state=FAKE)
+    assert bwd_call(L, variant=3, grads=g2, a=a2) == 4                       # ... and takes no dbeta
+    assert bwd_call(L, variant=3, grads=g2, a=args(beta=None, erase_b=None, initial_state=FAKE)) == 1   # needs the gates
     assert bwd_call(L, variant=1 | 0x100) == 2                               # raw inputs: unsupported
     assert bwd_call(L, dtype=0) == 2 and bwd_call(L, dk=64) == 2             # fp32 I/O, dk = 64
     assert bwd_call(L, dv=96) == 2
@@ -273,6 +278,7 @@ def test_backward_workspace_sizes(L):
     rec_kda = rec + 512 - 16                                                 # Gamma_C as 128 floats
     want_kda = up(bh * NC * rec_kda) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
     assert L.gdr_backward_workspace_size(2, 1, B, T, H, 128, 128) == want_kda
-    assert L.gdr_backward_workspace_size(3, 1, B, T, H, 128, 128) == 0       # GDN-2
+    assert L.gdr_backward_workspace_size(3, 1, B, T, H, 128, 128) == \
+        up(bh * NC * rev) + up(bh * NC * rev) + 2 * up(bh * NC * 128 * 128 * 4) + 2 * up(bh * 128 * 128 * 4) + 256
     assert L.gdr_backward_workspace_size(1, 0, B, T, H, 128, 128) == 0       # fp32 I/O
     assert L.gdr_backward_workspace_size(1, 1, B, 0, H, 128, 128) == 0

@@ -1,5 +1,5 @@
-"""GPU parity of the chunked backward (DeltaNet, Gated DeltaNet, KDA, KLA)
-against the fp64 reverse-mode oracle, through the C ABI.
+"""GPU parity of the chunked backward (all five variants) against the fp64
+reverse-mode oracle, through the C ABI.
 
 The backward re-runs the forward's chunk products and carry, runs the
 end-state-gradient recurrence on the forward's carry kernel over the chunks in
@@ -17,10 +17,10 @@ import torch
 import gated_delta_rule_forward_b200 as gdr
 import oracle
 from gated_delta_rule_forward_b200.inputs import make_inputs, random_output_grad, random_state
-from parity_util import assert_close, select, to_dev
+from parity_util import assert_close, assert_close_gate_grad, select, to_dev
 
 pytestmark = pytest.mark.gpu
-VARS = ["deltanet", "gdn", "kda", "kla"]
+VARS = ["deltanet", "gdn", "kda", "gdn2", "kla"]
 
 
 def run_backward(variant, B, T, H, dv=128, seed=0, s0=True, d_final=True, do_scale=1.0, scale=None, edit=None):
@@ -33,19 +33,27 @@ def run_backward(variant, B, T, H, dv=128, seed=0, s0=True, d_final=True, do_sca
     dS = random_state(B, H, dk, dv, seed + 2, scale=1.0) if d_final else None
     dO = random_output_grad(B, T, H, dv, seed + 3, scale=do_scale)
     dd = to_dev(d)
-    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, beta=dd["beta"], log_g=dd["log_g"],
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, **gates(dd),
                      initial_state=None if S0 is None else S0.cuda(),
                      d_final_state=None if dS is None else dS.cuda(), scale=scale)
     gdr.device_status()
-    ref = oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"],
-                          initial_state=S0, d_final=dS, scale=scale)
+    ref = oracle.backward(variant, d["q"], d["k"], d["v"], dO, **gates(d), initial_state=S0, d_final=dS,
+                          scale=scale)
     return g, ref
+
+
+def gates(d):
+    return {x: d[x] for x in ("beta", "log_g", "erase_b", "write_w")}
 
 
 def check_grads(g, ref, variant, what=""):
     for name in ("q", "k", "v"):
         assert_close(g[name], ref[name], torch.bfloat16, f"{what} d{name}")
-    assert_close(g["beta"], ref["beta"], torch.bfloat16, f"{what} d{'eta' if variant == 'kla' else 'beta'}")
+    if variant == "gdn2":
+        assert_close_gate_grad(g["erase_b"], ref["erase_b"], f"{what} d erase_b")
+        assert_close_gate_grad(g["write_w"], ref["write_w"], f"{what} d write_w")
+    else:
+        assert_close(g["beta"], ref["beta"], torch.bfloat16, f"{what} d{'eta' if variant == 'kla' else 'beta'}")
     if variant != "deltanet":
         assert_close(g["log_g"], ref["log_g"], torch.bfloat16, f"{what} dlog_g")
     assert_close(g["initial_state"], ref["initial_state"], torch.bfloat16, f"{what} d initial state")
@@ -68,12 +76,13 @@ def test_backward_short_sequences(T):
 
 
 @pytest.mark.parametrize("T", [1, 20, 37, 65])
-def test_backward_short_sequences_channel_decay(T):
-    """KDA's chunk products factor the decay around token 31 of a chunk, or
-    around the last token of a shorter one: chunks of 1, 20 and 37 tokens and
-    a 1-token tail."""
-    g, ref = run_backward("kda", 1, T, 2, seed=31)
-    check_grads(g, ref, "kda", f"T={T}")
+@pytest.mark.parametrize("variant", ["kda", "gdn2"])
+def test_backward_short_sequences_channel_decay(variant, T):
+    """The channel-decay chunk products factor the decay around token 31 of a
+    chunk, or around the last token of a shorter one: chunks of 1, 20 and 37
+    tokens and a 1-token tail."""
+    g, ref = run_backward(variant, 1, T, 2, seed=31)
+    check_grads(g, ref, variant, f"T={T}")
 
 
 def test_backward_without_states():
@@ -146,7 +155,7 @@ def test_backward_decay_beyond_the_guard_is_reported():
     gdr.device_status()   # the flag is cleared once read
 
 
-@pytest.mark.parametrize("variant", ["gdn", "kla", "kda"])
+@pytest.mark.parametrize("variant", ["gdn", "kla", "kda", "gdn2"])
 def test_backward_350m_layer_sampled(variant):
     """The 350M layer (B=8, T=2048, H=8, full size, in the launch configuration of
     a training step), checked against the oracle on two of its sequences."""
@@ -156,13 +165,11 @@ def test_backward_350m_layer_sampled(variant):
     d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.bfloat16, seed=26)
     dO = random_output_grad(B, T, H, dv, 27)
     dd = to_dev(d)
-    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, beta=dd["beta"], log_g=dd["log_g"],
-                     scale=scale)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant=variant, **gates(dd), scale=scale)
     gdr.device_status()
     for b in (0, B - 1):
         s = select(d, b=slice(b, b + 1))
-        ref = oracle.backward(variant, s["q"], s["k"], s["v"], dO[b:b + 1], beta=s["beta"], log_g=s["log_g"],
-                              scale=scale)
+        ref = oracle.backward(variant, s["q"], s["k"], s["v"], dO[b:b + 1], **gates(s), scale=scale)
         gb = {k: (None if x is None else x[b:b + 1]) for k, x in g.items()}
         check_grads(gb, ref, variant, f"sequence {b}")
 
@@ -196,7 +203,7 @@ def test_backward_long_context_sampled():
         check_grads(gh, ref, "gdn", f"head {h}")
 
 
-@pytest.mark.parametrize("variant", ["gdn", "kla", "kda"])
+@pytest.mark.parametrize("variant", ["gdn", "kla", "kda", "gdn2"])
 def test_backward_segmented(variant):
     """Few long sequences (B*H = 2, 65 chunks): both carries run in segments (13
     of 5 chunks) from an initial state and a final-state gradient."""
