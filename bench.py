@@ -56,8 +56,9 @@ WORKLOADS = {
     "gdn_fwd_350m_raw": ("gdn", 8, 2048, 8, 128, 128),
     "gdn_bwd_350m": ("gdn", 8, 2048, 8, 128, 128),
     "kda_bwd_1p3b": ("kda", 4, 4096, 16, 128, 128),
+    "gdn2_bwd_1p3b": ("gdn2", 4, 4096, 16, 128, 128),
 }
-BWD_WORKLOADS = {"gdn_bwd_350m", "kda_bwd_1p3b"}   # the chunked backward (gradients of o and the final state)
+BWD_WORKLOADS = {"gdn_bwd_350m", "kda_bwd_1p3b", "gdn2_bwd_1p3b"}   # the chunked backward (gradients of o and the final state)
 RAW_WORKLOADS = {"gdn_fwd_350m_raw"}   # raw projections and logits in; the kernels apply the transforms
 DEFAULT = "gdn_fwd_64k"
 DECODE_STEPS = 1024         # the decode chain after the long-context prefill
@@ -152,9 +153,14 @@ def bwd_bytes(variant, B, T, H, dk, dv, io_bytes=2):
     written once (no initial state, no final-state gradient)."""
     th = B * T * H
     b = th * (2 * dk + 2 * dv) * io_bytes + th * (2 * dk + dv) * io_bytes
-    b += th * 4 * 2                                    # beta in, d beta out
+    if variant != "gdn2":
+        b += th * 4 * 2                                # beta in, d beta out
     if variant in ("gdn", "kla"):
         b += th * 4 * 2                                # log decay in, its gradient out
+    elif variant in ("kda", "gdn2"):
+        b += th * dk * 4 * 2                           # per-channel log decay in, its gradient out
+    if variant == "gdn2":
+        b += 2 * th * dk * 4 * 2                       # erase and write gates in, their gradients out
     b += B * H * dk * dv * 4                           # initial state's gradient
     return b
 
@@ -319,8 +325,7 @@ def run_backward_workload(name, K, W, world, seed=0):
 
     def step(i):
         d = sets[i % 2]
-        gdr.backward(d["q"], d["k"], d["v"], grads[i % 2], variant=variant, beta=d["beta"], log_g=d["log_g"],
-                     scale=dk ** -0.5)
+        gdr.backward(d["q"], d["k"], d["v"], grads[i % 2], variant=variant, **gates(d), scale=dk ** -0.5)
 
     for i in range(W):
         step(i)
@@ -553,7 +558,7 @@ def cpu_baseline(name):
         dO = random_output_grad(1, T, H, dv, 1)
         passes, t0 = 0, time.perf_counter()
         while passes == 0 or time.perf_counter() - t0 < 2.0:
-            oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"], scale=dk ** -0.5)
+            oracle.backward(variant, d["q"], d["k"], d["v"], dO, **gates(d), scale=dk ** -0.5)
             passes += 1
         dt = time.perf_counter() - t0
         return {"value": passes * T / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
@@ -659,8 +664,7 @@ def reference(args):
         from gated_delta_rule_forward_b200.inputs import random_output_grad
         d = make_inputs(variant, 1, T, H, dk, dv, dtype=torch.bfloat16, seed=0)
         dO = random_output_grad(1, T, H, dv, 1)
-        run = lambda: oracle.backward(variant, d["q"], d["k"], d["v"], dO, beta=d["beta"], log_g=d["log_g"],
-                                      scale=dk ** -0.5)
+        run = lambda: oracle.backward(variant, d["q"], d["k"], d["v"], dO, **gates(d), scale=dk ** -0.5)
         tokens = T
         sample = f"the backward of 1 of {B} sequences x {T} tokens x {H} heads per step, fp64"
     else:           # forward: one of the B sequences per step (its first tokens if it is long)
