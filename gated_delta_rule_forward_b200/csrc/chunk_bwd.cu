@@ -1,6 +1,6 @@
-// Chunk-parallel kernels of the chunked backward for DeltaNet, Gated DeltaNet,
-// KDA and KLA.  "Gated DeltaNet-2" (technical core) asks
-// for a gate-aware backward that keeps the chunkwise structure; this one
+// Chunk-parallel kernels of the chunked backward for the five variants.
+// "Gated DeltaNet-2" (technical core) asks for a gate-aware backward that
+// keeps the chunkwise structure; this one
 // reverses the forward's chunk algebra ("Kaczmarz Linear Attention", KLA
 // update rule and implementation):
 //     forward, per chunk:  E = U' - W S0,  O = Qg S0 + P E,  S_C = Gamma_C S0 + Kt^T E
@@ -15,8 +15,9 @@
 // is local to a chunk given its start state S0 and dS; bwd_local_kernel
 // computes them per chunk, dE included (the records carry beta in P and Kt,
 // so the carry's own residual is Diag(beta) dE, which cannot be divided
-// back where beta vanishes).  With g the chunk-local cumulative log decay,
-// D_tr = e^(g_t - g_r) for r <= t, e = e^g and f = e^(g_C - g):
+// back where beta vanishes).  With scalar decay, g the chunk-local cumulative
+// log decay, D_tr = e^(g_t - g_r) for r <= t, e = e^g and f = e^(g_C - g)
+// (channel decay and GDN-2's gates: see bwd_local_kernel):
 //     dE = Diag(f) K dS + P^T dO,  P = scale tril(D o Q K^T)
 //     G = K K^T,  A = tril(Diag(beta) (D o G), -1),  T = (I + A)^-1
 //     E = T Diag(beta) V - T Diag(beta e) K S0,  dW = -dE S0^T,  dP = tril(dO E^T)
@@ -35,6 +36,9 @@
 // The reverse carry's fp16 operands need the gradients near unit scale: dO and
 // the final-state gradient are scaled by a power of two s (max |.| to [0.5, 1)),
 // and the local kernel and the initial-state gradient divide it out again.
+// The forward carry keeps every chunk's start state in fp16 for scalar decay
+// (the operand its MMAs took) and in fp32 for channel decay; the reverse carry
+// keeps its states in fp32.
 #include <algorithm>
 #include <type_traits>
 #include <cuda_bf16.h>

@@ -1,5 +1,6 @@
-// Chunked backward of the five variants: its chunk-parallel kernels (chunk_bwd.cu) and the orchestration over
-// the forward's preparation and carry kernels (chunk_split.cu).
+// Chunked backward of the five variants: its chunk-parallel kernels
+// (chunk_bwd.cu) and the orchestration over the forward's preparation and
+// carry kernels (chunk_split.cu).
 #pragma once
 #include <cstdint>
 #include <string>
@@ -14,8 +15,8 @@ struct BwdProblem {
   const void *d_o;         // [B,T,H,dv] I/O dtype: gradient of the outputs
   const float *d_final;    // [B,H,dk,dv] gradient of the final state, or null (zero)
   void *dq, *dk, *dv;      // [B,T,H,dk], [B,T,H,dk], [B,T,H,dv] I/O dtype
-  float *dbeta;            // [B,T,H]: d beta, or d eta for KLA
-  float *dlog_g;           // [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA); null for DeltaNet
+  float *dbeta;            // [B,T,H]: d beta, or d eta for KLA; null for GDN-2
+  float *dlog_g;           // [B,T,H] (GDN, KLA) or [B,T,H,dk] (KDA, GDN-2); null for DeltaNet
   float *d_s0;             // [B,H,dk,dv] gradient of the initial state, or null
   float *d_erase, *d_write;   // [B,T,H,dk] GDN-2's erase and write gate gradients
 };
