@@ -130,25 +130,50 @@ def chunk_span_log2(log_g):
     return float(np.abs(g - g[:, :, 31:32]).max() / np.log(2.0))
 
 
-def test_backward_strong_channel_decay():
-    """KDA with its decay doubled: factors up to 2^102 within a chunk, inside
+@pytest.mark.parametrize("variant", ["kda", "gdn2"])
+def test_backward_strong_channel_decay(variant):
+    """Channel decay doubled: factors up to 2^90-2^120 within a chunk, inside
     the forward's factoring range (2^120)."""
     def edit(d):
         d["log_g"] = (d["log_g"] * 2.0).contiguous()
         span = chunk_span_log2(d["log_g"])
-        assert 90.0 < span < 120.0, span
-    g, ref = run_backward("kda", 1, 192, 2, seed=25, edit=edit)
-    check_grads(g, ref, "kda", "strong channel decay")
+        assert 85.0 < span < 120.0, span
+    g, ref = run_backward(variant, 1, 192, 2, seed=25, edit=edit)
+    check_grads(g, ref, variant, "strong channel decay")
 
 
-def test_backward_decay_beyond_the_guard_is_reported():
-    """KDA with a decay of e^-5 per token on every channel spans 2^230 within
-    a chunk: the backward returns normally and reports GDR_ERR_RANGE."""
-    d = to_dev(make_inputs("kda", 1, 130, 2, seed=32))
+def test_backward_gdn2_tied_gates_is_kda():
+    """GDN-2 with b = w = beta on every channel is KDA ("Gated DeltaNet-2", what
+    is new): its q, k, v and log g gradients are KDA's, and the gate gradients
+    summed over the channels, sum_i (d b_i + d w_i), are KDA's d beta."""
+    B, T, H = 2, 200, 3
+    d = make_inputs("gdn2", B, T, H, dtype=torch.bfloat16, seed=34, gdn2_tied=True)
+    S0 = random_state(B, H, 128, 128, 35)
+    dS = random_state(B, H, 128, 128, 36, scale=1.0)
+    dO = random_output_grad(B, T, H, 128, 37)
+    dd = to_dev(d)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant="gdn2", **gates(dd), initial_state=S0.cuda(),
+                     d_final_state=dS.cuda(), scale=128 ** -0.5)
+    gdr.device_status()
+    beta = d["erase_b"][..., 0].contiguous()
+    ref = oracle.backward("kda", d["q"], d["k"], d["v"], dO, beta=beta, log_g=d["log_g"], initial_state=S0, d_final=dS,
+                          scale=128 ** -0.5)
+    for name in ("q", "k", "v"):
+        assert_close(g[name], ref[name], torch.bfloat16, f"d{name}")
+    assert_close(g["log_g"], ref["log_g"], torch.bfloat16, "dlog_g")
+    assert_close(g["initial_state"], ref["initial_state"], torch.bfloat16, "d initial state")
+    assert_close(g["erase_b"].sum(-1) + g["write_w"].sum(-1), ref["beta"], torch.bfloat16, "sum d b + d w = d beta")
+
+
+@pytest.mark.parametrize("variant", ["kda", "gdn2"])
+def test_backward_decay_beyond_the_guard_is_reported(variant):
+    """A decay of e^-5 per token on every channel spans 2^230 within a chunk:
+    the backward returns normally and reports GDR_ERR_RANGE."""
+    d = to_dev(make_inputs(variant, 1, 130, 2, seed=32))
     d["log_g"] = torch.full_like(d["log_g"], -5.0)
     dO = random_output_grad(1, 130, 2, 128, 33).cuda()
     gdr.device_status()
-    gdr.backward(d["q"], d["k"], d["v"], dO, variant="kda", beta=d["beta"], log_g=d["log_g"])
+    gdr.backward(d["q"], d["k"], d["v"], dO, variant=variant, **gates(d))
     with pytest.raises(gdr.GdrError) as e:
         gdr.device_status()
     assert e.value.status == 6, str(e.value)
