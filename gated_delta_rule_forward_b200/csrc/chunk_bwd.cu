@@ -601,10 +601,10 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   const float *dS = p.dss + rc * DK * DV;
   auto row = [&](int t) { return (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h; };
   // GDN-2 scratch: [I - A^d | P^d | dA^d] (C x C each) and [da | dd] (C x d_k), (d o f) dS (C x d_v)
-  float *scZ = reinterpret_cast<float *>(p.scr_f + static_cast<size_t>(blockIdx.x) * p.rb_f);
-  float *scPd = scZ + C * C, *scAd = scPd + C * C;
-  float *scDa = reinterpret_cast<float *>(p.scr_r + rc * p.rb_r);
-  float *scDd = scDa + C * DK, *scDv = scDd + C * DK;
+  float *scZ = G2 ? reinterpret_cast<float *>(p.scr_f + static_cast<size_t>(blockIdx.x) * p.rb_f) : nullptr;
+  float *scPd = G2 ? scZ + C * C : nullptr, *scAd = G2 ? scPd + C * C : nullptr;
+  float *scDa = G2 ? reinterpret_cast<float *>(p.scr_r + rc * p.rb_r) : nullptr;
+  float *scDd = G2 ? scDa + C * DK : nullptr, *scDv = G2 ? scDd + C * DK : nullptr;
 
   // ---- inputs: bf16 tiles (zero past T)
 #pragma unroll
