@@ -167,6 +167,22 @@ __device__ __forceinline__ float at(const FacG<TR, GM> &m, int r, int c) {
   return __bfloat162float(m.x[t * m.ld + i]) * gt * ex2(m.sg * (m.g[t * LDG + i] - m.ref[i]));
 }
 
+// ... or such a gated key tile staged in shared memory as fp32 (rows of LDG).
+template <bool TR>
+struct FacF {
+  using elem = float;
+  static constexpr bool kTr = TR;
+  static constexpr bool kGlobal = false;
+  static constexpr bool kExact = false;
+  const float *x, *g, *ref;
+  float sg;
+};
+template <bool TR>
+__device__ __forceinline__ float at(const FacF<TR> &m, int r, int c) {
+  const int t = TR ? c : r, i = TR ? r : c;
+  return m.x[t * LDG + i] * ex2(m.sg * (m.g[t * LDG + i] - m.ref[i]));
+}
+
 // The warp tile of rows m0 .. m0 + 15 and columns n0 .. n0 + 8 NT - 1 of an M x N
 // product shared by W warps.
 template <int M, int N, int W = 8>
@@ -762,12 +778,40 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   auto afac = [&](const float *ref, float sg) { return FacG<false, 1>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
   auto dfac = [&](const float *ref, float sg) { return FacG<false, 2>{sK, LDB, n, sgam, ref, sg, ebp, wwp, gld}; };
   auto gate = [&](const float *gp, int t, int i) { return t < n ? __ldg(gp + t * gld + i) : 0.f; };
+  // At d_v = 128 the gated key tiles a = b o k and d = (w - b) o k are staged in
+  // shared memory (fp32, rows of LDG) where a region of that size is free: for
+  // the two Gram products, for P^a and P^d, and for the dk and dq products.
+  constexpr bool GST = G2 && DV == 128;
+  auto stage_gated = [&](float *ta, float *td) {
+#pragma unroll
+    for (int u = tid; u < C * DK / 4; u += NTL) {
+      const int t = u / (DK / 4), i4 = 4 * (u % (DK / 4));
+      float4 e4 = make_float4(0.f, 0.f, 0.f, 0.f), w4 = e4;
+      if (t < n) {
+        e4 = __ldg(reinterpret_cast<const float4 *>(ebp + t * gld + i4));
+        w4 = __ldg(reinterpret_cast<const float4 *>(wwp + t * gld + i4));
+      }
+      const float k0 = __bfloat162float(sK[t * LDB + i4]), k1 = __bfloat162float(sK[t * LDB + i4 + 1]),
+                  k2 = __bfloat162float(sK[t * LDB + i4 + 2]), k3 = __bfloat162float(sK[t * LDB + i4 + 3]);
+      if (ta != nullptr)
+        *reinterpret_cast<float4 *>(ta + t * LDG + i4) = make_float4(e4.x * k0, e4.y * k1, e4.z * k2, e4.w * k3);
+      if (td != nullptr)
+        *reinterpret_cast<float4 *>(td + t * LDG + i4) =
+            make_float4((w4.x - e4.x) * k0, (w4.y - e4.y) * k1, (w4.z - e4.z) * k2, (w4.w - e4.w) * k3);
+    }
+  };
+  // the staged tiles' views (regions: E and W at the start and at the end, W and dE for P^a and P^d)
+  auto fsT = [&](const float *tile, const float *ref, float sg) { return FacF<true>{tile, sgam, ref, sg}; };
 
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
     float g[CC::NT][4];
     zero(g);
-    if constexpr (G2) {
+    if constexpr (GST) {
+      stage_gated(sE, sW);
+      __syncthreads();
+      wmm<CC::NT, false>(g, kfac(sgm, 1.f), fsT(sE, sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (G2) {
       wmm<CC::NT, false>(g, kfac(sgm, 1.f), afacT(sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
@@ -791,7 +835,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     {
       float g[CC::NT][4];
       zero(g);
-      wmm<CC::NT, false>(g, kfac(sgm, 1.f), dfacT(sgm, -1.f), DK, mc, nc, lane);
+      if constexpr (GST) {
+        wmm<CC::NT, false>(g, kfac(sgm, 1.f), fsT(sW, sgm, -1.f), DK, mc, nc, lane);
+      } else {
+        wmm<CC::NT, false>(g, kfac(sgm, 1.f), dfacT(sgm, -1.f), DK, mc, nc, lane);
+      }
       each(g, mc, nc, lane,
            [&](int t, int r, float &x) { scZ[t * C + r] = r == t ? 1.f : (r < t ? -x : 0.f); });
     }
@@ -853,13 +901,19 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   }
   each(dqT, mt, nt, lane, [&](int i, int t, float &x) { x *= p.scale * (CHAN ? ex2(sgam[t * LDG + i]) : see[t]); });
   __syncthreads();   // S0's staging is read: P may overwrite it
+  if constexpr (GST) {   // a over W (dead since E), d over dE (nothing yet) for P^a and P^d
+    stage_gated(sW, sdE);
+    __syncthreads();
+  }
   // ---- dE = Diag(f) K dS + P^T dO, P = scale tril(D o Q K^T) (into dP's tile first).  The
   // reverse carry's own dE is Diag(beta) dE (its records carry beta in P and Kt), so it is
   // recomputed here rather than divided by beta.
   {
     float gq[CC::NT][4];
     zero(gq);
-    if constexpr (G2) {
+    if constexpr (GST) {
+      wmm<CC::NT, false>(gq, qa(), fsT(sW, sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (G2) {
       wmm<CC::NT, false>(gq, qa(), afacT(sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
@@ -873,7 +927,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   if constexpr (G2) {   // P^d to scratch
     float gq[CC::NT][4];
     zero(gq);
-    wmm<CC::NT, false>(gq, qa(), dfacT(sgm, -1.f), DK, mc, nc, lane);
+    if constexpr (GST) {
+      wmm<CC::NT, false>(gq, qa(), fsT(sdE, sgm, -1.f), DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(gq, qa(), dfacT(sgm, -1.f), DK, mc, nc, lane);
+    }
     each(gq, mc, nc, lane, [&](int t, int r, float &x) { scPd[t * C + r] = r <= t ? p.scale * x : 0.f; });
   }
   __syncthreads();
@@ -1195,11 +1253,20 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   __syncthreads();
   // ---- dk += N1 K + N1^T K + N2^T Q   (as K^T N1^T, K^T N1, Q^T N2)
   if constexpr (G2) {
+    if constexpr (GST) {   // a over E (X is dead), d over W (dW^T is dead)
+      stage_gated(sE, sW);
+      __syncthreads();
+    }
     {   // dKa = dA (a o b) + dA^d (d o b): dk += a_ o dKa, dg += dKa o Ka
       float acc[KC::NT][4];
       zero(acc);
-      wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
-      wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{scAd, C}, C, mt, nt, lane);
+      if constexpr (GST) {
+        wmm<KC::NT, false>(acc, fsT(sE, sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
+        wmm<KC::NT, false>(acc, fsT(sW, sgm, -1.f), FT{scAd, C}, C, mt, nt, lane);
+      } else {
+        wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
+        wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{scAd, C}, C, mt, nt, lane);
+      }
       each_je(acc, mt, nt, lane, [&](int j, int e, int i, int t, float &x) {
         x *= ex2(sgam[t * LDG + i] - sgm[i]);
         add_dg(j, e, x * __bfloat162float(sK[t * LDB + i]));
@@ -1222,8 +1289,13 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     {   // dq += a_ o (N2a (a o b) + N2d (d o b))
       float acc[KC::NT][4];
       zero(acc);
-      wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
-      wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{sT, LD}, C, mt, nt, lane);
+      if constexpr (GST) {
+        wmm<KC::NT, false>(acc, fsT(sE, sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+        wmm<KC::NT, false>(acc, fsT(sW, sgm, -1.f), FT{sT, LD}, C, mt, nt, lane);
+      } else {
+        wmm<KC::NT, false>(acc, afacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+        wmm<KC::NT, false>(acc, dfacT(sgm, -1.f), FT{sT, LD}, C, mt, nt, lane);
+      }
       each_je(acc, mt, nt, lane,
               [&](int j, int e, int i, int t, float &x) { dqT[j][e] += x * ex2(sgam[t * LDG + i] - sgm[i]); });
     }
