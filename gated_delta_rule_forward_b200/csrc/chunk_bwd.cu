@@ -802,6 +802,36 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   };
   // the staged tiles' views (regions: E and W at the start and at the end, W and dE for P^a and P^d)
   auto fsT = [&](const float *tile, const float *ref, float sg) { return FacF<true>{tile, sgam, ref, sg}; };
+  // KDA at d_v = 128: the factored tiles x o 2^(sg (gamma - ref)) (x = K, or Q) staged whole as fp32
+  // (rows of LDG) where a region of that size is free, the same values the factored views compute
+  constexpr bool KST = CHAN && !G2 && DV == 128;
+  auto stage_fac = [&](float *dst, bool from_q, const float *ref, float sg) {
+#pragma unroll
+    for (int u = tid; u < C * DK / 4; u += NTL) {
+      const int t = u / (DK / 4), i4 = 4 * (u % (DK / 4));
+      float x[4];
+      if (from_q) {
+        if constexpr (QVG) {
+          uint2 raw = make_uint2(0u, 0u);
+          if (t < n) raw = __ldg(reinterpret_cast<const uint2 *>(p.q + row(t) * DK + i4));
+          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+          const float2 a0 = __bfloat1622float2(h2[0]), a1 = __bfloat1622float2(h2[1]);
+          x[0] = a0.x; x[1] = a0.y; x[2] = a1.x; x[3] = a1.y;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = __bfloat162float(sQ[t * LDB + i4 + e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __bfloat162float(sK[t * LDB + i4 + e]);
+      }
+      const float4 g4 = *reinterpret_cast<const float4 *>(sgam + t * LDG + i4);
+      const float4 r4 = *reinterpret_cast<const float4 *>(ref + i4);
+      *reinterpret_cast<float4 *>(dst + t * LDG + i4) =
+          make_float4(x[0] * ex2(sg * (g4.x - r4.x)), x[1] * ex2(sg * (g4.y - r4.y)), x[2] * ex2(sg * (g4.z - r4.z)),
+                      x[3] * ex2(sg * (g4.w - r4.w)));
+    }
+  };
 
   // ---- A = tril(Diag(beta) (D o K K^T), -1), stored transposed and tf32-rounded for the solve
   {
@@ -813,6 +843,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       wmm<CC::NT, false>(g, kfac(sgm, 1.f), fsT(sE, sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (G2) {
       wmm<CC::NT, false>(g, kfac(sgm, 1.f), afacT(sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (KST) {   // K o a_ over E, K o b over W
+      stage_fac(sE, false, sgm, 1.f);
+      stage_fac(sW, false, sgm, -1.f);
+      __syncthreads();
+      wmm1<CC::NT, false>(g, F{sE, LDG}, FT{sW, LDG}, DK, mc, nc, lane);
     } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
@@ -863,6 +898,10 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     zero(w);
     if constexpr (G2) {
       wmm<CK::NT, false>(w, TX{sT, LD}, kfac(szero, 1.f), C, mk, nk, lane);
+    } else if constexpr (KST) {   // K o e over E (E not yet computed)
+      stage_fac(sE, false, szero, 1.f);
+      __syncthreads();
+      wmm<CK::NT, false>(w, TX{sT, LD}, F{sE, LDG}, C, mk, nk, lane, sbeta);
     } else if constexpr (CHAN) {
       wmm<CK::NT, false>(w, TX{sT, LD}, kfac(szero, 1.f), C, mk, nk, lane, sbeta);
     } else {
@@ -915,6 +954,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       wmm<CC::NT, false>(gq, qa(), fsT(sW, sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (G2) {
       wmm<CC::NT, false>(gq, qa(), afacT(sgm, -1.f), DK, mc, nc, lane);
+    } else if constexpr (KST) {   // Q o a_ over W (dead since E), K o b over dE (nothing yet)
+      stage_fac(sW, true, sgm, 1.f);
+      stage_fac(sdE, false, sgm, -1.f);
+      __syncthreads();
+      wmm1<CC::NT, false>(gq, F{sW, LDG}, FT{sdE, LDG}, DK, mc, nc, lane);
     } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(gq, qa(), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
@@ -1179,7 +1223,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     zero(a1);
     zero(a2);
     wmm1<CC::NT, false>(a1, F{sdE, LDF}, vmT(), DV, mc, nc, lane);
-    if constexpr (CHAN) {
+    if constexpr (KST) {   // K o e over E (dead since dW)
+      stage_fac(sE, false, szero, 1.f);
+      __syncthreads();
+      wmm1<CC::NT, false>(a2, FT{sW, LDC}, FT{sE, LDG}, DK, mc, nc, lane);
+    } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
     } else {
       wmm1<CC::NT, false>(a2, FT{sW, LDC}, BKT{sK, LDB}, DK, mc, nc, lane);
@@ -1228,9 +1276,17 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     wmm<CC::NT, false>(acc, BK{sO, LDBV}, vmT(), DV, mc, nc, lane);
     each(acc, mc, nc, lane, [&](int t, int r, float &x) { sT[t * LD + r] = r <= t ? p.scale * x : 0.f; });
   } else {
+    if constexpr (KST) {   // K o a_ over E (X is dead), K o b over W (dW^T is dead), Q o a_ over dE
+      stage_fac(sE, false, sgm, 1.f);
+      stage_fac(sW, false, sgm, -1.f);
+      stage_fac(sdE, true, sgm, 1.f);
+      __syncthreads();
+    }
     float g[CC::NT][4];
     zero(g);
-    if constexpr (CHAN) {
+    if constexpr (KST) {
+      wmm1<CC::NT, false>(g, F{sE, LDG}, FT{sW, LDG}, DK, mc, nc, lane);
+    } else if constexpr (CHAN) {
       wmm1<CC::NT, false>(g, kfac(sgm, 1.f), kfacT(sgm, -1.f), DK, mc, nc, lane);
     } else {
       wmm<CC::NT, false>(g, BK{sK, LDB}, BKT{sK, LDB}, DK, mc, nc, lane);
@@ -1313,7 +1369,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   } else {
     float acc[KC::NT][4];
     zero(acc);
-    if constexpr (CHAN) {
+    if constexpr (KST) {
+      wmm<KC::NT, false>(acc, FT{sW, LDG}, FT{sA, LD}, C, mt, nt, lane);
+    } else if constexpr (CHAN) {
       wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sA, LD}, C, mt, nt, lane);
     } else {
       wmm1<KC::NT, false>(acc, BKT{sK, LDB}, FT{sA, LD}, C, mt, nt, lane);
@@ -1324,7 +1382,10 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       dkT[j][e] += x;
     });
     zero(acc);
-    if constexpr (CHAN) {
+    if constexpr (KST) {
+      wmm<KC::NT, false>(acc, FT{sE, LDG}, F{sA, LD}, C, mt, nt, lane);
+      wmm<KC::NT, false>(acc, FT{sdE, LDG}, F{sP, LDC}, C, mt, nt, lane);
+    } else if constexpr (CHAN) {
       wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
       wmm<KC::NT, false>(acc, qaT(), F{sP, LDC}, C, mt, nt, lane);
     } else {
@@ -1342,7 +1403,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   } else if constexpr (CHAN) {
     float acc[KC::NT][4];
     zero(acc);
-    wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+    if constexpr (KST) {
+      wmm<KC::NT, false>(acc, FT{sW, LDG}, FT{sP, LDC}, C, mt, nt, lane);
+    } else {
+      wmm<KC::NT, false>(acc, kfacT(sgm, -1.f), FT{sP, LDC}, C, mt, nt, lane);
+    }
     each_je(acc, mt, nt, lane,
             [&](int j, int e, int i, int t, float &x) { dqT[j][e] += x * ex2(sgam[t * LDG + i] - sgm[i]); });
   } else {
