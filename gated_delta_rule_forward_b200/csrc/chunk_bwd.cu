@@ -837,10 +837,11 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   {
     float g[CC::NT][4];
     zero(g);
-    if constexpr (GST) {
+    if constexpr (GST) {   // a over E, d over W, K o a_ over dE (nothing yet)
       stage_gated(sE, sW);
+      stage_fac(sdE, false, sgm, 1.f);
       __syncthreads();
-      wmm<CC::NT, false>(g, kfac(sgm, 1.f), fsT(sE, sgm, -1.f), DK, mc, nc, lane);
+      wmm<CC::NT, false>(g, F{sdE, LDG}, fsT(sE, sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (G2) {
       wmm<CC::NT, false>(g, kfac(sgm, 1.f), afacT(sgm, -1.f), DK, mc, nc, lane);
     } else if constexpr (KST) {   // K o a_ over E, K o b over W
@@ -871,7 +872,7 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       float g[CC::NT][4];
       zero(g);
       if constexpr (GST) {
-        wmm<CC::NT, false>(g, kfac(sgm, 1.f), fsT(sW, sgm, -1.f), DK, mc, nc, lane);
+        wmm<CC::NT, false>(g, F{sdE, LDG}, fsT(sW, sgm, -1.f), DK, mc, nc, lane);
       } else {
         wmm<CC::NT, false>(g, kfac(sgm, 1.f), dfacT(sgm, -1.f), DK, mc, nc, lane);
       }
@@ -1213,8 +1214,15 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
       each(a1, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = x; });
     }
     zero(a2);
-    wmm<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
-    __syncthreads();
+    if constexpr (GST) {   // K o e over E, once every warp has read tU there
+      __syncthreads();
+      stage_fac(sE, false, szero, 1.f);
+      __syncthreads();
+      wmm<CC::NT, false>(a2, FT{sW, LDC}, FT{sE, LDG}, DK, mc, nc, lane);
+    } else {
+      wmm<CC::NT, false>(a2, FT{sW, LDC}, kfacT(szero, 1.f), DK, mc, nc, lane);
+      __syncthreads();
+    }
     wmm<CC::NT, false>(a2, F{sA, LD}, FT{scZ, C}, C, mc, nc, lane);
     __syncthreads();
     each(a2, mc, nc, lane, [&](int t, int r, float &x) { sA[t * LD + r] = x; });
@@ -1309,8 +1317,9 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   __syncthreads();
   // ---- dk += N1 K + N1^T K + N2^T Q   (as K^T N1^T, K^T N1, Q^T N2)
   if constexpr (G2) {
-    if constexpr (GST) {   // a over E (X is dead), d over W (dW^T is dead)
+    if constexpr (GST) {   // a over E (X is dead), d over W (dW^T is dead), K o a_ over dE (dead)
       stage_gated(sE, sW);
+      stage_fac(sdE, false, sgm, 1.f);
       __syncthreads();
     }
     {   // dKa = dA (a o b) + dA^d (d o b): dk += a_ o dKa, dg += dKa o Ka
@@ -1332,12 +1341,20 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
     {   // da += b o (dA^T Ka + N2a^T Qa),  dd += b o (dA^d^T Ka + N2d^T Qa)
       float acc[KC::NT][4];
       zero(acc);
-      wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
+      if constexpr (GST) {
+        wmm<KC::NT, false>(acc, FT{sdE, LDG}, F{sA, LD}, C, mt, nt, lane);
+      } else {
+        wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{sA, LD}, C, mt, nt, lane);
+      }
       wmm<KC::NT, false>(acc, qaT(), F{sP, LDC}, C, mt, nt, lane);
       each(acc, mt, nt, lane,
            [&](int i, int t, float &x) { scDa[t * DK + i] += x * ex2(sgm[i] - sgam[t * LDG + i]); });
       zero(acc);
-      wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{scAd, C}, C, mt, nt, lane);
+      if constexpr (GST) {
+        wmm<KC::NT, false>(acc, FT{sdE, LDG}, F{scAd, C}, C, mt, nt, lane);
+      } else {
+        wmm<KC::NT, false>(acc, kfacT(sgm, 1.f), F{scAd, C}, C, mt, nt, lane);
+      }
       wmm<KC::NT, false>(acc, qaT(), F{sT, LD}, C, mt, nt, lane);
       each(acc, mt, nt, lane,
            [&](int i, int t, float &x) { scDd[t * DK + i] += x * ex2(sgm[i] - sgam[t * LDG + i]); });
