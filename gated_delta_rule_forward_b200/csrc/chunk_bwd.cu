@@ -546,9 +546,10 @@ struct LocalSmem {
 //     at the chunk's last token; dlog_g = per-channel suffix sums of dg over the chunk.
 //
 // Precision: fp32 operands are split into two tf32 parts (wmm) except in the
-// products that take one pass (wmm1): dT, X = dT T^T and dA; KDA's factored
-// Gram and P products; and, with scalar decay, the dk and dq products with N1
-// and N2.  Measured against the fp64 oracle (the 350M layer and small ragged
+// products that take one pass (wmm1): dT, X = dT T^T and dA (not for GDN-2,
+// whose d erase is a small difference of gradients built from them); KDA's
+// factored Gram and P products; and, with scalar decay, the dk and dq products
+// with N1 and N2.  Measured against the fp64 oracle (the 350M layer and small ragged
 // and strong-decay cases of every variant), this moved no gradient past 5e-3
 // of its RMS (d log g 6.0e-3 -> 5.8e-3, dk 2.3e-3 -> 4.8e-3); one pass for
 // E, dW or the dE, U', W products moved d log g to 1.5-2.9e-2, and KDA's dk
@@ -570,6 +571,11 @@ struct LocalSmem {
 //     da o a + dd o d summed over the chunk and e^(gamma_C) o rowsum(dS o S0) at its last token.
 // I - A^d, P^d, dA^d, da, dd and the (d o f) dS term go through global scratch: this
 // chunk's slots of the forward and reverse records, which nothing reads any more.
+//
+// At d_v = 128 (KDA and GDN-2) the factored and gated key / query tiles are
+// staged whole in shared memory as fp32 wherever a region of that size is
+// free between its own uses (E, W, dE), so that a fragment element is one
+// load rather than a factor evaluation; elsewhere the views evaluate them.
 constexpr int NTL = 512;
 template <int DV, bool CHAN, bool G2 = false>
 __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) {
@@ -585,8 +591,8 @@ __global__ void __launch_bounds__(NTL, 1) bwd_local_kernel(const LocalParams p) 
   __nv_bfloat16 *sV = reinterpret_cast<__nv_bfloat16 *>(sm + L::V);
   __nv_bfloat16 *sO = reinterpret_cast<__nv_bfloat16 *>(sm + L::O);
   float *sdE = reinterpret_cast<float *>(sm + L::DE);
-  float *sE = reinterpret_cast<float *>(sm + L::E);    // E, later X = dT T^T
-  float *sW = reinterpret_cast<float *>(sm + L::W);    // W, later dW^T
+  float *sE = reinterpret_cast<float *>(sm + L::E);    // E, later X = dT T^T (and staged tiles between)
+  float *sW = reinterpret_cast<float *>(sm + L::W);    // W, later dW^T (and staged tiles between)
   float *sA = reinterpret_cast<float *>(sm + L::A);    // A^T for the solve, later dT, dA, N1
   float *sT = reinterpret_cast<float *>(sm + L::TT);   // T
   float *sP = reinterpret_cast<float *>(sm + L::P);    // dP, later N2
