@@ -264,7 +264,7 @@ size_t gdr_backward_workspace_size(int variant, int dtype, int B, int T, int H, 
  * d_final_state [B,H,dk,dv] fp32 or NULL (zero).  The tensor-core carries use
  * fp16 operands with fp32 accumulation, like the forward's chunked path: the
  * gradients match an exact backward to a few 1e-3 of their RMS (measured
- * worst cases: d log g 1.5e-2 on long channel-decay sequences; GDN-2's gate
+ * worst cases: d log g up to 1.7e-2 on long channel-decay sequences; GDN-2's gate
  * gradients, which the carries' fp16 rounding reaches in proportion to the
  * terms they are built from, ~5e-4 of the largest gradient of a chunk); the
  * gradients are rescaled internally by a power of two so that d_o's range
