@@ -16,7 +16,7 @@ EXPORTS = (
     "gdr_forward_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
     "gdr_forward_launches", "gdr_forward_kernel_name", "gdr_status_string",
     "gdr_last_error", "gdr_version", "gdr_device_status", "gdr_forward_chunked_noalloc",
-    "gdr_forward_plan", "gdr_backward_workspace_size", "gdr_backward",
+    "gdr_forward_plan", "gdr_forward_segment_parts", "gdr_backward_workspace_size", "gdr_backward",
 )
 
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_ALIGNMENT",
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
             L.gdr_forward_launches.restype = i
             L.gdr_forward_plan.argtypes = [i] * 6 + [ctypes.POINTER(i)] * 3
             L.gdr_forward_plan.restype = i
+            L.gdr_forward_segment_parts.argtypes = [i] * 6 + [ctypes.POINTER(i)] * 2
+            L.gdr_forward_segment_parts.restype = i
             L.gdr_forward_kernel_name.argtypes = [i] * 8
             L.gdr_forward_kernel_name.restype = ctypes.c_char_p
             L.gdr_status_string.argtypes = [i]

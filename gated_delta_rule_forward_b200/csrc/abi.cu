@@ -104,7 +104,7 @@ gdr_status_t validate_gates(int variant, const float *beta, const float *log_g, 
 
 extern "C" {
 
-int gdr_version(void) { return 100; }
+int gdr_version(void) { return 101; }
 
 const char *gdr_status_string(gdr_status_t s) {
   switch (s) {
@@ -175,6 +175,18 @@ gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms,
   if (B < 0 || T < 0 || H < 0 || sms < 0) return fail(GDR_ERR_INVALID_ARG, "B, T, H and sms must be >= 0");
   if (!segments || !segment_chunks || !split_chunk) return fail(GDR_ERR_INVALID_ARG, "output pointer is NULL");
   gdr_split_plan(variant, B, T, H, dv, sms, segments, segment_chunks, split_chunk);
+  return GDR_OK;
+}
+
+gdr_status_t gdr_forward_segment_parts(int variant, int B, int T, int H, int dv, int sms, int *parts,
+                                       int *part_chunks) {
+  take_raw(variant);
+  if (!valid_variant(variant)) return fail(GDR_ERR_INVALID_ARG, "unknown variant");
+  if (!valid_dim(dv)) return fail(GDR_ERR_INVALID_ARG, "dv must be 64 or 128");
+  if (B < 0 || T < 0 || H < 0 || sms < 0) return fail(GDR_ERR_INVALID_ARG, "B, T, H and sms must be >= 0");
+  if (!parts || !part_chunks) return fail(GDR_ERR_INVALID_ARG, "output pointer is NULL");
+  int g = 0, l = 0, c = 0;
+  gdr_split_plan(variant, B, T, H, dv, sms, &g, &l, &c, parts, part_chunks);
   return GDR_OK;
 }
 

@@ -1385,6 +1385,7 @@ enum CarryFlags : int {
   CARRY_FAULT_MISSING_COPY = 32,   // host fault injection (see the issuer's prologue)
   CARRY_WRITE_STATES = 64,   // write every chunk's start state to `states` ([B,H,NC,d_k,d_v], fp32)
   CARRY_STATES_F16 = 128,    // ... in fp16 instead: the state as this kernel's MMAs take it
+  CARRY_SNAPSHOTS = 256,     // write the state at every interior chunk c_first + c that is a multiple of snap_len
 };
 
 struct CarryParams {
@@ -1404,6 +1405,11 @@ struct CarryParams {
   size_t s_final_b_seg_stride;
   __nv_bfloat16 *o;
   void *states;    // CARRY_WRITE_STATES output, indexed by (b, h, chunk)
+  // CARRY_SNAPSHOTS: the state at chunk x = n snap_len goes to snap (pass A) or
+  // snap_b (pass B) + (n - 1) snap_stride, packed [B, H, d_k, d_v] within a slot
+  int snap_len;
+  float *snap, *snap_b;
+  size_t snap_stride;
 };
 
 // max |x_i| over 16 values as a tree (four levels instead of a chain of 16).
@@ -1680,6 +1686,12 @@ __global__ void __launch_bounds__(carry::NTHREADS_CARRY, 1) chunk_carry_kernel(c
 #pragma unroll
           for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
         }
+      }
+      if ((flags & CARRY_SNAPSHOTS) && has_v && c > 0 && (c_first + c) % p.snap_len == 0) {
+        float *dst = (pass_b ? p.snap_b : p.snap) + static_cast<size_t>((c_first + c) / p.snap_len - 1) * p.snap_stride +
+                     ((static_cast<size_t>(b) * p.H + h) * DK + 32 * part) * p.dv + v;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) dst[static_cast<size_t>(k) * p.dv] = S[k];
       }
 
       // E^T = U'^T + Y_W, tokens 16 part .. 16 part + 15; U'^T is read from the
@@ -2003,48 +2015,143 @@ cudaError_t launch_prep_chan(const FwdProblem &p, int NC, uint8_t *ws, const Pre
   return e;
 }
 
-// Segment-start states for one (b, h) and 16 value columns per CTA, in fp32:
+// Start states of phase 2's parts (see SegPlan), for one (b, h) and 16 value
+// columns per CTA, in fp32.  The segment starts form the chain
 //     S_start[0] = s0 (zeros if null),  S_start[1] = D_0,
-//     S_start[g + 1] = M_g S_start[g] + D_g  (g = 1 .. G - 2).
-// D_0 is segment 0's end state from s0 itself; for g >= 1, M_g is the transition
-// map of segment g (the carry from the identity with the values taken as zero,
-// d_k x d_k, stored at index g - 1) and D_g its end state from zero (d_k x d_v).
-__global__ void __launch_bounds__(256) segment_chain_kernel(const float *s0, const float *M, const float *D,
-                                                            float *S_start, int G, int H, int dv) {
-  __shared__ float Sc[DK][16];
+//     S_start[g + 1] = M_g S_start[g] + D_g  (g = 1 .. G - 2),
+// where D_0 is segment 0's end state from s0 itself and, for g >= 1, M_g is the
+// transition map of segment g (the carry from the identity with the values
+// taken as zero, d_k x d_k, stored at index g - 1) and D_g its end state from
+// zero (d_k x d_v).  A part that starts j chunks into segment g (0 < j < L)
+// starts from the same affine map after j chunks, which phase 1 leaves as
+// snapshots of both carries: S = M_g(j) S_start[g] + D_g(j), or D_0(j) itself
+// in segment 0.  `items` lists the steps in order: a chain step (0x8000 | part
+// << 8 | g) forms S_start[g + 1] and, where a part starts there, writes it as
+// that part's state; a part step (its index) forms a part inside a segment.
+// Part 0 is S_start[0].
+struct ChainItems {
+  static constexpr int kMax = 16 + 64;
+  int n = 0;
+  uint16_t it[kMax];
+};
+namespace chain {
+constexpr int NT = 512;                         // threads: 32 row groups x 16 k-slices
+constexpr int SC_FLOATS = DK * 16 + (DK / 8) * 4;   // S_start[g] for 16 columns, padded (see sc_at)
+constexpr size_t SMEM_BYTES = 2 * 8 * NT * 16;  // two steps' maps, 8 float4 per thread
+// Row k of the 16-column start state: the 16 k-slices of a warp read rows 8
+// apart, so each group of 8 rows is shifted by 4 banks.
+__device__ __forceinline__ int sc_at(int k) { return k * 16 + (k >> 3) * 4; }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+}  // namespace chain
+// Each thread forms a 4 x 16 block of the product (rows 4 rg .. 4 rg + 3, the
+// CTA's 16 columns) over its 8-wide k-slice; the 16 k-slices of a row group
+// (half a warp) then sum by shuffles, each lane keeping 4 of the 64 values.
+// The maps of the next step are copied into shared memory (each thread its
+// own 8 float4) while the current one is formed.
+__global__ void __launch_bounds__(chain::NT, 1) segment_chain_kernel(const float *s0, const float *M, const float *D,
+                                                                    const float *snapM, const float *snapD,
+                                                                    float *S_part, const ChainItems items, int L,
+                                                                    int Lp, int H, int dv) {
+  using namespace chain;
+  __shared__ __align__(16) float Sc[SC_FLOATS];
+  extern __shared__ float4 stage[];   // [2][8][NT]
   const int sl = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const size_t BH = static_cast<size_t>(gridDim.z) * H, bh = static_cast<size_t>(b) * H + h;
-  for (int e = tid; e < DK * 16; e += blockDim.x) {
-    const int i = e >> 4, j = e & 15;
-    const size_t at = (bh * DK + i) * dv + 16 * sl + j;
-    const float x = s0 != nullptr ? s0[at] : 0.f;
-    Sc[i][j] = x;
-    S_start[at] = x;
+  const size_t slot = BH * DK * dv, mslot = BH * DK * DK;
+  const int rg = tid >> 4, ks = tid & 15;
+  const int r0 = 4 * rg, kb = 8 * ks;
+  // after the reduction: row 4 rg + ks / 4, columns 4 (ks % 4) .. + 3 of the CTA's 16
+  const int orow = r0 + (ks >> 2), ocol = 4 * (ks & 3);
+  const size_t at = (bh * DK + orow) * dv + 16 * sl + ocol;
+  for (int e = tid; e < DK * 16; e += NT) {
+    const int k = e >> 4, j = e & 15;
+    const size_t a = (bh * DK + k) * dv + 16 * sl + j;
+    const float x = s0 != nullptr ? s0[a] : 0.f;
+    Sc[sc_at(k) + j] = x;
+    S_part[a] = x;
   }
-  __syncthreads();
-  const int i = tid >> 1, j0 = 8 * (tid & 1);
-  for (int g = 0; g + 1 < G; ++g) {
-    const size_t at = ((g * BH + bh) * DK + i) * dv + 16 * sl + j0;
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = D[at + j];
-    const float *Mi = g > 0 ? M + (((g - 1) * BH + bh) * DK + i) * DK : nullptr;
-    for (int k = 0; g > 0 && k < DK; k += 4) {
-      const float4 m = __ldg(reinterpret_cast<const float4 *>(Mi + k));
+  // the map of step n, or null where the step copies
+  auto map_of = [&](int n) -> const float * {
+    const int it = items.it[n];
+    const int g = (it & 0x8000) ? (it & 0xff) : it * Lp / L;
+    if (g == 0) return nullptr;
+    return (it & 0x8000) ? M + (g - 1) * mslot : snapM + (it - 1) * mslot;
+  };
+  // this thread's part of a map: float4 j = 2 rho + half is M[r0 + rho][kb + 4 half .. + 3]
+  auto fetch = [&](int n, int buf) {
+    const float *m = n < items.n ? map_of(n) : nullptr;
+    if (m != nullptr) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        acc[j] = fmaf(m.x, Sc[k][j0 + j], fmaf(m.y, Sc[k + 1][j0 + j],
-                 fmaf(m.z, Sc[k + 2][j0 + j], fmaf(m.w, Sc[k + 3][j0 + j], acc[j]))));
+        cp_async16(&stage[(buf * 8 + j) * NT + tid], m + (bh * DK + r0 + (j >> 1)) * DK + kb + 4 * (j & 1));
     }
-    __syncthreads();
-    const size_t out = (((g + 1) * BH + bh) * DK + i) * dv + 16 * sl + j0;
+    cp_async_commit();
+  };
+  fetch(0, 0);
+  __syncthreads();
+  for (int n = 0; n < items.n; ++n) {
+    const int it = items.it[n];
+    const bool chain_step = (it & 0x8000) != 0;
+    const bool has_map = map_of(n) != nullptr;   // uniform over the CTA
+    fetch(n + 1, (n + 1) & 1);
+    const float *Dp = chain_step ? D + (it & 0xff) * slot : snapD + (it - 1) * slot;
+    const float4 dd = __ldg(reinterpret_cast<const float4 *>(Dp + at));
+    float acc[64];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      Sc[i][j0 + j] = acc[j];
-      S_start[out + j] = acc[j];
+    for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+    cp_async_wait_one();   // this step's map (the thread's own copies)
+    if (has_map) {
+      const float4 *st = stage + (n & 1) * 8 * NT + tid;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float4 mr[4];
+#pragma unroll
+        for (int rho = 0; rho < 4; ++rho) mr[rho] = st[(2 * rho + half) * NT];
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const float4 *sr = reinterpret_cast<const float4 *>(&Sc[sc_at(kb + 4 * half + kq)]);
+          float sv[16];
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 x = sr[j4];
+            sv[4 * j4] = x.x; sv[4 * j4 + 1] = x.y; sv[4 * j4 + 2] = x.z; sv[4 * j4 + 3] = x.w;
+          }
+#pragma unroll
+          for (int rho = 0; rho < 4; ++rho) {
+            const float m = kq == 0 ? mr[rho].x : kq == 1 ? mr[rho].y : kq == 2 ? mr[rho].z : mr[rho].w;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc[16 * rho + c] = fmaf(m, sv[c], acc[16 * rho + c]);
+          }
+        }
+      }
     }
-    __syncthreads();
+    // sum over the 16 k-slices: each round keeps the half of the values that
+    // its lane bit selects; lane ks ends with values 4 ks .. 4 ks + 3
+#pragma unroll
+    for (int w = 32, mask = 8; w >= 4; w >>= 1, mask >>= 1) {
+      const bool up = (ks & mask) != 0;
+#pragma unroll
+      for (int e = 0; e < w; ++e) {
+        const float send = up ? acc[e] : acc[w + e];
+        acc[e] = (up ? acc[w + e] : acc[e]) + __shfl_xor_sync(0xffffffffu, send, mask);
+      }
+    }
+    const float4 out = make_float4(acc[0] + dd.x, acc[1] + dd.y, acc[2] + dd.z, acc[3] + dd.w);
+    if (chain_step) {
+      __syncthreads();   // every thread is done reading S_start[g]
+      *reinterpret_cast<float4 *>(&Sc[sc_at(orow) + ocol]) = out;
+      const int part = (it >> 8) & 0x7f;
+      if (part > 0) *reinterpret_cast<float4 *>(S_part + part * slot + at) = out;
+      __syncthreads();
+    } else {
+      *reinterpret_cast<float4 *>(S_part + it * slot + at) = out;
+    }
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 struct CarryLaunch {
@@ -2059,6 +2166,9 @@ struct CarryLaunch {
   float *s_final_b = nullptr;
   size_t s_final_b_stride = 0;
   void *states = nullptr;    // CARRY_WRITE_STATES output
+  int snap_len = 0;          // CARRY_SNAPSHOTS
+  float *snap = nullptr, *snap_b = nullptr;
+  size_t snap_stride = 0;
 };
 
 // `pdl`: launched with programmatic stream serialization, so that its CTAs may
@@ -2090,6 +2200,7 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
   cp.s_final_b = l.s_final_b; cp.s_final_b_seg_stride = l.s_final_b_stride;
   cp.o = static_cast<__nv_bfloat16 *>(p.o);
   cp.states = l.states;
+  cp.snap_len = l.snap_len; cp.snap = l.snap; cp.snap_b = l.snap_b; cp.snap_stride = l.snap_stride;
   // GDR_FAULT=wait (host-side fault injection for the failure-path tests): CTA
   // (0, 0, 0) never copies chunk 1's record, so its waits give up after their
   // limit (about a second).
@@ -2111,11 +2222,23 @@ cudaError_t launch_carry(const FwdProblem &p, int NC, const uint8_t *ws, const C
 // D_0 is already S_start[1] and segment 0 needs no M; M_g (g >= 1) is the
 // carry from the identity with the values taken as zero.  That is 2G - 3
 // state-only CTAs per (b, h), all resident at once.  A chain kernel turns the
-// maps into segment start states; phase 2 runs every segment from its start
-// with outputs.  The sequential depth drops from NC chunks to about 2 NC / G.
+// maps into start states; phase 2 runs the sequence from them with outputs.
+//
+// Phase 2 needs one CTA per part where phase 1 needs about two per segment, so
+// it may cut the sequence finer: P parts of Lp chunks.  A part that starts
+// inside segment g (g < G - 1) starts from the segment's map and offset after
+// the chunks before it, which phase 1's two carries leave there as snapshots;
+// no part may start inside the last segment, which phase 1 does not run.  The
+// plan minimises the sequential time in units of about 0.4 us, measured on the
+// 64k-token sweep: a phase-1 chunk (no outputs) 4, a phase-2 chunk 5, a
+// product of the chain 10.  The sequential depth drops from NC chunks to about
+// L + Lp.
 struct SegPlan {
-  int G = 1, L = 0;
+  int G = 1, L = 0;    // phase 1: segments of L chunks
+  int P = 1, Lp = 0;   // phase 2: parts of Lp chunks (P = G, Lp = L unless cut finer)
+  bool finer() const { return G > 1 && Lp != L; }
 };
+constexpr int kMaxParts = 64;
 // SMs of the current device, 0 if there is none.
 int device_sms() {
   int dev = 0, sms = 0;
@@ -2125,6 +2248,14 @@ int device_sms() {
     return 0;
   }
   return sms;
+}
+// Products the chain kernel forms for a plan: one per segment start after the
+// second, one per part starting strictly inside a segment other than the first.
+int seg_products(int G, int L, int P, int Lp) {
+  int n = G - 2;
+  for (int p = 1; p < P; ++p)
+    if (p * Lp >= L && (p * Lp) % L != 0) ++n;
+  return n;
 }
 SegPlan seg_plan_for(int B, int H, int dv, int NC, int sms) {
   SegPlan sp;
@@ -2136,16 +2267,54 @@ SegPlan seg_plan_for(int B, int H, int dv, int NC, int sms) {
   if (G < 3) return sp;
   sp.L = (NC + G - 1) / G;
   sp.G = (NC + sp.L - 1) / sp.L;
+  sp.P = sp.G;
+  sp.Lp = sp.L;
+  auto cost = [](int G1, int L1, int P, int Lp) { return 4LL * L1 + 5LL * Lp + 10LL * seg_products(G1, L1, P, Lp); };
+  long long best = cost(sp.G, sp.L, sp.P, sp.Lp);
+  const int pmax = static_cast<int>(std::min<long long>(std::min<long long>(sms / bh, NC), kMaxParts));
+  const SegPlan base = sp;
+  for (int P0 = base.G + 1; P0 <= pmax; ++P0) {
+    const int Lp = (NC + P0 - 1) / P0, P = (NC + Lp - 1) / Lp;
+    if (P <= base.G) continue;
+    // the shortest phase-1 segments that leave no part start inside the last one
+    for (int L1 = base.L; L1 <= base.L + Lp; ++L1) {
+      const int G1 = (NC + L1 - 1) / L1;
+      if (G1 < 3) break;
+      if (static_cast<long long>(G1 - 1) * L1 < static_cast<long long>(P - 1) * Lp) continue;
+      const long long c = cost(G1, L1, P, Lp);
+      if (c < best) {
+        best = c;
+        sp.G = G1; sp.L = L1; sp.P = P; sp.Lp = Lp;
+      }
+      break;
+    }
+  }
   return sp;
 }
 SegPlan seg_plan(int B, int H, int dv, int NC) {
   if (dv != 128 || NC < 64) return seg_plan_for(B, H, dv, NC, 0);
   return seg_plan_for(B, H, dv, NC, device_sms());
 }
+// The chain kernel's steps for a plan (see segment_chain_kernel); false if a
+// part would start inside the last segment.
+bool chain_items(const SegPlan &sp, ChainItems *ci) {
+  ci->n = 0;
+  int p = 1;
+  for (int g = 0; g + 1 < sp.G; ++g) {
+    for (; p < sp.P && p * sp.Lp < (g + 1) * sp.L; ++p) ci->it[ci->n++] = static_cast<uint16_t>(p);
+    int at_start = 0;
+    if (p < sp.P && p * sp.Lp == (g + 1) * sp.L) at_start = p++;
+    ci->it[ci->n++] = static_cast<uint16_t>(0x8000 | (at_start << 8) | g);
+  }
+  return p == sp.P;
+}
+// Floats of the maps, offsets, part start states and snapshots.
 size_t seg_extra_floats(int B, int H, int dv, const SegPlan &sp) {
   if (sp.G == 1) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
-  return (sp.G - 2) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.G * bh * DK * dv;
+  size_t n = (sp.G - 2) * bh * DK * DK + (sp.G - 1) * bh * DK * dv + sp.P * bh * DK * dv;
+  if (sp.finer()) n += (sp.P - 1) * bh * (DK * dv + DK * DK);
+  return n;
 }
 
 // Pipelined sweep.  The carry runs B*H CTAs, one per SM, and leaves the other
@@ -2250,9 +2419,16 @@ cudaError_t launch_segmented(const FwdProblem &p, int NC, const SegPlan &sp, con
                              const float *s0, float *s_final, int flags2, void *states, cudaStream_t stream,
                              std::string *err) {
   const size_t bh = static_cast<size_t>(p.B) * p.H;
+  ChainItems items;
+  if (!chain_items(sp, &items)) {
+    *err = "segment plan: ";
+    return cudaErrorInvalidValue;
+  }
   float *Mb = reinterpret_cast<float *>(maps);
   float *Db = Mb + (sp.G - 2) * bh * DK * DK;
   float *Ss = Db + (sp.G - 1) * bh * DK * p.dv;
+  float *snapD = Ss + sp.P * bh * DK * p.dv;               // used when the parts are finer
+  float *snapM = snapD + (sp.P - 1) * bh * DK * p.dv;
   CarryLaunch m;   // phase 1, pass A: end states of segments 0 .. G-2 (segment 0 from s0, the rest from zero)
   m.segments = sp.G - 1; m.seg_len = sp.L;
   m.flags = CARRY_NO_OUTPUT | CARRY_S0_FIRST;
@@ -2262,16 +2438,30 @@ cudaError_t launch_segmented(const FwdProblem &p, int NC, const SegPlan &sp, con
   m.segments_b = sp.G - 2; m.seg_first_b = 1;
   m.flags_b = CARRY_IDENTITY | CARRY_NO_VALUES | CARRY_NO_OUTPUT;
   m.s_final_b = Mb; m.s_final_b_stride = bh * DK * DK;
+  if (sp.finer()) {   // both passes leave their state where a part starts inside the segment
+    m.flags |= CARRY_SNAPSHOTS;
+    m.flags_b |= CARRY_SNAPSHOTS;
+    m.snap_len = sp.Lp;
+    m.snap = snapD; m.snap_b = snapM;
+    m.snap_stride = bh * DK * p.dv;
+  }
   cudaError_t e = launch_carry<MODE>(p, NC, records, m, true, stream, err);
   if (e != cudaSuccess) return e;
-  segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), 256, 0, stream>>>(s0, Mb, Db, Ss, sp.G, p.H, p.dv);
+  e = cudaFuncSetAttribute(segment_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(chain::SMEM_BYTES));
+  if (e != cudaSuccess) {
+    *err = "cudaFuncSetAttribute: ";
+    return e;
+  }
+  segment_chain_kernel<<<dim3(p.dv / 16, p.H, p.B), chain::NT, chain::SMEM_BYTES, stream>>>(
+      s0, Mb, Db, snapM, snapD, Ss, items, sp.L, sp.Lp, p.H, p.dv);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = "segment chain launch: ";
     return e;
   }
-  CarryLaunch f;   // phase 2: every segment from its start
-  f.segments = sp.G; f.seg_len = sp.L;
+  CarryLaunch f;   // phase 2: every part from its start
+  f.segments = sp.P; f.seg_len = sp.Lp;
   f.flags = CARRY_LAST_FINAL | flags2;
   f.s0 = Ss; f.s0_stride = bh * DK * p.dv;
   f.s_final = s_final;
@@ -2422,12 +2612,14 @@ size_t gdr_split_workspace_bytes(int variant, int B, int T, int H, int dv) {
 }
 
 void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,
-                    int *split_chunk) {
+                    int *split_chunk, int *parts, int *part_chunks) {
   const int NC = (T + 63) / 64;
   const gdr::tc::SegPlan sp = gdr::tc::seg_plan_for(B, H, dv, NC, sms);
   *segments = sp.G;
   *segment_chunks = sp.L;
   *split_chunk = sp.G == 1 ? gdr::tc::pipe_plan_for(variant, B, H, NC, sms).c_split : 0;
+  if (parts != nullptr) *parts = sp.G == 1 ? 1 : sp.P;
+  if (part_chunks != nullptr) *part_chunks = sp.G == 1 ? sp.L : sp.Lp;
 }
 
 int gdr_split_launches(int variant, int B, int T, int H, int dv) {

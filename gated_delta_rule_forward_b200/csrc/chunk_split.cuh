@@ -15,9 +15,10 @@ size_t gdr_split_record_bytes(int variant, int dv);   // bytes of one (b, h, chu
 // Bytes of the segmented carry's maps, offsets and start states on the current device (0 when not segmented).
 size_t gdr_split_segment_bytes(int B, int T, int H, int dv);
 int gdr_split_launches(int variant, int B, int T, int H, int dv);   // kernel launches of one two-kernel-path call
-// The two-kernel path's schedule on a device with `sms` SMs (no device query).
+// The two-kernel path's schedule on a device with `sms` SMs (no device query);
+// parts / part_chunks (either may be null): the segmented carry's second phase.
 void gdr_split_plan(int variant, int B, int T, int H, int dv, int sms, int *segments, int *segment_chunks,
-                    int *split_chunk);
+                    int *split_chunk, int *parts = nullptr, int *part_chunks = nullptr);
 // ws_bytes: the workspace at ws; a segmented plan that needs more runs unsegmented.
 cudaError_t gdr_launch_split(const gdr::FwdProblem &p, void *ws, size_t ws_bytes, cudaStream_t stream,
                              std::string *err);

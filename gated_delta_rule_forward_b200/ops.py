@@ -224,9 +224,13 @@ def forward_kernel_name(variant, dtype, B, T, H, dk, dv, chunk=0) -> str:
 
 def forward_plan(variant, B, T, H, dv, sms) -> dict:
     """How the two-kernel chunked path schedules this problem on a device with
-    ``sms`` SMs (host-only): segments per sequence, chunks per segment, and the
-    chunk where the pipelined sweep cuts each sequence (0: serial)."""
-    g, lc, cs = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    ``sms`` SMs (host-only): segments per sequence and chunks per segment (the
+    segmented carry's maps), the parts per sequence and chunks per part of its
+    carry with outputs, and the chunk where the pipelined sweep cuts each
+    sequence (0: serial)."""
+    g, lc, cs, pa, pc = (ctypes.c_int() for _ in range(5))
     check(lib().gdr_forward_plan(variant_id(variant), B, T, H, dv, sms, ctypes.byref(g), ctypes.byref(lc),
                                  ctypes.byref(cs)))
-    return {"segments": g.value, "segment_chunks": lc.value, "split_chunk": cs.value}
+    check(lib().gdr_forward_segment_parts(variant_id(variant), B, T, H, dv, sms, ctypes.byref(pa), ctypes.byref(pc)))
+    return {"segments": g.value, "segment_chunks": lc.value, "parts": pa.value, "part_chunks": pc.value,
+            "split_chunk": cs.value}

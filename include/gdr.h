@@ -125,7 +125,8 @@ typedef struct {
  * 0 for every other path.  When few sequences of many chunks would leave
  * most of the device idle (B * H small, dv = 128, T >= 4033), the carry runs
  * in segments and the size adds their transition maps and start states
- * (fp32, a few MB).  The workspace is caller-owned scratch, overwritten by
+ * and, where the carry with outputs is cut finer than the maps, the maps'
+ * snapshots at the part starts (fp32, a few to a few tens of MB).  The workspace is caller-owned scratch, overwritten by
  * every call; its contents are not needed after the call completes on the
  * stream.
  */
@@ -147,7 +148,8 @@ size_t gdr_forward_workspace_size(int variant, int dtype, int B, int T, int H,
  *      sequential carry kernel: all five variants with bf16 I/O and dk = 128;
  *      needs the workspace.  Where the carry's B * H CTAs leave SMs idle it
  *      reschedules: for few long sequences, segment maps, a chain of segment
- *      start states, then the segments in parallel; for a mid-size B * H,
+ *      start states, then the segments (or finer parts, see
+ *      gdr_forward_segment_parts) in parallel; for a mid-size B * H,
  *      the sweep cut in two, with the second part's preparation beside the
  *      first part's carry.  Its kernels are chained on `stream` by
  *      programmatic dependent launch; the call returns after enqueueing them,
@@ -311,6 +313,18 @@ const char *gdr_forward_kernel_name(int variant, int dtype, int B, int T, int H,
  */
 gdr_status_t gdr_forward_plan(int variant, int B, int T, int H, int dv, int sms, int *segments,
                               int *segment_chunks, int *split_chunk);
+
+/*
+ * The second phase of a segmented plan (same arguments and errors as
+ * gdr_forward_plan).  The segment maps come from a first phase of about two
+ * CTAs per segment; the carry with outputs needs one CTA per part, so it may
+ * cut each sequence finer, into *parts parts of *part_chunks chunks (the last
+ * one ragged), each starting from the map and offset of its segment after the
+ * chunks before it.  Without segmenting: 1 part of all chunks; where phase 2
+ * does not cut finer: the segments themselves.
+ */
+gdr_status_t gdr_forward_segment_parts(int variant, int B, int T, int H, int dv, int sms, int *parts,
+                                       int *part_chunks);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device-side

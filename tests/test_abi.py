@@ -184,7 +184,7 @@ def test_two_kernel_schedule_on_a_148_sm_device(L):
     assert _plan(L, 4, 4, 4096, 16) == (1, 64, 39)     # 1.3B KLA
     assert _plan(L, 2, 4, 4096, 16) == (1, 64, 53)     # 1.3B KDA
     assert _plan(L, 3, 4, 4096, 16) == (1, 64, 51)     # 1.3B GDN-2
-    assert _plan(L, 1, 1, 65536, 16) == (6, 171, 0)    # 64k: six segments of 171 chunks
+    assert _plan(L, 1, 1, 65536, 16) == (6, 183, 0)    # 64k: six segments of 183 chunks (phase 1)
     assert _plan(L, 1, 1, 4100, 2) == (13, 5, 0)       # the segmented GPU test: 13 segments of 5
     assert _plan(L, 1, 2, 4480, 3) == (12, 6, 0)       # and its other shape: 12 of 6
     for v in range(5):                                  # the pipelined GPU tests (24 chunks)
@@ -195,6 +195,56 @@ def test_two_kernel_schedule_on_a_148_sm_device(L):
     assert _plan(L, 1, 1, 65536, 16, dv=64)[0] == 1    # segmenting needs dv = 128
     assert _plan(L, 1, 0, 5000, 8) == (1, 79, 0)       # no sequences: nothing to divide by
     assert _plan(L, 1, 4, 4096, 16, sms=0) == (1, 64, 0)
+
+
+def _parts(L, variant, B, T, H, dv=128, sms=148):
+    pa, pc = ctypes.c_int(-1), ctypes.c_int(-1)
+    st = L.gdr_forward_segment_parts(variant, B, T, H, dv, sms, ctypes.byref(pa), ctypes.byref(pc))
+    assert st == 0, L.gdr_last_error()
+    return pa.value, pc.value
+
+
+def test_segment_parts_on_a_148_sm_device(L):
+    """The segmented carry's second phase: one CTA per part, so it may cut finer
+    than the maps' segments (B200, 148 SMs)."""
+    assert _parts(L, 1, 1, 65536, 16) == (9, 114)     # 64k: nine parts, 144 CTAs
+    assert _parts(L, 1, 1, 7041, 17) == (7, 16)       # the finer-parts GPU test (5 segments of 24)
+    assert _plan(L, 1, 1, 7041, 17) == (5, 24, 0)
+    assert _parts(L, 1, 1, 5000, 12) == (7, 12)       # a short sequence: the chain's products cost more
+    assert _parts(L, 1, 1, 4100, 2) == (13, 5)        # the segmented GPU test: the segments themselves
+    assert _parts(L, 1, 8, 2048, 8) == (1, 32)        # not segmented: one part
+    assert _parts(L, 1, 1, 65536, 16, dv=64) == (1, 1024)
+    assert _parts(L, 1, 1, 1 << 20, 1) == (61, 269)   # at most 64 parts
+    g = ctypes.c_int()
+    assert L.gdr_forward_segment_parts(9, 1, 64, 1, 128, 148, ctypes.byref(g), ctypes.byref(g)) == 1
+    assert L.gdr_forward_segment_parts(1, 1, 64, 1, 128, -1, ctypes.byref(g), ctypes.byref(g)) == 1
+    assert L.gdr_forward_segment_parts(1, 1, 64, 1, 128, 148, ctypes.byref(g), None) == 1
+
+
+def test_segment_plan_invariants(L):
+    """Every segmented plan over a grid of shapes and device sizes: the segments
+    and the parts each cover the sequence with a ragged last one; phase 1
+    (2G - 3 CTAs per sequence) and phase 2 (one per part) fit the SMs; and no part
+    starts strictly inside the last segment, which phase 1 does not run (its
+    start states come from the maps after the chunks before them)."""
+    n = 0
+    for sms in (132, 148, 160):
+        for B, H in ((1, 1), (1, 2), (1, 3), (2, 3), (1, 5), (1, 8), (1, 12), (1, 16), (2, 8), (1, 24), (1, 40)):
+            for T in (4033, 4100, 5000, 8150, 12345, 40000, 65536, 100000, 1 << 20):
+                NC = (T + 63) // 64
+                G, Lc, _ = _plan(L, 1, B, T, H, sms=sms)
+                P, Lp = _parts(L, 1, B, T, H, sms=sms)
+                if G == 1:
+                    assert (P, Lp) == (1, Lc)
+                    continue
+                n += 1
+                bh = B * H
+                assert G >= 3 and (G - 1) * Lc < NC <= G * Lc
+                assert (P - 1) * Lp < NC <= P * Lp
+                assert (2 * G - 3) * bh <= sms and P * bh <= sms and P <= max(G, 64)
+                assert (P - 1) * Lp <= (G - 1) * Lc
+                assert P >= G and (P == G) == (Lp == Lc)
+    assert n > 100
 
 
 def test_two_kernel_schedule_rejects_bad_arguments(L):
@@ -212,8 +262,10 @@ def test_empty_batch_workspace_query(L):
 
 def test_forward_plan_binding():
     import gated_delta_rule_forward_b200 as gdr
-    assert gdr.forward_plan("gdn", 8, 2048, 8, 128, 148) == {"segments": 1, "segment_chunks": 32, "split_chunk": 20}
-    assert gdr.forward_plan("kla", 1, 65536, 16, 128, 148) == {"segments": 6, "segment_chunks": 171, "split_chunk": 0}
+    assert gdr.forward_plan("gdn", 8, 2048, 8, 128, 148) == {"segments": 1, "segment_chunks": 32, "parts": 1,
+                                                             "part_chunks": 32, "split_chunk": 20}
+    assert gdr.forward_plan("kla", 1, 65536, 16, 128, 148) == {"segments": 6, "segment_chunks": 183, "parts": 9,
+                                                               "part_chunks": 114, "split_chunk": 0}
     with pytest.raises(gdr.GdrError):
         gdr.forward_plan("gdn", 8, 2048, 8, 96, 148)
 

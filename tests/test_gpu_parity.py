@@ -195,6 +195,25 @@ def test_pipelined_sweep_no_states():
     assert_close(o, o_ref, torch.bfloat16, "o")
 
 
+@pytest.mark.parametrize("variant,s0", [("gdn", True), ("kla", True), ("kda", True), ("gdn2", True),
+                                        ("gdn", False)])
+def test_segmented_carry_finer_parts(variant, s0):
+    """Phase 2 cut finer than phase 1's segments: B=1, H=17, T=7041 (111 chunks,
+    the last of one token) runs the maps over 5 segments of 24 chunks and the
+    carry with outputs over 7 parts of 16 (the last one 15).  Part starts fall
+    inside segment 0 (chunk 16: the state itself), inside later segments
+    (chunks 32, 64, 80: map and offset after the chunks before them, applied to
+    the segment's start) and on segment starts (chunks 48, 96).  Compared
+    element by element with the oracle."""
+    B, T, H = 1, 7041, 17
+    plan = gdr.forward_plan(variant, B, T, H, 128, 148)
+    assert (plan["segments"], plan["segment_chunks"], plan["parts"], plan["part_chunks"]) == (5, 24, 7, 16)
+    assert gdr.forward_launches(variant, torch.bfloat16, B, T, H, 128, 128, 0) == 4
+    o, S, o_ref, S_ref = run_both(variant, B, T, H, 128, 128, torch.bfloat16, 0, seed=41, s0=s0)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
 def test_segmented_carry_no_initial_state():
     """Segmented carry from a zero state, B=2 H=3 T=4480 (70 chunks, 12 segments
     of 6): segment 0 then starts from zeros like every other segment's offset."""
