@@ -135,6 +135,83 @@ def test_chunk_equations_match_the_oracle(variant):
         np.testing.assert_allclose(g["log_g"], g_ref["log_g"][0, :, 0], rtol=0, atol=1e-10)
 
 
+@pytest.mark.parametrize("variant", ["deltanet", "gdn", "kda"])
+def test_segmented_carry_with_finer_parts_matches_the_oracle(variant):
+    """The segmented carry as the library plans it for B=1, H=17, T=7041 on 148
+    SMs (111 chunks, the last of one token): phase 1 runs segment 0 from S0 and
+    the other segments but the last from zero (offsets D_g) and from the
+    identity without values (maps M_g), leaving snapshots of both at every
+    multiple of the part length inside a segment; the chain forms the segment
+    starts S[g+1] = M_g S[g] + D_g and, in the same pass, each part start inside
+    segment g as M_g(j) S[g] + D_g(j) (D_0(j) itself in segment 0); phase 2 runs
+    the parts from their starts.  Here with chunks of 8 tokens and small d_k,
+    d_v, against the token-by-token oracle.  beta and the decay are weakened
+    (x 0.05, x 0.01) so that a segment's start state still shows at its end:
+    with the recipe's gates the maps M_g(j) fall below 1e-20 and the test
+    would not see their products."""
+    import gated_delta_rule_forward_b200 as gdr
+    plan = gdr.forward_plan(variant, 1, 7041, 17, 128, 148)
+    G, L, P, Lp = plan["segments"], plan["segment_chunks"], plan["parts"], plan["part_chunks"]
+    assert P > G and Lp < L
+    NC = 111
+    B, T, H, dk, dv, scale = 1, (NC - 1) * C + 1, 1, 6, 5, 0.7
+    d = make_inputs(variant, B, T, H, dk, dv, dtype=torch.float32, seed=17)
+    d = {k: (None if v is None else v.double().numpy()) for k, v in d.items()}
+    d["beta"] = 0.05 * d["beta"]
+    if d["log_g"] is not None:
+        d["log_g"] = 0.01 * d["log_g"]
+    s0 = np.random.default_rng(17).standard_normal((dk, dv))
+    o_ref, S_ref = oracle.forward(variant, **d, initial_state=s0[None, None], scale=scale)
+    lg = (np.zeros((T, dk)) if variant == "deltanet" else
+          np.repeat(d["log_g"][0, :, 0][:, None], dk, axis=1) if variant == "gdn" else d["log_g"][0, :, 0])
+    # per-chunk quantities (none depends on the state) and each chunk's affine map S -> A S + Bc
+    _, _, saved = chunk_forward(d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0], d["beta"][0, :, 0], lg, s0,
+                                scale)
+    assert len(saved) == NC
+    for sv in saved:
+        sv["U"] = sv["T"] @ (sv["b"][:, None] * sv["V"])
+        sv["A"] = np.diag(np.exp(sv["gam"][-1])) - sv["Kt"].T @ sv["W"]
+        sv["Bc"] = sv["Kt"].T @ sv["U"]
+
+    def sweep(x, c0, c1, values=True, snaps=None):
+        for c in range(c0, c1):
+            if snaps is not None and c > c0 and c % Lp == 0:
+                snaps[c // Lp] = x.copy()
+            x = saved[c]["A"] @ x + (saved[c]["Bc"] if values else 0)
+        return x
+
+    # phase 1
+    Dend, Mend, snapD, snapM = {}, {}, {}, {}
+    for g in range(G - 1):
+        Dend[g] = sweep(s0 if g == 0 else np.zeros((dk, dv)), g * L, min(NC, (g + 1) * L), snaps=snapD)
+    for g in range(1, G - 1):
+        Mend[g] = sweep(np.eye(dk), g * L, min(NC, (g + 1) * L), values=False, snaps=snapM)
+    # the chain, in the kernel's order: part starts inside segment g, then segment start g + 1
+    starts, Sg, p = {0: s0}, s0, 1
+    for g in range(G - 1):
+        while p < P and p * Lp < (g + 1) * L:
+            starts[p] = snapD[p] if g == 0 else snapM[p] @ Sg + snapD[p]
+            p += 1
+        Sg = Dend[0] if g == 0 else Mend[g] @ Sg + Dend[g]
+        if p < P and p * Lp == (g + 1) * L:
+            starts[p] = Sg
+            p += 1
+    assert p == P and sorted(starts) == list(range(P))
+    # phase 2: every part from its start, with outputs
+    o = np.zeros((T, dv))
+    for q in range(P):
+        x = starts[q]
+        for c in range(q * Lp, min(NC, (q + 1) * Lp)):
+            sv = saved[c]
+            o[sv["sl"]] = scale * sv["Qg"] @ x + sv["P"] @ (sv["U"] - sv["W"] @ x)
+            x = sv["A"] @ x + sv["Bc"]
+    np.testing.assert_allclose(o, o_ref[0, :, 0], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(x, S_ref[0, 0], rtol=0, atol=1e-10)
+    # the maps matter: the last part's start moves by more than 1e-3 without its M S[g] term
+    g_last = ((P - 1) * Lp - 1) // L
+    assert np.abs(Mend[g_last] @ Dend[g_last - 1]).max() > 1e-3 if g_last >= 2 else True
+
+
 @pytest.mark.parametrize("variant", ["gdn", "kda"])
 def test_two_record_carry_step_matches_the_oracle(variant):
     """One carry step over two records (c, c+1), from their single-chunk quantities
@@ -152,7 +229,8 @@ def test_two_record_carry_step_matches_the_oracle(variant):
     rng = np.random.default_rng(9)
     S = rng.standard_normal((dk, dv))
     o_ref, S_ref = oracle.forward(variant, **d, initial_state=S[None, None], scale=scale)
-    lg = (np.repeat(d["log_g"][0, :, 0][:, None], dk, axis=1) if variant == "gdn" else d["log_g"][0, :, 0])
+    lg = (np.zeros((T, dk)) if variant == "deltanet" else
+          np.repeat(d["log_g"][0, :, 0][:, None], dk, axis=1) if variant == "gdn" else d["log_g"][0, :, 0])
     _, _, sv = chunk_forward(d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0], d["beta"][0, :, 0], lg, S, scale)
     a, b = sv
     ga, gb = np.exp(a["gam"][-1]), np.exp(b["gam"][-1])      # per-channel end decays

@@ -258,6 +258,30 @@ def test_backward_segmented_finer_parts(variant):
         check_grads({**gh, "log_g": None}, {**ref, "log_g": None}, variant, f"head {h}")
 
 
+def test_backward_segmented_long_memory():
+    """Both backward carries segmented (5 segments of 24 chunks, 7 parts of 16)
+    where the maps keep most of a state over a segment: DeltaNet with beta
+    scaled by 0.1 (see test_segmented_carry_long_memory); heads 0 and 16."""
+    B, T, H = 1, 7041, 17
+    scale = 128 ** -0.5
+    d = make_inputs("deltanet", B, T, H, dtype=torch.bfloat16, seed=49)
+    d["beta"] = (0.1 * d["beta"]).contiguous()
+    S0 = random_state(B, H, 128, 128, 50)
+    dS = random_state(B, H, 128, 128, 51, scale=1.0)
+    dO = random_output_grad(B, T, H, 128, 52)
+    dd = to_dev(d)
+    g = gdr.backward(dd["q"], dd["k"], dd["v"], dO.cuda(), variant="deltanet", **gates(dd), initial_state=S0.cuda(),
+                     d_final_state=dS.cuda(), scale=scale)
+    gdr.device_status()
+    for h in (0, H - 1):
+        s = select(d, h=slice(h, h + 1))
+        ref = oracle.backward("deltanet", s["q"], s["k"], s["v"], dO[:, :, h:h + 1], **gates(s),
+                              initial_state=S0[:, h:h + 1], d_final=dS[:, h:h + 1], scale=scale)
+        gh = {k: (None if x is None else (x[:, h:h + 1] if k == "initial_state" else x[:, :, h:h + 1]))
+              for k, x in g.items()}
+        check_grads(gh, ref, "deltanet", f"head {h}")
+
+
 @pytest.mark.parametrize("variant", ["gdn", "kla", "kda", "gdn2"])
 def test_backward_segmented(variant):
     """Few long sequences (B*H = 2, 65 chunks): both carries run in segments (13

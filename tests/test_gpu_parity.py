@@ -214,6 +214,27 @@ def test_segmented_carry_finer_parts(variant, s0):
     assert_close(S, S_ref, torch.bfloat16, "S")
 
 
+@pytest.mark.parametrize("shape", [(1, 4100, 2), (1, 7041, 17)])
+def test_segmented_carry_long_memory(shape):
+    """The segmented carry where a segment's start state still shows at its
+    end: DeltaNet (no decay) with beta scaled by 0.1, so that the maps M_g and
+    M_g(j) keep most of a state over a segment (with the recipe's gates they
+    fall below 1e-20 and a wrong map product would go unseen).  Both plans: 13
+    segments of 5 chunks, and 5 segments of 24 with 7 parts of 16."""
+    B, T, H = shape
+    assert gdr.forward_launches("deltanet", torch.bfloat16, B, T, H, 128, 128, 0) == 4
+    d = make_inputs("deltanet", B, T, H, 128, 128, dtype=torch.bfloat16, seed=47)
+    d["beta"] = (0.1 * d["beta"]).contiguous()
+    S0 = random_state(B, H, 128, 128, 48)
+    dd = to_dev(d)
+    o, S = gdr.forward(dd["q"], dd["k"], dd["v"], variant="deltanet", **gate_kwargs(dd), initial_state=S0.cuda(),
+                       chunk=0)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle.forward("deltanet", **d, initial_state=S0)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S")
+
+
 def test_segmented_carry_no_initial_state():
     """Segmented carry from a zero state, B=2 H=3 T=4480 (70 chunks, 12 segments
     of 6): segment 0 then starts from zeros like every other segment's offset."""
